@@ -1,0 +1,312 @@
+"""Throughput of the KDA chunked forward on the 32K-token, 96-head prefill (B=1, T=32768, H=96,
+K=V=128, bf16 in/out, fp32 state, lower_bound=-5).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one kda_fwd over the whole workload (the full hot path: prologue, intra-chunk solve,
+chunk recurrence and epilogue in one kernel).  Inputs are seeded synthetic tensors resident in
+HBM; they are 4 GB, far larger than the 126 MB L2, so no flush is needed between steps.  For N > 1
+each rank runs an independent replica of the workload (the operator has no cross-GPU step):
+weak scaling, value = all ranks' token-heads / max-over-ranks time.  Prints one JSON line on rank 0.
+
+--impl reference times the CPU fp64 oracle on the host cores instead, on a bounded sample of the
+same workload (it is the only reference implementation available).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "KDA fwd Mtok·head/s at H=96,T=32K; TFLOP/s as % of binding roofline"
+UNIT = "Mtok·head/s"
+T_TOK, HEADS, D = 32768, 96, 128
+CHUNK = 64
+BYTES_PER_TOKEN_HEAD = 4 * 2 * D + 2 + 2 * D          # q, k, v, g in; raw beta in; o out
+FLOPS_PER_TOKEN_HEAD = 6 * D * D + 2 * CHUNK * D + 3 * 2 * CHUNK * D + 2 * CHUNK * D + CHUNK * CHUNK // 3
+STATE_OUT_BYTES_PER_UNIT = D * D * 4                  # fp32 final state written; initial state is zero (NULL)
+WORKLOAD = "prefill B=1 T=32768 H=96 K=V=128 bf16, lower_bound=-5, zero initial state, final state out"
+
+
+def algorithmic_bytes(tokens, heads, units):
+    return BYTES_PER_TOKEN_HEAD * tokens * heads + STATE_OUT_BYTES_PER_UNIT * units
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"kda_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(target_s=15.0):
+    """Times the fp64 oracle on a bounded sample of the prefill: the first m heads over the
+    first L tokens, sized from a short calibration to take about target_s seconds."""
+    import oracle
+    import kda_inputs
+
+    cores = os.cpu_count() or 1
+    oracle.build()
+    x = kda_inputs.make_random("prefill", [T_TOK], HEADS, seed=0)
+    def run(m, L):
+        sl = lambda t: t[:, :L, :m].contiguous()
+        t0 = time.perf_counter()
+        oracle.kda_fwd(sl(x.q), sl(x.k), sl(x.v), sl(x.g), sl(x.beta), x.scale, x.A_log[:m], x.dt_bias[:m],
+                       x.lower_bound, initial_state=None, cu_seqlens=torch.tensor([0, L], dtype=torch.int32),
+                       num_threads=cores)
+        return time.perf_counter() - t0
+    m = min(HEADS, cores)
+    cal = run(m, 1024)
+    L = int(min(T_TOK, max(1024, 1024 * target_s / max(cal, 1e-3))))
+    dt = run(m, L)
+    return {"value": m * L / dt / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"heads 0..{m - 1}, tokens 0..{L - 1} of the prefill workload (fp64 C oracle, "
+                      f"OpenMP over heads), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    steps = []
+    cb = None
+    for i in range(args.warmup + args.steps):
+        cb = cpu_oracle_sample(target_s=min(20.0, 150.0 / max(1, args.warmup + args.steps)))
+        if i >= args.warmup:
+            steps.append(cb["value"])
+    v = statistics.median(steps)
+    cb["value"] = v
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample": cb["sample"]},
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=HEADS,
+                    help="heads of the prefill workload (default 96; fewer only for small profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import kda_inputs
+    import kimi_delta_attention_24_b200 as kda
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    kda.load()
+    if args.heads == HEADS:
+        x = kda_inputs.make_workload("prefill", seed=rank, device=dev)
+    else:
+        x = kda_inputs.make_random("prefill", [T_TOK], args.heads, seed=rank, device=dev)
+    B, T, H, K = x.q.shape
+    N = x.num_seqs
+    out = torch.empty_like(x.v)
+    final = torch.empty(N, H, K, K, dtype=torch.float32, device=dev)
+    ws = torch.zeros(kda.get_workspace_size(B * T, H, N), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.fwd(x.q, x.k, x.v, x.g, x.beta, x.scale, out, ws, x.A_log, x.dt_bias, x.lower_bound,
+                None, final, x.cu_seqlens, stream=stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert kda.read_device_status(ws) == 0
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    kernel_ms = max_over_ranks(statistics.mean(launch_ms), world)
+    status = kda.read_device_status(ws)
+    ms_per_step = total_ms / args.steps
+    token_heads = B * T * H
+    value = world * token_heads / (ms_per_step * 1e-3) / 1e6
+
+    # end to end through the public API with pinned host buffers: H2D inputs, kernel, D2H outputs
+    host = {n: getattr(x, n).cpu().pin_memory() for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "cu_seqlens")}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    fin_h = torch.empty(final.shape, dtype=final.dtype).pin_memory()
+    dev_bufs = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
+
+    def e2e_step():
+        for n, t in host.items():
+            dev_bufs[n].copy_(t, non_blocking=True)
+        kda.fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["g"], dev_bufs["beta"], x.scale, out, ws,
+                dev_bufs["A_log"], dev_bufs["dt_bias"], x.lower_bound, None, final, dev_bufs["cu_seqlens"],
+                stream=stream.cuda_stream)
+        out_h.copy_(out, non_blocking=True)
+        fin_h.copy_(final, non_blocking=True)
+
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+        e2e = {"value": world * token_heads / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    hbm_peak, tf_peak, peak_kind = load_peaks()
+    alg_bytes = algorithmic_bytes(B * T, H, N)
+    achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+    flops = FLOPS_PER_TOKEN_HEAD * token_heads
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            traffic = json.load(f).get("kda_chunked_prefill_bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD if H == HEADS else WORKLOAD.replace("H=96", f"H={H}"), "batch": B, "seq_len": T, "heads": H, "head_dim": K, "chunk": CHUNK,
+                   "parallelism": f"replicas{world}", "l2": "inputs (4.0 GB) exceed L2 (126 MB); no flush"},
+        "tflops": flops / (kernel_ms * 1e-3) / 1e12,
+        "tflops_frac_of_bf16_peak": flops / (kernel_ms * 1e-3) / 1e12 / tf_peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kernel_ms},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "device_status": status,
+    }
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample()
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

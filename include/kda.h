@@ -1,0 +1,114 @@
+/*
+ * kda.h — C ABI of the B200 (sm_100a) Kimi Delta Attention forward library (libkda_b200.so).
+ *
+ * The operation.  Kimi Delta Attention is a gated delta rule with a per-channel decay:
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = scale * S_t^T q_t
+ * with, applied inside the kernels (the flags use_qk_l2norm_in_kernel, use_beta_sigmoid_in_kernel,
+ * use_gate_in_kernel and safe_gate of fla's chunk_kda, all on):
+ *     q <- q / sqrt(|q|^2 + 1e-6),  k likewise,  beta <- sigmoid(beta),
+ *     log alpha_c = lower_bound * sigmoid(exp(A_log[h]) * (g_c + dt_bias[h, c])).
+ * The argument order of kda_fwd follows FlashKDA's `fwd` (q, k, v, g, beta, scale, out, workspace,
+ * A_log, dt_bias, lower_bound, initial_state, final_state, cu_seqlens) as printed in the vLLM PR
+ * #54859 report ("[Kimi-K3] Bump FlashKDA to fix unstable inverse", section 关键源码片段); the
+ * workspace query follows `get_workspace_size(T, H, N)` on the same page; the support predicate
+ * follows `is_flashkda_supported(128, torch.bfloat16, lower_bound)` there.  Shapes and the
+ * batch-mode call (cu_seqlens = None) follow "What CUDA Version Is Required to Use FlashKDA?",
+ * section Usage Examples.  This C ABI adds explicit sizes and a stream.
+ *
+ * Layouts (all contiguous, row-major, device memory, every pointer 16-byte aligned):
+ *   q, k, g   bf16  [batch, seqlen, H, K]      (packed varlen: batch = 1, seqlen = total tokens)
+ *   v, out    bf16  [batch, seqlen, H, V]
+ *   beta      bf16  [batch, seqlen, H]          raw, before the sigmoid
+ *   A_log     fp32  [H];    dt_bias fp32 [H, K]
+ *   initial_state / final_state  fp32 [N, H, K, V] holding S[k][v]   (state_transposed = 0)
+ *                                fp32 [N, H, V, K] holding S^T        (state_transposed = 1)
+ *   cu_seqlens int32 [N + 1]: cu[0] = 0, non-decreasing, cu[N] = seqlen (batch must be 1)
+ * K = V = 128 is the supported head size; lower_bound must lie in [-5, 0].
+ *
+ * Ownership.  The caller owns every buffer.  The library allocates no device memory, keeps no
+ * per-call state, never synchronises the stream and never copies device data to the host
+ * (except kda_read_device_status, which exists to do exactly that).  Outputs are written in
+ * place on `stream`.  initial_state may alias final_state: each unit reads its state before
+ * writing it.  Rows of `out` outside [0, cu[N]) are not touched.
+ *
+ * Errors.  Argument problems are found on the host before anything is launched and nothing is
+ * written.  A launch failure returns KDA_ERR_CUDA.  The chunked kernel bounds every wait it
+ * performs; if a bound is exceeded it records KDA_ERR_DEVICE_TIMEOUT in the workspace status
+ * word and the affected work is skipped — read it with kda_read_device_status.
+ */
+#ifndef KDA_B200_H_
+#define KDA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st* kda_stream_t;
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARGUMENT = 1,   /* null pointer, bad shape, misaligned pointer, bad flag */
+  KDA_ERR_UNSUPPORTED = 2,        /* head dim != 128 or lower_bound outside [-5, 0] */
+  KDA_ERR_WORKSPACE_TOO_SMALL = 3,
+  KDA_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+  KDA_ERR_DEVICE_TIMEOUT = 5      /* a bounded device-side wait ran out (see kda_read_device_status) */
+} kda_status_t;
+
+/* 1 when (head_dim, dtype, lower_bound) is a configuration this library runs: head_dim = 128,
+ * bf16 inputs (dtype_is_bf16 != 0) and -5 <= lower_bound <= 0; otherwise 0.  Mirrors
+ * is_flashkda_supported(128, torch.bfloat16, lower_bound). */
+int kda_is_supported(int head_dim, int dtype_is_bf16, float lower_bound);
+
+/* Bytes of device workspace kda_fwd needs for (total tokens T, heads H, sequences N), as
+ * get_workspace_size(T, H, N).  Depends only on its arguments; the workspace needs no
+ * initialisation by the caller beyond being zero-filled once before first use (it carries the
+ * sticky device status word). */
+size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+
+/* The chunked forward pass (the product path): one fused kernel per call.
+ *   scale          multiplies the output (o = scale * S^T qhat); it never enters the state.
+ *   workspace      device buffer of at least kda_workspace_size(batch*seqlen, H, N) bytes,
+ *                  zero-filled once by the caller before its first use.
+ *   initial_state  NULL means a zero state.   final_state  NULL means it is not written.
+ *   cu_seqlens     NULL selects batch mode: N = batch sequences of length seqlen each.
+ *   num_seqs       N; with cu_seqlens it must be the number of documents, without it batch
+ *                  (0 is accepted and means batch).
+ *   state_transposed  0: state is S[k][v];  1: state is stored transposed (S^T, [V][K]).
+ * Returns KDA_OK once the work is enqueued on `stream`. */
+kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                     float scale, void* out, void* workspace, size_t workspace_bytes,
+                     const float* A_log, const float* dt_bias, float lower_bound,
+                     const float* initial_state, float* final_state, const int32_t* cu_seqlens,
+                     int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
+                     int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
+                     kda_stream_t stream);
+
+/* The same operation evaluated token by token on CUDA cores (one thread per state column):
+ * no chunking, no tensor cores.  Same arguments, layouts and errors as kda_fwd (the workspace
+ * may be NULL with workspace_bytes = 0).  It is the GPU restatement of the recurrence and the
+ * basis of single-token decoding; it is much slower than kda_fwd on long prefills. */
+kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, float scale, void* out, void* workspace,
+                               size_t workspace_bytes, const float* A_log, const float* dt_bias,
+                               float lower_bound, const float* initial_state, float* final_state,
+                               const int32_t* cu_seqlens, int32_t batch, int64_t seqlen,
+                               int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v,
+                               int32_t num_seqs, int32_t state_transposed, kda_stream_t stream);
+
+/* Synchronises `stream`, reads the workspace's sticky status word, clears it, and returns
+ * KDA_OK or the recorded device error (KDA_ERR_DEVICE_TIMEOUT).  KDA_ERR_CUDA if the copy fails. */
+kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream);
+
+/* A static, human-readable name for a status code. */
+const char* kda_status_string(kda_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_H_ */

@@ -1,0 +1,173 @@
+"""B200 (sm_100a) Kimi Delta Attention forward: Python binding of libkda_b200.so.
+
+Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream.
+
+    fwd(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
+        initial_state, final_state, cu_seqlens)          # FlashKDA-style, writes in place
+    get_workspace_size(T, H, N)
+    is_supported(head_dim, dtype, lower_bound)
+    chunk_kda(q, k, v, g, beta, ...) -> (out, final_state)  # fla-style, allocates outputs
+    fwd_recurrent(...)                                     # token-serial CUDA-core kernel
+
+The argument order of ``fwd`` follows FlashKDA's ``fwd`` as printed in the vLLM PR #54859 report
+(test_flashkda_near_collinear_keys_remain_finite); ``chunk_kda`` follows the fla call on the page
+"What CUDA Version Is Required to Use FlashKDA?", section Usage Examples.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["fwd", "fwd_recurrent", "get_workspace_size", "is_supported", "chunk_kda",
+           "read_device_status", "KDAError", "library_path", "load"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "lib", "libkda_b200.so")
+_lib = None
+
+_STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARGUMENT", 2: "KDA_ERR_UNSUPPORTED",
+           3: "KDA_ERR_WORKSPACE_TOO_SMALL", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_DEVICE_TIMEOUT"}
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Loads libkda_b200.so.  Raises if it has not been built: there is no fallback path."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is not built; run `python -m kimi_delta_attention_24_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    fwd_args = [vp, vp, vp, vp, vp, f32, vp, vp, ctypes.c_size_t, vp, vp, f32, vp, vp, vp,
+                i32, i64, i32, i32, i32, i32, i32, vp]
+    for name in ("kda_fwd", "kda_fwd_recurrent"):
+        fn = getattr(lib, name)
+        fn.argtypes = fwd_args
+        fn.restype = ctypes.c_int
+    lib.kda_workspace_size.argtypes = [i64, i32, i32]
+    lib.kda_workspace_size.restype = ctypes.c_size_t
+    lib.kda_is_supported.argtypes = [ctypes.c_int, ctypes.c_int, f32]
+    lib.kda_is_supported.restype = ctypes.c_int
+    lib.kda_read_device_status.argtypes = [vp, vp]
+    lib.kda_read_device_status.restype = ctypes.c_int
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def get_workspace_size(T: int, H: int, N: int) -> int:
+    return int(load().kda_workspace_size(int(T), int(H), int(N)))
+
+
+def is_supported(head_dim: int, dtype=torch.bfloat16, lower_bound: float = -5.0) -> bool:
+    return bool(load().kda_is_supported(int(head_dim), int(dtype == torch.bfloat16), float(lower_bound)))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype, device):
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _call(fn_name, q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
+          initial_state, final_state, cu_seqlens, state_transposed, stream):
+    lib = load()
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (out, "out")):
+        _check(t, n, torch.bfloat16, dev)
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (initial_state, "initial_state"),
+                 (final_state, "final_state")):
+        _check(t, n, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if workspace is not None:
+        _check(workspace, "workspace", torch.uint8, dev)
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, K]")
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = getattr(lib, fn_name)(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(out), _ptr(workspace),
+            0 if workspace is None else workspace.numel(), _ptr(A_log), _ptr(dt_bias), float(lower_bound),
+            _ptr(initial_state), _ptr(final_state), _ptr(cu_seqlens), B, T, H, K, V, N,
+            int(bool(state_transposed)), ctypes.c_void_p(stream))
+    if st != 0:
+        raise KDAError(st, fn_name)
+
+
+def fwd(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
+        initial_state=None, final_state=None, cu_seqlens=None, state_transposed=False, stream=None):
+    """The chunked forward (tcgen05 kernel).  Writes ``out`` and ``final_state`` in place."""
+    _call("kda_fwd", q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
+          initial_state, final_state, cu_seqlens, state_transposed, stream)
+
+
+def fwd_recurrent(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
+                  initial_state=None, final_state=None, cu_seqlens=None, state_transposed=False,
+                  stream=None):
+    """The token-serial CUDA-core kernel (same contract as ``fwd``)."""
+    _call("kda_fwd_recurrent", q, k, v, g, beta, scale, out, workspace, A_log, dt_bias,
+          lower_bound, initial_state, final_state, cu_seqlens, state_transposed, stream)
+
+
+def read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the workspace's device status code."""
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device).cuda_stream
+    with torch.cuda.device(workspace.device):
+        return int(load().kda_read_device_status(_ptr(workspace), ctypes.c_void_p(stream)))
+
+
+def chunk_kda(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=False,
+              A_log=None, dt_bias=None, lower_bound=-5.0, cu_seqlens=None,
+              transpose_state_layout=False, recurrent=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """fla-style call with the in-kernel L2 norm, beta sigmoid and safe gate always on.
+
+    Returns ``(out, final_state)``; ``final_state`` is None unless ``output_final_state``.
+    With ``transpose_state_layout`` the states are [N, H, V, K] (S transposed)."""
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    if scale is None:
+        scale = K ** -0.5
+    if A_log is None:
+        A_log = torch.zeros(H, dtype=torch.float32, device=q.device)
+    if dt_bias is None:
+        dt_bias = torch.zeros(H, K, dtype=torch.float32, device=q.device)
+    out = torch.empty_like(v)
+    final = None
+    if output_final_state:
+        shape = (N, H, V, K) if transpose_state_layout else (N, H, K, V)
+        final = torch.empty(shape, dtype=torch.float32, device=q.device)
+    ws = torch.zeros(get_workspace_size(B * T, H, N), dtype=torch.uint8, device=q.device)
+    fn = fwd_recurrent if recurrent else fwd
+    fn(q, k, v, g, beta, scale, out, ws, A_log, dt_bias, lower_bound, initial_state, final,
+       cu_seqlens, state_transposed=transpose_state_layout)
+    return out, final

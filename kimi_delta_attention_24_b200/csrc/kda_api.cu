@@ -1,0 +1,164 @@
+// C ABI of the KDA forward library: argument validation, workspace layout and launches.
+// The declarations and the contract live in include/kda.h.
+#include <math.h>
+
+#include "kda_common.cuh"
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Shape {
+  int64_t total_tokens;
+  int32_t num_seqs;
+};
+
+// Validates everything the host can check without touching device memory.
+kda_status_t validate(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                      const void* out, const float* A_log, const float* dt_bias, float lower_bound,
+                      const float* initial_state, const float* final_state,
+                      const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
+                      int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
+                      int32_t state_transposed, float scale, Shape* shape) {
+  if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
+  if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !g || !beta || !out || !A_log || !dt_bias) return KDA_ERR_INVALID_ARGUMENT;
+  if (batch < 0 || seqlen < 0 || num_heads <= 0 || num_seqs < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (state_transposed != 0 && state_transposed != 1) return KDA_ERR_INVALID_ARGUMENT;
+  if (!isfinite(scale)) return KDA_ERR_INVALID_ARGUMENT;
+  const void* vec[] = {q, k, v, g, out};
+  for (const void* p : vec)
+    if (!aligned(p, 16)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!aligned(beta, 2) || !aligned(A_log, 4) || !aligned(dt_bias, 16)) return KDA_ERR_INVALID_ARGUMENT;
+  if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (cu_seqlens) {
+    if (!aligned(cu_seqlens, 4) || batch != 1) return KDA_ERR_INVALID_ARGUMENT;
+    if (seqlen > INT32_MAX) return KDA_ERR_INVALID_ARGUMENT;  // cu_seqlens is int32
+    shape->num_seqs = num_seqs;
+  } else {
+    if (num_seqs != 0 && num_seqs != batch) return KDA_ERR_INVALID_ARGUMENT;
+    shape->num_seqs = batch;
+  }
+  shape->total_tokens = (int64_t)batch * seqlen;
+  if ((int64_t)shape->num_seqs * num_heads > INT32_MAX) return KDA_ERR_INVALID_ARGUMENT;
+  return KDA_OK;
+}
+
+kda::FwdParams make_params(const void* q, const void* k, const void* v, const void* g,
+                           const void* beta, float scale, void* out, const float* A_log,
+                           const float* dt_bias, float lower_bound, const float* initial_state,
+                           float* final_state, const int32_t* cu_seqlens, int64_t seqlen,
+                           int32_t num_heads, int32_t num_seqs, int32_t state_transposed,
+                           uint32_t* status) {
+  kda::FwdParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.g = static_cast<const __nv_bfloat16*>(g);
+  p.beta = static_cast<const __nv_bfloat16*>(beta);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.A_log = A_log;
+  p.dt_bias = dt_bias;
+  p.initial_state = initial_state;
+  p.final_state = final_state;
+  p.cu_seqlens = cu_seqlens;
+  p.seqlen = seqlen;
+  p.num_heads = num_heads;
+  p.num_seqs = num_seqs;
+  p.scale = scale;
+  p.lower_bound = lower_bound;
+  p.state_transposed = state_transposed;
+  p.status = status;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_is_supported(int head_dim, int dtype_is_bf16, float lower_bound) {
+  return head_dim == kda::kHeadDim && dtype_is_bf16 != 0 && lower_bound >= -5.0f &&
+         lower_bound <= 0.0f;
+}
+
+size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  (void)total_tokens;
+  const size_t units = (size_t)(num_seqs > 0 ? num_seqs : 0) * (size_t)(num_heads > 0 ? num_heads : 0);
+  return kda::kWorkspaceHeader + round_up(units * sizeof(int32_t), 256);
+}
+
+kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                     float scale, void* out, void* workspace, size_t workspace_bytes,
+                     const float* A_log, const float* dt_bias, float lower_bound,
+                     const float* initial_state, float* final_state, const int32_t* cu_seqlens,
+                     int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
+                     int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
+                     kda_stream_t stream) {
+  Shape shape;
+  kda_status_t st = validate(q, k, v, g, beta, out, A_log, dt_bias, lower_bound, initial_state,
+                             final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k,
+                             head_dim_v, num_seqs, state_transposed, scale, &shape);
+  if (st != KDA_OK) return st;
+  if (!workspace || !aligned(workspace, 256)) return KDA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < kda_workspace_size(shape.total_tokens, num_heads, shape.num_seqs))
+    return KDA_ERR_WORKSPACE_TOO_SMALL;
+  kda::FwdParams p = make_params(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
+                                 initial_state, final_state, cu_seqlens, seqlen, num_heads,
+                                 shape.num_seqs, state_transposed, static_cast<uint32_t*>(workspace));
+  if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
+  return kda::launch_chunked(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
+                                                                                        : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, float scale, void* out, void* workspace,
+                               size_t workspace_bytes, const float* A_log, const float* dt_bias,
+                               float lower_bound, const float* initial_state, float* final_state,
+                               const int32_t* cu_seqlens, int32_t batch, int64_t seqlen,
+                               int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v,
+                               int32_t num_seqs, int32_t state_transposed, kda_stream_t stream) {
+  (void)workspace_bytes;
+  Shape shape;
+  kda_status_t st = validate(q, k, v, g, beta, out, A_log, dt_bias, lower_bound, initial_state,
+                             final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k,
+                             head_dim_v, num_seqs, state_transposed, scale, &shape);
+  if (st != KDA_OK) return st;
+  kda::FwdParams p = make_params(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
+                                 initial_state, final_state, cu_seqlens, seqlen, num_heads,
+                                 shape.num_seqs, state_transposed, static_cast<uint32_t*>(workspace));
+  if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
+  return kda::launch_recurrent(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream) {
+  if (!workspace) return KDA_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  return (word & kda::kStatusTimeout) ? KDA_ERR_DEVICE_TIMEOUT : KDA_OK;
+}
+
+const char* kda_status_string(kda_status_t status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARGUMENT: return "KDA_ERR_INVALID_ARGUMENT";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_WORKSPACE_TOO_SMALL: return "KDA_ERR_WORKSPACE_TOO_SMALL";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// Shared host/device definitions of the KDA forward library (not part of the public ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+constexpr int kHeadDim = 128;        // K = V = 128, the only supported head size
+constexpr float kL2Eps = 1e-6f;      // inside the square root of the q/k L2 norm
+
+// Device status word (first 4 bytes of the workspace), sticky until read by the host.
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr size_t kWorkspaceHeader = 256;  // status word + padding; the rest is per-unit tables
+
+// Arguments of one forward call, after host-side validation.
+struct FwdParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* g;
+  const __nv_bfloat16* beta;
+  __nv_bfloat16* out;
+  const float* A_log;
+  const float* dt_bias;
+  const float* initial_state;  // may be null
+  float* final_state;          // may be null
+  const int32_t* cu_seqlens;   // null: batch mode
+  int64_t seqlen;              // batch mode: tokens per sequence
+  int32_t num_heads;
+  int32_t num_seqs;
+  float scale;
+  float lower_bound;
+  int32_t state_transposed;
+  uint32_t* status;            // workspace status word, may be null (recurrent path)
+};
+
+// Token range [bos, eos) of sequence n.
+__device__ __forceinline__ void seq_range(const FwdParams& p, int n, int64_t& bos, int64_t& eos) {
+  if (p.cu_seqlens) {
+    bos = p.cu_seqlens[n];
+    eos = p.cu_seqlens[n + 1];
+  } else {
+    bos = (int64_t)n * p.seqlen;
+    eos = bos + p.seqlen;
+  }
+}
+
+// Launchers (defined in the kernel translation units).  Return the launch's cudaError_t.
+cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
+cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream);
+
+}  // namespace kda

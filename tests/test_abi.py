@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad arguments on the
+host before touching a GPU (CPU only: no call here reaches a kernel launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kimi_delta_attention_24_b200 as kda
+from kimi_delta_attention_24_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load()
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "kda_fwd" in names and "kda_workspace_size" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    for code, name in [(0, b"KDA_OK"), (1, b"KDA_ERR_INVALID_ARGUMENT"), (2, b"KDA_ERR_UNSUPPORTED"),
+                       (3, b"KDA_ERR_WORKSPACE_TOO_SMALL"), (4, b"KDA_ERR_CUDA"),
+                       (5, b"KDA_ERR_DEVICE_TIMEOUT")]:
+        assert lib.kda_status_string(code) == name
+
+
+def test_support_predicate(lib):
+    assert lib.kda_is_supported(128, 1, -5.0) == 1
+    assert lib.kda_is_supported(128, 1, 0.0) == 1
+    assert lib.kda_is_supported(128, 1, -5.5) == 0
+    assert lib.kda_is_supported(128, 1, 0.5) == 0
+    assert lib.kda_is_supported(64, 1, -5.0) == 0
+    assert lib.kda_is_supported(128, 0, -5.0) == 0
+
+
+def test_workspace_size_depends_on_units(lib):
+    a = lib.kda_workspace_size(32768, 96, 1)
+    b = lib.kda_workspace_size(1, 96, 1)
+    assert a == b and a >= 256 and a % 256 == 0
+    assert lib.kda_workspace_size(100, 32, 8) >= 256 + 4 * 32 * 8
+
+
+# Fake device pointers: aligned, never dereferenced because validation fails first.
+P = 0x10000000
+
+
+def call(lib, name="kda_fwd", **kw):
+    a = dict(q=P, k=P, v=P, g=P, beta=P, scale=0.088, out=P, ws=P, ws_bytes=1 << 20, A_log=P,
+             dt_bias=P, lb=-5.0, s0=None, sT=None, cu=None, batch=1, seqlen=64, H=1, K=128, V=128,
+             N=1, transposed=0)
+    a.update(kw)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return getattr(lib, name)(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]), a["scale"],
+                              vp(a["out"]), vp(a["ws"]), a["ws_bytes"], vp(a["A_log"]), vp(a["dt_bias"]),
+                              a["lb"], vp(a["s0"]), vp(a["sT"]), vp(a["cu"]), a["batch"], a["seqlen"],
+                              a["H"], a["K"], a["V"], a["N"], a["transposed"], None)
+
+
+@pytest.mark.parametrize("name", ["kda_fwd", "kda_fwd_recurrent"])
+def test_host_validation(lib, name):
+    assert call(lib, name, K=64) == 2
+    assert call(lib, name, V=64) == 2
+    assert call(lib, name, lb=-5.01) == 2
+    assert call(lib, name, lb=0.1) == 2
+    assert call(lib, name, lb=float("nan")) == 2
+    assert call(lib, name, q=None) == 1
+    assert call(lib, name, out=P + 8) == 1          # misaligned
+    assert call(lib, name, H=0) == 1
+    assert call(lib, name, seqlen=-1) == 1
+    assert call(lib, name, transposed=2) == 1
+    assert call(lib, name, cu=P, batch=2) == 1      # varlen needs batch 1
+    assert call(lib, name, N=3) == 1                # batch mode: N must equal batch
+    assert call(lib, name, scale=float("inf")) == 1
+    assert call(lib, name, s0=P + 4) == 1
+
+
+def test_workspace_checks(lib):
+    assert call(lib, ws=None) == 1
+    assert call(lib, ws=P + 16) == 1                # workspace must be 256-byte aligned
+    assert call(lib, ws_bytes=16, H=4) == 3
+    # empty problems launch nothing and succeed
+    assert call(lib, batch=0, N=0) == 0
+    assert call(lib, "kda_fwd_recurrent", batch=0, N=0) == 0
+
+
+def test_read_status_rejects_null(lib):
+    assert lib.kda_read_device_status(None, None) == 1
+
+
+def test_python_binding_requires_built_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(kda, "_lib", None)
+    monkeypatch.setattr(kda, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        kda.load()

@@ -1,0 +1,172 @@
+"""GPU parity: the CUDA kernels (through the C ABI) against the fp64 CPU oracle.
+
+Tolerances (fixed for this operator): output max-abs <= 3e-2 and relative L2 <= 1e-2;
+final state relative L2 <= 1e-2; every element finite.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kda_inputs
+import kimi_delta_attention_24_b200 as kda
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+O_MAX_ABS = 3e-2
+O_REL_L2 = 1e-2
+S_REL_L2 = 1e-2
+IMPLS = ["chunked", "recurrent"]
+
+
+def rel_l2(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def run_gpu(x, impl="chunked", state_transposed=False, alias=False, dev="cuda:0"):
+    xd = x.to(dev)
+    B, T, H, K = xd.q.shape
+    N = xd.num_seqs
+    out = torch.full_like(xd.v, float("nan"))
+    s0 = xd.initial_state
+    if s0 is not None and state_transposed:
+        s0 = s0.transpose(-1, -2).contiguous()
+    final = None
+    if x.output_final_state:
+        final = s0 if alias else torch.full((N, H, K, K), float("nan"), dtype=torch.float32, device=dev)
+    ws = torch.zeros(kda.get_workspace_size(B * T, H, N), dtype=torch.uint8, device=dev)
+    fn = kda.fwd if impl == "chunked" else kda.fwd_recurrent
+    fn(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.scale, out, ws, xd.A_log, xd.dt_bias, xd.lower_bound,
+       s0, final, xd.cu_seqlens, state_transposed=state_transposed)
+    assert kda.read_device_status(ws) == 0
+    o = out.float().cpu().double().numpy()
+    s = None if final is None else final.cpu().double().numpy()
+    return o, s
+
+
+def check(o, s, o_ref, s_ref, what=""):
+    assert np.isfinite(o).all(), f"{what}: non-finite output"
+    err = np.max(np.abs(o - o_ref))
+    rl = rel_l2(o, o_ref)
+    assert err <= O_MAX_ABS and rl <= O_REL_L2, f"{what}: o max-abs {err:.3e}, rel-L2 {rl:.3e}"
+    if s_ref is not None:
+        assert np.isfinite(s).all(), f"{what}: non-finite state"
+        rs = rel_l2(s, s_ref)
+        assert rs <= S_REL_L2, f"{what}: state rel-L2 {rs:.3e}"
+    return err, rl
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("name", ["tiny", "tail", "varlen", "collinear", "usage"])
+def test_workload_parity(cuda_device, name, impl):
+    x = kda_inputs.make_workload(name)
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    o, s = run_gpu(x, impl)
+    check(o, s, o_ref, s_ref, f"{name}/{impl}")
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_prefill_sampled_heads(cuda_device, impl):
+    """The 32K x 96-head prefill, in the bench's launch configuration; the oracle recomputes a
+    sample of heads over the whole sequence."""
+    x = kda_inputs.make_workload("prefill", device=cuda_device)
+    o, s = run_gpu(x, impl)
+    heads = [0, 41, 95]
+    sl = lambda t: t[:, :, heads].contiguous().cpu()
+    o_ref, s_ref = oracle.kda_fwd(sl(x.q), sl(x.k), sl(x.v), sl(x.g), sl(x.beta), x.scale,
+                                  x.A_log[heads].cpu(), x.dt_bias[heads].cpu(), x.lower_bound,
+                                  initial_state=x.initial_state[:, heads].cpu(),
+                                  cu_seqlens=x.cu_seqlens.cpu())
+    check(o[:, :, heads], s[:, heads], o_ref, s_ref, f"prefill/{impl}")
+
+
+def test_chunk_tails_and_empty_documents(cuda_device):
+    lens = [1, 2, 15, 16, 17, 0, 63, 64, 65, 0, 127, 128, 129, 200]
+    x = kda_inputs.make_random("t", lens, 2, seed=21, state_std=0.2)
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    for impl in IMPLS:
+        o, s = run_gpu(x, impl)
+        check(o, s, o_ref, s_ref, f"tails/{impl}")
+    # zero-length documents hand their initial state through
+    np.testing.assert_array_equal(s[5], x.initial_state[5].double().numpy())
+
+
+@pytest.mark.parametrize("lb", [0.0, -0.5, -2.0])
+def test_lower_bounds(cuda_device, lb):
+    x = kda_inputs.make_random("t", [300, 77], 3, seed=22, state_std=0.1, lower_bound=lb)
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    check(*run_gpu(x), o_ref, s_ref, f"lb={lb}")
+
+
+def test_saturated_gates_and_extreme_beta(cuda_device):
+    x = kda_inputs.make_random("t", [256, 100], 2, seed=23, state_std=0.1)
+    x.g[:, :128].fill_(60.0)            # log alpha = -5 on every channel (fastest decay)
+    x.g[:, 128:200].fill_(-60.0)        # log alpha ~ 0 (no decay)
+    x.beta[:, ::3].fill_(30.0)          # beta = 1
+    x.beta[:, 1::3].fill_(-30.0)        # beta ~ 0
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    check(*run_gpu(x), o_ref, s_ref, "saturated")
+
+
+def test_transposed_state_and_aliasing(cuda_device):
+    x = kda_inputs.make_random("t", [150, 64], 2, seed=24, state_std=0.3)
+    o_ref, s_ref = oracle.fwd_inputs(x, state_transposed=True)
+    for impl in IMPLS:
+        check(*run_gpu(x, impl, state_transposed=True), o_ref, s_ref, f"transposed/{impl}")
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    for impl in IMPLS:
+        check(*run_gpu(x, impl, alias=True), o_ref, s_ref, f"alias/{impl}")
+
+
+def test_batch_mode(cuda_device):
+    x = kda_inputs.make_random("t", None, 4, seed=25, varlen=False, batch=3, seqlen=190, state_std=0.1)
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    for impl in IMPLS:
+        check(*run_gpu(x, impl), o_ref, s_ref, f"batch/{impl}")
+
+
+def test_varlen_matches_independent_documents_on_gpu(cuda_device):
+    x = kda_inputs.make_random("t", [70, 129, 5], 2, seed=26, state_std=0.1)
+    o, s = run_gpu(x)
+    cu = x.cu_seqlens.tolist()
+    for n in range(3):
+        a, b = cu[n], cu[n + 1]
+        xn = kda_inputs.KDAInputs("doc", x.q[:, a:b].contiguous(), x.k[:, a:b].contiguous(),
+                                  x.v[:, a:b].contiguous(), x.g[:, a:b].contiguous(),
+                                  x.beta[:, a:b].contiguous(), x.A_log, x.dt_bias, x.lower_bound, x.scale,
+                                  x.initial_state[n:n + 1].contiguous(),
+                                  torch.tensor([0, b - a], dtype=torch.int32))
+        on, sn = run_gpu(xn)
+        np.testing.assert_allclose(o[:, a:b], on, rtol=0, atol=1e-6)
+        np.testing.assert_allclose(s[n:n + 1], sn, rtol=0, atol=1e-6)
+
+
+def test_split_resume_on_gpu(cuda_device):
+    x = kda_inputs.make_random("t", [400], 2, seed=27, state_std=0.1)
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    t1 = 173
+    part = lambda a, b, s0: kda_inputs.KDAInputs(
+        "p", x.q[:, a:b].contiguous(), x.k[:, a:b].contiguous(), x.v[:, a:b].contiguous(),
+        x.g[:, a:b].contiguous(), x.beta[:, a:b].contiguous(), x.A_log, x.dt_bias, x.lower_bound,
+        x.scale, s0, torch.tensor([0, b - a], dtype=torch.int32))
+    oa, sa = run_gpu(part(0, t1, x.initial_state))
+    ob, sb = run_gpu(part(t1, 400, torch.from_numpy(sa).float()))
+    check(np.concatenate([oa, ob], axis=1), sb, o_ref, s_ref, "split-resume")
+
+
+def test_chunked_is_deterministic(cuda_device):
+    x = kda_inputs.make_workload("varlen")
+    o1, s1 = run_gpu(x)
+    o2, s2 = run_gpu(x)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_chunk_kda_convenience(cuda_device):
+    x = kda_inputs.make_workload("usage").to(cuda_device)
+    out, final = kda.chunk_kda(x.q, x.k, x.v, x.g, x.beta, scale=x.scale, A_log=x.A_log,
+                               dt_bias=x.dt_bias, lower_bound=x.lower_bound)
+    assert final is None
+    o_ref, _ = oracle.fwd_inputs(x.to("cpu"))
+    check(out.float().cpu().double().numpy(), None, o_ref, None, "chunk_kda")
