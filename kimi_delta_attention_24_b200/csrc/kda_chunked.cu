@@ -3,34 +3,36 @@
 // Kimi Delta Attention (FlashKDA `fwd`, fla `chunk_kda`; vLLM PR #54859 report and "What CUDA
 // Version Is Required to Use FlashKDA?", Usage Examples) is the gated delta rule
 //     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = scale S_t^T q_t.
-// The kernel walks the unit's tokens in chunks of C = 64 and uses the chunked (WY/UT) form:
-// with Gamma the in-chunk cumulative log-decay, A the strictly-lower gated key Gram matrix,
-// T = (I + A)^{-1}, W = T diag(beta) (Khat * e^Gamma), U = T diag(beta) V,
-// P = scale * tril_incl((Qhat * e^Gamma)(Khat * e^-Gamma)^T):
-//     Delta = U - W S,   O = Qtil S + P Delta,   S <- Diag(e^{Gamma_C}) S + Ktil^T Delta,
-// Qtil = scale * Qhat * e^Gamma, Ktil = Khat * e^{Gamma_C - Gamma}.  The output is rewritten as
-// O = (Qtil - P W) S + P U so that the recurrence needs two MMAs per chunk.
+// The kernel walks the unit's tokens in chunks of C = 64 and uses the chunked (WY/UT) form.  With
+// Gamma the in-chunk cumulative log-decay, Khat/Qhat the L2-normalised keys/queries,
+//   A = strict_tril(diag(beta) (Khat e^Gamma)(Khat e^-Gamma)^T),  T = (I + A)^{-1},
+//   P = scale * tril((Qhat e^Gamma)(Khat e^-Gamma)^T),  T_b = T diag(beta),
+//   W = T_b (Khat e^Gamma),  U = T_b V,  Qtil = scale Qhat e^Gamma,  Ktil = Khat e^{Gamma_C - Gamma},
+// each chunk does
+//   Delta = U - W S,   O = Qtil S + P Delta = (Qtil - P W) S + P U,
+//   S <- Diag(e^{Gamma_C}) S + Ktil^T Delta.
 //
-// Per chunk (all on-chip; HBM sees the raw inputs once and the output once):
-//   TMA       q, k, g, v tiles [64 tokens x 128] bf16, 128-byte swizzle, into shared memory.
-//   prologue  (CUDA cores) L2 norms, sigmoid(beta), safe gate, block-relative Gamma, and the bf16
-//             MMA operands with exponent referencing per 16-row sub-block (every factor within
-//             [e^-80, e^80] for lower_bound >= -5).
-//   MMA_AP    [LK; LQ] x R_I^T for the 4 sub-blocks -> gated K K^T and Q K^T blocks (TMEM).
-//   assemble  A (fp32, shared) and P (bf16 operand).
-//   solve     T = (I + A)^{-1} by fp32 forward substitution; T_beta = T diag(beta), kept as a
-//             bf16 pair hi + lo (about 16 significant bits).
-//   MMA_PT    P (T_hi + T_lo), read back as a hi + lo pair.
-//   MMA_X     [T_beta; P T_beta] x [Khat e^Gamma | V] -> [W U; PW PU] (TMEM), hi and lo parts.
-//   MMA1      [W; Qtil - PW] x S -> [W S; (Qtil - PW) S]
-//   ep1       Delta = U - W S (bf16 hi + lo operands), O = (Qtil - PW) S + P U -> global bf16.
-//   MMA2      Ktil^T (Delta_hi + Delta_lo); ep2: S = e^{Gamma_C} S + Ktil^T Delta (fp32 registers)
-//             + bf16 copy.
-// The hi + lo pairs matter when keys are nearly collinear: T then has entries close to -beta
-// that cancel against the diagonal, and the chunk's Delta rows telescope, so single bf16
-// rounding of T_beta, P T_beta or Delta would cost several percent of the state.
-// The state stays in registers (fp32 master) and shared memory (bf16 MMA operand) for the
-// whole sequence.
+// Per chunk (everything on-chip; HBM sees the raw inputs once and the output once):
+//   prologue  (CUDA cores) raw q, k, g rows straight from global memory into registers; L2 norms,
+//             sigmoid(beta), safe gate alpha = exp(lower_bound * sigmoid(exp(A_log)(g + dt_bias)));
+//             decays as running products of alpha inside each 16-row sub-block (exponent
+//             referencing: every factor stays in [e^-80, e^80] for lower_bound >= -5); the bf16 MMA
+//             operands, with the norms, beta and scale folded in.  v arrives by TMA.
+//   MMA_AP    [LK; LQ] x R_I^T per 16-row sub-block I -> the gated K K^T and Q K^T blocks (TMEM).
+//   assemble  A (fp32, shared memory) and P (bf16 operand).
+//   solve     T = (I + A)^{-1}: the four 16x16 diagonal blocks by forward substitution, then the
+//             off-diagonal blocks T_IJ = -T_II sum_K A_IK T_KJ, all in fp32; T_b as a bf16 hi+lo pair.
+//   MMA_PT    P (T_hi + T_lo), read back as a hi+lo pair.
+//   MMA_X     [T_b; P T_b] (hi + lo) x [Khat e^Gamma | V] -> [W | U; P W | P U] in TMEM.
+//   WQ        [-W; Qtil - P W] written back to TMEM as the A operand of MMA1.
+//   MMA1      accumulates [-W; Qtil - P W] x S onto [U; P U]  ->  [Delta; O].
+//   ep1       Delta (bf16 hi+lo operand), O -> global bf16.
+//   MMA2      Ktil^T (Delta_hi + Delta_lo); ep2: S = e^{Gamma_C} S + Ktil^T Delta (fp32 registers),
+//             plus its bf16 copy (the B operand of the next MMA1).
+// The hi+lo pairs matter when keys are nearly collinear: T then has entries close to -beta that
+// cancel against the diagonal, and a chunk's Delta rows telescope, so a single bf16 rounding of
+// T_b, P T_b or Delta would cost several percent of the state.  Ktil is built from the raw bf16 k
+// (its 1/|k| is applied to Delta) so that equal keys round identically.
 #include <cuda.h>
 
 #include "kda_common.cuh"
@@ -45,48 +47,50 @@ constexpr int C = 64;          // chunk length
 constexpr int D = kHeadDim;    // 128
 constexpr int kThreads = 256;  // 8 warps
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
 
-// Shared-memory map (bytes from a 1024-aligned base).
-constexpr uint32_t OFF_Q = 0;            // q tile -> Qb = scale/|q| * q * e^Gamma (bf16)
-constexpr uint32_t OFF_K = 16384;        // k tile -> Ktil (MN-major A operand of MMA2)
-constexpr uint32_t OFF_G = 32768;        // g tile -> Xk = khat * e^Gamma (MN-major B of MMA_X)
-constexpr uint32_t OFF_V = 49152;        // v tile (MN-major B of MMA_X)
-constexpr uint32_t OFF_U = 65536;        // union region (73728 bytes)
-constexpr uint32_t OFF_LKQ = OFF_U;      //   [LK; LQ] K-major, 2 k-blocks x 128 rows
-constexpr uint32_t OFF_R = OFF_U + 32768;  // R_0..R_3 K-major, 2 k-blocks x 160 rows
+// Shared-memory map (bytes from a 1024-aligned base).  "MN tile" = [2 blocks of 64 columns]
+// [64 rows][128 B] with the 128-byte swizzle; "K tile" = [2 blocks of 64 K][rows][128 B].
+constexpr uint32_t OFF_V = 0;            // v (TMA), MN-major B of MMA_X
+constexpr uint32_t OFF_XK = 16384;       // Khat e^Gamma, MN-major B of MMA_X
+constexpr uint32_t OFF_QB = 32768;       // Qtil (bf16), read when forming Qtil - P W
+constexpr uint32_t OFF_KT = 49152;       // Ktil (raw k), MN-major A of MMA2
+constexpr uint32_t OFF_SCR = 65536;      // scratch, 73728 bytes:
+constexpr uint32_t OFF_LKQ = OFF_SCR;    //   [LK; LQ] K tile, 128 rows (prologue -> MMA_AP)
+constexpr uint32_t OFF_R = OFF_SCR + 32768;  //   R_0..R_3 K tile, 160 rows (prologue -> MMA_AP)
 constexpr uint32_t R_KBLK = 160 * 128;
-constexpr uint32_t OFF_AS = OFF_U;       //   A (fp32, 64 x 68)
+constexpr uint32_t OFF_AS = OFF_SCR;             // A fp32 64 x 68 (assemble -> solve)
+constexpr uint32_t OFF_TS = OFF_SCR + 17408;     // T fp32 64 x 68 (solve)
+constexpr uint32_t OFF_YS = OFF_SCR + 17408 * 2; // solve temporaries, 3 x 16 x 16 fp32
 constexpr uint32_t AS_LD = 68;
-constexpr uint32_t OFF_WQ = OFF_U + 18432;   // [W; Qtil - PW] K-major, 2 k-blocks x 128 rows
-constexpr uint32_t OFF_DL = OFF_U + 18432;   // Delta (hi), MN-major B, 2 n-blocks x 64 rows (after MMA1)
-constexpr uint32_t OFF_DLLO = OFF_U + 34816; // Delta (lo)
-constexpr uint32_t OFF_TL = OFF_U + 51200;   // [T_lo; (P T_beta)_lo] 128 x 64, K-major
-constexpr uint32_t OFF_TP = OFF_U + 73728;   // [T_beta; P] (later [T_beta; P T_beta]) 128 x 64
-constexpr uint32_t OFF_S = OFF_TP + 16384;   // S bf16, MN-major B, 2 n-blocks x 128 rows
-constexpr uint32_t OFF_SC = OFF_S + 32768;   // scalars
-constexpr uint32_t SC_BETA = 0;              // float[64]
-constexpr uint32_t SC_IK = 256;              // float[64] 1/|k|
-constexpr uint32_t SC_IQS = 512;             // float[64] scale/|q|
-constexpr uint32_t SC_GAM = 768;             // float[128] e^{Gamma_C}
-constexpr uint32_t SC_CARRY = 1280;          // float[4][128]
-constexpr uint32_t SC_LEND = 3328;           // float[4][128]
-constexpr uint32_t SC_BAR = 5376;            // 2 mbarriers
-constexpr uint32_t SC_TMEM = 5392;
-constexpr uint32_t SC_ABORT = 5396;
-constexpr uint32_t SMEM_BYTES = OFF_SC + 5504;
+constexpr uint32_t OFF_TP = OFF_SCR + 40960;     // [T_hi; P -> (P T)_hi] 128 x 64, K tile
+constexpr uint32_t OFF_TL = OFF_SCR + 57344;     // [T_lo; (P T)_lo]
+constexpr uint32_t OFF_DL = OFF_SCR;             // Delta hi, MN tile (ep1 -> MMA2)
+constexpr uint32_t OFF_DLLO = OFF_SCR + 16384;   // Delta lo
+constexpr uint32_t OFF_S = OFF_SCR + 73728;      // S bf16, MN-major B of MMA1, 2 blocks x 128 rows
+constexpr uint32_t OFF_SC = OFF_S + 32768;       // scalars
+constexpr uint32_t SC_BETA = 0;                  // float[64]
+constexpr uint32_t SC_IK = 256;                  // float[64] 1/|k_r| (0 for rows past the end)
+constexpr uint32_t SC_GAM = 512;                 // float[128] e^{Gamma_C}
+constexpr uint32_t SC_TOT = 1024;                // float[8][128] per-warp alpha products
+constexpr uint32_t SC_BAR = 5120;                // 2 mbarriers
+constexpr uint32_t SC_TMEM = 5136;
+constexpr uint32_t SC_ABORT = 5140;
+constexpr uint32_t SMEM_BYTES = OFF_SC + 5248;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 
 // first row of R_I inside the R tile: 0, 16, 48, 96 (R_I holds 16 (I+1) rows)
 __host__ __device__ constexpr uint32_t row_off(int I) { return 8u * I * (I + 1); }
 
-// TMEM column map (512 allocated).
-constexpr uint32_t TM_AP = 0;    // 4 x 64 (sub-block products), later P T_beta, later [W PW | U PU]
-constexpr uint32_t TM_X = 0;
-constexpr uint32_t TM_REC = 256; // MMA1 / MMA2 results
-constexpr uint32_t kTmemCols = 512;
+// TMEM columns: AP products at row_off(I) (N = 16 (I+1)), then P T at 0..63, then
+// [W PW] at 0..127 and [U PU] at 128..255; [-W; Qtil - PW] packed bf16 at 0..63; MMA1 and MMA2
+// accumulate at 128..255.
+constexpr uint32_t TM_WQ = 0;
+constexpr uint32_t TM_UP = 128;
+constexpr uint32_t kTmemCols = 256;
 
 struct TensorMaps {
-  CUtensorMap q, k, v, g;
+  CUtensorMap v;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -96,22 +100,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
 }
-// Eight floats as a bf16 pair: hi = bf16(x), lo = bf16(x - hi).
-__device__ __forceinline__ void split_pack(const float* x, uint4& hi, uint4& lo) {
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(x[2 * u], x[2 * u + 1]);
-    const float2 bf = __bfloat1622float2(b);
-    const __nv_bfloat162 c = __floats2bfloat162_rn(x[2 * u] - bf.x, x[2 * u + 1] - bf.y);
-    h[u] = *reinterpret_cast<const uint32_t*>(&b);
-    l[u] = *reinterpret_cast<const uint32_t*>(&c);
-  }
-  hi = make_uint4(h[0], h[1], h[2], h[3]);
-  lo = make_uint4(l[0], l[1], l[2], l[3]);
+// x as a bf16 pair hi = bf16(x), lo = bf16(x - hi), two values at a time.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 __device__ __forceinline__ float fast_sigmoid(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
-
+__device__ __forceinline__ uint2 ldg_u2(const __nv_bfloat16* p) {
+  return __ldg(reinterpret_cast<const uint2*>(p));
+}
 __device__ __forceinline__ void bar_sync() { __syncthreads(); }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -121,15 +121,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(sm);
   float* sc_beta = reinterpret_cast<float*>(sm + OFF_SC + SC_BETA);
   float* sc_ik = reinterpret_cast<float*>(sm + OFF_SC + SC_IK);
-  float* sc_iqs = reinterpret_cast<float*>(sm + OFF_SC + SC_IQS);
   float* sc_gam = reinterpret_cast<float*>(sm + OFF_SC + SC_GAM);
-  float* sc_carry = reinterpret_cast<float*>(sm + OFF_SC + SC_CARRY);
-  float* sc_lend = reinterpret_cast<float*>(sm + OFF_SC + SC_LEND);
+  float* sc_tot = reinterpret_cast<float*>(sm + OFF_SC + SC_TOT);
   uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + OFF_SC + SC_BAR);
   uint64_t* mma_bar = tma_bar + 1;
   uint32_t* sc_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SC + SC_TMEM);
   volatile int* sc_abort = reinterpret_cast<volatile int*>(sm + OFF_SC + SC_ABORT);
   float* As = reinterpret_cast<float*>(sm + OFF_AS);
+  float* Ts = reinterpret_cast<float*>(sm + OFF_TS);
+  float* Ys = reinterpret_cast<float*>(sm + OFF_YS);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -146,10 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(mma_bar, 1);
     *sc_abort = 0;
     fence_mbar_init();
-    prefetch_tmap(&maps.q);
-    prefetch_tmap(&maps.k);
     prefetch_tmap(&maps.v);
-    prefetch_tmap(&maps.g);
   }
   if (warp == 0) {
     tmem_alloc(sc_tmem, kTmemCols);
@@ -159,8 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   bar_sync();
   tc_fence_after();
   const uint32_t tmem = *sc_tmem;
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;  // this warp's TMEM lane quarter
 
-  // ---- initial state: thread owns row k = 32*quarter + lane, columns [64*half, 64*half + 64)
+  // ---- state: thread owns row k = 32*quarter + lane, columns [64*half, 64*half + 64)
   const int srow = 32 * quarter + lane;
   const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
   float S[64];
@@ -187,34 +185,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   store_state_bf16();
 
-  // per-lane constants of the prologue mapping: warp w owns chunk rows 8w..8w+7, lane owns
-  // channels 4*lane .. 4*lane+3
+  // prologue mapping: warp w owns chunk rows 8w..8w+7, lane owns channels 4*lane..4*lane+3
   const float gate_a = __expf(p.A_log[h]);
   const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+  // exp(-a (g + dt)) = exp2(ga * g + gb)
+  const float ga = -gate_a * kLog2e;
+  const float gb[4] = {ga * dtb.x, ga * dtb.y, ga * dtb.z, ga * dtb.w};
+  const float lb2 = p.lower_bound * kLog2e;
   const int kb = lane >> 4;                       // 64-channel block
   const uint32_t lane_chunk = (lane & 15) >> 1;   // 16-byte chunk within the 128-byte row
   const uint32_t lane_sub = (lane & 1) * 8;       // byte within the chunk
-  const int blk = warp >> 1;                      // sub-block of this warp's rows
+  const int blk = warp >> 1;                      // 16-row sub-block of this warp's rows
+  const bool upper_half = warp & 1;               // rows 8..15 of the sub-block
 
   uint32_t tma_phase = 0, mma_phase = 0;
-  auto issue_tma = [&](int64_t t0, bool qgv, bool kk) {
-    const int c2 = (int)t0;
-    for (int b = 0; b < 2; ++b) {
-      if (qgv) {
-        tma_load_3d(sm + OFF_Q + b * 8192, &maps.q, tma_bar, 64 * b, h, c2);
-        tma_load_3d(sm + OFF_G + b * 8192, &maps.g, tma_bar, 64 * b, h, c2);
-        tma_load_3d(sm + OFF_V + b * 8192, &maps.v, tma_bar, 64 * b, h, c2);
-      }
-      if (kk) tma_load_3d(sm + OFF_K + b * 8192, &maps.k, tma_bar, 64 * b, h, c2);
-    }
-  };
   if (tid == 0 && nchunks > 0) {
-    mbar_arrive_expect_tx(tma_bar, 4 * 16384);
-    issue_tma(bos, true, true);
+    mbar_arrive_expect_tx(tma_bar, 16384);
+    tma_load_3d(sm + OFF_V, &maps.v, tma_bar, 0, h, (int)bos);
+    tma_load_3d(sm + OFF_V + 8192, &maps.v, tma_bar, 64, h, (int)bos);
   }
 
-  // Waits on an mbarrier phase; on timeout records the device error.  Every thread then meets
-  // at a barrier and reads the shared abort flag, so all threads leave the loop together.
   auto wait_all = [&](uint64_t* bar, uint32_t& phase) -> bool {
     const bool ok = mbar_wait(bar, phase, kWaitLimitNs);
     phase ^= 1u;
@@ -225,7 +215,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     bar_sync();
     return *sc_abort == 0;
   };
-  // Makes this thread's shared-memory writes and TMEM reads visible/ordered before an MMA issue.
   auto publish = [&]() {
     fence_proxy_async();
     tc_fence_before();
@@ -235,41 +224,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = bos + (int64_t)c * C;
     const int len = (int)((eos - t0) < (int64_t)C ? (eos - t0) : (int64_t)C);
-    if (!wait_all(tma_bar, tma_phase)) break;
 
     // ================================================================ prologue
     {
-      // raw q, k (bf16) of this thread's 8 rows x 4 channels
       uint2 qr[8], kr[8];
-      float la[8][4];
+      float al[8][4];
       float ssq[8], ssk[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = 8 * warp + i;
-        const uint32_t off = kb * 8192 + sw128(r, lane_chunk) + lane_sub;
         const bool valid = r < len;
-        qr[i] = valid ? *reinterpret_cast<const uint2*>(sm + OFF_Q + off) : make_uint2(0, 0);
-        kr[i] = valid ? *reinterpret_cast<const uint2*>(sm + OFF_K + off) : make_uint2(0, 0);
-        const uint2 gr = *reinterpret_cast<const uint2*>(sm + OFF_G + off);
+        const size_t off = ((size_t)(t0 + r) * H + h) * D + 4 * lane;
+        uint2 gr = make_uint2(0, 0);
+        qr[i] = make_uint2(0, 0);
+        kr[i] = make_uint2(0, 0);
+        if (valid) {
+          qr[i] = ldg_u2(p.q + off);
+          kr[i] = ldg_u2(p.k + off);
+          gr = ldg_u2(p.g + off);
+        }
         const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
         const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
         ssq[i] = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
         ssk[i] = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
         const float2 g01 = unpack_bf16(gr.x), g23 = unpack_bf16(gr.y);
-        const float lb = p.lower_bound;
-        la[i][0] = valid ? lb * fast_sigmoid(gate_a * (g01.x + dtb.x)) : 0.f;
-        la[i][1] = valid ? lb * fast_sigmoid(gate_a * (g01.y + dtb.y)) : 0.f;
-        la[i][2] = valid ? lb * fast_sigmoid(gate_a * (g23.x + dtb.z)) : 0.f;
-        la[i][3] = valid ? lb * fast_sigmoid(gate_a * (g23.y + dtb.w)) : 0.f;
-      }
-      // row sums of squares: transpose-reduce 16 values over the 32 lanes
-      float v16[16];
+        const float gv[4] = {g01.x, g01.y, g23.x, g23.y};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v16[i] = ssq[i];
-        v16[8 + i] = ssk[i];
+        for (int j = 0; j < 4; ++j) {
+          // alpha = 2^(lb*log2e * sigmoid(a (g + dt)))
+          const float z = exp2f(fmaf(ga, gv[j], gb[j]));
+          const float sig = __fdividef(1.0f, 1.0f + z);
+          al[i][j] = valid ? exp2f(lb2 * sig) : 1.0f;
+        }
       }
+      // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
+      // total of value (l >> 1): q rows 0..7, then k rows 0..7
+      float inv;
       {
+        float v16[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v16[i] = ssq[i];
+          v16[8 + i] = ssk[i];
+        }
         const bool b4 = lane & 16;
         float w8[8];
 #pragma unroll
@@ -297,66 +294,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool b1 = lane & 2;
         float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
         w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
-        // lane holds the total of index (lane >> 1): q rows 0..7, then k rows 0..7
-        const float inv = rsqrtf(w1 + kL2Eps);
+        inv = rsqrtf(w1 + kL2Eps);
+      }
+      // beta of row 8w + lane (lanes 0..7), broadcast to the warp
+      float beta_l = 0.f;
+      if (lane < 8) {
+        const int r = 8 * warp + lane;
+        if (r < len) beta_l = fast_sigmoid(__bfloat162float(p.beta[(size_t)(t0 + r) * H + h]));
+        sc_beta[r] = beta_l;
+      }
+      float iq[8], ik[8], bt[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          ssq[i] = __shfl_sync(0xffffffffu, inv, 2 * i);        // 1/|q_r|
-          ssk[i] = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);   // 1/|k_r|
-        }
+      for (int i = 0; i < 8; ++i) {
+        iq[i] = __shfl_sync(0xffffffffu, inv, 2 * i) * p.scale;
+        ik[i] = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);
+        bt[i] = __shfl_sync(0xffffffffu, beta_l, i);
       }
       if (lane < 8) {
         const int r = 8 * warp + lane;
-        float ik = ssk[0], iq = ssq[0];
+        float v = ik[0];
 #pragma unroll
-        for (int i = 1; i < 8; ++i) {
-          if (lane == i) {
-            ik = ssk[i];
-            iq = ssq[i];
-          }
-        }
-        const bool valid = r < len;
-        sc_ik[r] = valid ? ik : 0.f;
-        sc_iqs[r] = valid ? p.scale * iq : 0.f;
-        const float rb = valid ? __bfloat162float(p.beta[(size_t)(t0 + r) * H + h]) : 0.f;
-        sc_beta[r] = valid ? fast_sigmoid(rb) : 0.f;
+        for (int i = 1; i < 8; ++i) v = (lane == i) ? ik[i] : v;
+        sc_ik[r] = (r < len) ? v : 0.f;
       }
-      // in-block cumulative log-decay (block = 16 rows = warps 2J, 2J+1)
+      // running products of alpha over this warp's 8 rows (prefix in place) and their suffixes
+      float suf[8][4];
 #pragma unroll
-      for (int i = 1; i < 8; ++i)
+      for (int j = 0; j < 4; ++j) {
+        suf[7][j] = 1.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) la[i][j] += la[i - 1][j];
-      if ((warp & 1) == 0)
-        reinterpret_cast<float4*>(sc_carry + blk * 128)[lane] = make_float4(la[7][0], la[7][1], la[7][2], la[7][3]);
-      bar_sync();
-      if (warp & 1) {
-        const float4 cr = reinterpret_cast<const float4*>(sc_carry + blk * 128)[lane];
+        for (int i = 6; i >= 0; --i) suf[i][j] = suf[i + 1][j] * al[i + 1][j];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          la[i][0] += cr.x;
-          la[i][1] += cr.y;
-          la[i][2] += cr.z;
-          la[i][3] += cr.w;
-        }
-        reinterpret_cast<float4*>(sc_lend + blk * 128)[lane] = make_float4(la[7][0], la[7][1], la[7][2], la[7][3]);
+        for (int i = 1; i < 8; ++i) al[i][j] *= al[i - 1][j];
       }
+      reinterpret_cast<float4*>(sc_tot + warp * 128)[lane] = make_float4(al[7][0], al[7][1], al[7][2], al[7][3]);
       bar_sync();
-      // b_J = e^{lambda_end(J)} for the 4 blocks, this lane's channels
+      // sub-block totals b_J = e^{Gamma at the end of J - Gamma at its start}
       float bJ[4][4];
 #pragma unroll
       for (int J = 0; J < 4; ++J) {
-        const float4 le = reinterpret_cast<const float4*>(sc_lend + J * 128)[lane];
-        bJ[J][0] = __expf(le.x);
-        bJ[J][1] = __expf(le.y);
-        bJ[J][2] = __expf(le.z);
-        bJ[J][3] = __expf(le.w);
+        const float4 t0v = reinterpret_cast<const float4*>(sc_tot + (2 * J) * 128)[lane];
+        const float4 t1v = reinterpret_cast<const float4*>(sc_tot + (2 * J + 1) * 128)[lane];
+        bJ[J][0] = t0v.x * t1v.x;
+        bJ[J][1] = t0v.y * t1v.y;
+        bJ[J][2] = t0v.z * t1v.z;
+        bJ[J][3] = t0v.w * t1v.w;
       }
-      float lend[4];
-      {
-        const float4 le = reinterpret_cast<const float4*>(sc_lend + blk * 128)[lane];
-        lend[0] = le.x; lend[1] = le.y; lend[2] = le.z; lend[3] = le.w;
-      }
-      float pre[4], post[4], rb[4], mid[4][4];
+      const float4 partner = reinterpret_cast<const float4*>(sc_tot + (warp ^ 1) * 128)[lane];
+      const float pt[4] = {partner.x, partner.y, partner.z, partner.w};
+      // e_i = prod of alpha from the sub-block start to row i; f_i = prod after row i to its end
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (upper_half) al[i][j] *= pt[j];
+          else suf[i][j] *= pt[j];
+        }
+      float pre[4], post[4], cI[4][4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float a = 1.f, z = 1.f;
@@ -367,23 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         pre[j] = a;
         post[j] = z;
-        rb[j] = 1.0f / bJ[blk][j];
-        // mid[I][j] = prod_{J = blk+1}^{I-1} b_J  (for I > blk)
         float m = 1.f;
 #pragma unroll
         for (int I = 0; I < 4; ++I) {
-          mid[I][j] = m;
+          cI[I][j] = (I == blk) ? 1.0f / bJ[blk][j] : m;
           if (I > blk) m *= bJ[I][j];
         }
       }
-      if (warp == 0) {
-        float4 gm;
-        gm.x = bJ[0][0] * bJ[1][0] * bJ[2][0] * bJ[3][0];
-        gm.y = bJ[0][1] * bJ[1][1] * bJ[2][1] * bJ[3][1];
-        gm.z = bJ[0][2] * bJ[1][2] * bJ[2][2] * bJ[3][2];
-        gm.w = bJ[0][3] * bJ[1][3] * bJ[2][3] * bJ[3][3];
-        reinterpret_cast<float4*>(sc_gam)[lane] = gm;
-      }
+      if (warp == 0)
+        reinterpret_cast<float4*>(sc_gam)[lane] =
+            make_float4(bJ[0][0] * bJ[1][0] * bJ[2][0] * bJ[3][0], bJ[0][1] * bJ[1][1] * bJ[2][1] * bJ[3][1],
+                        bJ[0][2] * bJ[1][2] * bJ[2][2] * bJ[3][2], bJ[0][3] * bJ[1][3] * bJ[2][3] * bJ[3][3]);
       // operands, one row at a time
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -392,47 +380,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
         const float qv[4] = {q01.x, q01.y, q23.x, q23.y};
         const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
-        float e[4], f[4];
+        float lk[4], lq[4], kf[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          e[j] = __expf(la[i][j]);
-          f[j] = __expf(lend[j] - la[i][j]);
+          const float kh = kv[j] * ik[i];
+          lq[j] = qv[j] * iq[i] * al[i][j];   // scale * qhat * e
+          lk[j] = kh * al[i][j];              // khat * e
+          kf[j] = kh * suf[i][j];             // khat * f
         }
-        const float iq = ssq[i] * p.scale, ik = ssk[i];
-        const uint32_t off64 = kb * 8192 + sw128(r, lane_chunk) + lane_sub;     // 64-row tiles
-        // LK (row r) and LQ (row 64 + r): K-major [2][128 rows][128 B]
-        {
-          const uint32_t offk = kb * 16384 + sw128(r, lane_chunk) + lane_sub;
-          const uint32_t offq = kb * 16384 + sw128(64 + r, lane_chunk) + lane_sub;
-          *reinterpret_cast<uint2*>(sm + OFF_LKQ + offk) =
-              make_uint2(pack_bf16(kv[0] * e[0], kv[1] * e[1]), pack_bf16(kv[2] * e[2], kv[3] * e[3]));
-          *reinterpret_cast<uint2*>(sm + OFF_LKQ + offq) =
-              make_uint2(pack_bf16(qv[0] * e[0], qv[1] * e[1]), pack_bf16(qv[2] * e[2], qv[3] * e[3]));
-        }
-        // R_I rows for I >= blk
+        const uint32_t offk = kb * 16384 + sw128(r, lane_chunk) + lane_sub;
+        const uint32_t offq = kb * 16384 + sw128(64 + r, lane_chunk) + lane_sub;
+        const uint32_t off64 = kb * 8192 + sw128(r, lane_chunk) + lane_sub;
+        const float b = bt[i];
+        *reinterpret_cast<uint2*>(sm + OFF_LKQ + offk) =
+            make_uint2(pack_bf16(lk[0] * b, lk[1] * b), pack_bf16(lk[2] * b, lk[3] * b));
+        *reinterpret_cast<uint2*>(sm + OFF_LKQ + offq) =
+            make_uint2(pack_bf16(lq[0], lq[1]), pack_bf16(lq[2], lq[3]));
 #pragma unroll
         for (int I = 0; I < 4; ++I) {
           if (I < blk) continue;
-          float fac[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) fac[j] = (I == blk) ? f[j] * rb[j] : f[j] * mid[I][j];
-          const uint32_t row = row_off(I) + r;
-          const uint32_t off = kb * R_KBLK + sw128(row, lane_chunk) + lane_sub;
+          const uint32_t off = kb * R_KBLK + sw128(row_off(I) + r, lane_chunk) + lane_sub;
           *reinterpret_cast<uint2*>(sm + OFF_R + off) =
-              make_uint2(pack_bf16(kv[0] * fac[0], kv[1] * fac[1]), pack_bf16(kv[2] * fac[2], kv[3] * fac[3]));
+              make_uint2(pack_bf16(kf[0] * cI[I][0], kf[1] * cI[I][1]), pack_bf16(kf[2] * cI[I][2], kf[3] * cI[I][3]));
         }
-        // Xk = khat e^Gamma (in place of g), Qb = scale qhat e^Gamma (in place of q),
-        // Ktil = k e^{Gamma_C - Gamma} (in place of k; 1/|k| is folded into Delta)
-        *reinterpret_cast<uint2*>(sm + OFF_G + off64) =
-            make_uint2(pack_bf16(kv[0] * e[0] * pre[0] * ik, kv[1] * e[1] * pre[1] * ik),
-                       pack_bf16(kv[2] * e[2] * pre[2] * ik, kv[3] * e[3] * pre[3] * ik));
-        *reinterpret_cast<uint2*>(sm + OFF_Q + off64) =
-            make_uint2(pack_bf16(qv[0] * e[0] * pre[0] * iq, qv[1] * e[1] * pre[1] * iq),
-                       pack_bf16(qv[2] * e[2] * pre[2] * iq, qv[3] * e[3] * pre[3] * iq));
-        *reinterpret_cast<uint2*>(sm + OFF_K + off64) =
-            make_uint2(pack_bf16(kv[0] * f[0] * post[0], kv[1] * f[1] * post[1]),
-                       pack_bf16(kv[2] * f[2] * post[2], kv[3] * f[3] * post[3]));
-        if (r >= len) *reinterpret_cast<uint2*>(sm + OFF_V + off64) = make_uint2(0, 0);
+        *reinterpret_cast<uint2*>(sm + OFF_XK + off64) =
+            make_uint2(pack_bf16(lk[0] * pre[0], lk[1] * pre[1]), pack_bf16(lk[2] * pre[2], lk[3] * pre[3]));
+        *reinterpret_cast<uint2*>(sm + OFF_QB + off64) =
+            make_uint2(pack_bf16(lq[0] * pre[0], lq[1] * pre[1]), pack_bf16(lq[2] * pre[2], lq[3] * pre[3]));
+        *reinterpret_cast<uint2*>(sm + OFF_KT + off64) =
+            make_uint2(pack_bf16(kv[0] * suf[i][0] * post[0], kv[1] * suf[i][1] * post[1]),
+                       pack_bf16(kv[2] * suf[i][2] * post[2], kv[3] * suf[i][3] * post[3]));
       }
     }
     publish();
@@ -440,14 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ MMA_AP
     if (tid == 0) {
       tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
 #pragma unroll
       for (int I = 0; I < 4; ++I) {
+        const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t a = sdesc_sw128(sbase + OFF_LKQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
           const uint64_t b = sdesc_sw128(sbase + OFF_R + (ks >> 2) * R_KBLK + row_off(I) * 128 + (ks & 3) * 32, 16, 1024);
-          umma_bf16(tmem + TM_AP + 64 * I, a, b, idesc, ks > 0);
+          umma_bf16(tmem + row_off(I), a, b, idesc, ks > 0);
         }
       }
       umma_commit(mma_bar);
@@ -461,45 +438,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool qside = R >= 64;
       const int r = R & 63;
       const int Ib = r >> 4;
-      const int q2 = quarter & 1;         // rows 32*q2 .. 32*q2+31 of this side
-      // s-range [32*half, 32*half+32) is entirely above the diagonal for rows < 32
-      const bool skip = (half == 1) && (q2 == 0);
-      float dsel[32];
+      const int q2 = quarter & 1;         // rows 32*q2 .. 32*q2+31 of this side: blocks 2 q2, 2 q2 + 1
+      const bool skip = (half == 1) && (q2 == 0);  // s in [32, 64) lies above the diagonal there
+      float d[32];
       if (!skip) {
         float d0[32], d1[32];
-        const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
-        tmem_ld32(tmem + lane_addr + TM_AP + 64 * (2 * q2) + 32 * half, d0);
-        tmem_ld32(tmem + lane_addr + TM_AP + 64 * (2 * q2 + 1) + 32 * half, d1);
+        tmem_ld32(tmem + lane_base + row_off(2 * q2) + 32 * half, d0);
+        tmem_ld32(tmem + lane_base + row_off(2 * q2 + 1) + 32 * half, d1);
         const bool odd = Ib & 1;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dsel[j] = odd ? d1[j] : d0[j];
+        for (int j = 0; j < 32; ++j) d[j] = odd ? d1[j] : d0[j];
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dsel[j] = 0.f;
+        for (int j = 0; j < 32; ++j) d[j] = 0.f;
       }
       if (!qside) {
-        const float rowscale = sc_beta[r] * sc_ik[r];
         float* dst = As + r * AS_LD + 32 * half;
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-          float4 o;
           const int s = 32 * half + j;
-          o.x = (s + 0 < r) ? rowscale * sc_ik[s + 0] * dsel[j + 0] : 0.f;
-          o.y = (s + 1 < r) ? rowscale * sc_ik[s + 1] * dsel[j + 1] : 0.f;
-          o.z = (s + 2 < r) ? rowscale * sc_ik[s + 2] * dsel[j + 2] : 0.f;
-          o.w = (s + 3 < r) ? rowscale * sc_ik[s + 3] * dsel[j + 3] : 0.f;
+          float4 o;
+          o.x = (s + 0 < r) ? d[j + 0] : 0.f;
+          o.y = (s + 1 < r) ? d[j + 1] : 0.f;
+          o.z = (s + 2 < r) ? d[j + 2] : 0.f;
+          o.w = (s + 3 < r) ? d[j + 3] : 0.f;
           *reinterpret_cast<float4*>(dst + j) = o;
         }
       } else {
-        const float rowscale = sc_iqs[r];
 #pragma unroll
         for (int cch = 0; cch < 4; ++cch) {
           float v8[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int j = 8 * cch + u;
-            const int s = 32 * half + j;
-            v8[u] = (s <= r) ? rowscale * sc_ik[s] * dsel[j] : 0.f;
+            const int s = 32 * half + 8 * cch + u;
+            v8[u] = (s <= r) ? d[8 * cch + u] : 0.f;
           }
           uint4 w;
           w.x = pack_bf16(v8[0], v8[1]);
@@ -514,39 +486,96 @@ __global__ void __launch_bounds__(kThreads, 1)
     bar_sync();
 
     // ================================================================ solve T = (I + A)^{-1}
-    if (tid < 64) {
-      const int j = tid;
-      float x[C];
+    // diagonal 16x16 blocks: warp I, lane j < 16 computes column j by forward substitution
+    if (warp < 4 && lane < 16) {
+      const int I = warp, j = lane;
+      const float* a = As + (16 * I) * AS_LD + 16 * I;
+      float x[16];
 #pragma unroll
-      for (int s = 0; s < C; ++s) x[s] = (s == j) ? 1.f : 0.f;
+      for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
 #pragma unroll
-      for (int r = 1; r < C; ++r) {
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      for (int i = 1; i < 16; ++i) {
+        float acc = 0.f;
 #pragma unroll
-        for (int s = 0; s < r; s += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(As + r * AS_LD + s);
-          a0 = fmaf(a.x, x[s], a0);
-          if (s + 1 < C) a1 = fmaf(a.y, x[s + 1], a1);
-          if (s + 2 < C) a2 = fmaf(a.z, x[s + 2], a2);
-          if (s + 3 < C) a3 = fmaf(a.w, x[s + 3], a3);
-        }
-        const float val = -((a0 + a1) + (a2 + a3));
-        x[r] = (r > j) ? val : x[r];
+        for (int m = 0; m < i; ++m) acc = fmaf(a[i * AS_LD + m], x[m], acc);
+        x[i] = (i > j) ? -acc : x[i];
       }
-      const float bj = sc_beta[j];
-      const uint32_t cbyte = (uint32_t)j * 2;
 #pragma unroll
-      for (int r = 0; r < C; ++r) {
-        const uint32_t off = sw128(r, cbyte >> 4) + (cbyte & 15);
-        const float tb = x[r] * bj;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(tb);
-        *reinterpret_cast<__nv_bfloat16*>(sm + OFF_TP + off) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(sm + OFF_TL + off) = __float2bfloat16_rn(tb - __bfloat162float(hi));
+      for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = x[i];
+    }
+    bar_sync();
+    // off-diagonal blocks by distance dd below the diagonal: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
+#pragma unroll 1
+    for (int dd = 1; dd < 4; ++dd) {
+      const int nblk = 4 - dd;
+      const int job = tid;                  // (block, row i, 4-column group)
+      const bool active = job < nblk * 64;
+      const int bI = dd + job / 64;         // block row I (J = I - dd)
+      const int bJ = bI - dd;
+      const int i = (job % 64) >> 2, cg = job & 3;
+      if (active) {
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        for (int K = bJ; K < bI; ++K) {
+          const float* arow = As + (16 * bI + i) * AS_LD + 16 * K;
+          const float* tcol = Ts + (16 * K) * AS_LD + 16 * bJ + 4 * cg;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const float a = arow[m];
+            const float4 t = *reinterpret_cast<const float4*>(tcol + m * AS_LD);
+            y0 = fmaf(a, t.x, y0);
+            y1 = fmaf(a, t.y, y1);
+            y2 = fmaf(a, t.z, y2);
+            y3 = fmaf(a, t.w, y3);
+          }
+        }
+        *reinterpret_cast<float4*>(Ys + (job / 64) * 256 + i * 16 + 4 * cg) = make_float4(y0, y1, y2, y3);
+      }
+      bar_sync();
+      if (active) {
+        const float* trow = Ts + (16 * bI + i) * AS_LD + 16 * bI;
+        const float* ycol = Ys + (job / 64) * 256 + 4 * cg;
+        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float t = (m <= i) ? trow[m] : 0.f;
+          const float4 y = *reinterpret_cast<const float4*>(ycol + m * 16);
+          z0 = fmaf(t, y.x, z0);
+          z1 = fmaf(t, y.y, z1);
+          z2 = fmaf(t, y.z, z2);
+          z3 = fmaf(t, y.w, z3);
+        }
+        *reinterpret_cast<float4*>(Ts + (16 * bI + i) * AS_LD + 16 * bJ + 4 * cg) = make_float4(-z0, -z1, -z2, -z3);
+      }
+      bar_sync();
+    }
+    // T_b = T diag(beta) as hi/lo bf16 into rows 0..63 of TP / TL (upper blocks are zero)
+    {
+      const int r = tid >> 2, c16 = tid & 3;   // row r, columns 16*c16 .. 16*c16+15
+      const int I = r >> 4;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c0 = 16 * c16 + 8 * hh;
+        uint4 wh, wl;
+        if (c16 > I) {
+          wh = make_uint4(0, 0, 0, 0);
+          wl = wh;
+        } else {
+          const float4 t0v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0);
+          const float4 t1v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0 + 4);
+          const float4 b0 = *reinterpret_cast<const float4*>(sc_beta + c0);
+          const float4 b1 = *reinterpret_cast<const float4*>(sc_beta + c0 + 4);
+          split2(t0v.x * b0.x, t0v.y * b0.y, wh.x, wl.x);
+          split2(t0v.z * b0.z, t0v.w * b0.w, wh.y, wl.y);
+          split2(t1v.x * b1.x, t1v.y * b1.y, wh.z, wl.z);
+          split2(t1v.z * b1.z, t1v.w * b1.w, wh.w, wl.w);
+        }
+        *reinterpret_cast<uint4*>(sm + OFF_TP + sw128(r, c0 >> 3)) = wh;
+        *reinterpret_cast<uint4*>(sm + OFF_TL + sw128(r, c0 >> 3)) = wl;
       }
     }
     publish();
 
-    // ================================================================ MMA_PT: [T_beta; P] x T_beta
+    // ================================================================ MMA_PT: [T_hi; P] x (T_hi + T_lo)
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
@@ -554,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t a = sdesc_sw128(sbase + OFF_TP + (ks & 3) * 32, 16, 1024);
         const uint64_t b = sdesc_sw128(sbase + (ks < 4 ? OFF_TP : OFF_TL) + (ks & 3) * 2048, 8192, 1024);
-        umma_bf16(tmem + TM_AP, a, b, idesc, ks > 0);
+        umma_bf16(tmem, a, b, idesc, ks > 0);
       }
       umma_commit(mma_bar);
     }
@@ -563,89 +592,94 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (quarter >= 2) {
       const int r = 32 * quarter + lane - 64;
       float d[32];
-      tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + TM_AP + 32 * half, d);
+      tmem_ld32(tmem + lane_base + 32 * half, d);
 #pragma unroll
       for (int cch = 0; cch < 4; ++cch) {
         uint4 wh, wl;
-        split_pack(&d[8 * cch], wh, wl);
+        split2(d[8 * cch + 0], d[8 * cch + 1], wh.x, wl.x);
+        split2(d[8 * cch + 2], d[8 * cch + 3], wh.y, wl.y);
+        split2(d[8 * cch + 4], d[8 * cch + 5], wh.z, wl.z);
+        split2(d[8 * cch + 6], d[8 * cch + 7], wh.w, wl.w);
         *reinterpret_cast<uint4*>(sm + OFF_TP + sw128(64 + r, 4 * half + cch)) = wh;
         *reinterpret_cast<uint4*>(sm + OFF_TL + sw128(64 + r, 4 * half + cch)) = wl;
       }
     }
     publish();
 
-    // ================================================================ MMA_X: [T_beta; P T_beta] x [Xk | V]
+    // ================================================================ MMA_X: [T_b; P T_b] x [Xk | V]
+    if (!wait_all(tma_bar, tma_phase)) break;   // v tile of this chunk
+    if (len < C) {  // rows past the document end (another document's or zero-filled) -> 0
+      for (int idx = tid; idx < 2 * (C - len) * 8; idx += kThreads) {
+        const int blk2 = idx / ((C - len) * 8), rem = idx % ((C - len) * 8);
+        const int r = len + rem / 8;
+        *reinterpret_cast<uint4*>(sm + OFF_V + blk2 * 8192 + sw128(r, rem & 7)) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async();
+      bar_sync();
+    }
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t a = sdesc_sw128(sbase + (ks < 4 ? OFF_TP : OFF_TL) + (ks & 3) * 32, 16, 1024);
-        const uint64_t bk = sdesc_sw128(sbase + OFF_G + (ks & 3) * 2048, 8192, 1024);
+        const uint64_t bk = sdesc_sw128(sbase + OFF_XK + (ks & 3) * 2048, 8192, 1024);
         const uint64_t bv = sdesc_sw128(sbase + OFF_V + (ks & 3) * 2048, 8192, 1024);
-        umma_bf16(tmem + TM_X, a, bk, idesc, ks > 0);
-        umma_bf16(tmem + TM_X + 128, a, bv, idesc, ks > 0);
+        umma_bf16(tmem + TM_WQ, a, bk, idesc, ks > 0);
+        umma_bf16(tmem + TM_UP, a, bv, idesc, ks > 0);
       }
       umma_commit(mma_bar);
     }
     if (!wait_all(mma_bar, mma_phase)) break;
     tc_fence_after();
+    // the v tile is free: fetch the next chunk's
+    if (tid == 0 && c + 1 < nchunks) {
+      mbar_arrive_expect_tx(tma_bar, 16384);
+      tma_load_3d(sm + OFF_V, &maps.v, tma_bar, 0, h, (int)(t0 + C));
+      tma_load_3d(sm + OFF_V + 8192, &maps.v, tma_bar, 64, h, (int)(t0 + C));
+    }
 
-    // ================================================================ [W; Qtil - PW] operand
+    // ================================================================ [-W; Qtil - PW] -> TMEM (bf16)
     {
       const int R = 32 * quarter + lane;
-      const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
+      uint32_t packed[32];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         float d[32];
-        tmem_ld32(tmem + lane_addr + TM_X + 64 * half + 32 * part, d);
+        tmem_ld32(tmem + lane_base + TM_WQ + 64 * half + 32 * part, d);
         if (R >= 64) {
           const int r = R - 64;
 #pragma unroll
           for (int cch = 0; cch < 4; ++cch) {
-            const uint32_t chunk = 4 * part + cch;  // within the 64-channel block `half`
-            const uint4 qb = *reinterpret_cast<const uint4*>(sm + OFF_Q + half * 8192 + sw128(r, chunk));
+            const uint4 qb = *reinterpret_cast<const uint4*>(sm + OFF_QB + half * 8192 + sw128(r, 4 * part + cch));
             const float2 a0 = unpack_bf16(qb.x), a1 = unpack_bf16(qb.y), a2 = unpack_bf16(qb.z),
                          a3 = unpack_bf16(qb.w);
-            d[8 * cch + 0] = a0.x - d[8 * cch + 0];
-            d[8 * cch + 1] = a0.y - d[8 * cch + 1];
-            d[8 * cch + 2] = a1.x - d[8 * cch + 2];
-            d[8 * cch + 3] = a1.y - d[8 * cch + 3];
-            d[8 * cch + 4] = a2.x - d[8 * cch + 4];
-            d[8 * cch + 5] = a2.y - d[8 * cch + 5];
-            d[8 * cch + 6] = a3.x - d[8 * cch + 6];
-            d[8 * cch + 7] = a3.y - d[8 * cch + 7];
+            packed[16 * part + 4 * cch + 0] = pack_bf16(a0.x - d[8 * cch + 0], a0.y - d[8 * cch + 1]);
+            packed[16 * part + 4 * cch + 1] = pack_bf16(a1.x - d[8 * cch + 2], a1.y - d[8 * cch + 3]);
+            packed[16 * part + 4 * cch + 2] = pack_bf16(a2.x - d[8 * cch + 4], a2.y - d[8 * cch + 5]);
+            packed[16 * part + 4 * cch + 3] = pack_bf16(a3.x - d[8 * cch + 6], a3.y - d[8 * cch + 7]);
           }
-        }
+        } else {
 #pragma unroll
-        for (int cch = 0; cch < 4; ++cch) {
-          uint4 w;
-          w.x = pack_bf16(d[8 * cch + 0], d[8 * cch + 1]);
-          w.y = pack_bf16(d[8 * cch + 2], d[8 * cch + 3]);
-          w.z = pack_bf16(d[8 * cch + 4], d[8 * cch + 5]);
-          w.w = pack_bf16(d[8 * cch + 6], d[8 * cch + 7]);
-          *reinterpret_cast<uint4*>(sm + OFF_WQ + half * 16384 + sw128(R, 4 * part + cch)) = w;
+          for (int u = 0; u < 16; ++u) packed[16 * part + u] = pack_bf16(-d[2 * u], -d[2 * u + 1]);
         }
       }
+      tc_fence_before();
+      bar_sync();   // every thread has read [W PW] before any column 0..63 is overwritten
+      tc_fence_after();
+      tmem_st32(tmem + lane_base + TM_WQ + 32 * half, packed);
+      tmem_wait_st();
     }
     publish();
 
-    // next chunk's q, g, v tiles may now be loaded (Qb read, Xk and V consumed by MMA_X)
-    const bool has_next = (c + 1 < nchunks);
-    if (tid == 0 && has_next) {
-      mbar_arrive_expect_tx(tma_bar, 4 * 16384);
-      issue_tma(t0 + C, true, false);
-    }
-
-    // ================================================================ MMA1: [W; Qtil - PW] x S
+    // ================================================================ MMA1: [U; PU] += [-W; Qtil - PW] x S
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t a = sdesc_sw128(sbase + OFF_WQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
         const uint64_t b = sdesc_sw128(sbase + OFF_S + ks * 2048, 16384, 1024);
-        umma_bf16(tmem + TM_REC, a, b, idesc, ks > 0);
+        umma_bf16_tmem_a(tmem + TM_UP, tmem + TM_WQ + 8 * ks, b, idesc, 1);
       }
       umma_commit(mma_bar);
     }
@@ -655,22 +689,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ ep1: Delta and O
     {
       const int R = 32 * quarter + lane;
-      const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
       const int r = R & 63;
-      const float ik = sc_ik[r];
+      const float ikr = sc_ik[r];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        float ws[32], uu[32];
-        tmem_ld32(tmem + lane_addr + TM_REC + 64 * half + 32 * part, ws);
-        tmem_ld32(tmem + lane_addr + TM_X + 128 + 64 * half + 32 * part, uu);
+        float d[32];
+        tmem_ld32(tmem + lane_base + TM_UP + 64 * half + 32 * part, d);
         if (R < 64) {
 #pragma unroll
           for (int cch = 0; cch < 4; ++cch) {
-            float dl[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) dl[u] = (uu[8 * cch + u] - ws[8 * cch + u]) * ik;
             uint4 wh, wl;
-            split_pack(dl, wh, wl);
+            split2(d[8 * cch + 0] * ikr, d[8 * cch + 1] * ikr, wh.x, wl.x);
+            split2(d[8 * cch + 2] * ikr, d[8 * cch + 3] * ikr, wh.y, wl.y);
+            split2(d[8 * cch + 4] * ikr, d[8 * cch + 5] * ikr, wh.z, wl.z);
+            split2(d[8 * cch + 6] * ikr, d[8 * cch + 7] * ikr, wh.w, wl.w);
             *reinterpret_cast<uint4*>(sm + OFF_DL + half * 8192 + sw128(r, 4 * part + cch)) = wh;
             *reinterpret_cast<uint4*>(sm + OFF_DLLO + half * 8192 + sw128(r, 4 * part + cch)) = wl;
           }
@@ -679,10 +711,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cch = 0; cch < 4; ++cch) {
             uint4 w;
-            w.x = pack_bf16(ws[8 * cch + 0] + uu[8 * cch + 0], ws[8 * cch + 1] + uu[8 * cch + 1]);
-            w.y = pack_bf16(ws[8 * cch + 2] + uu[8 * cch + 2], ws[8 * cch + 3] + uu[8 * cch + 3]);
-            w.z = pack_bf16(ws[8 * cch + 4] + uu[8 * cch + 4], ws[8 * cch + 5] + uu[8 * cch + 5]);
-            w.w = pack_bf16(ws[8 * cch + 6] + uu[8 * cch + 6], ws[8 * cch + 7] + uu[8 * cch + 7]);
+            w.x = pack_bf16(d[8 * cch + 0], d[8 * cch + 1]);
+            w.y = pack_bf16(d[8 * cch + 2], d[8 * cch + 3]);
+            w.z = pack_bf16(d[8 * cch + 4], d[8 * cch + 5]);
+            w.w = pack_bf16(d[8 * cch + 6], d[8 * cch + 7]);
             reinterpret_cast<uint4*>(orow)[cch] = w;
           }
         }
@@ -690,30 +722,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     publish();
 
-    // ================================================================ MMA2: Ktil^T x Delta
+    // ================================================================ MMA2: Ktil^T x (Delta_hi + Delta_lo)
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t idesc = idesc_bf16(128, 128, true, true);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t a = sdesc_sw128(sbase + OFF_K + (ks & 3) * 2048, 8192, 1024);
+        const uint64_t a = sdesc_sw128(sbase + OFF_KT + (ks & 3) * 2048, 8192, 1024);
         const uint64_t b = sdesc_sw128(sbase + (ks < 4 ? OFF_DL : OFF_DLLO) + (ks & 3) * 2048, 8192, 1024);
-        umma_bf16(tmem + TM_REC, a, b, idesc, ks > 0);
+        umma_bf16(tmem + TM_UP, a, b, idesc, ks > 0);
       }
       umma_commit(mma_bar);
     }
     if (!wait_all(mma_bar, mma_phase)) break;
     tc_fence_after();
-    if (tid == 0 && has_next) issue_tma(t0 + C, false, true);
 
     // ================================================================ ep2: state update
     {
-      const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
       const float gam = sc_gam[srow];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         float d[32];
-        tmem_ld32(tmem + lane_addr + TM_REC + 64 * half + 32 * part, d);
+        tmem_ld32(tmem + lane_base + TM_UP + 64 * half + 32 * part, d);
 #pragma unroll
         for (int j = 0; j < 32; ++j) S[32 * part + j] = fmaf(gam, S[32 * part + j], d[j]);
       }
@@ -778,9 +808,7 @@ cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream) {
   if (units == 0) return cudaSuccess;
   const int64_t tokens = p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs;
   TensorMaps maps;
-  if (!make_token_map(&maps.q, p.q, tokens, p.num_heads) || !make_token_map(&maps.k, p.k, tokens, p.num_heads) ||
-      !make_token_map(&maps.v, p.v, tokens, p.num_heads) || !make_token_map(&maps.g, p.g, tokens, p.num_heads))
-    return cudaErrorInvalidValue;
+  if (!make_token_map(&maps.v, p.v, tokens, p.num_heads)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
