@@ -1,4 +1,5 @@
-// Chunked KDA forward for sm_100a: one fused kernel, one CTA per (sequence, head) unit.
+// Chunked KDA forward for sm_100a: one fused, warp-specialised kernel, one CTA per (sequence,
+// head) unit.
 //
 // Kimi Delta Attention (FlashKDA `fwd`, fla `chunk_kda`; vLLM PR #54859 report and "What CUDA
 // Version Is Required to Use FlashKDA?", Usage Examples) is the gated delta rule
@@ -12,27 +13,37 @@
 //   Delta = U - W S,   O = Qtil S + P Delta = (Qtil - P W) S + P U,
 //   S <- Diag(e^{Gamma_C}) S + Ktil^T Delta.
 //
-// Per chunk (everything on-chip; HBM sees the raw inputs once and the output once):
-//   prologue  (CUDA cores) raw q, k, g rows straight from global memory into registers; L2 norms,
-//             sigmoid(beta), safe gate alpha = exp(lower_bound * sigmoid(exp(A_log)(g + dt_bias)));
-//             decays as running products of alpha inside each 16-row sub-block (exponent
-//             referencing: every factor stays in [e^-80, e^80] for lower_bound >= -5); the bf16 MMA
-//             operands, with the norms, beta and scale folded in.  v arrives by TMA.
-//   MMA_AP    [LK; LQ] x R_I^T per 16-row sub-block I -> the gated K K^T and Q K^T blocks (TMEM).
-//   assemble  A (fp32, shared memory) and P (bf16 operand).
-//   solve     T = (I + A)^{-1}: the four 16x16 diagonal blocks by forward substitution, then the
-//             off-diagonal blocks T_IJ = -T_II sum_K A_IK T_KJ, all in fp32; T_b as a bf16 hi+lo pair.
-//   MMA_PT    P (T_hi + T_lo), read back as a hi+lo pair.
-//   MMA_X     [T_b; P T_b] (hi + lo) x [Khat e^Gamma | V] -> [W | U; P W | P U] in TMEM.
-//   WQ        [-W; Qtil - P W] written back to TMEM as the A operand of MMA1.
-//   MMA1      accumulates [-W; Qtil - P W] x S onto [U; P U]  ->  [Delta; O].
-//   ep1       Delta (bf16 hi+lo operand), O -> global bf16.
-//   MMA2      Ktil^T (Delta_hi + Delta_lo); ep2: S = e^{Gamma_C} S + Ktil^T Delta (fp32 registers),
-//             plus its bf16 copy (the B operand of the next MMA1).
-// The hi+lo pairs matter when keys are nearly collinear: T then has entries close to -beta that
-// cancel against the diagonal, and a chunk's Delta rows telescope, so a single bf16 rounding of
-// T_b, P T_b or Delta would cost several percent of the state.  Ktil is built from the raw bf16 k
-// (its 1/|k| is applied to Delta) so that equal keys round identically.
+// Roles (512 threads):
+//   warp 0 (one thread)  issues every tcgen05 MMA, polling two dependency streams: the
+//                        intra-chunk stream (AP, PT, Xk, Xv of chunk c+1) and the recurrence
+//                        stream (MMA1, MMA2 of chunk c), so each runs as soon as its inputs exist.
+//   warp 1 (one thread)  TMA loads of the q and k tiles (a single stage, refilled as soon as the
+//                        intra warps have read it) and of the v tile.
+//   warps 4..11 (intra)  per chunk:
+//       prologue  raw q, k (shared memory), g (registers, prefetched one chunk ahead); L2 norms,
+//                 sigmoid(beta), safe gate alpha = exp(lower_bound * sigmoid(exp(A_log)(g + dt_bias)));
+//                 decays as running products of alpha inside each 16-row sub-block (exponent
+//                 referencing: every factor stays in [e^-80, e^80] for lower_bound >= -5); the bf16
+//                 MMA operands with the norms, beta and scale folded in.
+//       assemble  A (fp32) and P (bf16) from the gated Gram blocks [LK; LQ] x R_I^T (MMA AP).
+//       solve     T = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution, off-diagonal
+//                 blocks T_IJ = -T_II sum_K A_IK T_KJ, in fp32; T_b kept as a bf16 hi+lo pair.
+//       PT        P (T_hi + T_lo) (MMA PT) read back as a hi+lo pair.
+//       WQ        [-W; Qtil - P W] from [T_b; P T_b] x Khat e^Gamma (MMA Xk), written to TMEM as
+//                 the A operand of MMA1.
+//   warps 12..15 (rec)   MMA Xv writes [U; P U] into TMEM; MMA1 accumulates [-W; Qtil - PW] x S onto
+//                 it, giving [Delta; O]; ep1 stores O and Delta (bf16 hi+lo); MMA2 accumulates
+//                 Ktil^T Delta onto the fp32 state kept in TMEM (pre-scaled by e^{Gamma_C}); ep2
+//                 refreshes the bf16 copy of S used as the B operand of the next MMA1.
+// HBM sees the raw inputs once and the output once.  The hi+lo pairs matter when keys are nearly
+// collinear: T then has entries close to -beta that cancel against the diagonal and a chunk's
+// Delta rows telescope, so a single bf16 rounding of T_b, P T_b or Delta would cost several
+// percent of the state.  Ktil is built from the raw bf16 k (its 1/|k| is applied to Delta) so that
+// equal keys round identically.
+//
+// Every wait is bounded (kWaitLimitNs of wall time without progress): on expiry the kernel
+// records KDA_ERR_DEVICE_TIMEOUT in the workspace status word, every role leaves its loop, and
+// the tensor memory is released.
 #include <cuda.h>
 
 #include "kda_common.cuh"
@@ -45,52 +56,63 @@ using namespace sm100;
 
 constexpr int C = 64;          // chunk length
 constexpr int D = kHeadDim;    // 128
-constexpr int kThreads = 256;  // 8 warps
+constexpr int kThreads = 512;  // 16 warps
+constexpr int kIntraWarp0 = 4, kIntraThreads = 256;
+constexpr int kRecWarp0 = 12, kRecThreads = 128;
+constexpr uint32_t kBarIntra = 1, kBarRec = 2;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Shared-memory map (bytes from a 1024-aligned base).  "MN tile" = [2 blocks of 64 columns]
 // [64 rows][128 B] with the 128-byte swizzle; "K tile" = [2 blocks of 64 K][rows][128 B].
-constexpr uint32_t OFF_V = 0;            // v (TMA), MN-major B of MMA_X
-constexpr uint32_t OFF_XK = 16384;       // Khat e^Gamma, MN-major B of MMA_X
-constexpr uint32_t OFF_QB = 32768;       // Qtil (bf16), read when forming Qtil - P W
-constexpr uint32_t OFF_KT = 49152;       // Ktil (raw k), MN-major A of MMA2
-constexpr uint32_t OFF_SCR = 65536;      // scratch, 73728 bytes:
-constexpr uint32_t OFF_LKQ = OFF_SCR;    //   [LK; LQ] K tile, 128 rows (prologue -> MMA_AP)
-constexpr uint32_t OFF_R = OFF_SCR + 32768;  //   R_0..R_3 K tile, 160 rows (prologue -> MMA_AP)
+constexpr uint32_t OFF_RQ = 0;           // q tile (TMA)
+constexpr uint32_t OFF_RK = 16384;       // k tile (TMA)
+constexpr uint32_t OFF_XK = 32768;       // Khat e^Gamma, MN-major B of MMA Xk
+constexpr uint32_t OFF_QB = 49152;       // Qtil (bf16), read when forming Qtil - P W
+constexpr uint32_t OFF_KT = 65536;       // Ktil (raw k), MN-major A of MMA2
+constexpr uint32_t OFF_DL = 81920;       // Delta hi, MN tile (ep1 -> MMA2)
+constexpr uint32_t OFF_DLLO = 98304;     // Delta lo
+constexpr uint32_t OFF_S = 114688;       // S bf16, MN-major B of MMA1, 2 blocks x 128 rows
+constexpr uint32_t OFF_SCR = 147456;     // scratch, 73728 bytes:
+constexpr uint32_t OFF_LKQ = OFF_SCR;            //   [LK; LQ] K tile, 128 rows (prologue -> AP)
+constexpr uint32_t OFF_R = OFF_SCR + 32768;      //   R_0..R_3 K tile, 160 rows (prologue -> AP)
 constexpr uint32_t R_KBLK = 160 * 128;
-constexpr uint32_t OFF_AS = OFF_SCR;             // A fp32 64 x 68 (assemble -> solve)
-constexpr uint32_t OFF_TS = OFF_SCR + 17408;     // T fp32 64 x 68 (solve)
-constexpr uint32_t OFF_YS = OFF_SCR + 17408 * 2; // solve temporaries, 3 x 16 x 16 fp32
+constexpr uint32_t OFF_TP = OFF_SCR;             //   [T_hi; P -> (P T)_hi] 128 x 64 K tile
+constexpr uint32_t OFF_AS = OFF_SCR + 16384;     //   A fp32 64 x 68 (assemble -> solve)
+constexpr uint32_t OFF_TL = OFF_SCR + 16384;     //   [T_lo; (P T)_lo] (after A is dead)
+constexpr uint32_t OFF_TS = OFF_SCR + 33792;     //   T fp32 64 x 68
+constexpr uint32_t OFF_YS = OFF_SCR + 51200;     //   solve temporaries 3 x 16 x 16 fp32
+constexpr uint32_t OFF_V = OFF_SCR + 54272;      //   v tile (TMA, after AP), MN-major B of MMA Xv
 constexpr uint32_t AS_LD = 68;
-constexpr uint32_t OFF_TP = OFF_SCR + 40960;     // [T_hi; P -> (P T)_hi] 128 x 64, K tile
-constexpr uint32_t OFF_TL = OFF_SCR + 57344;     // [T_lo; (P T)_lo]
-constexpr uint32_t OFF_DL = OFF_SCR;             // Delta hi, MN tile (ep1 -> MMA2)
-constexpr uint32_t OFF_DLLO = OFF_SCR + 16384;   // Delta lo
-constexpr uint32_t OFF_S = OFF_SCR + 73728;      // S bf16, MN-major B of MMA1, 2 blocks x 128 rows
-constexpr uint32_t OFF_SC = OFF_S + 32768;       // scalars
-constexpr uint32_t SC_BETA = 0;                  // float[64]
-constexpr uint32_t SC_IK = 256;                  // float[64] 1/|k_r| (0 for rows past the end)
-constexpr uint32_t SC_GAM = 512;                 // float[128] e^{Gamma_C}
-constexpr uint32_t SC_TOT = 1024;                // float[8][128] per-warp alpha products
-constexpr uint32_t SC_BAR = 5120;                // 2 mbarriers
-constexpr uint32_t SC_TMEM = 5136;
-constexpr uint32_t SC_ABORT = 5140;
-constexpr uint32_t SMEM_BYTES = OFF_SC + 5248;
+constexpr uint32_t OFF_SC = OFF_SCR + 73728;     // scalars
+constexpr uint32_t SC_BETA = 0;                  // float[2][64]
+constexpr uint32_t SC_IK = 512;                  // float[2][64] 1/|k_r| (0 past the end)
+constexpr uint32_t SC_GAM = 1024;                // float[2][128] e^{Gamma_C}
+constexpr uint32_t SC_TOT = 2048;                // float[8][128] per-warp alpha products
+constexpr uint32_t SC_BAR = 6144;                // mbarriers
+constexpr uint32_t SC_TMEM = 6400;
+constexpr uint32_t SC_ABORT = 6404;
+constexpr uint32_t SMEM_BYTES = OFF_SC + 6528;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+
+// mbarrier indices
+enum {
+  B_RAW_FULL, B_RAW_EMPTY, B_V_FULL, B_OPS0, B_OPS1, B_KT, B_AP, B_TB, B_PT, B_TP, B_XK, B_XV, B_WQ,
+  B_MMA1, B_DELTA, B_MMA2, B_S, B_COUNT
+};
 
 // first row of R_I inside the R tile: 0, 16, 48, 96 (R_I holds 16 (I+1) rows)
 __host__ __device__ constexpr uint32_t row_off(int I) { return 8u * I * (I + 1); }
 
-// TMEM columns: AP products at row_off(I) (N = 16 (I+1)), then P T at 0..63, then
-// [W PW] at 0..127 and [U PU] at 128..255; [-W; Qtil - PW] packed bf16 at 0..63; MMA1 and MMA2
-// accumulate at 128..255.
-constexpr uint32_t TM_WQ = 0;
-constexpr uint32_t TM_UP = 128;
-constexpr uint32_t kTmemCols = 256;
+// TMEM columns: intra area 0..255 (AP products at row_off(I), P T at 0..63, [W PW] at 0..127,
+// [-W; Qtil - PW] packed bf16 at 0..63); [U PU] -> [Delta O] at 256..383; fp32 state at 384..511.
+constexpr uint32_t TM_UP = 256;
+constexpr uint32_t TM_S = 384;
+constexpr uint32_t kTmemCols = 512;
 
 struct TensorMaps {
-  CUtensorMap v;
+  CUtensorMap q, k, v;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -112,224 +134,315 @@ __device__ __forceinline__ float fast_sigmoid(float x) { return __fdividef(1.0f,
 __device__ __forceinline__ uint2 ldg_u2(const __nv_bfloat16* p) {
   return __ldg(reinterpret_cast<const uint2*>(p));
 }
-__device__ __forceinline__ void bar_sync() { __syncthreads(); }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    chunked_kernel(const __grid_constant__ TensorMaps maps, FwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sbase = smem_u32(sm);
+struct Shared {
+  uint8_t* sm;
+  uint32_t sbase;
+  uint64_t* bar;
+  volatile int* abort;
+  uint32_t tmem;
+};
+
+// Bounded wait on a phase; returns false once the abort flag is up (set here on time-out).
+__device__ __forceinline__ bool wait_bar(const Shared& S_, int b, uint32_t parity, uint32_t* status) {
+  uint64_t* bar = S_.bar + b;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63) == 0) {
+      if (*S_.abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *S_.abort = 1;
+        if (status) atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ MMA issuer
+__device__ void mma_issuer(const Shared& S_, const FwdParams& p, int nchunks) {
+  const uint32_t sbase = S_.sbase, tmem = S_.tmem;
+  uint64_t* bar = S_.bar;
+  int ci = 0, ist = 0;  // intra stream: chunk, stage (0 AP, 1 PT, 2 Xk, 3 Xv)
+  int cr = 0, rst = 0;  // recurrence stream: chunk, stage (0 MMA1, 1 MMA2)
+  uint64_t last = globaltimer_ns();
+  while (cr < nchunks) {
+    if (*S_.abort) return;
+    bool progressed = false;
+    // ---- recurrence stream (priority)
+    if (rst == 0) {
+      if (ci > cr && mbar_test(bar + B_WQ, cr & 1) && mbar_test(bar + B_S, cr & 1)) {
+        tc_fence_after();
+        constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t b = sdesc_sw128(sbase + OFF_S + ks * 2048, 16384, 1024);
+          umma_bf16_tmem_a(tmem + TM_UP, tmem + 8 * ks, b, idesc, 1);
+        }
+        umma_commit(bar + B_MMA1);
+        rst = 1;
+        progressed = true;
+      }
+    } else {
+      if (mbar_test(bar + B_DELTA, cr & 1) && mbar_test(bar + B_KT, cr & 1)) {
+        tc_fence_after();
+        constexpr uint32_t idesc = idesc_bf16(128, 128, true, true);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t a = sdesc_sw128(sbase + OFF_KT + (ks & 3) * 2048, 8192, 1024);
+          const uint64_t b = sdesc_sw128(sbase + (ks < 4 ? OFF_DL : OFF_DLLO) + (ks & 3) * 2048, 8192, 1024);
+          umma_bf16(tmem + TM_S, a, b, idesc, 1);
+        }
+        umma_commit(bar + B_MMA2);
+        rst = 0;
+        ++cr;
+        progressed = true;
+      }
+    }
+    // ---- intra-chunk stream
+    if (ci < nchunks) {
+      if (ist == 0) {
+        // AP(ci) overwrites the TMEM area that holds WQ(ci-1): MMA1(ci-1) must be issued first
+        const bool wq_consumed = (ci == 0) || (cr > ci - 1) || (cr == ci - 1 && rst == 1);
+        if (wq_consumed && mbar_test(bar + B_OPS0 + (ci & 1), (ci >> 1) & 1)) {
+          tc_fence_after();
+#pragma unroll
+          for (int I = 0; I < 4; ++I) {
+            const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint64_t a = sdesc_sw128(sbase + OFF_LKQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+              const uint64_t b =
+                  sdesc_sw128(sbase + OFF_R + (ks >> 2) * R_KBLK + row_off(I) * 128 + (ks & 3) * 32, 16, 1024);
+              umma_bf16(tmem + row_off(I), a, b, idesc, ks > 0);
+            }
+          }
+          umma_commit(bar + B_AP);
+          ist = 1;
+          progressed = true;
+        }
+      } else if (ist == 1) {
+        if (mbar_test(bar + B_TB, ci & 1)) {
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t a = sdesc_sw128(sbase + OFF_TP + (ks & 3) * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(sbase + (ks < 4 ? OFF_TP : OFF_TL) + (ks & 3) * 2048, 8192, 1024);
+            umma_bf16(tmem, a, b, idesc, ks > 0);
+          }
+          umma_commit(bar + B_PT);
+          ist = 2;
+          progressed = true;
+        }
+      } else if (ist == 2) {
+        if (mbar_test(bar + B_TP, ci & 1)) {
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t a = sdesc_sw128(sbase + (ks < 4 ? OFF_TP : OFF_TL) + (ks & 3) * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(sbase + OFF_XK + (ks & 3) * 2048, 8192, 1024);
+            umma_bf16(tmem, a, b, idesc, ks > 0);
+          }
+          umma_commit(bar + B_XK);
+          ist = 3;
+          progressed = true;
+        }
+      } else {
+        // Xv(ci) writes [U PU] where [Delta O](ci-1) lives until ep1(ci-1) has read it
+        const bool up_free = (ci == 0) || mbar_test(bar + B_DELTA, (ci - 1) & 1);
+        if (up_free && mbar_test(bar + B_V_FULL, ci & 1)) {
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t a = sdesc_sw128(sbase + (ks < 4 ? OFF_TP : OFF_TL) + (ks & 3) * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(sbase + OFF_V + (ks & 3) * 2048, 8192, 1024);
+            umma_bf16(tmem + TM_UP, a, b, idesc, ks > 0);
+          }
+          umma_commit(bar + B_XV);
+          ist = 0;
+          ++ci;
+          progressed = true;
+        }
+      }
+    }
+    if (progressed) {
+      last = globaltimer_ns();
+    } else {
+      __nanosleep(64);
+      if (globaltimer_ns() - last > kWaitLimitNs) {
+        *S_.abort = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+        return;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ TMA producer
+__device__ void tma_producer(const Shared& S_, const TensorMaps& maps, const FwdParams& p, int h,
+                             int64_t bos, int nchunks) {
+  uint8_t* sm = S_.sm;
+  uint64_t* bar = S_.bar;
+  for (int c = 0; c < nchunks; ++c) {
+    const int t0 = (int)(bos + (int64_t)c * C);
+    if (c > 0 && !wait_bar(S_, B_RAW_EMPTY, (c - 1) & 1, p.status)) return;
+    mbar_arrive_expect_tx(bar + B_RAW_FULL, 32768);
+    tma_load_3d(sm + OFF_RQ, &maps.q, bar + B_RAW_FULL, 0, h, t0);
+    tma_load_3d(sm + OFF_RQ + 8192, &maps.q, bar + B_RAW_FULL, 64, h, t0);
+    tma_load_3d(sm + OFF_RK, &maps.k, bar + B_RAW_FULL, 0, h, t0);
+    tma_load_3d(sm + OFF_RK + 8192, &maps.k, bar + B_RAW_FULL, 64, h, t0);
+    // the v tile lands in the scratch once MMA AP has consumed the Gram operands
+    if (!wait_bar(S_, B_AP, c & 1, p.status)) return;
+    mbar_arrive_expect_tx(bar + B_V_FULL, 16384);
+    tma_load_3d(sm + OFF_V, &maps.v, bar + B_V_FULL, 0, h, t0);
+    tma_load_3d(sm + OFF_V + 8192, &maps.v, bar + B_V_FULL, 64, h, t0);
+  }
+}
+
+// ------------------------------------------------------------------------------ intra warps
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t bos, int64_t eos,
+                            int nchunks, int itid) {
+  uint8_t* sm = S_.sm;
+  const uint32_t tmem = S_.tmem;
+  const int H = p.num_heads;
+  const int iw = itid >> 5, lane = itid & 31;
+  const int quarter = iw & 3, ihalf = iw >> 2;       // TMEM lane quarter, column half
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
   float* sc_beta = reinterpret_cast<float*>(sm + OFF_SC + SC_BETA);
   float* sc_ik = reinterpret_cast<float*>(sm + OFF_SC + SC_IK);
   float* sc_gam = reinterpret_cast<float*>(sm + OFF_SC + SC_GAM);
   float* sc_tot = reinterpret_cast<float*>(sm + OFF_SC + SC_TOT);
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + OFF_SC + SC_BAR);
-  uint64_t* mma_bar = tma_bar + 1;
-  uint32_t* sc_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SC + SC_TMEM);
-  volatile int* sc_abort = reinterpret_cast<volatile int*>(sm + OFF_SC + SC_ABORT);
   float* As = reinterpret_cast<float*>(sm + OFF_AS);
   float* Ts = reinterpret_cast<float*>(sm + OFF_TS);
   float* Ys = reinterpret_cast<float*>(sm + OFF_YS);
+  volatile int* abort_flag = S_.abort;
+  auto sync = [&]() { named_bar(kBarIntra, kIntraThreads); };
 
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int quarter = warp & 3, half = warp >> 2;
-  const int H = p.num_heads;
-  const int n = blockIdx.x / H, h = blockIdx.x % H;
-  int64_t bos, eos;
-  seq_range(p, n, bos, eos);
-  const int64_t seq_len = eos - bos;
-  const int nchunks = (int)((seq_len + C - 1) / C);
-
-  if (tid == 0) {
-    mbar_init(tma_bar, 1);
-    mbar_init(mma_bar, 1);
-    *sc_abort = 0;
-    fence_mbar_init();
-    prefetch_tmap(&maps.v);
-  }
-  if (warp == 0) {
-    tmem_alloc(sc_tmem, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  bar_sync();
-  tc_fence_after();
-  const uint32_t tmem = *sc_tmem;
-  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;  // this warp's TMEM lane quarter
-
-  // ---- state: thread owns row k = 32*quarter + lane, columns [64*half, 64*half + 64)
-  const int srow = 32 * quarter + lane;
-  const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
-  float S[64];
-#pragma unroll
-  for (int j = 0; j < 64; ++j) {
-    const int col = 64 * half + j;
-    float s = 0.f;
-    if (p.initial_state)
-      s = p.state_transposed ? p.initial_state[soff + (size_t)col * D + srow]
-                             : p.initial_state[soff + (size_t)srow * D + col];
-    S[j] = s;
-  }
-  auto store_state_bf16 = [&]() {
-    uint8_t* base = sm + OFF_S + half * (128 * 128);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint4 w;
-      w.x = pack_bf16(S[8 * c + 0], S[8 * c + 1]);
-      w.y = pack_bf16(S[8 * c + 2], S[8 * c + 3]);
-      w.z = pack_bf16(S[8 * c + 4], S[8 * c + 5]);
-      w.w = pack_bf16(S[8 * c + 6], S[8 * c + 7]);
-      *reinterpret_cast<uint4*>(base + sw128(srow, c)) = w;
-    }
-  };
-  store_state_bf16();
-
-  // prologue mapping: warp w owns chunk rows 8w..8w+7, lane owns channels 4*lane..4*lane+3
+  // prologue mapping: warp iw owns chunk rows 8 iw .. 8 iw + 7, lane owns channels 4 lane .. +3
   const float gate_a = __expf(p.A_log[h]);
   const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-  // exp(-a (g + dt)) = exp2(ga * g + gb)
-  const float ga = -gate_a * kLog2e;
+  const float ga = -gate_a * kLog2e;                 // exp(-a (g + dt)) = exp2(ga g + gb)
   const float gb[4] = {ga * dtb.x, ga * dtb.y, ga * dtb.z, ga * dtb.w};
   const float lb2 = p.lower_bound * kLog2e;
-  const int kb = lane >> 4;                       // 64-channel block
-  const uint32_t lane_chunk = (lane & 15) >> 1;   // 16-byte chunk within the 128-byte row
-  const uint32_t lane_sub = (lane & 1) * 8;       // byte within the chunk
-  const int blk = warp >> 1;                      // 16-row sub-block of this warp's rows
-  const bool upper_half = warp & 1;               // rows 8..15 of the sub-block
+  const int kb = lane >> 4;
+  const uint32_t lane_chunk = (lane & 15) >> 1;
+  const uint32_t lane_sub = (lane & 1) * 8;
+  const int blk = iw >> 1;
+  const bool upper_half = iw & 1;
 
-  uint32_t tma_phase = 0, mma_phase = 0;
-  if (tid == 0 && nchunks > 0) {
-    mbar_arrive_expect_tx(tma_bar, 16384);
-    tma_load_3d(sm + OFF_V, &maps.v, tma_bar, 0, h, (int)bos);
-    tma_load_3d(sm + OFF_V + 8192, &maps.v, tma_bar, 64, h, (int)bos);
-  }
-
-  auto wait_all = [&](uint64_t* bar, uint32_t& phase) -> bool {
-    const bool ok = mbar_wait(bar, phase, kWaitLimitNs);
-    phase ^= 1u;
-    if (!ok) {
-      *sc_abort = 1;
-      if (p.status) atomicOr(p.status, kStatusTimeout);
+  uint2 gr[8];  // raw g of the chunk being prepared (loaded one chunk ahead)
+  auto load_g = [&](int c) {
+    const int64_t t0 = bos + (int64_t)c * C;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t t = t0 + 8 * iw + i;
+      gr[i] = (c < nchunks && t < eos) ? ldg_u2(p.g + ((size_t)t * H + h) * D + 4 * lane) : make_uint2(0, 0);
     }
-    bar_sync();
-    return *sc_abort == 0;
   };
-  auto publish = [&]() {
-    fence_proxy_async();
-    tc_fence_before();
-    bar_sync();
-  };
+  load_g(0);
 
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = bos + (int64_t)c * C;
     const int len = (int)((eos - t0) < (int64_t)C ? (eos - t0) : (int64_t)C);
+    const int slot = c & 1;
 
-    // ================================================================ prologue
-    {
-      uint2 qr[8], kr[8];
-      float al[8][4];
-      float ssq[8], ssk[8];
+    // ============================================================== prologue
+    wait_bar(S_, B_RAW_FULL, c & 1, p.status);
+    uint2 qr[8], kr[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * warp + i;
-        const bool valid = r < len;
-        const size_t off = ((size_t)(t0 + r) * H + h) * D + 4 * lane;
-        uint2 gr = make_uint2(0, 0);
-        qr[i] = make_uint2(0, 0);
-        kr[i] = make_uint2(0, 0);
-        if (valid) {
-          qr[i] = ldg_u2(p.q + off);
-          kr[i] = ldg_u2(p.k + off);
-          gr = ldg_u2(p.g + off);
-        }
-        const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
-        const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
-        ssq[i] = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
-        ssk[i] = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
-        const float2 g01 = unpack_bf16(gr.x), g23 = unpack_bf16(gr.y);
-        const float gv[4] = {g01.x, g01.y, g23.x, g23.y};
+    for (int i = 0; i < 8; ++i) {
+      const int r = 8 * iw + i;
+      const uint32_t off = kb * 8192 + sw128(r, lane_chunk) + lane_sub;
+      const bool valid = r < len;
+      qr[i] = valid ? *reinterpret_cast<const uint2*>(sm + OFF_RQ + off) : make_uint2(0, 0);
+      kr[i] = valid ? *reinterpret_cast<const uint2*>(sm + OFF_RK + off) : make_uint2(0, 0);
+    }
+    sync();
+    if (*abort_flag) break;
+    if (itid == 0) mbar_arrive(S_.bar + B_RAW_EMPTY);
+
+    float a[8][4];  // alpha
+    float ssq[8], ssk[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // alpha = 2^(lb*log2e * sigmoid(a (g + dt)))
-          const float z = exp2f(fmaf(ga, gv[j], gb[j]));
-          const float sig = __fdividef(1.0f, 1.0f + z);
-          al[i][j] = valid ? exp2f(lb2 * sig) : 1.0f;
-        }
-      }
-      // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
-      // total of value (l >> 1): q rows 0..7, then k rows 0..7
-      float inv;
-      {
-        float v16[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v16[i] = ssq[i];
-          v16[8 + i] = ssk[i];
-        }
-        const bool b4 = lane & 16;
-        float w8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float send = b4 ? v16[j] : v16[j + 8];
-          const float keep = b4 ? v16[j + 8] : v16[j];
-          w8[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-        }
-        const bool b3 = lane & 8;
-        float w4[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float send = b3 ? w8[j] : w8[j + 4];
-          const float keep = b3 ? w8[j + 4] : w8[j];
-          w4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-        const bool b2 = lane & 4;
-        float w2[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const float send = b2 ? w4[j] : w4[j + 2];
-          const float keep = b2 ? w4[j + 2] : w4[j];
-          w2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        }
-        const bool b1 = lane & 2;
-        float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
-        w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
-        inv = rsqrtf(w1 + kL2Eps);
-      }
-      // beta of row 8w + lane (lanes 0..7), broadcast to the warp
-      float beta_l = 0.f;
-      if (lane < 8) {
-        const int r = 8 * warp + lane;
-        if (r < len) beta_l = fast_sigmoid(__bfloat162float(p.beta[(size_t)(t0 + r) * H + h]));
-        sc_beta[r] = beta_l;
-      }
-      float iq[8], ik[8], bt[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        iq[i] = __shfl_sync(0xffffffffu, inv, 2 * i) * p.scale;
-        ik[i] = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);
-        bt[i] = __shfl_sync(0xffffffffu, beta_l, i);
-      }
-      if (lane < 8) {
-        const int r = 8 * warp + lane;
-        float v = ik[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) v = (lane == i) ? ik[i] : v;
-        sc_ik[r] = (r < len) ? v : 0.f;
-      }
-      // running products of alpha over this warp's 8 rows (prefix in place) and their suffixes
-      float suf[8][4];
+    for (int i = 0; i < 8; ++i) {
+      const int r = 8 * iw + i;
+      const bool valid = r < len;
+      const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
+      const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
+      ssq[i] = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
+      ssk[i] = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
+      const float2 g01 = unpack_bf16(gr[i].x), g23 = unpack_bf16(gr[i].y);
+      const float gv[4] = {g01.x, g01.y, g23.x, g23.y};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        suf[7][j] = 1.f;
-#pragma unroll
-        for (int i = 6; i >= 0; --i) suf[i][j] = suf[i + 1][j] * al[i + 1][j];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) al[i][j] *= al[i - 1][j];
+        const float sig = rcp_approx(1.0f + ex2_approx(fmaf(ga, gv[j], gb[j])));
+        a[i][j] = valid ? ex2_approx(lb2 * sig) : 1.0f;
       }
-      reinterpret_cast<float4*>(sc_tot + warp * 128)[lane] = make_float4(al[7][0], al[7][1], al[7][2], al[7][3]);
-      bar_sync();
-      // sub-block totals b_J = e^{Gamma at the end of J - Gamma at its start}
+    }
+    // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
+    // total of value (l >> 1): q rows 0..7, then k rows 0..7
+    float inv;
+    {
+      float v16[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v16[i] = ssq[i];
+        v16[8 + i] = ssk[i];
+      }
+      const bool b4 = lane & 16;
+      float w8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        w8[j] = (b4 ? v16[j + 8] : v16[j]) + __shfl_xor_sync(0xffffffffu, b4 ? v16[j] : v16[j + 8], 16);
+      const bool b3 = lane & 8;
+      float w4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w4[j] = (b3 ? w8[j + 4] : w8[j]) + __shfl_xor_sync(0xffffffffu, b3 ? w8[j] : w8[j + 4], 8);
+      const bool b2 = lane & 4;
+      float w2[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        w2[j] = (b2 ? w4[j + 2] : w4[j]) + __shfl_xor_sync(0xffffffffu, b2 ? w4[j] : w4[j + 2], 4);
+      const bool b1 = lane & 2;
+      float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
+      w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
+      inv = rsqrtf(w1 + kL2Eps);
+    }
+    float beta_l = 0.f;
+    if (lane < 8) {
+      const int r = 8 * iw + lane;
+      if (r < len) beta_l = fast_sigmoid(__bfloat162float(p.beta[(size_t)(t0 + r) * H + h]));
+    }
+    // per-warp alpha totals -> sub-block totals b_J
+    float tot[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float t = a[0][j];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) t *= a[i][j];
+      tot[j] = t;
+    }
+    reinterpret_cast<float4*>(sc_tot + iw * 128)[lane] = make_float4(tot[0], tot[1], tot[2], tot[3]);
+    sync();
+    float pre[4], post[4], cI[4][4], gam[4], pt[4];
+    {
       float bJ[4][4];
 #pragma unroll
       for (int J = 0; J < 4; ++J) {
@@ -340,27 +453,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         bJ[J][2] = t0v.z * t1v.z;
         bJ[J][3] = t0v.w * t1v.w;
       }
-      const float4 partner = reinterpret_cast<const float4*>(sc_tot + (warp ^ 1) * 128)[lane];
-      const float pt[4] = {partner.x, partner.y, partner.z, partner.w};
-      // e_i = prod of alpha from the sub-block start to row i; f_i = prod after row i to its end
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (upper_half) al[i][j] *= pt[j];
-          else suf[i][j] *= pt[j];
-        }
-      float pre[4], post[4], cI[4][4];
+      const float4 pv = reinterpret_cast<const float4*>(sc_tot + (iw ^ 1) * 128)[lane];
+      pt[0] = pv.x; pt[1] = pv.y; pt[2] = pv.z; pt[3] = pv.w;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float a = 1.f, z = 1.f;
+        float pa = 1.f, z = 1.f;
 #pragma unroll
         for (int J = 0; J < 4; ++J) {
-          if (J < blk) a *= bJ[J][j];
+          if (J < blk) pa *= bJ[J][j];
           if (J > blk) z *= bJ[J][j];
         }
-        pre[j] = a;
+        pre[j] = pa;
         post[j] = z;
+        gam[j] = bJ[0][j] * bJ[1][j] * bJ[2][j] * bJ[3][j];
         float m = 1.f;
 #pragma unroll
         for (int I = 0; I < 4; ++I) {
@@ -368,34 +473,71 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (I > blk) m *= bJ[I][j];
         }
       }
-      if (warp == 0)
-        reinterpret_cast<float4*>(sc_gam)[lane] =
-            make_float4(bJ[0][0] * bJ[1][0] * bJ[2][0] * bJ[3][0], bJ[0][1] * bJ[1][1] * bJ[2][1] * bJ[3][1],
-                        bJ[0][2] * bJ[1][2] * bJ[2][2] * bJ[3][2], bJ[0][3] * bJ[1][3] * bJ[2][3] * bJ[3][3]);
-      // operands, one row at a time
+    }
+    // the scratch and the scalar slot still serve the chunk two back / MMA Xv of the previous
+    // chunk until MMA Xv has run (and, through it, ep1 of the chunk before)
+    if (c > 0) wait_bar(S_, B_XV, (c - 1) & 1, p.status);
+    sync();
+    if (*abort_flag) break;
+    {
+      const float ikr = __shfl_sync(0xffffffffu, inv, 16 + 2 * (lane & 7));  // 1/|k| of row 8 iw + (lane & 7)
+      if (lane < 8) {
+        const int r = 8 * iw + lane;
+        sc_beta[slot * 64 + r] = beta_l;
+        sc_ik[slot * 64 + r] = (r < len) ? ikr : 0.f;
+      }
+    }
+    if (iw == 0) reinterpret_cast<float4*>(sc_gam + slot * 128)[lane] = make_float4(gam[0], gam[1], gam[2], gam[3]);
+
+    // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i
+    {
+      float run[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) run[j] = upper_half ? pt[j] : 1.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int r = 8 * warp + i;
+        const int r = 8 * iw + i;
+        const float iq = __shfl_sync(0xffffffffu, inv, 2 * i) * p.scale;
+        const float ik = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);
+        const float b = __shfl_sync(0xffffffffu, beta_l, i);
         const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
         const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
         const float qv[4] = {q01.x, q01.y, q23.x, q23.y};
         const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
-        float lk[4], lq[4], kf[4];
+        float lk[4], lq[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float kh = kv[j] * ik[i];
-          lq[j] = qv[j] * iq[i] * al[i][j];   // scale * qhat * e
-          lk[j] = kh * al[i][j];              // khat * e
-          kf[j] = kh * suf[i][j];             // khat * f
+          run[j] *= a[i][j];
+          lq[j] = qv[j] * iq * run[j];   // scale * qhat * e
+          lk[j] = kv[j] * ik * run[j];   // khat * e
         }
         const uint32_t offk = kb * 16384 + sw128(r, lane_chunk) + lane_sub;
         const uint32_t offq = kb * 16384 + sw128(64 + r, lane_chunk) + lane_sub;
         const uint32_t off64 = kb * 8192 + sw128(r, lane_chunk) + lane_sub;
-        const float b = bt[i];
         *reinterpret_cast<uint2*>(sm + OFF_LKQ + offk) =
             make_uint2(pack_bf16(lk[0] * b, lk[1] * b), pack_bf16(lk[2] * b, lk[3] * b));
-        *reinterpret_cast<uint2*>(sm + OFF_LKQ + offq) =
-            make_uint2(pack_bf16(lq[0], lq[1]), pack_bf16(lq[2], lq[3]));
+        *reinterpret_cast<uint2*>(sm + OFF_LKQ + offq) = make_uint2(pack_bf16(lq[0], lq[1]), pack_bf16(lq[2], lq[3]));
+        *reinterpret_cast<uint2*>(sm + OFF_XK + off64) =
+            make_uint2(pack_bf16(lk[0] * pre[0], lk[1] * pre[1]), pack_bf16(lk[2] * pre[2], lk[3] * pre[3]));
+        *reinterpret_cast<uint2*>(sm + OFF_QB + off64) =
+            make_uint2(pack_bf16(lq[0] * pre[0], lq[1] * pre[1]), pack_bf16(lq[2] * pre[2], lq[3] * pre[3]));
+      }
+    }
+    // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end
+    uint2 kt_pack[8];
+    {
+      float run[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) run[j] = upper_half ? 1.f : pt[j];
+#pragma unroll
+      for (int i = 7; i >= 0; --i) {
+        const int r = 8 * iw + i;
+        const float ik = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);
+        const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
+        const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
+        float kf[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) kf[j] = kv[j] * ik * run[j];   // khat * f
 #pragma unroll
         for (int I = 0; I < 4; ++I) {
           if (I < blk) continue;
@@ -403,48 +545,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint2*>(sm + OFF_R + off) =
               make_uint2(pack_bf16(kf[0] * cI[I][0], kf[1] * cI[I][1]), pack_bf16(kf[2] * cI[I][2], kf[3] * cI[I][3]));
         }
-        *reinterpret_cast<uint2*>(sm + OFF_XK + off64) =
-            make_uint2(pack_bf16(lk[0] * pre[0], lk[1] * pre[1]), pack_bf16(lk[2] * pre[2], lk[3] * pre[3]));
-        *reinterpret_cast<uint2*>(sm + OFF_QB + off64) =
-            make_uint2(pack_bf16(lq[0] * pre[0], lq[1] * pre[1]), pack_bf16(lq[2] * pre[2], lq[3] * pre[3]));
-        *reinterpret_cast<uint2*>(sm + OFF_KT + off64) =
-            make_uint2(pack_bf16(kv[0] * suf[i][0] * post[0], kv[1] * suf[i][1] * post[1]),
-                       pack_bf16(kv[2] * suf[i][2] * post[2], kv[3] * suf[i][3] * post[3]));
+        kt_pack[i] = make_uint2(pack_bf16(kv[0] * (run[0] * post[0]), kv[1] * (run[1] * post[1])),
+                                pack_bf16(kv[2] * (run[2] * post[2]), kv[3] * (run[3] * post[3])));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) run[j] *= a[i][j];
       }
     }
-    publish();
+    load_g(c + 1);
+    fence_proxy_async();
+    sync();
+    if (itid == 0) mbar_arrive(S_.bar + B_OPS0 + slot);
+    // Ktil: the previous chunk's is read by MMA2 until it has run
+    if (c > 0) wait_bar(S_, B_MMA2, (c - 1) & 1, p.status);
+    sync();
+    if (*abort_flag) break;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 8 * iw + i;
+      *reinterpret_cast<uint2*>(sm + OFF_KT + kb * 8192 + sw128(r, lane_chunk) + lane_sub) = kt_pack[i];
+    }
+    fence_proxy_async();
+    sync();
+    if (itid == 0) mbar_arrive(S_.bar + B_KT);
 
-    // ================================================================ MMA_AP
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int I = 0; I < 4; ++I) {
-        const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t a = sdesc_sw128(sbase + OFF_LKQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(sbase + OFF_R + (ks >> 2) * R_KBLK + row_off(I) * 128 + (ks & 3) * 32, 16, 1024);
-          umma_bf16(tmem + row_off(I), a, b, idesc, ks > 0);
-        }
-      }
-      umma_commit(mma_bar);
-    }
-    if (!wait_all(mma_bar, mma_phase)) break;
+    // ============================================================== assemble A and P
+    wait_bar(S_, B_AP, c & 1, p.status);
+    sync();
+    if (*abort_flag) break;
     tc_fence_after();
-
-    // ================================================================ assemble A and P
     {
-      const int R = 32 * quarter + lane;  // accumulator row
+      const int R = 32 * quarter + lane;
       const bool qside = R >= 64;
       const int r = R & 63;
       const int Ib = r >> 4;
-      const int q2 = quarter & 1;         // rows 32*q2 .. 32*q2+31 of this side: blocks 2 q2, 2 q2 + 1
-      const bool skip = (half == 1) && (q2 == 0);  // s in [32, 64) lies above the diagonal there
+      const int q2 = quarter & 1;
+      const bool skip = (ihalf == 1) && (q2 == 0);
       float d[32];
       if (!skip) {
         float d0[32], d1[32];
-        tmem_ld32(tmem + lane_base + row_off(2 * q2) + 32 * half, d0);
-        tmem_ld32(tmem + lane_base + row_off(2 * q2 + 1) + 32 * half, d1);
+        tmem_ld32(tmem + lane_base + row_off(2 * q2) + 32 * ihalf, d0);
+        tmem_ld32(tmem + lane_base + row_off(2 * q2 + 1) + 32 * ihalf, d1);
         const bool odd = Ib & 1;
 #pragma unroll
         for (int j = 0; j < 32; ++j) d[j] = odd ? d1[j] : d0[j];
@@ -453,10 +593,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j) d[j] = 0.f;
       }
       if (!qside) {
-        float* dst = As + r * AS_LD + 32 * half;
+        float* dst = As + r * AS_LD + 32 * ihalf;
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-          const int s = 32 * half + j;
+          const int s = 32 * ihalf + j;
           float4 o;
           o.x = (s + 0 < r) ? d[j + 0] : 0.f;
           o.y = (s + 1 < r) ? d[j + 1] : 0.f;
@@ -470,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v8[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int s = 32 * half + 8 * cch + u;
+            const int s = 32 * ihalf + 8 * cch + u;
             v8[u] = (s <= r) ? d[8 * cch + u] : 0.f;
           }
           uint4 w;
@@ -478,59 +618,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.y = pack_bf16(v8[2], v8[3]);
           w.z = pack_bf16(v8[4], v8[5]);
           w.w = pack_bf16(v8[6], v8[7]);
-          *reinterpret_cast<uint4*>(sm + OFF_TP + sw128(64 + r, 4 * half + cch)) = w;
+          *reinterpret_cast<uint4*>(sm + OFF_TP + sw128(64 + r, 4 * ihalf + cch)) = w;
         }
       }
     }
     tc_fence_before();
-    bar_sync();
+    sync();
 
-    // ================================================================ solve T = (I + A)^{-1}
-    // diagonal 16x16 blocks: warp I, lane j < 16 computes column j by forward substitution
-    if (warp < 4 && lane < 16) {
-      const int I = warp, j = lane;
-      const float* a = As + (16 * I) * AS_LD + 16 * I;
+    // ============================================================== solve T = (I + A)^{-1}
+    if (iw < 4 && lane < 16) {
+      const int I = iw, j = lane;
+      const float* ab = As + (16 * I) * AS_LD + 16 * I;
       float x[16];
 #pragma unroll
       for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
+      // right-looking substitution: once x[m] is final, fold it into every later row
 #pragma unroll
-      for (int i = 1; i < 16; ++i) {
-        float acc = 0.f;
+      for (int m = 0; m < 15; ++m) {
+        const float xm = x[m];
 #pragma unroll
-        for (int m = 0; m < i; ++m) acc = fmaf(a[i * AS_LD + m], x[m], acc);
-        x[i] = (i > j) ? -acc : x[i];
+        for (int i = m + 1; i < 16; ++i) x[i] = fmaf(-ab[i * AS_LD + m], xm, x[i]);
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = x[i];
+      for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = (i >= j) ? x[i] : 0.f;
     }
-    bar_sync();
-    // off-diagonal blocks by distance dd below the diagonal: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
+    sync();
 #pragma unroll 1
     for (int dd = 1; dd < 4; ++dd) {
       const int nblk = 4 - dd;
-      const int job = tid;                  // (block, row i, 4-column group)
+      const int job = itid;
       const bool active = job < nblk * 64;
-      const int bI = dd + job / 64;         // block row I (J = I - dd)
-      const int bJ = bI - dd;
+      const int bI = dd + job / 64;
+      const int bJ2 = bI - dd;
       const int i = (job % 64) >> 2, cg = job & 3;
       if (active) {
         float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-        for (int K = bJ; K < bI; ++K) {
+        for (int K = bJ2; K < bI; ++K) {
           const float* arow = As + (16 * bI + i) * AS_LD + 16 * K;
-          const float* tcol = Ts + (16 * K) * AS_LD + 16 * bJ + 4 * cg;
+          const float* tcol = Ts + (16 * K) * AS_LD + 16 * bJ2 + 4 * cg;
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            const float a = arow[m];
+            const float av = arow[m];
             const float4 t = *reinterpret_cast<const float4*>(tcol + m * AS_LD);
-            y0 = fmaf(a, t.x, y0);
-            y1 = fmaf(a, t.y, y1);
-            y2 = fmaf(a, t.z, y2);
-            y3 = fmaf(a, t.w, y3);
+            y0 = fmaf(av, t.x, y0);
+            y1 = fmaf(av, t.y, y1);
+            y2 = fmaf(av, t.z, y2);
+            y3 = fmaf(av, t.w, y3);
           }
         }
         *reinterpret_cast<float4*>(Ys + (job / 64) * 256 + i * 16 + 4 * cg) = make_float4(y0, y1, y2, y3);
       }
-      bar_sync();
+      sync();
       if (active) {
         const float* trow = Ts + (16 * bI + i) * AS_LD + 16 * bI;
         const float* ycol = Ys + (job / 64) * 256 + 4 * cg;
@@ -544,14 +682,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           z2 = fmaf(t, y.z, z2);
           z3 = fmaf(t, y.w, z3);
         }
-        *reinterpret_cast<float4*>(Ts + (16 * bI + i) * AS_LD + 16 * bJ + 4 * cg) = make_float4(-z0, -z1, -z2, -z3);
+        *reinterpret_cast<float4*>(Ts + (16 * bI + i) * AS_LD + 16 * bJ2 + 4 * cg) = make_float4(-z0, -z1, -z2, -z3);
       }
-      bar_sync();
+      sync();
     }
-    // T_b = T diag(beta) as hi/lo bf16 into rows 0..63 of TP / TL (upper blocks are zero)
     {
-      const int r = tid >> 2, c16 = tid & 3;   // row r, columns 16*c16 .. 16*c16+15
+      const int r = itid >> 2, c16 = itid & 3;
       const int I = r >> 4;
+      const float* sb = sc_beta + slot * 64;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int c0 = 16 * c16 + 8 * hh;
@@ -562,8 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const float4 t0v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0);
           const float4 t1v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0 + 4);
-          const float4 b0 = *reinterpret_cast<const float4*>(sc_beta + c0);
-          const float4 b1 = *reinterpret_cast<const float4*>(sc_beta + c0 + 4);
+          const float4 b0 = *reinterpret_cast<const float4*>(sb + c0);
+          const float4 b1 = *reinterpret_cast<const float4*>(sb + c0 + 4);
           split2(t0v.x * b0.x, t0v.y * b0.y, wh.x, wl.x);
           split2(t0v.z * b0.z, t0v.w * b0.w, wh.y, wl.y);
           split2(t1v.x * b1.x, t1v.y * b1.y, wh.z, wl.z);
@@ -573,26 +711,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(sm + OFF_TL + sw128(r, c0 >> 3)) = wl;
       }
     }
-    publish();
+    fence_proxy_async();
+    sync();
+    if (itid == 0) mbar_arrive(S_.bar + B_TB);
 
-    // ================================================================ MMA_PT: [T_hi; P] x (T_hi + T_lo)
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t a = sdesc_sw128(sbase + OFF_TP + (ks & 3) * 32, 16, 1024);
-        const uint64_t b = sdesc_sw128(sbase + (ks < 4 ? OFF_TP : OFF_TL) + (ks & 3) * 2048, 8192, 1024);
-        umma_bf16(tmem, a, b, idesc, ks > 0);
-      }
-      umma_commit(mma_bar);
-    }
-    if (!wait_all(mma_bar, mma_phase)) break;
+    // ============================================================== P T_b
+    wait_bar(S_, B_PT, c & 1, p.status);
+    if (len < C) wait_bar(S_, B_V_FULL, c & 1, p.status);
+    sync();
+    if (*abort_flag) break;
     tc_fence_after();
     if (quarter >= 2) {
       const int r = 32 * quarter + lane - 64;
       float d[32];
-      tmem_ld32(tmem + lane_base + 32 * half, d);
+      tmem_ld32(tmem + lane_base + 32 * ihalf, d);
 #pragma unroll
       for (int cch = 0; cch < 4; ++cch) {
         uint4 wh, wl;
@@ -600,58 +732,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         split2(d[8 * cch + 2], d[8 * cch + 3], wh.y, wl.y);
         split2(d[8 * cch + 4], d[8 * cch + 5], wh.z, wl.z);
         split2(d[8 * cch + 6], d[8 * cch + 7], wh.w, wl.w);
-        *reinterpret_cast<uint4*>(sm + OFF_TP + sw128(64 + r, 4 * half + cch)) = wh;
-        *reinterpret_cast<uint4*>(sm + OFF_TL + sw128(64 + r, 4 * half + cch)) = wl;
+        *reinterpret_cast<uint4*>(sm + OFF_TP + sw128(64 + r, 4 * ihalf + cch)) = wh;
+        *reinterpret_cast<uint4*>(sm + OFF_TL + sw128(64 + r, 4 * ihalf + cch)) = wl;
       }
     }
-    publish();
-
-    // ================================================================ MMA_X: [T_b; P T_b] x [Xk | V]
-    if (!wait_all(tma_bar, tma_phase)) break;   // v tile of this chunk
-    if (len < C) {  // rows past the document end (another document's or zero-filled) -> 0
-      for (int idx = tid; idx < 2 * (C - len) * 8; idx += kThreads) {
+    if (len < C) {
+      // rows of the v tile past the document end (another document's, or zero-filled) -> 0
+      for (int idx = itid; idx < 2 * (C - len) * 8; idx += kIntraThreads) {
         const int blk2 = idx / ((C - len) * 8), rem = idx % ((C - len) * 8);
-        const int r = len + rem / 8;
-        *reinterpret_cast<uint4*>(sm + OFF_V + blk2 * 8192 + sw128(r, rem & 7)) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sm + OFF_V + blk2 * 8192 + sw128(len + rem / 8, rem & 7)) = make_uint4(0, 0, 0, 0);
       }
-      fence_proxy_async();
-      bar_sync();
     }
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t a = sdesc_sw128(sbase + (ks < 4 ? OFF_TP : OFF_TL) + (ks & 3) * 32, 16, 1024);
-        const uint64_t bk = sdesc_sw128(sbase + OFF_XK + (ks & 3) * 2048, 8192, 1024);
-        const uint64_t bv = sdesc_sw128(sbase + OFF_V + (ks & 3) * 2048, 8192, 1024);
-        umma_bf16(tmem + TM_WQ, a, bk, idesc, ks > 0);
-        umma_bf16(tmem + TM_UP, a, bv, idesc, ks > 0);
-      }
-      umma_commit(mma_bar);
-    }
-    if (!wait_all(mma_bar, mma_phase)) break;
-    tc_fence_after();
-    // the v tile is free: fetch the next chunk's
-    if (tid == 0 && c + 1 < nchunks) {
-      mbar_arrive_expect_tx(tma_bar, 16384);
-      tma_load_3d(sm + OFF_V, &maps.v, tma_bar, 0, h, (int)(t0 + C));
-      tma_load_3d(sm + OFF_V + 8192, &maps.v, tma_bar, 64, h, (int)(t0 + C));
-    }
+    fence_proxy_async();
+    tc_fence_before();
+    sync();
+    if (itid == 0) mbar_arrive(S_.bar + B_TP);
 
-    // ================================================================ [-W; Qtil - PW] -> TMEM (bf16)
+    // ============================================================== [-W; Qtil - PW] -> TMEM
+    wait_bar(S_, B_XK, c & 1, p.status);
+    sync();
+    if (*abort_flag) break;
+    tc_fence_after();
     {
       const int R = 32 * quarter + lane;
       uint32_t packed[32];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         float d[32];
-        tmem_ld32(tmem + lane_base + TM_WQ + 64 * half + 32 * part, d);
+        tmem_ld32(tmem + lane_base + 64 * ihalf + 32 * part, d);
         if (R >= 64) {
           const int r = R - 64;
 #pragma unroll
           for (int cch = 0; cch < 4; ++cch) {
-            const uint4 qb = *reinterpret_cast<const uint4*>(sm + OFF_QB + half * 8192 + sw128(r, 4 * part + cch));
+            const uint4 qb = *reinterpret_cast<const uint4*>(sm + OFF_QB + ihalf * 8192 + sw128(r, 4 * part + cch));
             const float2 a0 = unpack_bf16(qb.x), a1 = unpack_bf16(qb.y), a2 = unpack_bf16(qb.z),
                          a3 = unpack_bf16(qb.w);
             packed[16 * part + 4 * cch + 0] = pack_bf16(a0.x - d[8 * cch + 0], a0.y - d[8 * cch + 1]);
@@ -665,36 +778,106 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      bar_sync();   // every thread has read [W PW] before any column 0..63 is overwritten
+      sync();  // every [W PW] column read before any is overwritten
       tc_fence_after();
-      tmem_st32(tmem + lane_base + TM_WQ + 32 * half, packed);
+      tmem_st32(tmem + lane_base + 32 * ihalf, packed);
       tmem_wait_st();
     }
-    publish();
+    tc_fence_before();
+    sync();
+    if (itid == 0) mbar_arrive(S_.bar + B_WQ);
+  }
+}
 
-    // ================================================================ MMA1: [U; PU] += [-W; Qtil - PW] x S
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+// ------------------------------------------------------------------------------ recurrence warps
+__device__ void rec_warps(const Shared& S_, const FwdParams& p, int n, int h, int64_t bos, int64_t eos,
+                          int nchunks, int rtid) {
+  uint8_t* sm = S_.sm;
+  const uint32_t tmem = S_.tmem;
+  const int H = p.num_heads;
+  const int quarter = rtid >> 5, lane = rtid & 31;
+  const int R = 32 * quarter + lane;  // TMEM lane: state row k, or chunk row (Delta / O)
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+  const float* sc_ik = reinterpret_cast<const float*>(sm + OFF_SC + SC_IK);
+  const float* sc_gam = reinterpret_cast<const float*>(sm + OFF_SC + SC_GAM);
+  const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
+
+  auto store_row_bf16 = [&](int part, const float (&v)[32]) {
+    // columns 32 part .. 32 part + 31 of row R of the bf16 state (MN tile of 128 rows)
+    uint8_t* base = sm + OFF_S + (part >> 1) * (128 * 128);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t b = sdesc_sw128(sbase + OFF_S + ks * 2048, 16384, 1024);
-        umma_bf16_tmem_a(tmem + TM_UP, tmem + TM_WQ + 8 * ks, b, idesc, 1);
-      }
-      umma_commit(mma_bar);
+    for (int c = 0; c < 4; ++c) {
+      uint4 w;
+      w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
+      w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
+      w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
+      w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
+      *reinterpret_cast<uint4*>(base + sw128(R, 4 * (part & 1) + c)) = w;
     }
-    if (!wait_all(mma_bar, mma_phase)) break;
-    tc_fence_after();
-
-    // ================================================================ ep1: Delta and O
-    {
-      const int R = 32 * quarter + lane;
-      const int r = R & 63;
-      const float ikr = sc_ik[r];
+  };
+  auto store_final = [&](int part, const float (&v)[32]) {
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
+    for (int j = 0; j < 32; ++j) {
+      const int col = 32 * part + j;
+      if (p.state_transposed) p.final_state[soff + (size_t)col * D + R] = v[j];
+      else p.final_state[soff + (size_t)R * D + col] = v[j];
+    }
+  };
+
+  // initial state: bf16 copy for MMA1(0); fp32 copy pre-scaled by e^{Gamma_C}(0) for MMA2(0)
+  {
+    bool ok = true;
+    if (nchunks > 0) ok = wait_bar(S_, B_OPS0, 0, p.status);
+    const float gam = (nchunks > 0 && ok) ? sc_gam[R] : 1.f;
+#pragma unroll 1
+    for (int part = 0; part < 4; ++part) {
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int col = 32 * part + j;
+        float s = 0.f;
+        if (p.initial_state)
+          s = p.state_transposed ? p.initial_state[soff + (size_t)col * D + R]
+                                 : p.initial_state[soff + (size_t)R * D + col];
+        v[j] = s;
+      }
+      if (nchunks == 0) {
+        if (p.final_state) store_final(part, v);
+        continue;
+      }
+      store_row_bf16(part, v);
+      uint32_t u[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam * v[j]);
+      tmem_st32(tmem + lane_base + TM_S + 32 * part, u);
+    }
+    if (nchunks == 0) return;
+    tmem_wait_st();
+    fence_proxy_async();
+    tc_fence_before();
+    named_bar(kBarRec, kRecThreads);
+    if (*S_.abort) return;
+    if (rtid == 0) mbar_arrive(S_.bar + B_S);
+  }
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int64_t t0 = bos + (int64_t)c * C;
+    const int len = (int)((eos - t0) < (int64_t)C ? (eos - t0) : (int64_t)C);
+    const int slot = c & 1;
+    // ============================================================== ep1: Delta and O
+    // the scalar slot of this chunk (1/|k|) is acquired from the intra warps' own barrier
+    wait_bar(S_, B_OPS0 + slot, (c >> 1) & 1, p.status);
+    wait_bar(S_, B_MMA1, c & 1, p.status);
+    named_bar(kBarRec, kRecThreads);
+    if (*S_.abort) break;
+    tc_fence_after();
+    {
+      const int r = R & 63;
+      const float ikr = sc_ik[slot * 64 + r];
+#pragma unroll 1
+      for (int part = 0; part < 4; ++part) {
         float d[32];
-        tmem_ld32(tmem + lane_base + TM_UP + 64 * half + 32 * part, d);
+        tmem_ld32(tmem + lane_base + TM_UP + 32 * part, d);
         if (R < 64) {
 #pragma unroll
           for (int cch = 0; cch < 4; ++cch) {
@@ -703,11 +886,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             split2(d[8 * cch + 2] * ikr, d[8 * cch + 3] * ikr, wh.y, wl.y);
             split2(d[8 * cch + 4] * ikr, d[8 * cch + 5] * ikr, wh.z, wl.z);
             split2(d[8 * cch + 6] * ikr, d[8 * cch + 7] * ikr, wh.w, wl.w);
-            *reinterpret_cast<uint4*>(sm + OFF_DL + half * 8192 + sw128(r, 4 * part + cch)) = wh;
-            *reinterpret_cast<uint4*>(sm + OFF_DLLO + half * 8192 + sw128(r, 4 * part + cch)) = wl;
+            const uint32_t off = (part >> 1) * 8192 + sw128(r, 4 * (part & 1) + cch);
+            *reinterpret_cast<uint4*>(sm + OFF_DL + off) = wh;
+            *reinterpret_cast<uint4*>(sm + OFF_DLLO + off) = wl;
           }
         } else if (r < len) {
-          __nv_bfloat16* orow = p.out + ((size_t)(t0 + r) * H + h) * D + 64 * half + 32 * part;
+          __nv_bfloat16* orow = p.out + ((size_t)(t0 + r) * H + h) * D + 32 * part;
 #pragma unroll
           for (int cch = 0; cch < 4; ++cch) {
             uint4 w;
@@ -720,52 +904,104 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    publish();
+    fence_proxy_async();
+    tc_fence_before();
+    named_bar(kBarRec, kRecThreads);
+    if (rtid == 0) mbar_arrive(S_.bar + B_DELTA);
 
-    // ================================================================ MMA2: Ktil^T x (Delta_hi + Delta_lo)
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(128, 128, true, true);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t a = sdesc_sw128(sbase + OFF_KT + (ks & 3) * 2048, 8192, 1024);
-        const uint64_t b = sdesc_sw128(sbase + (ks < 4 ? OFF_DL : OFF_DLLO) + (ks & 3) * 2048, 8192, 1024);
-        umma_bf16(tmem + TM_UP, a, b, idesc, ks > 0);
-      }
-      umma_commit(mma_bar);
-    }
-    if (!wait_all(mma_bar, mma_phase)) break;
+    // ============================================================== ep2: state
+    wait_bar(S_, B_MMA2, c & 1, p.status);
+    const bool last = (c + 1 == nchunks);
+    if (!last) wait_bar(S_, B_OPS0 + ((c + 1) & 1), ((c + 1) >> 1) & 1, p.status);
+    named_bar(kBarRec, kRecThreads);
+    if (*S_.abort) break;
     tc_fence_after();
-
-    // ================================================================ ep2: state update
     {
-      const float gam = sc_gam[srow];
+      const float gam = last ? 1.f : sc_gam[((c + 1) & 1) * 128 + R];
+#pragma unroll 1
+      for (int part = 0; part < 4; ++part) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + TM_S + 32 * part, v);
+        if (last) {
+          if (p.final_state) store_final(part, v);
+        } else {
+          store_row_bf16(part, v);
+          uint32_t u[32];
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        float d[32];
-        tmem_ld32(tmem + lane_base + TM_UP + 64 * half + 32 * part, d);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) S[32 * part + j] = fmaf(gam, S[32 * part + j], d[j]);
+          for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam * v[j]);
+          tmem_st32(tmem + lane_base + TM_S + 32 * part, u);
+        }
       }
-      store_state_bf16();
+      if (!last) tmem_wait_st();
     }
-    publish();
+    if (last) break;
+    fence_proxy_async();
+    tc_fence_before();
+    named_bar(kBarRec, kRecThreads);
+    if (rtid == 0) mbar_arrive(S_.bar + B_S);
   }
+}
 
-  // ---- final state
-  if (p.final_state && *sc_abort == 0) {
-#pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      const int col = 64 * half + j;
-      if (p.state_transposed) p.final_state[soff + (size_t)col * D + srow] = S[j];
-      else p.final_state[soff + (size_t)srow * D + col] = S[j];
-    }
+__global__ void __launch_bounds__(kThreads, 1)
+    chunked_kernel(const __grid_constant__ TensorMaps maps, FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Shared S_;
+  S_.sm = sm;
+  S_.sbase = smem_u32(sm);
+  S_.bar = reinterpret_cast<uint64_t*>(sm + OFF_SC + SC_BAR);
+  S_.abort = reinterpret_cast<volatile int*>(sm + OFF_SC + SC_ABORT);
+  uint32_t* sc_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SC + SC_TMEM);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int H = p.num_heads;
+  const int n = blockIdx.x / H, h = blockIdx.x % H;
+  int64_t bos, eos;
+  seq_range(p, n, bos, eos);
+  const int nchunks = (int)((eos - bos + C - 1) / C);
+
+  if (tid == 0) {
+    for (int b = 0; b < B_COUNT; ++b) mbar_init(S_.bar + b, 1);
+    *S_.abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.k);
+    prefetch_tmap(&maps.v);
+  }
+  if (warp == 0) {
+    tmem_alloc(sc_tmem, kTmemCols);
+    tmem_relinquish();
   }
   tc_fence_before();
-  bar_sync();
+  __syncthreads();
+  tc_fence_after();
+  S_.tmem = *sc_tmem;
+
+  // register budget per warpgroup: control 56, intra 168, recurrence 96 (4*56 + 8*168 + 4*96 warps-worth
+  // of 32-thread rows = 62464 <= 65536)
+  if (warp < kIntraWarp0) {
+    setmaxnreg_dec<56>();
+    if (warp == 0) {
+      if (lane == 0) mma_issuer(S_, p, nchunks);
+      __syncwarp();
+    } else if (warp == 1) {
+      if (lane == 0) tma_producer(S_, maps, p, h, bos, nchunks);
+      __syncwarp();
+    }
+  } else if (warp < kRecWarp0) {
+    setmaxnreg_inc<168>();
+    intra_warps(S_, p, h, bos, eos, nchunks, tid - 32 * kIntraWarp0);
+  } else {
+    setmaxnreg_dec<96>();
+    rec_warps(S_, p, n, h, bos, eos, nchunks, tid - 32 * kRecWarp0);
+  }
+
+  tc_fence_before();
+  __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(S_.tmem, kTmemCols);
   }
 }
 
@@ -808,7 +1044,9 @@ cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream) {
   if (units == 0) return cudaSuccess;
   const int64_t tokens = p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs;
   TensorMaps maps;
-  if (!make_token_map(&maps.v, p.v, tokens, p.num_heads)) return cudaErrorInvalidValue;
+  if (!make_token_map(&maps.q, p.q, tokens, p.num_heads) || !make_token_map(&maps.k, p.k, tokens, p.num_heads) ||
+      !make_token_map(&maps.v, p.v, tokens, p.num_heads))
+    return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
