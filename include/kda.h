@@ -100,6 +100,25 @@ kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, cons
                                int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v,
                                int32_t num_seqs, int32_t state_transposed, kda_stream_t stream);
 
+/* kda_fwd for callers that cannot allocate device memory (for example runtimes that plan every
+ * device buffer ahead of time and forbid libraries from calling cudaMalloc, or code that must not
+ * trigger cudaMalloc's device-wide synchronisation).  The pages have no counterpart to this entry
+ * point.  Same arguments and results as kda_fwd, minus the workspace: it uses a device array that
+ * lives in the library (16.6 KB per GPU, held until the process exits) and allocates nothing.
+ *   - At most 4096 (sequence, head) units per call; more returns KDA_ERR_WORKSPACE_TOO_SMALL.
+ *   - The first call on a device looks up the array's address on that device; make it before any
+ *     stream capture.
+ *   - All calls share the array: calls that overlap on the GPU race on it.
+ *   - Each call clears the array's status word; device time-outs are not reported by this call. */
+kda_status_t kda_fwd_static_workspace(const void* q, const void* k, const void* v, const void* g,
+                                      const void* beta, float scale, void* out, const float* A_log,
+                                      const float* dt_bias, float lower_bound,
+                                      const float* initial_state, float* final_state,
+                                      const int32_t* cu_seqlens, int32_t batch, int64_t seqlen,
+                                      int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v,
+                                      int32_t num_seqs, int32_t state_transposed,
+                                      kda_stream_t stream);
+
 /* Synchronises `stream`, reads the workspace's sticky status word, clears it, and returns
  * KDA_OK or the recorded device error (KDA_ERR_DEVICE_TIMEOUT).  KDA_ERR_CUDA if the copy fails. */
 kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream);
