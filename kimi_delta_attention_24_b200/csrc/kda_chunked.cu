@@ -346,7 +346,8 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
   const int blk = iw >> 1;
   const bool upper_half = iw & 1;
 
-  uint2 gr[8];  // raw g of the chunk being prepared (loaded one chunk ahead)
+  uint2 gr[8];        // raw g of the chunk being prepared (loaded one chunk ahead)
+  float beta_raw = 0.f;  // raw beta of row 8 iw + lane (lanes 0..7), loaded with g
   auto load_g = [&](int c) {
     const int64_t t0 = bos + (int64_t)c * C;
 #pragma unroll
@@ -354,8 +355,19 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
       const int64_t t = t0 + 8 * iw + i;
       gr[i] = (c < nchunks && t < eos) ? ldg_u2(p.g + ((size_t)t * H + h) * D + 4 * lane) : make_uint2(0, 0);
     }
+    const int64_t tb = t0 + 8 * iw + (lane & 7);
+    beta_raw = (c < nchunks && tb < eos) ? __bfloat162float(p.beta[(size_t)tb * H + h]) : 0.f;
   };
   load_g(0);
+  // shared-memory byte offset of this thread's 8 bytes of row 8 iw + i inside a 128-byte-row tile
+  uint32_t xo[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) xo[i] = (uint32_t)((8 * iw + i) * 128) + (((lane_chunk ^ i) & 7u) << 4) + lane_sub;
+  const uint32_t sbase = S_.sbase;
+  const uint32_t a_rq = sbase + OFF_RQ + kb * 8192, a_rk = sbase + OFF_RK + kb * 8192;
+  const uint32_t a_lk = sbase + OFF_LKQ + kb * 16384, a_lq = a_lk + 64 * 128;
+  const uint32_t a_xk = sbase + OFF_XK + kb * 8192, a_qb = sbase + OFF_QB + kb * 8192, a_kt = sbase + OFF_KT + kb * 8192;
+  const uint32_t a_r = sbase + OFF_R + kb * R_KBLK;
 
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = bos + (int64_t)c * C;
@@ -367,11 +379,9 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
     uint2 qr[8], kr[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int r = 8 * iw + i;
-      const uint32_t off = kb * 8192 + sw128(r, lane_chunk) + lane_sub;
-      const bool valid = r < len;
-      qr[i] = valid ? *reinterpret_cast<const uint2*>(sm + OFF_RQ + off) : make_uint2(0, 0);
-      kr[i] = valid ? *reinterpret_cast<const uint2*>(sm + OFF_RK + off) : make_uint2(0, 0);
+      const bool valid = 8 * iw + i < len;
+      qr[i] = valid ? lds64(a_rq + xo[i]) : make_uint2(0, 0);
+      kr[i] = valid ? lds64(a_rk + xo[i]) : make_uint2(0, 0);
     }
     sync();
     if (*abort_flag) break;
@@ -425,10 +435,13 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
       w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
       inv = rsqrtf(w1 + kL2Eps);
     }
-    float beta_l = 0.f;
-    if (lane < 8) {
-      const int r = 8 * iw + lane;
-      if (r < len) beta_l = fast_sigmoid(__bfloat162float(p.beta[(size_t)(t0 + r) * H + h]));
+    const float beta_l = (lane < 8 && 8 * iw + lane < len) ? fast_sigmoid(beta_raw) : 0.f;
+    float iqv[8], ikv[8], btv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      iqv[i] = __shfl_sync(0xffffffffu, inv, 2 * i) * p.scale;
+      ikv[i] = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);
+      btv[i] = __shfl_sync(0xffffffffu, beta_l, i);
     }
     // per-warp alpha totals -> sub-block totals b_J
     float tot[4];
@@ -496,10 +509,6 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
       for (int j = 0; j < 4; ++j) run[j] = upper_half ? pt[j] : 1.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int r = 8 * iw + i;
-        const float iq = __shfl_sync(0xffffffffu, inv, 2 * i) * p.scale;
-        const float ik = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);
-        const float b = __shfl_sync(0xffffffffu, beta_l, i);
         const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
         const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
         const float qv[4] = {q01.x, q01.y, q23.x, q23.y};
@@ -508,19 +517,14 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           run[j] *= a[i][j];
-          lq[j] = qv[j] * iq * run[j];   // scale * qhat * e
-          lk[j] = kv[j] * ik * run[j];   // khat * e
+          lk[j] = kv[j] * (run[j] * ikv[i]);   // khat * e
+          lq[j] = qv[j] * (run[j] * iqv[i]);   // scale * qhat * e
         }
-        const uint32_t offk = kb * 16384 + sw128(r, lane_chunk) + lane_sub;
-        const uint32_t offq = kb * 16384 + sw128(64 + r, lane_chunk) + lane_sub;
-        const uint32_t off64 = kb * 8192 + sw128(r, lane_chunk) + lane_sub;
-        *reinterpret_cast<uint2*>(sm + OFF_LKQ + offk) =
-            make_uint2(pack_bf16(lk[0] * b, lk[1] * b), pack_bf16(lk[2] * b, lk[3] * b));
-        *reinterpret_cast<uint2*>(sm + OFF_LKQ + offq) = make_uint2(pack_bf16(lq[0], lq[1]), pack_bf16(lq[2], lq[3]));
-        *reinterpret_cast<uint2*>(sm + OFF_XK + off64) =
-            make_uint2(pack_bf16(lk[0] * pre[0], lk[1] * pre[1]), pack_bf16(lk[2] * pre[2], lk[3] * pre[3]));
-        *reinterpret_cast<uint2*>(sm + OFF_QB + off64) =
-            make_uint2(pack_bf16(lq[0] * pre[0], lq[1] * pre[1]), pack_bf16(lq[2] * pre[2], lq[3] * pre[3]));
+        const float b = btv[i];
+        sts64(a_lk + xo[i], bf16x2(lk[0] * b, lk[1] * b), bf16x2(lk[2] * b, lk[3] * b));
+        sts64(a_lq + xo[i], bf16x2(lq[0], lq[1]), bf16x2(lq[2], lq[3]));
+        sts64(a_xk + xo[i], bf16x2(lk[0] * pre[0], lk[1] * pre[1]), bf16x2(lk[2] * pre[2], lk[3] * pre[3]));
+        sts64(a_qb + xo[i], bf16x2(lq[0] * pre[0], lq[1] * pre[1]), bf16x2(lq[2] * pre[2], lq[3] * pre[3]));
       }
     }
     // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end
@@ -531,22 +535,19 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
       for (int j = 0; j < 4; ++j) run[j] = upper_half ? 1.f : pt[j];
 #pragma unroll
       for (int i = 7; i >= 0; --i) {
-        const int r = 8 * iw + i;
-        const float ik = __shfl_sync(0xffffffffu, inv, 16 + 2 * i);
         const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
         const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
         float kf[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) kf[j] = kv[j] * ik * run[j];   // khat * f
+        for (int j = 0; j < 4; ++j) kf[j] = kv[j] * (run[j] * ikv[i]);   // khat * f
 #pragma unroll
         for (int I = 0; I < 4; ++I) {
           if (I < blk) continue;
-          const uint32_t off = kb * R_KBLK + sw128(row_off(I) + r, lane_chunk) + lane_sub;
-          *reinterpret_cast<uint2*>(sm + OFF_R + off) =
-              make_uint2(pack_bf16(kf[0] * cI[I][0], kf[1] * cI[I][1]), pack_bf16(kf[2] * cI[I][2], kf[3] * cI[I][3]));
+          sts64(a_r + row_off(I) * 128 + xo[i], bf16x2(kf[0] * cI[I][0], kf[1] * cI[I][1]),
+                bf16x2(kf[2] * cI[I][2], kf[3] * cI[I][3]));
         }
-        kt_pack[i] = make_uint2(pack_bf16(kv[0] * (run[0] * post[0]), kv[1] * (run[1] * post[1])),
-                                pack_bf16(kv[2] * (run[2] * post[2]), kv[3] * (run[3] * post[3])));
+        kt_pack[i] = make_uint2(bf16x2(kv[0] * (run[0] * post[0]), kv[1] * (run[1] * post[1])),
+                                bf16x2(kv[2] * (run[2] * post[2]), kv[3] * (run[3] * post[3])));
 #pragma unroll
         for (int j = 0; j < 4; ++j) run[j] *= a[i][j];
       }
@@ -560,10 +561,7 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
     sync();
     if (*abort_flag) break;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = 8 * iw + i;
-      *reinterpret_cast<uint2*>(sm + OFF_KT + kb * 8192 + sw128(r, lane_chunk) + lane_sub) = kt_pack[i];
-    }
+    for (int i = 0; i < 8; ++i) sts64(a_kt + xo[i], kt_pack[i].x, kt_pack[i].y);
     fence_proxy_async();
     sync();
     if (itid == 0) mbar_arrive(S_.bar + B_KT);
@@ -643,46 +641,72 @@ __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t
       for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = (i >= j) ? x[i] : 0.f;
     }
     sync();
+    // off-diagonal blocks by distance dd below the diagonal, one warp per block:
+    // T_IJ = -T_II (sum_{K=J}^{I-1} A_IK T_KJ), each 16x16x16 product on mma.sync m16n8k8 tf32
+    // with both operands split hi + lo (three products), i.e. fp32-level accuracy
 #pragma unroll 1
     for (int dd = 1; dd < 4; ++dd) {
-      const int nblk = 4 - dd;
-      const int job = itid;
-      const bool active = job < nblk * 64;
-      const int bI = dd + job / 64;
-      const int bJ2 = bI - dd;
-      const int i = (job % 64) >> 2, cg = job & 3;
-      if (active) {
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+      if (iw < 4 - dd) {
+        const int bI = dd + iw, bJ2 = iw;
+        const int g = lane >> 2, t = lane & 3;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         for (int K = bJ2; K < bI; ++K) {
-          const float* arow = As + (16 * bI + i) * AS_LD + 16 * K;
-          const float* tcol = Ts + (16 * K) * AS_LD + 16 * bJ2 + 4 * cg;
 #pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const float av = arow[m];
-            const float4 t = *reinterpret_cast<const float4*>(tcol + m * AS_LD);
-            y0 = fmaf(av, t.x, y0);
-            y1 = fmaf(av, t.y, y1);
-            y2 = fmaf(av, t.z, y2);
-            y3 = fmaf(av, t.w, y3);
+          for (int ks = 0; ks < 2; ++ks) {
+            const float* ab = As + (16 * bI + g) * AS_LD + 16 * K + 8 * ks + t;
+            uint32_t ah[4], al[4];
+            tf32_split(ab[0], ah[0], al[0]);
+            tf32_split(ab[8 * AS_LD], ah[1], al[1]);
+            tf32_split(ab[4], ah[2], al[2]);
+            tf32_split(ab[8 * AS_LD + 4], ah[3], al[3]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const float* tb = Ts + (16 * K + 8 * ks + t) * AS_LD + 16 * bJ2 + 8 * nt + g;
+              uint32_t bh0, bl0, bh1, bl1;
+              tf32_split(tb[0], bh0, bl0);
+              tf32_split(tb[4 * AS_LD], bh1, bl1);
+              mma_tf32(acc[nt], ah, bh0, bh1);
+              mma_tf32(acc[nt], ah, bl0, bl1);
+              mma_tf32(acc[nt], al, bh0, bh1);
+            }
           }
         }
-        *reinterpret_cast<float4*>(Ys + (job / 64) * 256 + i * 16 + 4 * cg) = make_float4(y0, y1, y2, y3);
-      }
-      sync();
-      if (active) {
-        const float* trow = Ts + (16 * bI + i) * AS_LD + 16 * bI;
-        const float* ycol = Ys + (job / 64) * 256 + 4 * cg;
-        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+        float* ys = Ys + iw * 256;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float t = (m <= i) ? trow[m] : 0.f;
-          const float4 y = *reinterpret_cast<const float4*>(ycol + m * 16);
-          z0 = fmaf(t, y.x, z0);
-          z1 = fmaf(t, y.y, z1);
-          z2 = fmaf(t, y.z, z2);
-          z3 = fmaf(t, y.w, z3);
+        for (int nt = 0; nt < 2; ++nt) {
+          ys[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
+          ys[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
+          ys[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
+          ys[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
         }
-        *reinterpret_cast<float4*>(Ts + (16 * bI + i) * AS_LD + 16 * bJ2 + 4 * cg) = make_float4(-z0, -z1, -z2, -z3);
+        __syncwarp();
+        float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const float* tr = Ts + (16 * bI + g) * AS_LD + 16 * bI + 8 * ks + t;
+          uint32_t ah[4], al[4];
+          tf32_split(tr[0], ah[0], al[0]);
+          tf32_split(tr[8 * AS_LD], ah[1], al[1]);
+          tf32_split(tr[4], ah[2], al[2]);
+          tf32_split(tr[8 * AS_LD + 4], ah[3], al[3]);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            uint32_t bh0, bl0, bh1, bl1;
+            tf32_split(ys[(8 * ks + t) * 16 + 8 * nt + g], bh0, bl0);
+            tf32_split(ys[(8 * ks + t + 4) * 16 + 8 * nt + g], bh1, bl1);
+            mma_tf32(z[nt], ah, bh0, bh1);
+            mma_tf32(z[nt], ah, bl0, bl1);
+            mma_tf32(z[nt], al, bh0, bh1);
+          }
+        }
+        float* to = Ts + (16 * bI) * AS_LD + 16 * bJ2;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          to[g * AS_LD + 8 * nt + 2 * t] = -z[nt][0];
+          to[g * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][1];
+          to[(g + 8) * AS_LD + 8 * nt + 2 * t] = -z[nt][2];
+          to[(g + 8) * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][3];
+        }
       }
       sync();
     }
