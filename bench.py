@@ -206,7 +206,7 @@ def main():
     N = x.num_seqs
     out = torch.empty_like(x.v)
     final = torch.empty(N, H, K, K, dtype=torch.float32, device=dev)
-    ws = torch.zeros(kda.get_workspace_size(B * T, H, N), dtype=torch.uint8, device=dev)
+    ws = kda.new_workspace(B * T, H, N, dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():

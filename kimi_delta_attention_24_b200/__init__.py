@@ -22,7 +22,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["fwd", "fwd_recurrent", "get_workspace_size", "is_supported", "chunk_kda",
+__all__ = ["fwd", "fwd_recurrent", "get_workspace_size", "new_workspace", "is_supported", "chunk_kda",
            "read_device_status", "KDAError", "library_path", "load"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +72,14 @@ def load():
 
 def get_workspace_size(T: int, H: int, N: int) -> int:
     return int(load().kda_workspace_size(int(T), int(H), int(N)))
+
+
+def new_workspace(T: int, H: int, N: int, device) -> torch.Tensor:
+    """A workspace for kda.fwd: uninitialised except for its 256-byte header (the status word),
+    which is zeroed."""
+    ws = torch.empty(get_workspace_size(T, H, N), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
 
 
 def is_supported(head_dim: int, dtype=torch.bfloat16, lower_bound: float = -5.0) -> bool:
@@ -166,7 +174,7 @@ def chunk_kda(q, k, v, g, beta, scale=None, initial_state=None, output_final_sta
     if output_final_state:
         shape = (N, H, V, K) if transpose_state_layout else (N, H, K, V)
         final = torch.empty(shape, dtype=torch.float32, device=q.device)
-    ws = torch.zeros(get_workspace_size(B * T, H, N), dtype=torch.uint8, device=q.device)
+    ws = new_workspace(B * T, H, N, q.device)
     fn = fwd_recurrent if recurrent else fwd
     fn(q, k, v, g, beta, scale, out, ws, A_log, dt_bias, lower_bound, initial_state, final,
        cu_seqlens, state_transposed=transpose_state_layout)

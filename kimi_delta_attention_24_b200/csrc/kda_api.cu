@@ -8,8 +8,6 @@ namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
 struct Shape {
   int64_t total_tokens;
   int32_t num_seqs;
@@ -77,6 +75,24 @@ kda::FwdParams make_params(const void* q, const void* k, const void* v, const vo
 
 }  // namespace
 
+kda_status_t kda::fwd_fused(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                            float scale, void* out, const float* A_log, const float* dt_bias, float lower_bound,
+                            const float* initial_state, float* final_state, const int32_t* cu_seqlens,
+                            int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
+                            int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed, uint32_t* status,
+                            cudaStream_t stream) {
+  Shape shape;
+  kda_status_t st = validate(q, k, v, g, beta, out, A_log, dt_bias, lower_bound, initial_state,
+                             final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k,
+                             head_dim_v, num_seqs, state_transposed, scale, &shape);
+  if (st != KDA_OK) return st;
+  kda::FwdParams p = make_params(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
+                                 initial_state, final_state, cu_seqlens, seqlen, num_heads,
+                                 shape.num_seqs, state_transposed, status);
+  if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
+  return kda::launch_chunked(p, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 extern "C" {
 
 int kda_is_supported(int head_dim, int dtype_is_bf16, float lower_bound) {
@@ -85,9 +101,7 @@ int kda_is_supported(int head_dim, int dtype_is_bf16, float lower_bound) {
 }
 
 size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
-  (void)total_tokens;
-  const size_t units = (size_t)(num_seqs > 0 ? num_seqs : 0) * (size_t)(num_heads > 0 ? num_heads : 0);
-  return kda::kWorkspaceHeader + round_up(units * sizeof(int32_t), 256);
+  return kda::split_workspace_bytes(total_tokens, num_heads, num_seqs);
 }
 
 kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -109,8 +123,8 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g,
                                  initial_state, final_state, cu_seqlens, seqlen, num_heads,
                                  shape.num_seqs, state_transposed, static_cast<uint32_t*>(workspace));
   if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
-  return kda::launch_chunked(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
-                                                                                        : KDA_ERR_CUDA;
+  return kda::launch_split(p, workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
+                                                                                                 : KDA_ERR_CUDA;
 }
 
 kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, const void* g,

@@ -44,24 +44,19 @@
 // Every wait is bounded (kWaitLimitNs of wall time without progress): on expiry the kernel
 // records KDA_ERR_DEVICE_TIMEOUT in the workspace status word, every role leaves its loop, and
 // the tensor memory is released.
-#include <cuda.h>
-
-#include "kda_common.cuh"
-#include "sm100.cuh"
+#include "kda_device.cuh"
 
 namespace kda {
 namespace {
 
 using namespace sm100;
 
-constexpr int C = 64;          // chunk length
+constexpr int C = kChunk;      // chunk length
 constexpr int D = kHeadDim;    // 128
 constexpr int kThreads = 512;  // 16 warps
 constexpr int kIntraWarp0 = 4, kIntraThreads = 256;
 constexpr int kRecWarp0 = 12, kRecThreads = 128;
 constexpr uint32_t kBarIntra = 1, kBarRec = 2;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr float kLog2e = 1.4426950408889634f;
 
 // Shared-memory map (bytes from a 1024-aligned base).  "MN tile" = [2 blocks of 64 columns]
 // [64 rows][128 B] with the 128-byte swizzle; "K tile" = [2 blocks of 64 K][rows][128 B].
@@ -102,8 +97,6 @@ enum {
   B_MMA1, B_DELTA, B_MMA2, B_S, B_COUNT
 };
 
-// first row of R_I inside the R tile: 0, 16, 48, 96 (R_I holds 16 (I+1) rows)
-__host__ __device__ constexpr uint32_t row_off(int I) { return 8u * I * (I + 1); }
 
 // TMEM columns: intra area 0..255 (AP products at row_off(I), P T at 0..63, [W PW] at 0..127,
 // [-W; Qtil - PW] packed bf16 at 0..63); [U PU] -> [Delta O] at 256..383; fp32 state at 384..511.
@@ -114,26 +107,6 @@ constexpr uint32_t kTmemCols = 512;
 struct TensorMaps {
   CUtensorMap q, k, v;
 };
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&t);
-}
-__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
-  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
-}
-// x as a bf16 pair hi = bf16(x), lo = bf16(x - hi), two values at a time.
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const float2 hf = __bfloat1622float2(h);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = *reinterpret_cast<const uint32_t*>(&l);
-}
-__device__ __forceinline__ float fast_sigmoid(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
-__device__ __forceinline__ uint2 ldg_u2(const __nv_bfloat16* p) {
-  return __ldg(reinterpret_cast<const uint2*>(p));
-}
 
 struct Shared {
   uint8_t* sm;
@@ -305,17 +278,6 @@ __device__ void tma_producer(const Shared& S_, const TensorMaps& maps, const Fwd
 }
 
 // ------------------------------------------------------------------------------ intra warps
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 __device__ void intra_warps(const Shared& S_, const FwdParams& p, int h, int64_t bos, int64_t eos,
                             int nchunks, int itid) {
   uint8_t* sm = S_.sm;
@@ -1031,36 +993,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiledFn>(ptr);
-  }();
-  return fn;
-}
-
-// [tokens, H, 128] bf16 viewed as 3-D (channel, head, token); box 64 channels x 1 head x 64 tokens.
-bool make_token_map(CUtensorMap* map, const void* base, int64_t tokens, int H) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(tokens > 0 ? tokens : 1)};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)C};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream) {
@@ -1071,16 +1003,9 @@ cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream) {
   if (!make_token_map(&maps.q, p.q, tokens, p.num_heads) || !make_token_map(&maps.k, p.k, tokens, p.num_heads) ||
       !make_token_map(&maps.v, p.v, tokens, p.num_heads))
     return cudaErrorInvalidValue;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  cudaError_t e = set_smem_once(chunked_kernel, SMEM_ALLOC, attr_set);
+  if (e != cudaSuccess) return e;
   chunked_kernel<<<(unsigned)units, kThreads, SMEM_ALLOC, stream>>>(maps, p);
   return cudaGetLastError();
 }

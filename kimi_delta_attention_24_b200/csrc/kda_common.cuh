@@ -51,6 +51,18 @@ __device__ __forceinline__ void seq_range(const FwdParams& p, int n, int64_t& bo
 
 // Launchers (defined in the kernel translation units).  Return the launch's cudaError_t.
 cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
+// The fused single-kernel chunked path (one CTA per (sequence, head); needs only the status word).
 cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream);
+// The split chunked path: chunk table, chunk-parallel intra-chunk kernel, recurrence kernel.
+cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream);
+size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+
+// Validates the arguments of a forward call and launches the fused chunked path with `status` as
+// the device status word (used by kda_fwd_static_workspace).
+kda_status_t fwd_fused(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+                       void* out, const float* A_log, const float* dt_bias, float lower_bound,
+                       const float* initial_state, float* final_state, const int32_t* cu_seqlens, int32_t batch,
+                       int64_t seqlen, int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
+                       int32_t state_transposed, uint32_t* status, cudaStream_t stream);
 
 }  // namespace kda

@@ -7,7 +7,10 @@
 // still own their inputs and outputs, but have nowhere to put kda_fwd's workspace.  This entry
 // point uses a workspace that lives in the library itself: a file-scope device array, allocated
 // once when the library's device code is loaded on a GPU and held by that GPU until the process
-// exits.
+// exits.  That array cannot hold the per-chunk intermediates of kda_fwd's split path (about 81 KB
+// per chunk and head), so this entry point runs the fused single-kernel chunked path, which keeps
+// every intermediate on chip and needs only the status word; its results agree with kda_fwd's to
+// rounding.
 //
 // Limits and behaviour:
 //   - The array holds the workspace of at most kStaticMaxUnits (sequence, head) units; larger
@@ -66,7 +69,7 @@ extern "C" kda_status_t kda_fwd_static_workspace(
   if (st != KDA_OK) return st;
   if (cudaMemsetAsync(ws, 0, kda::kWorkspaceHeader, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KDA_ERR_CUDA;
-  return kda_fwd(q, k, v, g, beta, scale, out, ws, kStaticWorkspaceBytes, A_log, dt_bias, lower_bound,
-                 initial_state, final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v,
-                 num_seqs, state_transposed, stream);
+  return kda::fwd_fused(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound, initial_state, final_state,
+                        cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v, num_seqs, state_transposed,
+                        static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
 }

@@ -1,0 +1,1099 @@
+// Chunked KDA forward for sm_100a, split into a chunk-parallel intra-chunk kernel and a
+// per-(sequence, head) recurrence kernel.
+//
+// Kimi Delta Attention (FlashKDA `fwd`, fla `chunk_kda`; vLLM PR #54859 report and "What CUDA
+// Version Is Required to Use FlashKDA?", Usage Examples) is the gated delta rule
+//     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = scale S_t^T q_t,
+// evaluated in chunks of C = 64 tokens in the WY/UT form.  With Gamma the in-chunk cumulative
+// log-decay and Khat/Qhat the L2-normalised keys/queries:
+//   A = strict_tril(diag(beta) (Khat e^Gamma)(Khat e^-Gamma)^T),  T = (I + A)^{-1},  T_b = T diag(beta),
+//   P = scale tril((Qhat e^Gamma)(Khat e^-Gamma)^T),  W = T_b (Khat e^Gamma),  U = T_b V,
+//   Qtil = scale Qhat e^Gamma,  Ktil = Khat e^{Gamma_C - Gamma},
+// and per chunk
+//   Delta = U - W S,   O = Qtil S + P Delta = (Qtil - P W) S + P U,   S <- Diag(e^{Gamma_C}) S + Ktil^T Delta.
+//
+// Everything that does not involve S is independent across chunks, so it runs in one CTA per
+// (chunk, head) spread over every SM (intra_kernel): the gate, the norms, the decays, the Gram
+// products, the solve and the products with T_b.  It leaves one "item" per (chunk, head) in the
+// workspace, stored as the byte image of the shared-memory tiles the recurrence consumes:
+//   [-W; Qtil - P W]   (A operand of MMA1)          [T_b; P T_b] hi and lo   (A operand of MMA Xv)
+//   Ktil (raw k scaled by the decays; A of MMA2)    1/|k_r| per row, e^{Gamma_C} per channel.
+// rec_kernel then walks each (sequence, head) chunk by chunk with the fp32 state in tensor memory:
+//   MMA Xv   [U; P U]  = [T_b; P T_b] (hi + lo) V
+//   MMA1     [Delta; O] = [U; P U] + [-W; Qtil - P W] S_bf16
+//   ep1      O -> out (bf16); Delta / |k| -> bf16 hi + lo in shared memory
+//   MMA2     S_tmem += Ktil^T Delta (hi + lo)      (S_tmem holds e^{Gamma_C} S on entry)
+//   ep2      S -> bf16 copy for the next MMA1; S_tmem <- e^{Gamma_C of the next chunk} S.
+// The hi+lo pairs matter when keys are nearly collinear (T then has entries near -beta that cancel
+// against the diagonal, and a chunk's Delta rows telescope), and Ktil is built from the raw bf16 k
+// with 1/|k| applied to Delta, so that equal keys round identically.
+//
+// Every wait is bounded (kWaitLimitNs of wall time): on expiry the kernel records
+// KDA_ERR_DEVICE_TIMEOUT in the workspace status word and the affected work is skipped.
+#include "kda_device.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+
+constexpr int C = kChunk;
+constexpr int D = kHeadDim;
+
+// ------------------------------------------------------------------------- item image (workspace)
+constexpr uint32_t IT_WQ = 0;          // [-W; Qtil - P W] bf16: 2 K-blocks x [128 rows][128 B], SW128
+constexpr uint32_t IT_TP = 32768;      // [T_b; P T_b] hi: [128 rows][128 B], SW128 (K = 64 tokens)
+constexpr uint32_t IT_TL = 49152;      // [T_b; P T_b] lo
+constexpr uint32_t IT_KT = 65536;      // Ktil: 2 channel blocks x [64 tokens][128 B], SW128
+constexpr uint32_t IT_IK = 81920;      // float[64] 1/|k_r| (0 past the end of the sequence)
+constexpr uint32_t IT_GAM = 82176;     // float[128] e^{Gamma_C}
+constexpr uint32_t IT_SC_BYTES = 768;  // IT_IK .. IT_GAM + 512
+constexpr uint32_t ITEM_BYTES = 82944;
+
+struct SplitArgs {
+  FwdParams p;
+  const int32_t* chunk_off;  // [N + 1] first global chunk of each sequence
+  uint8_t* items;            // ITEM_BYTES per (global chunk, head), chunk-major
+};
+
+// ------------------------------------------------------------------------- chunk table
+// chunk_off[n] = sum over m < n of ceil(len_m / C); one block of 1024 threads.
+__global__ void __launch_bounds__(1024) chunk_table_kernel(FwdParams p, int32_t* chunk_off) {
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    carry = 0;
+    chunk_off[0] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < p.num_seqs; base += 1024) {
+    const int n = base + tid;
+    int32_t cnt = 0;
+    if (n < p.num_seqs) {
+      int64_t bos, eos;
+      seq_range(p, n, bos, eos);
+      const int64_t len = eos > bos ? eos - bos : 0;
+      cnt = (int32_t)((len + C - 1) / C);
+    }
+    int32_t x = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t w = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_tot[lane] = w;  // inclusive
+    }
+    __syncthreads();
+    const int32_t incl = carry + x + (warp > 0 ? warp_tot[warp - 1] : 0);
+    if (n < p.num_seqs) chunk_off[n + 1] = incl;
+    __syncthreads();
+    if (tid == 1023) carry = incl;
+    __syncthreads();
+  }
+}
+
+// Sequence of global chunk gc: the largest n with chunk_off[n] <= gc (skips empty sequences).
+__device__ __forceinline__ int seq_of_chunk(const int32_t* co, int nseq, int64_t gc) {
+  int lo = 0, hi = nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)co[mid] <= gc) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ========================================================================= intra-chunk kernel
+// 256 threads, two CTAs per SM.  Shared-memory map (bytes from a 1024-aligned base); "MN tile" =
+// 2 blocks of 64 columns x [64 rows][128 B] with the 128-byte swizzle, "K tile" = 2 blocks of 64 K
+// x [rows][128 B].
+constexpr int kIntraThreads = 256;
+constexpr uint32_t I_RQ = 0;        // q tile (TMA); becomes XK once q, k sit in registers
+constexpr uint32_t I_RK = 16384;    // k tile (TMA); becomes QB
+constexpr uint32_t I_XK = 0;        // Khat e^Gamma (pre-scaled to the chunk start), MN tile, B of MMA Xk
+constexpr uint32_t I_QB = 16384;    // Qtil, MN tile, read when forming Qtil - P W
+constexpr uint32_t I_LKQ = 32768;   // [LK; LQ] K tile, 128 rows (A of MMA AP)
+constexpr uint32_t I_R = 65536;     // R_0..R_3 K tile, 160 rows (B of MMA AP)
+constexpr uint32_t I_RKBLK = 160 * 128;
+constexpr uint32_t I_TP = 32768;    // after MMA AP: [T_b hi; P -> (P T_b) hi], 128 rows x 64
+constexpr uint32_t I_TL = 49152;    //               [T_b lo; (P T_b) lo]
+constexpr uint32_t I_AS = 65536;    //               A fp32 64 x 68
+constexpr uint32_t I_TS = 82944;    //               T fp32 64 x 68
+constexpr uint32_t I_YS = 100352;   //               solve temporaries 3 x 16 x 16 fp32
+constexpr uint32_t AS_LD = 68;
+constexpr uint32_t I_SC = 106496;   // scalars
+constexpr uint32_t I_TOT = I_SC;            // float[8][128] per-warp alpha products
+constexpr uint32_t I_BETA = I_SC + 4096;    // float[64]
+constexpr uint32_t I_BAR = I_SC + 4352;     // 2 mbarriers
+constexpr uint32_t I_TMEM = I_SC + 4368;    // allocated TMEM address
+constexpr uint32_t I_ABORT = I_SC + 4372;
+constexpr uint32_t I_SMEM = I_SC + 4480;
+constexpr uint32_t I_ALLOC = I_SMEM + 1024;
+static_assert(I_YS + 3072 <= I_SC, "intra shared-memory map");
+static_assert(2 * (I_ALLOC + 1024) <= 233472, "two intra CTAs per SM");
+constexpr uint32_t kIntraTmemCols = 256;
+
+struct IntraMaps {
+  CUtensorMap q, k;
+};
+
+__global__ void __launch_bounds__(kIntraThreads, 2)
+    intra_kernel(const __grid_constant__ IntraMaps maps, const SplitArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const FwdParams& p = args.p;
+  const int H = p.num_heads;
+  const int64_t gc = blockIdx.x / H;
+  const int h = blockIdx.x % H;
+  const int32_t* co = args.chunk_off;
+  if (gc >= (int64_t)co[p.num_seqs]) return;
+  const int n = seq_of_chunk(co, p.num_seqs, gc);
+  int64_t bos, eos;
+  seq_range(p, n, bos, eos);
+  const int64_t t0 = bos + (gc - co[n]) * C;
+  const int len = (int)((eos - t0) < (int64_t)C ? (eos - t0) : (int64_t)C);
+  uint8_t* item = args.items + ((size_t)gc * H + h) * ITEM_BYTES;
+
+  const int itid = threadIdx.x;
+  const int iw = itid >> 5, lane = itid & 31;
+  const uint32_t sbase = smem_u32(sm);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + I_BAR);  // [0] q/k tiles landed, [1] MMA done
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + I_ABORT);
+  float* sc_tot = reinterpret_cast<float*>(sm + I_TOT);
+  float* sc_beta = reinterpret_cast<float*>(sm + I_BETA);
+  float* As = reinterpret_cast<float*>(sm + I_AS);
+  float* Ts = reinterpret_cast<float*>(sm + I_TS);
+  float* Ys = reinterpret_cast<float*>(sm + I_YS);
+  auto sync = [&]() { __syncthreads(); };
+
+  if (itid == 0) {
+    mbar_init(bar + 0, 1);
+    mbar_init(bar + 1, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.k);
+    mbar_arrive_expect_tx(bar + 0, 32768);
+    tma_load_3d(sm + I_RQ, &maps.q, bar + 0, 0, h, (int)t0);
+    tma_load_3d(sm + I_RQ + 8192, &maps.q, bar + 0, 64, h, (int)t0);
+    tma_load_3d(sm + I_RK, &maps.k, bar + 0, 0, h, (int)t0);
+    tma_load_3d(sm + I_RK + 8192, &maps.k, bar + 0, 64, h, (int)t0);
+  }
+  if (iw == 0) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(sm + I_TMEM), kIntraTmemCols);
+    tmem_relinquish();
+  }
+
+  // prologue mapping: warp iw owns chunk rows 8 iw .. 8 iw + 7, lane owns channels 4 lane .. +3
+  const float gate_a = __expf(p.A_log[h]);
+  const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+  const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
+  const float gb[4] = {ga * dtb.x, ga * dtb.y, ga * dtb.z, ga * dtb.w};
+  const float lb2 = p.lower_bound * kLog2e;
+  const int kb = lane >> 4;
+  const uint32_t lane_chunk = (lane & 15) >> 1;
+  const uint32_t lane_sub = (lane & 1) * 8;
+  const int blk = iw >> 1;
+  const bool upper_half = iw & 1;
+  const int quarter = iw & 3, ihalf = iw >> 2;  // TMEM lane quarter, column half
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+
+  uint2 gr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t t = t0 + 8 * iw + i;
+    gr[i] = (8 * iw + i < len) ? ldg_u2(p.g + ((size_t)t * H + h) * D + 4 * lane) : make_uint2(0, 0);
+  }
+  const float beta_raw =
+      (8 * iw + (lane & 7) < len) ? __bfloat162float(p.beta[(size_t)(t0 + 8 * iw + (lane & 7)) * H + h]) : 0.f;
+  // shared-memory byte offset of this thread's 8 bytes of row 8 iw + i inside a 128-byte-row tile
+  uint32_t xo[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) xo[i] = (uint32_t)((8 * iw + i) * 128) + (((lane_chunk ^ i) & 7u) << 4) + lane_sub;
+  const uint32_t a_rq = sbase + I_RQ + kb * 8192, a_rk = sbase + I_RK + kb * 8192;
+  const uint32_t a_lk = sbase + I_LKQ + kb * 16384, a_lq = a_lk + 64 * 128;
+  const uint32_t a_xk = sbase + I_XK + kb * 8192, a_qb = sbase + I_QB + kb * 8192;
+  const uint32_t a_r = sbase + I_R + kb * I_RKBLK;
+
+  tc_fence_before();
+  sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + I_TMEM);
+
+  // ================================================================ prologue
+  bounded_wait(bar + 0, 0, abort_flag, p.status);
+  uint2 qr[8], kr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool valid = 8 * iw + i < len;
+    qr[i] = valid ? lds64(a_rq + xo[i]) : make_uint2(0, 0);
+    kr[i] = valid ? lds64(a_rk + xo[i]) : make_uint2(0, 0);
+  }
+  float a[8][4];  // alpha
+  float ssq[8], ssk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool valid = 8 * iw + i < len;
+    const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
+    const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
+    ssq[i] = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
+    ssk[i] = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
+    const float2 g01 = unpack_bf16(gr[i].x), g23 = unpack_bf16(gr[i].y);
+    const float gv[4] = {g01.x, g01.y, g23.x, g23.y};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float sig = rcp_approx(1.0f + ex2_approx(fmaf(ga, gv[j], gb[j])));
+      a[i][j] = valid ? ex2_approx(lb2 * sig) : 1.0f;
+    }
+  }
+  // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
+  // total of value (l >> 1): q rows 0..7, then k rows 0..7
+  float inv;
+  {
+    float v16[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v16[i] = ssq[i];
+      v16[8 + i] = ssk[i];
+    }
+    const bool b4 = lane & 16;
+    float w8[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      w8[j] = (b4 ? v16[j + 8] : v16[j]) + __shfl_xor_sync(0xffffffffu, b4 ? v16[j] : v16[j + 8], 16);
+    const bool b3 = lane & 8;
+    float w4[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w4[j] = (b3 ? w8[j + 4] : w8[j]) + __shfl_xor_sync(0xffffffffu, b3 ? w8[j] : w8[j + 4], 8);
+    const bool b2 = lane & 4;
+    float w2[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      w2[j] = (b2 ? w4[j + 2] : w4[j]) + __shfl_xor_sync(0xffffffffu, b2 ? w4[j] : w4[j + 2], 4);
+    const bool b1 = lane & 2;
+    float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
+    w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
+    inv = rsqrtf(w1 + kL2Eps);
+  }
+  const float beta_l = (lane < 8 && 8 * iw + lane < len) ? fast_sigmoid(beta_raw) : 0.f;
+  const float inv_s = inv * (lane < 16 ? p.scale : 1.f);  // scale folded into 1/|q|
+  {
+    const float ikr = __shfl_sync(0xffffffffu, inv, 16 + 2 * (lane & 7));  // 1/|k| of row 8 iw + (lane & 7)
+    if (lane < 8) {
+      const int r = 8 * iw + lane;
+      sc_beta[r] = beta_l;
+      reinterpret_cast<float*>(item + IT_IK)[r] = (r < len) ? ikr : 0.f;
+    }
+  }
+  // per-warp alpha totals -> sub-block totals b_J
+  {
+    float tot[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float t = a[0][j];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) t *= a[i][j];
+      tot[j] = t;
+    }
+    reinterpret_cast<float4*>(sc_tot + iw * 128)[lane] = make_float4(tot[0], tot[1], tot[2], tot[3]);
+  }
+  sync();  // also: every thread holds its q, k rows, so the raw tiles may be overwritten
+  // sub-block totals b_J = prod of alpha over rows 16 J .. 16 J + 15 (channels 4 lane .. + 3)
+  auto load_bJ = [&](float (&bJ)[4][4]) {
+#pragma unroll
+    for (int J = 0; J < 4; ++J) {
+      const float4 t0v = reinterpret_cast<const float4*>(sc_tot + (2 * J) * 128)[lane];
+      const float4 t1v = reinterpret_cast<const float4*>(sc_tot + (2 * J + 1) * 128)[lane];
+      bJ[J][0] = t0v.x * t1v.x;
+      bJ[J][1] = t0v.y * t1v.y;
+      bJ[J][2] = t0v.z * t1v.z;
+      bJ[J][3] = t0v.w * t1v.w;
+    }
+  };
+  float pre[4], pt[4];
+  {
+    float bJ[4][4];
+    load_bJ(bJ);
+    const float4 pv = reinterpret_cast<const float4*>(sc_tot + (iw ^ 1) * 128)[lane];
+    pt[0] = pv.x;
+    pt[1] = pv.y;
+    pt[2] = pv.z;
+    pt[3] = pv.w;
+    float gam[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float pa = 1.f;
+#pragma unroll
+      for (int J = 0; J < 4; ++J)
+        if (J < blk) pa *= bJ[J][j];
+      pre[j] = pa;
+      gam[j] = bJ[0][j] * bJ[1][j] * bJ[2][j] * bJ[3][j];
+    }
+    if (iw == 0) reinterpret_cast<float4*>(item + IT_GAM)[lane] = make_float4(gam[0], gam[1], gam[2], gam[3]);
+  }
+
+  // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i
+  {
+    float run[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) run[j] = upper_half ? pt[j] : 1.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
+      const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
+      const float qv[4] = {q01.x, q01.y, q23.x, q23.y};
+      const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
+      const float iq = __shfl_sync(0xffffffffu, inv_s, 2 * i), ik = __shfl_sync(0xffffffffu, inv_s, 16 + 2 * i);
+      const float b = __shfl_sync(0xffffffffu, beta_l, i);
+      float lk[4], lq[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        run[j] *= a[i][j];
+        lk[j] = kv[j] * (run[j] * ik);  // khat * e
+        lq[j] = qv[j] * (run[j] * iq);  // scale * qhat * e
+      }
+      sts64(a_lk + xo[i], bf16x2(lk[0] * b, lk[1] * b), bf16x2(lk[2] * b, lk[3] * b));
+      sts64(a_lq + xo[i], bf16x2(lq[0], lq[1]), bf16x2(lq[2], lq[3]));
+      sts64(a_xk + xo[i], bf16x2(lk[0] * pre[0], lk[1] * pre[1]), bf16x2(lk[2] * pre[2], lk[3] * pre[3]));
+      sts64(a_qb + xo[i], bf16x2(lq[0] * pre[0], lq[1] * pre[1]), bf16x2(lq[2] * pre[2], lq[3] * pre[3]));
+    }
+  }
+  // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end; Ktil goes
+  // straight to the item (same swizzled image as a shared-memory MN tile)
+  {
+    float post[4], cI[4][4];
+    {
+      float bJ[4][4];
+      load_bJ(bJ);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float z = 1.f;
+#pragma unroll
+        for (int J = 0; J < 4; ++J)
+          if (J > blk) z *= bJ[J][j];
+        post[j] = z;
+        float m = 1.f;
+#pragma unroll
+        for (int I = 0; I < 4; ++I) {
+          cI[I][j] = (I == blk) ? 1.0f / bJ[blk][j] : m;
+          if (I > blk) m *= bJ[I][j];
+        }
+      }
+    }
+    float run[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) run[j] = upper_half ? 1.f : pt[j];
+    uint8_t* kt_dst = item + IT_KT + kb * 8192;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+      const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
+      const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
+      const float ik = __shfl_sync(0xffffffffu, inv_s, 16 + 2 * i);
+      float kf[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) kf[j] = kv[j] * (run[j] * ik);  // khat * f
+#pragma unroll
+      for (int I = 0; I < 4; ++I) {
+        if (I < blk) continue;
+        sts64(a_r + row_off(I) * 128 + xo[i], bf16x2(kf[0] * cI[I][0], kf[1] * cI[I][1]),
+              bf16x2(kf[2] * cI[I][2], kf[3] * cI[I][3]));
+      }
+      *reinterpret_cast<uint2*>(kt_dst + xo[i]) =
+          make_uint2(bf16x2(kv[0] * (run[0] * post[0]), kv[1] * (run[1] * post[1])),
+                     bf16x2(kv[2] * (run[2] * post[2]), kv[3] * (run[3] * post[3])));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) run[j] *= a[i][j];
+    }
+  }
+  fence_proxy_async();
+  if (__syncthreads_or(*abort_flag)) goto done;
+
+  // ================================================================ MMA AP: [LK; LQ] x R_I^T
+  if (itid == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int I = 0; I < 4; ++I) {
+      const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = sdesc_sw128(sbase + I_LKQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(sbase + I_R + (ks >> 2) * I_RKBLK + row_off(I) * 128 + (ks & 3) * 32, 16, 1024);
+        umma_bf16(tmem + row_off(I), ad, bd, idesc, ks > 0);
+      }
+    }
+    umma_commit(bar + 1);
+  }
+  bounded_wait(bar + 1, 0, abort_flag, p.status);
+  if (__syncthreads_or(*abort_flag)) goto done;
+  tc_fence_after();
+
+  // ================================================================ assemble A (fp32) and P (bf16)
+  {
+    const int R = 32 * quarter + lane;
+    const bool qside = R >= 64;
+    const int r = R & 63;
+    const int Ib = r >> 4;
+    const int q2 = quarter & 1;
+    const bool skip = (ihalf == 1) && (q2 == 0);
+    float d[32];
+    if (!skip) {
+      float d0[32], d1[32];
+      tmem_ld32(tmem + lane_base + row_off(2 * q2) + 32 * ihalf, d0);
+      tmem_ld32(tmem + lane_base + row_off(2 * q2 + 1) + 32 * ihalf, d1);
+      const bool odd = Ib & 1;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) d[j] = odd ? d1[j] : d0[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) d[j] = 0.f;
+    }
+    if (!qside) {
+      float* dst = As + r * AS_LD + 32 * ihalf;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const int s = 32 * ihalf + j;
+        float4 o;
+        o.x = (s + 0 < r) ? d[j + 0] : 0.f;
+        o.y = (s + 1 < r) ? d[j + 1] : 0.f;
+        o.z = (s + 2 < r) ? d[j + 2] : 0.f;
+        o.w = (s + 3 < r) ? d[j + 3] : 0.f;
+        *reinterpret_cast<float4*>(dst + j) = o;
+      }
+    } else {
+#pragma unroll
+      for (int cch = 0; cch < 4; ++cch) {
+        float v8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int s = 32 * ihalf + 8 * cch + u;
+          v8[u] = (s <= r) ? d[8 * cch + u] : 0.f;
+        }
+        uint4 w;
+        w.x = pack_bf16(v8[0], v8[1]);
+        w.y = pack_bf16(v8[2], v8[3]);
+        w.z = pack_bf16(v8[4], v8[5]);
+        w.w = pack_bf16(v8[6], v8[7]);
+        *reinterpret_cast<uint4*>(sm + I_TP + sw128(64 + r, 4 * ihalf + cch)) = w;
+      }
+    }
+  }
+  sync();
+
+  // ================================================================ solve T = (I + A)^{-1}
+  if (iw < 4 && lane < 16) {
+    const int I = iw, j = lane;
+    const float* ab = As + (16 * I) * AS_LD + 16 * I;
+    float x[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
+    // right-looking substitution: once x[m] is final, fold it into every later row
+#pragma unroll
+    for (int m = 0; m < 15; ++m) {
+      const float xm = x[m];
+#pragma unroll
+      for (int i = m + 1; i < 16; ++i) x[i] = fmaf(-ab[i * AS_LD + m], xm, x[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = (i >= j) ? x[i] : 0.f;
+  }
+  sync();
+  // off-diagonal blocks by distance dd below the diagonal, one warp per block:
+  // T_IJ = -T_II (sum_{K=J}^{I-1} A_IK T_KJ), each 16x16x16 product on mma.sync m16n8k8 tf32
+  // with both operands split hi + lo (three products), i.e. fp32-level accuracy
+#pragma unroll 1
+  for (int dd = 1; dd < 4; ++dd) {
+    if (iw < 4 - dd) {
+      const int bI = dd + iw, bJ2 = iw;
+      const int g = lane >> 2, t = lane & 3;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int K = bJ2; K < bI; ++K) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const float* ab = As + (16 * bI + g) * AS_LD + 16 * K + 8 * ks + t;
+          uint32_t ah[4], al[4];
+          tf32_split(ab[0], ah[0], al[0]);
+          tf32_split(ab[8 * AS_LD], ah[1], al[1]);
+          tf32_split(ab[4], ah[2], al[2]);
+          tf32_split(ab[8 * AS_LD + 4], ah[3], al[3]);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const float* tb = Ts + (16 * K + 8 * ks + t) * AS_LD + 16 * bJ2 + 8 * nt + g;
+            uint32_t bh0, bl0, bh1, bl1;
+            tf32_split(tb[0], bh0, bl0);
+            tf32_split(tb[4 * AS_LD], bh1, bl1);
+            mma_tf32(acc[nt], ah, bh0, bh1);
+            mma_tf32(acc[nt], ah, bl0, bl1);
+            mma_tf32(acc[nt], al, bh0, bh1);
+          }
+        }
+      }
+      float* ys = Ys + iw * 256;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        ys[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
+        ys[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
+        ys[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
+        ys[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
+      }
+      __syncwarp();
+      float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        const float* tr = Ts + (16 * bI + g) * AS_LD + 16 * bI + 8 * ks + t;
+        uint32_t ah[4], al[4];
+        tf32_split(tr[0], ah[0], al[0]);
+        tf32_split(tr[8 * AS_LD], ah[1], al[1]);
+        tf32_split(tr[4], ah[2], al[2]);
+        tf32_split(tr[8 * AS_LD + 4], ah[3], al[3]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          uint32_t bh0, bl0, bh1, bl1;
+          tf32_split(ys[(8 * ks + t) * 16 + 8 * nt + g], bh0, bl0);
+          tf32_split(ys[(8 * ks + t + 4) * 16 + 8 * nt + g], bh1, bl1);
+          mma_tf32(z[nt], ah, bh0, bh1);
+          mma_tf32(z[nt], ah, bl0, bl1);
+          mma_tf32(z[nt], al, bh0, bh1);
+        }
+      }
+      float* to = Ts + (16 * bI) * AS_LD + 16 * bJ2;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        to[g * AS_LD + 8 * nt + 2 * t] = -z[nt][0];
+        to[g * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][1];
+        to[(g + 8) * AS_LD + 8 * nt + 2 * t] = -z[nt][2];
+        to[(g + 8) * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][3];
+      }
+    }
+    sync();
+  }
+  // T_b = T diag(beta) as a bf16 hi + lo pair, rows 0..63 of TP / TL
+  {
+    const int r = itid >> 2, c16 = itid & 3;
+    const int I = r >> 4;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int c0 = 16 * c16 + 8 * hh;
+      uint4 wh, wl;
+      if (c16 > I) {
+        wh = make_uint4(0, 0, 0, 0);
+        wl = wh;
+      } else {
+        const float4 t0v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0);
+        const float4 t1v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0 + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(sc_beta + c0);
+        const float4 b1 = *reinterpret_cast<const float4*>(sc_beta + c0 + 4);
+        split2(t0v.x * b0.x, t0v.y * b0.y, wh.x, wl.x);
+        split2(t0v.z * b0.z, t0v.w * b0.w, wh.y, wl.y);
+        split2(t1v.x * b1.x, t1v.y * b1.y, wh.z, wl.z);
+        split2(t1v.z * b1.z, t1v.w * b1.w, wh.w, wl.w);
+      }
+      *reinterpret_cast<uint4*>(sm + I_TP + sw128(r, c0 >> 3)) = wh;
+      *reinterpret_cast<uint4*>(sm + I_TL + sw128(r, c0 >> 3)) = wl;
+    }
+  }
+  fence_proxy_async();
+  sync();
+
+  // ================================================================ MMA PT: P (T_hi + T_lo)
+  if (itid == 0) {
+    tc_fence_after();
+    constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint64_t ad = sdesc_sw128(sbase + I_TP + (ks & 3) * 32, 16, 1024);
+      const uint64_t bd = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 2048, 8192, 1024);
+      umma_bf16(tmem, ad, bd, idesc, ks > 0);
+    }
+    umma_commit(bar + 1);
+  }
+  bounded_wait(bar + 1, 1, abort_flag, p.status);
+  if (__syncthreads_or(*abort_flag)) goto done;
+  tc_fence_after();
+  if (quarter >= 2) {
+    const int r = 32 * quarter + lane - 64;
+    float d[32];
+    tmem_ld32(tmem + lane_base + 32 * ihalf, d);
+#pragma unroll
+    for (int cch = 0; cch < 4; ++cch) {
+      uint4 wh, wl;
+      split2(d[8 * cch + 0], d[8 * cch + 1], wh.x, wl.x);
+      split2(d[8 * cch + 2], d[8 * cch + 3], wh.y, wl.y);
+      split2(d[8 * cch + 4], d[8 * cch + 5], wh.z, wl.z);
+      split2(d[8 * cch + 6], d[8 * cch + 7], wh.w, wl.w);
+      *reinterpret_cast<uint4*>(sm + I_TP + sw128(64 + r, 4 * ihalf + cch)) = wh;
+      *reinterpret_cast<uint4*>(sm + I_TL + sw128(64 + r, 4 * ihalf + cch)) = wl;
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  sync();
+
+  // ================================================================ MMA Xk: [T_b; P T_b] x Khat e^Gamma
+  if (itid == 0) {
+    tc_fence_after();
+    constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint64_t ad = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 32, 16, 1024);
+      const uint64_t bd = sdesc_sw128(sbase + I_XK + (ks & 3) * 2048, 8192, 1024);
+      umma_bf16(tmem, ad, bd, idesc, ks > 0);
+    }
+    umma_commit(bar + 1);
+    // [T_b; P T_b] hi and lo are final: copy both tiles to the item while the MMA runs
+    bulk_store(item + IT_TP, sm + I_TP, 32768);
+    bulk_commit();
+  }
+  bounded_wait(bar + 1, 0, abort_flag, p.status);
+  if (__syncthreads_or(*abort_flag)) goto done;
+  tc_fence_after();
+
+  // ================================================================ [-W; Qtil - P W] -> item
+  {
+    const int R = 32 * quarter + lane;
+    uint8_t* dst = item + IT_WQ + ihalf * 16384 + R * 128;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      float d[32];
+      tmem_ld32(tmem + lane_base + 64 * ihalf + 32 * part, d);
+#pragma unroll
+      for (int cch = 0; cch < 4; ++cch) {
+        uint4 w;
+        if (R >= 64) {
+          const uint4 qb = *reinterpret_cast<const uint4*>(sm + I_QB + ihalf * 8192 + sw128(R - 64, 4 * part + cch));
+          const float2 a0 = unpack_bf16(qb.x), a1 = unpack_bf16(qb.y), a2 = unpack_bf16(qb.z), a3 = unpack_bf16(qb.w);
+          w.x = pack_bf16(a0.x - d[8 * cch + 0], a0.y - d[8 * cch + 1]);
+          w.y = pack_bf16(a1.x - d[8 * cch + 2], a1.y - d[8 * cch + 3]);
+          w.z = pack_bf16(a2.x - d[8 * cch + 4], a2.y - d[8 * cch + 5]);
+          w.w = pack_bf16(a3.x - d[8 * cch + 6], a3.y - d[8 * cch + 7]);
+        } else {
+          w.x = pack_bf16(-d[8 * cch + 0], -d[8 * cch + 1]);
+          w.y = pack_bf16(-d[8 * cch + 2], -d[8 * cch + 3]);
+          w.z = pack_bf16(-d[8 * cch + 4], -d[8 * cch + 5]);
+          w.w = pack_bf16(-d[8 * cch + 6], -d[8 * cch + 7]);
+        }
+        *reinterpret_cast<uint4*>(dst + ((((uint32_t)(4 * part + cch) ^ (uint32_t)R) & 7u) << 4)) = w;
+      }
+    }
+  }
+
+done:
+  tc_fence_before();
+  sync();
+  if (itid == 0) bulk_wait_all();
+  if (iw == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kIntraTmemCols);
+  }
+}
+
+// ========================================================================= recurrence kernel
+// 384 threads: warp 0 issues the MMAs, warp 1 loads, warps 4..11 run the epilogues (warp w reads
+// TMEM lanes 32 (w % 4) .. + 31, columns 64 ((w - 4) / 4) .. + 63).  One CTA per (sequence, head).
+constexpr int kRecThreads = 384;
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kBarEpi = 1;
+constexpr uint32_t R_TPV = 0;         // 2 stages x [TP 16K][TL 16K][V 16K]
+constexpr uint32_t R_TPV_STAGE = 49152;
+constexpr uint32_t R_WQ = 98304;      // 2 stages x 32K
+constexpr uint32_t R_KT = 163840;     // 2 stages x 16K
+constexpr uint32_t R_SD = 196608;     // 32K: S bf16 (MN tile, 2 blocks x 128 rows) or Delta hi (16K) + lo (16K)
+constexpr uint32_t R_SC = 229376;     // 2 stages x 768: 1/|k| and e^{Gamma_C}
+constexpr uint32_t R_BAR = R_SC + 2 * IT_SC_BYTES;
+constexpr uint32_t R_TMEM = R_BAR + 8 * 20;
+constexpr uint32_t R_ABORT = R_TMEM + 4;
+constexpr uint32_t R_SMEM = R_BAR + 256;
+constexpr uint32_t R_ALLOC = R_SMEM + 1024;
+static_assert(R_ALLOC <= 232448, "recurrence shared-memory budget");
+constexpr uint32_t TM_UP = 0;    // [U; P U] -> [Delta; O]
+constexpr uint32_t TM_S = 128;   // fp32 state (lane = k, column = v)
+constexpr uint32_t kRecTmemCols = 256;
+
+enum {
+  RB_TPV_FULL = 0,   // 2
+  RB_TPV_EMPTY = 2,  // 2 (MMA Xv commit + epilogue after ep1)
+  RB_WQ_FULL = 4,
+  RB_WQ_EMPTY = 6,
+  RB_KT_FULL = 8,
+  RB_KT_EMPTY = 10,
+  RB_VZ = 12,        // tail rows of the v tile zeroed
+  RB_MMA1 = 13,
+  RB_DELTA = 14,
+  RB_MMA2 = 15,
+  RB_S = 16,
+  RB_FINAL = 17,
+  RB_COUNT = 18
+};
+
+struct RecMaps {
+  CUtensorMap v;
+};
+
+__global__ void __launch_bounds__(kRecThreads, 1)
+    rec_kernel(const __grid_constant__ RecMaps maps, const SplitArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const FwdParams& p = args.p;
+  const int H = p.num_heads;
+  const int n = blockIdx.x / H, h = blockIdx.x % H;
+  int64_t bos, eos;
+  seq_range(p, n, bos, eos);
+  const int nch = (int)((eos - bos + C - 1) / C);
+  const int64_t item0 = (int64_t)args.chunk_off[n];
+  const uint32_t sbase = smem_u32(sm);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + R_BAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + R_ABORT);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  auto chunk_len = [&](int c) -> int {
+    const int64_t rem = eos - (bos + (int64_t)c * C);
+    return (int)(rem < (int64_t)C ? rem : (int64_t)C);
+  };
+  auto item_ptr = [&](int c) -> const uint8_t* {
+    return args.items + ((size_t)(item0 + c) * H + h) * ITEM_BYTES;
+  };
+  auto wait = [&](int b, uint32_t parity) { return bounded_wait(bar + b, parity, abort_flag, p.status); };
+
+  if (tid == 0) {
+    for (int b = 0; b < RB_COUNT; ++b) mbar_init(bar + b, (b == RB_TPV_EMPTY || b == RB_TPV_EMPTY + 1) ? 2 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&maps.v);
+  }
+  if (warp == 0) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(sm + R_TMEM), kRecTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + R_TMEM);
+
+  if (warp == 1) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0) {
+      int armed[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};  // last chunk armed per (TPV, WQ, KT) stage
+      for (int c = 0; c < nch; ++c) {
+        const int s = c & 1;
+        const uint32_t par = ((c >> 1) - 1) & 1;
+        const uint8_t* it = item_ptr(c);
+        if (c >= 2 && !wait(RB_TPV_EMPTY + s, par)) break;
+        armed[0][s] = c;
+        mbar_arrive_expect_tx(bar + RB_TPV_FULL + s, 32768 + 16384 + IT_SC_BYTES);
+        bulk_load(sm + R_TPV + s * R_TPV_STAGE, it + IT_TP, 16384, bar + RB_TPV_FULL + s);
+        bulk_load(sm + R_TPV + s * R_TPV_STAGE + 16384, it + IT_TL, 16384, bar + RB_TPV_FULL + s);
+        bulk_load(sm + R_SC + s * IT_SC_BYTES, it + IT_IK, IT_SC_BYTES, bar + RB_TPV_FULL + s);
+        const int t0 = (int)(bos + (int64_t)c * C);
+        tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 32768, &maps.v, bar + RB_TPV_FULL + s, 0, h, t0);
+        tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 40960, &maps.v, bar + RB_TPV_FULL + s, 64, h, t0);
+        if (c >= 2 && !wait(RB_WQ_EMPTY + s, par)) break;
+        armed[1][s] = c;
+        mbar_arrive_expect_tx(bar + RB_WQ_FULL + s, 32768);
+        bulk_load(sm + R_WQ + s * 32768, it + IT_WQ, 16384, bar + RB_WQ_FULL + s);
+        bulk_load(sm + R_WQ + s * 32768 + 16384, it + IT_WQ + 16384, 16384, bar + RB_WQ_FULL + s);
+        if (c >= 2 && !wait(RB_KT_EMPTY + s, par)) break;
+        armed[2][s] = c;
+        mbar_arrive_expect_tx(bar + RB_KT_FULL + s, 16384);
+        bulk_load(sm + R_KT + s * 16384, it + IT_KT, 16384, bar + RB_KT_FULL + s);
+      }
+      // leave no copy in flight: wait for the last armed phase of every stage
+      for (int kind = 0; kind < 3; ++kind)
+        for (int s = 0; s < 2; ++s)
+          if (armed[kind][s] >= 0)
+            mbar_wait(bar + (kind == 0 ? RB_TPV_FULL : kind == 1 ? RB_WQ_FULL : RB_KT_FULL) + s,
+                      (armed[kind][s] >> 1) & 1, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nch > 0) {
+      auto issue_xv = [&](int c) -> bool {
+        const int s = c & 1;
+        if (!wait(RB_TPV_FULL + s, (c >> 1) & 1)) return false;
+        if (chunk_len(c) < C && !wait(RB_VZ, 0)) return false;
+        tc_fence_after();
+        constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+        const uint32_t st = sbase + R_TPV + s * R_TPV_STAGE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t ad = sdesc_sw128(st + (ks < 4 ? 0 : 16384) + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(st + 32768 + (ks & 3) * 2048, 8192, 1024);
+          umma_bf16(tmem + TM_UP, ad, bd, idesc, ks > 0);
+        }
+        umma_commit(bar + RB_TPV_EMPTY + s);
+        return true;
+      };
+      if (issue_xv(0)) {
+        for (int c = 0; c < nch; ++c) {
+          const int s = c & 1;
+          const uint32_t par = (c >> 1) & 1;
+          if (!wait(RB_WQ_FULL + s, par) || !wait(RB_S, c & 1)) break;
+          tc_fence_after();
+          {
+            constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint64_t ad = sdesc_sw128(sbase + R_WQ + s * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(sbase + R_SD + ks * 2048, 16384, 1024);
+              umma_bf16(tmem + TM_UP, ad, bd, idesc, 1);
+            }
+          }
+          umma_commit(bar + RB_MMA1);
+          umma_commit(bar + RB_WQ_EMPTY + s);
+          if (!wait(RB_DELTA, c & 1) || !wait(RB_KT_FULL + s, par)) break;
+          tc_fence_after();
+          {
+            constexpr uint32_t idesc = idesc_bf16(128, 128, true, true);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint64_t ad = sdesc_sw128(sbase + R_KT + s * 16384 + (ks & 3) * 2048, 8192, 1024);
+              const uint64_t bd = sdesc_sw128(sbase + R_SD + (ks < 4 ? 0 : 16384) + (ks & 3) * 2048, 8192, 1024);
+              umma_bf16(tmem + TM_S, ad, bd, idesc, 1);
+            }
+          }
+          umma_commit(bar + RB_MMA2);
+          umma_commit(bar + RB_KT_EMPTY + s);
+          if (c + 1 < nch && !issue_xv(c + 1)) break;
+        }
+      }
+      // every MMA issued has completed before the tensor memory is released
+      umma_commit(bar + RB_FINAL);
+      mbar_wait(bar + RB_FINAL, 0, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue warps
+    const int et = tid - 128;
+    const int quarter = warp & 3, half = (warp - 4) >> 2;
+    const int R = 32 * quarter + lane;  // TMEM lane: state row k, or chunk row (Delta / O)
+    const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+    const uint32_t col0 = 64 * half;
+    const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
+    auto epi_sync = [&]() { named_bar(kBarEpi, kEpiThreads); };
+    // a barrier whose answer (has any role aborted?) is the same for every epilogue thread
+    auto epi_sync_abort = [&]() { return named_bar_or(kBarEpi, kEpiThreads, *abort_flag != 0); };
+    const float* sc_ik = reinterpret_cast<const float*>(sm + R_SC);
+    const float* sc_gam = reinterpret_cast<const float*>(sm + R_SC + (IT_GAM - IT_IK));
+
+    auto store_s_bf16 = [&](int part, const float (&v)[32]) {
+      // columns col0 + 32 part .. + 31 of row R of the bf16 state (MN tile, block `half`, 128 rows)
+      uint8_t* base = sm + R_SD + half * 16384;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint4 w;
+        w.x = pack_bf16(v[8 * cc + 0], v[8 * cc + 1]);
+        w.y = pack_bf16(v[8 * cc + 2], v[8 * cc + 3]);
+        w.z = pack_bf16(v[8 * cc + 4], v[8 * cc + 5]);
+        w.w = pack_bf16(v[8 * cc + 6], v[8 * cc + 7]);
+        *reinterpret_cast<uint4*>(base + sw128(R, 4 * part + cc)) = w;
+      }
+    };
+    auto load_state = [&](int part, float (&v)[32]) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const uint32_t col = col0 + 32 * part + j;
+        float s = 0.f;
+        if (p.initial_state)
+          s = p.state_transposed ? p.initial_state[soff + (size_t)col * D + R] : p.initial_state[soff + (size_t)R * D + col];
+        v[j] = s;
+      }
+    };
+    auto store_final = [&](int part, const float (&v)[32]) {
+      if (p.state_transposed) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) p.final_state[soff + (size_t)(col0 + 32 * part + j) * D + R] = v[j];
+      } else {
+        float4* dst = reinterpret_cast<float4*>(p.final_state + soff + (size_t)R * D + col0 + 32 * part);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      }
+    };
+
+    if (nch == 0) {
+      if (p.final_state) {
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          load_state(part, v);
+          store_final(part, v);
+        }
+      }
+    } else {
+      // initial state: bf16 copy for MMA1(0); fp32 copy pre-scaled by e^{Gamma_C}(0) for MMA2(0)
+      wait(RB_TPV_FULL, 0);
+      const float gam0 = sc_gam[R];
+#pragma unroll 1
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        load_state(part, v);
+        store_s_bf16(part, v);
+        uint32_t u[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam0 * v[j]);
+        tmem_st32(tmem + lane_base + TM_S + col0 + 32 * part, u);
+      }
+      tmem_wait_st();
+      fence_proxy_async();
+      tc_fence_before();
+      epi_sync();
+      if (et == 0) mbar_arrive(bar + RB_S);
+
+      for (int c = 0; c < nch; ++c) {
+        const int s = c & 1;
+        const int len = chunk_len(c);
+        const int64_t t0 = bos + (int64_t)c * C;
+        wait(RB_TPV_FULL + s, (c >> 1) & 1);
+        if (len < C) {
+          // rows of the v tile past the sequence end (another sequence's, or zero-filled) -> 0
+          if (epi_sync_abort()) break;
+          uint8_t* vt = sm + R_TPV + s * R_TPV_STAGE + 32768;
+          for (int idx = et; idx < 2 * (C - len) * 8; idx += kEpiThreads) {
+            const int b2 = idx / ((C - len) * 8), rem = idx % ((C - len) * 8);
+            *reinterpret_cast<uint4*>(vt + b2 * 8192 + sw128(len + rem / 8, rem & 7)) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async();
+          epi_sync();
+          if (et == 0) mbar_arrive(bar + RB_VZ);
+        }
+        // ---------------------------------------------------- ep1: Delta and O
+        wait(RB_MMA1, c & 1);
+        if (epi_sync_abort()) break;
+        tc_fence_after();
+        {
+          const int r = R & 63;
+          const float ikr = sc_ik[s * (IT_SC_BYTES / 4) + r];
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part) {
+            float d[32];
+            tmem_ld32(tmem + lane_base + TM_UP + col0 + 32 * part, d);
+            if (R < 64) {
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) {
+                uint4 wh, wl;
+                split2(d[8 * cc + 0] * ikr, d[8 * cc + 1] * ikr, wh.x, wl.x);
+                split2(d[8 * cc + 2] * ikr, d[8 * cc + 3] * ikr, wh.y, wl.y);
+                split2(d[8 * cc + 4] * ikr, d[8 * cc + 5] * ikr, wh.z, wl.z);
+                split2(d[8 * cc + 6] * ikr, d[8 * cc + 7] * ikr, wh.w, wl.w);
+                const uint32_t off = half * 8192 + sw128(r, 4 * part + cc);
+                *reinterpret_cast<uint4*>(sm + R_SD + off) = wh;
+                *reinterpret_cast<uint4*>(sm + R_SD + 16384 + off) = wl;
+              }
+            } else if (r < len) {
+              uint4* orow = reinterpret_cast<uint4*>(p.out + ((size_t)(t0 + r) * H + h) * D + col0 + 32 * part);
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) {
+                uint4 w;
+                w.x = pack_bf16(d[8 * cc + 0], d[8 * cc + 1]);
+                w.y = pack_bf16(d[8 * cc + 2], d[8 * cc + 3]);
+                w.z = pack_bf16(d[8 * cc + 4], d[8 * cc + 5]);
+                w.w = pack_bf16(d[8 * cc + 6], d[8 * cc + 7]);
+                orow[cc] = w;
+              }
+            }
+          }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        epi_sync();
+        if (et == 0) {
+          mbar_arrive(bar + RB_DELTA);
+          mbar_arrive(bar + RB_TPV_EMPTY + s);
+        }
+        // ---------------------------------------------------- ep2: state
+        const bool last = (c + 1 == nch);
+        wait(RB_MMA2, c & 1);
+        if (!last) wait(RB_TPV_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1);
+        if (epi_sync_abort()) break;
+        tc_fence_after();
+        {
+          const float gam = last ? 1.f : sc_gam[((c + 1) & 1) * (IT_SC_BYTES / 4) + R];
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part) {
+            float v[32];
+            tmem_ld32(tmem + lane_base + TM_S + col0 + 32 * part, v);
+            if (last) {
+              if (p.final_state) store_final(part, v);
+            } else {
+              store_s_bf16(part, v);
+              uint32_t u[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam * v[j]);
+              tmem_st32(tmem + lane_base + TM_S + col0 + 32 * part, u);
+            }
+          }
+          if (!last) tmem_wait_st();
+        }
+        if (last) break;
+        fence_proxy_async();
+        tc_fence_before();
+        epi_sync();
+        if (et == 0) mbar_arrive(bar + RB_S);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kRecTmemCols);
+  }
+}
+
+bool g_intra_attr[64] = {};
+bool g_rec_attr[64] = {};
+
+}  // namespace
+
+size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  const int64_t n = num_seqs > 0 ? num_seqs : 0;
+  const int64_t t = total_tokens > 0 ? total_tokens : 0;
+  const int64_t max_chunks = (t + (int64_t)(C - 1) * n) / C;
+  const size_t table = ((size_t)(n + 1) * sizeof(int32_t) + 1023) / 1024 * 1024;
+  return kWorkspaceHeader + table + (size_t)max_chunks * (size_t)(num_heads > 0 ? num_heads : 0) * ITEM_BYTES;
+}
+
+cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream) {
+  const int64_t units = (int64_t)p.num_seqs * p.num_heads;
+  if (units == 0) return cudaSuccess;
+  const int64_t tokens = p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs;
+  const int64_t max_chunks = (tokens + (int64_t)(C - 1) * p.num_seqs) / C;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  SplitArgs args;
+  args.p = p;
+  args.chunk_off = reinterpret_cast<int32_t*>(ws + kWorkspaceHeader);
+  args.items = ws + kWorkspaceHeader + ((size_t)(p.num_seqs + 1) * sizeof(int32_t) + 1023) / 1024 * 1024;
+
+  IntraMaps im;
+  RecMaps rm;
+  if (!make_token_map(&im.q, p.q, tokens, p.num_heads) || !make_token_map(&im.k, p.k, tokens, p.num_heads) ||
+      !make_token_map(&rm.v, p.v, tokens, p.num_heads))
+    return cudaErrorInvalidValue;
+  cudaError_t e = set_smem_once(intra_kernel, I_ALLOC, g_intra_attr);
+  if (e != cudaSuccess) return e;
+  e = set_smem_once(rec_kernel, R_ALLOC, g_rec_attr);
+  if (e != cudaSuccess) return e;
+
+  chunk_table_kernel<<<1, 1024, 0, stream>>>(p, const_cast<int32_t*>(args.chunk_off));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t intra_blocks = max_chunks * p.num_heads;
+  if (intra_blocks > 0) {
+    if (intra_blocks > INT32_MAX) return cudaErrorInvalidValue;
+    intra_kernel<<<(unsigned)intra_blocks, kIntraThreads, I_ALLOC, stream>>>(im, args);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  rec_kernel<<<(unsigned)units, kRecThreads, R_ALLOC, stream>>>(rm, args);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -52,11 +52,15 @@ def test_support_predicate(lib):
     assert lib.kda_is_supported(128, 0, -5.0) == 0
 
 
-def test_workspace_size_depends_on_units(lib):
+def test_workspace_size_covers_every_chunk_and_head(lib):
+    # one 81 KB item per (chunk, head): 512 chunks x 96 heads at T = 32768
+    item = 82944
     a = lib.kda_workspace_size(32768, 96, 1)
-    b = lib.kda_workspace_size(1, 96, 1)
-    assert a == b and a >= 256 and a % 256 == 0
-    assert lib.kda_workspace_size(100, 32, 8) >= 256 + 4 * 32 * 8
+    assert a >= 512 * 96 * item and a % 256 == 0
+    assert lib.kda_workspace_size(1, 96, 1) >= 96 * item
+    # 8 sequences of 100 tokens or fewer hold at most (100 + 63 * 8) / 64 chunks in total
+    assert lib.kda_workspace_size(100, 32, 8) >= (100 + 63 * 8) // 64 * 32 * item
+    assert lib.kda_workspace_size(0, 32, 0) >= 256
 
 
 # Fake device pointers: aligned, never dereferenced because validation fails first.

@@ -35,7 +35,7 @@ def run_gpu(x, impl="chunked", state_transposed=False, alias=False, dev="cuda:0"
     final = None
     if x.output_final_state:
         final = s0 if alias else torch.full((N, H, K, K), float("nan"), dtype=torch.float32, device=dev)
-    ws = torch.zeros(kda.get_workspace_size(B * T, H, N), dtype=torch.uint8, device=dev)
+    ws = kda.new_workspace(B * T, H, N, dev)
     fn = kda.fwd if impl == "chunked" else kda.fwd_recurrent
     fn(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.scale, out, ws, xd.A_log, xd.dt_bias, xd.lower_bound,
        s0, final, xd.cu_seqlens, state_transposed=state_transposed)

@@ -42,7 +42,7 @@ def test_static_workspace_matches_kda_fwd(cuda_device):
     N = x.num_seqs
     ref_out = torch.empty_like(x.v)
     ref_final = torch.empty(N, H, K, K, dtype=torch.float32, device=cuda_device)
-    ws = torch.zeros(kda.get_workspace_size(B * T, H, N), dtype=torch.uint8, device=cuda_device)
+    ws = kda.new_workspace(B * T, H, N, cuda_device)
     kda.fwd(x.q, x.k, x.v, x.g, x.beta, x.scale, ref_out, ws, x.A_log, x.dt_bias, x.lower_bound,
             x.initial_state, ref_final, x.cu_seqlens)
     torch.cuda.synchronize()
