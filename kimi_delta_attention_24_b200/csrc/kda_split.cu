@@ -698,11 +698,14 @@ done:
 }
 
 // ========================================================================= recurrence kernel
-// 384 threads: warp 0 issues the MMAs, warp 1 loads, warps 4..11 run the epilogues (warp w reads
-// TMEM lanes 32 (w % 4) .. + 31, columns 64 ((w - 4) / 4) .. + 63).  One CTA per (sequence, head).
-constexpr int kRecThreads = 384;
-constexpr int kEpiThreads = 256;
-constexpr uint32_t kBarEpi = 1;
+// One CTA per (sequence, head), 640 threads: warp 0 issues the MMAs, warp 1 loads (and zeroes the
+// v rows past a sequence's end), warps 4..19 run the epilogues; warp w reads TMEM lanes
+// 32 (w % 4) .. + 31 and columns 32 cb .. + 31, cb = (w - 4) / 4.  The per-chunk critical path is
+// MMA1 -> ep1 (Delta rows only) -> MMA2 -> ep2; MMA Xv of the next chunk goes into the other
+// [U; P U] buffer in two halves that fill the tensor pipe while ep1 and ep2 run.
+constexpr int kRecThreads = 640;
+constexpr int kEpiThreads = 512;
+constexpr uint32_t kBarEpi = 1, kBarDelta = 2;
 constexpr uint32_t R_TPV = 0;         // 2 stages x [TP 16K][TL 16K][V 16K]
 constexpr uint32_t R_TPV_STAGE = 49152;
 constexpr uint32_t R_WQ = 98304;      // 2 stages x 32K
@@ -710,18 +713,19 @@ constexpr uint32_t R_KT = 163840;     // 2 stages x 16K
 constexpr uint32_t R_SD = 196608;     // 32K: S bf16 (MN tile, 2 blocks x 128 rows) or Delta hi (16K) + lo (16K)
 constexpr uint32_t R_SC = 229376;     // 2 stages x 768: 1/|k| and e^{Gamma_C}
 constexpr uint32_t R_BAR = R_SC + 2 * IT_SC_BYTES;
-constexpr uint32_t R_TMEM = R_BAR + 8 * 20;
+constexpr uint32_t R_TMEM = R_BAR + 8 * 24;
 constexpr uint32_t R_ABORT = R_TMEM + 4;
 constexpr uint32_t R_SMEM = R_BAR + 256;
 constexpr uint32_t R_ALLOC = R_SMEM + 1024;
 static_assert(R_ALLOC <= 232448, "recurrence shared-memory budget");
-constexpr uint32_t TM_UP = 0;    // [U; P U] -> [Delta; O]
-constexpr uint32_t TM_S = 128;   // fp32 state (lane = k, column = v)
-constexpr uint32_t kRecTmemCols = 256;
+constexpr uint32_t TM_UP = 0;    // 2 buffers x 128 columns: [U; P U] -> [Delta; O] of chunk c in buffer c % 2
+constexpr uint32_t TM_S = 256;   // fp32 state (lane = k, column = v)
+constexpr uint32_t kRecTmemCols = 512;
+constexpr int kRecPrefetch = 4;  // chunks the loader pulls into L2 ahead of its stage loads
 
 enum {
-  RB_TPV_FULL = 0,   // 2
-  RB_TPV_EMPTY = 2,  // 2 (MMA Xv commit + epilogue after ep1)
+  RB_TPV_FULL = 0,   // 2 stages
+  RB_TPV_EMPTY = 2,  // 2 stages; count 2: the commit after MMA Xv, and the Delta warps after ep1
   RB_WQ_FULL = 4,
   RB_WQ_EMPTY = 6,
   RB_KT_FULL = 8,
@@ -779,91 +783,133 @@ __global__ void __launch_bounds__(kRecThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + R_TMEM);
 
   if (warp == 1) {
-    // ------------------------------------------------------------ loader
-    if (lane == 0) {
-      int armed[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};  // last chunk armed per (TPV, WQ, KT) stage
-      for (int c = 0; c < nch; ++c) {
-        const int s = c & 1;
-        const uint32_t par = ((c >> 1) - 1) & 1;
-        const uint8_t* it = item_ptr(c);
-        if (c >= 2 && !wait(RB_TPV_EMPTY + s, par)) break;
-        armed[0][s] = c;
-        mbar_arrive_expect_tx(bar + RB_TPV_FULL + s, 32768 + 16384 + IT_SC_BYTES);
-        bulk_load(sm + R_TPV + s * R_TPV_STAGE, it + IT_TP, 16384, bar + RB_TPV_FULL + s);
-        bulk_load(sm + R_TPV + s * R_TPV_STAGE + 16384, it + IT_TL, 16384, bar + RB_TPV_FULL + s);
-        bulk_load(sm + R_SC + s * IT_SC_BYTES, it + IT_IK, IT_SC_BYTES, bar + RB_TPV_FULL + s);
-        const int t0 = (int)(bos + (int64_t)c * C);
-        tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 32768, &maps.v, bar + RB_TPV_FULL + s, 0, h, t0);
-        tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 40960, &maps.v, bar + RB_TPV_FULL + s, 64, h, t0);
-        if (c >= 2 && !wait(RB_WQ_EMPTY + s, par)) break;
-        armed[1][s] = c;
-        mbar_arrive_expect_tx(bar + RB_WQ_FULL + s, 32768);
-        bulk_load(sm + R_WQ + s * 32768, it + IT_WQ, 16384, bar + RB_WQ_FULL + s);
-        bulk_load(sm + R_WQ + s * 32768 + 16384, it + IT_WQ + 16384, 16384, bar + RB_WQ_FULL + s);
-        if (c >= 2 && !wait(RB_KT_EMPTY + s, par)) break;
-        armed[2][s] = c;
-        mbar_arrive_expect_tx(bar + RB_KT_FULL + s, 16384);
-        bulk_load(sm + R_KT + s * 16384, it + IT_KT, 16384, bar + RB_KT_FULL + s);
+    // ------------------------------------------------------------ loader (lane 0 issues; the
+    // whole warp zeroes the v rows past the end of the sequence in the last chunk)
+    int armed[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};  // last chunk armed per (TPV, WQ, KT) stage
+    auto prefetch = [&](int c) {
+      if (c >= nch) return;
+      prefetch_l2(item_ptr(c), ITEM_BYTES);
+      const int t0 = (int)(bos + (int64_t)c * C);
+      tma_prefetch_3d(&maps.v, 0, h, t0);
+      tma_prefetch_3d(&maps.v, 64, h, t0);
+    };
+    if (lane == 0)
+      for (int c = 0; c < kRecPrefetch; ++c) prefetch(c);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1;
+      const uint32_t par = ((c >> 1) - 1) & 1;
+      const uint8_t* it = item_ptr(c);
+      int ok = 1;
+      if (lane == 0) {
+        prefetch(c + kRecPrefetch);
+        if (c >= 2 && !wait(RB_TPV_EMPTY + s, par)) ok = 0;
+        if (ok) {
+          armed[0][s] = c;
+          mbar_arrive_expect_tx(bar + RB_TPV_FULL + s, 32768 + 16384 + IT_SC_BYTES);
+          bulk_load(sm + R_TPV + s * R_TPV_STAGE, it + IT_TP, 16384, bar + RB_TPV_FULL + s);
+          bulk_load(sm + R_TPV + s * R_TPV_STAGE + 16384, it + IT_TL, 16384, bar + RB_TPV_FULL + s);
+          bulk_load(sm + R_SC + s * IT_SC_BYTES, it + IT_IK, IT_SC_BYTES, bar + RB_TPV_FULL + s);
+          const int t0 = (int)(bos + (int64_t)c * C);
+          tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 32768, &maps.v, bar + RB_TPV_FULL + s, 0, h, t0);
+          tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 40960, &maps.v, bar + RB_TPV_FULL + s, 64, h, t0);
+        }
+        if (ok && c >= 2 && !wait(RB_WQ_EMPTY + s, par)) ok = 0;
+        if (ok) {
+          armed[1][s] = c;
+          mbar_arrive_expect_tx(bar + RB_WQ_FULL + s, 32768);
+          bulk_load(sm + R_WQ + s * 32768, it + IT_WQ, 16384, bar + RB_WQ_FULL + s);
+          bulk_load(sm + R_WQ + s * 32768 + 16384, it + IT_WQ + 16384, 16384, bar + RB_WQ_FULL + s);
+        }
+        if (ok && c >= 2 && !wait(RB_KT_EMPTY + s, par)) ok = 0;
+        if (ok) {
+          armed[2][s] = c;
+          mbar_arrive_expect_tx(bar + RB_KT_FULL + s, 16384);
+          bulk_load(sm + R_KT + s * 16384, it + IT_KT, 16384, bar + RB_KT_FULL + s);
+        }
+        if (ok && chunk_len(c) < C && !wait(RB_TPV_FULL + s, (c >> 1) & 1)) ok = 0;
       }
-      // leave no copy in flight: wait for the last armed phase of every stage
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const int len = chunk_len(c);
+      if (len < C) {
+        // rows of the v tile past the sequence end (another sequence's, or zero-filled) -> 0
+        uint8_t* vt = sm + R_TPV + s * R_TPV_STAGE + 32768;
+        for (int idx = lane; idx < 2 * (C - len) * 8; idx += 32) {
+          const int b2 = idx / ((C - len) * 8), rem = idx % ((C - len) * 8);
+          *reinterpret_cast<uint4*>(vt + b2 * 8192 + sw128(len + rem / 8, rem & 7)) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar + RB_VZ);
+      }
+    }
+    // leave no copy in flight: wait for the last armed phase of every stage
+    if (lane == 0)
       for (int kind = 0; kind < 3; ++kind)
         for (int s = 0; s < 2; ++s)
           if (armed[kind][s] >= 0)
             mbar_wait(bar + (kind == 0 ? RB_TPV_FULL : kind == 1 ? RB_WQ_FULL : RB_KT_FULL) + s,
                       (armed[kind][s] >> 1) & 1, kWaitLimitNs);
-    }
     __syncwarp();
   } else if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nch > 0) {
-      auto issue_xv = [&](int c) -> bool {
+      constexpr uint32_t idesc_k = idesc_bf16(128, 128, false, true);  // A K-major, B MN-major
+      constexpr uint32_t idesc_m = idesc_bf16(128, 128, true, true);   // A and B MN-major
+      // half `part` of MMA Xv: [U; P U] (+)= [T_b; P T_b]_{hi / lo} V into buffer c % 2
+      auto issue_xv = [&](int c, int part) -> bool {
         const int s = c & 1;
-        if (!wait(RB_TPV_FULL + s, (c >> 1) & 1)) return false;
-        if (chunk_len(c) < C && !wait(RB_VZ, 0)) return false;
-        tc_fence_after();
-        constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+        if (part == 0) {
+          if (!wait(RB_TPV_FULL + s, (c >> 1) & 1)) return false;
+          if (chunk_len(c) < C && !wait(RB_VZ, 0)) return false;
+          // the buffer held [Delta; O] of chunk c - 2, read by ep1(c - 2): ep2(c - 2) followed it
+          // on every epilogue warp before S(c - 1) arrived, and MMA1(c - 1) waited for S(c - 1)
+          tc_fence_after();
+        }
         const uint32_t st = sbase + R_TPV + s * R_TPV_STAGE;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t ad = sdesc_sw128(st + (ks < 4 ? 0 : 16384) + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(st + 32768 + (ks & 3) * 2048, 8192, 1024);
-          umma_bf16(tmem + TM_UP, ad, bd, idesc, ks > 0);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const uint64_t ad = sdesc_sw128(st + 16384 * part + k4 * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(st + 32768 + k4 * 2048, 8192, 1024);
+          umma_bf16(tmem + TM_UP + 128 * (c & 1), ad, bd, idesc_k, part + k4 > 0);
         }
-        umma_commit(bar + RB_TPV_EMPTY + s);
+        if (part == 1) umma_commit(bar + RB_TPV_EMPTY + s);
         return true;
       };
-      if (issue_xv(0)) {
-        for (int c = 0; c < nch; ++c) {
-          const int s = c & 1;
-          const uint32_t par = (c >> 1) & 1;
-          if (!wait(RB_WQ_FULL + s, par) || !wait(RB_S, c & 1)) break;
-          tc_fence_after();
-          {
-            constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+      bool ok = issue_xv(0, 0) && issue_xv(0, 1);
+      for (int c = 0; ok && c < nch; ++c) {
+        const int s = c & 1;
+        const uint32_t par = (c >> 1) & 1;
+        // MMA1: [Delta; O] = [U; P U] + [-W; Qtil - P W] S
+        if (!wait(RB_WQ_FULL + s, par) || !wait(RB_S, c & 1)) break;
+        tc_fence_after();
+        {
+          const uint32_t wq = sbase + R_WQ + s * 32768;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint64_t ad = sdesc_sw128(sbase + R_WQ + s * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sbase + R_SD + ks * 2048, 16384, 1024);
-              umma_bf16(tmem + TM_UP, ad, bd, idesc, 1);
-            }
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t ad = sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sbase + R_SD + ks * 2048, 16384, 1024);
+            umma_bf16(tmem + TM_UP + 128 * (c & 1), ad, bd, idesc_k, 1);
           }
-          umma_commit(bar + RB_MMA1);
-          umma_commit(bar + RB_WQ_EMPTY + s);
-          if (!wait(RB_DELTA, c & 1) || !wait(RB_KT_FULL + s, par)) break;
-          tc_fence_after();
-          {
-            constexpr uint32_t idesc = idesc_bf16(128, 128, true, true);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint64_t ad = sdesc_sw128(sbase + R_KT + s * 16384 + (ks & 3) * 2048, 8192, 1024);
-              const uint64_t bd = sdesc_sw128(sbase + R_SD + (ks < 4 ? 0 : 16384) + (ks & 3) * 2048, 8192, 1024);
-              umma_bf16(tmem + TM_S, ad, bd, idesc, 1);
-            }
-          }
-          umma_commit(bar + RB_MMA2);
-          umma_commit(bar + RB_KT_EMPTY + s);
-          if (c + 1 < nch && !issue_xv(c + 1)) break;
         }
+        umma_commit(bar + RB_MMA1);
+        umma_commit(bar + RB_WQ_EMPTY + s);
+        if (c + 1 < nch && !issue_xv(c + 1, 0)) break;
+        // MMA2: S_tmem += Ktil^T Delta (hi + lo)
+        if (!wait(RB_KT_FULL + s, par) || !wait(RB_DELTA, c & 1)) break;
+        tc_fence_after();
+        {
+          const uint32_t kt = sbase + R_KT + s * 16384;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t ad = sdesc_sw128(kt + (ks & 3) * 2048, 8192, 1024);
+            const uint64_t bd = sdesc_sw128(sbase + R_SD + (ks < 4 ? 0 : 16384) + (ks & 3) * 2048, 8192, 1024);
+            umma_bf16(tmem + TM_S, ad, bd, idesc_m, 1);
+          }
+        }
+        umma_commit(bar + RB_MMA2);
+        umma_commit(bar + RB_KT_EMPTY + s);
+        if (c + 1 < nch) ok = issue_xv(c + 1, 1);
       }
       // every MMA issued has completed before the tensor memory is released
       umma_commit(bar + RB_FINAL);
@@ -873,20 +919,20 @@ __global__ void __launch_bounds__(kRecThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue warps
     const int et = tid - 128;
-    const int quarter = warp & 3, half = (warp - 4) >> 2;
+    const int quarter = warp & 3, cb = (warp - 4) >> 2;
     const int R = 32 * quarter + lane;  // TMEM lane: state row k, or chunk row (Delta / O)
+    const bool delta_rows = quarter < 2;
     const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-    const uint32_t col0 = 64 * half;
+    const uint32_t col0 = 32 * cb;      // this thread's 32 columns
     const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
-    auto epi_sync = [&]() { named_bar(kBarEpi, kEpiThreads); };
-    // a barrier whose answer (has any role aborted?) is the same for every epilogue thread
+    // a barrier of all epilogue warps whose answer (has any role aborted?) is the same for all
     auto epi_sync_abort = [&]() { return named_bar_or(kBarEpi, kEpiThreads, *abort_flag != 0); };
     const float* sc_ik = reinterpret_cast<const float*>(sm + R_SC);
     const float* sc_gam = reinterpret_cast<const float*>(sm + R_SC + (IT_GAM - IT_IK));
 
-    auto store_s_bf16 = [&](int part, const float (&v)[32]) {
-      // columns col0 + 32 part .. + 31 of row R of the bf16 state (MN tile, block `half`, 128 rows)
-      uint8_t* base = sm + R_SD + half * 16384;
+    auto store_s_bf16 = [&](const float (&v)[32]) {
+      // columns col0 .. + 31 of row R of the bf16 state (MN tile, block cb / 2, 128 rows)
+      uint8_t* base = sm + R_SD + (cb >> 1) * 16384;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint4 w;
@@ -894,25 +940,34 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         w.y = pack_bf16(v[8 * cc + 2], v[8 * cc + 3]);
         w.z = pack_bf16(v[8 * cc + 4], v[8 * cc + 5]);
         w.w = pack_bf16(v[8 * cc + 6], v[8 * cc + 7]);
-        *reinterpret_cast<uint4*>(base + sw128(R, 4 * part + cc)) = w;
+        *reinterpret_cast<uint4*>(base + sw128(R, 4 * (cb & 1) + cc)) = w;
       }
     };
-    auto load_state = [&](int part, float (&v)[32]) {
+    auto load_state = [&](float (&v)[32]) {
+      if (!p.initial_state) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const uint32_t col = col0 + 32 * part + j;
-        float s = 0.f;
-        if (p.initial_state)
-          s = p.state_transposed ? p.initial_state[soff + (size_t)col * D + R] : p.initial_state[soff + (size_t)R * D + col];
-        v[j] = s;
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+      } else if (p.state_transposed) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = p.initial_state[soff + (size_t)(col0 + j) * D + R];
+      } else {
+        const float4* src = reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)R * D + col0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 t = src[j];
+          v[4 * j] = t.x;
+          v[4 * j + 1] = t.y;
+          v[4 * j + 2] = t.z;
+          v[4 * j + 3] = t.w;
+        }
       }
     };
-    auto store_final = [&](int part, const float (&v)[32]) {
+    auto store_final = [&](const float (&v)[32]) {
       if (p.state_transposed) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) p.final_state[soff + (size_t)(col0 + 32 * part + j) * D + R] = v[j];
+        for (int j = 0; j < 32; ++j) p.final_state[soff + (size_t)(col0 + j) * D + R] = v[j];
       } else {
-        float4* dst = reinterpret_cast<float4*>(p.final_state + soff + (size_t)R * D + col0 + 32 * part);
+        float4* dst = reinterpret_cast<float4*>(p.final_state + soff + (size_t)R * D + col0);
 #pragma unroll
         for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
       }
@@ -920,74 +975,66 @@ __global__ void __launch_bounds__(kRecThreads, 1)
 
     if (nch == 0) {
       if (p.final_state) {
-        for (int part = 0; part < 2; ++part) {
-          float v[32];
-          load_state(part, v);
-          store_final(part, v);
-        }
+        float v[32];
+        load_state(v);
+        store_final(v);
       }
     } else {
       // initial state: bf16 copy for MMA1(0); fp32 copy pre-scaled by e^{Gamma_C}(0) for MMA2(0)
       wait(RB_TPV_FULL, 0);
-      const float gam0 = sc_gam[R];
-#pragma unroll 1
-      for (int part = 0; part < 2; ++part) {
+      {
+        const float gam0 = sc_gam[R];
         float v[32];
-        load_state(part, v);
-        store_s_bf16(part, v);
+        load_state(v);
+        store_s_bf16(v);
         uint32_t u[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam0 * v[j]);
-        tmem_st32(tmem + lane_base + TM_S + col0 + 32 * part, u);
+        tmem_st32(tmem + lane_base + TM_S + col0, u);
       }
       tmem_wait_st();
       fence_proxy_async();
       tc_fence_before();
-      epi_sync();
+      named_bar(kBarEpi, kEpiThreads);
       if (et == 0) mbar_arrive(bar + RB_S);
 
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
         const int len = chunk_len(c);
         const int64_t t0 = bos + (int64_t)c * C;
-        wait(RB_TPV_FULL + s, (c >> 1) & 1);
-        if (len < C) {
-          // rows of the v tile past the sequence end (another sequence's, or zero-filled) -> 0
-          if (epi_sync_abort()) break;
-          uint8_t* vt = sm + R_TPV + s * R_TPV_STAGE + 32768;
-          for (int idx = et; idx < 2 * (C - len) * 8; idx += kEpiThreads) {
-            const int b2 = idx / ((C - len) * 8), rem = idx % ((C - len) * 8);
-            *reinterpret_cast<uint4*>(vt + b2 * 8192 + sw128(len + rem / 8, rem & 7)) = make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async();
-          epi_sync();
-          if (et == 0) mbar_arrive(bar + RB_VZ);
-        }
-        // ---------------------------------------------------- ep1: Delta and O
+        const uint32_t up = tmem + lane_base + TM_UP + 128 * (c & 1) + col0;
+        // ---------------------------------------------------- ep1: Delta (rows 0..63) and O (rows 64..127)
+        if (delta_rows) wait(RB_TPV_FULL + s, (c >> 1) & 1);  // 1/|k| of this chunk
         wait(RB_MMA1, c & 1);
         if (epi_sync_abort()) break;
         tc_fence_after();
         {
-          const int r = R & 63;
-          const float ikr = sc_ik[s * (IT_SC_BYTES / 4) + r];
-#pragma unroll 1
-          for (int part = 0; part < 2; ++part) {
-            float d[32];
-            tmem_ld32(tmem + lane_base + TM_UP + col0 + 32 * part, d);
-            if (R < 64) {
+          float d[32];
+          tmem_ld32(up, d);
+          if (delta_rows) {
+            const float ikr = sc_ik[s * (IT_SC_BYTES / 4) + R];
 #pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                uint4 wh, wl;
-                split2(d[8 * cc + 0] * ikr, d[8 * cc + 1] * ikr, wh.x, wl.x);
-                split2(d[8 * cc + 2] * ikr, d[8 * cc + 3] * ikr, wh.y, wl.y);
-                split2(d[8 * cc + 4] * ikr, d[8 * cc + 5] * ikr, wh.z, wl.z);
-                split2(d[8 * cc + 6] * ikr, d[8 * cc + 7] * ikr, wh.w, wl.w);
-                const uint32_t off = half * 8192 + sw128(r, 4 * part + cc);
-                *reinterpret_cast<uint4*>(sm + R_SD + off) = wh;
-                *reinterpret_cast<uint4*>(sm + R_SD + 16384 + off) = wl;
-              }
-            } else if (r < len) {
-              uint4* orow = reinterpret_cast<uint4*>(p.out + ((size_t)(t0 + r) * H + h) * D + col0 + 32 * part);
+            for (int cc = 0; cc < 4; ++cc) {
+              uint4 wh, wl;
+              split2(d[8 * cc + 0] * ikr, d[8 * cc + 1] * ikr, wh.x, wl.x);
+              split2(d[8 * cc + 2] * ikr, d[8 * cc + 3] * ikr, wh.y, wl.y);
+              split2(d[8 * cc + 4] * ikr, d[8 * cc + 5] * ikr, wh.z, wl.z);
+              split2(d[8 * cc + 6] * ikr, d[8 * cc + 7] * ikr, wh.w, wl.w);
+              const uint32_t off = (cb >> 1) * 8192 + sw128(R, 4 * (cb & 1) + cc);
+              *reinterpret_cast<uint4*>(sm + R_SD + off) = wh;
+              *reinterpret_cast<uint4*>(sm + R_SD + 16384 + off) = wl;
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar(kBarDelta, kEpiThreads / 2);
+            if (et == 0) {
+              mbar_arrive(bar + RB_DELTA);
+              mbar_arrive(bar + RB_TPV_EMPTY + s);
+            }
+          } else {
+            const int r = R - 64;
+            if (r < len) {
+              uint4* orow = reinterpret_cast<uint4*>(p.out + ((size_t)(t0 + r) * H + h) * D + col0);
 #pragma unroll
               for (int cc = 0; cc < 4; ++cc) {
                 uint4 w;
@@ -998,14 +1045,8 @@ __global__ void __launch_bounds__(kRecThreads, 1)
                 orow[cc] = w;
               }
             }
+            tc_fence_before();
           }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        epi_sync();
-        if (et == 0) {
-          mbar_arrive(bar + RB_DELTA);
-          mbar_arrive(bar + RB_TPV_EMPTY + s);
         }
         // ---------------------------------------------------- ep2: state
         const bool last = (c + 1 == nch);
@@ -1014,27 +1055,24 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         if (epi_sync_abort()) break;
         tc_fence_after();
         {
-          const float gam = last ? 1.f : sc_gam[((c + 1) & 1) * (IT_SC_BYTES / 4) + R];
-#pragma unroll 1
-          for (int part = 0; part < 2; ++part) {
-            float v[32];
-            tmem_ld32(tmem + lane_base + TM_S + col0 + 32 * part, v);
-            if (last) {
-              if (p.final_state) store_final(part, v);
-            } else {
-              store_s_bf16(part, v);
-              uint32_t u[32];
+          float v[32];
+          tmem_ld32(tmem + lane_base + TM_S + col0, v);
+          if (last) {
+            if (p.final_state) store_final(v);
+          } else {
+            const float gam = sc_gam[((c + 1) & 1) * (IT_SC_BYTES / 4) + R];
+            store_s_bf16(v);
+            uint32_t u[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam * v[j]);
-              tmem_st32(tmem + lane_base + TM_S + col0 + 32 * part, u);
-            }
+            for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam * v[j]);
+            tmem_st32(tmem + lane_base + TM_S + col0, u);
+            tmem_wait_st();
           }
-          if (!last) tmem_wait_st();
         }
         if (last) break;
         fence_proxy_async();
         tc_fence_before();
-        epi_sync();
+        named_bar(kBarEpi, kEpiThreads);
         if (et == 0) mbar_arrive(bar + RB_S);
       }
     }
