@@ -698,19 +698,27 @@ done:
 }
 
 // ========================================================================= recurrence kernel
-// One CTA per (sequence, head), 640 threads: warp 0 issues the MMAs, warp 1 loads (and zeroes the
-// v rows past a sequence's end), warps 4..19 run the epilogues; warp w reads TMEM lanes
-// 32 (w % 4) .. + 31 and columns 32 cb .. + 31, cb = (w - 4) / 4.  The per-chunk critical path is
-// MMA1 -> ep1 (Delta rows only) -> MMA2 -> ep2; MMA Xv of the next chunk goes into the other
-// [U; P U] buffer in two halves that fill the tensor pipe while ep1 and ep2 run.
+// One CTA per (sequence, head).  The state is carried transposed, S^T (lane = v, column = k), so
+// that every state-side MMA operand lives in tensor memory and the epilogues on the per-chunk
+// critical path never touch shared memory:
+//   MMA Xv   [U^T | (P U)^T]   = V^T [T_b; P T_b]^T           (A = V tile, MN-major; B = TP / TL images)
+//   MMA1     [Delta^T | O^T]  += S^T_bf16 [-W; Qtil - P W]^T  (A = S^T in TMEM; B = WQ image, K-major)
+//   ep1      Delta^T / |k| -> bf16 hi + lo into TMEM (A of MMA2); O^T -> staging tile -> TMA store
+//   MMA2     S^T_tmem += Delta^T (hi + lo) Ktil                (A in TMEM; B = Ktil image, MN-major)
+//   ep2      S^T -> bf16 into TMEM (A of the next MMA1); S^T_tmem <- S^T Diag(e^{Gamma_C} of the next chunk).
+// 640 threads: warp 0 issues the MMAs, warp 1 loads (and zeroes the v rows past a sequence's end),
+// warps 4..19 run the epilogues; warp w reads TMEM lanes 32 (w % 4) .. + 31 and columns
+// 32 cb .. + 31, cb = (w - 4) / 4 (ep1: cb 0, 1 hold Delta^T, cb 2, 3 hold O^T).  MMA Xv of the next
+// chunk goes into the other accumulator buffer in two halves that fill the tensor pipe while ep1
+// and ep2 run.
 constexpr int kRecThreads = 640;
 constexpr int kEpiThreads = 512;
-constexpr uint32_t kBarEpi = 1, kBarDelta = 2;
+constexpr uint32_t kBarEpi = 1, kBarDelta = 2, kBarOut = 3;
 constexpr uint32_t R_TPV = 0;         // 2 stages x [TP 16K][TL 16K][V 16K]
 constexpr uint32_t R_TPV_STAGE = 49152;
 constexpr uint32_t R_WQ = 98304;      // 2 stages x 32K
 constexpr uint32_t R_KT = 163840;     // 2 stages x 16K
-constexpr uint32_t R_SD = 196608;     // 32K: S bf16 (MN tile, 2 blocks x 128 rows) or Delta hi (16K) + lo (16K)
+constexpr uint32_t R_OST = 196608;    // 2 x 16K: O staging tile (same layout as the TMA box of `out`)
 constexpr uint32_t R_SC = 229376;     // 2 stages x 768: 1/|k| and e^{Gamma_C}
 constexpr uint32_t R_BAR = R_SC + 2 * IT_SC_BYTES;
 constexpr uint32_t R_TMEM = R_BAR + 8 * 24;
@@ -718,8 +726,11 @@ constexpr uint32_t R_ABORT = R_TMEM + 4;
 constexpr uint32_t R_SMEM = R_BAR + 256;
 constexpr uint32_t R_ALLOC = R_SMEM + 1024;
 static_assert(R_ALLOC <= 232448, "recurrence shared-memory budget");
-constexpr uint32_t TM_UP = 0;    // 2 buffers x 128 columns: [U; P U] -> [Delta; O] of chunk c in buffer c % 2
-constexpr uint32_t TM_S = 256;   // fp32 state (lane = k, column = v)
+constexpr uint32_t TM_ACC = 0;   // 2 buffers x 128 columns: [U^T | (PU)^T] -> [Delta^T | O^T] of chunk c in buffer c % 2
+constexpr uint32_t TM_ST = 256;  // fp32 S^T (lane = v, column = k)
+constexpr uint32_t TM_SB = 384;  // S^T as bf16 pairs (A of MMA1), 64 columns
+constexpr uint32_t TM_DH = 448;  // Delta^T hi as bf16 pairs (A of MMA2), 32 columns
+constexpr uint32_t TM_DL = 480;  // Delta^T lo
 constexpr uint32_t kRecTmemCols = 512;
 constexpr int kRecPrefetch = 4;  // chunks the loader pulls into L2 ahead of its stage loads
 
@@ -740,7 +751,7 @@ enum {
 };
 
 struct RecMaps {
-  CUtensorMap v;
+  CUtensorMap v, out;
 };
 
 __global__ void __launch_bounds__(kRecThreads, 1)
@@ -772,6 +783,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.v);
+    prefetch_tmap(&maps.out);
   }
   if (warp == 0) {
     tmem_alloc(reinterpret_cast<uint32_t*>(sm + R_TMEM), kRecTmemCols);
@@ -854,24 +866,25 @@ __global__ void __launch_bounds__(kRecThreads, 1)
   } else if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nch > 0) {
-      constexpr uint32_t idesc_k = idesc_bf16(128, 128, false, true);  // A K-major, B MN-major
-      constexpr uint32_t idesc_m = idesc_bf16(128, 128, true, true);   // A and B MN-major
-      // half `part` of MMA Xv: [U; P U] (+)= [T_b; P T_b]_{hi / lo} V into buffer c % 2
+      constexpr uint32_t idesc_xv = idesc_bf16(128, 128, true, false);   // A MN-major (V), B K-major
+      constexpr uint32_t idesc_1 = idesc_bf16(128, 128, false, false);   // A in TMEM, B K-major
+      constexpr uint32_t idesc_2 = idesc_bf16(128, 128, false, true);    // A in TMEM, B MN-major
+      // half `part` of MMA Xv into accumulator buffer c % 2: V^T [T_b; P T_b]_{hi / lo}^T
       auto issue_xv = [&](int c, int part) -> bool {
         const int s = c & 1;
         if (part == 0) {
           if (!wait(RB_TPV_FULL + s, (c >> 1) & 1)) return false;
           if (chunk_len(c) < C && !wait(RB_VZ, 0)) return false;
-          // the buffer held [Delta; O] of chunk c - 2, read by ep1(c - 2): ep2(c - 2) followed it
-          // on every epilogue warp before S(c - 1) arrived, and MMA1(c - 1) waited for S(c - 1)
+          // the buffer held [Delta^T | O^T] of chunk c - 2, read by ep1(c - 2): ep2(c - 2) followed
+          // it on every epilogue warp before S(c - 1) arrived, and MMA1(c - 1) waited for S(c - 1)
           tc_fence_after();
         }
         const uint32_t st = sbase + R_TPV + s * R_TPV_STAGE;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
-          const uint64_t ad = sdesc_sw128(st + 16384 * part + k4 * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(st + 32768 + k4 * 2048, 8192, 1024);
-          umma_bf16(tmem + TM_UP + 128 * (c & 1), ad, bd, idesc_k, part + k4 > 0);
+          const uint64_t ad = sdesc_sw128(st + 32768 + k4 * 2048, 8192, 1024);
+          const uint64_t bd = sdesc_sw128(st + 16384 * part + k4 * 32, 16, 1024);
+          umma_bf16(tmem + TM_ACC + 128 * (c & 1), ad, bd, idesc_xv, part + k4 > 0);
         }
         if (part == 1) umma_commit(bar + RB_TPV_EMPTY + s);
         return true;
@@ -880,31 +893,29 @@ __global__ void __launch_bounds__(kRecThreads, 1)
       for (int c = 0; ok && c < nch; ++c) {
         const int s = c & 1;
         const uint32_t par = (c >> 1) & 1;
-        // MMA1: [Delta; O] = [U; P U] + [-W; Qtil - P W] S
+        // MMA1: [Delta^T | O^T] += S^T [-W; Qtil - P W]^T
         if (!wait(RB_WQ_FULL + s, par) || !wait(RB_S, c & 1)) break;
         tc_fence_after();
         {
           const uint32_t wq = sbase + R_WQ + s * 32768;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t ad = sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sbase + R_SD + ks * 2048, 16384, 1024);
-            umma_bf16(tmem + TM_UP + 128 * (c & 1), ad, bd, idesc_k, 1);
+            const uint64_t bd = sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            umma_bf16_tmem_a(tmem + TM_ACC + 128 * (c & 1), tmem + TM_SB + 8 * ks, bd, idesc_1, 1);
           }
         }
         umma_commit(bar + RB_MMA1);
         umma_commit(bar + RB_WQ_EMPTY + s);
         if (c + 1 < nch && !issue_xv(c + 1, 0)) break;
-        // MMA2: S_tmem += Ktil^T Delta (hi + lo)
+        // MMA2: S^T += Delta^T (hi + lo) Ktil
         if (!wait(RB_KT_FULL + s, par) || !wait(RB_DELTA, c & 1)) break;
         tc_fence_after();
         {
           const uint32_t kt = sbase + R_KT + s * 16384;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t ad = sdesc_sw128(kt + (ks & 3) * 2048, 8192, 1024);
-            const uint64_t bd = sdesc_sw128(sbase + R_SD + (ks < 4 ? 0 : 16384) + (ks & 3) * 2048, 8192, 1024);
-            umma_bf16(tmem + TM_S, ad, bd, idesc_m, 1);
+            const uint64_t bd = sdesc_sw128(kt + (ks & 3) * 2048, 8192, 1024);
+            umma_bf16_tmem_a(tmem + TM_ST, tmem + (ks < 4 ? TM_DH : TM_DL) + 8 * (ks & 3), bd, idesc_2, 1);
           }
         }
         umma_commit(bar + RB_MMA2);
@@ -920,80 +931,79 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     // ------------------------------------------------------------ epilogue warps
     const int et = tid - 128;
     const int quarter = warp & 3, cb = (warp - 4) >> 2;
-    const int R = 32 * quarter + lane;  // TMEM lane: state row k, or chunk row (Delta / O)
-    const bool delta_rows = quarter < 2;
+    const int v = 32 * quarter + lane;  // TMEM lane: the state / output column v
     const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-    const uint32_t col0 = 32 * cb;      // this thread's 32 columns
+    const uint32_t col0 = 32 * cb;      // this thread's 32 columns (k for the state; tokens in ep1)
     const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
     // a barrier of all epilogue warps whose answer (has any role aborted?) is the same for all
     auto epi_sync_abort = [&]() { return named_bar_or(kBarEpi, kEpiThreads, *abort_flag != 0); };
     const float* sc_ik = reinterpret_cast<const float*>(sm + R_SC);
     const float* sc_gam = reinterpret_cast<const float*>(sm + R_SC + (IT_GAM - IT_IK));
+    const bool out_issuer = (cb == 2 && quarter == 0 && lane == 0);  // first thread of the O warps (warp 12)
 
-    auto store_s_bf16 = [&](const float (&v)[32]) {
-      // columns col0 .. + 31 of row R of the bf16 state (MN tile, block cb / 2, 128 rows)
-      uint8_t* base = sm + R_SD + (cb >> 1) * 16384;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint4 w;
-        w.x = pack_bf16(v[8 * cc + 0], v[8 * cc + 1]);
-        w.y = pack_bf16(v[8 * cc + 2], v[8 * cc + 3]);
-        w.z = pack_bf16(v[8 * cc + 4], v[8 * cc + 5]);
-        w.w = pack_bf16(v[8 * cc + 6], v[8 * cc + 7]);
-        *reinterpret_cast<uint4*>(base + sw128(R, 4 * (cb & 1) + cc)) = w;
-      }
-    };
-    auto load_state = [&](float (&v)[32]) {
+    // state columns: S^T[v][k] = S[k][v], k = col0 + j
+    auto load_state = [&](float (&x)[32]) {
       if (!p.initial_state) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        for (int j = 0; j < 32; ++j) x[j] = 0.f;
       } else if (p.state_transposed) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = p.initial_state[soff + (size_t)(col0 + j) * D + R];
-      } else {
-        const float4* src = reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)R * D + col0);
+        const float4* src = reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)v * D + col0);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float4 t = src[j];
-          v[4 * j] = t.x;
-          v[4 * j + 1] = t.y;
-          v[4 * j + 2] = t.z;
-          v[4 * j + 3] = t.w;
+          x[4 * j] = t.x;
+          x[4 * j + 1] = t.y;
+          x[4 * j + 2] = t.z;
+          x[4 * j + 3] = t.w;
         }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = p.initial_state[soff + (size_t)(col0 + j) * D + v];
       }
     };
-    auto store_final = [&](const float (&v)[32]) {
+    auto store_final = [&](const float (&x)[32]) {
       if (p.state_transposed) {
+        float4* dst = reinterpret_cast<float4*>(p.final_state + soff + (size_t)v * D + col0);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) p.final_state[soff + (size_t)(col0 + j) * D + R] = v[j];
+        for (int j = 0; j < 8; ++j) dst[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
       } else {
-        float4* dst = reinterpret_cast<float4*>(p.final_state + soff + (size_t)R * D + col0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        for (int j = 0; j < 32; ++j) p.final_state[soff + (size_t)(col0 + j) * D + v] = x[j];
       }
+    };
+    // bf16 copy (A of MMA1) and the fp32 copy scaled column-wise by gam (the next chunk's decay)
+    auto store_state = [&](const float (&x)[32], const float* gam) {
+      uint32_t b[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) b[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
+      tmem_st16(tmem + lane_base + TM_SB + col0 / 2, b);
+      uint32_t u[32];
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 g = *reinterpret_cast<const float4*>(gam + col0 + j);
+        u[j] = __float_as_uint(g.x * x[j]);
+        u[j + 1] = __float_as_uint(g.y * x[j + 1]);
+        u[j + 2] = __float_as_uint(g.z * x[j + 2]);
+        u[j + 3] = __float_as_uint(g.w * x[j + 3]);
+      }
+      tmem_st32(tmem + lane_base + TM_ST + col0, u);
+      tmem_wait_st();
     };
 
     if (nch == 0) {
       if (p.final_state) {
-        float v[32];
-        load_state(v);
-        store_final(v);
+        float x[32];
+        load_state(x);
+        store_final(x);
       }
     } else {
-      // initial state: bf16 copy for MMA1(0); fp32 copy pre-scaled by e^{Gamma_C}(0) for MMA2(0)
+      // initial state: bf16 copy for MMA1(0); fp32 copy scaled by e^{Gamma_C}(0) for MMA2(0)
       wait(RB_TPV_FULL, 0);
       {
-        const float gam0 = sc_gam[R];
-        float v[32];
-        load_state(v);
-        store_s_bf16(v);
-        uint32_t u[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam0 * v[j]);
-        tmem_st32(tmem + lane_base + TM_S + col0, u);
+        float x[32];
+        load_state(x);
+        store_state(x, sc_gam);
       }
-      tmem_wait_st();
-      fence_proxy_async();
       tc_fence_before();
       named_bar(kBarEpi, kEpiThreads);
       if (et == 0) mbar_arrive(bar + RB_S);
@@ -1002,51 +1012,62 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         const int s = c & 1;
         const int len = chunk_len(c);
         const int64_t t0 = bos + (int64_t)c * C;
-        const uint32_t up = tmem + lane_base + TM_UP + 128 * (c & 1) + col0;
-        // ---------------------------------------------------- ep1: Delta (rows 0..63) and O (rows 64..127)
-        if (delta_rows) wait(RB_TPV_FULL + s, (c >> 1) & 1);  // 1/|k| of this chunk
+        const uint32_t acc = tmem + lane_base + TM_ACC + 128 * (c & 1);
+        // ---------------------------------------------------- ep1: Delta^T (columns 0..63), O^T (64..127)
+        if (cb < 2) wait(RB_TPV_FULL + s, (c >> 1) & 1);  // 1/|k| of this chunk
         wait(RB_MMA1, c & 1);
         if (epi_sync_abort()) break;
         tc_fence_after();
-        {
+        if (cb < 2) {
           float d[32];
-          tmem_ld32(up, d);
-          if (delta_rows) {
-            const float ikr = sc_ik[s * (IT_SC_BYTES / 4) + R];
+          tmem_ld32(acc + col0, d);
+          const float* ik = sc_ik + s * (IT_SC_BYTES / 4) + col0;  // 1/|k_t| of tokens col0 .. + 31
+          uint32_t hi[16], lo[16];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              uint4 wh, wl;
-              split2(d[8 * cc + 0] * ikr, d[8 * cc + 1] * ikr, wh.x, wl.x);
-              split2(d[8 * cc + 2] * ikr, d[8 * cc + 3] * ikr, wh.y, wl.y);
-              split2(d[8 * cc + 4] * ikr, d[8 * cc + 5] * ikr, wh.z, wl.z);
-              split2(d[8 * cc + 6] * ikr, d[8 * cc + 7] * ikr, wh.w, wl.w);
-              const uint32_t off = (cb >> 1) * 8192 + sw128(R, 4 * (cb & 1) + cc);
-              *reinterpret_cast<uint4*>(sm + R_SD + off) = wh;
-              *reinterpret_cast<uint4*>(sm + R_SD + 16384 + off) = wl;
+          for (int j = 0; j < 32; j += 4) {
+            const float4 f = *reinterpret_cast<const float4*>(ik + j);
+            split2(d[j] * f.x, d[j + 1] * f.y, hi[j / 2], lo[j / 2]);
+            split2(d[j + 2] * f.z, d[j + 3] * f.w, hi[j / 2 + 1], lo[j / 2 + 1]);
+          }
+          tmem_st16(tmem + lane_base + TM_DH + col0 / 2, hi);
+          tmem_st16(tmem + lane_base + TM_DL + col0 / 2, lo);
+          tmem_wait_st();
+          tc_fence_before();
+          named_bar(kBarDelta, kEpiThreads / 2);
+          if (et == 0) {
+            mbar_arrive(bar + RB_DELTA);
+            mbar_arrive(bar + RB_TPV_EMPTY + s);
+          }
+        } else {
+          float d[32];
+          tmem_ld32(acc + col0, d);  // O^T of tokens tb .. tb + 31
+          const int tb = (int)col0 - 64;
+          if (len == C) {
+            // staging tile [2 blocks of 64 v][64 tokens][128 B], 128-byte swizzle (the TMA box layout)
+            uint8_t* ost = sm + R_OST + (c & 1) * 16384 + (v >> 6) * 8192;
+            if (out_issuer) bulk_wait_read<1>();  // the store of chunk c - 2 has read this buffer
+            named_bar(kBarOut, kEpiThreads / 2);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = tb + j;
+              *reinterpret_cast<__nv_bfloat16*>(ost + sw128(t, (v & 63) >> 3) + (v & 7) * 2) = __float2bfloat16_rn(d[j]);
             }
             fence_proxy_async();
-            tc_fence_before();
-            named_bar(kBarDelta, kEpiThreads / 2);
-            if (et == 0) {
-              mbar_arrive(bar + RB_DELTA);
-              mbar_arrive(bar + RB_TPV_EMPTY + s);
+            named_bar(kBarOut, kEpiThreads / 2);
+            if (out_issuer) {
+              const uint8_t* base = sm + R_OST + (c & 1) * 16384;
+              tma_store_3d(&maps.out, base, 0, h, (int)t0);
+              tma_store_3d(&maps.out, base + 8192, 64, h, (int)t0);
+              bulk_commit();
             }
           } else {
-            const int r = R - 64;
-            if (r < len) {
-              uint4* orow = reinterpret_cast<uint4*>(p.out + ((size_t)(t0 + r) * H + h) * D + col0);
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                uint4 w;
-                w.x = pack_bf16(d[8 * cc + 0], d[8 * cc + 1]);
-                w.y = pack_bf16(d[8 * cc + 2], d[8 * cc + 3]);
-                w.z = pack_bf16(d[8 * cc + 4], d[8 * cc + 5]);
-                w.w = pack_bf16(d[8 * cc + 6], d[8 * cc + 7]);
-                orow[cc] = w;
-              }
+            // the last chunk of a sequence: only rows below len belong to it
+            for (int j = 0; j < 32; ++j) {
+              const int t = tb + j;
+              if (t < len) p.out[((size_t)(t0 + t) * H + h) * D + v] = __float2bfloat16_rn(d[j]);
             }
-            tc_fence_before();
           }
+          tc_fence_before();
         }
         // ---------------------------------------------------- ep2: state
         const bool last = (c + 1 == nch);
@@ -1055,26 +1076,20 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         if (epi_sync_abort()) break;
         tc_fence_after();
         {
-          float v[32];
-          tmem_ld32(tmem + lane_base + TM_S + col0, v);
+          float x[32];
+          tmem_ld32(tmem + lane_base + TM_ST + col0, x);
           if (last) {
-            if (p.final_state) store_final(v);
+            if (p.final_state) store_final(x);
           } else {
-            const float gam = sc_gam[((c + 1) & 1) * (IT_SC_BYTES / 4) + R];
-            store_s_bf16(v);
-            uint32_t u[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(gam * v[j]);
-            tmem_st32(tmem + lane_base + TM_S + col0, u);
-            tmem_wait_st();
+            store_state(x, sc_gam + ((c + 1) & 1) * (IT_SC_BYTES / 4));
           }
         }
         if (last) break;
-        fence_proxy_async();
         tc_fence_before();
         named_bar(kBarEpi, kEpiThreads);
         if (et == 0) mbar_arrive(bar + RB_S);
       }
+      if (out_issuer) bulk_wait_all();
     }
   }
 
@@ -1113,7 +1128,7 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
   IntraMaps im;
   RecMaps rm;
   if (!make_token_map(&im.q, p.q, tokens, p.num_heads) || !make_token_map(&im.k, p.k, tokens, p.num_heads) ||
-      !make_token_map(&rm.v, p.v, tokens, p.num_heads))
+      !make_token_map(&rm.v, p.v, tokens, p.num_heads) || !make_token_map(&rm.out, p.out, tokens, p.num_heads))
     return cudaErrorInvalidValue;
   cudaError_t e = set_smem_once(intra_kernel, I_ALLOC, g_intra_attr);
   if (e != cudaSuccess) return e;
