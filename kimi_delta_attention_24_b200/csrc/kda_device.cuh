@@ -64,6 +64,25 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
   }
 }
 
+// Bounded wait that polls without suspending (lowest wake-up latency, for the few threads on a
+// critical path).  Same contract as bounded_wait.
+__device__ __forceinline__ bool bounded_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             uint32_t* status) {
+  if (sm100::mbar_test(bar, parity)) return true;
+  const uint64_t t0 = sm100::globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (sm100::mbar_test(bar, parity)) return true;
+    if ((n & 255) == 0) {
+      if (*abort) return false;
+      if (sm100::globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        if (status) atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,

@@ -713,7 +713,7 @@ done:
 // and ep2 run.
 constexpr int kRecThreads = 640;
 constexpr int kEpiThreads = 512;
-constexpr uint32_t kBarEpi = 1, kBarDelta = 2, kBarOut = 3;
+constexpr uint32_t kBarEpi = 1, kBarDelta = 2, kBarOut = 3, kBarOutGo = 4;
 constexpr uint32_t R_TPV = 0;         // 2 stages x [TP 16K][TL 16K][V 16K]
 constexpr uint32_t R_TPV_STAGE = 49152;
 constexpr uint32_t R_WQ = 98304;      // 2 stages x 32K
@@ -745,9 +745,10 @@ enum {
   RB_MMA1 = 13,
   RB_DELTA = 14,
   RB_MMA2 = 15,
-  RB_S = 16,
-  RB_FINAL = 17,
-  RB_COUNT = 18
+  RB_S = 16,         // bf16 S^T written (A of the next MMA1)
+  RB_ST = 17,        // fp32 S^T rescaled by the next chunk's decay (accumulator of the next MMA2)
+  RB_FINAL = 18,
+  RB_COUNT = 19
 };
 
 struct RecMaps {
@@ -777,6 +778,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     return args.items + ((size_t)(item0 + c) * H + h) * ITEM_BYTES;
   };
   auto wait = [&](int b, uint32_t parity) { return bounded_wait(bar + b, parity, abort_flag, p.status); };
+  auto spin = [&](int b, uint32_t parity) { return bounded_spin(bar + b, parity, abort_flag, p.status); };
 
   if (tid == 0) {
     for (int b = 0; b < RB_COUNT; ++b) mbar_init(bar + b, (b == RB_TPV_EMPTY || b == RB_TPV_EMPTY + 1) ? 2 : 1);
@@ -894,7 +896,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         const int s = c & 1;
         const uint32_t par = (c >> 1) & 1;
         // MMA1: [Delta^T | O^T] += S^T [-W; Qtil - P W]^T
-        if (!wait(RB_WQ_FULL + s, par) || !wait(RB_S, c & 1)) break;
+        if (!wait(RB_WQ_FULL + s, par) || !spin(RB_S, c & 1)) break;
         tc_fence_after();
         {
           const uint32_t wq = sbase + R_WQ + s * 32768;
@@ -908,7 +910,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         umma_commit(bar + RB_WQ_EMPTY + s);
         if (c + 1 < nch && !issue_xv(c + 1, 0)) break;
         // MMA2: S^T += Delta^T (hi + lo) Ktil
-        if (!wait(RB_KT_FULL + s, par) || !wait(RB_DELTA, c & 1)) break;
+        if (!wait(RB_KT_FULL + s, par) || !spin(RB_DELTA, c & 1) || !spin(RB_ST, c & 1)) break;
         tc_fence_after();
         {
           const uint32_t kt = sbase + R_KT + s * 16384;
@@ -971,12 +973,16 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         for (int j = 0; j < 32; ++j) p.final_state[soff + (size_t)(col0 + j) * D + v] = x[j];
       }
     };
-    // bf16 copy (A of MMA1) and the fp32 copy scaled column-wise by gam (the next chunk's decay)
-    auto store_state = [&](const float (&x)[32], const float* gam) {
+    // bf16 copy (A of MMA1)
+    auto store_state_bf16 = [&](const float (&x)[32]) {
       uint32_t b[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) b[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
       tmem_st16(tmem + lane_base + TM_SB + col0 / 2, b);
+      tmem_wait_st();
+    };
+    // fp32 copy scaled column-wise by gam (the next chunk's decay): the accumulator of the next MMA2
+    auto store_state_scaled = [&](const float (&x)[32], const float* gam) {
       uint32_t u[32];
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
@@ -1002,11 +1008,15 @@ __global__ void __launch_bounds__(kRecThreads, 1)
       {
         float x[32];
         load_state(x);
-        store_state(x, sc_gam);
+        store_state_bf16(x);
+        store_state_scaled(x, sc_gam);
       }
       tc_fence_before();
       named_bar(kBarEpi, kEpiThreads);
-      if (et == 0) mbar_arrive(bar + RB_S);
+      if (et == 0) {
+        mbar_arrive(bar + RB_S);
+        mbar_arrive(bar + RB_ST);
+      }
 
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
@@ -1015,7 +1025,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         const uint32_t acc = tmem + lane_base + TM_ACC + 128 * (c & 1);
         // ---------------------------------------------------- ep1: Delta^T (columns 0..63), O^T (64..127)
         if (cb < 2) wait(RB_TPV_FULL + s, (c >> 1) & 1);  // 1/|k| of this chunk
-        wait(RB_MMA1, c & 1);
+        spin(RB_MMA1, c & 1);
         if (epi_sync_abort()) break;
         tc_fence_after();
         if (cb < 2) {
@@ -1038,7 +1048,9 @@ __global__ void __launch_bounds__(kRecThreads, 1)
             mbar_arrive(bar + RB_DELTA);
             mbar_arrive(bar + RB_TPV_EMPTY + s);
           }
+          named_bar_arrive(kBarOutGo, kEpiThreads);  // the O warps start once Delta^T is out
         } else {
+          named_bar(kBarOutGo, kEpiThreads);
           float d[32];
           tmem_ld32(acc + col0, d);  // O^T of tokens tb .. tb + 31
           const int tb = (int)col0 - 64;
@@ -1071,23 +1083,25 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         }
         // ---------------------------------------------------- ep2: state
         const bool last = (c + 1 == nch);
-        wait(RB_MMA2, c & 1);
+        spin(RB_MMA2, c & 1);
         if (!last) wait(RB_TPV_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1);
         if (epi_sync_abort()) break;
         tc_fence_after();
-        {
-          float x[32];
-          tmem_ld32(tmem + lane_base + TM_ST + col0, x);
-          if (last) {
-            if (p.final_state) store_final(x);
-          } else {
-            store_state(x, sc_gam + ((c + 1) & 1) * (IT_SC_BYTES / 4));
-          }
+        float x[32];
+        tmem_ld32(tmem + lane_base + TM_ST + col0, x);
+        if (last) {
+          if (p.final_state) store_final(x);
+          break;
         }
-        if (last) break;
+        store_state_bf16(x);
         tc_fence_before();
         named_bar(kBarEpi, kEpiThreads);
         if (et == 0) mbar_arrive(bar + RB_S);
+        // off the critical path (MMA1 of the next chunk runs meanwhile): the rescaled fp32 state
+        store_state_scaled(x, sc_gam + ((c + 1) & 1) * (IT_SC_BYTES / 4));
+        tc_fence_before();
+        named_bar(kBarEpi, kEpiThreads);
+        if (et == 0) mbar_arrive(bar + RB_ST);
       }
       if (out_issuer) bulk_wait_all();
     }

@@ -54,6 +54,10 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Arrives on a named barrier without waiting for it.
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 // Named barrier that also ORs a predicate over the participating threads: every thread gets the
 // same answer.
 __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t count, bool pred) {
