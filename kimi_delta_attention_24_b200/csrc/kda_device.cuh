@@ -115,6 +115,19 @@ inline bool make_token_map(CUtensorMap* map, const void* base, int64_t tokens, i
   return r == CUDA_SUCCESS;
 }
 
+// Number of SMs of the current device (looked up once per device); 0 on error.
+inline int sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
 // Sets the dynamic shared-memory limit of `kernel` once per device.
 template <typename Kernel>
 inline cudaError_t set_smem_once(Kernel kernel, uint32_t bytes, bool (&done)[64]) {

@@ -134,9 +134,9 @@ constexpr uint32_t AS_LD = 68;
 constexpr uint32_t I_SC = 106496;   // scalars
 constexpr uint32_t I_TOT = I_SC;            // float[8][128] per-warp alpha products
 constexpr uint32_t I_BETA = I_SC + 4096;    // float[64]
-constexpr uint32_t I_BAR = I_SC + 4352;     // 2 mbarriers
-constexpr uint32_t I_TMEM = I_SC + 4368;    // allocated TMEM address
-constexpr uint32_t I_ABORT = I_SC + 4372;
+constexpr uint32_t I_BAR = I_SC + 4352;     // 3 mbarriers
+constexpr uint32_t I_TMEM = I_SC + 4376;    // allocated TMEM address
+constexpr uint32_t I_ABORT = I_SC + 4380;
 constexpr uint32_t I_SMEM = I_SC + 4480;
 constexpr uint32_t I_ALLOC = I_SMEM + 1024;
 static_assert(I_YS + 3072 <= I_SC, "intra shared-memory map");
@@ -144,30 +144,29 @@ static_assert(2 * (I_ALLOC + 1024) <= 233472, "two intra CTAs per SM");
 constexpr uint32_t kIntraTmemCols = 256;
 
 struct IntraMaps {
-  CUtensorMap q, k;
+  CUtensorMap q, k, g;
 };
 
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ uint32_t bf16x2_of(float2 v) { return bf16x2(v.x, v.y); }
+
+// Persistent: every CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ... in chunk-major order
+// (item = global chunk * H + head), pulling its next item's q, k and g tiles into L2 while it works.
 __global__ void __launch_bounds__(kIntraThreads, 2)
     intra_kernel(const __grid_constant__ IntraMaps maps, const SplitArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const FwdParams& p = args.p;
   const int H = p.num_heads;
-  const int64_t gc = blockIdx.x / H;
-  const int h = blockIdx.x % H;
   const int32_t* co = args.chunk_off;
-  if (gc >= (int64_t)co[p.num_seqs]) return;
-  const int n = seq_of_chunk(co, p.num_seqs, gc);
-  int64_t bos, eos;
-  seq_range(p, n, bos, eos);
-  const int64_t t0 = bos + (gc - co[n]) * C;
-  const int len = (int)((eos - t0) < (int64_t)C ? (eos - t0) : (int64_t)C);
-  uint8_t* item = args.items + ((size_t)gc * H + h) * ITEM_BYTES;
 
   const int itid = threadIdx.x;
   const int iw = itid >> 5, lane = itid & 31;
   const uint32_t sbase = smem_u32(sm);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + I_BAR);  // [0] q/k tiles landed, [1] MMA done
+  // [0] q/k tiles landed, [1] MMA done, [2] final drain
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + I_BAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + I_ABORT);
   float* sc_tot = reinterpret_cast<float*>(sm + I_TOT);
   float* sc_beta = reinterpret_cast<float*>(sm + I_BETA);
@@ -179,27 +178,58 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   if (itid == 0) {
     mbar_init(bar + 0, 1);
     mbar_init(bar + 1, 1);
+    mbar_init(bar + 2, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.q);
     prefetch_tmap(&maps.k);
-    mbar_arrive_expect_tx(bar + 0, 32768);
-    tma_load_3d(sm + I_RQ, &maps.q, bar + 0, 0, h, (int)t0);
-    tma_load_3d(sm + I_RQ + 8192, &maps.q, bar + 0, 64, h, (int)t0);
-    tma_load_3d(sm + I_RK, &maps.k, bar + 0, 0, h, (int)t0);
-    tma_load_3d(sm + I_RK + 8192, &maps.k, bar + 0, 64, h, (int)t0);
+    prefetch_tmap(&maps.g);
   }
   if (iw == 0) {
     tmem_alloc(reinterpret_cast<uint32_t*>(sm + I_TMEM), kIntraTmemCols);
     tmem_relinquish();
   }
+  tc_fence_before();
+  sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + I_TMEM);
+
+  // one thread waits on the mbarrier, the others in the CTA barrier; the answer (abort?) is uniform
+  uint32_t raw_par = 0, mma_par = 0;
+  bool raw_pending = false;  // thread 0: a q/k load is armed and has not been seen to land
+  auto cta_wait = [&](int b, uint32_t& par) -> bool {
+    if (itid == 0 && bounded_wait(bar + b, par, abort_flag, p.status) && b == 0) raw_pending = false;
+    par ^= 1;
+    return __syncthreads_or(*abort_flag) != 0;
+  };
+  // item = gc * H + h advances by gridDim.x = step_gc * H + step_h per iteration (no division)
+  struct Loc {
+    int h, len;
+    int64_t t0, gc;
+  };
+  auto locate = [&](int64_t gc, int h) {
+    Loc L;
+    L.gc = gc;
+    L.h = h;
+    const int n = seq_of_chunk(co, p.num_seqs, gc);
+    int64_t bos, eos;
+    seq_range(p, n, bos, eos);
+    L.t0 = bos + (gc - co[n]) * C;
+    L.len = (int)((eos - L.t0) < (int64_t)C ? (eos - L.t0) : (int64_t)C);
+    return L;
+  };
+  const int step_gc = (int)(gridDim.x / (unsigned)H), step_h = (int)(gridDim.x % (unsigned)H);
+  auto advance = [&](int64_t& gc, int& h) {
+    gc += step_gc;
+    h += step_h;
+    if (h >= H) {
+      h -= H;
+      ++gc;
+    }
+  };
+  const int64_t total_gc = co[p.num_seqs];
 
   // prologue mapping: warp iw owns chunk rows 8 iw .. 8 iw + 7, lane owns channels 4 lane .. +3
-  const float gate_a = __expf(p.A_log[h]);
-  const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-  const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
-  const float gb[4] = {ga * dtb.x, ga * dtb.y, ga * dtb.z, ga * dtb.w};
-  const float lb2 = p.lower_bound * kLog2e;
   const int kb = lane >> 4;
   const uint32_t lane_chunk = (lane & 15) >> 1;
   const uint32_t lane_sub = (lane & 1) * 8;
@@ -207,15 +237,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const bool upper_half = iw & 1;
   const int quarter = iw & 3, ihalf = iw >> 2;  // TMEM lane quarter, column half
   const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-
-  uint2 gr[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t t = t0 + 8 * iw + i;
-    gr[i] = (8 * iw + i < len) ? ldg_u2(p.g + ((size_t)t * H + h) * D + 4 * lane) : make_uint2(0, 0);
-  }
-  const float beta_raw =
-      (8 * iw + (lane & 7) < len) ? __bfloat162float(p.beta[(size_t)(t0 + 8 * iw + (lane & 7)) * H + h]) : 0.f;
+  const float lb2 = p.lower_bound * kLog2e;
   // shared-memory byte offset of this thread's 8 bytes of row 8 iw + i inside a 128-byte-row tile
   uint32_t xo[8];
 #pragma unroll
@@ -225,472 +247,517 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const uint32_t a_xk = sbase + I_XK + kb * 8192, a_qb = sbase + I_QB + kb * 8192;
   const uint32_t a_r = sbase + I_R + kb * I_RKBLK;
 
-  tc_fence_before();
-  sync();
-  tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + I_TMEM);
-
-  // ================================================================ prologue
-  bounded_wait(bar + 0, 0, abort_flag, p.status);
-  uint2 qr[8], kr[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const bool valid = 8 * iw + i < len;
-    qr[i] = valid ? lds64(a_rq + xo[i]) : make_uint2(0, 0);
-    kr[i] = valid ? lds64(a_rk + xo[i]) : make_uint2(0, 0);
-  }
-  float a[8][4];  // alpha
-  float ssq[8], ssk[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const bool valid = 8 * iw + i < len;
-    const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
-    const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
-    ssq[i] = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
-    ssk[i] = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
-    const float2 g01 = unpack_bf16(gr[i].x), g23 = unpack_bf16(gr[i].y);
-    const float gv[4] = {g01.x, g01.y, g23.x, g23.y};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float sig = rcp_approx(1.0f + ex2_approx(fmaf(ga, gv[j], gb[j])));
-      a[i][j] = valid ? ex2_approx(lb2 * sig) : 1.0f;
+  int64_t cur_gc = blockIdx.x / (unsigned)H;
+  int cur_h = (int)(blockIdx.x % (unsigned)H);
+  for (; cur_gc < total_gc; advance(cur_gc, cur_h)) {
+    const Loc L = locate(cur_gc, cur_h);
+    const int h = L.h, len = L.len;
+    const int64_t t0 = L.t0;
+    uint8_t* item = args.items + ((size_t)L.gc * H + h) * ITEM_BYTES;
+    if (itid == 0) {
+      raw_pending = true;
+      mbar_arrive_expect_tx(bar + 0, 32768);
+      tma_load_3d(sm + I_RQ, &maps.q, bar + 0, 0, h, (int)t0);
+      tma_load_3d(sm + I_RQ + 8192, &maps.q, bar + 0, 64, h, (int)t0);
+      tma_load_3d(sm + I_RK, &maps.k, bar + 0, 0, h, (int)t0);
+      tma_load_3d(sm + I_RK + 8192, &maps.k, bar + 0, 64, h, (int)t0);
+      int64_t ngc = cur_gc;
+      int nh = cur_h;
+      advance(ngc, nh);
+      if (ngc < total_gc) {
+        const Loc N = locate(ngc, nh);
+        tma_prefetch_3d(&maps.q, 0, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.q, 64, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.k, 0, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.k, 64, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.g, 0, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.g, 64, N.h, (int)N.t0);
+      }
     }
-  }
-  // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
-  // total of value (l >> 1): q rows 0..7, then k rows 0..7
-  float inv;
-  {
-    float v16[16];
+    const float gate_a = __expf(p.A_log[h]);
+    const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+    const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
+    const float2 ga2 = splat2(ga);
+    const float2 gb2[2] = {make_float2(ga * dtb.x, ga * dtb.y), make_float2(ga * dtb.z, ga * dtb.w)};
+    uint2 gr[8];
+    {
+      const __nv_bfloat16* gp = p.g + ((size_t)(t0 + 8 * iw) * H + h) * D + 4 * lane;
+      const uint32_t row_stride = (uint32_t)H * D;  // elements between consecutive tokens
+#pragma unroll
+      for (int i = 0; i < 8; ++i) gr[i] = (8 * iw + i < len) ? ldg_u2(gp + i * row_stride) : make_uint2(0, 0);
+    }
+    const float beta_raw =
+        (8 * iw + (lane & 7) < len)
+            ? __bfloat162float(p.beta[(size_t)(t0 + 8 * iw) * H + h + (uint32_t)(lane & 7) * (uint32_t)H])
+            : 0.f;
+
+    // ================================================================ prologue
+    if (cta_wait(0, raw_par)) break;
+    uint2 qr[8], kr[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      v16[i] = ssq[i];
-      v16[8 + i] = ssk[i];
+      const bool valid = 8 * iw + i < len;
+      qr[i] = valid ? lds64(a_rq + xo[i]) : make_uint2(0, 0);
+      kr[i] = valid ? lds64(a_rk + xo[i]) : make_uint2(0, 0);
     }
-    const bool b4 = lane & 16;
-    float w8[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      w8[j] = (b4 ? v16[j + 8] : v16[j]) + __shfl_xor_sync(0xffffffffu, b4 ? v16[j] : v16[j + 8], 16);
-    const bool b3 = lane & 8;
-    float w4[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      w4[j] = (b3 ? w8[j + 4] : w8[j]) + __shfl_xor_sync(0xffffffffu, b3 ? w8[j] : w8[j + 4], 8);
-    const bool b2 = lane & 4;
-    float w2[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-      w2[j] = (b2 ? w4[j + 2] : w4[j]) + __shfl_xor_sync(0xffffffffu, b2 ? w4[j] : w4[j + 2], 4);
-    const bool b1 = lane & 2;
-    float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
-    w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
-    inv = rsqrtf(w1 + kL2Eps);
-  }
-  const float beta_l = (lane < 8 && 8 * iw + lane < len) ? fast_sigmoid(beta_raw) : 0.f;
-  const float inv_s = inv * (lane < 16 ? p.scale : 1.f);  // scale folded into 1/|q|
-  {
-    const float ikr = __shfl_sync(0xffffffffu, inv, 16 + 2 * (lane & 7));  // 1/|k| of row 8 iw + (lane & 7)
-    if (lane < 8) {
-      const int r = 8 * iw + lane;
-      sc_beta[r] = beta_l;
-      reinterpret_cast<float*>(item + IT_IK)[r] = (r < len) ? ikr : 0.f;
-    }
-  }
-  // per-warp alpha totals -> sub-block totals b_J
-  {
-    float tot[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float t = a[0][j];
-#pragma unroll
-      for (int i = 1; i < 8; ++i) t *= a[i][j];
-      tot[j] = t;
-    }
-    reinterpret_cast<float4*>(sc_tot + iw * 128)[lane] = make_float4(tot[0], tot[1], tot[2], tot[3]);
-  }
-  sync();  // also: every thread holds its q, k rows, so the raw tiles may be overwritten
-  // sub-block totals b_J = prod of alpha over rows 16 J .. 16 J + 15 (channels 4 lane .. + 3)
-  auto load_bJ = [&](float (&bJ)[4][4]) {
-#pragma unroll
-    for (int J = 0; J < 4; ++J) {
-      const float4 t0v = reinterpret_cast<const float4*>(sc_tot + (2 * J) * 128)[lane];
-      const float4 t1v = reinterpret_cast<const float4*>(sc_tot + (2 * J + 1) * 128)[lane];
-      bJ[J][0] = t0v.x * t1v.x;
-      bJ[J][1] = t0v.y * t1v.y;
-      bJ[J][2] = t0v.z * t1v.z;
-      bJ[J][3] = t0v.w * t1v.w;
-    }
-  };
-  float pre[4], pt[4];
-  {
-    float bJ[4][4];
-    load_bJ(bJ);
-    const float4 pv = reinterpret_cast<const float4*>(sc_tot + (iw ^ 1) * 128)[lane];
-    pt[0] = pv.x;
-    pt[1] = pv.y;
-    pt[2] = pv.z;
-    pt[3] = pv.w;
-    float gam[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float pa = 1.f;
-#pragma unroll
-      for (int J = 0; J < 4; ++J)
-        if (J < blk) pa *= bJ[J][j];
-      pre[j] = pa;
-      gam[j] = bJ[0][j] * bJ[1][j] * bJ[2][j] * bJ[3][j];
-    }
-    if (iw == 0) reinterpret_cast<float4*>(item + IT_GAM)[lane] = make_float4(gam[0], gam[1], gam[2], gam[3]);
-  }
-
-  // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i
-  {
-    float run[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) run[j] = upper_half ? pt[j] : 1.f;
+    float2 a2[8][2];  // alpha of channels (4 lane, +1), (4 lane + 2, +3)
+    float ssq[8], ssk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
+      const bool valid = 8 * iw + i < len;
       const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
       const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
-      const float qv[4] = {q01.x, q01.y, q23.x, q23.y};
-      const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
-      const float iq = __shfl_sync(0xffffffffu, inv_s, 2 * i), ik = __shfl_sync(0xffffffffu, inv_s, 16 + 2 * i);
-      const float b = __shfl_sync(0xffffffffu, beta_l, i);
-      float lk[4], lq[4];
+      const float2 sq = fma2(q23, q23, mul2(q01, q01)), sk = fma2(k23, k23, mul2(k01, k01));
+      ssq[i] = sq.x + sq.y;
+      ssk[i] = sk.x + sk.y;
+      const float2 gv[2] = {unpack_bf16(gr[i].x), unpack_bf16(gr[i].y)};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        run[j] *= a[i][j];
-        lk[j] = kv[j] * (run[j] * ik);  // khat * e
-        lq[j] = qv[j] * (run[j] * iq);  // scale * qhat * e
+      for (int m = 0; m < 2; ++m) {
+        const float2 x = fma2(ga2, gv[m], gb2[m]);
+        const float2 d = make_float2(1.0f + ex2_approx(x.x), 1.0f + ex2_approx(x.y));
+        const float2 y = mul2(splat2(lb2), make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+        a2[i][m] = valid ? make_float2(ex2_approx(y.x), ex2_approx(y.y)) : make_float2(1.f, 1.f);
       }
-      sts64(a_lk + xo[i], bf16x2(lk[0] * b, lk[1] * b), bf16x2(lk[2] * b, lk[3] * b));
-      sts64(a_lq + xo[i], bf16x2(lq[0], lq[1]), bf16x2(lq[2], lq[3]));
-      sts64(a_xk + xo[i], bf16x2(lk[0] * pre[0], lk[1] * pre[1]), bf16x2(lk[2] * pre[2], lk[3] * pre[3]));
-      sts64(a_qb + xo[i], bf16x2(lq[0] * pre[0], lq[1] * pre[1]), bf16x2(lq[2] * pre[2], lq[3] * pre[3]));
     }
-  }
-  // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end; Ktil goes
-  // straight to the item (same swizzled image as a shared-memory MN tile)
-  {
-    float post[4], cI[4][4];
+    // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
+    // total of value (l >> 1): q rows 0..7, then k rows 0..7
+    float inv;
     {
-      float bJ[4][4];
-      load_bJ(bJ);
+      float v16[16];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float z = 1.f;
+      for (int i = 0; i < 8; ++i) {
+        v16[i] = ssq[i];
+        v16[8 + i] = ssk[i];
+      }
+      const bool b4 = lane & 16;
+      float w8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        w8[j] = (b4 ? v16[j + 8] : v16[j]) + __shfl_xor_sync(0xffffffffu, b4 ? v16[j] : v16[j + 8], 16);
+      const bool b3 = lane & 8;
+      float w4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w4[j] = (b3 ? w8[j + 4] : w8[j]) + __shfl_xor_sync(0xffffffffu, b3 ? w8[j] : w8[j + 4], 8);
+      const bool b2 = lane & 4;
+      float w2[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        w2[j] = (b2 ? w4[j + 2] : w4[j]) + __shfl_xor_sync(0xffffffffu, b2 ? w4[j] : w4[j + 2], 4);
+      const bool b1 = lane & 2;
+      float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
+      w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
+      inv = rsqrtf(w1 + kL2Eps);
+    }
+    const float beta_l = (lane < 8 && 8 * iw + lane < len) ? fast_sigmoid(beta_raw) : 0.f;
+    const float inv_s = inv * (lane < 16 ? p.scale : 1.f);  // scale folded into 1/|q|
+    {
+      const float ikr = __shfl_sync(0xffffffffu, inv, 16 + 2 * (lane & 7));  // 1/|k| of row 8 iw + (lane & 7)
+      if (lane < 8) {
+        const int r = 8 * iw + lane;
+        sc_beta[r] = beta_l;
+        reinterpret_cast<float*>(item + IT_IK)[r] = (r < len) ? ikr : 0.f;
+      }
+    }
+    // per-warp alpha totals -> sub-block totals b_J
+    {
+      float2 t[2] = {a2[0][0], a2[0][1]};
+#pragma unroll
+      for (int i = 1; i < 8; ++i) {
+        t[0] = mul2(t[0], a2[i][0]);
+        t[1] = mul2(t[1], a2[i][1]);
+      }
+      reinterpret_cast<float4*>(sc_tot + iw * 128)[lane] = make_float4(t[0].x, t[0].y, t[1].x, t[1].y);
+    }
+    sync();  // also: every thread holds its q, k rows, so the raw tiles may be overwritten
+    // sub-block totals b_J = prod of alpha over rows 16 J .. 16 J + 15 (channels 4 lane .. + 3)
+    auto load_bJ = [&](float2 (&bJ)[4][2]) {
+#pragma unroll
+      for (int J = 0; J < 4; ++J) {
+        const float4 t0v = reinterpret_cast<const float4*>(sc_tot + (2 * J) * 128)[lane];
+        const float4 t1v = reinterpret_cast<const float4*>(sc_tot + (2 * J + 1) * 128)[lane];
+        bJ[J][0] = mul2(make_float2(t0v.x, t0v.y), make_float2(t1v.x, t1v.y));
+        bJ[J][1] = mul2(make_float2(t0v.z, t0v.w), make_float2(t1v.z, t1v.w));
+      }
+    };
+    float2 pre[2], pt[2];
+    {
+      float2 bJ[4][2];
+      load_bJ(bJ);
+      const float4 pv = reinterpret_cast<const float4*>(sc_tot + (iw ^ 1) * 128)[lane];
+      pt[0] = make_float2(pv.x, pv.y);
+      pt[1] = make_float2(pv.z, pv.w);
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        float2 pa = make_float2(1.f, 1.f);
 #pragma unroll
         for (int J = 0; J < 4; ++J)
-          if (J > blk) z *= bJ[J][j];
-        post[j] = z;
-        float m = 1.f;
+          if (J < blk) pa = mul2(pa, bJ[J][m]);
+        pre[m] = pa;
+      }
+      if (iw == 0) {
+        const float2 g0 = mul2(mul2(bJ[0][0], bJ[1][0]), mul2(bJ[2][0], bJ[3][0]));
+        const float2 g1 = mul2(mul2(bJ[0][1], bJ[1][1]), mul2(bJ[2][1], bJ[3][1]));
+        reinterpret_cast<float4*>(item + IT_GAM)[lane] = make_float4(g0.x, g0.y, g1.x, g1.y);
+      }
+    }
+
+    // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i
+    {
+      float2 run[2];
 #pragma unroll
-        for (int I = 0; I < 4; ++I) {
-          cI[I][j] = (I == blk) ? 1.0f / bJ[blk][j] : m;
-          if (I > blk) m *= bJ[I][j];
+      for (int m = 0; m < 2; ++m) run[m] = upper_half ? pt[m] : make_float2(1.f, 1.f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 qv[2] = {unpack_bf16(qr[i].x), unpack_bf16(qr[i].y)};
+        const float2 kv[2] = {unpack_bf16(kr[i].x), unpack_bf16(kr[i].y)};
+        const float2 iq = splat2(__shfl_sync(0xffffffffu, inv_s, 2 * i));
+        const float2 ik = splat2(__shfl_sync(0xffffffffu, inv_s, 16 + 2 * i));
+        const float2 b = splat2(__shfl_sync(0xffffffffu, beta_l, i));
+        float2 lk[2], lq[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          run[m] = mul2(run[m], a2[i][m]);
+          lk[m] = mul2(kv[m], mul2(run[m], ik));  // khat * e
+          lq[m] = mul2(qv[m], mul2(run[m], iq));  // scale * qhat * e
         }
+        sts64(a_lk + xo[i], bf16x2_of(mul2(lk[0], b)), bf16x2_of(mul2(lk[1], b)));
+        sts64(a_lq + xo[i], bf16x2_of(lq[0]), bf16x2_of(lq[1]));
+        sts64(a_xk + xo[i], bf16x2_of(mul2(lk[0], pre[0])), bf16x2_of(mul2(lk[1], pre[1])));
+        sts64(a_qb + xo[i], bf16x2_of(mul2(lq[0], pre[0])), bf16x2_of(mul2(lq[1], pre[1])));
       }
     }
-    float run[4];
+    // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end; Ktil goes
+    // straight to the item (same swizzled image as a shared-memory MN tile)
+    {
+      float2 post[2], cI[4][2];
+      {
+        float2 bJ[4][2];
+        load_bJ(bJ);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) run[j] = upper_half ? 1.f : pt[j];
-    uint8_t* kt_dst = item + IT_KT + kb * 8192;
+        for (int m = 0; m < 2; ++m) {
+          float2 z = make_float2(1.f, 1.f);
 #pragma unroll
-    for (int i = 7; i >= 0; --i) {
-      const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
-      const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
-      const float ik = __shfl_sync(0xffffffffu, inv_s, 16 + 2 * i);
-      float kf[4];
+          for (int J = 0; J < 4; ++J)
+            if (J > blk) z = mul2(z, bJ[J][m]);
+          post[m] = z;
+          float2 mm = make_float2(1.f, 1.f);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) kf[j] = kv[j] * (run[j] * ik);  // khat * f
-#pragma unroll
-      for (int I = 0; I < 4; ++I) {
-        if (I < blk) continue;
-        sts64(a_r + row_off(I) * 128 + xo[i], bf16x2(kf[0] * cI[I][0], kf[1] * cI[I][1]),
-              bf16x2(kf[2] * cI[I][2], kf[3] * cI[I][3]));
-      }
-      *reinterpret_cast<uint2*>(kt_dst + xo[i]) =
-          make_uint2(bf16x2(kv[0] * (run[0] * post[0]), kv[1] * (run[1] * post[1])),
-                     bf16x2(kv[2] * (run[2] * post[2]), kv[3] * (run[3] * post[3])));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) run[j] *= a[i][j];
-    }
-  }
-  fence_proxy_async();
-  if (__syncthreads_or(*abort_flag)) goto done;
-
-  // ================================================================ MMA AP: [LK; LQ] x R_I^T
-  if (itid == 0) {
-    tc_fence_after();
-#pragma unroll
-    for (int I = 0; I < 4; ++I) {
-      const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = sdesc_sw128(sbase + I_LKQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sbase + I_R + (ks >> 2) * I_RKBLK + row_off(I) * 128 + (ks & 3) * 32, 16, 1024);
-        umma_bf16(tmem + row_off(I), ad, bd, idesc, ks > 0);
-      }
-    }
-    umma_commit(bar + 1);
-  }
-  bounded_wait(bar + 1, 0, abort_flag, p.status);
-  if (__syncthreads_or(*abort_flag)) goto done;
-  tc_fence_after();
-
-  // ================================================================ assemble A (fp32) and P (bf16)
-  {
-    const int R = 32 * quarter + lane;
-    const bool qside = R >= 64;
-    const int r = R & 63;
-    const int Ib = r >> 4;
-    const int q2 = quarter & 1;
-    const bool skip = (ihalf == 1) && (q2 == 0);
-    float d[32];
-    if (!skip) {
-      float d0[32], d1[32];
-      tmem_ld32(tmem + lane_base + row_off(2 * q2) + 32 * ihalf, d0);
-      tmem_ld32(tmem + lane_base + row_off(2 * q2 + 1) + 32 * ihalf, d1);
-      const bool odd = Ib & 1;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) d[j] = odd ? d1[j] : d0[j];
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) d[j] = 0.f;
-    }
-    if (!qside) {
-      float* dst = As + r * AS_LD + 32 * ihalf;
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const int s = 32 * ihalf + j;
-        float4 o;
-        o.x = (s + 0 < r) ? d[j + 0] : 0.f;
-        o.y = (s + 1 < r) ? d[j + 1] : 0.f;
-        o.z = (s + 2 < r) ? d[j + 2] : 0.f;
-        o.w = (s + 3 < r) ? d[j + 3] : 0.f;
-        *reinterpret_cast<float4*>(dst + j) = o;
-      }
-    } else {
-#pragma unroll
-      for (int cch = 0; cch < 4; ++cch) {
-        float v8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int s = 32 * ihalf + 8 * cch + u;
-          v8[u] = (s <= r) ? d[8 * cch + u] : 0.f;
-        }
-        uint4 w;
-        w.x = pack_bf16(v8[0], v8[1]);
-        w.y = pack_bf16(v8[2], v8[3]);
-        w.z = pack_bf16(v8[4], v8[5]);
-        w.w = pack_bf16(v8[6], v8[7]);
-        *reinterpret_cast<uint4*>(sm + I_TP + sw128(64 + r, 4 * ihalf + cch)) = w;
-      }
-    }
-  }
-  sync();
-
-  // ================================================================ solve T = (I + A)^{-1}
-  if (iw < 4 && lane < 16) {
-    const int I = iw, j = lane;
-    const float* ab = As + (16 * I) * AS_LD + 16 * I;
-    float x[16];
-#pragma unroll
-    for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
-    // right-looking substitution: once x[m] is final, fold it into every later row
-#pragma unroll
-    for (int m = 0; m < 15; ++m) {
-      const float xm = x[m];
-#pragma unroll
-      for (int i = m + 1; i < 16; ++i) x[i] = fmaf(-ab[i * AS_LD + m], xm, x[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = (i >= j) ? x[i] : 0.f;
-  }
-  sync();
-  // off-diagonal blocks by distance dd below the diagonal, one warp per block:
-  // T_IJ = -T_II (sum_{K=J}^{I-1} A_IK T_KJ), each 16x16x16 product on mma.sync m16n8k8 tf32
-  // with both operands split hi + lo (three products), i.e. fp32-level accuracy
-#pragma unroll 1
-  for (int dd = 1; dd < 4; ++dd) {
-    if (iw < 4 - dd) {
-      const int bI = dd + iw, bJ2 = iw;
-      const int g = lane >> 2, t = lane & 3;
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      for (int K = bJ2; K < bI; ++K) {
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const float* ab = As + (16 * bI + g) * AS_LD + 16 * K + 8 * ks + t;
-          uint32_t ah[4], al[4];
-          tf32_split(ab[0], ah[0], al[0]);
-          tf32_split(ab[8 * AS_LD], ah[1], al[1]);
-          tf32_split(ab[4], ah[2], al[2]);
-          tf32_split(ab[8 * AS_LD + 4], ah[3], al[3]);
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            const float* tb = Ts + (16 * K + 8 * ks + t) * AS_LD + 16 * bJ2 + 8 * nt + g;
-            uint32_t bh0, bl0, bh1, bl1;
-            tf32_split(tb[0], bh0, bl0);
-            tf32_split(tb[4 * AS_LD], bh1, bl1);
-            mma_tf32(acc[nt], ah, bh0, bh1);
-            mma_tf32(acc[nt], ah, bl0, bl1);
-            mma_tf32(acc[nt], al, bh0, bh1);
+          for (int I = 0; I < 4; ++I) {
+            cI[I][m] = (I == blk) ? make_float2(1.0f / bJ[blk][m].x, 1.0f / bJ[blk][m].y) : mm;
+            if (I > blk) mm = mul2(mm, bJ[I][m]);
           }
         }
       }
-      float* ys = Ys + iw * 256;
+      float2 run[2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        ys[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
-        ys[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
-        ys[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
-        ys[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
+      for (int m = 0; m < 2; ++m) run[m] = upper_half ? make_float2(1.f, 1.f) : pt[m];
+      uint8_t* kt_dst = item + IT_KT + kb * 8192;
+#pragma unroll
+      for (int i = 7; i >= 0; --i) {
+        const float2 kv[2] = {unpack_bf16(kr[i].x), unpack_bf16(kr[i].y)};
+        const float2 ik = splat2(__shfl_sync(0xffffffffu, inv_s, 16 + 2 * i));
+        float2 kf[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) kf[m] = mul2(kv[m], mul2(run[m], ik));  // khat * f
+#pragma unroll
+        for (int I = 0; I < 4; ++I) {
+          if (I < blk) continue;
+          sts64(a_r + row_off(I) * 128 + xo[i], bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
+        }
+        *reinterpret_cast<uint2*>(kt_dst + xo[i]) =
+            make_uint2(bf16x2_of(mul2(kv[0], mul2(run[0], post[0]))), bf16x2_of(mul2(kv[1], mul2(run[1], post[1]))));
+#pragma unroll
+        for (int m = 0; m < 2; ++m) run[m] = mul2(run[m], a2[i][m]);
       }
-      __syncwarp();
-      float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    }
+    fence_proxy_async();
+    if (__syncthreads_or(*abort_flag)) break;
+
+    // ================================================================ MMA AP: [LK; LQ] x R_I^T
+    if (itid == 0) {
+      tc_fence_after();
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        const float* tr = Ts + (16 * bI + g) * AS_LD + 16 * bI + 8 * ks + t;
-        uint32_t ah[4], al[4];
-        tf32_split(tr[0], ah[0], al[0]);
-        tf32_split(tr[8 * AS_LD], ah[1], al[1]);
-        tf32_split(tr[4], ah[2], al[2]);
-        tf32_split(tr[8 * AS_LD + 4], ah[3], al[3]);
+      for (int I = 0; I < 4; ++I) {
+        const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          uint32_t bh0, bl0, bh1, bl1;
-          tf32_split(ys[(8 * ks + t) * 16 + 8 * nt + g], bh0, bl0);
-          tf32_split(ys[(8 * ks + t + 4) * 16 + 8 * nt + g], bh1, bl1);
-          mma_tf32(z[nt], ah, bh0, bh1);
-          mma_tf32(z[nt], ah, bl0, bl1);
-          mma_tf32(z[nt], al, bh0, bh1);
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t ad = sdesc_sw128(sbase + I_LKQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sbase + I_R + (ks >> 2) * I_RKBLK + row_off(I) * 128 + (ks & 3) * 32, 16, 1024);
+          umma_bf16(tmem + row_off(I), ad, bd, idesc, ks > 0);
         }
       }
-      float* to = Ts + (16 * bI) * AS_LD + 16 * bJ2;
+      umma_commit(bar + 1);
+    }
+    if (cta_wait(1, mma_par)) break;
+    tc_fence_after();
+
+    // ================================================================ assemble A (fp32) and P (bf16)
+    {
+      const int R = 32 * quarter + lane;
+      const bool qside = R >= 64;
+      const int r = R & 63;
+      const int Ib = r >> 4;
+      const int q2 = quarter & 1;
+      const bool skip = (ihalf == 1) && (q2 == 0);
+      float d[32];
+      if (!skip) {
+        float d0[32], d1[32];
+        tmem_ld32(tmem + lane_base + row_off(2 * q2) + 32 * ihalf, d0);
+        tmem_ld32(tmem + lane_base + row_off(2 * q2 + 1) + 32 * ihalf, d1);
+        const bool odd = Ib & 1;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        to[g * AS_LD + 8 * nt + 2 * t] = -z[nt][0];
-        to[g * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][1];
-        to[(g + 8) * AS_LD + 8 * nt + 2 * t] = -z[nt][2];
-        to[(g + 8) * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][3];
+        for (int j = 0; j < 32; ++j) d[j] = odd ? d1[j] : d0[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) d[j] = 0.f;
+      }
+      if (!qside) {
+        float* dst = As + r * AS_LD + 32 * ihalf;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const int s = 32 * ihalf + j;
+          float4 o;
+          o.x = (s + 0 < r) ? d[j + 0] : 0.f;
+          o.y = (s + 1 < r) ? d[j + 1] : 0.f;
+          o.z = (s + 2 < r) ? d[j + 2] : 0.f;
+          o.w = (s + 3 < r) ? d[j + 3] : 0.f;
+          *reinterpret_cast<float4*>(dst + j) = o;
+        }
+      } else {
+#pragma unroll
+        for (int cch = 0; cch < 4; ++cch) {
+          float v8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int s = 32 * ihalf + 8 * cch + u;
+            v8[u] = (s <= r) ? d[8 * cch + u] : 0.f;
+          }
+          uint4 w;
+          w.x = pack_bf16(v8[0], v8[1]);
+          w.y = pack_bf16(v8[2], v8[3]);
+          w.z = pack_bf16(v8[4], v8[5]);
+          w.w = pack_bf16(v8[6], v8[7]);
+          *reinterpret_cast<uint4*>(sm + I_TP + sw128(64 + r, 4 * ihalf + cch)) = w;
+        }
       }
     }
     sync();
-  }
-  // T_b = T diag(beta) as a bf16 hi + lo pair, rows 0..63 of TP / TL
-  {
-    const int r = itid >> 2, c16 = itid & 3;
-    const int I = r >> 4;
+
+    // ================================================================ solve T = (I + A)^{-1}
+    if (iw < 4 && lane < 16) {
+      const int I = iw, j = lane;
+      const float* ab = As + (16 * I) * AS_LD + 16 * I;
+      float x[16];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int c0 = 16 * c16 + 8 * hh;
-      uint4 wh, wl;
-      if (c16 > I) {
-        wh = make_uint4(0, 0, 0, 0);
-        wl = wh;
-      } else {
-        const float4 t0v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0);
-        const float4 t1v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0 + 4);
-        const float4 b0 = *reinterpret_cast<const float4*>(sc_beta + c0);
-        const float4 b1 = *reinterpret_cast<const float4*>(sc_beta + c0 + 4);
-        split2(t0v.x * b0.x, t0v.y * b0.y, wh.x, wl.x);
-        split2(t0v.z * b0.z, t0v.w * b0.w, wh.y, wl.y);
-        split2(t1v.x * b1.x, t1v.y * b1.y, wh.z, wl.z);
-        split2(t1v.z * b1.z, t1v.w * b1.w, wh.w, wl.w);
+      for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
+      // right-looking substitution: once x[m] is final, fold it into every later row
+#pragma unroll
+      for (int m = 0; m < 15; ++m) {
+        const float xm = x[m];
+#pragma unroll
+        for (int i = m + 1; i < 16; ++i) x[i] = fmaf(-ab[i * AS_LD + m], xm, x[i]);
       }
-      *reinterpret_cast<uint4*>(sm + I_TP + sw128(r, c0 >> 3)) = wh;
-      *reinterpret_cast<uint4*>(sm + I_TL + sw128(r, c0 >> 3)) = wl;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = (i >= j) ? x[i] : 0.f;
     }
-  }
-  fence_proxy_async();
-  sync();
+    sync();
+    // off-diagonal blocks by distance dd below the diagonal, one warp per block:
+    // T_IJ = -T_II (sum_{K=J}^{I-1} A_IK T_KJ), each 16x16x16 product on mma.sync m16n8k8 tf32
+    // with both operands split hi + lo (three products), i.e. fp32-level accuracy
+#pragma unroll 1
+    for (int dd = 1; dd < 4; ++dd) {
+      if (iw < 4 - dd) {
+        const int bI = dd + iw, bJ2 = iw;
+        const int g = lane >> 2, t = lane & 3;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int K = bJ2; K < bI; ++K) {
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const float* ab = As + (16 * bI + g) * AS_LD + 16 * K + 8 * ks + t;
+            uint32_t ah[4], al[4];
+            tf32_split(ab[0], ah[0], al[0]);
+            tf32_split(ab[8 * AS_LD], ah[1], al[1]);
+            tf32_split(ab[4], ah[2], al[2]);
+            tf32_split(ab[8 * AS_LD + 4], ah[3], al[3]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const float* tb = Ts + (16 * K + 8 * ks + t) * AS_LD + 16 * bJ2 + 8 * nt + g;
+              uint32_t bh0, bl0, bh1, bl1;
+              tf32_split(tb[0], bh0, bl0);
+              tf32_split(tb[4 * AS_LD], bh1, bl1);
+              mma_tf32(acc[nt], ah, bh0, bh1);
+              mma_tf32(acc[nt], ah, bl0, bl1);
+              mma_tf32(acc[nt], al, bh0, bh1);
+            }
+          }
+        }
+        float* ys = Ys + iw * 256;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          ys[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
+          ys[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
+          ys[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
+          ys[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
+        }
+        __syncwarp();
+        float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const float* tr = Ts + (16 * bI + g) * AS_LD + 16 * bI + 8 * ks + t;
+          uint32_t ah[4], al[4];
+          tf32_split(tr[0], ah[0], al[0]);
+          tf32_split(tr[8 * AS_LD], ah[1], al[1]);
+          tf32_split(tr[4], ah[2], al[2]);
+          tf32_split(tr[8 * AS_LD + 4], ah[3], al[3]);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            uint32_t bh0, bl0, bh1, bl1;
+            tf32_split(ys[(8 * ks + t) * 16 + 8 * nt + g], bh0, bl0);
+            tf32_split(ys[(8 * ks + t + 4) * 16 + 8 * nt + g], bh1, bl1);
+            mma_tf32(z[nt], ah, bh0, bh1);
+            mma_tf32(z[nt], ah, bl0, bl1);
+            mma_tf32(z[nt], al, bh0, bh1);
+          }
+        }
+        float* to = Ts + (16 * bI) * AS_LD + 16 * bJ2;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          to[g * AS_LD + 8 * nt + 2 * t] = -z[nt][0];
+          to[g * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][1];
+          to[(g + 8) * AS_LD + 8 * nt + 2 * t] = -z[nt][2];
+          to[(g + 8) * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][3];
+        }
+      }
+      sync();
+    }
+    // T_b = T diag(beta) as a bf16 hi + lo pair, rows 0..63 of TP / TL
+    {
+      const int r = itid >> 2, c16 = itid & 3;
+      const int I = r >> 4;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c0 = 16 * c16 + 8 * hh;
+        uint4 wh, wl;
+        if (c16 > I) {
+          wh = make_uint4(0, 0, 0, 0);
+          wl = wh;
+        } else {
+          const float4 t0v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0);
+          const float4 t1v = *reinterpret_cast<const float4*>(Ts + r * AS_LD + c0 + 4);
+          const float4 b0 = *reinterpret_cast<const float4*>(sc_beta + c0);
+          const float4 b1 = *reinterpret_cast<const float4*>(sc_beta + c0 + 4);
+          split2(t0v.x * b0.x, t0v.y * b0.y, wh.x, wl.x);
+          split2(t0v.z * b0.z, t0v.w * b0.w, wh.y, wl.y);
+          split2(t1v.x * b1.x, t1v.y * b1.y, wh.z, wl.z);
+          split2(t1v.z * b1.z, t1v.w * b1.w, wh.w, wl.w);
+        }
+        *reinterpret_cast<uint4*>(sm + I_TP + sw128(r, c0 >> 3)) = wh;
+        *reinterpret_cast<uint4*>(sm + I_TL + sw128(r, c0 >> 3)) = wl;
+      }
+    }
+    fence_proxy_async();
+    sync();
 
-  // ================================================================ MMA PT: P (T_hi + T_lo)
-  if (itid == 0) {
+    // ================================================================ MMA PT: P (T_hi + T_lo)
+    if (itid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = sdesc_sw128(sbase + I_TP + (ks & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 2048, 8192, 1024);
+        umma_bf16(tmem, ad, bd, idesc, ks > 0);
+      }
+      umma_commit(bar + 1);
+    }
+    if (cta_wait(1, mma_par)) break;
     tc_fence_after();
-    constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint64_t ad = sdesc_sw128(sbase + I_TP + (ks & 3) * 32, 16, 1024);
-      const uint64_t bd = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 2048, 8192, 1024);
-      umma_bf16(tmem, ad, bd, idesc, ks > 0);
-    }
-    umma_commit(bar + 1);
-  }
-  bounded_wait(bar + 1, 1, abort_flag, p.status);
-  if (__syncthreads_or(*abort_flag)) goto done;
-  tc_fence_after();
-  if (quarter >= 2) {
-    const int r = 32 * quarter + lane - 64;
-    float d[32];
-    tmem_ld32(tmem + lane_base + 32 * ihalf, d);
-#pragma unroll
-    for (int cch = 0; cch < 4; ++cch) {
-      uint4 wh, wl;
-      split2(d[8 * cch + 0], d[8 * cch + 1], wh.x, wl.x);
-      split2(d[8 * cch + 2], d[8 * cch + 3], wh.y, wl.y);
-      split2(d[8 * cch + 4], d[8 * cch + 5], wh.z, wl.z);
-      split2(d[8 * cch + 6], d[8 * cch + 7], wh.w, wl.w);
-      *reinterpret_cast<uint4*>(sm + I_TP + sw128(64 + r, 4 * ihalf + cch)) = wh;
-      *reinterpret_cast<uint4*>(sm + I_TL + sw128(64 + r, 4 * ihalf + cch)) = wl;
-    }
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  sync();
-
-  // ================================================================ MMA Xk: [T_b; P T_b] x Khat e^Gamma
-  if (itid == 0) {
-    tc_fence_after();
-    constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint64_t ad = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 32, 16, 1024);
-      const uint64_t bd = sdesc_sw128(sbase + I_XK + (ks & 3) * 2048, 8192, 1024);
-      umma_bf16(tmem, ad, bd, idesc, ks > 0);
-    }
-    umma_commit(bar + 1);
-    // [T_b; P T_b] hi and lo are final: copy both tiles to the item while the MMA runs
-    bulk_store(item + IT_TP, sm + I_TP, 32768);
-    bulk_commit();
-  }
-  bounded_wait(bar + 1, 0, abort_flag, p.status);
-  if (__syncthreads_or(*abort_flag)) goto done;
-  tc_fence_after();
-
-  // ================================================================ [-W; Qtil - P W] -> item
-  {
-    const int R = 32 * quarter + lane;
-    uint8_t* dst = item + IT_WQ + ihalf * 16384 + R * 128;
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
+    if (quarter >= 2) {
+      const int r = 32 * quarter + lane - 64;
       float d[32];
-      tmem_ld32(tmem + lane_base + 64 * ihalf + 32 * part, d);
+      tmem_ld32(tmem + lane_base + 32 * ihalf, d);
 #pragma unroll
       for (int cch = 0; cch < 4; ++cch) {
-        uint4 w;
-        if (R >= 64) {
-          const uint4 qb = *reinterpret_cast<const uint4*>(sm + I_QB + ihalf * 8192 + sw128(R - 64, 4 * part + cch));
-          const float2 a0 = unpack_bf16(qb.x), a1 = unpack_bf16(qb.y), a2 = unpack_bf16(qb.z), a3 = unpack_bf16(qb.w);
-          w.x = pack_bf16(a0.x - d[8 * cch + 0], a0.y - d[8 * cch + 1]);
-          w.y = pack_bf16(a1.x - d[8 * cch + 2], a1.y - d[8 * cch + 3]);
-          w.z = pack_bf16(a2.x - d[8 * cch + 4], a2.y - d[8 * cch + 5]);
-          w.w = pack_bf16(a3.x - d[8 * cch + 6], a3.y - d[8 * cch + 7]);
-        } else {
-          w.x = pack_bf16(-d[8 * cch + 0], -d[8 * cch + 1]);
-          w.y = pack_bf16(-d[8 * cch + 2], -d[8 * cch + 3]);
-          w.z = pack_bf16(-d[8 * cch + 4], -d[8 * cch + 5]);
-          w.w = pack_bf16(-d[8 * cch + 6], -d[8 * cch + 7]);
-        }
-        *reinterpret_cast<uint4*>(dst + ((((uint32_t)(4 * part + cch) ^ (uint32_t)R) & 7u) << 4)) = w;
+        uint4 wh, wl;
+        split2(d[8 * cch + 0], d[8 * cch + 1], wh.x, wl.x);
+        split2(d[8 * cch + 2], d[8 * cch + 3], wh.y, wl.y);
+        split2(d[8 * cch + 4], d[8 * cch + 5], wh.z, wl.z);
+        split2(d[8 * cch + 6], d[8 * cch + 7], wh.w, wl.w);
+        *reinterpret_cast<uint4*>(sm + I_TP + sw128(64 + r, 4 * ihalf + cch)) = wh;
+        *reinterpret_cast<uint4*>(sm + I_TL + sw128(64 + r, 4 * ihalf + cch)) = wl;
       }
     }
+    fence_proxy_async();
+    tc_fence_before();
+    sync();
+
+    // ================================================================ MMA Xk: [T_b; P T_b] x Khat e^Gamma
+    if (itid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(sbase + I_XK + (ks & 3) * 2048, 8192, 1024);
+        umma_bf16(tmem, ad, bd, idesc, ks > 0);
+      }
+      umma_commit(bar + 1);
+      // [T_b; P T_b] hi and lo are final: copy both tiles to the item while the MMA runs
+      bulk_store(item + IT_TP, sm + I_TP, 32768);
+      bulk_commit();
+    }
+    if (cta_wait(1, mma_par)) break;
+    tc_fence_after();
+
+    // ================================================================ [-W; Qtil - P W] -> item
+    {
+      const int R = 32 * quarter + lane;
+      uint8_t* dst = item + IT_WQ + ihalf * 16384 + R * 128;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float d[32];
+        tmem_ld32(tmem + lane_base + 64 * ihalf + 32 * part, d);
+#pragma unroll
+        for (int cch = 0; cch < 4; ++cch) {
+          uint4 w;
+          if (R >= 64) {
+            const uint4 qb = *reinterpret_cast<const uint4*>(sm + I_QB + ihalf * 8192 + sw128(R - 64, 4 * part + cch));
+            const float2 a0 = unpack_bf16(qb.x), a1 = unpack_bf16(qb.y), a2 = unpack_bf16(qb.z), a3 = unpack_bf16(qb.w);
+            w.x = pack_bf16(a0.x - d[8 * cch + 0], a0.y - d[8 * cch + 1]);
+            w.y = pack_bf16(a1.x - d[8 * cch + 2], a1.y - d[8 * cch + 3]);
+            w.z = pack_bf16(a2.x - d[8 * cch + 4], a2.y - d[8 * cch + 5]);
+            w.w = pack_bf16(a3.x - d[8 * cch + 6], a3.y - d[8 * cch + 7]);
+          } else {
+            w.x = pack_bf16(-d[8 * cch + 0], -d[8 * cch + 1]);
+            w.y = pack_bf16(-d[8 * cch + 2], -d[8 * cch + 3]);
+            w.z = pack_bf16(-d[8 * cch + 4], -d[8 * cch + 5]);
+            w.w = pack_bf16(-d[8 * cch + 6], -d[8 * cch + 7]);
+          }
+          *reinterpret_cast<uint4*>(dst + ((((uint32_t)(4 * part + cch) ^ (uint32_t)R) & 7u) << 4)) = w;
+        }
+      }
+    }
+
+    // the next item's TMA overwrites XK / QB (read above and by MMA Xk, which has completed) and its
+    // passes overwrite TP / TL: the bulk copy of this item's TP / TL must have read them
+    tc_fence_before();
+    if (itid == 0) bulk_wait_read<0>();
+    sync();
   }
 
-done:
   tc_fence_before();
   sync();
-  if (itid == 0) bulk_wait_all();
+  if (itid == 0) {
+    // after an abort, copies or MMAs may still be in flight: let them land before leaving
+    if (*abort_flag) {
+      if (raw_pending) mbar_wait(bar + 0, raw_par ^ 1, kWaitLimitNs);
+      umma_commit(bar + 2);
+      mbar_wait(bar + 2, 0, kWaitLimitNs);
+    }
+    bulk_wait_all();
+  }
+  sync();
   if (iw == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kIntraTmemCols);
@@ -1142,6 +1209,7 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
   IntraMaps im;
   RecMaps rm;
   if (!make_token_map(&im.q, p.q, tokens, p.num_heads) || !make_token_map(&im.k, p.k, tokens, p.num_heads) ||
+      !make_token_map(&im.g, p.g, tokens, p.num_heads) ||
       !make_token_map(&rm.v, p.v, tokens, p.num_heads) || !make_token_map(&rm.out, p.out, tokens, p.num_heads))
     return cudaErrorInvalidValue;
   cudaError_t e = set_smem_once(intra_kernel, I_ALLOC, g_intra_attr);
@@ -1152,9 +1220,12 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
   chunk_table_kernel<<<1, 1024, 0, stream>>>(p, const_cast<int32_t*>(args.chunk_off));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t intra_blocks = max_chunks * p.num_heads;
+  // persistent: two CTAs per SM, each walking its share of the items
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int64_t items = max_chunks * p.num_heads;
+  const int64_t intra_blocks = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
   if (intra_blocks > 0) {
-    if (intra_blocks > INT32_MAX) return cudaErrorInvalidValue;
     intra_kernel<<<(unsigned)intra_blocks, kIntraThreads, I_ALLOC, stream>>>(im, args);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
