@@ -3,9 +3,12 @@ K=V=128, bf16 in/out, fp32 state, lower_bound=-5).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-One step = one kda_fwd over the whole workload (the full hot path: prologue, intra-chunk solve,
-chunk recurrence and epilogue in one kernel).  Inputs are seeded synthetic tensors resident in
-HBM; they are 4 GB, far larger than the 126 MB L2, so no flush is needed between steps.  For N > 1
+One step = one kda_fwd over the whole workload: the full hot path in three launches (chunk table,
+the chunk-parallel intra-chunk kernel with the gate, norms, decays, Gram products and solve, and
+the per-(sequence, head) recurrence kernel with the output and final-state epilogues).  Inputs are
+seeded synthetic tensors resident in HBM; they are 4 GB, far larger than the 126 MB L2, so no
+flush is needed between steps.  The roofline block treats the whole call as the kernel: the
+pages' algorithmic bytes of the operation over its measured duration.  For N > 1
 each rank runs an independent replica of the workload (the operator has no cross-GPU step):
 weak scaling, value = all ranks' token-heads / max-over-ranks time.  Prints one JSON line on rank 0.
 
@@ -35,6 +38,7 @@ BYTES_PER_TOKEN_HEAD = 4 * 2 * D + 2 + 2 * D          # q, k, v, g in; raw beta 
 FLOPS_PER_TOKEN_HEAD = 6 * D * D + 2 * CHUNK * D + 3 * 2 * CHUNK * D + 2 * CHUNK * D + CHUNK * CHUNK // 3
 STATE_OUT_BYTES_PER_UNIT = D * D * 4                  # fp32 final state written; initial state is zero (NULL)
 WORKLOAD = "prefill B=1 T=32768 H=96 K=V=128 bf16, lower_bound=-5, zero initial state, final state out"
+LAUNCHES_PER_CALL = 3  # chunk table, intra-chunk kernel, recurrence kernel
 
 
 def algorithmic_bytes(tokens, heads, units):
@@ -147,7 +151,10 @@ def cpu_oracle_sample(target_s=15.0):
         return time.perf_counter() - t0
     m = min(HEADS, cores)
     cal = run(m, 1024)
-    L = int(min(T_TOK, max(1024, 1024 * target_s / max(cal, 1e-3))))
+    # grow the sample to about target_s: first the token count, then the heads (multiples of cores)
+    scale = target_s / max(cal, 1e-3)
+    L = int(min(T_TOK, max(1024, 1024 * scale)))
+    m = int(min(HEADS, max(m, m * scale * 1024 / L // m * m)))
     dt = run(m, L)
     return {"value": m * L / dt / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"heads 0..{m - 1}, tokens 0..{L - 1} of the prefill workload (fp64 C oracle, "
@@ -277,10 +284,10 @@ def main():
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
     flops = FLOPS_PER_TOKEN_HEAD * token_heads
     traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
+    tp = os.path.join(ROOT, "profiles", "kda_fwd_prefill_h96_traffic.json")
+    if os.path.exists(tp) and H == HEADS:
         with open(tp) as f:
-            traffic = json.load(f).get("kda_chunked_prefill_bytes_per_launch")
+            traffic = json.load(f).get("dram_bytes_per_call")
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -294,7 +301,7 @@ def main():
                      "frac": achieved / hbm_peak, "traffic": traffic, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kernel_ms},
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": LAUNCHES_PER_CALL * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
     }

@@ -65,15 +65,18 @@ typedef enum {
 int kda_is_supported(int head_dim, int dtype_is_bf16, float lower_bound);
 
 /* Bytes of device workspace kda_fwd needs for (total tokens T, heads H, sequences N), as
- * get_workspace_size(T, H, N).  Depends only on its arguments; the workspace needs no
- * initialisation by the caller beyond being zero-filled once before first use (it carries the
- * sticky device status word). */
+ * get_workspace_size(T, H, N): a 256-byte header (the sticky device status word), the chunk
+ * table, and 82,944 bytes of intermediates per (chunk, head) for at most (T + 63 N) / 64 chunks
+ * (4.08 GB at T = 32768, H = 96, N = 1).  Depends only on its arguments.  Only the header needs
+ * initialisation by the caller: zero it once before first use. */
 size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
-/* The chunked forward pass (the product path): one fused kernel per call.
+/* The chunked forward pass (the product path): three launches per call (chunk table, the
+ * chunk-parallel intra-chunk kernel, the per-(sequence, head) recurrence kernel).
  *   scale          multiplies the output (o = scale * S^T qhat); it never enters the state.
- *   workspace      device buffer of at least kda_workspace_size(batch*seqlen, H, N) bytes,
- *                  zero-filled once by the caller before its first use.
+ *   workspace      device buffer of at least kda_workspace_size(batch*seqlen, H, N) bytes, its
+ *                  first 256 bytes zeroed once by the caller before its first use; calls that
+ *                  share a workspace must be ordered (the same stream, or events).
  *   initial_state  NULL means a zero state.   final_state  NULL means it is not written.
  *   cu_seqlens     NULL selects batch mode: N = batch sequences of length seqlen each.
  *   num_seqs       N; with cu_seqlens it must be the number of documents, without it batch
@@ -103,8 +106,11 @@ kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, cons
 /* kda_fwd for callers that cannot allocate device memory (for example runtimes that plan every
  * device buffer ahead of time and forbid libraries from calling cudaMalloc, or code that must not
  * trigger cudaMalloc's device-wide synchronisation).  The pages have no counterpart to this entry
- * point.  Same arguments and results as kda_fwd, minus the workspace: it uses a device array that
- * lives in the library (16.6 KB per GPU, held until the process exits) and allocates nothing.
+ * point.  Same arguments as kda_fwd, minus the workspace: it uses a device array that lives in the
+ * library (16.6 KB per GPU, held until the process exits) and allocates nothing.  That array holds
+ * no per-chunk intermediates, so it runs the fused single-kernel path (one CTA per (sequence,
+ * head), every intermediate on chip): results agree with kda_fwd's to rounding, and it is slower
+ * on long prefills.
  *   - At most 4096 (sequence, head) units per call; more returns KDA_ERR_WORKSPACE_TOO_SMALL.
  *   - The first call on a device looks up the array's address on that device; make it before any
  *     stream capture.

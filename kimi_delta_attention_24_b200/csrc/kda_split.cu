@@ -799,7 +799,6 @@ constexpr uint32_t TM_SB = 384;  // S^T as bf16 pairs (A of MMA1), 64 columns
 constexpr uint32_t TM_DH = 448;  // Delta^T hi as bf16 pairs (A of MMA2), 32 columns
 constexpr uint32_t TM_DL = 480;  // Delta^T lo
 constexpr uint32_t kRecTmemCols = 512;
-constexpr int kRecPrefetch = 4;  // chunks the loader pulls into L2 ahead of its stage loads
 
 enum {
   RB_TPV_FULL = 0,   // 2 stages
@@ -867,22 +866,12 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     // ------------------------------------------------------------ loader (lane 0 issues; the
     // whole warp zeroes the v rows past the end of the sequence in the last chunk)
     int armed[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};  // last chunk armed per (TPV, WQ, KT) stage
-    auto prefetch = [&](int c) {
-      if (c >= nch) return;
-      prefetch_l2(item_ptr(c), ITEM_BYTES);
-      const int t0 = (int)(bos + (int64_t)c * C);
-      tma_prefetch_3d(&maps.v, 0, h, t0);
-      tma_prefetch_3d(&maps.v, 64, h, t0);
-    };
-    if (lane == 0)
-      for (int c = 0; c < kRecPrefetch; ++c) prefetch(c);
     for (int c = 0; c < nch; ++c) {
       const int s = c & 1;
       const uint32_t par = ((c >> 1) - 1) & 1;
       const uint8_t* it = item_ptr(c);
       int ok = 1;
       if (lane == 0) {
-        prefetch(c + kRecPrefetch);
         if (c >= 2 && !wait(RB_TPV_EMPTY + s, par)) ok = 0;
         if (ok) {
           armed[0][s] = c;
