@@ -52,8 +52,9 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
   if (sm100::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = sm100::globaltimer_ns();
   for (uint32_t n = 1;; ++n) {
-    if (sm100::mbar_try_wait(bar, parity)) return true;
-    if ((n & 63) == 0) {
+    // sleeps until the phase completes (or 20 us pass), so a waiting thread takes no issue slots
+    if (sm100::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((n & 7) == 0) {
       if (*abort) return false;
       if (sm100::globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort = 1;

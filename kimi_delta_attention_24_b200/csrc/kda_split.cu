@@ -246,6 +246,14 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const uint32_t a_lk = sbase + I_LKQ + kb * 16384, a_lq = a_lk + 64 * 128;
   const uint32_t a_xk = sbase + I_XK + kb * 8192, a_qb = sbase + I_QB + kb * 8192;
   const uint32_t a_r = sbase + I_R + kb * I_RKBLK;
+  // matrix descriptors of the MMA operand tiles (thread 0 issues; k-steps are offsets)
+  const uint64_t d_lkq = sdesc_sw128(sbase + I_LKQ, 16, 1024);   // K-major, 128 rows
+  const uint64_t d_r = sdesc_sw128(sbase + I_R, 16, 1024);       // K-major, 160 rows
+  const uint64_t d_tpk = sdesc_sw128(sbase + I_TP, 16, 1024);    // [T; P] / [T; PT] as K-major A
+  const uint64_t d_tlk = sdesc_sw128(sbase + I_TL, 16, 1024);
+  const uint64_t d_tpm = sdesc_sw128(sbase + I_TP, 8192, 1024);  // T_b hi / lo as MN-major B
+  const uint64_t d_tlm = sdesc_sw128(sbase + I_TL, 8192, 1024);
+  const uint64_t d_xk = sdesc_sw128(sbase + I_XK, 8192, 1024);   // MN-major B
 
   int64_t cur_gc = blockIdx.x / (unsigned)H;
   int cur_h = (int)(blockIdx.x % (unsigned)H);
@@ -482,8 +490,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
         const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t ad = sdesc_sw128(sbase + I_LKQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sbase + I_R + (ks >> 2) * I_RKBLK + row_off(I) * 128 + (ks & 3) * 32, 16, 1024);
+          const uint64_t ad = sdesc_add(d_lkq, (ks >> 2) * 16384 + (ks & 3) * 32);
+          const uint64_t bd = sdesc_add(d_r, (ks >> 2) * I_RKBLK + row_off(I) * 128 + (ks & 3) * 32);
           umma_bf16(tmem + row_off(I), ad, bd, idesc, ks > 0);
         }
       }
@@ -665,8 +673,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = sdesc_sw128(sbase + I_TP + (ks & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 2048, 8192, 1024);
+        const uint64_t ad = sdesc_add(d_tpk, (ks & 3) * 32);
+        const uint64_t bd = sdesc_add(ks < 4 ? d_tpm : d_tlm, (ks & 3) * 2048);
         umma_bf16(tmem, ad, bd, idesc, ks > 0);
       }
       umma_commit(bar + 1);
@@ -698,8 +706,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = sdesc_sw128(sbase + (ks < 4 ? I_TP : I_TL) + (ks & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sbase + I_XK + (ks & 3) * 2048, 8192, 1024);
+        const uint64_t ad = sdesc_add(ks < 4 ? d_tpk : d_tlk, (ks & 3) * 32);
+        const uint64_t bd = sdesc_add(d_xk, (ks & 3) * 2048);
         umma_bf16(tmem, ad, bd, idesc, ks > 0);
       }
       umma_commit(bar + 1);
