@@ -129,7 +129,7 @@ constexpr uint32_t I_TP = 32768;    // after MMA AP: [T_b hi; P -> (P T_b) hi], 
 constexpr uint32_t I_TL = 49152;    //               [T_b lo; (P T_b) lo]
 constexpr uint32_t I_AS = 65536;    //               A fp32 64 x 68
 constexpr uint32_t I_TS = 82944;    //               T fp32 64 x 68
-constexpr uint32_t I_YS = 100352;   //               solve temporaries 3 x 16 x 16 fp32
+constexpr uint32_t I_YS = 100352;   //               solve temporaries 8 x 16 x 8 fp32
 constexpr uint32_t AS_LD = 68;
 constexpr uint32_t I_SC = 106496;   // scalars
 constexpr uint32_t I_TOT = I_SC;            // float[8][128] per-warp alpha products
@@ -139,7 +139,7 @@ constexpr uint32_t I_TMEM = I_SC + 4376;    // allocated TMEM address
 constexpr uint32_t I_ABORT = I_SC + 4380;
 constexpr uint32_t I_SMEM = I_SC + 4480;
 constexpr uint32_t I_ALLOC = I_SMEM + 1024;
-static_assert(I_YS + 3072 <= I_SC, "intra shared-memory map");
+static_assert(I_YS + 4096 <= I_SC, "intra shared-memory map");
 static_assert(2 * (I_ALLOC + 1024) <= 233472, "two intra CTAs per SM");
 constexpr uint32_t kIntraTmemCols = 256;
 
@@ -485,15 +485,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     // ================================================================ MMA AP: [LK; LQ] x R_I^T
     if (itid == 0) {
       tc_fence_after();
+      // the four right operands R_0..R_3 are consecutive rows of one tile: a single N = 160 product
+      constexpr uint32_t idesc = idesc_bf16(128, 160, false, false);
 #pragma unroll
-      for (int I = 0; I < 4; ++I) {
-        const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), false, false);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t ad = sdesc_add(d_lkq, (ks >> 2) * 16384 + (ks & 3) * 32);
-          const uint64_t bd = sdesc_add(d_r, (ks >> 2) * I_RKBLK + row_off(I) * 128 + (ks & 3) * 32);
-          umma_bf16(tmem + row_off(I), ad, bd, idesc, ks > 0);
-        }
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = sdesc_add(d_lkq, (ks >> 2) * 16384 + (ks & 3) * 32);
+        const uint64_t bd = sdesc_add(d_r, (ks >> 2) * I_RKBLK + (ks & 3) * 32);
+        umma_bf16(tmem, ad, bd, idesc, ks > 0);
       }
       umma_commit(bar + 1);
     }
@@ -570,72 +568,68 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       for (int i = 0; i < 16; ++i) Ts[(16 * I + i) * AS_LD + 16 * I + j] = (i >= j) ? x[i] : 0.f;
     }
     sync();
-    // off-diagonal blocks by distance dd below the diagonal, one warp per block:
-    // T_IJ = -T_II (sum_{K=J}^{I-1} A_IK T_KJ), each 16x16x16 product on mma.sync m16n8k8 tf32
-    // with both operands split hi + lo (three products), i.e. fp32-level accuracy
+    // off-diagonal blocks by distance dd below the diagonal: T_IJ = -T_II (sum_{K=J}^{I-1} A_IK T_KJ),
+    // each 16x16x16 product on mma.sync m16n8k8 tf32 with both operands split hi + lo (three
+    // products, fp32-level accuracy).  Warp w takes block J = w / 2 and the 8 columns nt = w % 2
+    // of it; the three partial products accumulate separately so their chains stay short.
 #pragma unroll 1
     for (int dd = 1; dd < 4; ++dd) {
-      if (iw < 4 - dd) {
-        const int bI = dd + iw, bJ2 = iw;
+      const int bJ2 = iw >> 1, nt = iw & 1, bI = bJ2 + dd;
+      if (bI < 4) {
         const int g = lane >> 2, t = lane & 3;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        for (int K = bJ2; K < bI; ++K) {
+        float hh[4] = {0.f, 0.f, 0.f, 0.f}, hl[4] = {0.f, 0.f, 0.f, 0.f}, lh[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const float* ab = As + (16 * bI + g) * AS_LD + 16 * K + 8 * ks + t;
-            uint32_t ah[4], al[4];
-            tf32_split(ab[0], ah[0], al[0]);
-            tf32_split(ab[8 * AS_LD], ah[1], al[1]);
-            tf32_split(ab[4], ah[2], al[2]);
-            tf32_split(ab[8 * AS_LD + 4], ah[3], al[3]);
+        for (int kk = 0; kk < 3; ++kk) {
+          if (kk < dd) {
+            const int K = bJ2 + kk;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            for (int ks = 0; ks < 2; ++ks) {
+              const float* ab = As + (16 * bI + g) * AS_LD + 16 * K + 8 * ks + t;
               const float* tb = Ts + (16 * K + 8 * ks + t) * AS_LD + 16 * bJ2 + 8 * nt + g;
-              uint32_t bh0, bl0, bh1, bl1;
-              tf32_split(tb[0], bh0, bl0);
-              tf32_split(tb[4 * AS_LD], bh1, bl1);
-              mma_tf32(acc[nt], ah, bh0, bh1);
-              mma_tf32(acc[nt], ah, bl0, bl1);
-              mma_tf32(acc[nt], al, bh0, bh1);
+              const float a0 = ab[0], a1 = ab[8 * AS_LD], a2v = ab[4], a3 = ab[8 * AS_LD + 4];
+              const float b0 = tb[0], b1 = tb[4 * AS_LD];
+              uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
+              tf32_split(a0, ah[0], al[0]);
+              tf32_split(a1, ah[1], al[1]);
+              tf32_split(a2v, ah[2], al[2]);
+              tf32_split(a3, ah[3], al[3]);
+              tf32_split(b0, bh0, bl0);
+              tf32_split(b1, bh1, bl1);
+              mma_tf32(hh, ah, bh0, bh1);
+              mma_tf32(hl, ah, bl0, bl1);
+              mma_tf32(lh, al, bh0, bh1);
             }
           }
         }
-        float* ys = Ys + iw * 256;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          ys[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
-          ys[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
-          ys[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
-          ys[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
-        }
+        // Y (16 x 8) through shared memory, then Z = T_II Y
+        float* ys = Ys + iw * 128;
+        ys[g * 8 + 2 * t] = hh[0] + (hl[0] + lh[0]);
+        ys[g * 8 + 2 * t + 1] = hh[1] + (hl[1] + lh[1]);
+        ys[(g + 8) * 8 + 2 * t] = hh[2] + (hl[2] + lh[2]);
+        ys[(g + 8) * 8 + 2 * t + 1] = hh[3] + (hl[3] + lh[3]);
         __syncwarp();
-        float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float zh[4] = {0.f, 0.f, 0.f, 0.f}, zm[4] = {0.f, 0.f, 0.f, 0.f}, zl[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
           const float* tr = Ts + (16 * bI + g) * AS_LD + 16 * bI + 8 * ks + t;
-          uint32_t ah[4], al[4];
-          tf32_split(tr[0], ah[0], al[0]);
-          tf32_split(tr[8 * AS_LD], ah[1], al[1]);
-          tf32_split(tr[4], ah[2], al[2]);
-          tf32_split(tr[8 * AS_LD + 4], ah[3], al[3]);
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            uint32_t bh0, bl0, bh1, bl1;
-            tf32_split(ys[(8 * ks + t) * 16 + 8 * nt + g], bh0, bl0);
-            tf32_split(ys[(8 * ks + t + 4) * 16 + 8 * nt + g], bh1, bl1);
-            mma_tf32(z[nt], ah, bh0, bh1);
-            mma_tf32(z[nt], ah, bl0, bl1);
-            mma_tf32(z[nt], al, bh0, bh1);
-          }
+          const float a0 = tr[0], a1 = tr[8 * AS_LD], a2v = tr[4], a3 = tr[8 * AS_LD + 4];
+          const float b0 = ys[(8 * ks + t) * 8 + g], b1 = ys[(8 * ks + t + 4) * 8 + g];
+          uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
+          tf32_split(a0, ah[0], al[0]);
+          tf32_split(a1, ah[1], al[1]);
+          tf32_split(a2v, ah[2], al[2]);
+          tf32_split(a3, ah[3], al[3]);
+          tf32_split(b0, bh0, bl0);
+          tf32_split(b1, bh1, bl1);
+          mma_tf32(zh, ah, bh0, bh1);
+          mma_tf32(zm, ah, bl0, bl1);
+          mma_tf32(zl, al, bh0, bh1);
         }
-        float* to = Ts + (16 * bI) * AS_LD + 16 * bJ2;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          to[g * AS_LD + 8 * nt + 2 * t] = -z[nt][0];
-          to[g * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][1];
-          to[(g + 8) * AS_LD + 8 * nt + 2 * t] = -z[nt][2];
-          to[(g + 8) * AS_LD + 8 * nt + 2 * t + 1] = -z[nt][3];
-        }
+        float* to = Ts + (16 * bI) * AS_LD + 16 * bJ2 + 8 * nt;
+        to[g * AS_LD + 2 * t] = -(zh[0] + (zm[0] + zl[0]));
+        to[g * AS_LD + 2 * t + 1] = -(zh[1] + (zm[1] + zl[1]));
+        to[(g + 8) * AS_LD + 2 * t] = -(zh[2] + (zm[2] + zl[2]));
+        to[(g + 8) * AS_LD + 2 * t + 1] = -(zh[3] + (zm[3] + zl[3]));
       }
       sync();
     }
