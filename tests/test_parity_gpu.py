@@ -92,6 +92,17 @@ def test_chunk_tails_and_empty_documents(cuda_device):
     np.testing.assert_array_equal(s[5], x.initial_state[5].double().numpy())
 
 
+def test_many_short_documents(cuda_device):
+    """1100 documents of 0..70 tokens: the per-sequence chunk table spans two 1024-wide scan
+    blocks, and many chunks end a document part-way."""
+    rng = np.random.default_rng(31)
+    lens = [int(v) for v in rng.integers(0, 71, size=1100)]
+    x = kda_inputs.make_random("t", lens, 1, seed=31, state_std=0.1)
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    o, s = run_gpu(x, "chunked")
+    check(o, s, o_ref, s_ref, "many documents")
+
+
 @pytest.mark.parametrize("lb", [0.0, -0.5, -2.0])
 def test_lower_bounds(cuda_device, lb):
     x = kda_inputs.make_random("t", [300, 77], 3, seed=22, state_std=0.1, lower_bound=lb)
