@@ -929,6 +929,12 @@ __global__ void __launch_bounds__(kRecThreads, 1)
       constexpr uint32_t idesc_xv = idesc_bf16(128, 128, true, false);   // A MN-major (V), B K-major
       constexpr uint32_t idesc_1 = idesc_bf16(128, 128, false, false);   // A in TMEM, B K-major
       constexpr uint32_t idesc_2 = idesc_bf16(128, 128, false, true);    // A in TMEM, B MN-major
+      // matrix descriptors of stage 0; stage 1 and the k-steps are constant offsets (one thread
+      // issues every MMA, so its per-MMA work is kept to an add)
+      const uint64_t dv0 = sdesc_sw128(sbase + R_TPV + 32768, 8192, 1024);  // V tile: MN-major A
+      const uint64_t dtp0 = sdesc_sw128(sbase + R_TPV, 16, 1024);           // TP / TL: K-major B
+      const uint64_t dwq0 = sdesc_sw128(sbase + R_WQ, 16, 1024);            // WQ: K-major B
+      const uint64_t dkt0 = sdesc_sw128(sbase + R_KT, 8192, 1024);          // Ktil: MN-major B
       // half `part` of MMA Xv into accumulator buffer c % 2: V^T [T_b; P T_b]_{hi / lo}^T
       auto issue_xv = [&](int c, int part) -> bool {
         const int s = c & 1;
@@ -939,13 +945,13 @@ __global__ void __launch_bounds__(kRecThreads, 1)
           // it on every epilogue warp before S(c - 1) arrived, and MMA1(c - 1) waited for S(c - 1)
           tc_fence_after();
         }
-        const uint32_t st = sbase + R_TPV + s * R_TPV_STAGE;
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const uint64_t ad = sdesc_sw128(st + 32768 + k4 * 2048, 8192, 1024);
-          const uint64_t bd = sdesc_sw128(st + 16384 * part + k4 * 32, 16, 1024);
-          umma_bf16(tmem + TM_ACC + 128 * (c & 1), ad, bd, idesc_xv, part + k4 > 0);
-        }
+        const uint64_t dv = dv0 + (uint32_t)s * (R_TPV_STAGE >> 4);
+        const uint64_t dtp = dtp0 + (uint32_t)s * (R_TPV_STAGE >> 4) + (uint32_t)part * (16384 >> 4);
+        const uint32_t acc = tmem + TM_ACC + 128 * (c & 1);
+        umma_bf16(acc, dv, dtp, idesc_xv, part);
+        umma_bf16(acc, dv + (2048 >> 4), dtp + 2, idesc_xv, 1);
+        umma_bf16(acc, dv + (4096 >> 4), dtp + 4, idesc_xv, 1);
+        umma_bf16(acc, dv + (6144 >> 4), dtp + 6, idesc_xv, 1);
         if (part == 1) umma_commit(bar + RB_TPV_EMPTY + s);
         return true;
       };
@@ -957,12 +963,11 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         if (!wait(RB_WQ_FULL + s, par) || !spin(RB_S, c & 1)) break;
         tc_fence_after();
         {
-          const uint32_t wq = sbase + R_WQ + s * 32768;
+          const uint64_t dwq = dwq0 + (uint32_t)s * (32768 >> 4);
+          const uint32_t acc = tmem + TM_ACC + 128 * (c & 1), sb = tmem + TM_SB;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t bd = sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-            umma_bf16_tmem_a(tmem + TM_ACC + 128 * (c & 1), tmem + TM_SB + 8 * ks, bd, idesc_1, 1);
-          }
+          for (int ks = 0; ks < 8; ++ks)
+            umma_bf16_tmem_a(acc, sb + 8 * ks, dwq + (ks >> 2) * (16384 >> 4) + (ks & 3) * 2, idesc_1, 1);
         }
         umma_commit(bar + RB_MMA1);
         umma_commit(bar + RB_WQ_EMPTY + s);
@@ -971,12 +976,11 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         if (!wait(RB_KT_FULL + s, par) || !spin(RB_DELTA, c & 1) || !spin(RB_ST, c & 1)) break;
         tc_fence_after();
         {
-          const uint32_t kt = sbase + R_KT + s * 16384;
+          const uint64_t dkt = dkt0 + (uint32_t)s * (16384 >> 4);
+          const uint32_t st = tmem + TM_ST, dh = tmem + TM_DH, dl = tmem + TM_DL;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t bd = sdesc_sw128(kt + (ks & 3) * 2048, 8192, 1024);
-            umma_bf16_tmem_a(tmem + TM_ST, tmem + (ks < 4 ? TM_DH : TM_DL) + 8 * (ks & 3), bd, idesc_2, 1);
-          }
+          for (int ks = 0; ks < 8; ++ks)
+            umma_bf16_tmem_a(st, (ks < 4 ? dh : dl) + 8 * (ks & 3), dkt + (ks & 3) * (2048 >> 4), idesc_2, 1);
         }
         umma_commit(bar + RB_MMA2);
         umma_commit(bar + RB_KT_EMPTY + s);
@@ -1083,7 +1087,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         const uint32_t acc = tmem + lane_base + TM_ACC + 128 * (c & 1);
         // ---------------------------------------------------- ep1: Delta^T (columns 0..63), O^T (64..127)
         if (cb < 2) wait(RB_TPV_FULL + s, (c >> 1) & 1);  // 1/|k| of this chunk
-        spin(RB_MMA1, c & 1);
+        wait(RB_MMA1, c & 1);
         if (epi_sync_abort()) break;
         tc_fence_after();
         if (cb < 2) {
@@ -1141,7 +1145,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         }
         // ---------------------------------------------------- ep2: state
         const bool last = (c + 1 == nch);
-        spin(RB_MMA2, c & 1);
+        wait(RB_MMA2, c & 1);
         if (!last) wait(RB_TPV_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1);
         if (epi_sync_abort()) break;
         tc_fence_after();
