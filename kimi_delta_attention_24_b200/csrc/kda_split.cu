@@ -269,6 +269,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       tma_load_3d(sm + I_RQ + 8192, &maps.q, bar + 0, 64, h, (int)t0);
       tma_load_3d(sm + I_RK, &maps.k, bar + 0, 0, h, (int)t0);
       tma_load_3d(sm + I_RK + 8192, &maps.k, bar + 0, 64, h, (int)t0);
+    }
+    if (itid == 32) {
       int64_t ngc = cur_gc;
       int nh = cur_h;
       advance(ngc, nh);
@@ -714,8 +716,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 
     // ================================================================ [-W; Qtil - P W] -> item
     {
+      // staged in the (now dead) A / T scratch as the item's byte image, then one bulk copy
       const int R = 32 * quarter + lane;
-      uint8_t* dst = item + IT_WQ + ihalf * 16384 + R * 128;
+      uint8_t* dst = sm + I_AS + ihalf * 16384 + R * 128;
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         float d[32];
@@ -739,6 +742,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
           *reinterpret_cast<uint4*>(dst + ((((uint32_t)(4 * part + cch) ^ (uint32_t)R) & 7u) << 4)) = w;
         }
       }
+    }
+    fence_proxy_async();
+    sync();
+    if (itid == 0) {
+      bulk_store(item + IT_WQ, sm + I_AS, 32768);
+      bulk_commit();
     }
 
     // the next item's TMA overwrites XK / QB (read above and by MMA Xk, which has completed) and its
