@@ -12,18 +12,14 @@
 // and per chunk
 //   Delta = U - W S,   O = Qtil S + P Delta = (Qtil - P W) S + P U,   S <- Diag(e^{Gamma_C}) S + Ktil^T Delta.
 //
-// Everything that does not involve S is independent across chunks, so it runs in one CTA per
-// (chunk, head) spread over every SM (intra_kernel): the gate, the norms, the decays, the Gram
+// Everything that does not involve S is independent across chunks, so it runs chunk-parallel over
+// every SM (intra_kernel, persistent, two CTAs per SM): the gate, the norms, the decays, the Gram
 // products, the solve and the products with T_b.  It leaves one "item" per (chunk, head) in the
-// workspace, stored as the byte image of the shared-memory tiles the recurrence consumes:
-//   [-W; Qtil - P W]   (A operand of MMA1)          [T_b; P T_b] hi and lo   (A operand of MMA Xv)
-//   Ktil (raw k scaled by the decays; A of MMA2)    1/|k_r| per row, e^{Gamma_C} per channel.
-// rec_kernel then walks each (sequence, head) chunk by chunk with the fp32 state in tensor memory:
-//   MMA Xv   [U; P U]  = [T_b; P T_b] (hi + lo) V
-//   MMA1     [Delta; O] = [U; P U] + [-W; Qtil - P W] S_bf16
-//   ep1      O -> out (bf16); Delta / |k| -> bf16 hi + lo in shared memory
-//   MMA2     S_tmem += Ktil^T Delta (hi + lo)      (S_tmem holds e^{Gamma_C} S on entry)
-//   ep2      S -> bf16 copy for the next MMA1; S_tmem <- e^{Gamma_C of the next chunk} S.
+// workspace, stored as the byte image of the shared-memory tiles the recurrence feeds its MMAs:
+//   [-W; Qtil - P W]   (B of MMA1, K-major)          [T_b; P T_b] hi and lo   (B of MMA Xv, K-major)
+//   Ktil (raw k scaled by the decays; B of MMA2)     1/|k_r| per row, e^{Gamma_C} per channel.
+// rec_kernel then walks each (sequence, head) chunk by chunk with the state transposed (S^T) and
+// every state-side operand in tensor memory (its own comment below gives the steps).
 // The hi+lo pairs matter when keys are nearly collinear (T then has entries near -beta that cancel
 // against the diagonal, and a chunk's Delta rows telescope), and Ktil is built from the raw bf16 k
 // with 1/|k| applied to Delta, so that equal keys round identically.
@@ -127,7 +123,8 @@ constexpr uint32_t I_R = 65536;     // R_0..R_3 K tile, 160 rows (B of MMA AP)
 constexpr uint32_t I_RKBLK = 160 * 128;
 constexpr uint32_t I_TP = 32768;    // after MMA AP: [T_b hi; P -> (P T_b) hi], 128 rows x 64
 constexpr uint32_t I_TL = 49152;    //               [T_b lo; (P T_b) lo]
-constexpr uint32_t I_AS = 65536;    //               A fp32 64 x 68
+constexpr uint32_t I_AS = 65536;    //               A fp32 64 x 68 (then, over AS and TS, the
+                                    //               [-W; Qtil - P W] image for the bulk copy)
 constexpr uint32_t I_TS = 82944;    //               T fp32 64 x 68
 constexpr uint32_t I_YS = 100352;   //               solve temporaries 8 x 16 x 8 fp32
 constexpr uint32_t AS_LD = 68;
