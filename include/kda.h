@@ -65,14 +65,24 @@ typedef enum {
 int kda_is_supported(int head_dim, int dtype_is_bf16, float lower_bound);
 
 /* Bytes of device workspace kda_fwd needs for (total tokens T, heads H, sequences N), as
- * get_workspace_size(T, H, N): a 256-byte header (the sticky device status word), the chunk
- * table, and 82,944 bytes of intermediates per (chunk, head) for at most (T + 63 N) / 64 chunks
- * (4.08 GB at T = 32768, H = 96, N = 1).  Depends only on its arguments.  Only the header needs
- * initialisation by the caller: zero it once before first use. */
+ * get_workspace_size(T, H, N): a 256-byte header (the sticky device status word and two item
+ * counters), the chunk table, 82,944 bytes of intermediates per (chunk, head) for at most
+ * (T + 63 N) / 64 chunks, and one 64 KB fp32 state per head for the sequence that is cut between
+ * two stages (4.08 GB at T = 32768, H = 96, N = 1).  Depends only on its arguments.  Only the
+ * header needs initialisation by the caller: zero it once before first use. */
 size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
-/* The chunked forward pass (the product path): three launches per call (chunk table, the
- * chunk-parallel intra-chunk kernel, the per-(sequence, head) recurrence kernel).
+/* Number of kernel launches one kda_fwd call with these sizes enqueues on the current device:
+ * 3 (chunk table, intra-chunk kernel, recurrence kernel), 5 when the call runs in two stages
+ * (N * H below the device's SM count: the chunk range is cut in two and the second intra-chunk
+ * launch overlaps the first recurrence), 2 when there are no chunks, 0 when N * H = 0.
+ * -1 if the device cannot be queried. */
+int kda_fwd_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+
+/* The chunked forward pass (the product path): chunk table, then the chunk-parallel intra-chunk
+ * kernel and the per-(sequence, head) recurrence kernel over one or two ranges of chunks, all on
+ * `stream` (launches after the first intra-chunk one are programmatic dependents of the launch
+ * before them: they may start while it drains and wait in-kernel for what they read).
  *   scale          multiplies the output (o = scale * S^T qhat); it never enters the state.
  *   workspace      device buffer of at least kda_workspace_size(batch*seqlen, H, N) bytes, its
  *                  first 256 bytes zeroed once by the caller before its first use; calls that

@@ -22,8 +22,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["fwd", "fwd_recurrent", "get_workspace_size", "new_workspace", "is_supported", "chunk_kda",
-           "read_device_status", "KDAError", "library_path", "load"]
+__all__ = ["fwd", "fwd_recurrent", "get_workspace_size", "fwd_launch_count", "new_workspace",
+           "is_supported", "chunk_kda", "read_device_status", "KDAError", "library_path", "load"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "lib", "libkda_b200.so")
@@ -60,6 +60,8 @@ def load():
         fn.restype = ctypes.c_int
     lib.kda_workspace_size.argtypes = [i64, i32, i32]
     lib.kda_workspace_size.restype = ctypes.c_size_t
+    lib.kda_fwd_launch_count.argtypes = [i64, i32, i32]
+    lib.kda_fwd_launch_count.restype = ctypes.c_int
     lib.kda_is_supported.argtypes = [ctypes.c_int, ctypes.c_int, f32]
     lib.kda_is_supported.restype = ctypes.c_int
     lib.kda_read_device_status.argtypes = [vp, vp]
@@ -74,9 +76,15 @@ def get_workspace_size(T: int, H: int, N: int) -> int:
     return int(load().kda_workspace_size(int(T), int(H), int(N)))
 
 
+def fwd_launch_count(T: int, H: int, N: int) -> int:
+    """Kernel launches one fwd call over (T tokens, H heads, N sequences) enqueues on the current
+    device (3, or 5 when the chunk range runs in two stages)."""
+    return int(load().kda_fwd_launch_count(int(T), int(H), int(N)))
+
+
 def new_workspace(T: int, H: int, N: int, device) -> torch.Tensor:
-    """A workspace for kda.fwd: uninitialised except for its 256-byte header (the status word),
-    which is zeroed."""
+    """A workspace for kda.fwd: uninitialised except for its 256-byte header (status word and item
+    counters), which is zeroed."""
     ws = torch.empty(get_workspace_size(T, H, N), dtype=torch.uint8, device=device)
     ws[:256].zero_()
     return ws

@@ -104,6 +104,10 @@ size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_s
   return kda::split_workspace_bytes(total_tokens, num_heads, num_seqs);
 }
 
+int kda_fwd_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  return kda::split_launch_count(total_tokens, num_heads, num_seqs);
+}
+
 kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
                      float scale, void* out, void* workspace, size_t workspace_bytes,
                      const float* A_log, const float* dt_bias, float lower_bound,

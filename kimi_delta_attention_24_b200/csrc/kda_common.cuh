@@ -56,6 +56,7 @@ cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream);
 // The split chunked path: chunk table, chunk-parallel intra-chunk kernel, recurrence kernel.
 cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream);
 size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
 // Validates the arguments of a forward call and launches the fused chunked path with `status` as
 // the device status word (used by kda_fwd_static_workspace).

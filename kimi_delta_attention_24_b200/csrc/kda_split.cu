@@ -24,6 +24,12 @@
 // against the diagonal, and a chunk's Delta rows telescope), and Ktil is built from the raw bf16 k
 // with 1/|k| applied to Delta, so that equal keys round identically.
 //
+// Launches, on one stream: chunk_table_kernel (chunk offsets, item counters), then intra and rec
+// over global chunks [0, g_cut), then intra and rec over [g_cut, end).  Each launch after the first
+// intra carries the programmatic-serialization attribute: when the recurrence (one CTA and one SM
+// per (sequence, head)) leaves SMs free, the second intra launch fills them while the first
+// recurrence runs.  g_cut = end (one stage) when there are at least as many units as SMs.
+//
 // Every wait is bounded (kWaitLimitNs of wall time): on expiry the kernel records
 // KDA_ERR_DEVICE_TIMEOUT in the workspace status word and the affected work is skipped.
 #include "kda_device.cuh"
@@ -50,17 +56,25 @@ struct SplitArgs {
   FwdParams p;
   const int32_t* chunk_off;  // [N + 1] first global chunk of each sequence
   uint8_t* items;            // ITEM_BYTES per (global chunk, head), chunk-major
+  int64_t item_begin, item_end;  // intra_kernel: items [item_begin, item_end) (item = chunk * H + head)
+  int64_t g0, g1;                // rec_kernel: global chunks [g0, g1) (g1 = INT64_MAX: to the end)
+  float* boundary;               // [H][128 * 128] S^T of the one sequence cut between two launches
+  unsigned long long* queue;     // intra_kernel: item counter (zeroed by chunk_table_kernel)
 };
+
+constexpr int kQueues = 2;  // item counters in the workspace header, one per intra launch
 
 // ------------------------------------------------------------------------- chunk table
 // chunk_off[n] = sum over m < n of ceil(len_m / C); one block of 1024 threads.
-__global__ void __launch_bounds__(1024) chunk_table_kernel(FwdParams p, int32_t* chunk_off) {
+__global__ void __launch_bounds__(1024) chunk_table_kernel(FwdParams p, int32_t* chunk_off,
+                                                           unsigned long long* queues) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
     carry = 0;
     chunk_off[0] = 0;
+    for (int i = 0; i < kQueues; ++i) queues[i] = 0;
   }
   __syncthreads();
   for (int base = 0; base < p.num_seqs; base += 1024) {
@@ -149,8 +163,9 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
 __device__ __forceinline__ uint32_t bf16x2_of(float2 v) { return bf16x2(v.x, v.y); }
 
-// Persistent: every CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ... in chunk-major order
-// (item = global chunk * H + head), pulling its next item's q, k and g tiles into L2 while it works.
+// Persistent: every CTA takes items [item_begin, item_end) in chunk-major order (item = global
+// chunk * H + head) from a shared counter, pulling its next item's q, k and g tiles into L2 while
+// it works on the current one.
 __global__ void __launch_bounds__(kIntraThreads, 2)
     intra_kernel(const __grid_constant__ IntraMaps maps, const SplitArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -199,7 +214,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     par ^= 1;
     return __syncthreads_or(*abort_flag) != 0;
   };
-  // item = gc * H + h advances by gridDim.x = step_gc * H + step_h per iteration (no division)
   struct Loc {
     int h, len;
     int64_t t0, gc;
@@ -214,15 +228,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     L.t0 = bos + (gc - co[n]) * C;
     L.len = (int)((eos - L.t0) < (int64_t)C ? (eos - L.t0) : (int64_t)C);
     return L;
-  };
-  const int step_gc = (int)(gridDim.x / (unsigned)H), step_h = (int)(gridDim.x % (unsigned)H);
-  auto advance = [&](int64_t& gc, int& h) {
-    gc += step_gc;
-    h += step_h;
-    if (h >= H) {
-      h -= H;
-      ++gc;
-    }
   };
   const int64_t total_gc = co[p.num_seqs];
 
@@ -252,10 +257,16 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const uint64_t d_tlm = sdesc_sw128(sbase + I_TL, 8192, 1024);
   const uint64_t d_xk = sdesc_sw128(sbase + I_XK, 8192, 1024);   // MN-major B
 
-  int64_t cur_gc = blockIdx.x / (unsigned)H;
-  int cur_h = (int)(blockIdx.x % (unsigned)H);
-  for (; cur_gc < total_gc; advance(cur_gc, cur_h)) {
-    const Loc L = locate(cur_gc, cur_h);
+  // Items (gc * H + h, chunk-major) come from a counter, so that a CTA that starts late (on an SM
+  // freed by another kernel) takes fewer.  Thread 32 takes the next item while the current one runs
+  // and publishes it in s_next[j & 1] (double-buffered: it is read after the item's last barrier).
+  __shared__ int64_t s_next[2];
+  const int64_t item_end = args.item_end < total_gc * H ? args.item_end : total_gc * H;
+  if (itid == 0) s_next[1] = args.item_begin + (int64_t)atomicAdd(args.queue, 1ull);
+  __syncthreads();
+  int64_t cur_it = s_next[1];
+  for (uint32_t j = 0; cur_it < item_end; ++j) {
+    const Loc L = locate(cur_it / H, (int)(cur_it % H));
     const int h = L.h, len = L.len;
     const int64_t t0 = L.t0;
     uint8_t* item = args.items + ((size_t)L.gc * H + h) * ITEM_BYTES;
@@ -267,20 +278,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       tma_load_3d(sm + I_RK, &maps.k, bar + 0, 0, h, (int)t0);
       tma_load_3d(sm + I_RK + 8192, &maps.k, bar + 0, 64, h, (int)t0);
     }
-    if (itid == 32) {
-      int64_t ngc = cur_gc;
-      int nh = cur_h;
-      advance(ngc, nh);
-      if (ngc < total_gc) {
-        const Loc N = locate(ngc, nh);
-        tma_prefetch_3d(&maps.q, 0, N.h, (int)N.t0);
-        tma_prefetch_3d(&maps.q, 64, N.h, (int)N.t0);
-        tma_prefetch_3d(&maps.k, 0, N.h, (int)N.t0);
-        tma_prefetch_3d(&maps.k, 64, N.h, (int)N.t0);
-        tma_prefetch_3d(&maps.g, 0, N.h, (int)N.t0);
-        tma_prefetch_3d(&maps.g, 64, N.h, (int)N.t0);
-      }
-    }
+    int64_t nxt = 0;
+    if (itid == 32) nxt = args.item_begin + (int64_t)atomicAdd(args.queue, 1ull);
+
     const float gate_a = __expf(p.A_log[h]);
     const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
     const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
@@ -300,6 +300,19 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 
     // ================================================================ prologue
     if (cta_wait(0, raw_par)) break;
+    if (itid == 32) {
+      // the counter's answer has had the q / k load's time to arrive; warm L2 for the next item
+      s_next[j & 1] = nxt;
+      if (nxt < item_end) {
+        const Loc N = locate(nxt / H, (int)(nxt % H));
+        tma_prefetch_3d(&maps.q, 0, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.q, 64, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.k, 0, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.k, 64, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.g, 0, N.h, (int)N.t0);
+        tma_prefetch_3d(&maps.g, 64, N.h, (int)N.t0);
+      }
+    }
     uint2 qr[8], kr[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -752,7 +765,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     tc_fence_before();
     if (itid == 0) bulk_wait_read<0>();
     sync();
+    cur_it = s_next[j & 1];
   }
+  // no item left for this CTA: a kernel launched after this one as a programmatic dependent may
+  // start its CTAs
+  griddep_launch_dependents();
 
   tc_fence_before();
   sync();
@@ -770,6 +787,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, kIntraTmemCols);
   }
+  // when launched as a programmatic dependent of a recurrence launch, completion of this grid
+  // implies completion of that one (the next recurrence launch reads its boundary states)
+  if (itid == 0) griddep_wait();
 }
 
 // ========================================================================= recurrence kernel
@@ -838,8 +858,21 @@ __global__ void __launch_bounds__(kRecThreads, 1)
   const int n = blockIdx.x / H, h = blockIdx.x % H;
   int64_t bos, eos;
   seq_range(p, n, bos, eos);
-  const int nch = (int)((eos - bos + C - 1) / C);
-  const int64_t item0 = (int64_t)args.chunk_off[n];
+  // launched as a programmatic dependent: let the next launch place its CTAs beside this grid's,
+  // then wait until the items this launch reads are complete
+  // This launch walks the sequence's chunks that fall in global chunks [g0, g1); a sequence cut at
+  // g0 or g1 takes or leaves its state in args.boundary (S^T, [v][k]).
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t co_n = args.chunk_off[n], co_n1 = args.chunk_off[n + 1];
+  const int64_t first = co_n > args.g0 ? co_n : args.g0, lastx = co_n1 < args.g1 ? co_n1 : args.g1;
+  const bool empty_seq = (co_n == co_n1);
+  if (empty_seq ? !(co_n >= args.g0 && co_n < args.g1) : (first >= lastx)) return;  // nothing here
+  const int c_begin = empty_seq ? 0 : (int)(first - co_n), c_end = empty_seq ? 0 : (int)(lastx - co_n);
+  const bool state_in_user = (c_begin == 0), state_out_user = (c_end == (int)(co_n1 - co_n));
+  bos += (int64_t)c_begin * C;
+  const int nch = c_end - c_begin;
+  const int64_t item0 = co_n + c_begin;
   const uint32_t sbase = smem_u32(sm);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + R_BAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + R_ABORT);
@@ -1004,20 +1037,26 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     const int v = 32 * quarter + lane;  // TMEM lane: the state / output column v
     const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
     const uint32_t col0 = 32 * cb;      // this thread's 32 columns (k for the state; tokens in ep1)
-    const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
     // a barrier of all epilogue warps whose answer (has any role aborted?) is the same for all
     auto epi_sync_abort = [&]() { return named_bar_or(kBarEpi, kEpiThreads, *abort_flag != 0); };
     const float* sc_ik = reinterpret_cast<const float*>(sm + R_SC);
     const float* sc_gam = reinterpret_cast<const float*>(sm + R_SC + (IT_GAM - IT_IK));
     const bool out_issuer = (cb == 2 && quarter == 0 && lane == 0);  // first thread of the O warps (warp 12)
 
-    // state columns: S^T[v][k] = S[k][v], k = col0 + j
+    // state columns: S^T[v][k] = S[k][v], k = col0 + j.  A sequence cut between two launches hands
+    // its state over in args.boundary (S^T, slot h); each thread stores only what it loaded itself
+    const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
+    float* const bnd = args.boundary + (size_t)h * D * D;
+    const float* const st_in = state_in_user ? (p.initial_state ? p.initial_state + soff : nullptr) : bnd;
+    float* const st_out = state_out_user ? (p.final_state ? p.final_state + soff : nullptr) : bnd;
+    const bool in_t = state_in_user ? p.state_transposed != 0 : true;
+    const bool out_t = state_out_user ? p.state_transposed != 0 : true;
     auto load_state = [&](float (&x)[32]) {
-      if (!p.initial_state) {
+      if (!st_in) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = 0.f;
-      } else if (p.state_transposed) {
-        const float4* src = reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)v * D + col0);
+      } else if (in_t) {
+        const float4* src = reinterpret_cast<const float4*>(st_in + (size_t)v * D + col0);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float4 t = src[j];
@@ -1028,17 +1067,18 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = p.initial_state[soff + (size_t)(col0 + j) * D + v];
+        for (int j = 0; j < 32; ++j) x[j] = st_in[(size_t)(col0 + j) * D + v];
       }
     };
     auto store_final = [&](const float (&x)[32]) {
-      if (p.state_transposed) {
-        float4* dst = reinterpret_cast<float4*>(p.final_state + soff + (size_t)v * D + col0);
+      if (!st_out) return;
+      if (out_t) {
+        float4* dst = reinterpret_cast<float4*>(st_out + (size_t)v * D + col0);
 #pragma unroll
         for (int j = 0; j < 8; ++j) dst[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) p.final_state[soff + (size_t)(col0 + j) * D + v] = x[j];
+        for (int j = 0; j < 32; ++j) st_out[(size_t)(col0 + j) * D + v] = x[j];
       }
     };
     // bf16 copy (A of MMA1)
@@ -1065,11 +1105,9 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     };
 
     if (nch == 0) {
-      if (p.final_state) {
-        float x[32];
-        load_state(x);
-        store_final(x);
-      }
+      float x[32];
+      load_state(x);
+      store_final(x);
     } else {
       // initial state: bf16 copy for MMA1(0); fp32 copy scaled by e^{Gamma_C}(0) for MMA2(0)
       wait(RB_TPV_FULL, 0);
@@ -1158,7 +1196,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         float x[32];
         tmem_ld32(tmem + lane_base + TM_ST + col0, x);
         if (last) {
-          if (p.final_state) store_final(x);
+          store_final(x);
           break;
         }
         store_state_bf16(x);
@@ -1188,24 +1226,51 @@ bool g_rec_attr[64] = {};
 
 }  // namespace
 
+namespace {
+
+constexpr size_t kQueueOffset = 128;  // two item counters inside the workspace header
+size_t table_bytes(int64_t n) { return ((size_t)(n + 1) * sizeof(int32_t) + 1023) / 1024 * 1024; }
+
+// Upper bound on the global chunks of N sequences holding T tokens in total.
+int64_t chunk_bound(int64_t tokens, int64_t n) { return (tokens + (int64_t)(C - 1) * n) / C; }
+
+// First global chunk of the second stage, or max_chunks when the call runs in one stage.
+// Two stages when the recurrence leaves SMs free (fewer units than SMs): the recurrence over the
+// first g_cut global chunks runs, one SM per unit, while the intra launch of the remaining chunks
+// already fills the other SMs, and all of them once that recurrence is done.  The second stage's
+// share f is sized so that its intra work about fits on the free SMs during the first recurrence:
+// f / (1 - f) = 2 (SMs - units) t_chunk / (H t_item), with t_chunk / t_item ~ 0.135 the measured
+// ratio of one recurrence chunk to one intra item on one CTA.
+int64_t stage_cut(int64_t max_chunks, int64_t units, int heads, int sms) {
+  if (units >= sms || heads <= 0) return max_chunks;
+  const double x = 0.27 * (double)(sms - units) / (double)heads;
+  const int64_t g_cut = max_chunks - (int64_t)((double)max_chunks * x / (1.0 + x));
+  return (g_cut <= 0 || g_cut >= max_chunks) ? max_chunks : g_cut;
+}
+
+}  // namespace
+
 size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
   const int64_t n = num_seqs > 0 ? num_seqs : 0;
   const int64_t t = total_tokens > 0 ? total_tokens : 0;
-  const int64_t max_chunks = (t + (int64_t)(C - 1) * n) / C;
-  const size_t table = ((size_t)(n + 1) * sizeof(int32_t) + 1023) / 1024 * 1024;
-  return kWorkspaceHeader + table + (size_t)max_chunks * (size_t)(num_heads > 0 ? num_heads : 0) * ITEM_BYTES;
+  const int64_t hh = num_heads > 0 ? num_heads : 0;
+  const int64_t max_chunks = chunk_bound(t, n);
+  return kWorkspaceHeader + table_bytes(n) + (size_t)max_chunks * (size_t)hh * ITEM_BYTES +
+         (size_t)hh * D * D * sizeof(float);
 }
 
 cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream) {
   const int64_t units = (int64_t)p.num_seqs * p.num_heads;
   if (units == 0) return cudaSuccess;
   const int64_t tokens = p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs;
-  const int64_t max_chunks = (tokens + (int64_t)(C - 1) * p.num_seqs) / C;
+  const int64_t max_chunks = chunk_bound(tokens, p.num_seqs);
+  const int64_t items = max_chunks * p.num_heads;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  SplitArgs args;
+  SplitArgs args{};
   args.p = p;
   args.chunk_off = reinterpret_cast<int32_t*>(ws + kWorkspaceHeader);
-  args.items = ws + kWorkspaceHeader + ((size_t)(p.num_seqs + 1) * sizeof(int32_t) + 1023) / 1024 * 1024;
+  args.items = ws + kWorkspaceHeader + table_bytes(p.num_seqs);
+  args.boundary = reinterpret_cast<float*>(args.items + (size_t)items * ITEM_BYTES);
 
   IntraMaps im;
   RecMaps rm;
@@ -1217,22 +1282,65 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
   if (e != cudaSuccess) return e;
   e = set_smem_once(rec_kernel, R_ALLOC, g_rec_attr);
   if (e != cudaSuccess) return e;
-
-  chunk_table_kernel<<<1, 1024, 0, stream>>>(p, const_cast<int32_t*>(args.chunk_off));
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // persistent: two CTAs per SM, each walking its share of the items
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
-  const int64_t items = max_chunks * p.num_heads;
-  const int64_t intra_blocks = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
-  if (intra_blocks > 0) {
-    intra_kernel<<<(unsigned)intra_blocks, kIntraThreads, I_ALLOC, stream>>>(im, args);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+
+  unsigned long long* queues = reinterpret_cast<unsigned long long*>(ws + kQueueOffset);
+  // a launch with the programmatic-serialization attribute may start its CTAs once every CTA of
+  // the previous launch in the stream has signalled or exited; the kernels wait (griddepcontrol)
+  // for what they read
+  auto launch = [&](auto kernel, int64_t grid, int threads, uint32_t smem, bool dependent, auto maps,
+                    const SplitArgs& a) -> cudaError_t {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = dependent ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, maps, a);
+  };
+  auto intra = [&](int64_t b, int64_t en, int q, bool dependent) -> cudaError_t {
+    if (en <= b) return cudaSuccess;
+    SplitArgs a = args;
+    a.item_begin = b;
+    a.item_end = en;
+    a.queue = queues + q;
+    const int64_t grid = en - b < 2 * (int64_t)sms ? en - b : 2 * (int64_t)sms;
+    return launch(intra_kernel, grid, kIntraThreads, I_ALLOC, dependent, im, a);
+  };
+  auto rec = [&](int64_t g0, int64_t g1) -> cudaError_t {
+    SplitArgs a = args;
+    a.g0 = g0;
+    a.g1 = g1;
+    return launch(rec_kernel, units, kRecThreads, R_ALLOC, true, rm, a);
+  };
+
+  chunk_table_kernel<<<1, 1024, 0, stream>>>(p, const_cast<int32_t*>(args.chunk_off), queues);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // only the sequence holding chunk g_cut is cut; it hands its state over in args.boundary
+  const int64_t g_cut = stage_cut(max_chunks, units, p.num_heads, sms);
+  if (g_cut >= max_chunks) {
+    if ((e = intra(0, items, 0, false)) != cudaSuccess) return e;
+    return rec(0, INT64_MAX);
   }
-  rec_kernel<<<(unsigned)units, kRecThreads, R_ALLOC, stream>>>(rm, args);
-  return cudaGetLastError();
+  if ((e = intra(0, g_cut * p.num_heads, 0, false)) != cudaSuccess) return e;
+  if ((e = rec(0, g_cut)) != cudaSuccess) return e;
+  if ((e = intra(g_cut * p.num_heads, items, 1, true)) != cudaSuccess) return e;
+  return rec(g_cut, INT64_MAX);
+}
+
+int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  const int64_t units = (int64_t)(num_seqs > 0 ? num_seqs : 0) * (num_heads > 0 ? num_heads : 0);
+  if (units == 0) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return -1;
+  const int64_t max_chunks = chunk_bound(total_tokens > 0 ? total_tokens : 0, num_seqs);
+  if (stage_cut(max_chunks, units, num_heads, sms) < max_chunks) return 5;
+  return max_chunks > 0 ? 3 : 2;
 }
 
 }  // namespace kda

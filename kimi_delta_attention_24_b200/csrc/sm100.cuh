@@ -70,6 +70,14 @@ __device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
 __device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Programmatic dependent launch.  launch_dependents: this CTA lets the next launch of the stream
+// that carries the programmatic-serialization attribute place its CTAs (they start once every CTA of
+// this grid has signalled or exited).  wait: blocks until the grids this one depends on have
+// completed and their memory is visible; returns at once in a grid launched without the attribute.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Named barrier that also ORs a predicate over the participating threads: every thread gets the
 // same answer.
 __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t count, bool pred) {

@@ -71,6 +71,8 @@ def test_prefill_sampled_heads(cuda_device, impl):
     """The 32K x 96-head prefill, in the bench's launch configuration; the oracle recomputes a
     sample of heads over the whole sequence."""
     x = kda_inputs.make_workload("prefill", device=cuda_device)
+    if impl == "chunked":
+        assert kda.fwd_launch_count(x.total_tokens, x.num_heads, x.num_seqs) == 5  # two stages
     o, s = run_gpu(x, impl)
     heads = [0, 41, 95]
     sl = lambda t: t[:, :, heads].contiguous().cpu()
@@ -90,6 +92,20 @@ def test_chunk_tails_and_empty_documents(cuda_device):
         check(o, s, o_ref, s_ref, f"tails/{impl}")
     # zero-length documents hand their initial state through
     np.testing.assert_array_equal(s[5], x.initial_state[5].double().numpy())
+
+
+@pytest.mark.parametrize("opt", ["plain", "transposed", "no_final", "alias"])
+def test_two_stage_schedule(cuda_device, opt):
+    """N * H below the SM count: the chunk range runs in two stages (five launches) and the
+    document holding the cut hands its state from the first recurrence launch to the second
+    through the workspace; empty documents sit on both sides of the cut."""
+    lens = [1000, 0, 2048, 77, 1, 3000, 0]
+    assert kda.fwd_launch_count(sum(lens), 4, len(lens)) == 5
+    x = kda_inputs.make_random("t", lens, 4, seed=32, state_std=0.1,
+                               output_final_state=opt != "no_final")
+    o_ref, s_ref = oracle.fwd_inputs(x, state_transposed=opt == "transposed")
+    o, s = run_gpu(x, "chunked", state_transposed=opt == "transposed", alias=opt == "alias")
+    check(o, s, o_ref, s_ref, f"two stages/{opt}")
 
 
 def test_many_short_documents(cuda_device):
