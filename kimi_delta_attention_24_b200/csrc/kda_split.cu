@@ -241,9 +241,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
   const float lb2 = p.lower_bound * kLog2e;
   // shared-memory byte offset of this thread's 8 bytes of row 8 iw + i inside a 128-byte-row tile
-  uint32_t xo[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) xo[i] = (uint32_t)((8 * iw + i) * 128) + (((lane_chunk ^ i) & 7u) << 4) + lane_sub;
+  const uint32_t xo_base = (uint32_t)(iw * 1024) + lane_sub, xo_l = lane_chunk << 4;
+#define xo(i) (xo_base + (uint32_t)((i) * 128) + (xo_l ^ (uint32_t)((i) << 4)))
   const uint32_t a_rq = sbase + I_RQ + kb * 8192, a_rk = sbase + I_RK + kb * 8192;
   const uint32_t a_lk = sbase + I_LKQ + kb * 16384, a_lq = a_lk + 64 * 128;
   const uint32_t a_xk = sbase + I_XK + kb * 8192, a_qb = sbase + I_QB + kb * 8192;
@@ -259,14 +258,19 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 
   // Items (gc * H + h, chunk-major) come from a counter, so that a CTA that starts late (on an SM
   // freed by another kernel) takes fewer.  Thread 32 takes the next item while the current one runs
-  // and publishes it in s_next[j & 1] (double-buffered: it is read after the item's last barrier).
-  __shared__ int64_t s_next[2];
+  // and publishes it with its chunk in s_next[j & 1] (double-buffered: read after the item's last
+  // barrier), so that the division by H is done once per item.
+  __shared__ int64_t s_next[2][2];  // {item, global chunk}
   const int64_t item_end = args.item_end < total_gc * H ? args.item_end : total_gc * H;
-  if (itid == 0) s_next[1] = args.item_begin + (int64_t)atomicAdd(args.queue, 1ull);
+  if (itid == 0) {
+    const int64_t it = args.item_begin + (int64_t)atomicAdd(args.queue, 1ull);
+    s_next[1][0] = it;
+    s_next[1][1] = it / H;
+  }
   __syncthreads();
-  int64_t cur_it = s_next[1];
+  int64_t cur_it = s_next[1][0], cur_gc = s_next[1][1];
   for (uint32_t j = 0; cur_it < item_end; ++j) {
-    const Loc L = locate(cur_it / H, (int)(cur_it % H));
+    const Loc L = locate(cur_gc, (int)(cur_it - cur_gc * H));
     const int h = L.h, len = L.len;
     const int64_t t0 = L.t0;
     uint8_t* item = args.items + ((size_t)L.gc * H + h) * ITEM_BYTES;
@@ -302,9 +306,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     if (cta_wait(0, raw_par)) break;
     if (itid == 32) {
       // the counter's answer has had the q / k load's time to arrive; warm L2 for the next item
-      s_next[j & 1] = nxt;
+      const int64_t ngc = nxt / H;
+      s_next[j & 1][0] = nxt;
+      s_next[j & 1][1] = ngc;
       if (nxt < item_end) {
-        const Loc N = locate(nxt / H, (int)(nxt % H));
+        const Loc N = locate(ngc, (int)(nxt - ngc * H));
         tma_prefetch_3d(&maps.q, 0, N.h, (int)N.t0);
         tma_prefetch_3d(&maps.q, 64, N.h, (int)N.t0);
         tma_prefetch_3d(&maps.k, 0, N.h, (int)N.t0);
@@ -317,8 +323,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const bool valid = 8 * iw + i < len;
-      qr[i] = valid ? lds64(a_rq + xo[i]) : make_uint2(0, 0);
-      kr[i] = valid ? lds64(a_rk + xo[i]) : make_uint2(0, 0);
+      qr[i] = valid ? lds64(a_rq + xo(i)) : make_uint2(0, 0);
+      kr[i] = valid ? lds64(a_rk + xo(i)) : make_uint2(0, 0);
     }
     float2 a2[8][2];  // alpha of channels (4 lane, +1), (4 lane + 2, +3)
     float ssq[8], ssk[8];
@@ -441,10 +447,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
           lk[m] = mul2(kv[m], mul2(run[m], ik));  // khat * e
           lq[m] = mul2(qv[m], mul2(run[m], iq));  // scale * qhat * e
         }
-        sts64(a_lk + xo[i], bf16x2_of(mul2(lk[0], b)), bf16x2_of(mul2(lk[1], b)));
-        sts64(a_lq + xo[i], bf16x2_of(lq[0]), bf16x2_of(lq[1]));
-        sts64(a_xk + xo[i], bf16x2_of(mul2(lk[0], pre[0])), bf16x2_of(mul2(lk[1], pre[1])));
-        sts64(a_qb + xo[i], bf16x2_of(mul2(lq[0], pre[0])), bf16x2_of(mul2(lq[1], pre[1])));
+        sts64(a_lk + xo(i), bf16x2_of(mul2(lk[0], b)), bf16x2_of(mul2(lk[1], b)));
+        sts64(a_lq + xo(i), bf16x2_of(lq[0]), bf16x2_of(lq[1]));
+        sts64(a_xk + xo(i), bf16x2_of(mul2(lk[0], pre[0])), bf16x2_of(mul2(lk[1], pre[1])));
+        sts64(a_qb + xo(i), bf16x2_of(mul2(lq[0], pre[0])), bf16x2_of(mul2(lq[1], pre[1])));
       }
     }
     // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end; Ktil goes
@@ -483,9 +489,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 #pragma unroll
         for (int I = 0; I < 4; ++I) {
           if (I < blk) continue;
-          sts64(a_r + row_off(I) * 128 + xo[i], bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
+          sts64(a_r + row_off(I) * 128 + xo(i), bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
         }
-        *reinterpret_cast<uint2*>(kt_dst + xo[i]) =
+        *reinterpret_cast<uint2*>(kt_dst + xo(i)) =
             make_uint2(bf16x2_of(mul2(kv[0], mul2(run[0], post[0]))), bf16x2_of(mul2(kv[1], mul2(run[1], post[1]))));
 #pragma unroll
         for (int m = 0; m < 2; ++m) run[m] = mul2(run[m], a2[i][m]);
@@ -765,7 +771,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     tc_fence_before();
     if (itid == 0) bulk_wait_read<0>();
     sync();
-    cur_it = s_next[j & 1];
+    cur_it = s_next[j & 1][0];
+    cur_gc = s_next[j & 1][1];
   }
   // no item left for this CTA: a kernel launched after this one as a programmatic dependent may
   // start its CTAs
