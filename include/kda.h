@@ -34,7 +34,11 @@
  * Errors.  Argument problems are found on the host before anything is launched and nothing is
  * written.  A launch failure returns KDA_ERR_CUDA.  The chunked kernel bounds every wait it
  * performs; if a bound is exceeded it records KDA_ERR_DEVICE_TIMEOUT in the workspace status
- * word and the affected work is skipped — read it with kda_read_device_status.
+ * word and the affected work is skipped — read it with kda_read_device_status.  The contents of
+ * cu_seqlens live on the device, so they are checked there: unless 0 = cu[0] <= cu[1] <= ... <=
+ * cu[N] = seqlen, the kernels record KDA_ERR_INVALID_ARGUMENT in the status word, never read or
+ * write outside the T tokens, and kda_fwd treats every document as empty (out is not written,
+ * final_state receives initial_state).
  */
 #ifndef KDA_B200_H_
 #define KDA_B200_H_
@@ -136,8 +140,17 @@ kda_status_t kda_fwd_static_workspace(const void* q, const void* k, const void* 
                                       kda_stream_t stream);
 
 /* Synchronises `stream`, reads the workspace's sticky status word, clears it, and returns
- * KDA_OK or the recorded device error (KDA_ERR_DEVICE_TIMEOUT).  KDA_ERR_CUDA if the copy fails. */
+ * KDA_OK or the recorded device error: KDA_ERR_DEVICE_TIMEOUT (a bounded wait ran out; reported
+ * first when both are recorded) or KDA_ERR_INVALID_ARGUMENT (cu_seqlens out of order).
+ * KDA_ERR_CUDA if the copy fails. */
 kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream);
+
+/* Self-test of the device time-out path.  Enqueues one CTA that waits, with the forward kernels'
+ * bounded wait, on a barrier phase that nothing completes; after limit_us microseconds
+ * (1 .. 1,000,000) the wait gives up and records KDA_ERR_DEVICE_TIMEOUT in the workspace status
+ * word, which kda_read_device_status then returns.  Nothing faults or hangs and the stream stays
+ * usable.  KDA_ERR_INVALID_ARGUMENT for a null or misaligned workspace or a limit out of range. */
+kda_status_t kda_selftest_wait_timeout(void* workspace, uint32_t limit_us, kda_stream_t stream);
 
 /* A static, human-readable name for a status code. */
 const char* kda_status_string(kda_status_t status);

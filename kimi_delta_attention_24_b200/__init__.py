@@ -23,7 +23,8 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["fwd", "fwd_recurrent", "get_workspace_size", "fwd_launch_count", "new_workspace",
-           "is_supported", "chunk_kda", "read_device_status", "KDAError", "library_path", "load"]
+           "is_supported", "chunk_kda", "read_device_status", "selftest_wait_timeout", "KDAError",
+           "library_path", "load"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "lib", "libkda_b200.so")
@@ -62,6 +63,8 @@ def load():
     lib.kda_workspace_size.restype = ctypes.c_size_t
     lib.kda_fwd_launch_count.argtypes = [i64, i32, i32]
     lib.kda_fwd_launch_count.restype = ctypes.c_int
+    lib.kda_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
+    lib.kda_selftest_wait_timeout.restype = ctypes.c_int
     lib.kda_is_supported.argtypes = [ctypes.c_int, ctypes.c_int, f32]
     lib.kda_is_supported.restype = ctypes.c_int
     lib.kda_read_device_status.argtypes = [vp, vp]
@@ -159,6 +162,17 @@ def read_device_status(workspace: torch.Tensor, stream=None) -> int:
         stream = torch.cuda.current_stream(workspace.device).cuda_stream
     with torch.cuda.device(workspace.device):
         return int(load().kda_read_device_status(_ptr(workspace), ctypes.c_void_p(stream)))
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_us: int = 2000, stream=None) -> None:
+    """Enqueues the device time-out self-test: a bounded wait on a barrier nothing completes,
+    which records KDA_ERR_DEVICE_TIMEOUT in the workspace status word after ``limit_us``."""
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device).cuda_stream
+    with torch.cuda.device(workspace.device):
+        st = int(load().kda_selftest_wait_timeout(_ptr(workspace), int(limit_us), ctypes.c_void_p(stream)))
+    if st != 0:
+        raise KDAError(st, "kda_selftest_wait_timeout")
 
 
 def chunk_kda(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=False,

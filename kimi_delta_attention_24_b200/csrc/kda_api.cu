@@ -164,7 +164,17 @@ kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream) {
     if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return KDA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
   }
-  return (word & kda::kStatusTimeout) ? KDA_ERR_DEVICE_TIMEOUT : KDA_OK;
+  if (word & kda::kStatusTimeout) return KDA_ERR_DEVICE_TIMEOUT;
+  return (word & kda::kStatusBadSeqlens) ? KDA_ERR_INVALID_ARGUMENT : KDA_OK;
+}
+
+kda_status_t kda_selftest_wait_timeout(void* workspace, uint32_t limit_us, kda_stream_t stream) {
+  if (!workspace || !aligned(workspace, 256) || limit_us == 0 || limit_us > 1000000u)
+    return KDA_ERR_INVALID_ARGUMENT;
+  return kda::launch_wait_timeout(static_cast<uint32_t*>(workspace), (uint64_t)limit_us * 1000u,
+                                  reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
 }
 
 const char* kda_status_string(kda_status_t status) {

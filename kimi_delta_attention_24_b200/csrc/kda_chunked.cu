@@ -946,6 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t bos, eos;
   seq_range(p, n, bos, eos);
   const int nchunks = (int)((eos - bos + C - 1) / C);
+  if (tid == 0 && h == 0 && p.status && !seq_entries_ok(p, n)) atomicOr(p.status, kStatusBadSeqlens);
 
   if (tid == 0) {
     for (int b = 0; b < B_COUNT; ++b) mbar_init(S_.bar + b, 1);

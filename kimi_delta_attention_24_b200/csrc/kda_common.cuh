@@ -14,6 +14,7 @@ constexpr float kL2Eps = 1e-6f;      // inside the square root of the q/k L2 nor
 
 // Device status word (first 4 bytes of the workspace), sticky until read by the host.
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBadSeqlens = 2u;  // cu_seqlens not ordered as 0 = cu[0] <= ... <= cu[N] = T
 constexpr size_t kWorkspaceHeader = 256;  // status word + padding; the rest is per-unit tables
 
 // Arguments of one forward call, after host-side validation.
@@ -38,15 +39,26 @@ struct FwdParams {
   uint32_t* status;            // workspace status word, may be null (recurrent path)
 };
 
-// Token range [bos, eos) of sequence n.
+// Token range [bos, eos) of sequence n, clamped to the call's T tokens so that a malformed
+// cu_seqlens (which the host cannot read without a sync) never sends a kernel outside the token
+// tensors; the kernels report it through kStatusBadSeqlens.
 __device__ __forceinline__ void seq_range(const FwdParams& p, int n, int64_t& bos, int64_t& eos) {
   if (p.cu_seqlens) {
-    bos = p.cu_seqlens[n];
-    eos = p.cu_seqlens[n + 1];
+    const int64_t b = p.cu_seqlens[n], e = p.cu_seqlens[n + 1];
+    bos = b < 0 ? 0 : (b > p.seqlen ? p.seqlen : b);
+    eos = e < bos ? bos : (e > p.seqlen ? p.seqlen : e);
   } else {
     bos = (int64_t)n * p.seqlen;
     eos = bos + p.seqlen;
   }
+}
+
+// Whether sequence n's entries of cu_seqlens are in order: cu[n] <= cu[n + 1], cu[0] = 0 and
+// cu[N] = T.  Together over all n they say that the documents tile the T tokens.
+__device__ __forceinline__ bool seq_entries_ok(const FwdParams& p, int n) {
+  if (!p.cu_seqlens) return true;
+  const int64_t b = p.cu_seqlens[n], e = p.cu_seqlens[n + 1];
+  return b <= e && (n > 0 || b == 0) && (n + 1 < p.num_seqs || e == p.seqlen);
 }
 
 // Launchers (defined in the kernel translation units).  Return the launch's cudaError_t.
@@ -57,6 +69,8 @@ cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream);
 size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+// One CTA whose bounded wait on a never-completed phase runs out after limit_ns (self-test).
+cudaError_t launch_wait_timeout(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
 
 // Validates the arguments of a forward call and launches the fused chunked path with `status` as
 // the device status word (used by kda_fwd_static_workspace).

@@ -48,7 +48,7 @@ __host__ __device__ constexpr uint32_t row_off(int I) { return 8u * I * (I + 1);
 // Bounded wait on a phase.  Returns false on time-out (after raising *abort and the status word)
 // or once *abort is up.
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                             uint32_t* status) {
+                                             uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
   if (sm100::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = sm100::globaltimer_ns();
   for (uint32_t n = 1;; ++n) {
@@ -56,7 +56,7 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
     if (sm100::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if ((n & 7) == 0) {
       if (*abort) return false;
-      if (sm100::globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (sm100::globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         if (status) atomicOr(status, kStatusTimeout);
         return false;

@@ -65,7 +65,9 @@ struct SplitArgs {
 constexpr int kQueues = 2;  // item counters in the workspace header, one per intra launch
 
 // ------------------------------------------------------------------------- chunk table
-// chunk_off[n] = sum over m < n of ceil(len_m / C); one block of 1024 threads.
+// chunk_off[n] = sum over m < n of ceil(len_m / C); one block of 1024 threads.  A cu_seqlens that
+// does not tile the T tokens in order gives every sequence zero chunks (so no later kernel reads a
+// token or writes an output) and raises kStatusBadSeqlens; the final states are then the initial ones.
 __global__ void __launch_bounds__(1024) chunk_table_kernel(FwdParams p, int32_t* chunk_off,
                                                            unsigned long long* queues) {
   __shared__ int32_t warp_tot[32];
@@ -76,7 +78,13 @@ __global__ void __launch_bounds__(1024) chunk_table_kernel(FwdParams p, int32_t*
     chunk_off[0] = 0;
     for (int i = 0; i < kQueues; ++i) queues[i] = 0;
   }
-  __syncthreads();
+  bool bad = false;
+  for (int n = tid; n < p.num_seqs; n += 1024) bad |= !seq_entries_ok(p, n);
+  if (__syncthreads_or(bad)) {
+    for (int n = tid; n <= p.num_seqs; n += 1024) chunk_off[n] = 0;
+    if (tid == 0 && p.status) atomicOr(p.status, kStatusBadSeqlens);
+    return;
+  }
   for (int base = 0; base < p.num_seqs; base += 1024) {
     const int n = base + tid;
     int32_t cnt = 0;
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const float lb2 = p.lower_bound * kLog2e;
   // shared-memory byte offset of this thread's 8 bytes of row 8 iw + i inside a 128-byte-row tile
   const uint32_t xo_base = (uint32_t)(iw * 1024) + lane_sub, xo_l = lane_chunk << 4;
-#define xo(i) (xo_base + (uint32_t)((i) * 128) + (xo_l ^ (uint32_t)((i) << 4)))
+  auto xo = [&](int i) { return xo_base + (uint32_t)(i * 128) + (xo_l ^ (uint32_t)(i << 4)); };
   const uint32_t a_rq = sbase + I_RQ + kb * 8192, a_rk = sbase + I_RK + kb * 8192;
   const uint32_t a_lk = sbase + I_LKQ + kb * 16384, a_lq = a_lk + 64 * 128;
   const uint32_t a_xk = sbase + I_XK + kb * 8192, a_qb = sbase + I_QB + kb * 8192;
@@ -815,7 +823,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 // and ep2 run.
 constexpr int kRecThreads = 640;
 constexpr int kEpiThreads = 512;
-constexpr uint32_t kBarEpi = 1, kBarDelta = 2, kBarOut = 3, kBarOutGo = 4;
+constexpr uint32_t kBarEpi = 1, kBarOut = 3, kBarOutGo = 4;
+constexpr uint32_t kEpiWarps = kEpiThreads / 32, kDeltaWarps = kEpiWarps / 2;
 constexpr uint32_t R_TPV = 0;         // 2 stages x [TP 16K][TL 16K][V 16K]
 constexpr uint32_t R_TPV_STAGE = 49152;
 constexpr uint32_t R_WQ = 98304;      // 2 stages x 32K
@@ -895,7 +904,13 @@ __global__ void __launch_bounds__(kRecThreads, 1)
   auto spin = [&](int b, uint32_t parity) { return bounded_spin(bar + b, parity, abort_flag, p.status); };
 
   if (tid == 0) {
-    for (int b = 0; b < RB_COUNT; ++b) mbar_init(bar + b, (b == RB_TPV_EMPTY || b == RB_TPV_EMPTY + 1) ? 2 : 1);
+    for (int b = 0; b < RB_COUNT; ++b) {
+      uint32_t count = 1;
+      if (b == RB_TPV_EMPTY || b == RB_TPV_EMPTY + 1) count = 1 + kDeltaWarps;  // the Xv commit, each Delta warp
+      if (b == RB_DELTA) count = kDeltaWarps;
+      if (b == RB_S) count = kEpiWarps;
+      mbar_init(bar + b, count);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.v);
@@ -1126,10 +1141,8 @@ __global__ void __launch_bounds__(kRecThreads, 1)
       }
       tc_fence_before();
       named_bar(kBarEpi, kEpiThreads);
-      if (et == 0) {
-        mbar_arrive(bar + RB_S);
-        mbar_arrive(bar + RB_ST);
-      }
+      if (lane == 0) mbar_arrive(bar + RB_S);
+      if (et == 0) mbar_arrive(bar + RB_ST);
 
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
@@ -1137,9 +1150,11 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         const int64_t t0 = bos + (int64_t)c * C;
         const uint32_t acc = tmem + lane_base + TM_ACC + 128 * (c & 1);
         // ---------------------------------------------------- ep1: Delta^T (columns 0..63), O^T (64..127)
+        // no barrier of all epilogue warps on the critical path: a failed wait raises the abort flag,
+        // the warp carries on (its results are then discarded) and every warp leaves the loop
+        // together at the barrier that closes ep2
         if (cb < 2) wait(RB_TPV_FULL + s, (c >> 1) & 1);  // 1/|k| of this chunk
         wait(RB_MMA1, c & 1);
-        if (epi_sync_abort()) break;
         tc_fence_after();
         if (cb < 2) {
           float d[32];
@@ -1156,8 +1171,8 @@ __global__ void __launch_bounds__(kRecThreads, 1)
           tmem_st16(tmem + lane_base + TM_DL + col0 / 2, lo);
           tmem_wait_st();
           tc_fence_before();
-          named_bar(kBarDelta, kEpiThreads / 2);
-          if (et == 0) {
+          __syncwarp();
+          if (lane == 0) {
             mbar_arrive(bar + RB_DELTA);
             mbar_arrive(bar + RB_TPV_EMPTY + s);
           }
@@ -1198,7 +1213,6 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         const bool last = (c + 1 == nch);
         wait(RB_MMA2, c & 1);
         if (!last) wait(RB_TPV_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1);
-        if (epi_sync_abort()) break;
         tc_fence_after();
         float x[32];
         tmem_ld32(tmem + lane_base + TM_ST + col0, x);
@@ -1208,12 +1222,14 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         }
         store_state_bf16(x);
         tc_fence_before();
-        named_bar(kBarEpi, kEpiThreads);
-        if (et == 0) mbar_arrive(bar + RB_S);
-        // off the critical path (MMA1 of the next chunk runs meanwhile): the rescaled fp32 state
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar + RB_S);
+        // off the critical path (MMA1 of the next chunk runs meanwhile): the rescaled fp32 state,
+        // then the one barrier of all epilogue warps per chunk, which also decides (for all of them)
+        // whether to stop; it keeps ep1 of the next chunk after every warp's reads of this stage
         store_state_scaled(x, sc_gam + ((c + 1) & 1) * (IT_SC_BYTES / 4));
         tc_fence_before();
-        named_bar(kBarEpi, kEpiThreads);
+        if (epi_sync_abort()) break;
         if (et == 0) mbar_arrive(bar + RB_ST);
       }
       if (out_issuer) bulk_wait_all();

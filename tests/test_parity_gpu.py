@@ -190,6 +190,42 @@ def test_chunked_is_deterministic(cuda_device):
     np.testing.assert_array_equal(s1, s2)
 
 
+def test_device_wait_timeout_is_reported(cuda_device):
+    """A bounded device wait on a barrier that nothing completes runs out, records
+    KDA_ERR_DEVICE_TIMEOUT in the status word (read and cleared once) and leaves the context
+    usable: a valid forward on the same workspace follows."""
+    x = kda_inputs.make_workload("tail")
+    ws = kda.new_workspace(x.total_tokens, x.num_heads, x.num_seqs, cuda_device)
+    kda.selftest_wait_timeout(ws, limit_us=2000)
+    assert kda.read_device_status(ws) == 5  # KDA_ERR_DEVICE_TIMEOUT
+    assert kda.read_device_status(ws) == 0  # cleared by the read
+    o_ref, s_ref = oracle.fwd_inputs(x)
+    check(*run_gpu(x), o_ref, s_ref, "valid call after a time-out")
+
+
+@pytest.mark.parametrize("bad", [[0, 200, 100, 350], [0, 100, 300, 100000], [0, 100, 300, 340],
+                                 [5, 100, 300, 350], [0, -20, 300, 350]])
+def test_malformed_cu_seqlens_reported_on_device(cuda_device, bad):
+    """Offsets that do not tile the T tokens in order are caught on the device: the call records
+    KDA_ERR_INVALID_ARGUMENT, touches no token outside [0, T), leaves out unwritten and hands the
+    initial state through; the same workspace then serves a valid call."""
+    x = kda_inputs.make_random("t", [100, 200, 50], 2, seed=40, state_std=0.1).to(cuda_device)
+    N, H = 3, 2
+    cu_bad = torch.tensor(bad, dtype=torch.int32, device=cuda_device)
+    ws = kda.new_workspace(x.total_tokens, H, N, cuda_device)
+    for fn in (kda.fwd, kda.fwd_recurrent):
+        out = torch.full_like(x.v, float("nan"))
+        fin = torch.full((N, H, 128, 128), float("nan"), device=cuda_device)
+        fn(x.q, x.k, x.v, x.g, x.beta, x.scale, out, ws, x.A_log, x.dt_bias, x.lower_bound,
+           x.initial_state, fin, cu_bad)
+        assert kda.read_device_status(ws) == 1  # KDA_ERR_INVALID_ARGUMENT
+        if fn is kda.fwd:
+            assert torch.isnan(out).all()
+            assert torch.equal(fin, x.initial_state)
+    o_ref, s_ref = oracle.fwd_inputs(x.to("cpu"))
+    check(*run_gpu(x.to("cpu")), o_ref, s_ref, "valid call after a malformed one")
+
+
 def test_chunk_kda_convenience(cuda_device):
     x = kda_inputs.make_workload("usage").to(cuda_device)
     out, final = kda.chunk_kda(x.q, x.k, x.v, x.g, x.beta, scale=x.scale, A_log=x.A_log,
