@@ -197,7 +197,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=HEADS,
                     help="heads of the prefill workload (default 96; fewer only for small profiling runs)")
@@ -264,25 +264,46 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
 
-    def e2e_step():
+    # Each step copies its inputs in on the compute stream, runs kda.fwd and copies o and the final
+    # state out on a second stream (the two directions use different copy engines), so step i's
+    # outputs travel back while step i + 1's inputs travel in.  Outputs alternate between two
+    # device buffers; a buffer is rewritten only after its previous copy-out has finished.
+    d2h_stream = torch.cuda.Stream(dev)
+    outs = [out, torch.empty_like(out)]
+    finals = [final, torch.empty_like(final)]
+    outs_h = [out_h, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
+    fins_h = [fin_h, torch.empty(final.shape, dtype=final.dtype).pin_memory()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]   # copy-out of buffer b finished
+    ready = [torch.cuda.Event(), torch.cuda.Event()]  # kda.fwd into buffer b finished
+
+    def e2e_step(i):
+        b = i & 1
         for n, t in host.items():
             dev_bufs[n].copy_(t, non_blocking=True)
-        kda.fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["g"], dev_bufs["beta"], x.scale, out, ws,
-                dev_bufs["A_log"], dev_bufs["dt_bias"], x.lower_bound, None, final, dev_bufs["cu_seqlens"],
-                stream=stream.cuda_stream)
-        out_h.copy_(out, non_blocking=True)
-        fin_h.copy_(final, non_blocking=True)
+        stream.wait_event(done[b])
+        kda.fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["g"], dev_bufs["beta"], x.scale, outs[b],
+                ws, dev_bufs["A_log"], dev_bufs["dt_bias"], x.lower_bound, None, finals[b],
+                dev_bufs["cu_seqlens"], stream=stream.cuda_stream)
+        ready[b].record(stream)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(ready[b])
+            outs_h[b].copy_(outs[b], non_blocking=True)
+            fins_h[b].copy_(finals[b], non_blocking=True)
+            done[b].record(d2h_stream)
 
     e2e = None
     if args.e2e_steps > 0:
-        e2e_step()
+        for b in range(2):
+            done[b].record(d2h_stream)
+        e2e_step(0)
         torch.cuda.synchronize()
         barrier(world)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        stream.wait_stream(d2h_stream)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
