@@ -310,6 +310,7 @@ def main():
         e2e = {"value": world * token_heads / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
+    in_bytes = sum(t.numel() * t.element_size() for t in (x.q, x.k, x.v, x.g, x.beta))
     hbm_peak, tf_peak, peak_kind = load_peaks()
     alg_bytes = algorithmic_bytes(B * T, H, N)
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
@@ -325,7 +326,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD if H == HEADS else WORKLOAD.replace("H=96", f"H={H}"), "batch": B, "seq_len": T, "heads": H, "head_dim": K, "chunk": CHUNK,
-                   "parallelism": f"replicas{world}", "l2": "inputs (4.0 GB) exceed L2 (126 MB); no flush"},
+                   "parallelism": f"replicas{world}",
+                   "l2": f"inputs ({in_bytes / 1e9:.2f} GB) exceed L2 (126 MB); no flush"},
         "tflops": flops / (kernel_ms * 1e-3) / 1e12,
         "tflops_frac_of_bf16_peak": flops / (kernel_ms * 1e-3) / 1e12 / tf_peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",

@@ -108,6 +108,60 @@ def test_two_stage_schedule(cuda_device, opt):
     check(o, s, o_ref, s_ref, f"two stages/{opt}")
 
 
+def _stage_cut(lens, H, sms):
+    """Where the launcher cuts the global chunk range (its documented sizing rule), or None."""
+    T, N = sum(lens), len(lens)
+    mc = (T + 63 * N) // 64
+    if N * H >= sms:
+        return None
+    x = 0.27 * (sms - N * H) / H
+    g = mc - int(mc * x / (1 + x))
+    return g if 0 < g < mc else None
+
+
+def _cut_layouts(H, sms):
+    """Seeded document layouts whose stage cut falls exactly on a document start, inside a
+    document, and on an empty document."""
+    rng = np.random.default_rng(33)
+    found = {}
+    for _ in range(20000):
+        n = int(rng.integers(2, 7))
+        lens = [int(v) * 64 + (int(rng.integers(0, 64)) if rng.random() < 0.3 else 0)
+                for v in rng.integers(0, 9, size=n)]
+        if sum(lens) == 0:
+            continue
+        g = _stage_cut(lens, H, sms)
+        if g is None:
+            continue
+        co = np.concatenate([[0], np.cumsum([(L + 63) // 64 for L in lens])])
+        if any(co[i] == g == co[i + 1] for i in range(n)):
+            kind = "empty document at the cut"
+        elif any(co[i] < g < co[i + 1] for i in range(n)):
+            kind = "cut inside a document"
+        elif g in co:
+            kind = "cut on a document start"
+        else:
+            continue
+        found.setdefault(kind, lens)
+        if len(found) == 3:
+            break
+    return found
+
+
+def test_stage_cut_positions(cuda_device):
+    """The two-stage schedule with the cut on a document start (no hand-over), inside a
+    document (state handed over through the workspace) and on an empty document."""
+    H = 2
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    layouts = _cut_layouts(H, sms)
+    assert len(layouts) == 3, layouts
+    for kind, lens in layouts.items():
+        assert kda.fwd_launch_count(sum(lens), H, len(lens)) == 5
+        x = kda_inputs.make_random("t", lens, H, seed=34, state_std=0.1)
+        o_ref, s_ref = oracle.fwd_inputs(x)
+        check(*run_gpu(x), o_ref, s_ref, f"{kind} {lens}")
+
+
 def test_many_short_documents(cuda_device):
     """1100 documents of 0..70 tokens: the per-sequence chunk table spans two 1024-wide scan
     blocks, and many chunks end a document part-way."""
