@@ -327,19 +327,18 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
         tma_prefetch_3d(&maps.g, 64, N.h, (int)N.t0);
       }
     }
-    uint2 qr[8], kr[8];
+    // k stays in registers (its tile becomes QB in pass 1); q is read again in pass 1, from the
+    // same 8 bytes that its XK value then overwrites
+    uint2 kr[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool valid = 8 * iw + i < len;
-      qr[i] = valid ? lds64(a_rq + xo(i)) : make_uint2(0, 0);
-      kr[i] = valid ? lds64(a_rk + xo(i)) : make_uint2(0, 0);
-    }
+    for (int i = 0; i < 8; ++i) kr[i] = (8 * iw + i < len) ? lds64(a_rk + xo(i)) : make_uint2(0, 0);
     float2 a2[8][2];  // alpha of channels (4 lane, +1), (4 lane + 2, +3)
     float ssq[8], ssk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const bool valid = 8 * iw + i < len;
-      const float2 q01 = unpack_bf16(qr[i].x), q23 = unpack_bf16(qr[i].y);
+      const uint2 qri = valid ? lds64(a_rq + xo(i)) : make_uint2(0, 0);
+      const float2 q01 = unpack_bf16(qri.x), q23 = unpack_bf16(qri.y);
       const float2 k01 = unpack_bf16(kr[i].x), k23 = unpack_bf16(kr[i].y);
       const float2 sq = fma2(q23, q23, mul2(q01, q01)), sk = fma2(k23, k23, mul2(k01, k01));
       ssq[i] = sq.x + sq.y;
@@ -443,7 +442,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       for (int m = 0; m < 2; ++m) run[m] = upper_half ? pt[m] : make_float2(1.f, 1.f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float2 qv[2] = {unpack_bf16(qr[i].x), unpack_bf16(qr[i].y)};
+        const uint2 qri = (8 * iw + i < len) ? lds64(a_rq + xo(i)) : make_uint2(0, 0);
+        const float2 qv[2] = {unpack_bf16(qri.x), unpack_bf16(qri.y)};
         const float2 kv[2] = {unpack_bf16(kr[i].x), unpack_bf16(kr[i].y)};
         const float2 iq = splat2(__shfl_sync(0xffffffffu, inv_s, 2 * i));
         const float2 ik = splat2(__shfl_sync(0xffffffffu, inv_s, 16 + 2 * i));
