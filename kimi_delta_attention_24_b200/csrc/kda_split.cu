@@ -265,20 +265,24 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const uint64_t d_xk = sdesc_sw128(sbase + I_XK, 8192, 1024);   // MN-major B
 
   // Items (gc * H + h, chunk-major) come from a counter, so that a CTA that starts late (on an SM
-  // freed by another kernel) takes fewer.  Thread 32 takes the next item while the current one runs
-  // and publishes it with its chunk in s_next[j & 1] (double-buffered: read after the item's last
-  // barrier), so that the division by H is done once per item.
-  __shared__ int64_t s_next[2][2];  // {item, global chunk}
+  // freed by another kernel) takes fewer.  Thread 32 takes the next item while the current one runs,
+  // locates it (sequence, first token, length) and publishes both in s_item / s_loc[j & 1]
+  // (double-buffered: read after the item's last barrier).
+  __shared__ int64_t s_item[2];
+  __shared__ Loc s_loc[2];
   const int64_t item_end = args.item_end < total_gc * H ? args.item_end : total_gc * H;
   if (itid == 0) {
     const int64_t it = args.item_begin + (int64_t)atomicAdd(args.queue, 1ull);
-    s_next[1][0] = it;
-    s_next[1][1] = it / H;
+    s_item[1] = it;
+    if (it < item_end) {
+      const int64_t gc = it / H;
+      s_loc[1] = locate(gc, (int)(it - gc * H));
+    }
   }
   __syncthreads();
-  int64_t cur_it = s_next[1][0], cur_gc = s_next[1][1];
+  int64_t cur_it = s_item[1];
   for (uint32_t j = 0; cur_it < item_end; ++j) {
-    const Loc L = locate(cur_gc, (int)(cur_it - cur_gc * H));
+    const Loc L = s_loc[(j + 1) & 1];
     const int h = L.h, len = L.len;
     const int64_t t0 = L.t0;
     uint8_t* item = args.items + ((size_t)L.gc * H + h) * ITEM_BYTES;
@@ -314,11 +318,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     if (cta_wait(0, raw_par)) break;
     if (itid == 32) {
       // the counter's answer has had the q / k load's time to arrive; warm L2 for the next item
-      const int64_t ngc = nxt / H;
-      s_next[j & 1][0] = nxt;
-      s_next[j & 1][1] = ngc;
+      s_item[j & 1] = nxt;
       if (nxt < item_end) {
+        const int64_t ngc = nxt / H;
         const Loc N = locate(ngc, (int)(nxt - ngc * H));
+        s_loc[j & 1] = N;
         tma_prefetch_3d(&maps.q, 0, N.h, (int)N.t0);
         tma_prefetch_3d(&maps.q, 64, N.h, (int)N.t0);
         tma_prefetch_3d(&maps.k, 0, N.h, (int)N.t0);
@@ -779,8 +783,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     tc_fence_before();
     if (itid == 0) bulk_wait_read<0>();
     sync();
-    cur_it = s_next[j & 1][0];
-    cur_gc = s_next[j & 1][1];
+    cur_it = s_item[j & 1];
   }
   // no item left for this CTA: a kernel launched after this one as a programmatic dependent may
   // start its CTAs
