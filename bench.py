@@ -116,15 +116,19 @@ class ClockSampler:
 
 
 def dist_setup(n_gpus):
+    """One process per GPU from the launcher's environment; NCCL on GPUs, gloo without (tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     return rank, world, local
 
 
@@ -138,9 +142,16 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(token_heads_per_rank, ms_per_step, world):
+    """Whole-job Mtok·head/s: every rank runs its own replica of the workload (weak scaling), and
+    the step time is the slowest rank's."""
+    return world * token_heads_per_rank / (ms_per_step * 1e-3) / 1e6
 
 
 def cpu_oracle_sample(target_s=15.0):
@@ -254,7 +265,7 @@ def main():
     status = kda.read_device_status(ws)
     ms_per_step = total_ms / args.steps
     token_heads = B * T * H
-    value = world * token_heads / (ms_per_step * 1e-3) / 1e6
+    value = replica_throughput(token_heads, ms_per_step, world)
 
     # end to end through the public API with pinned host buffers: H2D inputs, kernel, D2H outputs
     host = {n: getattr(x, n).cpu().pin_memory() for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "cu_seqlens")}
@@ -307,7 +318,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
-        e2e = {"value": world * token_heads / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+        e2e = {"value": replica_throughput(token_heads, e2e_ms, world), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     in_bytes = sum(t.numel() * t.element_size() for t in (x.q, x.k, x.v, x.g, x.beta))
