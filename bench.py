@@ -275,26 +275,34 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
 
-    # Each step copies its inputs in on the compute stream, runs kda.fwd and copies o and the final
-    # state out on a second stream (the two directions use different copy engines), so step i's
-    # outputs travel back while step i + 1's inputs travel in.  Outputs alternate between two
-    # device buffers; a buffer is rewritten only after its previous copy-out has finished.
+    # Each step copies its inputs in on a copy-in stream, runs kda.fwd on the compute stream and
+    # copies o and the final state out on a copy-out stream (the two directions use different copy
+    # engines).  Inputs and outputs alternate between two device buffer sets, so step i + 1's
+    # inputs travel in while step i computes and step i - 1's outputs travel back; a set is
+    # rewritten only after the work that read it has finished.
+    h2d_stream = torch.cuda.Stream(dev)
     d2h_stream = torch.cuda.Stream(dev)
+    ins = [dev_bufs, {n: torch.empty_like(t) for n, t in dev_bufs.items()}]
     outs = [out, torch.empty_like(out)]
     finals = [final, torch.empty_like(final)]
     outs_h = [out_h, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
     fins_h = [fin_h, torch.empty(final.shape, dtype=final.dtype).pin_memory()]
-    done = [torch.cuda.Event(), torch.cuda.Event()]   # copy-out of buffer b finished
-    ready = [torch.cuda.Event(), torch.cuda.Event()]  # kda.fwd into buffer b finished
+    in_ready = [torch.cuda.Event(), torch.cuda.Event()]  # inputs of set b copied in
+    ready = [torch.cuda.Event(), torch.cuda.Event()]     # kda.fwd on set b finished
+    done = [torch.cuda.Event(), torch.cuda.Event()]      # copy-out of set b finished
 
     def e2e_step(i):
         b = i & 1
-        for n, t in host.items():
-            dev_bufs[n].copy_(t, non_blocking=True)
+        d = ins[b]
+        with torch.cuda.stream(h2d_stream):
+            h2d_stream.wait_event(ready[b])
+            for n, t in host.items():
+                d[n].copy_(t, non_blocking=True)
+            in_ready[b].record(h2d_stream)
+        stream.wait_event(in_ready[b])
         stream.wait_event(done[b])
-        kda.fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["g"], dev_bufs["beta"], x.scale, outs[b],
-                ws, dev_bufs["A_log"], dev_bufs["dt_bias"], x.lower_bound, None, finals[b],
-                dev_bufs["cu_seqlens"], stream=stream.cuda_stream)
+        kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], x.scale, outs[b], ws, d["A_log"], d["dt_bias"],
+                x.lower_bound, None, finals[b], d["cu_seqlens"], stream=stream.cuda_stream)
         ready[b].record(stream)
         with torch.cuda.stream(d2h_stream):
             d2h_stream.wait_event(ready[b])
@@ -305,6 +313,7 @@ def main():
     e2e = None
     if args.e2e_steps > 0:
         for b in range(2):
+            ready[b].record(stream)
             done[b].record(d2h_stream)
         e2e_step(0)
         torch.cuda.synchronize()
@@ -312,8 +321,10 @@ def main():
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        h2d_stream.wait_stream(stream)  # the first copy-in starts inside the timed region
         for i in range(args.e2e_steps):
             e2e_step(i)
+        stream.wait_stream(h2d_stream)
         stream.wait_stream(d2h_stream)
         e1.record(stream)
         torch.cuda.synchronize()
