@@ -136,10 +136,10 @@ __device__ __forceinline__ int seq_of_chunk(const int32_t* co, int nseq, int64_t
 // 2 blocks of 64 columns x [64 rows][128 B] with the 128-byte swizzle, "K tile" = 2 blocks of 64 K
 // x [rows][128 B].
 constexpr int kIntraThreads = 256;
-constexpr uint32_t I_RQ = 0;        // q tile (TMA); becomes XK once q, k sit in registers
-constexpr uint32_t I_RK = 16384;    // k tile (TMA); becomes QB
-constexpr uint32_t I_XK = 0;        // Khat e^Gamma (pre-scaled to the chunk start), MN tile, B of MMA Xk
-constexpr uint32_t I_QB = 16384;    // Qtil, MN tile, read when forming Qtil - P W
+constexpr uint32_t I_RQ = 0;        // q tile (TMA); becomes XK row by row in pass 1
+constexpr uint32_t I_RK = 16384;    // k tile (TMA); becomes QB once k sits in registers
+constexpr uint32_t I_XK = 0;        // -Khat e^Gamma (pre-scaled to the chunk start), MN tile, B of MMA Xk
+constexpr uint32_t I_QB = 16384;    // Qtil, MN tile, B of the MMA that seeds [0; Qtil]
 constexpr uint32_t I_LKQ = 32768;   // [LK; LQ] K tile, 128 rows (A of MMA AP)
 constexpr uint32_t I_R = 65536;     // R_0..R_3 K tile, 160 rows (B of MMA AP)
 constexpr uint32_t I_RKBLK = 160 * 128;
@@ -161,6 +161,7 @@ constexpr uint32_t I_ALLOC = I_SMEM + 1024;
 static_assert(I_YS + 4096 <= I_SC, "intra shared-memory map");
 static_assert(2 * (I_ALLOC + 1024) <= 233472, "two intra CTAs per SM");
 constexpr uint32_t kIntraTmemCols = 256;
+constexpr uint32_t kIdCol = 192;  // [0; I_64] as bf16 (32 columns), A of the MMA that seeds [0; Qtil]
 
 struct IntraMaps {
   CUtensorMap q, k, g;
@@ -213,6 +214,19 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   sync();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + I_TMEM);
+  // A = [0; I_64] (128 x 64 bf16, two per column, low half first) in columns kIdCol .. + 31, which
+  // no accumulator reaches (the Gram product uses columns 0 .. 159)
+  if (iw < 4) {
+    const int r = 32 * iw + lane - 64;  // identity row, or negative in the zero half
+    uint32_t u[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) u[c] = (r >= 0 && (r >> 1) == c) ? ((r & 1) ? 0x3F800000u : 0x3F80u) : 0u;
+    tmem_st32(tmem + ((uint32_t)(32 * iw) << 16) + kIdCol, u);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  sync();
+  tc_fence_after();
 
   // one thread waits on the mbarrier, the others in the CTA barrier; the answer (abort?) is uniform
   uint32_t raw_par = 0, mma_par = 0;
@@ -263,6 +277,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const uint64_t d_tpm = sdesc_sw128(sbase + I_TP, 8192, 1024);  // T_b hi / lo as MN-major B
   const uint64_t d_tlm = sdesc_sw128(sbase + I_TL, 8192, 1024);
   const uint64_t d_xk = sdesc_sw128(sbase + I_XK, 8192, 1024);   // MN-major B
+  const uint64_t d_qb = sdesc_sw128(sbase + I_QB, 8192, 1024);   // MN-major B
 
   // Items (gc * H + h, chunk-major) come from a counter, so that a CTA that starts late (on an SM
   // freed by another kernel) takes fewer.  Thread 32 takes the next item while the current one runs,
@@ -439,8 +454,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       }
     }
 
-    // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i
+    // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i.  XK is
+    // written negated, so that MMA Xk subtracts [W; P W] from the [0; Qtil] it starts from
     {
+      const float2 npre[2] = {make_float2(-pre[0].x, -pre[0].y), make_float2(-pre[1].x, -pre[1].y)};
       float2 run[2];
 #pragma unroll
       for (int m = 0; m < 2; ++m) run[m] = upper_half ? pt[m] : make_float2(1.f, 1.f);
@@ -461,7 +478,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
         }
         sts64(a_lk + xo(i), bf16x2_of(mul2(lk[0], b)), bf16x2_of(mul2(lk[1], b)));
         sts64(a_lq + xo(i), bf16x2_of(lq[0]), bf16x2_of(lq[1]));
-        sts64(a_xk + xo(i), bf16x2_of(mul2(lk[0], pre[0])), bf16x2_of(mul2(lk[1], pre[1])));
+        sts64(a_xk + xo(i), bf16x2_of(mul2(lk[0], npre[0])), bf16x2_of(mul2(lk[1], npre[1])));
         sts64(a_qb + xo(i), bf16x2_of(mul2(lq[0], pre[0])), bf16x2_of(mul2(lq[1], pre[1])));
       }
     }
@@ -724,15 +741,20 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     tc_fence_before();
     sync();
 
-    // ================================================================ MMA Xk: [T_b; P T_b] x Khat e^Gamma
+    // ================================================================ MMA Xk: [0; Qtil] - [T_b; P T_b] x Khat e^Gamma
     if (itid == 0) {
       tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);  // B MN-major (A K-major or in TMEM)
+      // [0; I_64] x Qtil seeds the accumulator with [0; Qtil] ...
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16_tmem_a(tmem, tmem + kIdCol + 8 * ks, sdesc_add(d_qb, ks * 2048), idesc, ks > 0);
+      // ... and [T_b; P T_b] (hi + lo) x (-Khat e^Gamma) completes [-W; Qtil - P W]
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t ad = sdesc_add(ks < 4 ? d_tpk : d_tlk, (ks & 3) * 32);
         const uint64_t bd = sdesc_add(d_xk, (ks & 3) * 2048);
-        umma_bf16(tmem, ad, bd, idesc, ks > 0);
+        umma_bf16(tmem, ad, bd, idesc, 1);
       }
       umma_commit(bar + 1);
       // [T_b; P T_b] hi and lo are final: copy both tiles to the item while the MMA runs
@@ -754,19 +776,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 #pragma unroll
         for (int cch = 0; cch < 4; ++cch) {
           uint4 w;
-          if (R >= 64) {
-            const uint4 qb = *reinterpret_cast<const uint4*>(sm + I_QB + ihalf * 8192 + sw128(R - 64, 4 * part + cch));
-            const float2 a0 = unpack_bf16(qb.x), a1 = unpack_bf16(qb.y), a2 = unpack_bf16(qb.z), a3 = unpack_bf16(qb.w);
-            w.x = pack_bf16(a0.x - d[8 * cch + 0], a0.y - d[8 * cch + 1]);
-            w.y = pack_bf16(a1.x - d[8 * cch + 2], a1.y - d[8 * cch + 3]);
-            w.z = pack_bf16(a2.x - d[8 * cch + 4], a2.y - d[8 * cch + 5]);
-            w.w = pack_bf16(a3.x - d[8 * cch + 6], a3.y - d[8 * cch + 7]);
-          } else {
-            w.x = pack_bf16(-d[8 * cch + 0], -d[8 * cch + 1]);
-            w.y = pack_bf16(-d[8 * cch + 2], -d[8 * cch + 3]);
-            w.z = pack_bf16(-d[8 * cch + 4], -d[8 * cch + 5]);
-            w.w = pack_bf16(-d[8 * cch + 6], -d[8 * cch + 7]);
-          }
+          w.x = pack_bf16(d[8 * cch + 0], d[8 * cch + 1]);
+          w.y = pack_bf16(d[8 * cch + 2], d[8 * cch + 3]);
+          w.z = pack_bf16(d[8 * cch + 4], d[8 * cch + 5]);
+          w.w = pack_bf16(d[8 * cch + 6], d[8 * cch + 7]);
           *reinterpret_cast<uint4*>(dst + ((((uint32_t)(4 * part + cch) ^ (uint32_t)R) & 7u) << 4)) = w;
         }
       }
@@ -778,8 +791,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       bulk_commit();
     }
 
-    // the next item's TMA overwrites XK / QB (read above and by MMA Xk, which has completed) and its
-    // passes overwrite TP / TL: the bulk copy of this item's TP / TL must have read them
+    // the next item's TMA overwrites XK / QB (read by MMA Xk, which has completed) and its passes
+    // overwrite TP / TL: the bulk copy of this item's TP / TL must have read them
     tc_fence_before();
     if (itid == 0) bulk_wait_read<0>();
     sync();
