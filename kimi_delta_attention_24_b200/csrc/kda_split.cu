@@ -421,7 +421,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       }
       reinterpret_cast<float4*>(sc_tot + iw * 128)[lane] = make_float4(t[0].x, t[0].y, t[1].x, t[1].y);
     }
-    sync();  // also: every thread holds its q, k rows, so the raw tiles may be overwritten
+    // the previous item's bulk copies have read TP / TL / AS, which the passes overwrite
+    if (itid == 0) bulk_wait_read<0>();
+    sync();  // also: every thread holds its k rows, so the k tile may be overwritten
     // sub-block totals b_J = prod of alpha over rows 16 J .. 16 J + 15 (channels 4 lane .. + 3)
     auto load_bJ = [&](float2 (&bJ)[4][2]) {
 #pragma unroll
@@ -617,8 +619,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     sync();
     // off-diagonal blocks by distance dd below the diagonal: T_IJ = -T_II (sum_{K=J}^{I-1} A_IK T_KJ),
     // each 16x16x16 product on mma.sync m16n8k8 tf32 with both operands split hi + lo (three
-    // products, fp32-level accuracy).  Warp w takes block J = w / 2 and the 8 columns nt = w % 2
-    // of it; the three partial products accumulate separately so their chains stay short.
+    // products, fp32-level accuracy).  Warp w takes block column J = w / 2 and its 8 columns
+    // nt = w % 2 all the way down: every T_KJ it reads in those columns it wrote itself, and the
+    // diagonal blocks are final, so the levels need no barrier across warps.  The three partial
+    // products accumulate separately so their chains stay short.
 #pragma unroll 1
     for (int dd = 1; dd < 4; ++dd) {
       const int bJ2 = iw >> 1, nt = iw & 1, bI = bJ2 + dd;
@@ -678,11 +682,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
         to[(g + 8) * AS_LD + 2 * t] = -(zh[2] + (zm[2] + zl[2]));
         to[(g + 8) * AS_LD + 2 * t + 1] = -(zh[3] + (zm[3] + zl[3]));
       }
-      sync();
+      __syncwarp();
     }
-    // T_b = T diag(beta) as a bf16 hi + lo pair, rows 0..63 of TP / TL
+    sync();
+    // T_b = T diag(beta) as a bf16 hi + lo pair, rows 0..63 of TP / TL (a warp takes 32 rows of one
+    // 16-column band, so its 16-byte reads of T hit distinct banks)
     {
-      const int r = itid >> 2, c16 = itid & 3;
+      const int r = itid & 63, c16 = itid >> 6;
       const int I = r >> 4;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -785,17 +791,15 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       }
     }
     fence_proxy_async();
+    tc_fence_before();  // this item's tensor-memory reads, before the next item's MMAs
     sync();
     if (itid == 0) {
       bulk_store(item + IT_WQ, sm + I_AS, 32768);
       bulk_commit();
     }
-
-    // the next item's TMA overwrites XK / QB (read by MMA Xk, which has completed) and its passes
-    // overwrite TP / TL: the bulk copy of this item's TP / TL must have read them
-    tc_fence_before();
-    if (itid == 0) bulk_wait_read<0>();
-    sync();
+    // no barrier here: the next item's TMA only overwrites XK / QB (read by MMA Xk, which has
+    // completed), and thread 0 lets the bulk copies finish reading TP / TL / AS before the barrier
+    // that precedes the next item's passes (which overwrite them)
     cur_it = s_item[j & 1];
   }
   // no item left for this CTA: a kernel launched after this one as a programmatic dependent may
