@@ -295,20 +295,23 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     }
   }
   __syncthreads();
+  // thread 0: the q and k tiles of an item (issued for the next item as soon as MMA Xk of the
+  // current one has read XK / QB, the tiles they land in)
+  auto load_qk = [&](const Loc& N) {
+    raw_pending = true;
+    mbar_arrive_expect_tx(bar + 0, 32768);
+    tma_load_3d(sm + I_RQ, &maps.q, bar + 0, 0, N.h, (int)N.t0);
+    tma_load_3d(sm + I_RQ + 8192, &maps.q, bar + 0, 64, N.h, (int)N.t0);
+    tma_load_3d(sm + I_RK, &maps.k, bar + 0, 0, N.h, (int)N.t0);
+    tma_load_3d(sm + I_RK + 8192, &maps.k, bar + 0, 64, N.h, (int)N.t0);
+  };
   int64_t cur_it = s_item[1];
+  if (itid == 0 && cur_it < item_end) load_qk(s_loc[1]);
   for (uint32_t j = 0; cur_it < item_end; ++j) {
     const Loc L = s_loc[(j + 1) & 1];
     const int h = L.h, len = L.len;
     const int64_t t0 = L.t0;
     uint8_t* item = args.items + ((size_t)L.gc * H + h) * ITEM_BYTES;
-    if (itid == 0) {
-      raw_pending = true;
-      mbar_arrive_expect_tx(bar + 0, 32768);
-      tma_load_3d(sm + I_RQ, &maps.q, bar + 0, 0, h, (int)t0);
-      tma_load_3d(sm + I_RQ + 8192, &maps.q, bar + 0, 64, h, (int)t0);
-      tma_load_3d(sm + I_RK, &maps.k, bar + 0, 0, h, (int)t0);
-      tma_load_3d(sm + I_RK + 8192, &maps.k, bar + 0, 64, h, (int)t0);
-    }
     int64_t nxt = 0;
     if (itid == 32) nxt = args.item_begin + (int64_t)atomicAdd(args.queue, 1ull);
 
@@ -769,6 +772,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     }
     if (cta_wait(1, mma_par)) break;
     tc_fence_after();
+    if (itid == 0 && s_item[j & 1] < item_end) load_qk(s_loc[j & 1]);
 
     // ================================================================ [-W; Qtil - P W] -> item
     {
