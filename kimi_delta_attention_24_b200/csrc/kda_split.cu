@@ -600,11 +600,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
         }
       }
     }
-    sync();
 
     // ================================================================ solve T = (I + A)^{-1}
-    if (iw < 4 && lane < 16) {
-      const int I = iw, j = lane;
+    // The diagonal blocks of A are rows / columns 0..31 of warp 0's share of the assembly and
+    // 32..63 of warp 5's: those two warps solve them at once, 16 lanes (one column each) per block.
+    if (iw == 0 || iw == 5) {
+      __syncwarp();
+      const int I = (iw == 0 ? 0 : 2) + (lane >> 4), j = lane & 15;
       const float* ab = As + (16 * I) * AS_LD + 16 * I;
       float x[16];
 #pragma unroll
