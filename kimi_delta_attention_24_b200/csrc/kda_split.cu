@@ -174,7 +174,16 @@ __device__ __forceinline__ uint32_t bf16x2_of(float2 v) { return bf16x2(v.x, v.y
 
 // Persistent: every CTA takes items [item_begin, item_end) in chunk-major order (item = global
 // chunk * H + head) from a shared counter, pulling its next item's q, k and g tiles into L2 while
-// it works on the current one.
+// it works on the current one and loading the next q, k tiles as soon as MMA Xk has freed them.
+// Per item (8 warps; warp iw owns rows 8 iw .. + 7 in the element-wise phases):
+//   prologue  norms, sigmoid(beta), the gate, per-warp decay products (q read, k kept in registers)
+//   pass 1    [LK; LQ] (Gram left operand), XK = -Khat e^Gamma and QB = Qtil (q read again)
+//   pass 2    R_0..R_3 (Gram right operand, one decay reference per row block) and Ktil (to the item)
+//   MMA AP    [LK; LQ] R^T (N = 160) -> assembly of A (fp32) and P (bf16)
+//   solve     diagonal 16 x 16 blocks by substitution (warps 0 and 5, which assembled them), then
+//             the off-diagonal blocks column by column on 3xTF32 mma.sync, warp-local levels
+//   T_b       hi + lo split; MMA PT: P T_b (hi + lo), read back as a hi + lo pair
+//   MMA Xk    [0; I] Qtil + [T_b; P T_b] (-XK) = [-W; Qtil - P W] in one accumulator -> bf16 image
 __global__ void __launch_bounds__(kIntraThreads, 2)
     intra_kernel(const __grid_constant__ IntraMaps maps, const SplitArgs args) {
   extern __shared__ uint8_t smem_raw[];
