@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const float2 x = fma2(ga2, gv[m], gb2[m]);
-        const float2 d = make_float2(1.0f + ex2_approx(x.x), 1.0f + ex2_approx(x.y));
+        const float2 d = fma2(make_float2(ex2_approx(x.x), ex2_approx(x.y)), splat2(1.f), splat2(1.f));
         const float2 y = mul2(splat2(lb2), make_float2(rcp_approx(d.x), rcp_approx(d.y)));
         a2[i][m] = valid ? make_float2(ex2_approx(y.x), ex2_approx(y.y)) : make_float2(1.f, 1.f);
       }
@@ -526,16 +526,19 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       for (int i = 7; i >= 0; --i) {
         const float2 kv[2] = {unpack_bf16(kr[i].x), unpack_bf16(kr[i].y)};
         const float2 ik = splat2(__shfl_sync(0xffffffffu, inv_s, 16 + 2 * i));
-        float2 kf[2];
+        float2 kr_f[2], kf[2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) kf[m] = mul2(kv[m], mul2(run[m], ik));  // khat * f
+        for (int m = 0; m < 2; ++m) {
+          kr_f[m] = mul2(kv[m], run[m]);  // raw k * f, shared by R (normalised) and Ktil
+          kf[m] = mul2(kr_f[m], ik);      // khat * f
+        }
 #pragma unroll
         for (int I = 0; I < 4; ++I) {
           if (I < blk) continue;
           sts64(a_r + row_off(I) * 128 + xo(i), bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
         }
         *reinterpret_cast<uint2*>(kt_dst + xo(i)) =
-            make_uint2(bf16x2_of(mul2(kv[0], mul2(run[0], post[0]))), bf16x2_of(mul2(kv[1], mul2(run[1], post[1]))));
+            make_uint2(bf16x2_of(mul2(kr_f[0], post[0])), bf16x2_of(mul2(kr_f[1], post[1])));
 #pragma unroll
         for (int m = 0; m < 2; ++m) run[m] = mul2(run[m], a2[i][m]);
       }
