@@ -162,6 +162,87 @@ def test_stage_cut_positions(cuda_device):
         check(*run_gpu(x), o_ref, s_ref, f"{kind} {lens}")
 
 
+# Byte layout of one (chunk, head) item that the intra-chunk kernel leaves in the workspace (an
+# internal format: the test decodes it to check each stage against the fp64 chunked form).
+_WS_HEADER, _ITEM = 256, 82944
+_IT_WQ, _IT_TP, _IT_TL, _IT_KT, _IT_IK, _IT_GAM = 0, 32768, 49152, 65536, 81920, 82176
+
+
+def _bf16_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _swizzled_tile(raw, rows):
+    """[rows][64] bf16 from a 128-byte-swizzled image: row r's 16-byte chunk c is stored at c ^ (r % 8)."""
+    u = np.frombuffer(raw, dtype=np.uint16).reshape(rows, 8, 8)
+    r = np.arange(rows)[:, None]
+    c = np.arange(8)[None, :]
+    return _bf16_to_f64(u[r, c ^ (r & 7)].reshape(rows, 64))
+
+
+def test_intra_chunk_stages_against_chunked_form(cuda_device):
+    """Each intra-chunk output against the fp64 chunked form of the same chunk: -W and Qtil - P W
+    (the MMA1 operand), T diag(beta) and P T diag(beta) (hi + lo pairs), Ktil (raw k with the decay
+    to the chunk end), 1/|k| and e^{Gamma_C}; full chunks and a 2-token tail."""
+    from oracle.chunked import chunk_intermediates
+    lens, H = [130, 64], 2
+    x = kda_inputs.make_random("t", lens, H, seed=41, state_std=0.1)
+    xd = x.to(cuda_device)
+    N = len(lens)
+    ws = kda.new_workspace(x.total_tokens, H, N, cuda_device)
+    out = torch.empty_like(xd.v)
+    kda.fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, x.scale, out, ws, xd.A_log, xd.dt_bias, x.lower_bound,
+            None, None, xd.cu_seqlens)
+    assert kda.read_device_status(ws) == 0
+    raw = ws.cpu().numpy().tobytes()
+    co = np.frombuffer(raw[_WS_HEADER:_WS_HEADER + 4 * (N + 1)], dtype=np.int32)
+    assert list(co) == [0, 3, 4]
+    items = _WS_HEADER + ((N + 1) * 4 + 1023) // 1024 * 1024
+    qh, kh, la, be = oracle.prologue(x.q, x.k, x.g, x.beta, x.A_log, x.dt_bias, x.lower_bound)
+    kraw = x.k.double().numpy()
+    cu = x.cu_seqlens.numpy()
+    worst = {}
+    for n in range(N):
+        t0, t1 = int(cu[n]), int(cu[n + 1])
+        for h in range(H):
+            chunks = chunk_intermediates(qh[0, t0:t1, h], kh[0, t0:t1, h], x.v[0, t0:t1, h].double().numpy(),
+                                         la[0, t0:t1, h], be[0, t0:t1, h], x.scale, 64)
+            for c, ref in enumerate(chunks):
+                L = ref["T"].shape[0]
+                off = items + ((int(co[n]) + c) * H + h) * _ITEM
+                it = raw[off:off + _ITEM]
+                wq = np.concatenate([_swizzled_tile(it[_IT_WQ + 16384 * kb:_IT_WQ + 16384 * (kb + 1)], 128)
+                                     for kb in range(2)], axis=1)
+                tb = _swizzled_tile(it[_IT_TP:_IT_TP + 16384], 128) + _swizzled_tile(it[_IT_TL:_IT_TL + 16384], 128)
+                kt = np.concatenate([_swizzled_tile(it[_IT_KT + 8192 * kb:_IT_KT + 8192 * (kb + 1)], 64)
+                                     for kb in range(2)], axis=1)
+                ik = np.frombuffer(it[_IT_IK:_IT_IK + 256], dtype=np.float32).astype(np.float64)
+                gam = np.frombuffer(it[_IT_GAM:_IT_GAM + 512], dtype=np.float32).astype(np.float64)
+                b = be[0, t0 + 64 * c:t0 + 64 * c + L, h]
+                Tb = ref["T"] * b[None, :]
+                kr = kraw[0, t0 + 64 * c:t0 + 64 * c + L, h]
+                ik_ref = 1.0 / np.sqrt((kr * kr).sum(axis=1) + 1e-6)
+                pairs = {
+                    "-W": (wq[:L], -ref["W"]),
+                    "Qtil - P W": (wq[64:64 + L], ref["Qt"] - ref["P"] @ ref["W"]),
+                    "T_b": (tb[:L, :L], Tb),
+                    "P T_b": (tb[64:64 + L, :L], ref["P"] @ Tb),
+                    "Ktil": (kt[:L], ref["Kt"] / ik_ref[:, None]),
+                    "1/|k|": (ik[:L], ik_ref),
+                    "e^Gamma_C": (gam, ref["gC"]),
+                }
+                assert np.all(ik[L:] == 0)  # rows past the end of the document
+                for name, (got, want) in pairs.items():
+                    assert np.isfinite(got).all(), name
+                    worst[name] = max(worst.get(name, 0.0), rel_l2(got, want))
+    # bf16 operands and outputs (-W, Qtil - P W, P T_b with P in bf16: a few 1e-3 measured), hi + lo
+    # pairs on an fp32 solve (T_b: ~6e-5), fp32 scalars (1/|k|: ~4e-8, e^Gamma_C: ~5e-6)
+    tol = {"-W": 1e-2, "Qtil - P W": 1e-2, "T_b": 1e-3, "P T_b": 2e-2, "Ktil": 5e-3, "1/|k|": 1e-6,
+           "e^Gamma_C": 1e-4}
+    for name, err in worst.items():
+        assert err <= tol[name], f"{name}: rel-L2 {err:.3e}"
+
+
 def test_many_short_documents(cuda_device):
     """1100 documents of 0..70 tokens: the per-sequence chunk table spans two 1024-wide scan
     blocks, and many chunks end a document part-way."""
