@@ -270,9 +270,11 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
 // ----------------------------------------------------------------------------------- warp MMA (solve)
 // tf32 split x = hi + lo with both parts representable in tf32.
 __device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
-  const float r = x - __uint_as_float(hi);
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+  // hi: x with the low 13 mantissa bits cleared (truncation); lo: the exact fp32 remainder,
+  // truncated the same way.  Two logic ops and a subtraction; the three products hi*hi, hi*lo and
+  // lo*hi then give x*y to about 2^-20 relative.
+  hi = __float_as_uint(x) & 0xFFFFE000u;
+  lo = __float_as_uint(x - __uint_as_float(hi)) & 0xFFFFE000u;
 }
 // D += A (16x8, row) * B (8x8, col), tf32 inputs, fp32 accumulate.
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
