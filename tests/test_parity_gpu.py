@@ -317,12 +317,19 @@ def test_split_resume_on_gpu(cuda_device):
     check(np.concatenate([oa, ob], axis=1), sb, o_ref, s_ref, "split-resume")
 
 
-def test_chunked_is_deterministic(cuda_device):
-    x = kda_inputs.make_workload("varlen")
+@pytest.mark.parametrize("layout", ["varlen", "two stages"])
+def test_chunked_is_deterministic(cuda_device, layout):
+    """Bitwise-equal results over repeated calls: items are taken from a counter in whatever order
+    the CTAs reach it, and the two-stage schedule overlaps launches, but no result depends on it."""
+    if layout == "varlen":
+        x = kda_inputs.make_workload("varlen")
+    else:
+        x = kda_inputs.make_random("t", [1000, 0, 2048, 77, 1, 3000, 0], 4, seed=32, state_std=0.1)
     o1, s1 = run_gpu(x)
-    o2, s2 = run_gpu(x)
-    np.testing.assert_array_equal(o1, o2)
-    np.testing.assert_array_equal(s1, s2)
+    for _ in range(4):
+        o2, s2 = run_gpu(x)
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(s1, s2)
 
 
 def test_device_wait_timeout_is_reported(cuda_device):
