@@ -1300,12 +1300,12 @@ int64_t chunk_bound(int64_t tokens, int64_t n) { return (tokens + (int64_t)(C - 
 // first g_cut global chunks runs, one SM per unit, while the intra launch of the remaining chunks
 // already fills the other SMs, and all of them once that recurrence is done.  The second stage's
 // share f is sized so that its intra work about fits on the free SMs during the first recurrence:
-// f / (1 - f) = 2 (SMs - units) t_chunk / (H t_item), with t_chunk / t_item ~ 0.15 the measured
-// ratio of one recurrence chunk to one intra item on one CTA (a sweep of the constant 2 t_chunk /
-// t_item from 0.24 to 0.40 has its optimum at 0.30).
+// f / (1 - f) = 2 (SMs - units) t_chunk / (H t_item), with t_chunk / t_item the ratio of one
+// recurrence chunk to one intra item on one CTA; the constant 2 t_chunk / t_item is set by a sweep
+// (flat optimum from 0.40 to 0.60 on the 96-head prefill; 0.45).
 int64_t stage_cut(int64_t max_chunks, int64_t units, int heads, int sms) {
   if (units >= sms || heads <= 0) return max_chunks;
-  const double x = 0.30 * (double)(sms - units) / (double)heads;
+  const double x = 0.45 * (double)(sms - units) / (double)heads;
   const int64_t g_cut = max_chunks - (int64_t)((double)max_chunks * x / (1.0 + x));
   return (g_cut <= 0 || g_cut >= max_chunks) ? max_chunks : g_cut;
 }

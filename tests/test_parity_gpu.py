@@ -114,7 +114,7 @@ def _stage_cut(lens, H, sms):
     mc = (T + 63 * N) // 64
     if N * H >= sms:
         return None
-    x = 0.30 * (sms - N * H) / H
+    x = 0.45 * (sms - N * H) / H
     g = mc - int(mc * x / (1 + x))
     return g if 0 < g < mc else None
 
