@@ -243,6 +243,19 @@ def test_intra_chunk_stages_against_chunked_form(cuda_device):
         assert err <= tol[name], f"{name}: rel-L2 {err:.3e}"
 
 
+def test_launch_count_follows_the_stage_rule(cuda_device):
+    """Two stages (5 launches) while N * H is below the SM count, one stage (3) from there on,
+    2 when there are no tokens (chunk table and recurrence only), 0 without units."""
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    assert kda.fwd_launch_count(32768, 96, 1) == 5
+    assert kda.fwd_launch_count(32768, sms, 1) == 3
+    assert kda.fwd_launch_count(4096, 32, 8) == (3 if 32 * 8 >= sms else 5)
+    assert kda.fwd_launch_count(0, 4, 1) == 2
+    assert kda.fwd_launch_count(100, 0, 1) == 0
+    assert kda.fwd_launch_count(100, 4, 0) == 0
+    assert kda.fwd_launch_count(64, 1, 1) == 3  # a single chunk: nothing to cut
+
+
 def test_many_short_documents(cuda_device):
     """1100 documents of 0..70 tokens: the per-sequence chunk table spans two 1024-wide scan
     blocks, and many chunks end a document part-way."""
