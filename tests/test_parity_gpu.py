@@ -83,6 +83,23 @@ def test_prefill_sampled_heads(cuda_device, impl):
     check(o[:, :, heads], s[:, heads], o_ref, s_ref, f"prefill/{impl}")
 
 
+@pytest.mark.parametrize("T,H", [(8192, 64), (4096, 160)])
+def test_other_head_counts_sampled(cuda_device, T, H):
+    """One long sequence at 64 heads (two stages, another cut) and at 160 heads (more units than
+    SMs: one stage); the oracle recomputes three heads over the whole sequence."""
+    x = kda_inputs.make_random("t", [T], H, seed=35, state_std=0.1, device=cuda_device)
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    assert kda.fwd_launch_count(T, H, 1) == (5 if H < sms else 3)
+    o, s = run_gpu(x, "chunked")
+    heads = [0, H // 2, H - 1]
+    sl = lambda t: t[:, :, heads].contiguous().cpu()
+    o_ref, s_ref = oracle.kda_fwd(sl(x.q), sl(x.k), sl(x.v), sl(x.g), sl(x.beta), x.scale,
+                                  x.A_log[heads].cpu(), x.dt_bias[heads].cpu(), x.lower_bound,
+                                  initial_state=x.initial_state[:, heads].cpu(),
+                                  cu_seqlens=x.cu_seqlens.cpu())
+    check(o[:, :, heads], s[:, heads], o_ref, s_ref, f"T={T} H={H}")
+
+
 def test_chunk_tails_and_empty_documents(cuda_device):
     lens = [1, 2, 15, 16, 17, 0, 63, 64, 65, 0, 127, 128, 129, 200]
     x = kda_inputs.make_random("t", lens, 2, seed=21, state_std=0.2)
