@@ -32,6 +32,7 @@
 //
 // Every wait is bounded (kWaitLimitNs of wall time): on expiry the kernel records
 // KDA_ERR_DEVICE_TIMEOUT in the workspace status word and the affected work is skipped.
+#include <type_traits>
 #include "kda_device.cuh"
 
 namespace kda {
@@ -326,7 +327,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 
     const float gate_a = __expf(p.A_log[h]);
     const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-    const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
+    // exp(-a (g + dt)) = exp2(ga g + gb); ga < 0 strictly, so that a row past the document end,
+    // loaded as g = -inf, gets x = +inf, log alpha = 0 and alpha = 1 with no select
+    const float ga0 = -gate_a * kLog2e;
+    const float ga = (ga0 > -1e-30f) ? -1e-30f : ga0;  // (a NaN stays NaN)
     const float2 ga2 = splat2(ga);
     const float2 gb2[2] = {make_float2(ga * dtb.x, ga * dtb.y), make_float2(ga * dtb.z, ga * dtb.w)};
     uint2 gr[8];
@@ -334,7 +338,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       const __nv_bfloat16* gp = p.g + ((size_t)(t0 + 8 * iw) * H + h) * D + 4 * lane;
       const uint32_t row_stride = (uint32_t)H * D;  // elements between consecutive tokens
 #pragma unroll
-      for (int i = 0; i < 8; ++i) gr[i] = (8 * iw + i < len) ? ldg_u2(gp + i * row_stride) : make_uint2(0, 0);
+      for (int i = 0; i < 8; ++i) gr[i] = (8 * iw + i < len) ? ldg_u2(gp + i * row_stride) : make_uint2(0xFF80FF80u, 0xFF80FF80u);
     }
     const float beta_raw =
         (8 * iw + (lane & 7) < len)
@@ -380,7 +384,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
         const float2 x = fma2(ga2, gv[m], gb2[m]);
         const float2 d = fma2(make_float2(ex2_approx(x.x), ex2_approx(x.y)), splat2(1.f), splat2(1.f));
         const float2 y = mul2(splat2(lb2), make_float2(rcp_approx(d.x), rcp_approx(d.y)));
-        a2[i][m] = valid ? make_float2(ex2_approx(y.x), ex2_approx(y.y)) : make_float2(1.f, 1.f);
+        a2[i][m] = make_float2(ex2_approx(y.x), ex2_approx(y.y));
       }
     }
     // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
@@ -497,50 +501,56 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       }
     }
     // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end; Ktil goes
-    // straight to the item (same swizzled image as a shared-memory MN tile)
+    // straight to the item (same swizzled image as a shared-memory MN tile).  Specialised on the
+    // warp's row block B, which writes R_B .. R_3
     {
-      float2 post[2], cI[4][2];
-      {
-        float2 bJ[4][2];
-        load_bJ(bJ);
+      float2 bJ[4][2];
+      load_bJ(bJ);
+      uint8_t* kt_dst = item + IT_KT + kb * 8192;
+      auto pass2 = [&](auto nb) {
+        constexpr int B = decltype(nb)::value;
+        float2 post[2], cI[4][2];
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
           float2 z = make_float2(1.f, 1.f);
 #pragma unroll
-          for (int J = 0; J < 4; ++J)
-            if (J > blk) z = mul2(z, bJ[J][m]);
+          for (int J = B + 1; J < 4; ++J) z = mul2(z, bJ[J][m]);
           post[m] = z;
+          cI[B][m] = make_float2(1.0f / bJ[B][m].x, 1.0f / bJ[B][m].y);
           float2 mm = make_float2(1.f, 1.f);
 #pragma unroll
-          for (int I = 0; I < 4; ++I) {
-            cI[I][m] = (I == blk) ? make_float2(1.0f / bJ[blk][m].x, 1.0f / bJ[blk][m].y) : mm;
-            if (I > blk) mm = mul2(mm, bJ[I][m]);
+          for (int I = B + 1; I < 4; ++I) {
+            cI[I][m] = mm;
+            mm = mul2(mm, bJ[I][m]);
           }
         }
-      }
-      float2 run[2];
+        float2 run[2];
 #pragma unroll
-      for (int m = 0; m < 2; ++m) run[m] = upper_half ? make_float2(1.f, 1.f) : pt[m];
-      uint8_t* kt_dst = item + IT_KT + kb * 8192;
+        for (int m = 0; m < 2; ++m) run[m] = upper_half ? make_float2(1.f, 1.f) : pt[m];
 #pragma unroll
-      for (int i = 7; i >= 0; --i) {
-        const float2 kv[2] = {unpack_bf16(kr[i].x), unpack_bf16(kr[i].y)};
-        const float2 ik = splat2(__shfl_sync(0xffffffffu, inv_s, 16 + 2 * i));
-        float2 kr_f[2], kf[2];
+        for (int i = 7; i >= 0; --i) {
+          const float2 kv[2] = {unpack_bf16(kr[i].x), unpack_bf16(kr[i].y)};
+          const float2 ik = splat2(__shfl_sync(0xffffffffu, inv_s, 16 + 2 * i));
+          float2 kr_f[2], kf[2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          kr_f[m] = mul2(kv[m], run[m]);  // raw k * f, shared by R (normalised) and Ktil
-          kf[m] = mul2(kr_f[m], ik);      // khat * f
+          for (int m = 0; m < 2; ++m) {
+            kr_f[m] = mul2(kv[m], run[m]);  // raw k * f, shared by R (normalised) and Ktil
+            kf[m] = mul2(kr_f[m], ik);      // khat * f
+          }
+#pragma unroll
+          for (int I = B; I < 4; ++I)
+            sts64(a_r + row_off(I) * 128 + xo(i), bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
+          *reinterpret_cast<uint2*>(kt_dst + xo(i)) =
+              make_uint2(bf16x2_of(mul2(kr_f[0], post[0])), bf16x2_of(mul2(kr_f[1], post[1])));
+#pragma unroll
+          for (int m = 0; m < 2; ++m) run[m] = mul2(run[m], a2[i][m]);
         }
-#pragma unroll
-        for (int I = 0; I < 4; ++I) {
-          if (I < blk) continue;
-          sts64(a_r + row_off(I) * 128 + xo(i), bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
-        }
-        *reinterpret_cast<uint2*>(kt_dst + xo(i)) =
-            make_uint2(bf16x2_of(mul2(kr_f[0], post[0])), bf16x2_of(mul2(kr_f[1], post[1])));
-#pragma unroll
-        for (int m = 0; m < 2; ++m) run[m] = mul2(run[m], a2[i][m]);
+      };
+      switch (blk) {
+        case 0: pass2(std::integral_constant<int, 0>()); break;
+        case 1: pass2(std::integral_constant<int, 1>()); break;
+        case 2: pass2(std::integral_constant<int, 2>()); break;
+        default: pass2(std::integral_constant<int, 3>()); break;
       }
     }
     fence_proxy_async();
