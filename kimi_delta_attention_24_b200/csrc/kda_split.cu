@@ -327,10 +327,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 
     const float gate_a = __expf(p.A_log[h]);
     const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-    // exp(-a (g + dt)) = exp2(ga g + gb); ga < 0 strictly, so that a row past the document end,
-    // loaded as g = -inf, gets x = +inf, log alpha = 0 and alpha = 1 with no select
-    const float ga0 = -gate_a * kLog2e;
-    const float ga = (ga0 > -1e-30f) ? -1e-30f : ga0;  // (a NaN stays NaN)
+    const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
     const float2 ga2 = splat2(ga);
     const float2 gb2[2] = {make_float2(ga * dtb.x, ga * dtb.y), make_float2(ga * dtb.z, ga * dtb.w)};
     uint2 gr[8];
@@ -338,7 +335,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       const __nv_bfloat16* gp = p.g + ((size_t)(t0 + 8 * iw) * H + h) * D + 4 * lane;
       const uint32_t row_stride = (uint32_t)H * D;  // elements between consecutive tokens
 #pragma unroll
-      for (int i = 0; i < 8; ++i) gr[i] = (8 * iw + i < len) ? ldg_u2(gp + i * row_stride) : make_uint2(0xFF80FF80u, 0xFF80FF80u);
+      for (int i = 0; i < 8; ++i) gr[i] = (8 * iw + i < len) ? ldg_u2(gp + i * row_stride) : make_uint2(0, 0);
     }
     const float beta_raw =
         (8 * iw + (lane & 7) < len)
@@ -384,7 +381,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
         const float2 x = fma2(ga2, gv[m], gb2[m]);
         const float2 d = fma2(make_float2(ex2_approx(x.x), ex2_approx(x.y)), splat2(1.f), splat2(1.f));
         const float2 y = mul2(splat2(lb2), make_float2(rcp_approx(d.x), rcp_approx(d.y)));
-        a2[i][m] = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+        a2[i][m] = valid ? make_float2(ex2_approx(y.x), ex2_approx(y.y)) : make_float2(1.f, 1.f);
       }
     }
     // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the

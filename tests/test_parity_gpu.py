@@ -304,12 +304,15 @@ def test_saturated_gates_and_extreme_beta(cuda_device):
 def test_extreme_gate_parameters(cuda_device):
     # A_log = -inf: exp(A_log) = 0 and log alpha = lb / 2 on every channel; A_log = -100: exp(A_log)
     # is below float range on the GPU and the gate is sigmoid(0) there too; A_log = 30: every gate
-    # saturates at log alpha = lb or 0.  Document lengths leave partial last chunks, whose masked
-    # rows must still get alpha = 1 (their gate input is driven to -inf, whatever A_log is).
+    # saturates at log alpha = lb or 0; dt_bias = +inf / -inf on some channels of head 3: log alpha
+    # = lb / 0 there.  Document lengths leave partial last chunks, whose masked rows must still get
+    # alpha = 1 whatever the gate parameters are.
     x = kda_inputs.make_random("t", [100, 37, 200], 4, seed=31, state_std=0.1)
     x.A_log[0] = float("-inf")
     x.A_log[1] = -100.0
     x.A_log[2] = 30.0
+    x.dt_bias[3, :16] = float("inf")
+    x.dt_bias[3, 16:24] = float("-inf")
     o_ref, s_ref = oracle.fwd_inputs(x)
     assert np.isfinite(o_ref).all() and np.isfinite(s_ref).all()
     for impl in IMPLS:
