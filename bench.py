@@ -36,12 +36,12 @@ T_TOK, HEADS, D = 32768, 96, 128
 CHUNK = 64
 BYTES_PER_TOKEN_HEAD = 4 * 2 * D + 2 + 2 * D          # q, k, v, g in; raw beta in; o out
 FLOPS_PER_TOKEN_HEAD = 6 * D * D + 2 * CHUNK * D + 3 * 2 * CHUNK * D + 2 * CHUNK * D + CHUNK * CHUNK // 3
-STATE_OUT_BYTES_PER_UNIT = D * D * 4                  # fp32 final state written; initial state is zero (NULL)
+STATE_OUT_BYTES_PER_UNIT = D * D * 4                  # fp32 final state per (sequence, head); initial state is zero (NULL)
 WORKLOAD = "prefill B=1 T=32768 H=96 K=V=128 bf16, lower_bound=-5, zero initial state, final state out"
 
 
-def algorithmic_bytes(tokens, heads, units):
-    return BYTES_PER_TOKEN_HEAD * tokens * heads + STATE_OUT_BYTES_PER_UNIT * units
+def algorithmic_bytes(tokens, heads, seqs):
+    return BYTES_PER_TOKEN_HEAD * tokens * heads + STATE_OUT_BYTES_PER_UNIT * seqs * heads
 
 
 def load_peaks():
