@@ -15,7 +15,8 @@
  * batch-mode call (cu_seqlens = None) follow "What CUDA Version Is Required to Use FlashKDA?",
  * section Usage Examples.  This C ABI adds explicit sizes and a stream.
  *
- * Layouts (all contiguous, row-major, device memory, every pointer 16-byte aligned):
+ * Layouts (all contiguous, row-major, device memory; q, k, v, g, out, dt_bias and the states
+ * 16-byte aligned, beta 2-byte, A_log and cu_seqlens 4-byte; batch * seqlen < 2^31 tokens):
  *   q, k, g   bf16  [batch, seqlen, H, K]      (packed varlen: batch = 1, seqlen = total tokens)
  *   v, out    bf16  [batch, seqlen, H, V]
  *   beta      bf16  [batch, seqlen, H]          raw, before the sigmoid

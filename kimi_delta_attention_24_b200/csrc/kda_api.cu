@@ -41,6 +41,7 @@ kda_status_t validate(const void* q, const void* k, const void* v, const void* g
     shape->num_seqs = batch;
   }
   shape->total_tokens = (int64_t)batch * seqlen;
+  if (shape->total_tokens > INT32_MAX) return KDA_ERR_INVALID_ARGUMENT;  // token coordinates are int32
   if ((int64_t)shape->num_seqs * num_heads > INT32_MAX) return KDA_ERR_INVALID_ARGUMENT;
   return KDA_OK;
 }

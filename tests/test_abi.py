@@ -96,6 +96,8 @@ def test_host_validation(lib, name):
     assert call(lib, name, N=3) == 1                # batch mode: N must equal batch
     assert call(lib, name, scale=float("inf")) == 1
     assert call(lib, name, s0=P + 4) == 1
+    assert call(lib, name, beta=P + 1) == 1         # beta needs 2-byte alignment
+    assert call(lib, name, batch=4, seqlen=1 << 30, N=4) == 1  # 2^32 tokens: int32 token coordinates
 
 
 def test_workspace_checks(lib):
