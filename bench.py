@@ -154,6 +154,50 @@ def replica_throughput(token_heads_per_rank, ms_per_step, world):
     return world * token_heads_per_rank / (ms_per_step * 1e-3) / 1e6
 
 
+DECODE_REQUESTS = 256
+
+
+def bench_decode(dev, steps, warmup, seed=0):
+    """The batched decode step on 256 requests x 96 heads, one token each, states updated in place
+    in a 256-slot pool (3.2 GB, far larger than L2): microseconds per step and achieved HBM GB/s of
+    its algorithmic bytes (state read + written, token inputs and output)."""
+    import kda_inputs
+    import kimi_delta_attention_24_b200 as kda
+
+    B, H = DECODE_REQUESTS, HEADS
+    x = kda_inputs.make_random("decode", None, H, seed=seed, varlen=False, batch=B, seqlen=1, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(seed + 7)
+    pool = torch.randn(B, H, D, D, generator=gen, device=dev) * 0.1
+    idx = torch.randperm(B, generator=gen, device=dev).to(torch.int32)
+    out = torch.empty_like(x.v)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.decode(x.q, x.k, x.v, x.g, x.beta, x.scale, out, x.A_log, x.dt_bias, x.lower_bound, pool, pool, idx,
+                   stream=stream.cuda_stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / steps
+    units = B * H
+    alg = units * (2 * D * D * 4 + BYTES_PER_TOKEN_HEAD)
+    hbm_peak, _, peak_kind = load_peaks()
+    gbs = alg / (us * 1e-6) / 1e9
+    return {"workload": f"decode: {B} requests x {H} heads, 1 token each, fp32 states in place in a {B}-slot pool",
+            "us_per_step": us, "requests_per_s": B / (us * 1e-6),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
+                         "bytes_per_unit": 2 * D * D * 4 + BYTES_PER_TOKEN_HEAD},
+            "gpu_launches": steps, "l2": "state pool (3.2 GB) exceeds L2; no flush"}
+
+
 def cpu_oracle_sample(target_s=15.0):
     """Times the fp64 oracle on a bounded sample of the prefill: the first m heads over the
     first L tokens, sized from a short calibration to take about target_s seconds."""
@@ -210,6 +254,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
     ap.add_argument("--heads", type=int, default=HEADS,
                     help="heads of the prefill workload (default 96; fewer only for small profiling runs)")
     args = ap.parse_args()
@@ -360,6 +405,8 @@ def main():
         "clocks": clk.summary(),
         "device_status": status,
     }
+    if not args.no_decode:
+        line["decode"] = bench_decode(dev, steps=max(args.steps, 10), warmup=args.warmup, seed=rank)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

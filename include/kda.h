@@ -38,7 +38,7 @@
  * word and the affected work is skipped — read it with kda_read_device_status.  The contents of
  * cu_seqlens live on the device, so they are checked there: unless 0 = cu[0] <= cu[1] <= ... <=
  * cu[N] = seqlen, the kernels record KDA_ERR_INVALID_ARGUMENT in the status word, never read or
- * write outside the T tokens, and kda_fwd treats every document as empty (out is not written,
+ * write outside the T tokens, and treat every document as empty (out is not written,
  * final_state receives initial_state).
  */
 #ifndef KDA_B200_H_
@@ -63,6 +63,21 @@ typedef enum {
   KDA_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
   KDA_ERR_DEVICE_TIMEOUT = 5      /* a bounded device-side wait ran out (see kda_read_device_status) */
 } kda_status_t;
+
+/* Input-transform flags (fla chunk_kda's use_gate_in_kernel, use_qk_l2norm_in_kernel and
+ * use_beta_sigmoid_in_kernel, as listed in "What CUDA Version Is Required to Use FlashKDA?",
+ * Usage Examples; 0 means all three transforms run in the kernel, as in kda_fwd).
+ *   KDA_FLAG_GATE_PRECOMPUTED  g holds fp32 log alpha [tokens, H, K] (natural log, <= 0): the safe
+ *                              gate is not applied and A_log / dt_bias are not read (may be NULL).
+ *                              kda_fwd_ex clamps it to [lower_bound, 0] (the safe-gate range);
+ *                              kda_decode uses it as given.
+ *   KDA_FLAG_NO_QK_L2NORM      q and k are used as given (no L2 normalisation).
+ *   KDA_FLAG_BETA_PRECOMPUTED  beta holds fp32 beta [tokens, H] (no sigmoid). */
+enum {
+  KDA_FLAG_GATE_PRECOMPUTED = 1,
+  KDA_FLAG_NO_QK_L2NORM = 2,
+  KDA_FLAG_BETA_PRECOMPUTED = 4
+};
 
 /* 1 when (head_dim, dtype, lower_bound) is a configuration this library runs: head_dim = 128,
  * bf16 inputs (dtype_is_bf16 != 0) and -5 <= lower_bound <= 0; otherwise 0.  Mirrors
@@ -106,6 +121,22 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g,
                      int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
                      kda_stream_t stream);
 
+/* kda_fwd with the input transforms selectable (fla chunk_kda's use_gate_in_kernel,
+ * use_qk_l2norm_in_kernel and use_beta_sigmoid_in_kernel; "What CUDA Version Is Required to Use
+ * FlashKDA?", Usage Examples): `flags` is a combination of the KDA_FLAG_* values, 0 giving
+ * kda_fwd.  With KDA_FLAG_GATE_PRECOMPUTED, g is fp32 log alpha [batch, seqlen, H, K] (16-byte
+ * aligned), A_log and dt_bias may be NULL, and each log alpha is clamped to [lower_bound, 0] (the
+ * range whose per-16-token exponent span the chunked kernels keep inside float range); with
+ * KDA_FLAG_BETA_PRECOMPUTED beta is fp32 [batch, seqlen, H] (4-byte aligned).  Same workspace,
+ * layouts and errors as kda_fwd otherwise. */
+kda_status_t kda_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        float scale, void* out, void* workspace, size_t workspace_bytes,
+                        const float* A_log, const float* dt_bias, float lower_bound,
+                        const float* initial_state, float* final_state, const int32_t* cu_seqlens,
+                        int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
+                        int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed, uint32_t flags,
+                        kda_stream_t stream);
+
 /* The same operation evaluated token by token on CUDA cores (one thread per state column):
  * no chunking, no tensor cores.  Same arguments, layouts and errors as kda_fwd (the workspace
  * may be NULL with workspace_bytes = 0).  It is the GPU restatement of the recurrence and the
@@ -121,16 +152,20 @@ kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, cons
 /* kda_fwd for callers that cannot allocate device memory (for example runtimes that plan every
  * device buffer ahead of time and forbid libraries from calling cudaMalloc, or code that must not
  * trigger cudaMalloc's device-wide synchronisation).  The pages have no counterpart to this entry
- * point.  Same arguments as kda_fwd, minus the workspace: it uses a device array that lives in the
- * library (16.6 KB per GPU, held until the process exits) and allocates nothing.  That array holds
- * no per-chunk intermediates, so it runs the fused single-kernel path (one CTA per (sequence,
- * head), every intermediate on chip): results agree with kda_fwd's to rounding, and it is slower
- * on long prefills.
- *   - At most 4096 (sequence, head) units per call; more returns KDA_ERR_WORKSPACE_TOO_SMALL.
+ * point.  Same arguments as kda_fwd, minus the workspace: its scratch is a 256-byte device array
+ * that lives in the library (held by every GPU that loads it until the process exits), and it
+ * allocates nothing.  That array holds no per-chunk intermediates, so it runs the fused
+ * single-kernel path (one CTA per (sequence, head), every intermediate on chip): results agree
+ * with kda_fwd's to rounding, and it is slower on long prefills.
+ *   - At most 4096 (sequence, head) units per call, a fixed limit of this entry point; more
+ *     returns KDA_ERR_WORKSPACE_TOO_SMALL.  Arguments are validated first (the same checks and
+ *     codes as kda_fwd), and a rejected call enqueues nothing.
  *   - The first call on a device looks up the array's address on that device; make it before any
  *     stream capture.
  *   - All calls share the array: calls that overlap on the GPU race on it.
- *   - Each call clears the array's status word; device time-outs are not reported by this call. */
+ *   - Each accepted call clears the array's status word, which is not reported: device time-outs
+ *     and out-of-order cu_seqlens go unreported here.  Out-of-order offsets still get kda_fwd's
+ *     empty-document rule (out not written, final_state = initial_state). */
 kda_status_t kda_fwd_static_workspace(const void* q, const void* k, const void* v, const void* g,
                                       const void* beta, float scale, void* out, const float* A_log,
                                       const float* dt_bias, float lower_bound,
@@ -140,9 +175,42 @@ kda_status_t kda_fwd_static_workspace(const void* q, const void* k, const void* 
                                       int32_t num_seqs, int32_t state_transposed,
                                       kda_stream_t stream);
 
+/* One recurrent step of a batch of requests, each advancing its own state in a state pool by
+ * `seqlen` tokens (1 for plain decoding, a few for speculative tokens): the decode path that
+ * serves Kimi-K3 beside the chunked prefill (vLLM PR #54859 report, sections 风险与影响 and
+ * 关联脉络).  For each (request b, head h) and each of its tokens in order:
+ *     S <- Diag(alpha) S;  delta = beta (v - S^T khat);  S <- S + khat delta^T;  o = scale S^T qhat
+ * with the same in-kernel transforms as kda_fwd unless `flags` switches them off (see the
+ * KDA_FLAG_* values).  Runs on CUDA cores, one CTA per (request, head), state in registers; bound
+ * by the state's HBM traffic (64 KB read + 64 KB written per unit).
+ *   q, k, v, out   bf16 [batch, seqlen, H, 128];  g bf16 [batch, seqlen, H, 128] (fp32 with
+ *                  KDA_FLAG_GATE_PRECOMPUTED);  beta bf16 [batch, seqlen, H] (fp32 with
+ *                  KDA_FLAG_BETA_PRECOMPUTED);  A_log fp32 [H], dt_bias fp32 [H, 128].
+ *   state_in / state_out  fp32 pools [num_slots, H, 128, 128] (S[k][v], or S^T with
+ *                  state_transposed = 1).  state_in NULL means zero states; state_out NULL means
+ *                  no write; they may be the same pool (in-place update).
+ *   state_indices  int32 [batch]: the pool slot of each request; NULL means slot b for request b.
+ *                  A negative index skips the request (nothing read or written: padding).  The
+ *                  non-negative indices of one call must be distinct.  An index >= num_slots
+ *                  also skips the request and records KDA_ERR_INVALID_ARGUMENT in the workspace
+ *                  status word when a workspace is given.
+ *   workspace      optional (NULL allowed): a device buffer of at least 256 bytes, 256-byte
+ *                  aligned, whose first 4 bytes are the sticky status word read by
+ *                  kda_read_device_status.
+ * Errors as kda_fwd (lower_bound is checked only when the gate is computed in the kernel).
+ * Pointers to q, k, v, g, out and the pools are 16-byte aligned, beta 2-byte (4 if fp32). */
+kda_status_t kda_decode(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        float scale, void* out, const float* A_log, const float* dt_bias,
+                        float lower_bound, const float* state_in, float* state_out,
+                        const int32_t* state_indices, int32_t batch, int32_t seqlen,
+                        int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int64_t num_slots,
+                        int32_t state_transposed, uint32_t flags, void* workspace,
+                        kda_stream_t stream);
+
 /* Synchronises `stream`, reads the workspace's sticky status word, clears it, and returns
  * KDA_OK or the recorded device error: KDA_ERR_DEVICE_TIMEOUT (a bounded wait ran out; reported
- * first when both are recorded) or KDA_ERR_INVALID_ARGUMENT (cu_seqlens out of order).
+ * first when both are recorded) or KDA_ERR_INVALID_ARGUMENT (cu_seqlens out of order, or a decode
+ * state index past the pool).
  * KDA_ERR_CUDA if the copy fails. */
 kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream);
 

@@ -9,6 +9,8 @@ PyTorch supplies device memory and the current stream.
     is_supported(head_dim, dtype, lower_bound)
     chunk_kda(q, k, v, g, beta, ...) -> (out, final_state)  # fla-style, allocates outputs
     fwd_recurrent(...)                                     # token-serial CUDA-core kernel
+    decode(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
+           state_in, state_out, state_indices)             # batched recurrent step on a state pool
 
 The argument order of ``fwd`` follows FlashKDA's ``fwd`` as printed in the vLLM PR #54859 report
 (test_flashkda_near_collinear_keys_remain_finite); ``chunk_kda`` follows the fla call on the page
@@ -22,7 +24,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["fwd", "fwd_recurrent", "get_workspace_size", "fwd_launch_count", "new_workspace",
+__all__ = ["fwd", "fwd_recurrent", "decode", "FLAG_GATE_PRECOMPUTED", "FLAG_NO_QK_L2NORM",
+           "FLAG_BETA_PRECOMPUTED", "get_workspace_size", "fwd_launch_count", "new_workspace",
            "is_supported", "chunk_kda", "read_device_status", "selftest_wait_timeout", "KDAError",
            "library_path", "load"]
 
@@ -32,6 +35,12 @@ _lib = None
 
 _STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARGUMENT", 2: "KDA_ERR_UNSUPPORTED",
            3: "KDA_ERR_WORKSPACE_TOO_SMALL", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_DEVICE_TIMEOUT"}
+
+
+# input-transform flags (include/kda.h: KDA_FLAG_*)
+FLAG_GATE_PRECOMPUTED = 1   # g holds fp32 log alpha
+FLAG_NO_QK_L2NORM = 2       # q, k used as given
+FLAG_BETA_PRECOMPUTED = 4   # beta holds fp32 beta
 
 
 class KDAError(RuntimeError):
@@ -59,6 +68,11 @@ def load():
         fn = getattr(lib, name)
         fn.argtypes = fwd_args
         fn.restype = ctypes.c_int
+    lib.kda_fwd_ex.argtypes = fwd_args[:-1] + [ctypes.c_uint32, vp]
+    lib.kda_fwd_ex.restype = ctypes.c_int
+    lib.kda_decode.argtypes = [vp, vp, vp, vp, vp, f32, vp, vp, vp, f32, vp, vp, vp, i32, i32, i32, i32, i32,
+                               i64, i32, ctypes.c_uint32, vp, vp]
+    lib.kda_decode.restype = ctypes.c_int
     lib.kda_workspace_size.argtypes = [i64, i32, i32]
     lib.kda_workspace_size.restype = ctypes.c_size_t
     lib.kda_fwd_launch_count.argtypes = [i64, i32, i32]
@@ -113,11 +127,13 @@ def _check(t: Optional[torch.Tensor], name: str, dtype, device):
 
 
 def _call(fn_name, q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
-          initial_state, final_state, cu_seqlens, state_transposed, stream):
+          initial_state, final_state, cu_seqlens, state_transposed, stream, flags=0):
     lib = load()
     dev = q.device
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (out, "out")):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
         _check(t, n, torch.bfloat16, dev)
+    _check(g, "g", torch.float32 if flags & FLAG_GATE_PRECOMPUTED else torch.bfloat16, dev)
+    _check(beta, "beta", torch.float32 if flags & FLAG_BETA_PRECOMPUTED else torch.bfloat16, dev)
     for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (initial_state, "initial_state"),
                  (final_state, "final_state")):
         _check(t, n, torch.float32, dev)
@@ -131,21 +147,25 @@ def _call(fn_name, q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lowe
     N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
-    with torch.cuda.device(dev):
-        st = getattr(lib, fn_name)(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(out), _ptr(workspace),
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(out), _ptr(workspace),
             0 if workspace is None else workspace.numel(), _ptr(A_log), _ptr(dt_bias), float(lower_bound),
             _ptr(initial_state), _ptr(final_state), _ptr(cu_seqlens), B, T, H, K, V, N,
-            int(bool(state_transposed)), ctypes.c_void_p(stream))
+            int(bool(state_transposed))]
+    if fn_name == "kda_fwd_ex":
+        args.append(int(flags))
+    with torch.cuda.device(dev):
+        st = getattr(lib, fn_name)(*args, ctypes.c_void_p(stream))
     if st != 0:
         raise KDAError(st, fn_name)
 
 
 def fwd(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
-        initial_state=None, final_state=None, cu_seqlens=None, state_transposed=False, stream=None):
-    """The chunked forward (tcgen05 kernel).  Writes ``out`` and ``final_state`` in place."""
-    _call("kda_fwd", q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
-          initial_state, final_state, cu_seqlens, state_transposed, stream)
+        initial_state=None, final_state=None, cu_seqlens=None, state_transposed=False, stream=None,
+        flags=0):
+    """The chunked forward (tcgen05 kernels).  Writes ``out`` and ``final_state`` in place.
+    ``flags`` (FLAG_*) switches input transforms off (kda_fwd_ex); 0 is kda_fwd."""
+    _call("kda_fwd_ex" if flags else "kda_fwd", q, k, v, g, beta, scale, out, workspace, A_log, dt_bias,
+          lower_bound, initial_state, final_state, cu_seqlens, state_transposed, stream, flags)
 
 
 def fwd_recurrent(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
@@ -154,6 +174,43 @@ def fwd_recurrent(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower
     """The token-serial CUDA-core kernel (same contract as ``fwd``)."""
     _call("kda_fwd_recurrent", q, k, v, g, beta, scale, out, workspace, A_log, dt_bias,
           lower_bound, initial_state, final_state, cu_seqlens, state_transposed, stream)
+
+
+def decode(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound, state_in=None, state_out=None,
+           state_indices=None, state_transposed=False, flags=0, workspace=None, stream=None):
+    """Batched recurrent step: request b advances pool slot ``state_indices[b]`` (b when None;
+    negative: skipped) by its ``T`` tokens and writes ``out`` in place.
+
+    q, k, v, out: bf16 [B, T, H, 128] (or [B, H, 128] for one token); g: bf16 raw gate, or fp32 log
+    alpha with FLAG_GATE_PRECOMPUTED; beta: bf16 [B, T, H] raw, or fp32 beta with
+    FLAG_BETA_PRECOMPUTED; state pools fp32 [slots, H, 128, 128] (state_in may be state_out)."""
+    lib = load()
+    if q.dim() == 3:
+        q, k, v, out, g = (t.unsqueeze(1) for t in (q, k, v, out, g))
+        beta = beta.unsqueeze(1)
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check(t, n, torch.bfloat16, dev)
+    _check(g, "g", torch.float32 if flags & FLAG_GATE_PRECOMPUTED else torch.bfloat16, dev)
+    _check(beta, "beta", torch.float32 if flags & FLAG_BETA_PRECOMPUTED else torch.bfloat16, dev)
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, torch.float32, dev)
+    _check(state_indices, "state_indices", torch.int32, dev)
+    if workspace is not None:
+        _check(workspace, "workspace", torch.uint8, dev)
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    pool = state_out if state_out is not None else state_in
+    slots = pool.shape[0] if pool is not None else B
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = lib.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(out),
+                            _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(state_in), _ptr(state_out),
+                            _ptr(state_indices), B, T, H, K, V, slots, int(bool(state_transposed)),
+                            int(flags), _ptr(workspace), ctypes.c_void_p(stream))
+    if st != 0:
+        raise KDAError(st, "kda_decode")
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
@@ -177,19 +234,31 @@ def selftest_wait_timeout(workspace: torch.Tensor, limit_us: int = 2000, stream=
 
 def chunk_kda(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=False,
               A_log=None, dt_bias=None, lower_bound=-5.0, cu_seqlens=None,
-              transpose_state_layout=False, recurrent=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """fla-style call with the in-kernel L2 norm, beta sigmoid and safe gate always on.
+              transpose_state_layout=False, recurrent=False, use_gate_in_kernel=True,
+              use_qk_l2norm_in_kernel=True, use_beta_sigmoid_in_kernel=True,
+              safe_gate=True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """fla-style call (flags as in the chunk_kda usage example).
 
+    ``use_gate_in_kernel=False``: ``g`` is fp32 log alpha (the safe gate already applied);
+    ``use_qk_l2norm_in_kernel=False``: q and k are used as given; ``use_beta_sigmoid_in_kernel=False``:
+    ``beta`` is fp32 beta.  ``safe_gate`` must stay True (the chunked kernels rely on the lower bound).
     Returns ``(out, final_state)``; ``final_state`` is None unless ``output_final_state``.
     With ``transpose_state_layout`` the states are [N, H, V, K] (S transposed)."""
+    if not safe_gate:
+        raise ValueError("safe_gate=False is not supported: the chunked kernels need lower_bound")
+    flags = ((0 if use_gate_in_kernel else FLAG_GATE_PRECOMPUTED)
+             | (0 if use_qk_l2norm_in_kernel else FLAG_NO_QK_L2NORM)
+             | (0 if use_beta_sigmoid_in_kernel else FLAG_BETA_PRECOMPUTED))
+    if recurrent and flags:
+        raise ValueError("the token-serial kernel runs the in-kernel transforms only")
     B, T, H, K = q.shape
     V = v.shape[-1]
     N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
     if scale is None:
         scale = K ** -0.5
-    if A_log is None:
+    if A_log is None and use_gate_in_kernel:
         A_log = torch.zeros(H, dtype=torch.float32, device=q.device)
-    if dt_bias is None:
+    if dt_bias is None and use_gate_in_kernel:
         dt_bias = torch.zeros(H, K, dtype=torch.float32, device=q.device)
     out = torch.empty_like(v)
     final = None
@@ -197,7 +266,10 @@ def chunk_kda(q, k, v, g, beta, scale=None, initial_state=None, output_final_sta
         shape = (N, H, V, K) if transpose_state_layout else (N, H, K, V)
         final = torch.empty(shape, dtype=torch.float32, device=q.device)
     ws = new_workspace(B * T, H, N, q.device)
-    fn = fwd_recurrent if recurrent else fwd
-    fn(q, k, v, g, beta, scale, out, ws, A_log, dt_bias, lower_bound, initial_state, final,
-       cu_seqlens, state_transposed=transpose_state_layout)
+    if recurrent:
+        fwd_recurrent(q, k, v, g, beta, scale, out, ws, A_log, dt_bias, lower_bound, initial_state, final,
+                      cu_seqlens, state_transposed=transpose_state_layout)
+    else:
+        fwd(q, k, v, g, beta, scale, out, ws, A_log, dt_bias, lower_bound, initial_state, final,
+            cu_seqlens, state_transposed=transpose_state_layout, flags=flags)
     return out, final

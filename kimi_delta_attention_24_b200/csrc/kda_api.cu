@@ -19,17 +19,21 @@ kda_status_t validate(const void* q, const void* k, const void* v, const void* g
                       const float* initial_state, const float* final_state,
                       const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
                       int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
-                      int32_t state_transposed, float scale, Shape* shape) {
+                      int32_t state_transposed, float scale, Shape* shape, uint32_t flags = 0) {
   if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
   if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !g || !beta || !out || !A_log || !dt_bias) return KDA_ERR_INVALID_ARGUMENT;
+  if ((flags & ~kda::kFlagMask) != 0) return KDA_ERR_INVALID_ARGUMENT;
+  const bool gate_in_kernel = !(flags & kda::kFlagGatePrecomputed);
+  if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_INVALID_ARGUMENT;
+  if (gate_in_kernel && (!A_log || !dt_bias)) return KDA_ERR_INVALID_ARGUMENT;
   if (batch < 0 || seqlen < 0 || num_heads <= 0 || num_seqs < 0) return KDA_ERR_INVALID_ARGUMENT;
   if (state_transposed != 0 && state_transposed != 1) return KDA_ERR_INVALID_ARGUMENT;
   if (!isfinite(scale)) return KDA_ERR_INVALID_ARGUMENT;
   const void* vec[] = {q, k, v, g, out};
   for (const void* p : vec)
     if (!aligned(p, 16)) return KDA_ERR_INVALID_ARGUMENT;
-  if (!aligned(beta, 2) || !aligned(A_log, 4) || !aligned(dt_bias, 16)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!aligned(beta, (flags & kda::kFlagBetaPrecomputed) ? 4 : 2)) return KDA_ERR_INVALID_ARGUMENT;
+  if (gate_in_kernel && (!aligned(A_log, 4) || !aligned(dt_bias, 16))) return KDA_ERR_INVALID_ARGUMENT;
   if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
     return KDA_ERR_INVALID_ARGUMENT;
   if (cu_seqlens) {
@@ -81,16 +85,21 @@ kda_status_t kda::fwd_fused(const void* q, const void* k, const void* v, const v
                             const float* initial_state, float* final_state, const int32_t* cu_seqlens,
                             int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
                             int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed, uint32_t* status,
-                            cudaStream_t stream) {
+                            int64_t max_units, cudaStream_t stream) {
   Shape shape;
   kda_status_t st = validate(q, k, v, g, beta, out, A_log, dt_bias, lower_bound, initial_state,
                              final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k,
                              head_dim_v, num_seqs, state_transposed, scale, &shape);
   if (st != KDA_OK) return st;
+  const int64_t units = (int64_t)shape.num_seqs * num_heads;
+  if (units > max_units) return KDA_ERR_WORKSPACE_TOO_SMALL;
+  if (!status) return KDA_ERR_INVALID_ARGUMENT;
+  if (units == 0) return KDA_OK;
   kda::FwdParams p = make_params(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
                                  initial_state, final_state, cu_seqlens, seqlen, num_heads,
                                  shape.num_seqs, state_transposed, status);
-  if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
+  // stream-ordered: a time-out recorded by an earlier call does not leak into this one
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), stream) != cudaSuccess) return KDA_ERR_CUDA;
   return kda::launch_chunked(p, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -109,17 +118,17 @@ int kda_fwd_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_se
   return kda::split_launch_count(total_tokens, num_heads, num_seqs);
 }
 
-kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                     float scale, void* out, void* workspace, size_t workspace_bytes,
-                     const float* A_log, const float* dt_bias, float lower_bound,
-                     const float* initial_state, float* final_state, const int32_t* cu_seqlens,
-                     int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
-                     int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
-                     kda_stream_t stream) {
+kda_status_t kda_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        float scale, void* out, void* workspace, size_t workspace_bytes,
+                        const float* A_log, const float* dt_bias, float lower_bound,
+                        const float* initial_state, float* final_state, const int32_t* cu_seqlens,
+                        int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
+                        int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed, uint32_t flags,
+                        kda_stream_t stream) {
   Shape shape;
   kda_status_t st = validate(q, k, v, g, beta, out, A_log, dt_bias, lower_bound, initial_state,
                              final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k,
-                             head_dim_v, num_seqs, state_transposed, scale, &shape);
+                             head_dim_v, num_seqs, state_transposed, scale, &shape, flags);
   if (st != KDA_OK) return st;
   if (!workspace || !aligned(workspace, 256)) return KDA_ERR_INVALID_ARGUMENT;
   if (workspace_bytes < kda_workspace_size(shape.total_tokens, num_heads, shape.num_seqs))
@@ -127,9 +136,22 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g,
   kda::FwdParams p = make_params(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
                                  initial_state, final_state, cu_seqlens, seqlen, num_heads,
                                  shape.num_seqs, state_transposed, static_cast<uint32_t*>(workspace));
+  p.flags = flags;
   if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
   return kda::launch_split(p, workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
                                                                                                  : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                     float scale, void* out, void* workspace, size_t workspace_bytes,
+                     const float* A_log, const float* dt_bias, float lower_bound,
+                     const float* initial_state, float* final_state, const int32_t* cu_seqlens,
+                     int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
+                     int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
+                     kda_stream_t stream) {
+  return kda_fwd_ex(q, k, v, g, beta, scale, out, workspace, workspace_bytes, A_log, dt_bias, lower_bound,
+                    initial_state, final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v,
+                    num_seqs, state_transposed, 0u, stream);
 }
 
 kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, const void* g,
@@ -154,6 +176,41 @@ kda_status_t kda_fwd_recurrent(const void* q, const void* k, const void* v, cons
              : KDA_ERR_CUDA;
 }
 
+kda_status_t kda_decode(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        float scale, void* out, const float* A_log, const float* dt_bias,
+                        float lower_bound, const float* state_in, float* state_out,
+                        const int32_t* state_indices, int32_t batch, int32_t seqlen,
+                        int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int64_t num_slots,
+                        int32_t state_transposed, uint32_t flags, void* workspace,
+                        kda_stream_t stream) {
+  if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
+  if ((flags & ~kda::kFlagMask) != 0) return KDA_ERR_INVALID_ARGUMENT;
+  const bool gate_in_kernel = !(flags & kda::kFlagGatePrecomputed);
+  if (gate_in_kernel && !(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_INVALID_ARGUMENT;
+  if (gate_in_kernel && (!A_log || !dt_bias)) return KDA_ERR_INVALID_ARGUMENT;
+  if (batch < 0 || seqlen < 0 || num_heads <= 0 || num_slots < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (state_transposed != 0 && state_transposed != 1) return KDA_ERR_INVALID_ARGUMENT;
+  if (!isfinite(scale)) return KDA_ERR_INVALID_ARGUMENT;
+  const void* vec[] = {q, k, v, g, out};
+  for (const void* p : vec)
+    if (!aligned(p, 16)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!aligned(beta, (flags & kda::kFlagBetaPrecomputed) ? 4 : 2)) return KDA_ERR_INVALID_ARGUMENT;
+  if (gate_in_kernel && (!aligned(A_log, 4) || !aligned(dt_bias, 16))) return KDA_ERR_INVALID_ARGUMENT;
+  if ((state_in && !aligned(state_in, 16)) || (state_out && !aligned(state_out, 16)))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (state_indices && !aligned(state_indices, 4)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!state_indices && (state_in || state_out) && num_slots < batch) return KDA_ERR_INVALID_ARGUMENT;
+  if (workspace && !aligned(workspace, 256)) return KDA_ERR_INVALID_ARGUMENT;
+  if ((int64_t)batch * seqlen > INT32_MAX || (int64_t)batch * num_heads > INT32_MAX)
+    return KDA_ERR_INVALID_ARGUMENT;
+  return kda::launch_decode(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound, state_in, state_out,
+                            state_indices, batch, seqlen, num_heads, num_slots, state_transposed, flags,
+                            static_cast<uint32_t*>(workspace), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
 kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream) {
   if (!workspace) return KDA_ERR_INVALID_ARGUMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -166,7 +223,7 @@ kda_status_t kda_read_device_status(void* workspace, kda_stream_t stream) {
     if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
   }
   if (word & kda::kStatusTimeout) return KDA_ERR_DEVICE_TIMEOUT;
-  return (word & kda::kStatusBadSeqlens) ? KDA_ERR_INVALID_ARGUMENT : KDA_OK;
+  return (word & (kda::kStatusBadSeqlens | kda::kStatusBadIndex)) ? KDA_ERR_INVALID_ARGUMENT : KDA_OK;
 }
 
 kda_status_t kda_selftest_wait_timeout(void* workspace, uint32_t limit_us, kda_stream_t stream) {

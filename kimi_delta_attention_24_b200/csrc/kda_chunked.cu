@@ -945,8 +945,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = blockIdx.x / H, h = blockIdx.x % H;
   int64_t bos, eos;
   seq_range(p, n, bos, eos);
-  const int nchunks = (int)((eos - bos + C - 1) / C);
   if (tid == 0 && h == 0 && p.status && !seq_entries_ok(p, n)) atomicOr(p.status, kStatusBadSeqlens);
+  // offsets out of order: every document is empty (as in the split path), so no two units can
+  // write the same output rows
+  if (!cta_seqlens_ok(p)) eos = bos;
+  const int nchunks = (int)((eos - bos + C - 1) / C);
 
   if (tid == 0) {
     for (int b = 0; b < B_COUNT; ++b) mbar_init(S_.bar + b, 1);

@@ -15,6 +15,13 @@ constexpr float kL2Eps = 1e-6f;      // inside the square root of the q/k L2 nor
 // Device status word (first 4 bytes of the workspace), sticky until read by the host.
 constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusBadSeqlens = 2u;  // cu_seqlens not ordered as 0 = cu[0] <= ... <= cu[N] = T
+constexpr uint32_t kStatusBadIndex = 4u;    // a decode state index at or past the pool's slot count
+
+// Input-transform flags (public values in kda.h).
+constexpr uint32_t kFlagGatePrecomputed = KDA_FLAG_GATE_PRECOMPUTED;  // g holds fp32 log alpha
+constexpr uint32_t kFlagNoQkL2Norm = KDA_FLAG_NO_QK_L2NORM;           // q, k used as given
+constexpr uint32_t kFlagBetaPrecomputed = KDA_FLAG_BETA_PRECOMPUTED;  // beta holds fp32 beta
+constexpr uint32_t kFlagMask = kFlagGatePrecomputed | kFlagNoQkL2Norm | kFlagBetaPrecomputed;
 constexpr size_t kWorkspaceHeader = 256;  // status word + padding; the rest is per-unit tables
 
 // Arguments of one forward call, after host-side validation.
@@ -37,6 +44,7 @@ struct FwdParams {
   float lower_bound;
   int32_t state_transposed;
   uint32_t* status;            // workspace status word, may be null (recurrent path)
+  uint32_t flags = 0;          // kFlag* input transforms switched off (split path only)
 };
 
 // Token range [bos, eos) of sequence n, clamped to the call's T tokens so that a malformed
@@ -61,6 +69,17 @@ __device__ __forceinline__ bool seq_entries_ok(const FwdParams& p, int n) {
   return b <= e && (n > 0 || b == 0) && (n + 1 < p.num_seqs || e == p.seqlen);
 }
 
+// Whether every entry of cu_seqlens is in order, computed by the whole CTA (every thread must call
+// it, with the same answer for all).  Kernels that own one (sequence, head) unit per CTA use it to
+// apply the empty-document rule: when the offsets do not tile the T tokens in order, every document
+// is treated as empty (no token read, no output row written, final state = initial state).
+__device__ __forceinline__ bool cta_seqlens_ok(const FwdParams& p) {
+  bool bad = false;
+  if (p.cu_seqlens)
+    for (int n = threadIdx.x; n < p.num_seqs; n += blockDim.x) bad |= !seq_entries_ok(p, n);
+  return __syncthreads_or(bad) == 0;
+}
+
 // Launchers (defined in the kernel translation units).  Return the launch's cudaError_t.
 cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 // The fused single-kernel chunked path (one CTA per (sequence, head); needs only the status word).
@@ -69,15 +88,23 @@ cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream);
 size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+// The batched recurrent decode step (kda_decode).
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+                          void* out, const float* A_log, const float* dt_bias, float lower_bound,
+                          const float* state_in, float* state_out, const int32_t* state_indices, int32_t batch,
+                          int32_t seqlen, int32_t num_heads, int64_t num_slots, int32_t state_transposed,
+                          uint32_t flags, uint32_t* status, cudaStream_t stream);
 // One CTA whose bounded wait on a never-completed phase runs out after limit_ns (self-test).
 cudaError_t launch_wait_timeout(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
 
-// Validates the arguments of a forward call and launches the fused chunked path with `status` as
-// the device status word (used by kda_fwd_static_workspace).
+// Validates the arguments of a forward call, rejects more than max_units (sequence, head) units with
+// KDA_ERR_WORKSPACE_TOO_SMALL, and only then clears the device status word `status` and launches
+// the fused chunked path with it (used by kda_fwd_static_workspace).  A rejected call enqueues
+// nothing.
 kda_status_t fwd_fused(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
                        void* out, const float* A_log, const float* dt_bias, float lower_bound,
                        const float* initial_state, float* final_state, const int32_t* cu_seqlens, int32_t batch,
                        int64_t seqlen, int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
-                       int32_t state_transposed, uint32_t* status, cudaStream_t stream);
+                       int32_t state_transposed, uint32_t* status, int64_t max_units, cudaStream_t stream);
 
 }  // namespace kda

@@ -116,6 +116,21 @@ inline bool make_token_map(CUtensorMap* map, const void* base, int64_t tokens, i
   return r == CUDA_SUCCESS;
 }
 
+// [tokens, H, 128] fp32 viewed as 3-D (channel, head, token); box 64 channels x 1 head x 64 tokens,
+// no swizzle (used only to pull tiles into L2 ahead of plain loads).
+inline bool make_token_map_f32(CUtensorMap* map, const void* base, int64_t tokens, int H) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)H, (cuuint64_t)(tokens > 0 ? tokens : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 4, (cuuint64_t)H * kHeadDim * 4};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kChunk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Number of SMs of the current device (looked up once per device); 0 on error.
 inline int sm_count() {
   static int cache[64] = {};

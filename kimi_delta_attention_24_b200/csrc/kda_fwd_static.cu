@@ -5,23 +5,26 @@
 // runtimes that plan every device buffer ahead of time and forbid libraries from calling
 // cudaMalloc, or code that must not pay cudaMalloc's implicit device-wide synchronisation.  They
 // still own their inputs and outputs, but have nowhere to put kda_fwd's workspace.  This entry
-// point uses a workspace that lives in the library itself: a file-scope device array, allocated
-// once when the library's device code is loaded on a GPU and held by that GPU until the process
-// exits.  That array cannot hold the per-chunk intermediates of kda_fwd's split path (about 81 KB
-// per chunk and head), so this entry point runs the fused single-kernel chunked path, which keeps
-// every intermediate on chip and needs only the status word; its results agree with kda_fwd's to
-// rounding.
+// point uses scratch that lives in the library itself: a file-scope device array, allocated once
+// when the library's device code is loaded on a GPU and held by that GPU until the process exits.
+// That array cannot hold the per-chunk intermediates of kda_fwd's split path (about 81 KB per
+// chunk and head), so this entry point runs the fused single-kernel chunked path, which keeps
+// every intermediate on chip; its only scratch is the device status word (the first 4 bytes of
+// the array; the rest of its 256 bytes pads it to the status-header size the kernels expect).
 //
 // Limits and behaviour:
-//   - The array holds the workspace of at most kStaticMaxUnits (sequence, head) units; larger
-//     problems are rejected with KDA_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+//   - At most kStaticMaxUnits (sequence, head) units per call, a fixed limit of this entry point:
+//     every CTA of the fused kernel scans all N + 1 offsets of cu_seqlens to apply the
+//     empty-document rule, so the limit also bounds that scan.  Larger problems are rejected with
+//     KDA_ERR_WORKSPACE_TOO_SMALL after the arguments have been validated and before anything is
+//     enqueued.
 //   - The array's device address is looked up once per device, on the first call made with that
 //     device current (cudaGetSymbolAddress).  Make that first call before any stream capture.
 //   - Every call shares the one array.  Calls whose kernels overlap on the GPU race on it; issue
 //     them on one stream, or otherwise order them.
-//   - Each call clears the array's status word first (stream-ordered), so a device-side time-out
-//     recorded by an earlier call does not leak into the next; the status itself is not reported
-//     to the caller by this entry point.
+//   - Each call clears the status word (stream-ordered) after validation, so a device-side time-out
+//     or malformed-offsets flag recorded by an earlier call does not leak into the next; the status
+//     itself is not reported to the caller by this entry point.
 //   - Nothing here calls cudaMalloc, cudaFree or any allocating library routine.
 #include <mutex>
 
@@ -30,7 +33,7 @@
 namespace {
 
 constexpr int32_t kStaticMaxUnits = 4096;
-constexpr size_t kStaticWorkspaceBytes = kda::kWorkspaceHeader + (size_t)kStaticMaxUnits * sizeof(int32_t);
+constexpr size_t kStaticWorkspaceBytes = kda::kWorkspaceHeader;
 
 static __device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceBytes];
 
@@ -61,15 +64,10 @@ extern "C" kda_status_t kda_fwd_static_workspace(
     float* final_state, const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
     int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
     kda_stream_t stream) {
-  const int64_t seqs = cu_seqlens ? (int64_t)num_seqs : (int64_t)batch;
-  if (seqs < 0 || num_heads < 0) return KDA_ERR_INVALID_ARGUMENT;
-  if (seqs * (int64_t)num_heads > kStaticMaxUnits) return KDA_ERR_WORKSPACE_TOO_SMALL;
   void* ws = nullptr;
-  kda_status_t st = static_workspace_address(&ws);
+  kda_status_t st = static_workspace_address(&ws);  // host-side lookup; writes no device memory
   if (st != KDA_OK) return st;
-  if (cudaMemsetAsync(ws, 0, kda::kWorkspaceHeader, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return KDA_ERR_CUDA;
   return kda::fwd_fused(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound, initial_state, final_state,
                         cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v, num_seqs, state_transposed,
-                        static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
+                        static_cast<uint32_t*>(ws), kStaticMaxUnits, reinterpret_cast<cudaStream_t>(stream));
 }

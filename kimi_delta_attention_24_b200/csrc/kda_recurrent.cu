@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(kVSlice) recurrent_kernel(FwdParams p) {
   seq_range(p, n, bos, eos);
   if (tid == 0 && h == 0 && blockIdx.y == 0 && p.status && !seq_entries_ok(p, n))
     atomicOr(p.status, kStatusBadSeqlens);
+  // offsets out of order: every document is empty, as in the chunked paths
+  if (!cta_seqlens_ok(p)) eos = bos;
 
   const size_t state_off = ((size_t)n * H + h) * (size_t)K * V;
   float S[K];

@@ -185,6 +185,10 @@ __device__ __forceinline__ uint32_t bf16x2_of(float2 v) { return bf16x2(v.x, v.y
 //             the off-diagonal blocks column by column on 3xTF32 mma.sync, warp-local levels
 //   T_b       hi + lo split; MMA PT: P T_b (hi + lo), read back as a hi + lo pair
 //   MMA Xk    [0; I] Qtil + [T_b; P T_b] (-XK) = [-W; Qtil - P W] in one accumulator -> bf16 image
+// kGatePre: g holds fp32 log alpha (the safe gate is not applied; values are clamped to
+// [lower_bound, 0], the range the exponent referencing relies on).  The other input flags (no q/k
+// L2 norm, fp32 beta) are uniform run-time branches.
+template <bool kGatePre>
 __global__ void __launch_bounds__(kIntraThreads, 2)
     intra_kernel(const __grid_constant__ IntraMaps maps, const SplitArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -325,22 +329,34 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     int64_t nxt = 0;
     if (itid == 32) nxt = args.item_begin + (int64_t)atomicAdd(args.queue, 1ull);
 
-    const float gate_a = __expf(p.A_log[h]);
-    const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-    const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
-    const float2 ga2 = splat2(ga);
-    const float2 gb2[2] = {make_float2(ga * dtb.x, ga * dtb.y), make_float2(ga * dtb.z, ga * dtb.w)};
+    float2 ga2, gb2[2];
     uint2 gr[8];
-    {
+    float4 gf[kGatePre ? 8 : 1];
+    if constexpr (!kGatePre) {
+      const float gate_a = __expf(p.A_log[h]);
+      const float4 dtb = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+      const float ga = -gate_a * kLog2e;  // exp(-a (g + dt)) = exp2(ga g + gb)
+      ga2 = splat2(ga);
+      gb2[0] = make_float2(ga * dtb.x, ga * dtb.y);
+      gb2[1] = make_float2(ga * dtb.z, ga * dtb.w);
       const __nv_bfloat16* gp = p.g + ((size_t)(t0 + 8 * iw) * H + h) * D + 4 * lane;
       const uint32_t row_stride = (uint32_t)H * D;  // elements between consecutive tokens
 #pragma unroll
       for (int i = 0; i < 8; ++i) gr[i] = (8 * iw + i < len) ? ldg_u2(gp + i * row_stride) : make_uint2(0, 0);
+    } else {
+      const float4* gp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.g) +
+                                                         ((size_t)(t0 + 8 * iw) * H + h) * D) + lane;
+      const uint32_t row_stride = (uint32_t)H * (D / 4);  // float4s between consecutive tokens
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        gf[i] = (8 * iw + i < len) ? __ldg(gp + i * row_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float beta_raw =
-        (8 * iw + (lane & 7) < len)
-            ? __bfloat162float(p.beta[(size_t)(t0 + 8 * iw) * H + h + (uint32_t)(lane & 7) * (uint32_t)H])
-            : 0.f;
+    float beta_raw = 0.f;
+    if (8 * iw + (lane & 7) < len) {
+      const size_t bi = (size_t)(t0 + 8 * iw) * H + h + (uint32_t)(lane & 7) * (uint32_t)H;
+      beta_raw = (p.flags & kFlagBetaPrecomputed) ? reinterpret_cast<const float*>(p.beta)[bi]
+                                                  : __bfloat162float(p.beta[bi]);
+    }
 
     // ================================================================ prologue
     if (cta_wait(0, raw_par)) break;
@@ -375,13 +391,23 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       const float2 sq = fma2(q23, q23, mul2(q01, q01)), sk = fma2(k23, k23, mul2(k01, k01));
       ssq[i] = sq.x + sq.y;
       ssk[i] = sk.x + sk.y;
-      const float2 gv[2] = {unpack_bf16(gr[i].x), unpack_bf16(gr[i].y)};
+      if constexpr (!kGatePre) {
+        const float2 gv[2] = {unpack_bf16(gr[i].x), unpack_bf16(gr[i].y)};
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const float2 x = fma2(ga2, gv[m], gb2[m]);
-        const float2 d = fma2(make_float2(ex2_approx(x.x), ex2_approx(x.y)), splat2(1.f), splat2(1.f));
-        const float2 y = mul2(splat2(lb2), make_float2(rcp_approx(d.x), rcp_approx(d.y)));
-        a2[i][m] = valid ? make_float2(ex2_approx(y.x), ex2_approx(y.y)) : make_float2(1.f, 1.f);
+        for (int m = 0; m < 2; ++m) {
+          const float2 x = fma2(ga2, gv[m], gb2[m]);
+          const float2 d = fma2(make_float2(ex2_approx(x.x), ex2_approx(x.y)), splat2(1.f), splat2(1.f));
+          const float2 y = mul2(splat2(lb2), make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+          a2[i][m] = valid ? make_float2(ex2_approx(y.x), ex2_approx(y.y)) : make_float2(1.f, 1.f);
+        }
+      } else {
+        // log alpha clamped to [lower_bound, 0], then alpha = 2^(log2 e * log alpha)
+        const float lg[4] = {gf[i].x, gf[i].y, gf[i].z, gf[i].w};
+        float al[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) al[c] = ex2_approx(fminf(fmaxf(lg[c], p.lower_bound), 0.f) * kLog2e);
+        a2[i][0] = valid ? make_float2(al[0], al[1]) : make_float2(1.f, 1.f);
+        a2[i][1] = valid ? make_float2(al[2], al[3]) : make_float2(1.f, 1.f);
       }
     }
     // row sums of squares: transpose-reduce 16 values over the 32 lanes; lane l ends with the
@@ -412,9 +438,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       const bool b1 = lane & 2;
       float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
       w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
-      inv = rsqrtf(w1 + kL2Eps);
+      inv = (p.flags & kFlagNoQkL2Norm) ? 1.f : rsqrtf(w1 + kL2Eps);
     }
-    const float beta_l = (lane < 8 && 8 * iw + lane < len) ? fast_sigmoid(beta_raw) : 0.f;
+    const float beta_l = (lane < 8 && 8 * iw + lane < len)
+                             ? ((p.flags & kFlagBetaPrecomputed) ? beta_raw : fast_sigmoid(beta_raw))
+                             : 0.f;
     const float inv_s = inv * (lane < 16 ? p.scale : 1.f);  // scale folded into 1/|q|
     {
       const float ikr = __shfl_sync(0xffffffffu, inv, 16 + 2 * (lane & 7));  // 1/|k| of row 8 iw + (lane & 7)
@@ -1289,7 +1317,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
   }
 }
 
-bool g_intra_attr[64] = {};
+bool g_intra_attr[2][64] = {};
 bool g_rec_attr[64] = {};
 
 }  // namespace
@@ -1343,11 +1371,14 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
 
   IntraMaps im;
   RecMaps rm;
+  const bool gate_pre = (p.flags & kFlagGatePrecomputed) != 0;
   if (!make_token_map(&im.q, p.q, tokens, p.num_heads) || !make_token_map(&im.k, p.k, tokens, p.num_heads) ||
-      !make_token_map(&im.g, p.g, tokens, p.num_heads) ||
+      !(gate_pre ? make_token_map_f32(&im.g, p.g, tokens, p.num_heads)
+                 : make_token_map(&im.g, p.g, tokens, p.num_heads)) ||
       !make_token_map(&rm.v, p.v, tokens, p.num_heads) || !make_token_map(&rm.out, p.out, tokens, p.num_heads))
     return cudaErrorInvalidValue;
-  cudaError_t e = set_smem_once(intra_kernel, I_ALLOC, g_intra_attr);
+  auto intra_fn = gate_pre ? intra_kernel<true> : intra_kernel<false>;
+  cudaError_t e = set_smem_once(intra_fn, I_ALLOC, g_intra_attr[gate_pre ? 1 : 0]);
   if (e != cudaSuccess) return e;
   e = set_smem_once(rec_kernel, R_ALLOC, g_rec_attr);
   if (e != cudaSuccess) return e;
@@ -1379,7 +1410,7 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
     a.item_end = en;
     a.queue = queues + q;
     const int64_t grid = en - b < 2 * (int64_t)sms ? en - b : 2 * (int64_t)sms;
-    return launch(intra_kernel, grid, kIntraThreads, I_ALLOC, dependent, im, a);
+    return launch(intra_fn, grid, kIntraThreads, I_ALLOC, dependent, im, a);
   };
   auto rec = [&](int64_t g0, int64_t g1) -> cudaError_t {
     SplitArgs a = args;

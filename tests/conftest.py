@@ -28,3 +28,15 @@ def cuda_device():
     import torch
 
     return torch.device("cuda:0")
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Writes the parity margins the GPU tests recorded (see margins.py) to stderr."""
+    try:
+        from margins import summary_lines
+    except ImportError:
+        return
+    lines = summary_lines()
+    if lines:
+        sys.stderr.write("\n" + "\n".join(lines) + "\n")
+        sys.stderr.flush()

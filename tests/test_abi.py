@@ -118,3 +118,55 @@ def test_python_binding_requires_built_library(tmp_path, monkeypatch):
     monkeypatch.setattr(kda, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         kda.load()
+
+
+def call_decode(lib, **kw):
+    a = dict(q=P, k=P, v=P, g=P, beta=P, scale=0.088, out=P, A_log=P, dt_bias=P, lb=-5.0, s_in=P, s_out=P,
+             idx=None, batch=4, seqlen=1, H=2, K=128, V=128, slots=4, transposed=0, flags=0, ws=None)
+    a.update(kw)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    fn = lib.kda_decode
+    fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int32] * 5 + \
+        [ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    return fn(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]), a["scale"], vp(a["out"]),
+              vp(a["A_log"]), vp(a["dt_bias"]), a["lb"], vp(a["s_in"]), vp(a["s_out"]), vp(a["idx"]),
+              a["batch"], a["seqlen"], a["H"], a["K"], a["V"], a["slots"], a["transposed"], a["flags"],
+              vp(a["ws"]), None)
+
+
+def test_decode_host_validation(lib):
+    assert call_decode(lib, K=64) == 2
+    assert call_decode(lib, lb=-6.0) == 2
+    assert call_decode(lib, q=None) == 1
+    assert call_decode(lib, A_log=None) == 1
+    assert call_decode(lib, out=P + 8) == 1
+    assert call_decode(lib, s_out=P + 4) == 1
+    assert call_decode(lib, flags=8) == 1                      # unknown flag bit
+    assert call_decode(lib, transposed=2) == 1
+    assert call_decode(lib, slots=3) == 1                      # no indices: request b uses slot b
+    assert call_decode(lib, ws=P + 16) == 1                    # workspace must be 256-byte aligned
+    assert call_decode(lib, beta=P + 2, flags=4) == 1          # fp32 beta needs 4-byte alignment
+    assert call_decode(lib, H=0) == 1
+    # a precomputed gate needs neither A_log nor dt_bias, and lower_bound is not checked
+    assert call_decode(lib, A_log=None, dt_bias=None, lb=-9.0, flags=1, batch=0) == 0
+    assert call_decode(lib, batch=0) == 0
+    assert call_decode(lib, seqlen=0) == 0
+
+
+def test_fwd_ex_flags_validation(lib):
+    fn = lib.kda_fwd_ex
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def ex(flags, A_log=P, dt_bias=P, beta=P, lb=-5.0, batch=1):
+        return fn(vp(P), vp(P), vp(P), vp(P), vp(beta), ctypes.c_float(0.088), vp(P), vp(P),
+                  ctypes.c_size_t(1 << 20), vp(A_log), vp(dt_bias), ctypes.c_float(lb), None, None, None,
+                  ctypes.c_int32(batch), ctypes.c_int64(64), ctypes.c_int32(1), ctypes.c_int32(128),
+                  ctypes.c_int32(128), ctypes.c_int32(batch), ctypes.c_int32(0), ctypes.c_uint32(flags), None)
+
+    assert ex(8) == 1                                    # unknown flag bit
+    assert ex(0, A_log=None) == 1                        # the in-kernel gate needs A_log
+    assert ex(1, A_log=None, dt_bias=None, batch=0) == 0  # a precomputed gate does not
+    assert ex(4, beta=P + 2) == 1                        # fp32 beta needs 4-byte alignment
+    assert ex(1, lb=-6.0) == 2                           # the clamp range must still be supported

@@ -9,6 +9,7 @@ import torch
 
 import kda_inputs
 import kimi_delta_attention_24_b200 as kda
+import margins
 import oracle
 
 pytestmark = pytest.mark.gpu
@@ -46,13 +47,18 @@ def run_gpu(x, impl="chunked", state_transposed=False, alias=False, dev="cuda:0"
 
 
 def check(o, s, o_ref, s_ref, what=""):
+    """Asserts the parity tolerances and records the margins (printed at the end of the session)."""
     assert np.isfinite(o).all(), f"{what}: non-finite output"
-    err = np.max(np.abs(o - o_ref))
+    err = np.max(np.abs(o - o_ref)) if o.size else 0.0
     rl = rel_l2(o, o_ref)
-    assert err <= O_MAX_ABS and rl <= O_REL_L2, f"{what}: o max-abs {err:.3e}, rel-L2 {rl:.3e}"
+    rs = None
     if s_ref is not None:
         assert np.isfinite(s).all(), f"{what}: non-finite state"
         rs = rel_l2(s, s_ref)
+    margins.record(what, err, rl, rs)
+    print(f"{what}: o max-abs {err:.3e}, o rel-L2 {rl:.3e}, state rel-L2 {rs if rs is None else f'{rs:.3e}'}")
+    assert err <= O_MAX_ABS and rl <= O_REL_L2, f"{what}: o max-abs {err:.3e}, rel-L2 {rl:.3e}"
+    if rs is not None:
         assert rs <= S_REL_L2, f"{what}: state rel-L2 {rs:.3e}"
     return err, rl
 
@@ -197,27 +203,66 @@ def _swizzled_tile(raw, rows):
     return _bf16_to_f64(u[r, c ^ (r & 7)].reshape(rows, 64))
 
 
-def test_intra_chunk_stages_against_chunked_form(cuda_device):
+def _stage_case(case):
+    """Inputs of the stage-level checks: random documents with a 2-token tail, the first four
+    chunks of the near-collinear stress case, and saturated gates (log alpha = lower_bound on every
+    channel) with beta = 1."""
+    if case == "random":
+        return kda_inputs.make_random("t", [130, 64], 2, seed=41, state_std=0.1)
+    if case == "collinear":
+        x = kda_inputs.make_workload("collinear")
+        T = 256
+        sl = lambda t: t[:, :T].contiguous()
+        return kda_inputs.KDAInputs("collinear256", sl(x.q), sl(x.k), sl(x.v), sl(x.g), sl(x.beta),
+                                    x.A_log, x.dt_bias, x.lower_bound, x.scale, x.initial_state,
+                                    torch.tensor([0, T], dtype=torch.int32))
+    if case == "saturated":
+        x = kda_inputs.make_random("t", [192, 70], 2, seed=42, state_std=0.1)
+        x.g.fill_(60.0)
+        x.beta.fill_(30.0)
+        return x
+    raise KeyError(case)
+
+
+# Stage tolerances (relative L2 against the fp64 chunked form; Qtil - P W against ||Qtil||).
+# Random inputs: bf16 operands and outputs (-W, Qtil - P W, P T_b with P in bf16: a few 1e-3),
+# hi + lo pairs on the fp32 / 3xTF32 solve (T_b: ~6e-5), fp32 scalars (1/|k|: ~4e-8, e^Gamma_C:
+# ~5e-6).  Near-collinear keys: the rows of W beyond the first cancel to a small fraction of the
+# first, so -W keeps bf16's absolute error on a smaller norm, and Qtil - P W cancels almost to
+# zero (hence the norm of its terms); T_b is an fp32-accurate solve whatever the conditioning.
+STAGE_TOL = {
+    "random": {"-W": 1e-2, "Qtil - P W": 1e-2, "T_b": 1e-3, "P T_b": 2e-2, "Ktil": 5e-3,
+               "1/|k|": 1e-6, "e^Gamma_C": 1e-4},
+    "collinear": {"-W": 2e-2, "Qtil - P W": 2e-2, "T_b": 1e-3, "P T_b": 2e-2, "Ktil": 5e-3,
+                  "1/|k|": 1e-6, "e^Gamma_C": 1e-4},
+    "saturated": {"-W": 1e-2, "Qtil - P W": 1e-2, "T_b": 1e-3, "P T_b": 2e-2, "Ktil": 5e-3,
+                  "1/|k|": 1e-6, "e^Gamma_C": 1e-4},
+}
+
+
+@pytest.mark.parametrize("case", ["random", "collinear", "saturated"])
+def test_intra_chunk_stages_against_chunked_form(cuda_device, case):
     """Each intra-chunk output against the fp64 chunked form of the same chunk: -W and Qtil - P W
     (the MMA1 operand), T diag(beta) and P T diag(beta) (hi + lo pairs), Ktil (raw k with the decay
-    to the chunk end), 1/|k| and e^{Gamma_C}; full chunks and a 2-token tail."""
+    to the chunk end), 1/|k| and e^{Gamma_C}; full chunks and partial tails."""
     from oracle.chunked import chunk_intermediates
-    lens, H = [130, 64], 2
-    x = kda_inputs.make_random("t", lens, H, seed=41, state_std=0.1)
+    x = _stage_case(case)
+    H = x.num_heads
+    N = x.num_seqs
     xd = x.to(cuda_device)
-    N = len(lens)
     ws = kda.new_workspace(x.total_tokens, H, N, cuda_device)
     out = torch.empty_like(xd.v)
     kda.fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, x.scale, out, ws, xd.A_log, xd.dt_bias, x.lower_bound,
             None, None, xd.cu_seqlens)
     assert kda.read_device_status(ws) == 0
     raw = ws.cpu().numpy().tobytes()
+    cu = x.cu_seqlens.numpy()
     co = np.frombuffer(raw[_WS_HEADER:_WS_HEADER + 4 * (N + 1)], dtype=np.int32)
-    assert list(co) == [0, 3, 4]
+    assert list(co) == list(np.concatenate([[0], np.cumsum([(int(cu[i + 1] - cu[i]) + 63) // 64
+                                                             for i in range(N)])]))
     items = _WS_HEADER + ((N + 1) * 4 + 1023) // 1024 * 1024
     qh, kh, la, be = oracle.prologue(x.q, x.k, x.g, x.beta, x.A_log, x.dt_bias, x.lower_bound)
     kraw = x.k.double().numpy()
-    cu = x.cu_seqlens.numpy()
     worst = {}
     for n in range(N):
         t0, t1 = int(cu[n]), int(cu[n + 1])
@@ -239,25 +284,30 @@ def test_intra_chunk_stages_against_chunked_form(cuda_device):
                 Tb = ref["T"] * b[None, :]
                 kr = kraw[0, t0 + 64 * c:t0 + 64 * c + L, h]
                 ik_ref = 1.0 / np.sqrt((kr * kr).sum(axis=1) + 1e-6)
+                # (got, want, norm the error is measured against): Qtil - P W is a difference whose
+                # terms cancel on nearly collinear keys (P W predicts Qtil almost exactly), so its
+                # error is measured against the size of its terms, ||Qtil||; the others against
+                # their own size
+                qpw = ref["Qt"] - ref["P"] @ ref["W"]
                 pairs = {
-                    "-W": (wq[:L], -ref["W"]),
-                    "Qtil - P W": (wq[64:64 + L], ref["Qt"] - ref["P"] @ ref["W"]),
-                    "T_b": (tb[:L, :L], Tb),
-                    "P T_b": (tb[64:64 + L, :L], ref["P"] @ Tb),
-                    "Ktil": (kt[:L], ref["Kt"] / ik_ref[:, None]),
-                    "1/|k|": (ik[:L], ik_ref),
-                    "e^Gamma_C": (gam, ref["gC"]),
+                    "-W": (wq[:L], -ref["W"], None),
+                    "Qtil - P W": (wq[64:64 + L], qpw, max(np.linalg.norm(qpw), np.linalg.norm(ref["Qt"]))),
+                    "T_b": (tb[:L, :L], Tb, None),
+                    "P T_b": (tb[64:64 + L, :L], ref["P"] @ Tb, None),
+                    "Ktil": (kt[:L], ref["Kt"] / ik_ref[:, None], None),
+                    "1/|k|": (ik[:L], ik_ref, None),
+                    "e^Gamma_C": (gam, ref["gC"], None),
                 }
                 assert np.all(ik[L:] == 0)  # rows past the end of the document
-                for name, (got, want) in pairs.items():
+                for name, (got, want, nrm) in pairs.items():
                     assert np.isfinite(got).all(), name
-                    worst[name] = max(worst.get(name, 0.0), rel_l2(got, want))
-    # bf16 operands and outputs (-W, Qtil - P W, P T_b with P in bf16: a few 1e-3 measured), hi + lo
-    # pairs on an fp32 solve (T_b: ~6e-5), fp32 scalars (1/|k|: ~4e-8, e^Gamma_C: ~5e-6)
-    tol = {"-W": 1e-2, "Qtil - P W": 1e-2, "T_b": 1e-3, "P T_b": 2e-2, "Ktil": 5e-3, "1/|k|": 1e-6,
-           "e^Gamma_C": 1e-4}
+                    err = rel_l2(got, want) if nrm is None else np.linalg.norm(got - want) / max(nrm, 1e-300)
+                    worst[name] = max(worst.get(name, 0.0), err)
+    print(f"stages/{case}: " + ", ".join(f"{k} {v:.2e}" for k, v in worst.items()))
     for name, err in worst.items():
-        assert err <= tol[name], f"{name}: rel-L2 {err:.3e}"
+        margins.note(f"stage {case} {name}: rel-L2 {err:.2e} (tol {STAGE_TOL[case][name]:.0e})")
+    for name, err in worst.items():
+        assert err <= STAGE_TOL[case][name], f"{case} {name}: rel-L2 {err:.3e}"
 
 
 def test_launch_count_follows_the_stage_rule(cuda_device):
@@ -409,9 +459,9 @@ def test_malformed_cu_seqlens_reported_on_device(cuda_device, bad):
         fn(x.q, x.k, x.v, x.g, x.beta, x.scale, out, ws, x.A_log, x.dt_bias, x.lower_bound,
            x.initial_state, fin, cu_bad)
         assert kda.read_device_status(ws) == 1  # KDA_ERR_INVALID_ARGUMENT
-        if fn is kda.fwd:
-            assert torch.isnan(out).all()
-            assert torch.equal(fin, x.initial_state)
+        # every document is treated as empty, on both paths
+        assert torch.isnan(out).all()
+        assert torch.equal(fin, x.initial_state)
     o_ref, s_ref = oracle.fwd_inputs(x.to("cpu"))
     check(*run_gpu(x.to("cpu")), o_ref, s_ref, "valid call after a malformed one")
 
