@@ -198,6 +198,50 @@ def bench_decode(dev, steps, warmup, seed=0):
             "gpu_launches": steps, "l2": "state pool (3.2 GB) exceeds L2; no flush"}
 
 
+BWD_TOKENS = 4096
+BWD_BYTES_PER_TOKEN_HEAD = BYTES_PER_TOKEN_HEAD + 2 * D + (4 * 2 * D + 2)  # + d_out in; dq, dk, dv, dg, dbeta out
+
+
+def bench_backward(dev, steps, warmup, seed=0):
+    """The backward pass (token-serial on CUDA cores, checkpointed) on the prefill's heads with
+    T = 4096 tokens: milliseconds per step, token-heads/s, and HBM GB/s of its algorithmic bytes
+    (inputs and d_out read once, the five token gradients written once)."""
+    import kda_inputs
+    import kimi_delta_attention_24_b200 as kda
+
+    x = kda_inputs.make_random("bwd", [BWD_TOKENS], HEADS, seed=seed, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(seed + 11)
+    d_out = torch.randn(x.v.shape, generator=gen, device=dev).to(torch.bfloat16)
+    ws = torch.empty(kda.bwd_workspace_size(BWD_TOKENS, HEADS, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.bwd(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, d_out,
+                cu_seqlens=x.cu_seqlens, workspace=ws, stream=stream.cuda_stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    th = BWD_TOKENS * HEADS
+    alg = BWD_BYTES_PER_TOKEN_HEAD * th
+    hbm_peak, _, peak_kind = load_peaks()
+    gbs = alg / (ms * 1e-3) / 1e9
+    return {"workload": f"backward: B=1 T={BWD_TOKENS} H={HEADS} K=V=128, gradients of every input",
+            "ms_per_step": ms, "value": th / (ms * 1e-3) / 1e6, "unit": UNIT,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
+                         "note": "token-serial CUDA-core kernel: bound by its per-token dependency chain, "
+                                 "not by HBM"},
+            "gpu_launches": steps}
+
+
 def cpu_oracle_sample(target_s=15.0):
     """Times the fp64 oracle on a bounded sample of the prefill: the first m heads over the
     first L tokens, sized from a short calibration to take about target_s seconds."""
@@ -255,6 +299,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--heads", type=int, default=HEADS,
                     help="heads of the prefill workload (default 96; fewer only for small profiling runs)")
     args = ap.parse_args()
@@ -407,6 +452,8 @@ def main():
     }
     if not args.no_decode:
         line["decode"] = bench_decode(dev, steps=max(args.steps, 10), warmup=args.warmup, seed=rank)
+    if not args.no_backward:
+        line["backward"] = bench_backward(dev, steps=2, warmup=1, seed=rank)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

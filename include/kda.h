@@ -137,6 +137,32 @@ kda_status_t kda_fwd_ex(const void* q, const void* k, const void* v, const void*
                         int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed, uint32_t flags,
                         kda_stream_t stream);
 
+/* The segment map of every (sequence, head) unit, for sequence-parallel prefill (KCP, the KDA
+ * context parallelism of torchtitan PR #4374): the forward pass is affine in the state a segment
+ * starts from, S_out = M S_in + B, with M (K x K) the product of the segment's per-token
+ * transitions (I - beta khat khat^T) Diag(alpha) and B (K x V) the state reached from zero.  Same
+ * inputs, workspace and flags as kda_fwd_ex (no scale, output or states); writes
+ *   map_M  fp32 [N, H, K, K]   (M[k][k'], row-major; 16-byte aligned)
+ *   map_B  fp32 [N, H, K, V]   (B[k][v])
+ * Runs the chunk table and the intra-chunk kernel once, then one recurrence launch of 2 N H CTAs
+ * (B from v and a zero state; M from v = 0 and the identity state).  An empty sequence gets
+ * M = I, B = 0.  Errors as kda_fwd. */
+kda_status_t kda_segment_map(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                             void* workspace, size_t workspace_bytes, const float* A_log,
+                             const float* dt_bias, float lower_bound, float* map_M, float* map_B,
+                             const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
+                             int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs, uint32_t flags,
+                             kda_stream_t stream);
+
+/* state_out = map_M state_in + map_B for `units` (sequence, head) units of 128 x 128 fp32: the
+ * fold of one segment map over a state (KCP's scan step).  map_M and map_B as kda_segment_map
+ * writes them; state_in / state_out in the layout `state_transposed` selects (S[k][v], or S^T);
+ * state_in NULL means a zero state (then map_M may be NULL too); state_out may alias state_in.
+ * One CTA per unit, fp32 on CUDA cores.  KDA_ERR_UNSUPPORTED for head_dim != 128,
+ * KDA_ERR_INVALID_ARGUMENT for null or misaligned (16-byte) pointers or a bad flag. */
+kda_status_t kda_state_affine(const float* map_M, const float* map_B, const float* state_in, float* state_out,
+                              int64_t units, int32_t head_dim, int32_t state_transposed, kda_stream_t stream);
+
 /* The same operation evaluated token by token on CUDA cores (one thread per state column):
  * no chunking, no tensor cores.  Same arguments, layouts and errors as kda_fwd (the workspace
  * may be NULL with workspace_bytes = 0).  It is the GPU restatement of the recurrence and the
@@ -206,6 +232,34 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const void*
                         int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int64_t num_slots,
                         int32_t state_transposed, uint32_t flags, void* workspace,
                         kda_stream_t stream);
+
+/* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): one fp32
+ * 128 x 128 checkpoint per (64-token chunk, head) for at most T / 64 + N + 1 chunk slots, and a
+ * 64-state scratch for each of up to min(N H, 256) CTAs.  Depends only on its arguments. */
+size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+
+/* The backward pass: gradients of sum(d_out * out) + sum(d_final * final_state) with respect to
+ * every input of kda_fwd (torchtitan trains Kimi-K3 through chunk_kda, and its varlen test checks
+ * the gradient as well as the forward: torchtitan PR #4374, Results).  Same inputs, layouts and
+ * errors as kda_fwd (state_transposed = 0: states and their gradients are [N, H, K, V]), plus
+ *   d_out        bf16 [batch, seqlen, H, V]   the output's gradient
+ *   d_final      fp32 [N, H, K, V] or NULL (zero)   the final state's gradient
+ * and writes
+ *   dq, dk, dg   bf16 [batch, seqlen, H, K];  dv bf16 [batch, seqlen, H, V];  dbeta bf16
+ *                [batch, seqlen, H] (w.r.t. the raw beta, before the sigmoid; dg w.r.t. the raw gate)
+ *   dA_log fp32 [H], ddt_bias fp32 [H, K]  (overwritten: zeroed, then summed over all tokens)
+ *   d_initial    fp32 [N, H, K, V] or NULL (not written)
+ * Token by token on CUDA cores, one persistent CTA per (sequence, head): a forward that stores a
+ * checkpoint every 64 tokens, then chunk by chunk from the last a rerun from the checkpoint and a
+ * reverse walk over its tokens.  Gradient pointers are 16-byte aligned (dbeta 2, dA_log 4).  With
+ * out-of-order cu_seqlens every document is treated as empty: the token gradients are not written
+ * and d_initial = d_final (there is no status word to report it). */
+kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+                     const float* A_log, const float* dt_bias, float lower_bound, const float* initial_state,
+                     const void* d_out, const float* d_final, void* dq, void* dk, void* dv, void* dg, void* dbeta,
+                     float* dA_log, float* ddt_bias, float* d_initial, void* workspace, size_t workspace_bytes,
+                     const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
+                     int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs, kda_stream_t stream);
 
 /* Synchronises `stream`, reads the workspace's sticky status word, clears it, and returns
  * KDA_OK or the recorded device error: KDA_ERR_DEVICE_TIMEOUT (a bounded wait ran out; reported

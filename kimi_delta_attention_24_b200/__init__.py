@@ -24,7 +24,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["fwd", "fwd_recurrent", "decode", "FLAG_GATE_PRECOMPUTED", "FLAG_NO_QK_L2NORM",
+__all__ = ["fwd", "fwd_recurrent", "decode", "segment_map", "state_affine", "bwd", "bwd_workspace_size", "FLAG_GATE_PRECOMPUTED", "FLAG_NO_QK_L2NORM",
            "FLAG_BETA_PRECOMPUTED", "get_workspace_size", "fwd_launch_count", "new_workspace",
            "is_supported", "chunk_kda", "read_device_status", "selftest_wait_timeout", "KDAError",
            "library_path", "load"]
@@ -73,6 +73,16 @@ def load():
     lib.kda_decode.argtypes = [vp, vp, vp, vp, vp, f32, vp, vp, vp, f32, vp, vp, vp, i32, i32, i32, i32, i32,
                                i64, i32, ctypes.c_uint32, vp, vp]
     lib.kda_decode.restype = ctypes.c_int
+    lib.kda_segment_map.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp, f32, vp, vp, vp,
+                                    i32, i64, i32, i32, i32, i32, ctypes.c_uint32, vp]
+    lib.kda_segment_map.restype = ctypes.c_int
+    lib.kda_state_affine.argtypes = [vp, vp, vp, vp, i64, i32, i32, vp]
+    lib.kda_state_affine.restype = ctypes.c_int
+    lib.kda_bwd_workspace_size.argtypes = [i64, i32, i32]
+    lib.kda_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.kda_bwd.argtypes = [vp, vp, vp, vp, vp, f32, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                            ctypes.c_size_t, vp, i32, i64, i32, i32, i32, i32, vp]
+    lib.kda_bwd.restype = ctypes.c_int
     lib.kda_workspace_size.argtypes = [i64, i32, i32]
     lib.kda_workspace_size.restype = ctypes.c_size_t
     lib.kda_fwd_launch_count.argtypes = [i64, i32, i32]
@@ -211,6 +221,88 @@ def decode(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound, state_in=N
                             int(flags), _ptr(workspace), ctypes.c_void_p(stream))
     if st != 0:
         raise KDAError(st, "kda_decode")
+
+
+def segment_map(q, k, v, g, beta, workspace, A_log, dt_bias, lower_bound, map_M, map_B, cu_seqlens=None,
+                flags=0, stream=None):
+    """The affine map S_out = M S_in + B of every (sequence, head) unit's tokens: writes map_M
+    (fp32 [N, H, K, K]) and map_B (fp32 [N, H, K, V]) in place (kda_segment_map)."""
+    lib = load()
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, dev)
+    _check(g, "g", torch.float32 if flags & FLAG_GATE_PRECOMPUTED else torch.bfloat16, dev)
+    _check(beta, "beta", torch.float32 if flags & FLAG_BETA_PRECOMPUTED else torch.bfloat16, dev)
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (map_M, "map_M"), (map_B, "map_B")):
+        _check(t, n, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _check(workspace, "workspace", torch.uint8, dev)
+    B, T, H, K = q.shape
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = lib.kda_segment_map(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(workspace),
+                                 workspace.numel(), _ptr(A_log), _ptr(dt_bias), float(lower_bound),
+                                 _ptr(map_M), _ptr(map_B), _ptr(cu_seqlens), B, T, H, K, v.shape[-1], N,
+                                 int(flags), ctypes.c_void_p(stream))
+    if st != 0:
+        raise KDAError(st, "kda_segment_map")
+
+
+def state_affine(map_M, map_B, state_in, state_out, state_transposed=False, stream=None):
+    """state_out = map_M state_in + map_B per (sequence, head) unit (state_in None: zero state);
+    state_out may be state_in (kda_state_affine)."""
+    lib = load()
+    dev = map_B.device
+    for t, n in ((map_M, "map_M"), (map_B, "map_B"), (state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, torch.float32, dev)
+    units = map_B.numel() // (map_B.shape[-1] * map_B.shape[-2])
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = lib.kda_state_affine(_ptr(map_M), _ptr(map_B), _ptr(state_in), _ptr(state_out), units,
+                                  map_B.shape[-1], int(bool(state_transposed)), ctypes.c_void_p(stream))
+    if st != 0:
+        raise KDAError(st, "kda_state_affine")
+
+
+def bwd_workspace_size(T: int, H: int, N: int) -> int:
+    return int(load().kda_bwd_workspace_size(int(T), int(H), int(N)))
+
+
+def bwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out, initial_state=None, d_final=None,
+        cu_seqlens=None, workspace=None, stream=None):
+    """Gradients of sum(d_out * o) + sum(d_final * final_state) w.r.t. every input (kda_bwd).
+    Returns a dict: dq, dk, dv, dg (bf16, shaped like the inputs), dbeta (bf16, like beta),
+    dA_log [H], ddt_bias [H, K] and d_initial [N, H, K, V] (fp32)."""
+    lib = load()
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (d_out, "d_out")):
+        _check(t, n, torch.bfloat16, dev)
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (initial_state, "initial_state"), (d_final, "d_final")):
+        _check(t, n, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_size(B * T, H, N), dtype=torch.uint8, device=dev)
+    r = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v), "dg": torch.empty_like(g),
+         "dbeta": torch.empty_like(beta), "dA_log": torch.empty(H, dtype=torch.float32, device=dev),
+         "ddt_bias": torch.empty(H, K, dtype=torch.float32, device=dev),
+         "d_initial": torch.empty(N, H, K, V, dtype=torch.float32, device=dev)}
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(A_log), _ptr(dt_bias),
+                         float(lower_bound), _ptr(initial_state), _ptr(d_out), _ptr(d_final), _ptr(r["dq"]),
+                         _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dg"]), _ptr(r["dbeta"]), _ptr(r["dA_log"]),
+                         _ptr(r["ddt_bias"]), _ptr(r["d_initial"]), _ptr(workspace), workspace.numel(),
+                         _ptr(cu_seqlens), B, T, H, K, V, N, ctypes.c_void_p(stream))
+    if st != 0:
+        raise KDAError(st, "kda_bwd")
+    return r
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:

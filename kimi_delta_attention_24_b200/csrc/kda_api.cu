@@ -19,12 +19,13 @@ kda_status_t validate(const void* q, const void* k, const void* v, const void* g
                       const float* initial_state, const float* final_state,
                       const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
                       int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
-                      int32_t state_transposed, float scale, Shape* shape, uint32_t flags = 0) {
+                      int32_t state_transposed, float scale, Shape* shape, uint32_t flags = 0,
+                      bool need_out = true) {
   if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
   if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_UNSUPPORTED;
   if ((flags & ~kda::kFlagMask) != 0) return KDA_ERR_INVALID_ARGUMENT;
   const bool gate_in_kernel = !(flags & kda::kFlagGatePrecomputed);
-  if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_INVALID_ARGUMENT;
+  if (!q || !k || !v || !g || !beta || (need_out && !out)) return KDA_ERR_INVALID_ARGUMENT;
   if (gate_in_kernel && (!A_log || !dt_bias)) return KDA_ERR_INVALID_ARGUMENT;
   if (batch < 0 || seqlen < 0 || num_heads <= 0 || num_seqs < 0) return KDA_ERR_INVALID_ARGUMENT;
   if (state_transposed != 0 && state_transposed != 1) return KDA_ERR_INVALID_ARGUMENT;
@@ -142,6 +143,47 @@ kda_status_t kda_fwd_ex(const void* q, const void* k, const void* v, const void*
                                                                                                  : KDA_ERR_CUDA;
 }
 
+kda_status_t kda_segment_map(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                             void* workspace, size_t workspace_bytes, const float* A_log,
+                             const float* dt_bias, float lower_bound, float* map_M, float* map_B,
+                             const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
+                             int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs, uint32_t flags,
+                             kda_stream_t stream) {
+  Shape shape;
+  kda_status_t st = validate(q, k, v, g, beta, nullptr, A_log, dt_bias, lower_bound, nullptr, nullptr,
+                             cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v, num_seqs, 0, 1.0f,
+                             &shape, flags, /*need_out=*/false);
+  if (st != KDA_OK) return st;
+  if (!map_M || !map_B || !aligned(map_M, 16) || !aligned(map_B, 16)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!workspace || !aligned(workspace, 256)) return KDA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < kda_workspace_size(shape.total_tokens, num_heads, shape.num_seqs))
+    return KDA_ERR_WORKSPACE_TOO_SMALL;
+  kda::FwdParams p = make_params(q, k, v, g, beta, 1.0f, nullptr, A_log, dt_bias, lower_bound, nullptr, nullptr,
+                                 cu_seqlens, seqlen, num_heads, shape.num_seqs, 0,
+                                 static_cast<uint32_t*>(workspace));
+  p.flags = flags;
+  if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
+  return kda::launch_segment_map(p, workspace, map_M, map_B, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_state_affine(const float* map_M, const float* map_B, const float* state_in, float* state_out,
+                              int64_t units, int32_t head_dim, int32_t state_transposed, kda_stream_t stream) {
+  if (head_dim != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
+  if (units < 0 || units > INT32_MAX || (state_transposed != 0 && state_transposed != 1))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (!map_B || !state_out || (state_in && !map_M)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!aligned(map_B, 16) || !aligned(state_out, 16) || (map_M && !aligned(map_M, 16)) ||
+      (state_in && !aligned(state_in, 16)))
+    return KDA_ERR_INVALID_ARGUMENT;
+  return kda::launch_state_affine(map_M, map_B, state_in, state_out, units, state_transposed,
+                                  reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
 kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
                      float scale, void* out, void* workspace, size_t workspace_bytes,
                      const float* A_log, const float* dt_bias, float lower_bound,
@@ -207,6 +249,40 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const void*
   return kda::launch_decode(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound, state_in, state_out,
                             state_indices, batch, seqlen, num_heads, num_slots, state_transposed, flags,
                             static_cast<uint32_t*>(workspace), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
+size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  return kda::bwd_workspace_bytes(total_tokens, num_heads, num_seqs);
+}
+
+kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+                     const float* A_log, const float* dt_bias, float lower_bound, const float* initial_state,
+                     const void* d_out, const float* d_final, void* dq, void* dk, void* dv, void* dg, void* dbeta,
+                     float* dA_log, float* ddt_bias, float* d_initial, void* workspace, size_t workspace_bytes,
+                     const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
+                     int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs, kda_stream_t stream) {
+  Shape shape;
+  kda_status_t st = validate(q, k, v, g, beta, d_out, A_log, dt_bias, lower_bound, initial_state, d_final,
+                             cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v, num_seqs, 0, scale,
+                             &shape);
+  if (st != KDA_OK) return st;
+  if (!dq || !dk || !dv || !dg || !dbeta || !dA_log || !ddt_bias) return KDA_ERR_INVALID_ARGUMENT;
+  const void* vec[] = {dq, dk, dv, dg, ddt_bias};
+  for (const void* p : vec)
+    if (!aligned(p, 16)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!aligned(dbeta, 2) || !aligned(dA_log, 4) || (d_initial && !aligned(d_initial, 16)))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (!workspace || !aligned(workspace, 256)) return KDA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < kda_bwd_workspace_size(shape.total_tokens, num_heads, shape.num_seqs))
+    return KDA_ERR_WORKSPACE_TOO_SMALL;
+  kda::FwdParams p = make_params(q, k, v, g, beta, scale, nullptr, A_log, dt_bias, lower_bound, initial_state,
+                                 nullptr, cu_seqlens, seqlen, num_heads, shape.num_seqs, 0, nullptr);
+  return kda::launch_bwd(p, static_cast<const __nv_bfloat16*>(d_out), d_final, static_cast<__nv_bfloat16*>(dq),
+                         static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv),
+                         static_cast<__nv_bfloat16*>(dg), static_cast<__nv_bfloat16*>(dbeta), dA_log, ddt_bias,
+                         d_initial, workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? KDA_OK
              : KDA_ERR_CUDA;
 }

@@ -88,6 +88,17 @@ cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream);
 size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+// The segment map (M, B) of every unit: the split path with the recurrence in map mode.
+cudaError_t launch_segment_map(const FwdParams& p, void* workspace, float* map_M, float* map_B,
+                               cudaStream_t stream);
+// S_out = M S_in + B for `units` (sequence, head) units (S_in null: zero).
+cudaError_t launch_state_affine(const float* M, const float* B, const float* S_in, float* S_out, int64_t units,
+                                int32_t transposed, cudaStream_t stream);
+// The backward pass (kda_bwd): workspace bytes, and the launch (zeroes dA_log / ddt_bias first).
+size_t bwd_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const float* d_final, __nv_bfloat16* dq,
+                       __nv_bfloat16* dk, __nv_bfloat16* dv, __nv_bfloat16* dg, __nv_bfloat16* dbeta, float* dA_log,
+                       float* ddt_bias, float* d_initial, void* workspace, cudaStream_t stream);
 // The batched recurrent decode step (kda_decode).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
                           void* out, const float* A_log, const float* dt_bias, float lower_bound,

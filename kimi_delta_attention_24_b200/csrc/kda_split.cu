@@ -61,6 +61,12 @@ struct SplitArgs {
   int64_t g0, g1;                // rec_kernel: global chunks [g0, g1) (g1 = INT64_MAX: to the end)
   float* boundary;               // [H][128 * 128] S^T of the one sequence cut between two launches
   unsigned long long* queue;     // intra_kernel: item counter (zeroed by chunk_table_kernel)
+  // rec_kernel map mode (the segment map S_out = M S_in + B of each unit): a grid of 2 N H CTAs;
+  // CTA u < N H computes B (v as given, zero initial state), CTA N H + u computes M (v = 0, identity
+  // initial state); each writes its final state [k][v] to map_B / map_M and no output.
+  int map_mode;
+  float* map_M;                  // [N, H, 128, 128]
+  float* map_B;                  // [N, H, 128, 128]
 };
 
 constexpr int kQueues = 2;  // item counters in the workspace header, one per intra launch
@@ -938,13 +944,18 @@ struct RecMaps {
   CUtensorMap v, out;
 };
 
+// kMap: map mode (see SplitArgs), compiled separately so that the forward's code is unchanged.
+template <bool kMap>
 __global__ void __launch_bounds__(kRecThreads, 1)
     rec_kernel(const __grid_constant__ RecMaps maps, const SplitArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const FwdParams& p = args.p;
   const int H = p.num_heads;
-  const int n = blockIdx.x / H, h = blockIdx.x % H;
+  const int units = p.num_seqs * H;
+  const bool map_part_M = kMap && (int)blockIdx.x >= units;  // map mode: this CTA computes M
+  const int ub = kMap ? (int)blockIdx.x % units : (int)blockIdx.x;
+  const int n = ub / H, h = ub % H;
   int64_t bos, eos;
   seq_range(p, n, bos, eos);
   // launched as a programmatic dependent: let the next launch place its CTAs beside this grid's,
@@ -1002,6 +1013,16 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     // ------------------------------------------------------------ loader (lane 0 issues; the
     // whole warp zeroes the v rows past the end of the sequence in the last chunk)
     int armed[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};  // last chunk armed per (TPV, WQ, KT) stage
+    if (map_part_M) {
+      // M of the segment map: v = 0.  Both stages' v tiles are zeroed once, before the first copy
+      // into either stage is armed, and never loaded
+      for (int idx = lane; idx < 2 * 16384 / 16; idx += 32) {
+        const int st = idx / 1024, off = (idx % 1024) * 16;
+        *reinterpret_cast<uint4*>(sm + R_TPV + st * R_TPV_STAGE + 32768 + off) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async();
+      __syncwarp();
+    }
     for (int c = 0; c < nch; ++c) {
       const int s = c & 1;
       const uint32_t par = ((c >> 1) - 1) & 1;
@@ -1011,13 +1032,15 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         if (c >= 2 && !wait(RB_TPV_EMPTY + s, par)) ok = 0;
         if (ok) {
           armed[0][s] = c;
-          mbar_arrive_expect_tx(bar + RB_TPV_FULL + s, 32768 + 16384 + IT_SC_BYTES);
+          mbar_arrive_expect_tx(bar + RB_TPV_FULL + s, 32768 + (map_part_M ? 0 : 16384) + IT_SC_BYTES);
           bulk_load(sm + R_TPV + s * R_TPV_STAGE, it + IT_TP, 16384, bar + RB_TPV_FULL + s);
           bulk_load(sm + R_TPV + s * R_TPV_STAGE + 16384, it + IT_TL, 16384, bar + RB_TPV_FULL + s);
           bulk_load(sm + R_SC + s * IT_SC_BYTES, it + IT_IK, IT_SC_BYTES, bar + RB_TPV_FULL + s);
-          const int t0 = (int)(bos + (int64_t)c * C);
-          tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 32768, &maps.v, bar + RB_TPV_FULL + s, 0, h, t0);
-          tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 40960, &maps.v, bar + RB_TPV_FULL + s, 64, h, t0);
+          if (!map_part_M) {
+            const int t0 = (int)(bos + (int64_t)c * C);
+            tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 32768, &maps.v, bar + RB_TPV_FULL + s, 0, h, t0);
+            tma_load_3d(sm + R_TPV + s * R_TPV_STAGE + 40960, &maps.v, bar + RB_TPV_FULL + s, 64, h, t0);
+          }
         }
         if (ok && c >= 2 && !wait(RB_WQ_EMPTY + s, par)) ok = 0;
         if (ok) {
@@ -1142,12 +1165,20 @@ __global__ void __launch_bounds__(kRecThreads, 1)
     // its state over in args.boundary (S^T, slot h); each thread stores only what it loaded itself
     const size_t soff = ((size_t)n * H + h) * (size_t)D * D;
     float* const bnd = args.boundary + (size_t)h * D * D;
-    const float* const st_in = state_in_user ? (p.initial_state ? p.initial_state + soff : nullptr) : bnd;
-    float* const st_out = state_out_user ? (p.final_state ? p.final_state + soff : nullptr) : bnd;
-    const bool in_t = state_in_user ? p.state_transposed != 0 : true;
-    const bool out_t = state_out_user ? p.state_transposed != 0 : true;
+    const float* st_in = state_in_user ? (p.initial_state ? p.initial_state + soff : nullptr) : bnd;
+    float* st_out = state_out_user ? (p.final_state ? p.final_state + soff : nullptr) : bnd;
+    bool in_t = state_in_user ? p.state_transposed != 0 : true;
+    bool out_t = state_out_user ? p.state_transposed != 0 : true;
+    if (kMap) {  // one stage: B from a zero state, M from the identity; both stored [k][v]
+      st_in = nullptr;
+      st_out = (map_part_M ? args.map_M : args.map_B) + soff;
+      in_t = out_t = false;
+    }
     auto load_state = [&](float (&x)[32]) {
-      if (!st_in) {
+      if (map_part_M) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = (col0 + j == (uint32_t)v) ? 1.f : 0.f;
+      } else if (!st_in) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = 0.f;
       } else if (in_t) {
@@ -1250,6 +1281,8 @@ __global__ void __launch_bounds__(kRecThreads, 1)
             mbar_arrive(bar + RB_TPV_EMPTY + s);
           }
           named_bar_arrive(kBarOutGo, kEpiThreads);  // the O warps start once Delta^T is out
+        } else if (kMap) {
+          named_bar(kBarOutGo, kEpiThreads);  // no output in map mode
         } else {
           named_bar(kBarOutGo, kEpiThreads);
           float d[32];
@@ -1318,7 +1351,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
 }
 
 bool g_intra_attr[2][64] = {};
-bool g_rec_attr[64] = {};
+bool g_rec_attr[2][64] = {};
 
 }  // namespace
 
@@ -1380,7 +1413,7 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
   auto intra_fn = gate_pre ? intra_kernel<true> : intra_kernel<false>;
   cudaError_t e = set_smem_once(intra_fn, I_ALLOC, g_intra_attr[gate_pre ? 1 : 0]);
   if (e != cudaSuccess) return e;
-  e = set_smem_once(rec_kernel, R_ALLOC, g_rec_attr);
+  e = set_smem_once(rec_kernel<false>, R_ALLOC, g_rec_attr[0]);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
@@ -1416,7 +1449,7 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
     SplitArgs a = args;
     a.g0 = g0;
     a.g1 = g1;
-    return launch(rec_kernel, units, kRecThreads, R_ALLOC, true, rm, a);
+    return launch(rec_kernel<false>, units, kRecThreads, R_ALLOC, true, rm, a);
   };
 
   chunk_table_kernel<<<1, 1024, 0, stream>>>(p, const_cast<int32_t*>(args.chunk_off), queues);
@@ -1431,6 +1464,69 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
   if ((e = rec(0, g_cut)) != cudaSuccess) return e;
   if ((e = intra(g_cut * p.num_heads, items, 1, true)) != cudaSuccess) return e;
   return rec(g_cut, INT64_MAX);
+}
+
+// The segment map of every (sequence, head) unit: chunk table, the intra-chunk kernel over every
+// item (once: the items do not depend on v or on the state), then one recurrence launch of 2 N H
+// CTAs in map mode (B from v and a zero state, M from v = 0 and the identity), as a programmatic
+// dependent of the intra launch.
+cudaError_t launch_segment_map(const FwdParams& p, void* workspace, float* map_M, float* map_B,
+                               cudaStream_t stream) {
+  const int64_t units = (int64_t)p.num_seqs * p.num_heads;
+  if (units == 0) return cudaSuccess;
+  const int64_t tokens = p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs;
+  const int64_t max_chunks = chunk_bound(tokens, p.num_seqs);
+  const int64_t items = max_chunks * p.num_heads;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  SplitArgs args{};
+  args.p = p;
+  args.chunk_off = reinterpret_cast<int32_t*>(ws + kWorkspaceHeader);
+  args.items = ws + kWorkspaceHeader + table_bytes(p.num_seqs);
+  args.boundary = reinterpret_cast<float*>(args.items + (size_t)items * ITEM_BYTES);
+  IntraMaps im;
+  RecMaps rm;
+  const bool gate_pre = (p.flags & kFlagGatePrecomputed) != 0;
+  if (!make_token_map(&im.q, p.q, tokens, p.num_heads) || !make_token_map(&im.k, p.k, tokens, p.num_heads) ||
+      !(gate_pre ? make_token_map_f32(&im.g, p.g, tokens, p.num_heads)
+                 : make_token_map(&im.g, p.g, tokens, p.num_heads)) ||
+      !make_token_map(&rm.v, p.v, tokens, p.num_heads) || !make_token_map(&rm.out, p.v, tokens, p.num_heads))
+    return cudaErrorInvalidValue;  // (no output in map mode: the out map is never used)
+  auto intra_fn = gate_pre ? intra_kernel<true> : intra_kernel<false>;
+  cudaError_t e = set_smem_once(intra_fn, I_ALLOC, g_intra_attr[gate_pre ? 1 : 0]);
+  if (e != cudaSuccess) return e;
+  e = set_smem_once(rec_kernel<true>, R_ALLOC, g_rec_attr[1]);
+  if (e != cudaSuccess) return e;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  unsigned long long* queues = reinterpret_cast<unsigned long long*>(ws + kQueueOffset);
+  chunk_table_kernel<<<1, 1024, 0, stream>>>(p, const_cast<int32_t*>(args.chunk_off), queues);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (items > 0) {
+    SplitArgs a = args;
+    a.item_begin = 0;
+    a.item_end = items;
+    a.queue = queues;
+    const int64_t grid = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
+    intra_fn<<<(unsigned)grid, kIntraThreads, I_ALLOC, stream>>>(im, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  SplitArgs a = args;
+  a.g0 = 0;
+  a.g1 = INT64_MAX;
+  a.map_mode = 1;
+  a.map_M = map_M;
+  a.map_B = map_B;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * units));
+  cfg.blockDim = dim3((unsigned)kRecThreads);
+  cfg.dynamicSmemBytes = R_ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, rec_kernel<true>, rm, a);
 }
 
 int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {

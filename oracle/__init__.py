@@ -56,6 +56,15 @@ def _load():
         lib.kda_oracle_prologue.argtypes = [_u16p, _u16p, _u16p, _u16p, _fp, _fp, ctypes.c_double,
                                             ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _dp, _dp,
                                             _dp, _dp]
+        lib.kda_oracle_fwd_f64.restype = ctypes.c_int
+        lib.kda_oracle_fwd_f64.argtypes = [_dp, _dp, _dp, _dp, _dp, ctypes.c_double, _dp, _dp, ctypes.c_double,
+                                           _dp, _dp, _dp, _i32p, ctypes.c_int32, ctypes.c_int64,
+                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+        lib.kda_oracle_bwd.restype = ctypes.c_int
+        lib.kda_oracle_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, ctypes.c_double, _dp, _dp, ctypes.c_double,
+                                       _dp, _dp, _dp, _i32p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                       ctypes.c_int32, ctypes.c_int32, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
+                                       ctypes.c_int32]
         lib.kda_oracle_core.restype = ctypes.c_int
         lib.kda_oracle_core.argtypes = [_dp, _dp, _dp, _dp, _dp, ctypes.c_double, _dp, _dp, _dp,
                                         _i32p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
@@ -181,3 +190,59 @@ def fwd_inputs(x, num_threads: int = 0, state_transposed: bool = False):
                    initial_state=s0, cu_seqlens=x.cu_seqlens,
                    output_final_state=x.output_final_state, state_transposed=state_transposed,
                    num_threads=num_threads)
+
+
+def kda_fwd_f64(q, k, v, g, beta, scale: float, A_log, dt_bias, lower_bound: float, initial_state=None,
+                cu_seqlens=None):
+    """The forward from fp64 raw inputs (no bf16 widening), states [N, H, K, V]: the function whose
+    finite differences pin ``kda_bwd``.  Returns (o, final_state)."""
+    lib = _load()
+    cu, total, H = _cu_and_shape(tuple(q.shape), cu_seqlens)
+    N = cu.size - 1
+    dk, dv = q.shape[-1], v.shape[-1]
+    qd, kd, vd, gd, bd, al, db = (_f64(x) for x in (q, k, v, g, beta, A_log, dt_bias))
+    s0 = None if initial_state is None else _f64(initial_state)
+    out = np.empty((total, H, dv))
+    sf = np.empty((N, H, dk, dv))
+    rc = lib.kda_oracle_fwd_f64(_ptr(qd, _dp), _ptr(kd, _dp), _ptr(vd, _dp), _ptr(gd, _dp), _ptr(bd, _dp),
+                                float(scale), _ptr(al, _dp), _ptr(db, _dp), float(lower_bound), _ptr(s0, _dp),
+                                _ptr(sf, _dp), _ptr(out, _dp), _ptr(cu, _i32p), int(N), int(total), int(H),
+                                int(dk), int(dv))
+    if rc != 0:
+        raise ValueError("oracle rejected the sizes or cu_seqlens")
+    return out.reshape(tuple(v.shape)), sf
+
+
+def kda_bwd(q, k, v, g, beta, scale: float, A_log, dt_bias, lower_bound: float, d_out, initial_state=None,
+            d_final=None, cu_seqlens=None, num_threads: int = 0):
+    """Gradients of sum(d_out * o) + sum(d_final * S_final) w.r.t. the raw inputs, in fp64 (inputs
+    are taken as fp64 values; bf16 tensors are widened exactly).  Returns a dict with dq, dk, dv, dg
+    (shaped like q), dbeta (like beta), dA_log [H], ddt_bias [H, K] and d_initial [N, H, K, V]."""
+    lib = _load()
+    cu, total, H = _cu_and_shape(tuple(q.shape), cu_seqlens)
+    N = cu.size - 1
+    dk, dv = q.shape[-1], v.shape[-1]
+    qd, kd, vd, gd, bd, al, db = (_f64(x) for x in (q, k, v, g, beta, A_log, dt_bias))
+    s0 = None if initial_state is None else _f64(initial_state)
+    do = _f64(d_out)
+    dF = None if d_final is None else _f64(d_final)
+    r = {n: np.empty((total, H, dk)) for n in ("dq", "dk", "dg")}
+    r["dv"] = np.empty((total, H, dv))
+    r["dbeta"] = np.empty((total, H))
+    r["dA_log"] = np.empty(H)
+    r["ddt_bias"] = np.empty((H, dk))
+    r["d_initial"] = np.empty((N, H, dk, dv))
+    rc = lib.kda_oracle_bwd(_ptr(qd, _dp), _ptr(kd, _dp), _ptr(vd, _dp), _ptr(gd, _dp), _ptr(bd, _dp),
+                            float(scale), _ptr(al, _dp), _ptr(db, _dp), float(lower_bound), _ptr(s0, _dp),
+                            _ptr(do, _dp), _ptr(dF, _dp), _ptr(cu, _i32p), int(N), int(total), int(H), int(dk),
+                            int(dv), _ptr(r["dq"], _dp), _ptr(r["dk"], _dp), _ptr(r["dv"], _dp), _ptr(r["dg"], _dp),
+                            _ptr(r["dbeta"], _dp), _ptr(r["dA_log"], _dp), _ptr(r["ddt_bias"], _dp),
+                            _ptr(r["d_initial"], _dp), int(num_threads))
+    if rc != 0:
+        raise ValueError("oracle rejected the sizes or cu_seqlens")
+    shp = tuple(q.shape)
+    for n in ("dq", "dk", "dg"):
+        r[n] = r[n].reshape(shp)
+    r["dv"] = r["dv"].reshape(tuple(v.shape))
+    r["dbeta"] = r["dbeta"].reshape(shp[:-1])
+    return r

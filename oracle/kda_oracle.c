@@ -237,3 +237,237 @@ int kda_oracle_core(const double* qhat, const double* khat, const double* v, con
     free(pred);
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------------
+ * Backward pass (gradients) — TEST INFRASTRUCTURE ONLY, like everything in this file.
+ *
+ * torchtitan trains through chunk_kda, and its varlen test checks the gradient as well as the
+ * forward (torchtitan PR #4374, Results: test_varlen_matches_independent_documents, "forward and
+ * gradient").  The adjoint below is the reverse-mode derivative of the token recurrence above,
+ * taken step by step in reverse token order.  For one token (with Stil = Diag(alpha) S_{t-1},
+ * p = Stil^T khat, delta = beta (v - p), S_t = Stil + khat delta^T, o_t = scale S_t^T qhat), given
+ * dS (the gradient of the loss w.r.t. S_t, from later tokens and the final state) and do_t:
+ *   dS     += scale qhat do^T                   dqhat  = scale S_t do
+ *   dkhat   = dS delta                          ddelta = dS^T khat
+ *   dbeta   = ddelta . (v - p)                  dv     = beta ddelta,   dp = -beta ddelta
+ *   dStil   = dS + khat dp^T                    dkhat += Stil dp
+ *   dalpha_c = sum_j dStil[c][j] S_{t-1}[c][j]  dS_{t-1} = Diag(alpha) dStil
+ * then back through the in-kernel transforms:
+ *   qhat = q / n (n = sqrt(sum q^2 + eps)):  dq = (dqhat - qhat (qhat . dqhat)) / n   (k alike)
+ *   beta = sigmoid(b):                       db = dbeta beta (1 - beta)
+ *   log alpha = lb sigmoid(x), x = e^A (g + dt):
+ *       dx = dalpha alpha lb sigmoid(x) (1 - sigmoid(x));  dg = dx e^A;  ddt += dx e^A;  dA += dx x
+ * The loss is sum(do * o) + sum(dfinal * S_final); d_initial is the gradient w.r.t. S_0.
+ * Inputs here are fp64 (raw values before the transforms), so that finite differences of
+ * kda_oracle_fwd_f64 can pin the adjoint.
+ * ------------------------------------------------------------------------------------------ */
+
+static void l2_normalize_d(const double* x, int d, double* out, double* norm) {
+    double ss = 0.0;
+    for (int c = 0; c < d; ++c) ss += x[c] * x[c];
+    double n = sqrt(ss + KDA_ORACLE_L2_EPS);
+    for (int c = 0; c < d; ++c) out[c] = x[c] / n;
+    if (norm) *norm = n;
+}
+
+/* Forward pass from fp64 raw inputs (same steps as kda_oracle_fwd; no bf16 widening).  States
+ * are [N,H,dk,dv] (S[k][v]). */
+int kda_oracle_fwd_f64(const double* q, const double* k, const double* v, const double* g,
+                       const double* beta, double scale, const double* A_log, const double* dt_bias,
+                       double lower_bound, const double* initial_state, double* final_state,
+                       double* out, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                       int32_t num_heads, int32_t dk, int32_t dv) {
+    if (dk <= 0 || dv <= 0 || num_heads <= 0 || total_tokens < 0) return 1;
+    if (check_cu(cu_seqlens, num_seqs, total_tokens)) return 1;
+    const size_t state_elems = (size_t)dk * dv;
+    double* S = (double*)malloc(sizeof(double) * state_elems);
+    double* qh = (double*)malloc(sizeof(double) * dk);
+    double* kh = (double*)malloc(sizeof(double) * dk);
+    double* la = (double*)malloc(sizeof(double) * dk);
+    double* pred = (double*)malloc(sizeof(double) * dv);
+    for (int32_t n = 0; n < num_seqs; ++n)
+        for (int32_t h = 0; h < num_heads; ++h) {
+            const size_t soff = ((size_t)n * num_heads + h) * state_elems;
+            load_state(S, initial_state ? initial_state + soff : NULL, 0, dk, dv);
+            const double a = exp(A_log[h]);
+            for (int64_t t = cu_seqlens[n]; t < cu_seqlens[n + 1]; ++t) {
+                const size_t row = (size_t)t * num_heads + h;
+                l2_normalize_d(q + row * dk, dk, qh, NULL);
+                l2_normalize_d(k + row * dk, dk, kh, NULL);
+                for (int c = 0; c < dk; ++c)
+                    la[c] = lower_bound * sigmoid(a * (g[row * dk + c] + dt_bias[(size_t)h * dk + c]));
+                recurrence_step(S, qh, kh, v + row * dv, la, sigmoid(beta[row]), scale, dk, dv, pred,
+                                out + row * dv);
+            }
+            store_state(S, final_state ? final_state + soff : NULL, 0, dk, dv);
+        }
+    free(S); free(qh); free(kh); free(la); free(pred);
+    return 0;
+}
+
+/* Gradients of sum(d_out * o) + sum(d_final * S_final) w.r.t. every input, fp64.  Shapes as
+ * kda_oracle_fwd_f64; d_final may be NULL (zero); dA_log [H] and ddt_bias [H,dk] are summed over
+ * sequences; d_initial [N,H,dk,dv] may be NULL. */
+int kda_oracle_bwd(const double* q, const double* k, const double* v, const double* g,
+                   const double* beta, double scale, const double* A_log, const double* dt_bias,
+                   double lower_bound, const double* initial_state, const double* d_out,
+                   const double* d_final, const int32_t* cu_seqlens, int32_t num_seqs,
+                   int64_t total_tokens, int32_t num_heads, int32_t dk, int32_t dv, double* dq,
+                   double* dkey, double* dval, double* dg, double* dbeta, double* dA_log,
+                   double* ddt_bias, double* d_initial, int32_t num_threads) {
+    if (dk <= 0 || dv <= 0 || num_heads <= 0 || total_tokens < 0) return 1;
+    if (check_cu(cu_seqlens, num_seqs, total_tokens)) return 1;
+    const int64_t units = (int64_t)num_seqs * num_heads;
+    const size_t se = (size_t)dk * dv;
+    /* per-unit partial sums of the per-head parameter gradients, added up after the loop */
+    double* part = (double*)calloc((size_t)(units > 0 ? units : 1) * (1 + dk), sizeof(double));
+    int failed = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(|:failed)
+    for (int64_t u = 0; u < units; ++u) {
+        const int32_t n = (int32_t)(u / num_heads), h = (int32_t)(u % num_heads);
+        const int64_t t0 = cu_seqlens[n], L = cu_seqlens[n + 1] - cu_seqlens[n];
+        const size_t soff = ((size_t)n * num_heads + h) * se;
+        const double ea = exp(A_log[h]);
+        /* the forward, keeping every state and every transformed input */
+        double* hist = (double*)malloc(sizeof(double) * se * (size_t)(L + 1));
+        double* qh = (double*)malloc(sizeof(double) * dk * (size_t)(L > 0 ? L : 1));
+        double* kh = (double*)malloc(sizeof(double) * dk * (size_t)(L > 0 ? L : 1));
+        double* nq = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        double* nk = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        double* xg = (double*)malloc(sizeof(double) * dk * (size_t)(L > 0 ? L : 1));
+        double* la = (double*)malloc(sizeof(double) * dk * (size_t)(L > 0 ? L : 1));
+        double* bt = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        double* pred = (double*)malloc(sizeof(double) * dv);
+        double* otmp = (double*)malloc(sizeof(double) * dv);
+        double* dS = (double*)malloc(sizeof(double) * se);
+        double* dSt = (double*)malloc(sizeof(double) * se);
+        double* St = (double*)malloc(sizeof(double) * se);
+        double* vec = (double*)malloc(sizeof(double) * (4 * (size_t)dk + 4 * (size_t)dv));
+        if (!hist || !qh || !kh || !nq || !nk || !xg || !la || !bt || !pred || !otmp || !dS || !dSt ||
+            !St || !vec) {
+            failed = 1;
+        } else {
+            load_state(hist, initial_state ? initial_state + soff : NULL, 0, dk, dv);
+            for (int64_t i = 0; i < L; ++i) {
+                const size_t row = (size_t)(t0 + i) * num_heads + h;
+                l2_normalize_d(q + row * dk, dk, qh + i * dk, nq + i);
+                l2_normalize_d(k + row * dk, dk, kh + i * dk, nk + i);
+                for (int c = 0; c < dk; ++c) {
+                    xg[i * dk + c] = ea * (g[row * dk + c] + dt_bias[(size_t)h * dk + c]);
+                    la[i * dk + c] = lower_bound * sigmoid(xg[i * dk + c]);
+                }
+                bt[i] = sigmoid(beta[row]);
+                memcpy(hist + (size_t)(i + 1) * se, hist + (size_t)i * se, sizeof(double) * se);
+                recurrence_step(hist + (size_t)(i + 1) * se, qh + i * dk, kh + i * dk, v + row * dv,
+                                la + i * dk, bt[i], scale, dk, dv, pred, otmp);
+            }
+            /* the reverse sweep */
+            double* dqh = vec;
+            double* dkh = vec + dk;
+            double* dal = vec + 2 * (size_t)dk;
+            double* alpha = vec + 3 * (size_t)dk;
+            double* p = vec + 4 * (size_t)dk;
+            double* delta = p + dv;
+            double* ddelta = delta + dv;
+            double* dp = ddelta + dv;
+            for (size_t e = 0; e < se; ++e) dS[e] = d_final ? d_final[soff + e] : 0.0;
+            double* ppart = part + (size_t)u * (1 + dk);
+            for (int64_t i = L - 1; i >= 0; --i) {
+                const size_t row = (size_t)(t0 + i) * num_heads + h;
+                const double* Sp = hist + (size_t)i * se;
+                const double* Sn = hist + (size_t)(i + 1) * se;
+                const double* qi = qh + i * dk;
+                const double* ki = kh + i * dk;
+                const double* doi = d_out + row * dv;
+                const double* vi = v + row * dv;
+                const double b = bt[i];
+                for (int c = 0; c < dk; ++c) alpha[c] = exp(la[i * dk + c]);
+                /* o_t = scale S_t^T qhat */
+                for (int c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        dS[(size_t)c * dv + j] += scale * qi[c] * doi[j];
+                        acc += Sn[(size_t)c * dv + j] * doi[j];
+                    }
+                    dqh[c] = scale * acc;
+                }
+                /* Stil, p, delta */
+                for (int c = 0; c < dk; ++c)
+                    for (int j = 0; j < dv; ++j) St[(size_t)c * dv + j] = alpha[c] * Sp[(size_t)c * dv + j];
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < dk; ++c) acc += St[(size_t)c * dv + j] * ki[c];
+                    p[j] = acc;
+                    delta[j] = b * (vi[j] - acc);
+                }
+                /* S_t = Stil + khat delta^T */
+                for (int c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) acc += dS[(size_t)c * dv + j] * delta[j];
+                    dkh[c] = acc;
+                }
+                double dbt = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < dk; ++c) acc += dS[(size_t)c * dv + j] * ki[c];
+                    ddelta[j] = acc;
+                    dbt += acc * (vi[j] - p[j]);
+                    dval[row * dv + j] = b * acc;
+                    dp[j] = -b * acc;
+                }
+                /* dStil = dS + khat dp^T;  dkhat += Stil dp;  dalpha;  dS_{t-1} = Diag(alpha) dStil */
+                for (int c = 0; c < dk; ++c) {
+                    double acc = 0.0, da = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        const double d = dS[(size_t)c * dv + j] + ki[c] * dp[j];
+                        dSt[(size_t)c * dv + j] = d;
+                        acc += St[(size_t)c * dv + j] * dp[j];
+                        da += d * Sp[(size_t)c * dv + j];
+                    }
+                    dkh[c] += acc;
+                    dal[c] = da;
+                }
+                for (int c = 0; c < dk; ++c)
+                    for (int j = 0; j < dv; ++j) dS[(size_t)c * dv + j] = alpha[c] * dSt[(size_t)c * dv + j];
+                /* back through the transforms */
+                double sq = 0.0, sk = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    sq += qi[c] * dqh[c];
+                    sk += ki[c] * dkh[c];
+                }
+                for (int c = 0; c < dk; ++c) {
+                    dq[row * dk + c] = (dqh[c] - qi[c] * sq) / nq[i];
+                    dkey[row * dk + c] = (dkh[c] - ki[c] * sk) / nk[i];
+                    const double sig = sigmoid(xg[i * dk + c]);
+                    const double dx = dal[c] * alpha[c] * lower_bound * sig * (1.0 - sig);
+                    dg[row * dk + c] = dx * ea;
+                    ppart[1 + c] += dx * ea;
+                    ppart[0] += dx * xg[i * dk + c];
+                }
+                dbeta[row] = dbt * b * (1.0 - b);
+            }
+            if (d_initial)
+                for (size_t e = 0; e < se; ++e) d_initial[soff + e] = dS[e];
+        }
+        free(hist); free(qh); free(kh); free(nq); free(nk); free(xg); free(la); free(bt); free(pred);
+        free(otmp); free(dS); free(dSt); free(St); free(vec);
+    }
+    if (!failed) {
+        for (int32_t h = 0; h < num_heads; ++h) {
+            dA_log[h] = 0.0;
+            for (int c = 0; c < dk; ++c) ddt_bias[(size_t)h * dk + c] = 0.0;
+        }
+        for (int64_t u = 0; u < units; ++u) {
+            const int32_t h = (int32_t)(u % num_heads);
+            dA_log[h] += part[(size_t)u * (1 + dk)];
+            for (int c = 0; c < dk; ++c) ddt_bias[(size_t)h * dk + c] += part[(size_t)u * (1 + dk) + 1 + c];
+        }
+    }
+    free(part);
+    return failed ? 2 : 0;
+}

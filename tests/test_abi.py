@@ -170,3 +170,33 @@ def test_fwd_ex_flags_validation(lib):
     assert ex(1, A_log=None, dt_bias=None, batch=0) == 0  # a precomputed gate does not
     assert ex(4, beta=P + 2) == 1                        # fp32 beta needs 4-byte alignment
     assert ex(1, lb=-6.0) == 2                           # the clamp range must still be supported
+
+
+def test_kcp_entry_points_validation(lib):
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    sm = lib.kda_segment_map
+    sm.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                           ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p]
+    sm.restype = ctypes.c_int
+
+    def seg(M=P, Bm=P, ws=P, ws_bytes=1 << 20, K=128, batch=1):
+        return sm(vp(P), vp(P), vp(P), vp(P), vp(P), vp(ws), ws_bytes, vp(P), vp(P), -5.0, vp(M), vp(Bm), None,
+                  batch, 64, 1, K, 128, batch, 0, None)
+
+    assert seg(M=None) == 1
+    assert seg(Bm=P + 8) == 1
+    assert seg(ws=None) == 1
+    assert seg(ws_bytes=16) == 3
+    assert seg(K=64) == 2
+    assert seg(batch=0) == 0
+    af = lib.kda_state_affine
+    af.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
+    af.restype = ctypes.c_int
+    assert af(vp(P), vp(P), vp(P), vp(P), 4, 64, 0, None) == 2
+    assert af(None, vp(P), vp(P), vp(P), 4, 128, 0, None) == 1   # a state input needs M
+    assert af(vp(P), None, vp(P), vp(P), 4, 128, 0, None) == 1
+    assert af(vp(P), vp(P), vp(P + 4), vp(P), 4, 128, 0, None) == 1
+    assert af(vp(P), vp(P), vp(P), vp(P), 4, 128, 2, None) == 1
+    assert af(vp(P), vp(P), vp(P), vp(P), 0, 128, 0, None) == 0

@@ -296,7 +296,9 @@ def test_intra_chunk_stages_against_chunked_form(cuda_device, case):
                     "P T_b": (tb[64:64 + L, :L], ref["P"] @ Tb, None),
                     "Ktil": (kt[:L], ref["Kt"] / ik_ref[:, None], None),
                     "1/|k|": (ik[:L], ik_ref, None),
-                    "e^Gamma_C": (gam, ref["gC"], None),
+                    # e^{Gamma_C} is a float32 product of decays: where the exact value is below
+                    # float32's normal range (64 saturated decays: e^-320) it is zero
+                    "e^Gamma_C": (gam, np.where(ref["gC"] < np.finfo(np.float32).tiny, 0.0, ref["gC"]), None),
                 }
                 assert np.all(ik[L:] == 0)  # rows past the end of the document
                 for name, (got, want, nrm) in pairs.items():
