@@ -121,14 +121,24 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g,
                      int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
                      kda_stream_t stream);
 
+/* Bytes of workspace kda_fwd_ex needs for head sizes (K, V): kda_workspace_size(T, H, N) when
+ * K = V = 128; for smaller head sizes also 128-wide copies of q, k, v, g, out, dt_bias and the
+ * states, into which the inputs are zero-padded. */
+size_t kda_workspace_size_ex(int64_t total_tokens, int32_t num_heads, int32_t num_seqs, int32_t head_dim_k,
+                             int32_t head_dim_v);
+
 /* kda_fwd with the input transforms selectable (fla chunk_kda's use_gate_in_kernel,
  * use_qk_l2norm_in_kernel and use_beta_sigmoid_in_kernel; "What CUDA Version Is Required to Use
  * FlashKDA?", Usage Examples): `flags` is a combination of the KDA_FLAG_* values, 0 giving
  * kda_fwd.  With KDA_FLAG_GATE_PRECOMPUTED, g is fp32 log alpha [batch, seqlen, H, K] (16-byte
  * aligned), A_log and dt_bias may be NULL, and each log alpha is clamped to [lower_bound, 0] (the
  * range whose per-16-token exponent span the chunked kernels keep inside float range); with
- * KDA_FLAG_BETA_PRECOMPUTED beta is fp32 [batch, seqlen, H] (4-byte aligned).  Same workspace,
- * layouts and errors as kda_fwd otherwise. */
+ * KDA_FLAG_BETA_PRECOMPUTED beta is fp32 [batch, seqlen, H] (4-byte aligned).
+ * Head sizes: besides K = V = 128, any K and V that are multiples of 8 up to 128 (fla's chunk_kda
+ * takes any head size).  Those run the same kernels on zero-padded 128-wide copies made in the
+ * workspace (size from kda_workspace_size_ex), which is exact: padded key channels are zero in q
+ * and k, padded value channels zero in v, so they add nothing and their state entries stay zero;
+ * layouts are the same with K and V in place of 128.  Same errors as kda_fwd otherwise. */
 kda_status_t kda_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
                         float scale, void* out, void* workspace, size_t workspace_bytes,
                         const float* A_log, const float* dt_bias, float lower_bound,
@@ -234,8 +244,9 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const void*
                         kda_stream_t stream);
 
 /* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): one fp32
- * 128 x 128 checkpoint per (64-token chunk, head) for at most T / 64 + N + 1 chunk slots, and a
- * 64-state scratch for each of up to min(N H, 256) CTAs.  Depends only on its arguments. */
+ * 128 x 128 checkpoint per (64-token chunk, head) for at most T / 64 + N + 1 chunk slots, a scratch
+ * of 64 states of 128 x 32 for each of up to min(4 N H, 512) CTAs, and four slices of per-channel
+ * partial sums (3 x 128 + 1 fp32 per token and head).  Depends only on its arguments. */
 size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
 /* The backward pass: gradients of sum(d_out * out) + sum(d_final * final_state) with respect to
@@ -249,9 +260,10 @@ size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t n
  *                [batch, seqlen, H] (w.r.t. the raw beta, before the sigmoid; dg w.r.t. the raw gate)
  *   dA_log fp32 [H], ddt_bias fp32 [H, K]  (overwritten: zeroed, then summed over all tokens)
  *   d_initial    fp32 [N, H, K, V] or NULL (not written)
- * Token by token on CUDA cores, one persistent CTA per (sequence, head): a forward that stores a
- * checkpoint every 64 tokens, then chunk by chunk from the last a rerun from the checkpoint and a
- * reverse walk over its tokens.  Gradient pointers are 16-byte aligned (dbeta 2, dA_log 4).  With
+ * Token by token on CUDA cores, four persistent CTAs per (sequence, head) (32 state columns each):
+ * a forward that stores a checkpoint every 64 tokens, then chunk by chunk from the last a rerun from
+ * the checkpoint and a reverse walk over its tokens; a second kernel sums the column slices and
+ * applies the derivatives of the in-kernel transforms.  Gradient pointers are 16-byte aligned (dbeta 2, dA_log 4).  With
  * out-of-order cu_seqlens every document is treated as empty: the token gradients are not written
  * and d_initial = d_final (there is no status word to report it). */
 kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,

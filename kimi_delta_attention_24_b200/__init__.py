@@ -24,7 +24,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["fwd", "fwd_recurrent", "decode", "segment_map", "state_affine", "bwd", "bwd_workspace_size", "FLAG_GATE_PRECOMPUTED", "FLAG_NO_QK_L2NORM",
+__all__ = ["get_workspace_size_ex", "fwd", "fwd_recurrent", "decode", "segment_map", "state_affine", "bwd", "bwd_workspace_size", "FLAG_GATE_PRECOMPUTED", "FLAG_NO_QK_L2NORM",
            "FLAG_BETA_PRECOMPUTED", "get_workspace_size", "fwd_launch_count", "new_workspace",
            "is_supported", "chunk_kda", "read_device_status", "selftest_wait_timeout", "KDAError",
            "library_path", "load"]
@@ -83,6 +83,8 @@ def load():
     lib.kda_bwd.argtypes = [vp, vp, vp, vp, vp, f32, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                             ctypes.c_size_t, vp, i32, i64, i32, i32, i32, i32, vp]
     lib.kda_bwd.restype = ctypes.c_int
+    lib.kda_workspace_size_ex.argtypes = [i64, i32, i32, i32, i32]
+    lib.kda_workspace_size_ex.restype = ctypes.c_size_t
     lib.kda_workspace_size.argtypes = [i64, i32, i32]
     lib.kda_workspace_size.restype = ctypes.c_size_t
     lib.kda_fwd_launch_count.argtypes = [i64, i32, i32]
@@ -109,10 +111,14 @@ def fwd_launch_count(T: int, H: int, N: int) -> int:
     return int(load().kda_fwd_launch_count(int(T), int(H), int(N)))
 
 
-def new_workspace(T: int, H: int, N: int, device) -> torch.Tensor:
-    """A workspace for kda.fwd: uninitialised except for its 256-byte header (status word and item
-    counters), which is zeroed."""
-    ws = torch.empty(get_workspace_size(T, H, N), dtype=torch.uint8, device=device)
+def get_workspace_size_ex(T: int, H: int, N: int, K: int = 128, V: int = 128) -> int:
+    return int(load().kda_workspace_size_ex(int(T), int(H), int(N), int(K), int(V)))
+
+
+def new_workspace(T: int, H: int, N: int, device, K: int = 128, V: int = 128) -> torch.Tensor:
+    """A workspace for kda.fwd (head sizes K, V): uninitialised except for its 256-byte header
+    (status word and item counters), which is zeroed."""
+    ws = torch.empty(get_workspace_size_ex(T, H, N, K, V), dtype=torch.uint8, device=device)
     ws[:256].zero_()
     return ws
 
@@ -174,7 +180,8 @@ def fwd(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound,
         flags=0):
     """The chunked forward (tcgen05 kernels).  Writes ``out`` and ``final_state`` in place.
     ``flags`` (FLAG_*) switches input transforms off (kda_fwd_ex); 0 is kda_fwd."""
-    _call("kda_fwd_ex" if flags else "kda_fwd", q, k, v, g, beta, scale, out, workspace, A_log, dt_bias,
+    ex = flags or q.shape[-1] != 128 or v.shape[-1] != 128
+    _call("kda_fwd_ex" if ex else "kda_fwd", q, k, v, g, beta, scale, out, workspace, A_log, dt_bias,
           lower_bound, initial_state, final_state, cu_seqlens, state_transposed, stream, flags)
 
 
@@ -357,7 +364,7 @@ def chunk_kda(q, k, v, g, beta, scale=None, initial_state=None, output_final_sta
     if output_final_state:
         shape = (N, H, V, K) if transpose_state_layout else (N, H, K, V)
         final = torch.empty(shape, dtype=torch.float32, device=q.device)
-    ws = new_workspace(B * T, H, N, q.device)
+    ws = new_workspace(B * T, H, N, q.device, K, V)
     if recurrent:
         fwd_recurrent(q, k, v, g, beta, scale, out, ws, A_log, dt_bias, lower_bound, initial_state, final,
                       cu_seqlens, state_transposed=transpose_state_layout)

@@ -19,7 +19,7 @@ LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libkda_b200.so")
 
 SOURCES = ["kda_api.cu", "kda_recurrent.cu", "kda_chunked.cu", "kda_split.cu", "kda_fwd_static.cu",
-           "kda_selftest.cu", "kda_decode.cu", "kda_kcp.cu", "kda_bwd.cu"]
+           "kda_selftest.cu", "kda_decode.cu", "kda_kcp.cu", "kda_bwd.cu", "kda_pad.cu"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH_FLAGS + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
                            f"-I{INCLUDE}", f"-I{CSRC}"]

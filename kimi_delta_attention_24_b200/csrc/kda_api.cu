@@ -13,6 +13,21 @@ struct Shape {
   int32_t num_seqs;
 };
 
+// Head sizes kda_fwd_ex runs by zero padding to 128: multiples of 8 (16-byte bf16 rows) up to 128.
+bool padded_head_dim_ok(int32_t d) { return d >= 8 && d <= kda::kHeadDim && d % 8 == 0; }
+
+// Bytes after the split path's workspace that zero padding needs: 128-wide q, k, v, out (bf16), g
+// (fp32, the wider of its two types), dt_bias, and the initial and final states.
+size_t pad_bytes(int64_t tokens, int32_t H, int32_t N, int32_t K, int32_t V) {
+  if (K == kda::kHeadDim && V == kda::kHeadDim) return 0;
+  const size_t rows = (size_t)(tokens > 0 ? tokens : 0) * (size_t)(H > 0 ? H : 0);
+  const size_t row_bf16 = kda::kHeadDim * 2, row_f32 = kda::kHeadDim * 4;
+  const size_t units = (size_t)(N > 0 ? N : 0) * (size_t)(H > 0 ? H : 0);
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  return 4 * up(rows * row_bf16) + up(rows * row_f32) + up((size_t)(H > 0 ? H : 0) * row_f32) +
+         2 * up(units * kda::kHeadDim * row_f32);
+}
+
 // Validates everything the host can check without touching device memory.
 kda_status_t validate(const void* q, const void* k, const void* v, const void* g, const void* beta,
                       const void* out, const float* A_log, const float* dt_bias, float lower_bound,
@@ -20,8 +35,12 @@ kda_status_t validate(const void* q, const void* k, const void* v, const void* g
                       const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
                       int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
                       int32_t state_transposed, float scale, Shape* shape, uint32_t flags = 0,
-                      bool need_out = true) {
-  if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
+                      bool need_out = true, bool any_head_dim = false) {
+  if (any_head_dim) {
+    if (!padded_head_dim_ok(head_dim_k) || !padded_head_dim_ok(head_dim_v)) return KDA_ERR_UNSUPPORTED;
+  } else if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) {
+    return KDA_ERR_UNSUPPORTED;
+  }
   if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_UNSUPPORTED;
   if ((flags & ~kda::kFlagMask) != 0) return KDA_ERR_INVALID_ARGUMENT;
   const bool gate_in_kernel = !(flags & kda::kFlagGatePrecomputed);
@@ -107,8 +126,7 @@ kda_status_t kda::fwd_fused(const void* q, const void* k, const void* v, const v
 extern "C" {
 
 int kda_is_supported(int head_dim, int dtype_is_bf16, float lower_bound) {
-  return head_dim == kda::kHeadDim && dtype_is_bf16 != 0 && lower_bound >= -5.0f &&
-         lower_bound <= 0.0f;
+  return head_dim == kda::kHeadDim && dtype_is_bf16 != 0 && lower_bound >= -5.0f && lower_bound <= 0.0f;
 }
 
 size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
@@ -117,6 +135,13 @@ size_t kda_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_s
 
 int kda_fwd_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
   return kda::split_launch_count(total_tokens, num_heads, num_seqs);
+}
+
+size_t kda_workspace_size_ex(int64_t total_tokens, int32_t num_heads, int32_t num_seqs, int32_t head_dim_k,
+                             int32_t head_dim_v) {
+  const size_t split = kda::split_workspace_bytes(total_tokens, num_heads, num_seqs);
+  if (head_dim_k == kda::kHeadDim && head_dim_v == kda::kHeadDim) return split;
+  return (split + 255) / 256 * 256 + pad_bytes(total_tokens, num_heads, num_seqs, head_dim_k, head_dim_v);
 }
 
 kda_status_t kda_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -129,18 +154,68 @@ kda_status_t kda_fwd_ex(const void* q, const void* k, const void* v, const void*
   Shape shape;
   kda_status_t st = validate(q, k, v, g, beta, out, A_log, dt_bias, lower_bound, initial_state,
                              final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k,
-                             head_dim_v, num_seqs, state_transposed, scale, &shape, flags);
+                             head_dim_v, num_seqs, state_transposed, scale, &shape, flags, true, true);
   if (st != KDA_OK) return st;
   if (!workspace || !aligned(workspace, 256)) return KDA_ERR_INVALID_ARGUMENT;
-  if (workspace_bytes < kda_workspace_size(shape.total_tokens, num_heads, shape.num_seqs))
+  if (workspace_bytes < kda_workspace_size_ex(shape.total_tokens, num_heads, shape.num_seqs, head_dim_k,
+                                              head_dim_v))
     return KDA_ERR_WORKSPACE_TOO_SMALL;
   kda::FwdParams p = make_params(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
                                  initial_state, final_state, cu_seqlens, seqlen, num_heads,
                                  shape.num_seqs, state_transposed, static_cast<uint32_t*>(workspace));
   p.flags = flags;
-  if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
-  return kda::launch_split(p, workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
-                                                                                                 : KDA_ERR_CUDA;
+  const int64_t units = (int64_t)shape.num_seqs * num_heads;
+  if (units == 0) return KDA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int K = head_dim_k, V = head_dim_v;
+  if (K == kda::kHeadDim && V == kda::kHeadDim)
+    return kda::launch_split(p, workspace, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+
+  // head sizes below 128: zero-pad into the workspace, run the 128-wide path, copy the results out
+  const int64_t rows = shape.total_tokens * num_heads;
+  const size_t row_bf16 = kda::kHeadDim * 2, row_f32 = kda::kHeadDim * 4;
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  uint8_t* cur = static_cast<uint8_t*>(workspace) +
+                 up(kda::split_workspace_bytes(shape.total_tokens, num_heads, shape.num_seqs));
+  auto take = [&](size_t bytes) {
+    uint8_t* r = cur;
+    cur += up(bytes);
+    return r;
+  };
+  void* q2 = take(rows * row_bf16);
+  void* k2 = take(rows * row_bf16);
+  void* v2 = take(rows * row_bf16);
+  void* o2 = take(rows * row_bf16);
+  void* g2 = take(rows * row_f32);
+  float* dt2 = reinterpret_cast<float*>(take((size_t)num_heads * row_f32));
+  float* s02 = reinterpret_cast<float*>(take((size_t)units * kda::kHeadDim * row_f32));
+  float* sf2 = reinterpret_cast<float*>(take((size_t)units * kda::kHeadDim * row_f32));
+  const bool gate_pre = (flags & kda::kFlagGatePrecomputed) != 0;
+  const int R = state_transposed ? V : K, C = state_transposed ? K : V;
+  bool ok = kda::launch_pad_rows(q, q2, rows, K, 2, s) == cudaSuccess &&
+            kda::launch_pad_rows(k, k2, rows, K, 2, s) == cudaSuccess &&
+            kda::launch_pad_rows(v, v2, rows, V, 2, s) == cudaSuccess &&
+            kda::launch_pad_rows(g, g2, rows, K, gate_pre ? 4 : 2, s) == cudaSuccess;
+  if (ok && !gate_pre) ok = kda::launch_pad_rows(dt_bias, dt2, num_heads, K, 4, s) == cudaSuccess;
+  if (ok && initial_state) ok = kda::launch_pad_state(initial_state, s02, units, R, C, s) == cudaSuccess;
+  if (!ok) return KDA_ERR_CUDA;
+  p.q = static_cast<const __nv_bfloat16*>(q2);
+  p.k = static_cast<const __nv_bfloat16*>(k2);
+  p.v = static_cast<const __nv_bfloat16*>(v2);
+  p.g = static_cast<const __nv_bfloat16*>(g2);
+  p.out = static_cast<__nv_bfloat16*>(o2);
+  p.dt_bias = gate_pre ? nullptr : dt2;
+  p.initial_state = initial_state ? s02 : nullptr;
+  p.final_state = final_state ? sf2 : nullptr;
+  if (kda::launch_split(p, workspace, s) != cudaSuccess) return KDA_ERR_CUDA;
+  // the documents cover every token when cu_seqlens is in order, so every padded output row was
+  // written; when it is not, the chunk table is all zero and `out` must stay untouched: the copy
+  // reads the chunk table's total first and skips
+  const int32_t* chunk_total = reinterpret_cast<const int32_t*>(static_cast<uint8_t*>(workspace) +
+                                                                kda::kWorkspaceHeader) + shape.num_seqs;
+  if (kda::launch_unpad_rows(o2, out, rows, V, 2, s, chunk_total) != cudaSuccess) return KDA_ERR_CUDA;
+  if (final_state && kda::launch_unpad_state(sf2, final_state, units, R, C, s) != cudaSuccess) return KDA_ERR_CUDA;
+  return KDA_OK;
 }
 
 kda_status_t kda_segment_map(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -191,6 +266,7 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const void* g,
                      int32_t batch, int64_t seqlen, int32_t num_heads, int32_t head_dim_k,
                      int32_t head_dim_v, int32_t num_seqs, int32_t state_transposed,
                      kda_stream_t stream) {
+  if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
   return kda_fwd_ex(q, k, v, g, beta, scale, out, workspace, workspace_bytes, A_log, dt_bias, lower_bound,
                     initial_state, final_state, cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v,
                     num_seqs, state_transposed, 0u, stream);

@@ -10,14 +10,17 @@
 //   dalpha_c = sum_j dStil[c][j] S_{t-1}[c][j];  dS_{t-1} = Diag(alpha) dStil,
 // followed by the derivatives of the in-kernel transforms (L2 norms, sigmoid of beta, safe gate).
 //
-// One CTA per (sequence, head) unit (persistent over units), 256 threads, the 128 x 128 state and
-// its gradient held in registers (a 16 x 4 block of each per thread, the layout of the decode
-// kernel).  The CTA first runs the forward over its sequence, storing the state at the start of
-// every 64-token chunk in the workspace; then, chunk by chunk from the last, it reruns the chunk's
-// forward from its checkpoint, storing the state before every token in a per-CTA scratch, and walks
-// the chunk's tokens backwards.  Sums over the state's rows run through shared memory across the
-// warps, sums over its columns through warp shuffles.  dA_log and dt_bias gradients are summed per
-// CTA and added to the outputs (zeroed first) with one atomic per value.
+// The columns of the state evolve independently, so one (sequence, head) unit is split over four
+// CTAs of 32 state columns each (persistent over (unit, slice) pairs, two CTAs per SM), 256 threads,
+// the slice of the state and of its gradient in registers (16 rows x 1 column per thread).  A CTA
+// first runs the forward over its sequence, storing the slice at the start of every 64-token chunk in
+// the workspace; then, chunk by chunk from the last, it reruns the chunk's forward from its
+// checkpoint, storing the slice before every token in a per-CTA scratch, and walks the chunk's tokens
+// backwards.  Sums over the state's rows run through shared memory across the warps, sums over its
+// columns through warp shuffles; what sums over all columns (dqhat, dkhat, dalpha per channel and
+// dbeta) is written per slice, and a second kernel adds the slices, applies the derivatives of the
+// L2 norms, the gate and the sigmoid, and adds the dA_log / dt_bias sums with one atomic per value
+// per CTA (the outputs are zeroed first).
 #include "kda_common.cuh"
 
 namespace kda {
@@ -26,7 +29,10 @@ namespace {
 constexpr int kBwdThreads = 256;
 constexpr int kBwdChunk = 64;
 constexpr int kRows = 16;  // state rows per thread: warp w holds rows 16 w .. 16 w + 15
+constexpr int kSlice = 32;  // state columns per CTA (one per lane)
+constexpr int kSlices = kHeadDim / kSlice;
 constexpr size_t kStateElems = (size_t)kHeadDim * kHeadDim;
+constexpr size_t kSliceElems = (size_t)kHeadDim * kSlice;
 
 struct BwdParams {
   FwdParams f;
@@ -40,8 +46,9 @@ struct BwdParams {
   float* dA_log;                // [H], zeroed before the launch
   float* ddt_bias;              // [H, K], zeroed before the launch
   float* d_initial;             // [N, H, K, V] or null
-  float* ckpt;                  // (T / 64 + N + 1) x H states: chunk-start checkpoints
-  float* scratch;               // gridDim.x x 64 states: the states before each token of a chunk
+  float* ckpt;                  // (T / 64 + N + 1) x H states: chunk-start checkpoints (by slice)
+  float* scratch;               // gridDim.x x 64 slices: the states before each token of a chunk
+  float* part;                  // per slice: dqhat, dkhat, dalpha [tokens, H, K]; then dbeta [slice][tokens, H]
 };
 
 struct TokenIn {
@@ -65,16 +72,48 @@ __device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, float a, float b, fl
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-// The transformed inputs of one token into shared memory (warps 0..5; a lane takes 4 channels).
-// `full`: also q, d_out and the gate's intermediates (the backward step); otherwise only what the
-// forward step reads (khat, alpha, beta, v).
-__device__ __forceinline__ void load_token(const BwdParams& P, size_t row, int h, float ea, TokenIn& s, bool full) {
+// One token's raw inputs, split over the CTA: warps 0..4 read 4 channels per lane of q, k, g, v and
+// d_out (warp 0 and 4 only for the backward step), lane 0 of warp 5 reads beta.  Fetched one token
+// ahead into registers, so that the global loads of token t + 1 overlap the work on token t.
+struct RawTok {
+  uint2 u;
+  float b;
+};
+
+__device__ __forceinline__ RawTok fetch_token(const BwdParams& P, size_t row, bool full) {
   const FwdParams& p = P.f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int D = kHeadDim;
+  RawTok r;
+  r.u = make_uint2(0, 0);
+  r.b = 0.f;
+  const __nv_bfloat16* src = nullptr;
+  if (warp == 0 && full) src = p.q;
+  else if (warp == 1) src = p.k;
+  else if (warp == 2) src = p.g;
+  else if (warp == 3) src = p.v;
+  else if (warp == 4 && full) src = P.d_out;
+  if (src) r.u = *reinterpret_cast<const uint2*>(src + row * D + 4 * lane);
+  if (warp == 5 && lane == 0) r.b = __bfloat162float(p.beta[row]);
+  return r;
+}
+
+__device__ __forceinline__ float4 bf16x4_of(uint2 u) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// The transformed inputs of one token into shared memory, from the fetched raw values.  `full`:
+// also qhat, d_out and the gate's intermediates (the backward step); otherwise only what the forward
+// step reads (khat, alpha, beta, v).  dt: this lane's 4 channels of dt_bias[h].
+__device__ __forceinline__ void stage_token(const BwdParams& P, const RawTok& r, float ea, float4 dt, TokenIn& s,
+                                            bool full) {
+  const FwdParams& p = P.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 || warp == 1) {
     if (warp == 0 && !full) return;
-    const float4 x4 = ld_bf16x4((warp == 0 ? p.q : p.k) + row * D + 4 * lane);
+    const float4 x4 = bf16x4_of(r.u);
     float ss = x4.x * x4.x + x4.y * x4.y + x4.z * x4.z + x4.w * x4.w;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -83,8 +122,7 @@ __device__ __forceinline__ void load_token(const BwdParams& P, size_t row, int h
     reinterpret_cast<float4*>(dst)[lane] = make_float4(x4.x / n, x4.y / n, x4.z / n, x4.w / n);
     if (lane == 0) (warp == 0 ? s.nq : s.nk) = n;
   } else if (warp == 2) {
-    const float4 g4 = ld_bf16x4(p.g + row * D + 4 * lane);
-    const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+    const float4 g4 = bf16x4_of(r.u);
     const float gv[4] = {g4.x, g4.y, g4.z, g4.w}, dts[4] = {dt.x, dt.y, dt.z, dt.w};
     float xs[4], sgs[4], as[4];
 #pragma unroll
@@ -99,11 +137,11 @@ __device__ __forceinline__ void load_token(const BwdParams& P, size_t row, int h
       reinterpret_cast<float4*>(s.sg)[lane] = make_float4(sgs[0], sgs[1], sgs[2], sgs[3]);
     }
   } else if (warp == 3) {
-    reinterpret_cast<float4*>(s.v)[lane] = ld_bf16x4(p.v + row * D + 4 * lane);
+    reinterpret_cast<float4*>(s.v)[lane] = bf16x4_of(r.u);
   } else if (warp == 4) {
-    if (full) reinterpret_cast<float4*>(s.d)[lane] = ld_bf16x4(P.d_out + row * D + 4 * lane);
+    if (full) reinterpret_cast<float4*>(s.d)[lane] = bf16x4_of(r.u);
   } else if (warp == 5 && lane == 0) {
-    s.b = sigmoid_acc(__bfloat162float(p.beta[row]));
+    s.b = sigmoid_acc(r.b);
   }
 }
 
@@ -122,34 +160,30 @@ __device__ __forceinline__ float transpose_reduce16(const float (&x)[16], int la
   return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
 }
 
-// Sum over the 8 warps of each thread's 4 column partials: red[w][4 lane + j].
-__device__ __forceinline__ float4 cross_warp_sum(float (*red)[kHeadDim], const float (&x)[4], int warp, int lane) {
-  reinterpret_cast<float4*>(red[warp])[lane] = make_float4(x[0], x[1], x[2], x[3]);
-  __syncthreads();
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    const float4 t = reinterpret_cast<const float4*>(red[w])[lane];
-    s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
-  }
-  return s;
-}
-
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(BwdParams P) {
+// One CTA per (unit, column slice): the state's 128 rows and the slice's kSlice columns (a 16 x 1
+// block per thread: warp w holds rows 16 w .. + 15, lane l column l of the slice).  The columns of
+// the state evolve independently, so each slice runs the whole token recurrence on its own; what
+// sums over columns (dqhat, dkhat, dalpha per row, dbeta) is written per slice and summed by
+// bwd_finish_kernel, which also applies the derivatives of the in-kernel transforms.
+__global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
   constexpr int D = kHeadDim;
   __shared__ __align__(16) TokenIn s;
-  __shared__ __align__(16) float red[2][8][D];
-  __shared__ __align__(16) float rows[3][D];  // dqhat, dkhat, dalpha of the token, per state row
+  __shared__ __align__(16) float red[2][8][kSlice];
   const FwdParams& p = P.f;
   const int H = p.num_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r0 = kRows * warp, c0 = 4 * lane;
+  const int r0 = kRows * warp;
   const int64_t units = (int64_t)p.num_seqs * H;
-  float* const scr = P.scratch + (size_t)blockIdx.x * kBwdChunk * kStateElems;
+  const int64_t work = units * kSlices;
+  float* const scr = P.scratch + (size_t)blockIdx.x * kBwdChunk * kSliceElems;
   const bool seqlens_ok = cta_seqlens_ok(p);
+  const int64_t rows_total = (p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs) * H;
 
-  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+  for (int64_t wi = blockIdx.x; wi < work; wi += gridDim.x) {
+    const int64_t u = wi / kSlices;
+    const int sl = (int)(wi - u * kSlices);
     const int n = (int)(u / H), h = (int)(u % H);
+    const int col = sl * kSlice + lane;  // this thread's state column (v)
     int64_t bos, eos;
     seq_range(p, n, bos, eos);
     if (!seqlens_ok) eos = bos;
@@ -158,232 +192,256 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(BwdParams P) {
     const size_t soff = ((size_t)n * H + h) * kStateElems;
     const int64_t ck0 = bos / kBwdChunk + n;  // this sequence's first checkpoint slot
     const float ea = expf(p.A_log[h]);
-    auto ck_ptr = [&](int c) { return P.ckpt + ((size_t)(ck0 + c) * H + h) * kStateElems; };
+    const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+    auto tok_row = [&](int64_t t) { return (size_t)t * H + h; };
+    // checkpoint c of this slice: [128 rows][kSlice]
+    auto ck_ptr = [&](int c) { return P.ckpt + (((size_t)(ck0 + c) * H + h) * kSlices + sl) * kSliceElems; };
+    float* const part_q = P.part + (size_t)sl * 3 * rows_total * D;  // per slice: dqhat, dkhat, dalpha rows
+    float* const part_k = part_q + (size_t)rows_total * D;
+    float* const part_a = part_k + (size_t)rows_total * D;
+    float* const part_b = P.part + (size_t)kSlices * 3 * rows_total * D + (size_t)sl * rows_total;
 
-    float S[kRows][4];
-    if (p.initial_state) {
+    float S[kRows];
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const float4 t = *reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)(r0 + i) * D + c0);
-        S[i][0] = t.x; S[i][1] = t.y; S[i][2] = t.z; S[i][3] = t.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) S[i][0] = S[i][1] = S[i][2] = S[i][3] = 0.f;
-    }
+    for (int i = 0; i < kRows; ++i) S[i] = p.initial_state ? p.initial_state[soff + (size_t)(r0 + i) * D + col] : 0.f;
     auto store_state = [&](float* dst) {
 #pragma unroll
-      for (int i = 0; i < kRows; ++i)
-        *reinterpret_cast<float4*>(dst + (size_t)(r0 + i) * D + c0) = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
+      for (int i = 0; i < kRows; ++i) dst[(r0 + i) * kSlice + lane] = S[i];
     };
     auto load_state = [&](const float* src) {
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const float4 t = *reinterpret_cast<const float4*>(src + (size_t)(r0 + i) * D + c0);
-        S[i][0] = t.x; S[i][1] = t.y; S[i][2] = t.z; S[i][3] = t.w;
-      }
+      for (int i = 0; i < kRows; ++i) S[i] = src[(r0 + i) * kSlice + lane];
     };
-    // one forward token on the registers' state (inputs in shared memory)
+    // the sum over the 8 warps of one value per thread (its column): red[w][lane]
+    auto col_sum = [&](float (*rd)[kSlice], float x) {
+      rd[warp][lane] = x;
+      __syncthreads();
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) t += rd[w][lane];
+      return t;
+    };
     auto forward_token = [&]() {
-      float pr[4] = {0.f, 0.f, 0.f, 0.f};
+      float pr = 0.f;
 #pragma unroll
       for (int i = 0; i < kRows; ++i) {
-        const float a = s.a[r0 + i], kk = s.k[r0 + i];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          S[i][j] *= a;
-          pr[j] = fmaf(S[i][j], kk, pr[j]);
-        }
+        S[i] *= s.a[r0 + i];
+        pr = fmaf(S[i], s.k[r0 + i], pr);
       }
-      const float4 pp = cross_warp_sum(red[0], pr, warp, lane);
-      const float4 vv = reinterpret_cast<const float4*>(s.v)[lane];
-      const float d[4] = {s.b * (vv.x - pp.x), s.b * (vv.y - pp.y), s.b * (vv.z - pp.z), s.b * (vv.w - pp.w)};
+      const float d = s.b * (s.v[col] - col_sum(red[0], pr));
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const float kk = s.k[r0 + i];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) S[i][j] = fmaf(kk, d[j], S[i][j]);
-      }
+      for (int i = 0; i < kRows; ++i) S[i] = fmaf(s.k[r0 + i], d, S[i]);
     };
 
     // ---------------------------------------------------------------- forward with checkpoints
+    RawTok rt = fetch_token(P, tok_row(bos), false);  // (L = 0: never staged)
     for (int c = 0; c < nch; ++c) {
       store_state(ck_ptr(c));
       const int64_t t_end = min(bos + (int64_t)(c + 1) * kBwdChunk, eos);
       for (int64_t t = bos + (int64_t)c * kBwdChunk; t < t_end; ++t) {
         __syncthreads();
-        load_token(P, (size_t)t * H + h, h, ea, s, false);
+        stage_token(P, rt, ea, dt, s, false);
+        if (t + 1 < eos) rt = fetch_token(P, tok_row(t + 1), false);
         __syncthreads();
         forward_token();
       }
     }
 
     // ---------------------------------------------------------------- backward, chunk by chunk
-    float dS[kRows][4];
-    if (P.d_final) {
+    float dS[kRows];
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const float4 t = *reinterpret_cast<const float4*>(P.d_final + soff + (size_t)(r0 + i) * D + c0);
-        dS[i][0] = t.x; dS[i][1] = t.y; dS[i][2] = t.z; dS[i][3] = t.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) dS[i][0] = dS[i][1] = dS[i][2] = dS[i][3] = 0.f;
-    }
-    float ddt[4] = {0.f, 0.f, 0.f, 0.f}, dA = 0.f;  // warp 2's gate-parameter sums (channels 4 lane ..)
+    for (int i = 0; i < kRows; ++i) dS[i] = P.d_final ? P.d_final[soff + (size_t)(r0 + i) * D + col] : 0.f;
 
     for (int c = nch - 1; c >= 0; --c) {
       const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
       const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
       // rerun the chunk's forward from its checkpoint, keeping the state before each token
       load_state(ck_ptr(c));
+      RawTok rf = fetch_token(P, tok_row(t_begin), false);
       for (int i = 0; i < len; ++i) {
-        store_state(scr + (size_t)i * kStateElems);
+        store_state(scr + (size_t)i * kSliceElems);
         __syncthreads();
-        load_token(P, (size_t)(t_begin + i) * H + h, h, ea, s, false);
+        stage_token(P, rf, ea, dt, s, false);
+        if (i + 1 < len) rf = fetch_token(P, tok_row(t_begin + i + 1), false);
         __syncthreads();
         forward_token();
       }
-      // the chunk's tokens backwards
+      // the chunk's tokens backwards; S holds S_{t-1} of the token at hand, loaded from the scratch
+      // (written by this thread above) during the token after it
+      RawTok rb = fetch_token(P, tok_row(t_begin + len - 1), true);
+      load_state(scr + (size_t)(len - 1) * kSliceElems);
       for (int i = len - 1; i >= 0; --i) {
-        const size_t row = (size_t)(t_begin + i) * H + h;
+        const size_t row = tok_row(t_begin + i);
         __syncthreads();
-        load_token(P, row, h, ea, s, true);
-        load_state(scr + (size_t)i * kStateElems);  // S_{t-1}: written by this thread above
+        stage_token(P, rb, ea, dt, s, true);
+        if (i > 0) rb = fetch_token(P, tok_row(t_begin + i - 1), true);
         __syncthreads();
         const float b = s.b, scale = p.scale;
-        // p = Stil^T khat
-        float pr[4] = {0.f, 0.f, 0.f, 0.f};
+        float pr = 0.f;
+#pragma unroll
+        for (int ii = 0; ii < kRows; ++ii) pr = fmaf(s.a[r0 + ii] * S[ii], s.k[r0 + ii], pr);
+        const float pj = col_sum(red[0], pr);
+        const float vj = s.v[col], doj = s.d[col];
+        const float dl = b * (vj - pj);
+        // dS += scale qhat do^T;  dqhat rows (this slice) = scale S_t do;  ddelta = dS^T khat
+        float rq[kRows], pd = 0.f;
 #pragma unroll
         for (int ii = 0; ii < kRows; ++ii) {
-          const float a = s.a[r0 + ii], kk = s.k[r0 + ii];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) pr[j] = fmaf(a * S[ii][j], kk, pr[j]);
-        }
-        const float4 pp = cross_warp_sum(red[0], pr, warp, lane);
-        const float4 vv = reinterpret_cast<const float4*>(s.v)[lane];
-        const float4 do4 = reinterpret_cast<const float4*>(s.d)[lane];
-        const float pj[4] = {pp.x, pp.y, pp.z, pp.w}, vj[4] = {vv.x, vv.y, vv.z, vv.w};
-        const float doj[4] = {do4.x, do4.y, do4.z, do4.w};
-        float dl[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dl[j] = b * (vj[j] - pj[j]);
-        // dS += scale qhat do^T; dqhat rows = scale S_t do; ddelta = dS^T khat
-        float rq[kRows], pd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ii = 0; ii < kRows; ++ii) {
-          const float a = s.a[r0 + ii], kk = s.k[r0 + ii], qq = s.q[r0 + ii];
-          float acc = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float st = fmaf(kk, dl[j], a * S[ii][j]);  // S_t
-            acc = fmaf(st, doj[j], acc);
-            dS[ii][j] = fmaf(scale * qq, doj[j], dS[ii][j]);
-            pd[j] = fmaf(dS[ii][j], kk, pd[j]);
-          }
-          rq[ii] = scale * acc;
-        }
-        const float4 dd = cross_warp_sum(red[1], pd, warp, lane);
-        const float ddl[4] = {dd.x, dd.y, dd.z, dd.w};
-        float dp[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dp[j] = -b * ddl[j];
-        if (warp == 0) {
-          // dv, and dbeta through the sigmoid
-          st_bf16x4(P.dv + row * D + c0, b * ddl[0], b * ddl[1], b * ddl[2], b * ddl[3]);
-          float db = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) db = fmaf(ddl[j], vj[j] - pj[j], db);
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
-          if (lane == 0) P.dbeta[row] = __float2bfloat16_rn(db * b * (1.f - b));
-        }
-        // dkhat = dS delta + Stil dp;  dStil = dS + khat dp^T;  dalpha;  dS <- Diag(alpha) dStil
-        float rk[kRows], ra[kRows];
-#pragma unroll
-        for (int ii = 0; ii < kRows; ++ii) {
-          const float a = s.a[r0 + ii], kk = s.k[r0 + ii];
-          float ak = 0.f, aa = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float st = a * S[ii][j];
-            ak = fmaf(dS[ii][j], dl[j], ak);
-            ak = fmaf(st, dp[j], ak);
-            const float dst = fmaf(kk, dp[j], dS[ii][j]);
-            aa = fmaf(dst, S[ii][j], aa);
-            dS[ii][j] = a * dst;
-          }
-          rk[ii] = ak;
-          ra[ii] = aa;
+          const float kk = s.k[r0 + ii];
+          rq[ii] = scale * fmaf(kk, dl, s.a[r0 + ii] * S[ii]) * doj;
+          dS[ii] = fmaf(scale * s.q[r0 + ii], doj, dS[ii]);
+          pd = fmaf(dS[ii], kk, pd);
         }
         const float tq = transpose_reduce16(rq, lane);
+        const float ddl = col_sum(red[1], pd);
+        const float dp = -b * ddl;
+        if (warp == 0) {
+          P.dv[row * D + col] = __float2bfloat16_rn(b * ddl);
+          float db = ddl * (vj - pj);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
+          if (lane == 0) part_b[row] = db;
+        }
+        // dkhat = dS delta + Stil dp;  dStil = dS + khat dp^T;  dalpha;  dS <- Diag(alpha) dStil
+        float rk[kRows];
+#pragma unroll
+        for (int ii = 0; ii < kRows; ++ii) rk[ii] = fmaf(dS[ii], dl, s.a[r0 + ii] * S[ii] * dp);
         const float tk = transpose_reduce16(rk, lane);
+        float ra[kRows];
+#pragma unroll
+        for (int ii = 0; ii < kRows; ++ii) {
+          const float dst = fmaf(s.k[r0 + ii], dp, dS[ii]);
+          ra[ii] = dst * S[ii];
+          dS[ii] = s.a[r0 + ii] * dst;
+        }
+        if (i > 0) load_state(scr + (size_t)(i - 1) * kSliceElems);  // the next token's S_{t-1}
         const float ta = transpose_reduce16(ra, lane);
         if ((lane & 1) == 0) {
-          rows[0][r0 + (lane >> 1)] = tq;
-          rows[1][r0 + (lane >> 1)] = tk;
-          rows[2][r0 + (lane >> 1)] = ta;
-        }
-        __syncthreads();
-        // back through the transforms: warp 0 q, warp 1 k, warp 2 the gate
-        if (warp == 0 || warp == 1) {
-          const float* xh = warp == 0 ? s.q : s.k;
-          const float4 x4 = reinterpret_cast<const float4*>(xh)[lane];
-          const float4 g4 = reinterpret_cast<const float4*>(rows[warp])[lane];
-          float dot = x4.x * g4.x + x4.y * g4.y + x4.z * g4.z + x4.w * g4.w;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-          const float inv = 1.f / (warp == 0 ? s.nq : s.nk);
-          st_bf16x4((warp == 0 ? P.dq : P.dk) + row * D + c0, (g4.x - x4.x * dot) * inv, (g4.y - x4.y * dot) * inv,
-                    (g4.z - x4.z * dot) * inv, (g4.w - x4.w * dot) * inv);
-        } else if (warp == 2) {
-          const float4 da4 = reinterpret_cast<const float4*>(rows[2])[lane];
-          const float4 a4 = reinterpret_cast<const float4*>(s.a)[lane];
-          const float4 x4 = reinterpret_cast<const float4*>(s.x)[lane];
-          const float4 s4 = reinterpret_cast<const float4*>(s.sg)[lane];
-          const float dal[4] = {da4.x, da4.y, da4.z, da4.w}, al[4] = {a4.x, a4.y, a4.z, a4.w};
-          const float xv[4] = {x4.x, x4.y, x4.z, x4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
-          float dg[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float dx = dal[j] * al[j] * p.lower_bound * sv[j] * (1.f - sv[j]);
-            dg[j] = dx * ea;
-            ddt[j] += dg[j];
-            dA = fmaf(dx, xv[j], dA);
-          }
-          st_bf16x4(P.dg + row * D + c0, dg[0], dg[1], dg[2], dg[3]);
+          const size_t o = row * D + r0 + (lane >> 1);
+          part_q[o] = tq;
+          part_k[o] = tk;
+          part_a[o] = ta;
         }
       }
     }
     if (P.d_initial) {
 #pragma unroll
-      for (int i = 0; i < kRows; ++i)
-        *reinterpret_cast<float4*>(P.d_initial + soff + (size_t)(r0 + i) * D + c0) =
-            make_float4(dS[i][0], dS[i][1], dS[i][2], dS[i][3]);
+      for (int i = 0; i < kRows; ++i) P.d_initial[soff + (size_t)(r0 + i) * D + col] = dS[i];
     }
-    if (warp == 2) {
+  }
+}
+
+// Per (token, head) row: the slices' partial sums, then the derivatives of the transforms
+// (dq and dk through the L2 norms, dg through the gate, dbeta through the sigmoid).  A CTA takes one
+// head and a run of tokens (one warp per token at a time, a lane per 4 channels) and adds its sums
+// of the gate-parameter gradients with one atomic per value.
+__global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t tokens, int tokens_per_cta) {
+  constexpr int D = kHeadDim;
+  __shared__ __align__(16) float s_dt[8][D];
+  __shared__ float s_dA[8];
+  const FwdParams& p = P.f;
+  if (!cta_seqlens_ok(p)) return;  // out-of-order offsets: no document ran, nothing to finish
+  const int H = p.num_heads;
+  const int h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rows_total = tokens * H;
+  const float ea = expf(p.A_log[h]);
+  const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+  const float dts[4] = {dt.x, dt.y, dt.z, dt.w};
+  float ddt[4] = {0.f, 0.f, 0.f, 0.f}, dA = 0.f;
+  const int64_t t_begin = (int64_t)blockIdx.x * tokens_per_cta;
+  const int64_t t_end = min(t_begin + tokens_per_cta, tokens);
+  for (int64_t t = t_begin + warp; t < t_end; t += 8) {
+    const size_t row = (size_t)t * H + h;
+    float gq[4] = {0.f, 0.f, 0.f, 0.f}, gk[4] = {0.f, 0.f, 0.f, 0.f}, ga[4] = {0.f, 0.f, 0.f, 0.f}, gb = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) atomicAdd(P.ddt_bias + (size_t)h * D + c0 + j, ddt[j]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dA += __shfl_xor_sync(0xffffffffu, dA, o);
-      if (lane == 0) atomicAdd(P.dA_log + h, dA);
+    for (int sl = 0; sl < kSlices; ++sl) {
+      const float* base = P.part + (size_t)sl * 3 * rows_total * D + row * D + 4 * lane;
+      const float4 a = *reinterpret_cast<const float4*>(base);
+      const float4 b = *reinterpret_cast<const float4*>(base + (size_t)rows_total * D);
+      const float4 c = *reinterpret_cast<const float4*>(base + 2 * (size_t)rows_total * D);
+      gq[0] += a.x; gq[1] += a.y; gq[2] += a.z; gq[3] += a.w;
+      gk[0] += b.x; gk[1] += b.y; gk[2] += b.z; gk[3] += b.w;
+      ga[0] += c.x; ga[1] += c.y; ga[2] += c.z; ga[3] += c.w;
+      gb += P.part[(size_t)kSlices * 3 * rows_total * D + (size_t)sl * rows_total + row];
     }
+    // dq, dk: (dxhat - xhat (xhat . dxhat)) / n
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const float4 x4 = ld_bf16x4((which == 0 ? p.q : p.k) + row * D + 4 * lane);
+      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+      float ss = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float nrm = sqrtf(ss + kL2Eps);
+      const float* gx = which == 0 ? gq : gk;
+      float dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dot += (xv[j] / nrm) * gx[j];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      float r[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) r[j] = (gx[j] - (xv[j] / nrm) * dot) / nrm;
+      st_bf16x4((which == 0 ? P.dq : P.dk) + row * D + 4 * lane, r[0], r[1], r[2], r[3]);
+    }
+    // dg through the gate; the sums for dt_bias and A_log
+    {
+      const float4 g4 = ld_bf16x4(p.g + row * D + 4 * lane);
+      const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+      float dg[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float x = ea * (gv[j] + dts[j]);
+        const float sg = sigmoid_acc(x);
+        const float al = expf(p.lower_bound * sg);
+        const float dx = ga[j] * al * p.lower_bound * sg * (1.f - sg);
+        dg[j] = dx * ea;
+        ddt[j] += dg[j];
+        dA = fmaf(dx, x, dA);
+      }
+      st_bf16x4(P.dg + row * D + 4 * lane, dg[0], dg[1], dg[2], dg[3]);
+    }
+    if (lane == 0) {
+      const float b = sigmoid_acc(__bfloat162float(p.beta[row]));
+      P.dbeta[row] = __float2bfloat16_rn(gb * b * (1.f - b));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dA += __shfl_xor_sync(0xffffffffu, dA, o);
+  reinterpret_cast<float4*>(s_dt[warp])[lane] = make_float4(ddt[0], ddt[1], ddt[2], ddt[3]);
+  if (lane == 0) s_dA[warp] = dA;
+  __syncthreads();
+  if (warp == 0) {
+    float t[4] = {0.f, 0.f, 0.f, 0.f}, a = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      const float4 x = reinterpret_cast<const float4*>(s_dt[w])[lane];
+      t[0] += x.x; t[1] += x.y; t[2] += x.z; t[3] += x.w;
+      a += s_dA[w];
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) atomicAdd(P.ddt_bias + (size_t)h * D + 4 * lane + j, t[j]);
+    if (lane == 0) atomicAdd(P.dA_log + h, a);
   }
 }
 
 }  // namespace
 
-// At most this many persistent CTAs (one per SM; more SMs than this are left to other work), so the
-// workspace size depends only on the problem's sizes.
-constexpr int64_t kBwdMaxCtas = 256;
+// At most this many persistent CTAs of the slice kernel (two per SM), so that the workspace size
+// depends only on the problem's sizes.
+constexpr int64_t kBwdMaxCtas = 512;
+constexpr int kFinishTokens = 64;  // tokens per CTA of the finishing kernel
 
 size_t bwd_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
   const int64_t t = total_tokens > 0 ? total_tokens : 0, n = num_seqs > 0 ? num_seqs : 0;
   const int64_t hh = num_heads > 0 ? num_heads : 0;
   const int64_t slots = t / kBwdChunk + n + 1;
-  const int64_t units = n * hh;
-  const int64_t ctas = units < kBwdMaxCtas ? units : kBwdMaxCtas;
-  return ((size_t)slots * hh + (size_t)ctas * kBwdChunk) * kStateElems * sizeof(float);
+  const int64_t work = n * hh * kSlices;
+  const int64_t ctas = work < kBwdMaxCtas ? work : kBwdMaxCtas;
+  const size_t ckpt = (size_t)slots * hh * kStateElems;
+  const size_t scratch = (size_t)ctas * kBwdChunk * kSliceElems;
+  const size_t part = (size_t)kSlices * (3 * (size_t)t * hh * kHeadDim + (size_t)t * hh);
+  return (ckpt + scratch + part) * sizeof(float);
 }
 
 cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const float* d_final, __nv_bfloat16* dq,
@@ -399,6 +457,9 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
   if (e != cudaSuccess || units == 0) return e;
   const int64_t tokens = f.cu_seqlens ? f.seqlen : f.seqlen * f.num_seqs;
   const int64_t slots = tokens / kBwdChunk + f.num_seqs + 1;
+  const int64_t work = units * kSlices;
+  int64_t grid = work < 2 * (int64_t)sms ? work : 2 * (int64_t)sms;
+  if (grid > kBwdMaxCtas) grid = kBwdMaxCtas;
   BwdParams P;
   P.f = f;
   P.d_out = d_out;
@@ -413,9 +474,12 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
   P.d_initial = d_initial;
   P.ckpt = static_cast<float*>(workspace);
   P.scratch = P.ckpt + (size_t)slots * f.num_heads * kStateElems;
-  int64_t grid = units < sms ? units : sms;
-  if (grid > kBwdMaxCtas) grid = kBwdMaxCtas;
+  const int64_t work_cap = work < kBwdMaxCtas ? work : kBwdMaxCtas;
+  P.part = P.scratch + (size_t)work_cap * kBwdChunk * kSliceElems;
   bwd_kernel<<<(unsigned)grid, kBwdThreads, 0, stream>>>(P);
+  if ((e = cudaGetLastError()) != cudaSuccess || tokens == 0) return e;
+  const dim3 fgrid((unsigned)((tokens + kFinishTokens - 1) / kFinishTokens), (unsigned)f.num_heads);
+  bwd_finish_kernel<<<fgrid, 256, 0, stream>>>(P, tokens, kFinishTokens);
   return cudaGetLastError();
 }
 

@@ -94,6 +94,14 @@ cudaError_t launch_segment_map(const FwdParams& p, void* workspace, float* map_M
 // S_out = M S_in + B for `units` (sequence, head) units (S_in null: zero).
 cudaError_t launch_state_affine(const float* M, const float* B, const float* S_in, float* S_out, int64_t units,
                                 int32_t transposed, cudaStream_t stream);
+// Zero padding of head sizes below 128 (kda_pad.cu): rows of w elements of esz bytes to / from
+// 128-wide rows, and [R][C] states to / from 128 x 128 ones.
+cudaError_t launch_pad_rows(const void* src, void* dst, int64_t rows, int w, int esz, cudaStream_t stream);
+// (rows are copied only if `nonzero` is null or *nonzero != 0)
+cudaError_t launch_unpad_rows(const void* src, void* dst, int64_t rows, int w, int esz, cudaStream_t stream,
+                              const int32_t* nonzero = nullptr);
+cudaError_t launch_pad_state(const float* src, float* dst, int64_t units, int R, int C, cudaStream_t stream);
+cudaError_t launch_unpad_state(const float* src, float* dst, int64_t units, int R, int C, cudaStream_t stream);
 // The backward pass (kda_bwd): workspace bytes, and the launch (zeroes dA_log / ddt_bias first).
 size_t bwd_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const float* d_final, __nv_bfloat16* dq,

@@ -200,3 +200,25 @@ def test_kcp_entry_points_validation(lib):
     assert af(vp(P), vp(P), vp(P + 4), vp(P), 4, 128, 0, None) == 1
     assert af(vp(P), vp(P), vp(P), vp(P), 4, 128, 2, None) == 1
     assert af(vp(P), vp(P), vp(P), vp(P), 0, 128, 0, None) == 0
+
+
+def test_fwd_ex_head_sizes(lib):
+    fn = lib.kda_fwd_ex
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def ex(K, V, ws_bytes=1 << 40):
+        return fn(vp(P), vp(P), vp(P), vp(P), vp(P), ctypes.c_float(0.088), vp(P), vp(P), ctypes.c_size_t(ws_bytes),
+                  vp(P), vp(P), ctypes.c_float(-5.0), None, None, None, ctypes.c_int32(0), ctypes.c_int64(64),
+                  ctypes.c_int32(1), ctypes.c_int32(K), ctypes.c_int32(V), ctypes.c_int32(0), ctypes.c_int32(0),
+                  ctypes.c_uint32(0), None)
+
+    assert ex(60, 64) == 2      # not a multiple of 8
+    assert ex(136, 128) == 2    # above 128
+    assert ex(0, 64) == 2
+    assert ex(64, 64) == 0      # empty batch: accepted, nothing launched
+    assert ex(64, 64, ws_bytes=16) == 3
+    # kda_fwd itself stays at 128 (FlashKDA's fwd)
+    assert call(lib, K=64, V=64) == 2
+    # padded sizes need room for the 128-wide copies; 128 needs exactly kda_workspace_size
+    assert lib.kda_workspace_size_ex(32768, 96, 1, 128, 128) == lib.kda_workspace_size(32768, 96, 1)
+    assert lib.kda_workspace_size_ex(4096, 8, 2, 64, 64) > lib.kda_workspace_size(4096, 8, 2) + 5 * 4096 * 8 * 256

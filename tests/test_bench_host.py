@@ -59,10 +59,13 @@ def test_peaks_come_from_the_measured_file():
 
 
 def test_traffic_summary_is_consistent():
-    """The committed DRAM traffic of one call is the sum of its launches' reads and writes and at
-    least the operator's own bytes (the items' round trip comes on top)."""
-    with open(os.path.join(ROOT, "profiles", "kda_fwd_prefill_h96_traffic.json")) as f:
+    """The committed DRAM traffic of one call (measured at 32 heads) is the sum of its launches'
+    reads and writes, at least the operator's own bytes at 32 heads (the items' round trip comes on
+    top), and scales to 96 heads by the head ratio."""
+    with open(os.path.join(ROOT, "profiles", "kda_fwd_prefill_h32_traffic.json")) as f:
         d = json.load(f)
-    total = sum(v["read"] + v["write"] for v in d["per_kernel"].values())
-    assert abs(total - d["dram_bytes_per_call"]) <= 1e-3 * d["dram_bytes_per_call"]
-    assert d["dram_bytes_per_call"] >= bench.algorithmic_bytes(32768, 96, 1)
+    total = sum(v["read"] + v["write"] for v in d["per_kernel_measured"].values())
+    assert abs(total - d["dram_bytes_per_call_measured"]) <= 1e-3 * d["dram_bytes_per_call_measured"]
+    assert d["dram_bytes_per_call_measured"] >= bench.algorithmic_bytes(32768, d["measured_heads"], 1)
+    assert d["scale_to_96_heads"] == 96 / d["measured_heads"]
+    assert abs(d["dram_bytes_per_call"] - d["scale_to_96_heads"] * d["dram_bytes_per_call_measured"]) <= 1e6
