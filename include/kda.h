@@ -244,8 +244,8 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const void*
                         kda_stream_t stream);
 
 /* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): one fp32
- * 128 x 128 checkpoint per (64-token chunk, head) for at most T / 64 + N + 1 chunk slots, a scratch
- * of 64 states of 128 x 32 for each of up to min(4 N H, 512) CTAs, and four slices of per-channel
+ * 128 x 128 checkpoint per (32-token chunk, head) for at most T / 32 + N + 1 chunk slots, a scratch
+ * of 32 states of 128 x 32 for each of up to min(4 N H, 512) CTAs, and four slices of per-channel
  * partial sums (3 x 128 + 1 fp32 per token and head).  Depends only on its arguments. */
 size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
@@ -261,7 +261,7 @@ size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t n
  *   dA_log fp32 [H], ddt_bias fp32 [H, K]  (overwritten: zeroed, then summed over all tokens)
  *   d_initial    fp32 [N, H, K, V] or NULL (not written)
  * Token by token on CUDA cores, four persistent CTAs per (sequence, head) (32 state columns each):
- * a forward that stores a checkpoint every 64 tokens, then chunk by chunk from the last a rerun from
+ * a forward that stores a checkpoint every 32 tokens, then chunk by chunk from the last a rerun from
  * the checkpoint and a reverse walk over its tokens; a second kernel sums the column slices and
  * applies the derivatives of the in-kernel transforms.  Gradient pointers are 16-byte aligned (dbeta 2, dA_log 4).  With
  * out-of-order cu_seqlens every document is treated as empty: the token gradients are not written

@@ -11,25 +11,28 @@
 // followed by the derivatives of the in-kernel transforms (L2 norms, sigmoid of beta, safe gate).
 //
 // The columns of the state evolve independently, so one (sequence, head) unit is split over four
-// CTAs of 32 state columns each (persistent over (unit, slice) pairs, two CTAs per SM), 256 threads,
-// the slice of the state and of its gradient in registers (16 rows x 1 column per thread).  A CTA
-// first runs the forward over its sequence, storing the slice at the start of every 64-token chunk in
-// the workspace; then, chunk by chunk from the last, it reruns the chunk's forward from its
+// CTAs of 32 state columns each (persistent over (unit, slice) pairs, two CTAs per SM, 256
+// threads).  Inside a CTA, warp w owns 4 columns over all 128 rows and lane l rows 4 l .. 4 l + 3,
+// so each thread holds a 4 x 4 block of the state and of its gradient, and the sums over rows that
+// the token chain needs (the prediction S^T khat and the delta gradient dS^T khat) are warp
+// shuffles: a warp runs the token recurrence on its columns without waiting for the others.  A CTA
+// first runs the forward over its sequence, storing its slice at the start of every 32-token chunk
+// in the workspace; then, chunk by chunk from the last, it reruns the chunk's forward from its
 // checkpoint, storing the slice before every token in a per-CTA scratch, and walks the chunk's tokens
-// backwards.  Sums over the state's rows run through shared memory across the warps, sums over its
-// columns through warp shuffles; what sums over all columns (dqhat, dkhat, dalpha per channel and
-// dbeta) is written per slice, and a second kernel adds the slices, applies the derivatives of the
-// L2 norms, the gate and the sigmoid, and adds the dA_log / dt_bias sums with one atomic per value
-// per CTA (the outputs are zeroed first).
+// backwards.  Each chunk's inputs are transformed once (norms, gate, sigmoid) into shared memory,
+// and the next token's scratch state is fetched during the current one.  What sums over columns
+// (dqhat, dkhat, dalpha per channel, dbeta) is added over the CTA's warps through shared memory (one
+// barrier per token) and written per slice; a second kernel adds the slices, applies the derivatives
+// of the L2 norms, the gate and the sigmoid, and adds the dA_log / dt_bias sums with one atomic per
+// value per CTA (the outputs are zeroed first).
 #include "kda_common.cuh"
 
 namespace kda {
 namespace {
 
 constexpr int kBwdThreads = 256;
-constexpr int kBwdChunk = 64;
-constexpr int kRows = 16;  // state rows per thread: warp w holds rows 16 w .. 16 w + 15
-constexpr int kSlice = 32;  // state columns per CTA (one per lane)
+constexpr int kBwdChunk = 32;  // tokens per checkpoint (and per staged chunk)
+constexpr int kSlice = 32;  // state columns per CTA (4 per warp)
 constexpr int kSlices = kHeadDim / kSlice;
 constexpr size_t kStateElems = (size_t)kHeadDim * kHeadDim;
 constexpr size_t kSliceElems = (size_t)kHeadDim * kSlice;
@@ -51,11 +54,6 @@ struct BwdParams {
   float* part;                  // per slice: dqhat, dkhat, dalpha [tokens, H, K]; then dbeta [slice][tokens, H]
 };
 
-struct TokenIn {
-  float q[kHeadDim], k[kHeadDim], a[kHeadDim], x[kHeadDim], sg[kHeadDim], v[kHeadDim], d[kHeadDim];
-  float nq, nk, b;
-};
-
 __device__ __forceinline__ float sigmoid_acc(float x) { return 1.0f / (1.0f + expf(-x)); }
 
 __device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16* p) {
@@ -72,107 +70,79 @@ __device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, float a, float b, fl
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-// One token's raw inputs, split over the CTA: warps 0..4 read 4 channels per lane of q, k, g, v and
-// d_out (warp 0 and 4 only for the backward step), lane 0 of warp 5 reads beta.  Fetched one token
-// ahead into registers, so that the global loads of token t + 1 overlap the work on token t.
-struct RawTok {
-  uint2 u;
-  float b;
+// Sum over the 32 lanes of a warp, every lane getting the totals.
+__device__ __forceinline__ void warp_allsum4(float (&x)[4]) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x[j] += __shfl_xor_sync(0xffffffffu, x[j], o);
+}
+__device__ __forceinline__ float warp_allsum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// A chunk's transformed inputs, staged in shared memory once per chunk (each warp transforms every
+// eighth token) and read by all warps: khat, qhat and alpha per channel, v and d_out on the slice's
+// columns, beta.
+struct ChunkIn {
+  float k[kBwdChunk][kHeadDim];
+  float q[kBwdChunk][kHeadDim];
+  float a[kBwdChunk][kHeadDim];
+  float v[kBwdChunk][kSlice];
+  float d[kBwdChunk][kSlice];
+  float b[kBwdChunk];
 };
 
-__device__ __forceinline__ RawTok fetch_token(const BwdParams& P, size_t row, bool full) {
+__device__ __forceinline__ void stage_chunk(const BwdParams& P, ChunkIn& s, int64_t t_begin, int len, int h,
+                                            int scol0, float ea, float4 dt, bool full) {
   const FwdParams& p = P.f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = p.num_heads;
   constexpr int D = kHeadDim;
-  RawTok r;
-  r.u = make_uint2(0, 0);
-  r.b = 0.f;
-  const __nv_bfloat16* src = nullptr;
-  if (warp == 0 && full) src = p.q;
-  else if (warp == 1) src = p.k;
-  else if (warp == 2) src = p.g;
-  else if (warp == 3) src = p.v;
-  else if (warp == 4 && full) src = P.d_out;
-  if (src) r.u = *reinterpret_cast<const uint2*>(src + row * D + 4 * lane);
-  if (warp == 5 && lane == 0) r.b = __bfloat162float(p.beta[row]);
-  return r;
-}
-
-__device__ __forceinline__ float4 bf16x4_of(uint2 u) {
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-  return make_float4(a.x, a.y, b.x, b.y);
-}
-
-// The transformed inputs of one token into shared memory, from the fetched raw values.  `full`:
-// also qhat, d_out and the gate's intermediates (the backward step); otherwise only what the forward
-// step reads (khat, alpha, beta, v).  dt: this lane's 4 channels of dt_bias[h].
-__device__ __forceinline__ void stage_token(const BwdParams& P, const RawTok& r, float ea, float4 dt, TokenIn& s,
-                                            bool full) {
-  const FwdParams& p = P.f;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 0 || warp == 1) {
-    if (warp == 0 && !full) return;
-    const float4 x4 = bf16x4_of(r.u);
-    float ss = x4.x * x4.x + x4.y * x4.y + x4.z * x4.z + x4.w * x4.w;
+  const float dts[4] = {dt.x, dt.y, dt.z, dt.w};
+  for (int i = warp; i < len; i += kBwdThreads / 32) {
+    const size_t row = (size_t)(t_begin + i) * H + h;
+    const float4 k4 = ld_bf16x4(p.k + row * D + 4 * lane);
+    const float4 g4 = ld_bf16x4(p.g + row * D + 4 * lane);
+    const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w};
+    const float nk = sqrtf(warp_allsum(kv[0] * kv[0] + kv[1] * kv[1] + kv[2] * kv[2] + kv[3] * kv[3]) + kL2Eps);
+    float av[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float n = sqrtf(ss + kL2Eps);
-    float* dst = warp == 0 ? s.q : s.k;
-    reinterpret_cast<float4*>(dst)[lane] = make_float4(x4.x / n, x4.y / n, x4.z / n, x4.w / n);
-    if (lane == 0) (warp == 0 ? s.nq : s.nk) = n;
-  } else if (warp == 2) {
-    const float4 g4 = bf16x4_of(r.u);
-    const float gv[4] = {g4.x, g4.y, g4.z, g4.w}, dts[4] = {dt.x, dt.y, dt.z, dt.w};
-    float xs[4], sgs[4], as[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      xs[j] = ea * (gv[j] + dts[j]);
-      sgs[j] = sigmoid_acc(xs[j]);
-      as[j] = expf(p.lower_bound * sgs[j]);
-    }
-    reinterpret_cast<float4*>(s.a)[lane] = make_float4(as[0], as[1], as[2], as[3]);
+    for (int j = 0; j < 4; ++j) av[j] = expf(p.lower_bound * sigmoid_acc(ea * (gv[j] + dts[j])));
+    reinterpret_cast<float4*>(s.k[i])[lane] = make_float4(kv[0] / nk, kv[1] / nk, kv[2] / nk, kv[3] / nk);
+    reinterpret_cast<float4*>(s.a[i])[lane] = make_float4(av[0], av[1], av[2], av[3]);
+    if (lane < kSlice / 4) reinterpret_cast<float4*>(s.v[i])[lane] = ld_bf16x4(p.v + row * D + scol0 + 4 * lane);
+    if (lane == 0) s.b[i] = sigmoid_acc(__bfloat162float(p.beta[row]));
     if (full) {
-      reinterpret_cast<float4*>(s.x)[lane] = make_float4(xs[0], xs[1], xs[2], xs[3]);
-      reinterpret_cast<float4*>(s.sg)[lane] = make_float4(sgs[0], sgs[1], sgs[2], sgs[3]);
+      const float4 q4 = ld_bf16x4(p.q + row * D + 4 * lane);
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+      const float nq = sqrtf(warp_allsum(qv[0] * qv[0] + qv[1] * qv[1] + qv[2] * qv[2] + qv[3] * qv[3]) + kL2Eps);
+      reinterpret_cast<float4*>(s.q[i])[lane] = make_float4(qv[0] / nq, qv[1] / nq, qv[2] / nq, qv[3] / nq);
+      if (lane < kSlice / 4) reinterpret_cast<float4*>(s.d[i])[lane] = ld_bf16x4(P.d_out + row * D + scol0 + 4 * lane);
     }
-  } else if (warp == 3) {
-    reinterpret_cast<float4*>(s.v)[lane] = bf16x4_of(r.u);
-  } else if (warp == 4) {
-    if (full) reinterpret_cast<float4*>(s.d)[lane] = bf16x4_of(r.u);
-  } else if (warp == 5 && lane == 0) {
-    s.b = sigmoid_acc(r.b);
   }
 }
 
-// Sum over the 32 lanes of 16 values at once: after the exchange, lanes 2 i and 2 i + 1 hold the
-// total of value i.
-__device__ __forceinline__ float transpose_reduce16(const float (&x)[16], int lane) {
-  float w8[8], w4[4], w2[2];
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) w8[j] = (b4 ? x[j + 8] : x[j]) + __shfl_xor_sync(0xffffffffu, b4 ? x[j] : x[j + 8], 16);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) w4[j] = (b3 ? w8[j + 4] : w8[j]) + __shfl_xor_sync(0xffffffffu, b3 ? w8[j] : w8[j + 4], 8);
-#pragma unroll
-  for (int j = 0; j < 2; ++j) w2[j] = (b2 ? w4[j + 2] : w4[j]) + __shfl_xor_sync(0xffffffffu, b2 ? w4[j] : w4[j + 2], 4);
-  float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
-  return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
-}
-
-// One CTA per (unit, column slice): the state's 128 rows and the slice's kSlice columns (a 16 x 1
-// block per thread: warp w holds rows 16 w .. + 15, lane l column l of the slice).  The columns of
-// the state evolve independently, so each slice runs the whole token recurrence on its own; what
-// sums over columns (dqhat, dkhat, dalpha per row, dbeta) is written per slice and summed by
-// bwd_finish_kernel, which also applies the derivatives of the in-kernel transforms.
+// One CTA per (unit, slice of 32 state columns); warp w owns columns 4 w .. 4 w + 3 of the slice over
+// all 128 rows, lane l rows 4 l .. 4 l + 3 (a 4 x 4 block of the state and of its gradient per
+// thread).  The columns of the state evolve independently, so every warp runs the token recurrence
+// on its own columns: the sums over rows (the prediction and the delta gradient) are warp shuffles,
+// and the token chain needs no barrier of the CTA.  Each chunk's inputs are transformed once into
+// shared memory.  What sums over columns (dqhat, dkhat, dalpha per row, dbeta) is summed over the
+// CTA's warps through shared memory (one barrier per token) and written per slice for
+// bwd_finish_kernel.  Checkpoints and the per-token scratch are stored per thread (16 contiguous
+// floats), since every thread reads back only what it wrote.
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
   constexpr int D = kHeadDim;
-  __shared__ __align__(16) TokenIn s;
-  __shared__ __align__(16) float red[2][8][kSlice];
+  extern __shared__ __align__(16) uint8_t bwd_smem[];
+  ChunkIn& s = *reinterpret_cast<ChunkIn*>(bwd_smem);
+  float (*part)[8][3][D] = reinterpret_cast<float (*)[8][3][D]>(bwd_smem + sizeof(ChunkIn));  // [buffer][warp]
+  float (*part_beta)[8] = reinterpret_cast<float (*)[8]>(bwd_smem + sizeof(ChunkIn) + 2 * 8 * 3 * D * sizeof(float));
   const FwdParams& p = P.f;
   const int H = p.num_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r0 = kRows * warp;
   const int64_t units = (int64_t)p.num_seqs * H;
   const int64_t work = units * kSlices;
   float* const scr = P.scratch + (size_t)blockIdx.x * kBwdChunk * kSliceElems;
@@ -183,7 +153,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
     const int64_t u = wi / kSlices;
     const int sl = (int)(wi - u * kSlices);
     const int n = (int)(u / H), h = (int)(u % H);
-    const int col = sl * kSlice + lane;  // this thread's state column (v)
+    const int scol0 = sl * kSlice;         // the slice's first state column
+    const int col0 = scol0 + 4 * warp;     // this warp's first state column (v)
     int64_t bos, eos;
     seq_range(p, n, bos, eos);
     if (!seqlens_ok) eos = bos;
@@ -193,141 +164,180 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
     const int64_t ck0 = bos / kBwdChunk + n;  // this sequence's first checkpoint slot
     const float ea = expf(p.A_log[h]);
     const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-    auto tok_row = [&](int64_t t) { return (size_t)t * H + h; };
-    // checkpoint c of this slice: [128 rows][kSlice]
+    // a slice state stored per thread: 16 contiguous floats at thread index tid
     auto ck_ptr = [&](int c) { return P.ckpt + (((size_t)(ck0 + c) * H + h) * kSlices + sl) * kSliceElems; };
-    float* const part_q = P.part + (size_t)sl * 3 * rows_total * D;  // per slice: dqhat, dkhat, dalpha rows
-    float* const part_k = part_q + (size_t)rows_total * D;
-    float* const part_a = part_k + (size_t)rows_total * D;
+    float* const part_q = P.part + (size_t)sl * 3 * rows_total * D;
     float* const part_b = P.part + (size_t)kSlices * 3 * rows_total * D + (size_t)sl * rows_total;
 
-    float S[kRows];
+    float S[4][4];  // S[4 lane + i][col0 + j]
 #pragma unroll
-    for (int i = 0; i < kRows; ++i) S[i] = p.initial_state ? p.initial_state[soff + (size_t)(r0 + i) * D + col] : 0.f;
-    auto store_state = [&](float* dst) {
+    for (int i = 0; i < 4; ++i) {
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (p.initial_state) t = *reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)(4 * lane + i) * D + col0);
+      S[i][0] = t.x; S[i][1] = t.y; S[i][2] = t.z; S[i][3] = t.w;
+    }
+    auto store_state = [&](float* base) {
+      float4* dst = reinterpret_cast<float4*>(base + (size_t)tid * 16);
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) dst[(r0 + i) * kSlice + lane] = S[i];
+      for (int i = 0; i < 4; ++i) dst[i] = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
     };
-    auto load_state = [&](const float* src) {
+    auto load_state = [&](const float* base) {
+      const float4* src = reinterpret_cast<const float4*>(base + (size_t)tid * 16);
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) S[i] = src[(r0 + i) * kSlice + lane];
+      for (int i = 0; i < 4; ++i) {
+        const float4 t = src[i];
+        S[i][0] = t.x; S[i][1] = t.y; S[i][2] = t.z; S[i][3] = t.w;
+      }
     };
-    // the sum over the 8 warps of one value per thread (its column): red[w][lane]
-    auto col_sum = [&](float (*rd)[kSlice], float x) {
-      rd[warp][lane] = x;
-      __syncthreads();
-      float t = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) t += rd[w][lane];
+    // the chunk's token i, this thread's rows and the warp's columns
+    auto row4 = [&](const float (*m)[D], int i) {
+      const float4 t = reinterpret_cast<const float4*>(m[i])[lane];
       return t;
     };
-    auto forward_token = [&]() {
-      float pr = 0.f;
+    auto forward_token = [&](int i) {
+      const float4 a4 = row4(s.a, i), k4 = row4(s.k, i);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
+      const float4 v4 = reinterpret_cast<const float4*>(s.v[i])[warp];
+      const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+      const float b = s.b[i];
+      float pr[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        S[i] *= s.a[r0 + i];
-        pr = fmaf(S[i], s.k[r0 + i], pr);
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          S[r][j] *= av[r];
+          pr[j] = fmaf(S[r][j], kv[r], pr[j]);
+        }
+      warp_allsum4(pr);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float d = b * (vv[j] - pr[j]);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) S[r][j] = fmaf(kv[r], d, S[r][j]);
       }
-      const float d = s.b * (s.v[col] - col_sum(red[0], pr));
-#pragma unroll
-      for (int i = 0; i < kRows; ++i) S[i] = fmaf(s.k[r0 + i], d, S[i]);
     };
 
     // ---------------------------------------------------------------- forward with checkpoints
-    RawTok rt = fetch_token(P, tok_row(bos), false);  // (L = 0: never staged)
     for (int c = 0; c < nch; ++c) {
+      const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
+      const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
       store_state(ck_ptr(c));
-      const int64_t t_end = min(bos + (int64_t)(c + 1) * kBwdChunk, eos);
-      for (int64_t t = bos + (int64_t)c * kBwdChunk; t < t_end; ++t) {
-        __syncthreads();
-        stage_token(P, rt, ea, dt, s, false);
-        if (t + 1 < eos) rt = fetch_token(P, tok_row(t + 1), false);
-        __syncthreads();
-        forward_token();
-      }
+      __syncthreads();  // the previous chunk's staged inputs are read
+      stage_chunk(P, s, t_begin, len, h, scol0, ea, dt, false);
+      __syncthreads();
+      for (int i = 0; i < len; ++i) forward_token(i);
     }
 
     // ---------------------------------------------------------------- backward, chunk by chunk
-    float dS[kRows];
+    float dS[4][4];
 #pragma unroll
-    for (int i = 0; i < kRows; ++i) dS[i] = P.d_final ? P.d_final[soff + (size_t)(r0 + i) * D + col] : 0.f;
-
+    for (int i = 0; i < 4; ++i) {
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (P.d_final) t = *reinterpret_cast<const float4*>(P.d_final + soff + (size_t)(4 * lane + i) * D + col0);
+      dS[i][0] = t.x; dS[i][1] = t.y; dS[i][2] = t.z; dS[i][3] = t.w;
+    }
+    int buf = 0;
     for (int c = nch - 1; c >= 0; --c) {
       const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
       const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
+      __syncthreads();  // the previous chunk's staged inputs and partials are read
+      stage_chunk(P, s, t_begin, len, h, scol0, ea, dt, true);
+      __syncthreads();
       // rerun the chunk's forward from its checkpoint, keeping the state before each token
       load_state(ck_ptr(c));
-      RawTok rf = fetch_token(P, tok_row(t_begin), false);
       for (int i = 0; i < len; ++i) {
         store_state(scr + (size_t)i * kSliceElems);
-        __syncthreads();
-        stage_token(P, rf, ea, dt, s, false);
-        if (i + 1 < len) rf = fetch_token(P, tok_row(t_begin + i + 1), false);
-        __syncthreads();
-        forward_token();
+        forward_token(i);
       }
-      // the chunk's tokens backwards; S holds S_{t-1} of the token at hand, loaded from the scratch
-      // (written by this thread above) during the token after it
-      RawTok rb = fetch_token(P, tok_row(t_begin + len - 1), true);
+      // the chunk's tokens backwards; S holds S_{t-1} of the token at hand (from the scratch)
       load_state(scr + (size_t)(len - 1) * kSliceElems);
       for (int i = len - 1; i >= 0; --i) {
-        const size_t row = tok_row(t_begin + i);
-        __syncthreads();
-        stage_token(P, rb, ea, dt, s, true);
-        if (i > 0) rb = fetch_token(P, tok_row(t_begin + i - 1), true);
-        __syncthreads();
-        const float b = s.b, scale = p.scale;
-        float pr = 0.f;
+        const size_t row = (size_t)(t_begin + i) * H + h;
+        const float4 a4 = row4(s.a, i), k4 = row4(s.k, i), q4 = row4(s.q, i);
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+        const float4 v4 = reinterpret_cast<const float4*>(s.v[i])[warp];
+        const float4 d4 = reinterpret_cast<const float4*>(s.d[i])[warp];
+        const float vv[4] = {v4.x, v4.y, v4.z, v4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        const float b = s.b[i], scale = p.scale;
+        // p = Stil^T khat (columns), delta
+        float pj[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ii = 0; ii < kRows; ++ii) pr = fmaf(s.a[r0 + ii] * S[ii], s.k[r0 + ii], pr);
-        const float pj = col_sum(red[0], pr);
-        const float vj = s.v[col], doj = s.d[col];
-        const float dl = b * (vj - pj);
-        // dS += scale qhat do^T;  dqhat rows (this slice) = scale S_t do;  ddelta = dS^T khat
-        float rq[kRows], pd = 0.f;
+        for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int ii = 0; ii < kRows; ++ii) {
-          const float kk = s.k[r0 + ii];
-          rq[ii] = scale * fmaf(kk, dl, s.a[r0 + ii] * S[ii]) * doj;
-          dS[ii] = fmaf(scale * s.q[r0 + ii], doj, dS[ii]);
-          pd = fmaf(dS[ii], kk, pd);
+          for (int j = 0; j < 4; ++j) pj[j] = fmaf(av[r] * S[r][j], kv[r], pj[j]);
+        warp_allsum4(pj);
+        float dl[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dl[j] = b * (vv[j] - pj[j]);
+        // dS += scale qhat do^T;  dqhat rows = scale S_t do;  ddelta = dS^T khat
+        float rq[4], dd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float acc = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc = fmaf(fmaf(kv[r], dl[j], av[r] * S[r][j]), dv[j], acc);
+            dS[r][j] = fmaf(scale * qv[r], dv[j], dS[r][j]);
+            dd[j] = fmaf(dS[r][j], kv[r], dd[j]);
+          }
+          rq[r] = scale * acc;
         }
-        const float tq = transpose_reduce16(rq, lane);
-        const float ddl = col_sum(red[1], pd);
-        const float dp = -b * ddl;
-        if (warp == 0) {
-          P.dv[row * D + col] = __float2bfloat16_rn(b * ddl);
-          float db = ddl * (vj - pj);
+        warp_allsum4(dd);
+        float dp[4], db = 0.f;
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
-          if (lane == 0) part_b[row] = db;
+        for (int j = 0; j < 4; ++j) {
+          dp[j] = -b * dd[j];
+          db = fmaf(dd[j], vv[j] - pj[j], db);
         }
+        if (lane == 0) st_bf16x4(P.dv + row * D + col0, b * dd[0], b * dd[1], b * dd[2], b * dd[3]);
         // dkhat = dS delta + Stil dp;  dStil = dS + khat dp^T;  dalpha;  dS <- Diag(alpha) dStil
-        float rk[kRows];
+        float rk[4], ra[4];
 #pragma unroll
-        for (int ii = 0; ii < kRows; ++ii) rk[ii] = fmaf(dS[ii], dl, s.a[r0 + ii] * S[ii] * dp);
-        const float tk = transpose_reduce16(rk, lane);
-        float ra[kRows];
+        for (int r = 0; r < 4; ++r) {
+          float ak = 0.f, aa = 0.f;
 #pragma unroll
-        for (int ii = 0; ii < kRows; ++ii) {
-          const float dst = fmaf(s.k[r0 + ii], dp, dS[ii]);
-          ra[ii] = dst * S[ii];
-          dS[ii] = s.a[r0 + ii] * dst;
+          for (int j = 0; j < 4; ++j) {
+            ak = fmaf(dS[r][j], dl[j], ak);
+            ak = fmaf(av[r] * S[r][j], dp[j], ak);
+            const float dst = fmaf(kv[r], dp[j], dS[r][j]);
+            aa = fmaf(dst, S[r][j], aa);
+            dS[r][j] = av[r] * dst;
+          }
+          rk[r] = ak;
+          ra[r] = aa;
         }
         if (i > 0) load_state(scr + (size_t)(i - 1) * kSliceElems);  // the next token's S_{t-1}
-        const float ta = transpose_reduce16(ra, lane);
-        if ((lane & 1) == 0) {
-          const size_t o = row * D + r0 + (lane >> 1);
-          part_q[o] = tq;
-          part_k[o] = tk;
-          part_a[o] = ta;
+        // the warps' row partials through shared memory, summed over the slice's 32 columns
+        reinterpret_cast<float4*>(part[buf][warp][0])[lane] = make_float4(rq[0], rq[1], rq[2], rq[3]);
+        reinterpret_cast<float4*>(part[buf][warp][1])[lane] = make_float4(rk[0], rk[1], rk[2], rk[3]);
+        reinterpret_cast<float4*>(part[buf][warp][2])[lane] = make_float4(ra[0], ra[1], ra[2], ra[3]);
+        if (lane == 0) part_beta[buf][warp] = db;
+        __syncthreads();
+        // 384 row sums: thread t sums entries t and t + 256 (of 3 x 128)
+        for (int e = tid; e < 3 * D; e += kBwdThreads) {
+          const int which = e / D, r = e % D;
+          float acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) acc += part[buf][w][which][r];
+          part_q[(size_t)which * rows_total * D + row * D + r] = acc;
         }
+        if (tid == 0) {
+          float acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) acc += part_beta[buf][w];
+          part_b[row] = acc;
+        }
+        buf ^= 1;  // the next token writes the other buffer; this one is read until the next barrier
       }
     }
     if (P.d_initial) {
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) P.d_initial[soff + (size_t)(r0 + i) * D + col] = dS[i];
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(P.d_initial + soff + (size_t)(4 * lane + i) * D + col0) =
+            make_float4(dS[i][0], dS[i][1], dS[i][2], dS[i][3]);
     }
+    __syncthreads();  // shared partials of this item are read before the next item writes them
   }
 }
 
@@ -476,7 +486,14 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
   P.scratch = P.ckpt + (size_t)slots * f.num_heads * kStateElems;
   const int64_t work_cap = work < kBwdMaxCtas ? work : kBwdMaxCtas;
   P.part = P.scratch + (size_t)work_cap * kBwdChunk * kSliceElems;
-  bwd_kernel<<<(unsigned)grid, kBwdThreads, 0, stream>>>(P);
+  const size_t smem = sizeof(ChunkIn) + (2 * 8 * 3 * kHeadDim + 2 * 8) * sizeof(float);
+  static bool attr_done[64] = {};
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if ((e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    attr_done[dev] = true;
+  }
+  bwd_kernel<<<(unsigned)grid, kBwdThreads, smem, stream>>>(P);
   if ((e = cudaGetLastError()) != cudaSuccess || tokens == 0) return e;
   const dim3 fgrid((unsigned)((tokens + kFinishTokens - 1) / kFinishTokens), (unsigned)f.num_heads);
   bwd_finish_kernel<<<fgrid, 256, 0, stream>>>(P, tokens, kFinishTokens);
