@@ -87,7 +87,10 @@ def kcp_forward(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_st
     is the sequences' initial state ([B, H, K, V], or [B, H, V, K] with ``state_transposed``), the
     same on every rank, None for zero.  Returns this rank's output segment and, with
     ``output_final_state``, the final states of the whole sequences (the same on every rank).
-    Every rank must call it with the same B, H and flags; segment lengths may differ."""
+    Every rank must call it with the same B, H and flags; segment lengths may differ but must be at
+    least one token."""
+    if q.shape[1] == 0:
+        raise ValueError("kcp_forward: every rank's segment must hold at least one token")
     ops = DeviceOps() if ops is None else ops
     comm = ProcessGroupComm(group) if comm is None else comm
     rank, world = comm.rank, comm.world

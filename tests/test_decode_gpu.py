@@ -200,3 +200,22 @@ def test_decode_matches_chunked_prefill_continuation(cuda_device):
         outs.append(o_t)
     o = torch.cat(outs, dim=1).float().cpu().double().numpy()
     check(o, state.cpu().double().numpy(), o_ref, s_ref, "prefill 300 + decode 5")
+
+
+def test_decode_zero_tokens_copies_states(cuda_device):
+    """seqlen = 0: no token, the requests' states go from the in pool to the out pool unchanged."""
+    B, H = 5, 2
+    gen = torch.Generator().manual_seed(66)
+    pool = torch.randn(7, H, 128, 128, generator=gen).to(cuda_device)
+    idx = torch.tensor([6, 0, -1, 3, 2], dtype=torch.int32, device=cuda_device)
+    dev = cuda_device
+    # zero-token views of real allocations, so that every pointer is valid and 16-byte aligned
+    q, k, v, g, out = (torch.zeros(B, 1, H, 128, dtype=torch.bfloat16, device=dev)[:, :0] for _ in range(5))
+    beta = torch.zeros(B, 1, H, dtype=torch.bfloat16, device=dev)[:, :0]
+    p_out = torch.full_like(pool, float("nan"))
+    kda.decode(q, k, v, g, beta, 0.088, out, torch.zeros(H, device=dev), torch.zeros(H, 128, device=dev), -5.0,
+               pool, p_out, idx)
+    torch.cuda.synchronize()
+    used = [6, 0, 3, 2]
+    assert torch.equal(p_out[used], pool[used])
+    assert torch.isnan(p_out[[1, 4, 5]]).all()
