@@ -214,32 +214,96 @@ def bench_backward(dev, steps, warmup, seed=0):
     d_out = torch.randn(x.v.shape, generator=gen, device=dev).to(torch.bfloat16)
     ws = torch.empty(kda.bwd_workspace_size(BWD_TOKENS, HEADS, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # the training forward stores the chunk-start states the backward starts from
+    ck = torch.empty(kda.checkpoint_size(BWD_TOKENS, HEADS, 1) // 4, dtype=torch.float32, device=dev)
+    fws = kda.new_workspace(BWD_TOKENS, HEADS, 1, dev)
+    out = torch.empty_like(x.v)
+    kda.fwd_checkpointed(x.q, x.k, x.v, x.g, x.beta, x.scale, out, fws, x.A_log, x.dt_bias, x.lower_bound, ck,
+                         cu_seqlens=x.cu_seqlens, stream=stream.cuda_stream)
 
-    def step():
-        kda.bwd(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, d_out,
-                cu_seqlens=x.cu_seqlens, workspace=ws, stream=stream.cuda_stream)
+    def timed(checkpoints):
+        def step():
+            kda.bwd(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, d_out,
+                    cu_seqlens=x.cu_seqlens, workspace=ws, stream=stream.cuda_stream, checkpoints=checkpoints)
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
 
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
+    ms = timed(ck)
+    ms_without = timed(None)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
-        step()
+        kda.fwd_checkpointed(x.q, x.k, x.v, x.g, x.beta, x.scale, out, fws, x.A_log, x.dt_bias, x.lower_bound, ck,
+                             cu_seqlens=x.cu_seqlens, stream=stream.cuda_stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    ms_fwd_ck = e0.elapsed_time(e1) / steps
     th = BWD_TOKENS * HEADS
     alg = BWD_BYTES_PER_TOKEN_HEAD * th
     hbm_peak, _, peak_kind = load_peaks()
     gbs = alg / (ms * 1e-3) / 1e9
-    return {"workload": f"backward: B=1 T={BWD_TOKENS} H={HEADS} K=V=128, gradients of every input",
+    return {"workload": f"backward: B=1 T={BWD_TOKENS} H={HEADS} K=V=128, gradients of every input, from the "
+                        "chunk-start states the checkpointing forward stored",
             "ms_per_step": ms, "value": th / (ms * 1e-3) / 1e6, "unit": UNIT,
+            "ms_per_step_without_checkpoints": ms_without,
+            "checkpointing_forward_ms": ms_fwd_ck,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
                          "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
                          "note": "token-serial CUDA-core kernel: bound by its per-token dependency chain, "
                                  "not by HBM"},
             "gpu_launches": steps}
+
+
+KCP_RANKS = 8
+
+
+def bench_kcp_rank(dev, steps, warmup, seed=0):
+    """The device work one rank of an 8-rank sequence-parallel prefill does on its 4096-token
+    segment of the 32K x 96-head prefill (the rank in the middle: segment map, the fold of four
+    earlier maps, the forward from the folded state, the fold of three later maps), timed on one GPU
+    with the other ranks' maps stood in by this rank's own (the all-gather is not included: every GPU
+    call here has one GPU)."""
+    import kda_inputs
+    import kimi_delta_attention_24_b200 as kda
+    from kimi_delta_attention_24_b200.kcp import DeviceOps
+
+    T = T_TOK // KCP_RANKS
+    x = kda_inputs.make_random("kcp", None, HEADS, seed=seed, varlen=False, batch=1, seqlen=T, device=dev)
+    ops = DeviceOps()
+    r = KCP_RANKS // 2
+
+    def step():
+        M, Bm = ops.segment_map(x.q, x.k, x.v, x.g, x.beta, x.A_log, x.dt_bias, x.lower_bound, 0)
+        S = None
+        for _ in range(r):
+            S = ops.fold(M, Bm, S, False)
+        _, S_end = ops.forward(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, S, 0, False)
+        for _ in range(KCP_RANKS - r - 1):
+            S_end = ops.fold(M, Bm, S_end, False)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"workload": f"sequence-parallel prefill, device work of rank {r} of {KCP_RANKS}: a {T}-token segment "
+                        f"of the B=1 T={T_TOK} H={HEADS} prefill (segment map, {KCP_RANKS - 1} folds, forward); "
+                        "the all-gather of the maps is not included",
+            "ms_per_step": ms, "segment_token_heads_per_s_M": T * HEADS / (ms * 1e-3) / 1e6,
+            "note": "one GPU only: measures a rank's device work, not a multi-GPU run"}
 
 
 def cpu_oracle_sample(target_s=15.0):
@@ -300,6 +364,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
+    ap.add_argument("--no-kcp", action="store_true", help="skip the sequence-parallel rank-work measurement")
     ap.add_argument("--heads", type=int, default=HEADS,
                     help="heads of the prefill workload (default 96; fewer only for small profiling runs)")
     args = ap.parse_args()
@@ -454,6 +519,8 @@ def main():
         line["decode"] = bench_decode(dev, steps=max(args.steps, 10), warmup=args.warmup, seed=rank)
     if not args.no_backward:
         line["backward"] = bench_backward(dev, steps=2, warmup=1, seed=rank)
+    if not args.no_kcp:
+        line["kcp_rank_work"] = bench_kcp_rank(dev, steps=5, warmup=2, seed=rank)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

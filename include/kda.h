@@ -224,7 +224,9 @@ kda_status_t kda_fwd_static_workspace(const void* q, const void* k, const void* 
  *                  KDA_FLAG_BETA_PRECOMPUTED);  A_log fp32 [H], dt_bias fp32 [H, 128].
  *   state_in / state_out  fp32 pools [num_slots, H, 128, 128] (S[k][v], or S^T with
  *                  state_transposed = 1).  state_in NULL means zero states; state_out NULL means
- *                  no write; they may be the same pool (in-place update).
+ *                  no write; they may be the same pool (in-place update).  With seqlen = 0 the
+ *                  requests' states are copied from state_in to state_out unchanged (the token
+ *                  tensors, A_log and dt_bias are then not read and may be NULL).
  *   state_indices  int32 [batch]: the pool slot of each request; NULL means slot b for request b.
  *                  A negative index skips the request (nothing read or written: padding).  The
  *                  non-negative indices of one call must be distinct.  An index >= num_slots
@@ -243,10 +245,26 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const void*
                         int32_t state_transposed, uint32_t flags, void* workspace,
                         kda_stream_t stream);
 
-/* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): one fp32
- * 128 x 128 checkpoint per (32-token chunk, head) for at most T / 32 + N + 1 chunk slots, a scratch
- * of 32 states of 128 x 32 for each of up to min(4 N H, 512) CTAs, and four slices of per-channel
- * partial sums (3 x 128 + 1 fp32 per token and head).  Depends only on its arguments. */
+/* Bytes of the checkpoints kda_fwd_checkpointed writes for (T, H, N): one fp32 128 x 128 state per
+ * (64-token chunk, head) for at most T / 64 + N + 1 chunk slots (3.2 GB at T = 32768, H = 96). */
+size_t kda_checkpoint_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
+
+/* kda_fwd (K = V = 128, the in-kernel transforms on) that also stores, for the backward pass, the
+ * state at the start of every 64-token chunk of every (sequence, head): fp32 S^T [v][k], 64 KB per
+ * (chunk, head), slot floor(bos_n / 64) + n + c for chunk c of sequence n (bos_n its first token).
+ * checkpoints: device, 16-byte aligned, at least kda_checkpoint_size bytes.  Otherwise as kda_fwd. */
+kda_status_t kda_fwd_checkpointed(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                  float scale, void* out, void* workspace, size_t workspace_bytes,
+                                  const float* A_log, const float* dt_bias, float lower_bound,
+                                  const float* initial_state, float* final_state, float* checkpoints,
+                                  size_t checkpoint_bytes, const int32_t* cu_seqlens, int32_t batch, int64_t seqlen,
+                                  int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
+                                  kda_stream_t stream);
+
+/* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): room for the
+ * checkpoints (as kda_checkpoint_size; used when the call is given none), a scratch of 64 states of
+ * 128 x 32 for each of up to min(4 N H, 512) CTAs, and four slices of per-channel partial sums
+ * (3 x 128 + 1 fp32 per token and head).  Depends only on its arguments. */
 size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
 /* The backward pass: gradients of sum(d_out * out) + sum(d_final * final_state) with respect to
@@ -255,20 +273,23 @@ size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t n
  * errors as kda_fwd (state_transposed = 0: states and their gradients are [N, H, K, V]), plus
  *   d_out        bf16 [batch, seqlen, H, V]   the output's gradient
  *   d_final      fp32 [N, H, K, V] or NULL (zero)   the final state's gradient
+ *   checkpoints  what kda_fwd_checkpointed stored for the same inputs, or NULL: then the backward
+ *                first runs the forward itself to make them (in the workspace)
  * and writes
  *   dq, dk, dg   bf16 [batch, seqlen, H, K];  dv bf16 [batch, seqlen, H, V];  dbeta bf16
  *                [batch, seqlen, H] (w.r.t. the raw beta, before the sigmoid; dg w.r.t. the raw gate)
  *   dA_log fp32 [H], ddt_bias fp32 [H, K]  (overwritten: zeroed, then summed over all tokens)
  *   d_initial    fp32 [N, H, K, V] or NULL (not written)
  * Token by token on CUDA cores, four persistent CTAs per (sequence, head) (32 state columns each):
- * a forward that stores a checkpoint every 32 tokens, then chunk by chunk from the last a rerun from
- * the checkpoint and a reverse walk over its tokens; a second kernel sums the column slices and
- * applies the derivatives of the in-kernel transforms.  Gradient pointers are 16-byte aligned (dbeta 2, dA_log 4).  With
+ * (without checkpoints) a forward that stores one every 64 tokens, then chunk by chunk from the
+ * last a rerun from the checkpoint and a reverse walk over its tokens; a second kernel sums the
+ * column slices and applies the derivatives of the in-kernel transforms.  Gradient pointers are 16-byte aligned (dbeta 2, dA_log 4).  With
  * out-of-order cu_seqlens every document is treated as empty: the token gradients are not written
  * and d_initial = d_final (there is no status word to report it). */
 kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
                      const float* A_log, const float* dt_bias, float lower_bound, const float* initial_state,
-                     const void* d_out, const float* d_final, void* dq, void* dk, void* dv, void* dg, void* dbeta,
+                     const void* d_out, const float* d_final, const float* checkpoints, void* dq, void* dk,
+                     void* dv, void* dg, void* dbeta,
                      float* dA_log, float* ddt_bias, float* d_initial, void* workspace, size_t workspace_bytes,
                      const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
                      int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs, kda_stream_t stream);

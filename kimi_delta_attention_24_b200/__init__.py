@@ -24,7 +24,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["get_workspace_size_ex", "fwd", "fwd_recurrent", "decode", "segment_map", "state_affine", "bwd", "bwd_workspace_size", "FLAG_GATE_PRECOMPUTED", "FLAG_NO_QK_L2NORM",
+__all__ = ["get_workspace_size_ex", "fwd", "fwd_recurrent", "decode", "segment_map", "state_affine", "bwd", "bwd_workspace_size",
+           "checkpoint_size", "fwd_checkpointed", "FLAG_GATE_PRECOMPUTED", "FLAG_NO_QK_L2NORM",
            "FLAG_BETA_PRECOMPUTED", "get_workspace_size", "fwd_launch_count", "new_workspace",
            "is_supported", "chunk_kda", "read_device_status", "selftest_wait_timeout", "KDAError",
            "library_path", "load"]
@@ -81,7 +82,12 @@ def load():
     lib.kda_bwd_workspace_size.argtypes = [i64, i32, i32]
     lib.kda_bwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_bwd.argtypes = [vp, vp, vp, vp, vp, f32, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                            ctypes.c_size_t, vp, i32, i64, i32, i32, i32, i32, vp]
+                            vp, ctypes.c_size_t, vp, i32, i64, i32, i32, i32, i32, vp]
+    lib.kda_checkpoint_size.argtypes = [i64, i32, i32]
+    lib.kda_checkpoint_size.restype = ctypes.c_size_t
+    lib.kda_fwd_checkpointed.argtypes = [vp, vp, vp, vp, vp, f32, vp, vp, ctypes.c_size_t, vp, vp, f32, vp, vp, vp,
+                                         ctypes.c_size_t, vp, i32, i64, i32, i32, i32, i32, vp]
+    lib.kda_fwd_checkpointed.restype = ctypes.c_int
     lib.kda_bwd.restype = ctypes.c_int
     lib.kda_workspace_size_ex.argtypes = [i64, i32, i32, i32, i32]
     lib.kda_workspace_size_ex.restype = ctypes.c_size_t
@@ -278,16 +284,49 @@ def bwd_workspace_size(T: int, H: int, N: int) -> int:
     return int(load().kda_bwd_workspace_size(int(T), int(H), int(N)))
 
 
+def checkpoint_size(T: int, H: int, N: int) -> int:
+    return int(load().kda_checkpoint_size(int(T), int(H), int(N)))
+
+
+def fwd_checkpointed(q, k, v, g, beta, scale, out, workspace, A_log, dt_bias, lower_bound, checkpoints,
+                     initial_state=None, final_state=None, cu_seqlens=None, stream=None):
+    """kda.fwd that also stores the state at the start of every 64-token chunk in ``checkpoints``
+    (fp32, at least checkpoint_size(T, H, N) bytes' worth) for kda.bwd (kda_fwd_checkpointed)."""
+    lib = load()
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (out, "out")):
+        _check(t, n, torch.bfloat16, dev)
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (initial_state, "initial_state"),
+                 (final_state, "final_state"), (checkpoints, "checkpoints")):
+        _check(t, n, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _check(workspace, "workspace", torch.uint8, dev)
+    B, T, H, K = q.shape
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = lib.kda_fwd_checkpointed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(out),
+                                      _ptr(workspace), workspace.numel(), _ptr(A_log), _ptr(dt_bias),
+                                      float(lower_bound), _ptr(initial_state), _ptr(final_state), _ptr(checkpoints),
+                                      checkpoints.numel() * 4, _ptr(cu_seqlens), B, T, H, K, v.shape[-1], N,
+                                      ctypes.c_void_p(stream))
+    if st != 0:
+        raise KDAError(st, "kda_fwd_checkpointed")
+
+
 def bwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out, initial_state=None, d_final=None,
-        cu_seqlens=None, workspace=None, stream=None):
-    """Gradients of sum(d_out * o) + sum(d_final * final_state) w.r.t. every input (kda_bwd).
-    Returns a dict: dq, dk, dv, dg (bf16, shaped like the inputs), dbeta (bf16, like beta),
-    dA_log [H], ddt_bias [H, K] and d_initial [N, H, K, V] (fp32)."""
+        cu_seqlens=None, workspace=None, stream=None, checkpoints=None):
+    """Gradients of sum(d_out * o) + sum(d_final * final_state) w.r.t. every input (kda_bwd), using
+    ``checkpoints`` from fwd_checkpointed when given.  Returns a dict: dq, dk, dv, dg (bf16, shaped
+    like the inputs), dbeta (bf16, like beta), dA_log [H], ddt_bias [H, K] and d_initial
+    [N, H, K, V] (fp32)."""
     lib = load()
     dev = q.device
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (d_out, "d_out")):
         _check(t, n, torch.bfloat16, dev)
-    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (initial_state, "initial_state"), (d_final, "d_final")):
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (initial_state, "initial_state"), (d_final, "d_final"),
+                 (checkpoints, "checkpoints")):
         _check(t, n, torch.float32, dev)
     _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
     B, T, H, K = q.shape
@@ -303,7 +342,8 @@ def bwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out, initial_sta
         stream = torch.cuda.current_stream(dev).cuda_stream
     with torch.cuda.device(dev):
         st = lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(A_log), _ptr(dt_bias),
-                         float(lower_bound), _ptr(initial_state), _ptr(d_out), _ptr(d_final), _ptr(r["dq"]),
+                         float(lower_bound), _ptr(initial_state), _ptr(d_out), _ptr(d_final), _ptr(checkpoints),
+                         _ptr(r["dq"]),
                          _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dg"]), _ptr(r["dbeta"]), _ptr(r["dA_log"]),
                          _ptr(r["ddt_bias"]), _ptr(r["d_initial"]), _ptr(workspace), workspace.numel(),
                          _ptr(cu_seqlens), B, T, H, K, V, N, ctypes.c_void_p(stream))

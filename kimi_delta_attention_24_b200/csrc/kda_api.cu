@@ -305,16 +305,17 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const void*
   if ((flags & ~kda::kFlagMask) != 0) return KDA_ERR_INVALID_ARGUMENT;
   const bool gate_in_kernel = !(flags & kda::kFlagGatePrecomputed);
   if (gate_in_kernel && !(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_INVALID_ARGUMENT;
-  if (gate_in_kernel && (!A_log || !dt_bias)) return KDA_ERR_INVALID_ARGUMENT;
   if (batch < 0 || seqlen < 0 || num_heads <= 0 || num_slots < 0) return KDA_ERR_INVALID_ARGUMENT;
+  // with no token nothing of the token tensors is read: they may be null (empty tensors)
+  if (seqlen > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARGUMENT;
+  if (seqlen > 0 && gate_in_kernel && (!A_log || !dt_bias)) return KDA_ERR_INVALID_ARGUMENT;
   if (state_transposed != 0 && state_transposed != 1) return KDA_ERR_INVALID_ARGUMENT;
   if (!isfinite(scale)) return KDA_ERR_INVALID_ARGUMENT;
   const void* vec[] = {q, k, v, g, out};
   for (const void* p : vec)
     if (!aligned(p, 16)) return KDA_ERR_INVALID_ARGUMENT;
   if (!aligned(beta, (flags & kda::kFlagBetaPrecomputed) ? 4 : 2)) return KDA_ERR_INVALID_ARGUMENT;
-  if (gate_in_kernel && (!aligned(A_log, 4) || !aligned(dt_bias, 16))) return KDA_ERR_INVALID_ARGUMENT;
+  if (gate_in_kernel && seqlen > 0 && (!aligned(A_log, 4) || !aligned(dt_bias, 16))) return KDA_ERR_INVALID_ARGUMENT;
   if ((state_in && !aligned(state_in, 16)) || (state_out && !aligned(state_out, 16)))
     return KDA_ERR_INVALID_ARGUMENT;
   if (state_indices && !aligned(state_indices, 4)) return KDA_ERR_INVALID_ARGUMENT;
@@ -333,9 +334,40 @@ size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t n
   return kda::bwd_workspace_bytes(total_tokens, num_heads, num_seqs);
 }
 
+size_t kda_checkpoint_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  return kda::checkpoint_bytes(total_tokens, num_heads, num_seqs);
+}
+
+kda_status_t kda_fwd_checkpointed(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                  float scale, void* out, void* workspace, size_t workspace_bytes,
+                                  const float* A_log, const float* dt_bias, float lower_bound,
+                                  const float* initial_state, float* final_state, float* checkpoints,
+                                  size_t checkpoint_bytes, const int32_t* cu_seqlens, int32_t batch, int64_t seqlen,
+                                  int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
+                                  kda_stream_t stream) {
+  Shape shape;
+  kda_status_t st = validate(q, k, v, g, beta, out, A_log, dt_bias, lower_bound, initial_state, final_state,
+                             cu_seqlens, batch, seqlen, num_heads, head_dim_k, head_dim_v, num_seqs, 0, scale,
+                             &shape);
+  if (st != KDA_OK) return st;
+  if (!workspace || !aligned(workspace, 256) || !checkpoints || !aligned(checkpoints, 16))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < kda_workspace_size(shape.total_tokens, num_heads, shape.num_seqs) ||
+      checkpoint_bytes < kda_checkpoint_size(shape.total_tokens, num_heads, shape.num_seqs))
+    return KDA_ERR_WORKSPACE_TOO_SMALL;
+  kda::FwdParams p = make_params(q, k, v, g, beta, scale, out, A_log, dt_bias, lower_bound,
+                                 initial_state, final_state, cu_seqlens, seqlen, num_heads,
+                                 shape.num_seqs, 0, static_cast<uint32_t*>(workspace));
+  if ((int64_t)shape.num_seqs * num_heads == 0) return KDA_OK;
+  return kda::launch_split(p, workspace, reinterpret_cast<cudaStream_t>(stream), checkpoints) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
 kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
                      const float* A_log, const float* dt_bias, float lower_bound, const float* initial_state,
-                     const void* d_out, const float* d_final, void* dq, void* dk, void* dv, void* dg, void* dbeta,
+                     const void* d_out, const float* d_final, const float* checkpoints, void* dq, void* dk,
+                     void* dv, void* dg, void* dbeta,
                      float* dA_log, float* ddt_bias, float* d_initial, void* workspace, size_t workspace_bytes,
                      const int32_t* cu_seqlens, int32_t batch, int64_t seqlen, int32_t num_heads,
                      int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs, kda_stream_t stream) {
@@ -348,7 +380,8 @@ kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g,
   const void* vec[] = {dq, dk, dv, dg, ddt_bias};
   for (const void* p : vec)
     if (!aligned(p, 16)) return KDA_ERR_INVALID_ARGUMENT;
-  if (!aligned(dbeta, 2) || !aligned(dA_log, 4) || (d_initial && !aligned(d_initial, 16)))
+  if (!aligned(dbeta, 2) || !aligned(dA_log, 4) || (d_initial && !aligned(d_initial, 16)) ||
+      (checkpoints && !aligned(checkpoints, 16)))
     return KDA_ERR_INVALID_ARGUMENT;
   if (!workspace || !aligned(workspace, 256)) return KDA_ERR_INVALID_ARGUMENT;
   if (workspace_bytes < kda_bwd_workspace_size(shape.total_tokens, num_heads, shape.num_seqs))
@@ -358,7 +391,7 @@ kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g,
   return kda::launch_bwd(p, static_cast<const __nv_bfloat16*>(d_out), d_final, static_cast<__nv_bfloat16*>(dq),
                          static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv),
                          static_cast<__nv_bfloat16*>(dg), static_cast<__nv_bfloat16*>(dbeta), dA_log, ddt_bias,
-                         d_initial, workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                         d_initial, checkpoints, workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? KDA_OK
              : KDA_ERR_CUDA;
 }

@@ -31,7 +31,8 @@ namespace kda {
 namespace {
 
 constexpr int kBwdThreads = 256;
-constexpr int kBwdChunk = 32;  // tokens per checkpoint (and per staged chunk)
+constexpr int kBwdChunk = 64;  // tokens per checkpoint: the forward's chunk, whose start states it can store
+constexpr int kStage = 32;     // tokens whose transformed inputs are staged in shared memory at once
 constexpr int kSlice = 32;  // state columns per CTA (4 per warp)
 constexpr int kSlices = kHeadDim / kSlice;
 constexpr size_t kStateElems = (size_t)kHeadDim * kHeadDim;
@@ -49,7 +50,8 @@ struct BwdParams {
   float* dA_log;                // [H], zeroed before the launch
   float* ddt_bias;              // [H, K], zeroed before the launch
   float* d_initial;             // [N, H, K, V] or null
-  float* ckpt;                  // (T / 64 + N + 1) x H states: chunk-start checkpoints (by slice)
+  const float* ckpt_in;         // the forward's checkpoints, or null (then computed into ckpt)
+  float* ckpt;                  // (T / 64 + N + 1) x H states: chunk-start checkpoints, S^T[v][k]
   float* scratch;               // gridDim.x x 64 slices: the states before each token of a chunk
   float* part;                  // per slice: dqhat, dkhat, dalpha [tokens, H, K]; then dbeta [slice][tokens, H]
 };
@@ -83,16 +85,16 @@ __device__ __forceinline__ float warp_allsum(float x) {
   return x;
 }
 
-// A chunk's transformed inputs, staged in shared memory once per chunk (each warp transforms every
-// eighth token) and read by all warps: khat, qhat and alpha per channel, v and d_out on the slice's
-// columns, beta.
+// Up to kStage tokens' transformed inputs, staged in shared memory (each warp transforms every eighth
+// token) and read by all warps: khat, qhat and alpha per channel, v and d_out on the slice's columns,
+// beta.
 struct ChunkIn {
-  float k[kBwdChunk][kHeadDim];
-  float q[kBwdChunk][kHeadDim];
-  float a[kBwdChunk][kHeadDim];
-  float v[kBwdChunk][kSlice];
-  float d[kBwdChunk][kSlice];
-  float b[kBwdChunk];
+  float k[kStage][kHeadDim];
+  float q[kStage][kHeadDim];
+  float a[kStage][kHeadDim];
+  float v[kStage][kSlice];
+  float d[kStage][kSlice];
+  float b[kStage];
 };
 
 __device__ __forceinline__ void stage_chunk(const BwdParams& P, ChunkIn& s, int64_t t_begin, int len, int h,
@@ -164,11 +166,6 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
     const int64_t ck0 = bos / kBwdChunk + n;  // this sequence's first checkpoint slot
     const float ea = expf(p.A_log[h]);
     const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-    // a slice state stored per thread: 16 contiguous floats at thread index tid
-    auto ck_ptr = [&](int c) { return P.ckpt + (((size_t)(ck0 + c) * H + h) * kSlices + sl) * kSliceElems; };
-    float* const part_q = P.part + (size_t)sl * 3 * rows_total * D;
-    float* const part_b = P.part + (size_t)kSlices * 3 * rows_total * D + (size_t)sl * rows_total;
-
     float S[4][4];  // S[4 lane + i][col0 + j]
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -176,6 +173,24 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
       if (p.initial_state) t = *reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)(4 * lane + i) * D + col0);
       S[i][0] = t.x; S[i][1] = t.y; S[i][2] = t.z; S[i][3] = t.w;
     }
+    // checkpoint of chunk c: the whole state, transposed (S^T[v][k]), as the forward stores it
+    const float* ck_base = P.ckpt_in ? P.ckpt_in : P.ckpt;
+    auto ck_ptr = [&](int c) { return ck_base + ((size_t)(ck0 + c) * H + h) * kStateElems; };
+    auto load_ckpt = [&](const float* base) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 t = *reinterpret_cast<const float4*>(base + (size_t)(col0 + j) * D + 4 * lane);
+        S[0][j] = t.x; S[1][j] = t.y; S[2][j] = t.z; S[3][j] = t.w;
+      }
+    };
+    auto store_ckpt = [&](float* base) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4*>(base + (size_t)(col0 + j) * D + 4 * lane) = make_float4(S[0][j], S[1][j], S[2][j], S[3][j]);
+    };
+    float* const part_q = P.part + (size_t)sl * 3 * rows_total * D;
+    float* const part_b = P.part + (size_t)kSlices * 3 * rows_total * D + (size_t)sl * rows_total;
+
     auto store_state = [&](float* base) {
       float4* dst = reinterpret_cast<float4*>(base + (size_t)tid * 16);
 #pragma unroll
@@ -218,14 +233,20 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
     };
 
     // ---------------------------------------------------------------- forward with checkpoints
-    for (int c = 0; c < nch; ++c) {
-      const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
-      const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
-      store_state(ck_ptr(c));
-      __syncthreads();  // the previous chunk's staged inputs are read
-      stage_chunk(P, s, t_begin, len, h, scol0, ea, dt, false);
-      __syncthreads();
-      for (int i = 0; i < len; ++i) forward_token(i);
+    // (only without the forward's checkpoints; each CTA writes its own 32 columns of them)
+    if (!P.ckpt_in) {
+      for (int c = 0; c < nch; ++c) {
+        const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
+        const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
+        store_ckpt(P.ckpt + ((size_t)(ck0 + c) * H + h) * kStateElems);
+        for (int h0 = 0; h0 < len; h0 += kStage) {
+          const int hl = min(kStage, len - h0);
+          __syncthreads();  // the previously staged inputs are read
+          stage_chunk(P, s, t_begin + h0, hl, h, scol0, ea, dt, false);
+          __syncthreads();
+          for (int i = 0; i < hl; ++i) forward_token(i);
+        }
+      }
     }
 
     // ---------------------------------------------------------------- backward, chunk by chunk
@@ -237,29 +258,16 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
       dS[i][0] = t.x; dS[i][1] = t.y; dS[i][2] = t.z; dS[i][3] = t.w;
     }
     int buf = 0;
-    for (int c = nch - 1; c >= 0; --c) {
-      const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
-      const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
-      __syncthreads();  // the previous chunk's staged inputs and partials are read
-      stage_chunk(P, s, t_begin, len, h, scol0, ea, dt, true);
-      __syncthreads();
-      // rerun the chunk's forward from its checkpoint, keeping the state before each token
-      load_state(ck_ptr(c));
-      for (int i = 0; i < len; ++i) {
-        store_state(scr + (size_t)i * kSliceElems);
-        forward_token(i);
-      }
-      // the chunk's tokens backwards; S holds S_{t-1} of the token at hand (from the scratch)
-      load_state(scr + (size_t)(len - 1) * kSliceElems);
-      for (int i = len - 1; i >= 0; --i) {
+    // one backward token: chunk token i (staged at si); S holds its S_{t-1}
+    auto backward_token = [&](int64_t t_begin, int i, int si) {
         const size_t row = (size_t)(t_begin + i) * H + h;
-        const float4 a4 = row4(s.a, i), k4 = row4(s.k, i), q4 = row4(s.q, i);
+        const float4 a4 = row4(s.a, si), k4 = row4(s.k, si), q4 = row4(s.q, si);
         const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
         const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-        const float4 v4 = reinterpret_cast<const float4*>(s.v[i])[warp];
-        const float4 d4 = reinterpret_cast<const float4*>(s.d[i])[warp];
+        const float4 v4 = reinterpret_cast<const float4*>(s.v[si])[warp];
+        const float4 d4 = reinterpret_cast<const float4*>(s.d[si])[warp];
         const float vv[4] = {v4.x, v4.y, v4.z, v4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        const float b = s.b[i], scale = p.scale;
+        const float b = s.b[si], scale = p.scale;
         // p = Stil^T khat (columns), delta
         float pj[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -329,7 +337,39 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
           part_b[row] = acc;
         }
         buf ^= 1;  // the next token writes the other buffer; this one is read until the next barrier
+    };
+    for (int c = nch - 1; c >= 0; --c) {
+      const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
+      const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
+      const int len0 = min(kStage, len);  // tokens of the first staged half
+      // rerun the chunk's forward from its checkpoint, keeping the state before each token; the
+      // second half is staged with what the backward needs and walked backwards right away
+      load_ckpt(ck_ptr(c));
+      __syncthreads();  // the previously staged inputs and partials are read
+      stage_chunk(P, s, t_begin, len0, h, scol0, ea, dt, false);
+      __syncthreads();
+      for (int i = 0; i < len0; ++i) {
+        store_state(scr + (size_t)i * kSliceElems);
+        forward_token(i);
       }
+      if (len > kStage) {
+        __syncthreads();
+        stage_chunk(P, s, t_begin + kStage, len - kStage, h, scol0, ea, dt, true);
+        __syncthreads();
+        for (int i = kStage; i < len; ++i) {
+          store_state(scr + (size_t)i * kSliceElems);
+          forward_token(i - kStage);
+        }
+        load_state(scr + (size_t)(len - 1) * kSliceElems);
+        for (int i = len - 1; i >= kStage; --i) backward_token(t_begin, i, i - kStage);
+      } else {
+        load_state(scr + (size_t)(len - 1) * kSliceElems);
+      }
+      // the first half backwards (S holds the state before its last token)
+      __syncthreads();
+      stage_chunk(P, s, t_begin, len0, h, scol0, ea, dt, true);
+      __syncthreads();
+      for (int i = len0 - 1; i >= 0; --i) backward_token(t_begin, i, i);
     }
     if (P.d_initial) {
 #pragma unroll
@@ -456,7 +496,8 @@ size_t bwd_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_
 
 cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const float* d_final, __nv_bfloat16* dq,
                        __nv_bfloat16* dk, __nv_bfloat16* dv, __nv_bfloat16* dg, __nv_bfloat16* dbeta, float* dA_log,
-                       float* ddt_bias, float* d_initial, void* workspace, cudaStream_t stream) {
+                       float* ddt_bias, float* d_initial, const float* checkpoints, void* workspace,
+                       cudaStream_t stream) {
   const int64_t units = (int64_t)f.num_seqs * f.num_heads;
   int dev = 0, sms = 0;
   cudaError_t qe = cudaGetDevice(&dev);
@@ -482,6 +523,7 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
   P.dA_log = dA_log;
   P.ddt_bias = ddt_bias;
   P.d_initial = d_initial;
+  P.ckpt_in = checkpoints;
   P.ckpt = static_cast<float*>(workspace);
   P.scratch = P.ckpt + (size_t)slots * f.num_heads * kStateElems;
   const int64_t work_cap = work < kBwdMaxCtas ? work : kBwdMaxCtas;

@@ -85,7 +85,9 @@ cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 // The fused single-kernel chunked path (one CTA per (sequence, head); needs only the status word).
 cudaError_t launch_chunked(const FwdParams& p, cudaStream_t stream);
 // The split chunked path: chunk table, chunk-parallel intra-chunk kernel, recurrence kernel.
-cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream);
+// ckpt (optional): also store the state at the start of every 64-token chunk (S^T, fp32) there.
+cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream, float* ckpt = nullptr);
+size_t checkpoint_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 // The segment map (M, B) of every unit: the split path with the recurrence in map mode.
@@ -106,7 +108,8 @@ cudaError_t launch_unpad_state(const float* src, float* dst, int64_t units, int 
 size_t bwd_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const float* d_final, __nv_bfloat16* dq,
                        __nv_bfloat16* dk, __nv_bfloat16* dv, __nv_bfloat16* dg, __nv_bfloat16* dbeta, float* dA_log,
-                       float* ddt_bias, float* d_initial, void* workspace, cudaStream_t stream);
+                       float* ddt_bias, float* d_initial, const float* checkpoints, void* workspace,
+                       cudaStream_t stream);
 // The batched recurrent decode step (kda_decode).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
                           void* out, const float* A_log, const float* dt_bias, float lower_bound,

@@ -67,6 +67,7 @@ struct SplitArgs {
   int map_mode;
   float* map_M;                  // [N, H, 128, 128]
   float* map_B;                  // [N, H, 128, 128]
+  float* ckpt;                   // checkpoint mode: [T / 64 + N + 1 slots][H][128 v][128 k] chunk-start states
 };
 
 constexpr int kQueues = 2;  // item counters in the workspace header, one per intra launch
@@ -944,8 +945,11 @@ struct RecMaps {
   CUtensorMap v, out;
 };
 
-// kMap: map mode (see SplitArgs), compiled separately so that the forward's code is unchanged.
-template <bool kMap>
+// kMode: kModeFwd, the forward; kModeMap, map mode (see SplitArgs); kModeCkpt, the forward that also
+// stores each chunk's starting state (S^T, fp32) in args.ckpt for the backward.  Compiled
+// separately, so that the forward's code is unchanged.
+constexpr int kModeFwd = 0, kModeMap = 1, kModeCkpt = 2;
+template <int kMode>
 __global__ void __launch_bounds__(kRecThreads, 1)
     rec_kernel(const __grid_constant__ RecMaps maps, const SplitArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -953,11 +957,13 @@ __global__ void __launch_bounds__(kRecThreads, 1)
   const FwdParams& p = args.p;
   const int H = p.num_heads;
   const int units = p.num_seqs * H;
+  constexpr bool kMap = kMode == kModeMap;
   const bool map_part_M = kMap && (int)blockIdx.x >= units;  // map mode: this CTA computes M
   const int ub = kMap ? (int)blockIdx.x % units : (int)blockIdx.x;
   const int n = ub / H, h = ub % H;
   int64_t bos, eos;
   seq_range(p, n, bos, eos);
+  const int64_t ck_slot0 = bos / C + n;  // checkpoint mode: the sequence's first checkpoint slot
   // launched as a programmatic dependent: let the next launch place its CTAs beside this grid's,
   // then wait until the items this launch reads are complete
   // This launch walks the sequence's chunks that fall in global chunks [g0, g1); a sequence cut at
@@ -1230,6 +1236,13 @@ __global__ void __launch_bounds__(kRecThreads, 1)
       tmem_wait_st();
     };
 
+    // checkpoint mode: S^T at the start of this sequence's chunk c (slot per (chunk, head), [v][k])
+    auto store_ckpt = [&](const float (&x)[32], int c) {
+      float4* dst = reinterpret_cast<float4*>(args.ckpt + ((size_t)(ck_slot0 + c) * H + h) * (size_t)D * D +
+                                              (size_t)v * D + col0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+    };
     if (nch == 0) {
       float x[32];
       load_state(x);
@@ -1240,6 +1253,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
       {
         float x[32];
         load_state(x);
+        if constexpr (kMode == kModeCkpt) store_ckpt(x, c_begin);
         store_state_bf16(x);
         store_state_scaled(x, sc_gam);
       }
@@ -1330,6 +1344,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar + RB_S);
+        if constexpr (kMode == kModeCkpt) store_ckpt(x, c_begin + c + 1);
         // off the critical path (MMA1 of the next chunk runs meanwhile): the rescaled fp32 state,
         // then the one barrier of all epilogue warps per chunk, which also decides (for all of them)
         // whether to stop; it keeps ep1 of the next chunk after every warp's reads of this stage
@@ -1351,7 +1366,7 @@ __global__ void __launch_bounds__(kRecThreads, 1)
 }
 
 bool g_intra_attr[2][64] = {};
-bool g_rec_attr[2][64] = {};
+bool g_rec_attr[3][64] = {};
 
 }  // namespace
 
@@ -1380,6 +1395,12 @@ int64_t stage_cut(int64_t max_chunks, int64_t units, int heads, int sms) {
 
 }  // namespace
 
+size_t checkpoint_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  const int64_t t = total_tokens > 0 ? total_tokens : 0, n = num_seqs > 0 ? num_seqs : 0;
+  const int64_t hh = num_heads > 0 ? num_heads : 0;
+  return (size_t)(t / C + n + 1) * (size_t)hh * D * D * sizeof(float);
+}
+
 size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
   const int64_t n = num_seqs > 0 ? num_seqs : 0;
   const int64_t t = total_tokens > 0 ? total_tokens : 0;
@@ -1389,7 +1410,7 @@ size_t split_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t nu
          (size_t)hh * D * D * sizeof(float);
 }
 
-cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream) {
+cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t stream, float* ckpt) {
   const int64_t units = (int64_t)p.num_seqs * p.num_heads;
   if (units == 0) return cudaSuccess;
   const int64_t tokens = p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs;
@@ -1413,7 +1434,8 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
   auto intra_fn = gate_pre ? intra_kernel<true> : intra_kernel<false>;
   cudaError_t e = set_smem_once(intra_fn, I_ALLOC, g_intra_attr[gate_pre ? 1 : 0]);
   if (e != cudaSuccess) return e;
-  e = set_smem_once(rec_kernel<false>, R_ALLOC, g_rec_attr[0]);
+  auto rec_fn = ckpt ? rec_kernel<kModeCkpt> : rec_kernel<kModeFwd>;
+  e = set_smem_once(rec_fn, R_ALLOC, g_rec_attr[ckpt ? 2 : 0]);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
@@ -1449,7 +1471,8 @@ cudaError_t launch_split(const FwdParams& p, void* workspace, cudaStream_t strea
     SplitArgs a = args;
     a.g0 = g0;
     a.g1 = g1;
-    return launch(rec_kernel<false>, units, kRecThreads, R_ALLOC, true, rm, a);
+    a.ckpt = ckpt;
+    return launch(rec_fn, units, kRecThreads, R_ALLOC, true, rm, a);
   };
 
   chunk_table_kernel<<<1, 1024, 0, stream>>>(p, const_cast<int32_t*>(args.chunk_off), queues);
@@ -1494,7 +1517,7 @@ cudaError_t launch_segment_map(const FwdParams& p, void* workspace, float* map_M
   auto intra_fn = gate_pre ? intra_kernel<true> : intra_kernel<false>;
   cudaError_t e = set_smem_once(intra_fn, I_ALLOC, g_intra_attr[gate_pre ? 1 : 0]);
   if (e != cudaSuccess) return e;
-  e = set_smem_once(rec_kernel<true>, R_ALLOC, g_rec_attr[1]);
+  e = set_smem_once(rec_kernel<kModeMap>, R_ALLOC, g_rec_attr[1]);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
@@ -1526,7 +1549,7 @@ cudaError_t launch_segment_map(const FwdParams& p, void* workspace, float* map_M
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, rec_kernel<true>, rm, a);
+  return cudaLaunchKernelEx(&cfg, rec_kernel<kModeMap>, rm, a);
 }
 
 int split_launch_count(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {

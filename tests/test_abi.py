@@ -152,6 +152,8 @@ def test_decode_host_validation(lib):
     # a precomputed gate needs neither A_log nor dt_bias, and lower_bound is not checked
     assert call_decode(lib, A_log=None, dt_bias=None, lb=-9.0, flags=1, batch=0) == 0
     assert call_decode(lib, batch=0) == 0     # no request: nothing launched
+    assert call_decode(lib, q=None, batch=0, seqlen=0) == 0  # no token: token tensors may be null
+    assert call_decode(lib, q=None, seqlen=1) == 1
 
 
 def test_fwd_ex_flags_validation(lib):

@@ -23,7 +23,7 @@ def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
 
 
-def run_case(dev, x, seed, with_final=True):
+def run_case(dev, x, seed, with_final=True, use_checkpoints=False):
     rng = np.random.default_rng(seed)
     d_out = torch.from_numpy(rng.standard_normal(x.v.shape)).to(torch.bfloat16)
     N, H = x.num_seqs, x.num_heads
@@ -31,9 +31,19 @@ def run_case(dev, x, seed, with_final=True):
     ref = oracle.kda_bwd(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, d_out,
                          initial_state=x.initial_state, d_final=d_final, cu_seqlens=x.cu_seqlens)
     xd = x.to(dev)
+    ck = None
+    if use_checkpoints:
+        # the training forward: output, final state and the chunk-start states for the backward
+        B, T = x.q.shape[:2]
+        ck = torch.empty(kda.checkpoint_size(B * T, H, N) // 4, dtype=torch.float32, device=dev)
+        out = torch.empty_like(xd.v)
+        ws = kda.new_workspace(B * T, H, N, dev)
+        kda.fwd_checkpointed(xd.q, xd.k, xd.v, xd.g, xd.beta, x.scale, out, ws, xd.A_log, xd.dt_bias, x.lower_bound,
+                             ck, initial_state=xd.initial_state, cu_seqlens=xd.cu_seqlens)
+        assert kda.read_device_status(ws) == 0
     got = kda.bwd(xd.q, xd.k, xd.v, xd.g, xd.beta, x.scale, xd.A_log, xd.dt_bias, x.lower_bound, d_out.to(dev),
                   initial_state=xd.initial_state, d_final=None if d_final is None else d_final.to(dev),
-                  cu_seqlens=xd.cu_seqlens)
+                  cu_seqlens=xd.cu_seqlens, checkpoints=ck)
     torch.cuda.synchronize()
     return got, ref
 
@@ -71,3 +81,38 @@ def test_bwd_many_units_more_than_sms(cuda_device):
     """200 (sequence, head) units: the persistent CTAs take several units each."""
     x = kda_inputs.make_random("t", [40, 70, 3, 100], 50, seed=114, state_std=0.1)
     check_grads(*run_case(cuda_device, x, 4), "200 units")
+
+
+@pytest.mark.parametrize("lens,H", [([130, 0, 64, 1, 200], 3), ([2000], 4), ([700, 9000], 12)])
+def test_bwd_with_forward_checkpoints(cuda_device, lens, H):
+    """The training path: kda_fwd_checkpointed stores the chunk-start states (the second shape runs
+    the forward in two stages, the third cuts a sequence between them) and kda_bwd starts from them."""
+    x = kda_inputs.make_random("t", lens, H, seed=115, state_std=0.2)
+    x.g[:, :, :, :64].fill_(-6.0)  # half the channels decay slowly: states carry across chunks
+    check_grads(*run_case(cuda_device, x, 5, use_checkpoints=True), f"checkpoints {lens} H={H}")
+
+
+def test_forward_checkpoints_are_chunk_start_states(cuda_device):
+    """The stored checkpoints equal the oracle's state after 64 c tokens (S^T layout)."""
+    lens, H = [300, 130], 2
+    x = kda_inputs.make_random("t", lens, H, seed=116, state_std=0.2)
+    x.g.fill_(-6.0)
+    xd = x.to(cuda_device)
+    ck = torch.full((kda.checkpoint_size(430, H, 2) // 4,), float("nan"), device=cuda_device)
+    out = torch.empty_like(xd.v)
+    ws = kda.new_workspace(430, H, 2, cuda_device)
+    kda.fwd_checkpointed(xd.q, xd.k, xd.v, xd.g, xd.beta, x.scale, out, ws, xd.A_log, xd.dt_bias, x.lower_bound, ck,
+                         initial_state=xd.initial_state, cu_seqlens=xd.cu_seqlens)
+    ck = ck.cpu().double().numpy().reshape(-1, H, 128, 128)
+    cu = x.cu_seqlens.tolist()
+    for n in range(2):
+        for c in range((lens[n] + 63) // 64):
+            t_end = cu[n] + 64 * c
+            sub = lambda t: t[:, cu[n]:t_end].contiguous()
+            _, s_ref = oracle.kda_fwd(sub(x.q), sub(x.k), sub(x.v), sub(x.g), sub(x.beta), x.scale, x.A_log,
+                                      x.dt_bias, x.lower_bound, initial_state=x.initial_state[n:n + 1],
+                                      cu_seqlens=torch.tensor([0, t_end - cu[n]], dtype=torch.int32))
+            slot = cu[n] // 64 + n + c
+            got = np.swapaxes(ck[slot], -1, -2)
+            err = rel_l2(got, s_ref[0])
+            assert np.isfinite(got).all() and err <= 1e-2, (n, c, err)

@@ -209,9 +209,9 @@ def test_decode_zero_tokens_copies_states(cuda_device):
     pool = torch.randn(7, H, 128, 128, generator=gen).to(cuda_device)
     idx = torch.tensor([6, 0, -1, 3, 2], dtype=torch.int32, device=cuda_device)
     dev = cuda_device
-    # zero-token views of real allocations, so that every pointer is valid and 16-byte aligned
-    q, k, v, g, out = (torch.zeros(B, 1, H, 128, dtype=torch.bfloat16, device=dev)[:, :0] for _ in range(5))
-    beta = torch.zeros(B, 1, H, dtype=torch.bfloat16, device=dev)[:, :0]
+    # empty token tensors (their data pointers are null: nothing of them is read)
+    q, k, v, g, out = (torch.zeros(B, 0, H, 128, dtype=torch.bfloat16, device=dev) for _ in range(5))
+    beta = torch.zeros(B, 0, H, dtype=torch.bfloat16, device=dev)
     p_out = torch.full_like(pool, float("nan"))
     kda.decode(q, k, v, g, beta, 0.088, out, torch.zeros(H, device=dev), torch.zeros(H, 128, device=dev), -5.0,
                pool, p_out, idx)
