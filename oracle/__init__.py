@@ -6,7 +6,8 @@ plain C token recurrence (``kda_oracle.c``), its ctypes wrapper, and two numpy c
 pin it (``brute`` — explicit products — and ``chunked`` — the chunked WY/UT form).
 
 Parity status: every function here is pinned by the ``-m "not gpu"`` tests against closed forms,
-invariants and brute force (see ``tests/test_oracle_pins.py``).  Agreement with upstream FlashKDA
+invariants and brute force (see ``tests/test_oracle_pins.py``); the backward (``kda_bwd``) against
+central finite differences of ``kda_fwd_f64`` and a closed form (``tests/test_oracle_bwd_pins.py``).  Agreement with upstream FlashKDA
 or fla outputs is unpinned: neither their code nor any of their outputs is available, so the
 state layout, the L2-norm epsilon and the gate form are readings (they are listed in the
 design notes).
