@@ -202,13 +202,27 @@ BWD_TOKENS = 4096
 BWD_BYTES_PER_TOKEN_HEAD = BYTES_PER_TOKEN_HEAD + 2 * D + (4 * 2 * D + 2)  # + d_out in; dq, dk, dv, dg, dbeta out
 
 
-def bench_backward(dev, steps, warmup, seed=0):
-    """The backward pass (token-serial on CUDA cores, checkpointed) on the prefill's heads with
-    T = 4096 tokens: milliseconds per step, token-heads/s, and HBM GB/s of its algorithmic bytes
-    (inputs and d_out read once, the five token gradients written once)."""
+# Chunked-form FLOPs of the backward per token-head (64-token chunks, K = V = 128; a multiply-add is 2
+# FLOPs): per (chunk, head), the chunk factors in both chunk-parallel kernels (the Gram and P blocks of
+# the four 16-row sub-blocks, the solve), the prep products (W, Qt - P W, P^T dO, (Qt - P W)^T dO), the
+# reverse state walk (Kt dS', W^T E) and the gradient products (W, U, dP, dT_b twice, dv, dKg; Delta,
+# dKt, dQs, dW; T^T dT, dA; the four decay-weighted products).
+_CB = 64
+_BWD_MACS_PER_CHUNK = (2 * (2 * 16 * 160 * D + _CB ** 3 // 6) + 3 * _CB * _CB * D + _CB * D * D
+                       + 2 * _CB * D * D
+                       + 7 * _CB * _CB * D + 4 * _CB * D * D + 2 * _CB ** 3 + 4 * 16 * 160 * D)
+BWD_FLOPS_PER_TOKEN_HEAD = 2 * _BWD_MACS_PER_CHUNK / _CB
+
+
+def bench_backward(dev, steps, warmup, seed=0, heads=HEADS):
+    """The backward pass (chunked, fp32 CUDA cores, from the checkpointing forward's states) on the
+    prefill's heads with T = 4096 tokens: milliseconds per step, token-heads/s, HBM GB/s of its
+    algorithmic bytes (inputs and d_out read once, the five token gradients written once) and
+    TFLOP/s of its chunked-form FLOPs."""
     import kda_inputs
     import kimi_delta_attention_24_b200 as kda
 
+    HEADS = heads  # noqa: N806 (the workload's head count)
     x = kda_inputs.make_random("bwd", [BWD_TOKENS], HEADS, seed=seed, device=dev)
     gen = torch.Generator(device=dev).manual_seed(seed + 11)
     d_out = torch.randn(x.v.shape, generator=gen, device=dev).to(torch.bfloat16)
@@ -257,8 +271,9 @@ def bench_backward(dev, steps, warmup, seed=0):
             "checkpointing_forward_ms": ms_fwd_ck,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
                          "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
-                         "note": "token-serial CUDA-core kernel: bound by its per-token dependency chain, "
-                                 "not by HBM"},
+                         "note": "chunked form on fp32 CUDA cores: latency-bound per chunk (about a fifth of "
+                                 "the fp32 FMA rate), not bound by HBM"},
+            "chunked_tflops": BWD_FLOPS_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e12,
             "gpu_launches": steps}
 
 
@@ -365,6 +380,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--no-kcp", action="store_true", help="skip the sequence-parallel rank-work measurement")
+    ap.add_argument("--bwd-heads", type=int, default=HEADS,
+                    help="heads of the backward workload (default 96; fewer only for small profiling runs)")
     ap.add_argument("--heads", type=int, default=HEADS,
                     help="heads of the prefill workload (default 96; fewer only for small profiling runs)")
     args = ap.parse_args()
@@ -518,7 +535,7 @@ def main():
     if not args.no_decode:
         line["decode"] = bench_decode(dev, steps=max(args.steps, 10), warmup=args.warmup, seed=rank)
     if not args.no_backward:
-        line["backward"] = bench_backward(dev, steps=2, warmup=1, seed=rank)
+        line["backward"] = bench_backward(dev, steps=2, warmup=1, seed=rank, heads=args.bwd_heads)
     if not args.no_kcp:
         line["kcp_rank_work"] = bench_kcp_rank(dev, steps=5, warmup=2, seed=rank)
     if world > 1:

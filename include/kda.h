@@ -261,10 +261,12 @@ kda_status_t kda_fwd_checkpointed(const void* q, const void* k, const void* v, c
                                   int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, int32_t num_seqs,
                                   kda_stream_t stream);
 
-/* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): room for the
- * checkpoints (as kda_checkpoint_size; used when the call is given none), a scratch of 64 states of
- * 128 x 32 for each of up to min(4 N H, 512) CTAs, and four slices of per-channel partial sums
- * (3 x 128 + 1 fp32 per token and head).  Depends only on its arguments. */
+/* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): the forward's
+ * workspace and the checkpoints and output it writes (used when the call is given no checkpoints),
+ * per (64-token chunk, head) the factors of the reverse state walk (160 KB) and dDelta (32 KB), one
+ * 128 x 128 state gradient per chunk slot and head, per-token partials (3 x 128 + 1 fp32 per token
+ * and head), and a scratch of 624 KB per CTA of the chunk-parallel kernels (at most 296).  Depends
+ * only on its arguments; its first 256 bytes hold the status word read by kda_read_device_status. */
 size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
 /* The backward pass: gradients of sum(d_out * out) + sum(d_final * final_state) with respect to
@@ -280,12 +282,13 @@ size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t n
  *                [batch, seqlen, H] (w.r.t. the raw beta, before the sigmoid; dg w.r.t. the raw gate)
  *   dA_log fp32 [H], ddt_bias fp32 [H, K]  (overwritten: zeroed, then summed over all tokens)
  *   d_initial    fp32 [N, H, K, V] or NULL (not written)
- * Token by token on CUDA cores, four persistent CTAs per (sequence, head) (32 state columns each):
- * (without checkpoints) a forward that stores one every 64 tokens, then chunk by chunk from the
- * last a rerun from the checkpoint and a reverse walk over its tokens; a second kernel sums the
- * column slices and applies the derivatives of the in-kernel transforms.  Gradient pointers are 16-byte aligned (dbeta 2, dA_log 4).  With
- * out-of-order cu_seqlens every document is treated as empty: the token gradients are not written
- * and d_initial = d_final (there is no status word to report it). */
+ * In the chunked form, on CUDA cores in fp32: (without checkpoints) the checkpointing forward; then
+ * per 64-token chunk, in parallel, the chunk's factors (gate, norms, decay-weighted Gram products,
+ * (I + A)^{-1}); per (sequence, head), from the last chunk to the first, the gradient of the state at
+ * every chunk boundary; per chunk, in parallel, the gradients of the chunk's inputs; and a last
+ * kernel for the derivatives of the in-kernel transforms.  Gradient pointers are 16-byte aligned
+ * (dbeta 2, dA_log 4).  With out-of-order cu_seqlens every document is treated as empty: the token
+ * gradients are not written, d_initial = d_final, and the workspace status word records it. */
 kda_status_t kda_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
                      const float* A_log, const float* dt_bias, float lower_bound, const float* initial_state,
                      const void* d_out, const float* d_final, const float* checkpoints, void* dq, void* dk,

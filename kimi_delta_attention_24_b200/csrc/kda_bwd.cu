@@ -1,42 +1,63 @@
-// Backward pass of the KDA forward (gradients of every input), token by token on CUDA cores.
+// Backward pass of the KDA forward (gradients of every input), in the chunked form.
 //
 // torchtitan trains Kimi-K3 through chunk_kda, and its varlen test checks the gradient as well
-// as the forward (torchtitan PR #4374, Results: test_varlen_matches_independent_documents).  For
-// one token, with Stil = Diag(alpha) S_{t-1}, p = Stil^T khat, delta = beta (v - p),
-// S_t = Stil + khat delta^T and o_t = scale S_t^T qhat, the reverse-mode step given dS (the
-// gradient w.r.t. S_t) and do_t is
-//   dS += scale qhat do^T;  dqhat = scale S_t do;  dkhat = dS delta + Stil dp;  ddelta = dS^T khat;
-//   dbeta = ddelta . (v - p);  dv = beta ddelta;  dp = -beta ddelta;  dStil = dS + khat dp^T;
-//   dalpha_c = sum_j dStil[c][j] S_{t-1}[c][j];  dS_{t-1} = Diag(alpha) dStil,
+// as the forward (torchtitan PR #4374, Results: test_varlen_matches_independent_documents).  The
+// forward of one 64-token chunk (rows r, state S at the chunk start; Gamma the in-chunk cumulative
+// log-decay, gamma its last row, khat / qhat the normalised keys / queries) is
+//   Kg = khat e^Gamma,  Qt = scale qhat e^Gamma,  Kt = khat e^{gamma - Gamma},
+//   M_rs = sum_c khat_rc khat_sc e^{Gamma_rc - Gamma_sc},  A = strict_tril(diag(beta) M),
+//   P = scale tril(qhat-khat gated the same way),  T = (I + A)^{-1},  T_b = T diag(beta),
+//   W = T_b Kg,  U = T_b V,  Delta = U - W S,  O = Qt S + P Delta,  S' = Diag(e^gamma) S + Kt^T Delta.
+// Reverse mode, given dO and dS' (the gradient of the chunk's end state):
+//   dDelta = P^T dO + Kt dS',   dS = Diag(e^gamma) dS' + (Qt - P W)^T dO - W^T Kt dS'   (to the chunk before),
+//   dKt = Delta dS'^T,  dQt = dO S^T + dP Kn,  dP = tril(dO Delta^T),  dW = -dDelta S^T,
+//   dT_b = dDelta V^T + dW Kg^T,  dV = T_b^T dDelta,  dKg = T_b^T dW,  dA = strict_tril(-T^T dT T^T)
+//   with dT = dT_b diag(beta),  dM = diag(beta) dA,  dbeta = colsum(dT_b o T) + rowsum(dA o M),
+// and the decay-weighted products that carry dM and dP back to khat and qhat never form e^{-Gamma}
+// alone: X1_r = sum_{s<r} dM_rs khat_s e^{Gamma_r - Gamma_s} and its transposed and P counterparts
+// are evaluated per 16-row sub-block against the decays at a sub-block boundary, so that every
+// factor lies in [e^{-80}, e^{80}] (|log alpha| <= 5).  Then
+//   dkhat = X1 + X2 + X4 + e^Gamma dKg + e^{gamma - Gamma} dKt,   dqhat = scale (X3 + e^Gamma dO S^T),
+//   dGamma = khat (X1 + e^Gamma dKg - X2 - X4 - e^{gamma - Gamma} dKt) + qhat dqhat,
+//   dlog alpha_r = sum_{r' >= r} dGamma_r' + dgamma,  dgamma = e^gamma rowsum(S o dS') + sum_r khat e^{gamma-Gamma} dKt,
 // followed by the derivatives of the in-kernel transforms (L2 norms, sigmoid of beta, safe gate).
 //
-// The columns of the state evolve independently, so one (sequence, head) unit is split over four
-// CTAs of 32 state columns each (persistent over (unit, slice) pairs, two CTAs per SM, 256
-// threads).  Inside a CTA, warp w owns 4 columns over all 128 rows and lane l rows 4 l .. 4 l + 3,
-// so each thread holds a 4 x 4 block of the state and of its gradient, and the sums over rows that
-// the token chain needs (the prediction S^T khat and the delta gradient dS^T khat) are warp
-// shuffles: a warp runs the token recurrence on its columns without waiting for the others.  A CTA
-// first runs the forward over its sequence, storing its slice at the start of every 32-token chunk
-// in the workspace; then, chunk by chunk from the last, it reruns the chunk's forward from its
-// checkpoint, storing the slice before every token in a per-CTA scratch, and walks the chunk's tokens
-// backwards.  Each chunk's inputs are transformed once (norms, gate, sigmoid) into shared memory,
-// and the next token's scratch state is fetched during the current one.  What sums over columns
-// (dqhat, dkhat, dalpha per channel, dbeta) is added over the CTA's warps through shared memory (one
-// barrier per token) and written per slice; a second kernel adds the slices, applies the derivatives
-// of the L2 norms, the gate and the sigmoid, and adds the dA_log / dt_bias sums with one atomic per
-// value per CTA (the outputs are zeroed first).
+// Launches: the checkpointing forward when no chunk-start states are given (the split path, which
+// stores S at every chunk start); bwd_prep_kernel (chunk-parallel: recomputes a chunk's factors and
+// stores W, Kt, P^T dO, (Qt - P W)^T dO and e^gamma); bwd_state_kernel (one CTA per (sequence, head),
+// chunks last to first: dDelta and the state gradient at every chunk boundary); bwd_grad_kernel
+// (chunk-parallel: recomputes the factors and forms the gradients above); bwd_finish_kernel (the
+// transforms, and dA_log / dt_bias summed with one atomic per value per CTA).  The chunk-parallel
+// kernels are persistent; each CTA keeps one chunk's intermediates in its own global scratch, which
+// stays in L2.  Arithmetic is fp32 on CUDA cores throughout.
 #include "kda_common.cuh"
 
 namespace kda {
 namespace {
 
 constexpr int kBwdThreads = 256;
-constexpr int kBwdChunk = 64;  // tokens per checkpoint: the forward's chunk, whose start states it can store
-constexpr int kStage = 32;     // tokens whose transformed inputs are staged in shared memory at once
-constexpr int kSlice = 32;  // state columns per CTA (4 per warp)
-constexpr int kSlices = kHeadDim / kSlice;
-constexpr size_t kStateElems = (size_t)kHeadDim * kHeadDim;
-constexpr size_t kSliceElems = (size_t)kHeadDim * kSlice;
+constexpr int C = 64;
+constexpr int D = kHeadDim;
+constexpr int kF = C * D;          // one 64 x 128 fp32 matrix
+constexpr int kQ = C * C;          // one 64 x 64 fp32 matrix
+constexpr size_t kStateElems = (size_t)D * D;
+
+// per-chunk outputs of bwd_prep_kernel, for bwd_state_kernel (floats)
+constexpr int PR_W = 0;            // W [64][128]
+constexpr int PR_KT = kF;          // Kt [64][128]
+constexpr int PR_PDO = 2 * kF;     // P^T dO [64][128]
+constexpr int PR_Y = 3 * kF;       // (Qt - P W)^T dO [128][128]
+constexpr int PR_EG = 3 * kF + D * D;  // e^gamma [128]
+constexpr int kPrepFloats = PR_EG + D;
+
+// per-CTA scratch (floats)
+constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_V = 4 * kF, SC_DO = 5 * kF;
+constexpr int SC_W = 6 * kF, SC_D = 7 * kF, SC_DKT = 8 * kF, SC_DQS = 9 * kF, SC_DW = 10 * kF;
+constexpr int SC_DKG = 11 * kF, SC_R = 12 * kF, SC_L = 13 * kF, SC_X = 14 * kF;
+constexpr int SC_M = 15 * kF, SC_P = SC_M + kQ, SC_T = SC_P + kQ, SC_TB = SC_T + kQ, SC_DP = SC_TB + kQ;
+constexpr int SC_DTB = SC_DP + kQ, SC_TMP = SC_DTB + kQ, SC_DA = SC_TMP + kQ;
+constexpr int SC_BETA = SC_DA + kQ, SC_EG = SC_BETA + C, SC_DGAM = SC_EG + D, SC_DB = SC_DGAM + D;
+constexpr int kScratchFloats = SC_DB + C + 64;
 
 struct BwdParams {
   FwdParams f;
@@ -50,10 +71,13 @@ struct BwdParams {
   float* dA_log;                // [H], zeroed before the launch
   float* ddt_bias;              // [H, K], zeroed before the launch
   float* d_initial;             // [N, H, K, V] or null
-  const float* ckpt_in;         // the forward's checkpoints, or null (then computed into ckpt)
-  float* ckpt;                  // (T / 64 + N + 1) x H states: chunk-start checkpoints, S^T[v][k]
-  float* scratch;               // gridDim.x x 64 slices: the states before each token of a chunk
-  float* part;                  // per slice: dqhat, dkhat, dalpha [tokens, H, K]; then dbeta [slice][tokens, H]
+  const float* ckpt;            // chunk-start states, S^T [v][k], slot bos / 64 + n + j for chunk j of sequence n
+  const int32_t* chunk_off;     // [N + 1] first global chunk of each sequence
+  float* prep;                  // kPrepFloats per (global chunk, head)
+  float* dsp;                   // per slot and head: dS' [k][v], the gradient of chunk j's end state (slot of chunk j)
+  float* dd;                    // kF per (global chunk, head): dDelta
+  float* part;                  // dqhat, dkhat, dlog alpha [tokens, H, K] each; then dbeta [tokens, H]
+  float* scratch;               // kScratchFloats per CTA of the chunk-parallel kernels
 };
 
 __device__ __forceinline__ float sigmoid_acc(float x) { return 1.0f / (1.0f + expf(-x)); }
@@ -72,321 +96,768 @@ __device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, float a, float b, fl
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-// Sum over the 32 lanes of a warp, every lane getting the totals.
-__device__ __forceinline__ void warp_allsum4(float (&x)[4]) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) x[j] += __shfl_xor_sync(0xffffffffu, x[j], o);
-}
-__device__ __forceinline__ float warp_allsum(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
+// ------------------------------------------------------------------------- generic fp32 GEMM
+// An operand: element (i, j) is p[i * ld + j], or p[j * ld + i] when t (transposed).
+struct Mat {
+  const float* p;
+  int ld;
+  bool t;
+};
+__device__ __forceinline__ Mat mat(const float* p, int ld, bool t = false) { return Mat{p, ld, t}; }
 
-// Up to kStage tokens' transformed inputs, staged in shared memory (each warp transforms every eighth
-// token) and read by all warps: khat, qhat and alpha per channel, v and d_out on the slice's columns,
-// beta.
-struct ChunkIn {
-  float k[kStage][kHeadDim];
-  float q[kStage][kHeadDim];
-  float a[kStage][kHeadDim];
-  float v[kStage][kSlice];
-  float d[kStage][kSlice];
-  float b[kStage];
+constexpr int GB_K = 64;   // depth of one staged slice
+struct GemmSmem {
+  float a[GB_K][64];
+  float b[GB_K][128];
 };
 
-__device__ __forceinline__ void stage_chunk(const BwdParams& P, ChunkIn& s, int64_t t_begin, int len, int h,
-                                            int scol0, float ea, float4 dt, bool full) {
-  const FwdParams& p = P.f;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int H = p.num_heads;
-  constexpr int D = kHeadDim;
-  const float dts[4] = {dt.x, dt.y, dt.z, dt.w};
-  for (int i = warp; i < len; i += kBwdThreads / 32) {
-    const size_t row = (size_t)(t_begin + i) * H + h;
-    const float4 k4 = ld_bf16x4(p.k + row * D + 4 * lane);
-    const float4 g4 = ld_bf16x4(p.g + row * D + 4 * lane);
-    const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w};
-    const float nk = sqrtf(warp_allsum(kv[0] * kv[0] + kv[1] * kv[1] + kv[2] * kv[2] + kv[3] * kv[3]) + kL2Eps);
-    float av[4];
+// Loads the GB_K x W slice (k0.., i0..) of an operand into s[k][i] (zero outside rows x depth),
+// element (i, k) being p[k * ld + i] (memory along i) or p[i * ld + k] (kmaj: memory along k, the
+// slice transposed on the way in).
+template <int W>
+__device__ __forceinline__ void gemm_load(float (*s)[W], const float* p, int ld, bool kmaj, int i0, int k0, int rows,
+                                          int depth) {
+  const int tid = threadIdx.x;
+  constexpr int kVec = GB_K * W / 4;  // float4s in the slice
+  if (!kmaj) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) av[j] = expf(p.lower_bound * sigmoid_acc(ea * (gv[j] + dts[j])));
-    reinterpret_cast<float4*>(s.k[i])[lane] = make_float4(kv[0] / nk, kv[1] / nk, kv[2] / nk, kv[3] / nk);
-    reinterpret_cast<float4*>(s.a[i])[lane] = make_float4(av[0], av[1], av[2], av[3]);
-    if (lane < kSlice / 4) reinterpret_cast<float4*>(s.v[i])[lane] = ld_bf16x4(p.v + row * D + scol0 + 4 * lane);
-    if (lane == 0) s.b[i] = sigmoid_acc(__bfloat162float(p.beta[row]));
-    if (full) {
-      const float4 q4 = ld_bf16x4(p.q + row * D + 4 * lane);
-      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-      const float nq = sqrtf(warp_allsum(qv[0] * qv[0] + qv[1] * qv[1] + qv[2] * qv[2] + qv[3] * qv[3]) + kL2Eps);
-      reinterpret_cast<float4*>(s.q[i])[lane] = make_float4(qv[0] / nq, qv[1] / nq, qv[2] / nq, qv[3] / nq);
-      if (lane < kSlice / 4) reinterpret_cast<float4*>(s.d[i])[lane] = ld_bf16x4(P.d_out + row * D + scol0 + 4 * lane);
+    for (int e = 0; e < (kVec + kBwdThreads - 1) / kBwdThreads; ++e) {
+      const int idx = tid + e * kBwdThreads;
+      if (kVec % kBwdThreads != 0 && idx >= kVec) break;
+      const int i4 = idx % (W / 4), k = idx / (W / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k0 + k < depth && i0 + 4 * i4 < rows)
+        v = *reinterpret_cast<const float4*>(p + (size_t)(k0 + k) * ld + i0 + 4 * i4);
+      *reinterpret_cast<float4*>(&s[k][4 * i4]) = v;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < (kVec + kBwdThreads - 1) / kBwdThreads; ++e) {
+      const int idx = tid + e * kBwdThreads;
+      if (kVec % kBwdThreads != 0 && idx >= kVec) break;
+      const int i = idx % W, k4 = idx / W;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 + i < rows && k0 + 4 * k4 < depth)
+        v = *reinterpret_cast<const float4*>(p + (size_t)(i0 + i) * ld + k0 + 4 * k4);
+      s[4 * k4 + 0][i] = v.x;
+      s[4 * k4 + 1][i] = v.y;
+      s[4 * k4 + 2][i] = v.z;
+      s[4 * k4 + 3][i] = v.w;
     }
   }
 }
 
-// One CTA per (unit, slice of 32 state columns); warp w owns columns 4 w .. 4 w + 3 of the slice over
-// all 128 rows, lane l rows 4 l .. 4 l + 3 (a 4 x 4 block of the state and of its gradient per
-// thread).  The columns of the state evolve independently, so every warp runs the token recurrence
-// on its own columns: the sums over rows (the prediction and the delta gradient) are warp shuffles,
-// and the token chain needs no barrier of the CTA.  Each chunk's inputs are transformed once into
-// shared memory.  What sums over columns (dqhat, dkhat, dalpha per row, dbeta) is summed over the
-// CTA's warps through shared memory (one barrier per token) and written per slice for
-// bwd_finish_kernel.  Checkpoints and the per-token scratch are stored per thread (16 contiguous
-// floats), since every thread reads back only what it wrote.
-__global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(BwdParams P) {
-  constexpr int D = kHeadDim;
-  extern __shared__ __align__(16) uint8_t bwd_smem[];
-  ChunkIn& s = *reinterpret_cast<ChunkIn*>(bwd_smem);
-  float (*part)[8][3][D] = reinterpret_cast<float (*)[8][3][D]>(bwd_smem + sizeof(ChunkIn));  // [buffer][warp]
-  float (*part_beta)[8] = reinterpret_cast<float (*)[8]>(bwd_smem + sizeof(ChunkIn) + 2 * 8 * 3 * D * sizeof(float));
+// C[i][j] = alpha sum_k A(i, k) B(k, j) (+ C[i][j] when acc), i < M, j < N; mask 1 keeps j < i,
+// mask 2 keeps j <= i (the rest is written as 0).  Output tiles of (16 RM) x 128: thread (ty, tx)
+// holds rows RM ty .. + RM - 1 and columns 4 tx .. + 3 and 64 + 4 tx .. + 3 (conflict-free
+// 16-byte reads of the B slice).  M, N, K multiples of 4; operands 16-byte aligned with ld a
+// multiple of 4.  All threads of the CTA call it; it ends with a barrier.
+template <int RM>
+__device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc, int mask,
+                       GemmSmem& sm) {
+  constexpr int BM = 16 * RM;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  float (*sa)[BM] = reinterpret_cast<float (*)[BM]>(&sm.a[0][0]);
+  for (int i0 = 0; i0 < M; i0 += BM) {
+    for (int j0 = 0; j0 < N; j0 += 128) {
+      float c[RM][8];
+#pragma unroll
+      for (int a = 0; a < RM; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) c[a][b] = 0.f;
+      for (int k0 = 0; k0 < K; k0 += GB_K) {
+        // A(i, k): memory along k when not transposed; B(k, j): memory along j when not transposed
+        gemm_load<BM>(sa, A.p, A.ld, !A.t, i0, k0, M, K);
+        gemm_load<128>(sm.b, B.p, B.ld, B.t, j0, k0, N, K);
+        __syncthreads();
+        const int kn = K - k0 < GB_K ? K - k0 : GB_K;
+#pragma unroll 4
+        for (int k = 0; k < kn; ++k) {
+          float ar[RM];
+          if constexpr (RM == 4) {
+            const float4 av = *reinterpret_cast<const float4*>(&sa[k][4 * ty]);
+            ar[0] = av.x;
+            ar[1] = av.y;
+            ar[2] = av.z;
+            ar[3] = av.w;
+          } else {
+#pragma unroll
+            for (int a = 0; a < RM; ++a) ar[a] = sa[k][RM * ty + a];
+          }
+          const float4 b0 = *reinterpret_cast<const float4*>(&sm.b[k][4 * tx]);
+          const float4 b1 = *reinterpret_cast<const float4*>(&sm.b[k][64 + 4 * tx]);
+          const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+          for (int a = 0; a < RM; ++a)
+#pragma unroll
+            for (int b = 0; b < 8; ++b) c[a][b] = fmaf(ar[a], br[b], c[a][b]);
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int a = 0; a < RM; ++a) {
+        const int i = i0 + RM * ty + a;
+        if (i >= M) continue;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int j = j0 + 64 * hf + 4 * tx;
+          if (j >= N) continue;
+          float4* dst = reinterpret_cast<float4*>(Cp + (size_t)i * ldc + j);
+          float4 o = make_float4(alpha * c[a][4 * hf], alpha * c[a][4 * hf + 1], alpha * c[a][4 * hf + 2],
+                                 alpha * c[a][4 * hf + 3]);
+          if (acc) {
+            const float4 old = *dst;
+            o.x += old.x;
+            o.y += old.y;
+            o.z += old.z;
+            o.w += old.w;
+          }
+          if (mask) {
+            const int lim = mask == 1 ? i : i + 1;  // keep j < lim
+            if (j + 0 >= lim) o.x = 0.f;
+            if (j + 1 >= lim) o.y = 0.f;
+            if (j + 2 >= lim) o.z = 0.f;
+            if (j + 3 >= lim) o.w = 0.f;
+          }
+          *dst = o;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void gemm(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc,
+                                     int mask, GemmSmem& sm) {
+  if (M <= 16) gemm_t<1>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
+  else gemm_t<4>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
+}
+
+// ------------------------------------------------------------------------- element-wise passes
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+__device__ __forceinline__ float4 sub4(float4 a, float4 b) { return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w); }
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+__device__ __forceinline__ float4 scl4(float4 a, float f) { return make_float4(a.x * f, a.y * f, a.z * f, a.w * f); }
+// the decays: exp of a difference of log-decays (exp(-inf) = 0)
+__device__ __forceinline__ float dexp(float x) { return __expf(x); }
+__device__ __forceinline__ float4 dexp4(float4 x) { return make_float4(dexp(x.x), dexp(x.y), dexp(x.z), dexp(x.w)); }
+struct F4x2 {
+  float4 a, b;
+};
+struct F4x4 {
+  float4 a, b, c, d;
+};
+
+// An element-wise pass over n4 float4 positions, kBatch per thread at a time: each thread evaluates
+// f at a batch of its positions (loads and arithmetic) before it stores any of their results with
+// st.  The buffers share one allocation, so the compiler would not move a load above an earlier
+// store by itself, and every position would cost a round trip to L2.
+template <int kBatch, typename F, typename S>
+__device__ __forceinline__ void ew(int n4, F f, S st) {
+  using V = decltype(f(0));
+  for (int base = threadIdx.x; base < n4; base += kBatch * kBwdThreads) {
+    V v[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int i = base + b * kBwdThreads;
+      if (i < n4) v[b] = f(i);
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int i = base + b * kBwdThreads;
+      if (i < n4) st(i, v[b]);
+    }
+  }
+}
+constexpr int kF4 = kF / 4, kQ4 = kQ / 4;  // float4s in a 64 x 128 / 64 x 64 matrix
+constexpr int kB1 = 8, kB2 = 4, kB4 = 2;  // batch sizes for results of 1, 2 and 4 float4s
+
+// ------------------------------------------------------------------------- per-chunk recomputation
+struct Chunk {
+  int n, h, len;
+  int64_t t0, gc, slot;
+};
+
+__device__ __forceinline__ int seq_of_chunk(const int32_t* co, int nseq, int64_t gc) {
+  int lo = 0, hi = nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)co[mid] <= gc) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ Chunk locate(const BwdParams& P, int64_t item) {
+  const int H = P.f.num_heads;
+  Chunk c;
+  c.gc = item / H;
+  c.h = (int)(item - c.gc * H);
+  c.n = seq_of_chunk(P.chunk_off, P.f.num_seqs, c.gc);
+  int64_t bos, eos;
+  seq_range(P.f, c.n, bos, eos);
+  const int64_t j = c.gc - P.chunk_off[c.n];
+  c.t0 = bos + j * C;
+  c.len = (int)(eos - c.t0 < C ? eos - c.t0 : C);
+  c.slot = bos / C + c.n + j;
+  return c;
+}
+
+// The factors of a chunk that do not involve the state, into the CTA's scratch s:
+//   kh, qh, Gamma (G), beta, e^gamma, Kg; V and dO (fp32, rows past the chunk's end zero);
+//   M (strict lower), P (lower, with scale), T = (I + A)^{-1}, T_b.
+// need_v: also V (the gradient kernel).
+__device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, bool need_v, GemmSmem& gsm,
+                              float* sT /* shared 64 x 65 */, float* sA /* shared 64 x 65 */) {
   const FwdParams& p = P.f;
   const int H = p.num_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t units = (int64_t)p.num_seqs * H;
-  const int64_t work = units * kSlices;
-  float* const scr = P.scratch + (size_t)blockIdx.x * kBwdChunk * kSliceElems;
-  const bool seqlens_ok = cta_seqlens_ok(p);
-  const int64_t rows_total = (p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs) * H;
+  const int h = ch.h, len = ch.len;
+  const float ea = expf(p.A_log[h]);
+  const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
+  const float dts[4] = {dt.x, dt.y, dt.z, dt.w};
+  // prologue: warp per row, lane per 4 channels; each warp loads four rows before it stores any
+  for (int r0 = warp; r0 < C; r0 += 4 * (kBwdThreads / 32)) {
+    float4 k4[4], q4[4], g4[4], v4[4], o4[4];
+    float br[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = r0 + u * (kBwdThreads / 32);
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      k4[u] = q4[u] = g4[u] = v4[u] = o4[u] = z;
+      br[u] = 0.f;
+      if (r < len) {
+        const size_t row = (size_t)(ch.t0 + r) * H + h;
+        k4[u] = ld_bf16x4(p.k + row * D + 4 * lane);
+        q4[u] = ld_bf16x4(p.q + row * D + 4 * lane);
+        g4[u] = ld_bf16x4(p.g + row * D + 4 * lane);
+        if (need_v) v4[u] = ld_bf16x4(p.v + row * D + 4 * lane);
+        o4[u] = ld_bf16x4(P.d_out + row * D + 4 * lane);
+        br[u] = __bfloat162float(p.beta[row]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = r0 + u * (kBwdThreads / 32);
+      float sk = k4[u].x * k4[u].x + k4[u].y * k4[u].y + k4[u].z * k4[u].z + k4[u].w * k4[u].w;
+      float sq = q4[u].x * q4[u].x + q4[u].y * q4[u].y + q4[u].z * q4[u].z + q4[u].w * q4[u].w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      }
+      const float ik = 1.0f / sqrtf(sk + kL2Eps), iq = 1.0f / sqrtf(sq + kL2Eps);
+      const float gv[4] = {g4[u].x, g4[u].y, g4[u].z, g4[u].w};
+      float la[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) la[j] = r < len ? p.lower_bound * sigmoid_acc(ea * (gv[j] + dts[j])) : 0.f;
+      st4(s + SC_KH + r * D + 4 * lane, scl4(k4[u], ik));
+      st4(s + SC_QH + r * D + 4 * lane, scl4(q4[u], iq));
+      st4(s + SC_G + r * D + 4 * lane, make_float4(la[0], la[1], la[2], la[3]));
+      if (need_v) st4(s + SC_V + r * D + 4 * lane, v4[u]);
+      st4(s + SC_DO + r * D + 4 * lane, o4[u]);
+      if (lane == 0) s[SC_BETA + r] = r < len ? sigmoid_acc(br[u]) : 0.f;
+    }
+  }
+  __syncthreads();
+  // Gamma: running sum down the rows, one thread per channel (16 rows read at a time)
+  if (tid < D) {
+    float acc = 0.f;
+    for (int r0 = 0; r0 < C; r0 += 16) {
+      float col[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) col[r] = s[SC_G + (r0 + r) * D + tid];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        acc += col[r];
+        s[SC_G + (r0 + r) * D + tid] = acc;
+      }
+    }
+    s[SC_EG + tid] = dexp(acc);
+  }
+  __syncthreads();
+  ew<kB1>(kF4, [&](int i) { return mul4(ld4(s + SC_KH + 4 * i), dexp4(ld4(s + SC_G + 4 * i))); },
+            [&](int i, float4 v) { st4(s + SC_KG + 4 * i, v); });
+  // M and P per row block I: (Y_r e^{Gamma_r - rho_I}) (khat_s e^{rho_I - Gamma_s})^T, rho_I = Gamma at
+  // the end of block I - 1 (0 for I = 0)
+  for (int I = 0; I < 4; ++I) {
+    const int ns = 16 * (I + 1);
+    const float* rho = s + SC_G + (16 * I - 1) * D;
+    ew<kB1>(ns * D / 4,
+              [&](int i) {
+                const int c = (4 * i) & (D - 1);
+                const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
+                return mul4(ld4(s + SC_KH + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + 4 * i))));
+              },
+              [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
+    ew<kB2>(16 * D / 4,
+          [&](int i) {
+            const int c = (4 * i) & (D - 1), e = 16 * I * D + 4 * i;
+            const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
+            const float4 f = dexp4(sub4(ld4(s + SC_G + e), r4));
+            return F4x2{mul4(ld4(s + SC_KH + e), f), mul4(ld4(s + SC_QH + e), f)};
+          },
+          [&](int i, F4x2 v) {
+            st4(s + SC_L + 4 * i, v.a);
+            st4(s + SC_L + 16 * D + 4 * i, v.b);
+          });
+    __syncthreads();
+    gemm(s + SC_M + 16 * I * C, C, mat(s + SC_L, D), mat(s + SC_R, D, true), 16, ns, D, 1.f, false, 0, gsm);
+    gemm(s + SC_P + 16 * I * C, C, mat(s + SC_L + 16 * D, D), mat(s + SC_R, D, true), 16, ns, D, p.scale, false, 0,
+         gsm);
+  }
+  // M strictly lower, P lower with its diagonal: the entries right of each block's segment are zero
+  ew<kB2>(kQ4,
+            [&](int i) {
+              const int r = (4 * i) >> 6, c = (4 * i) & (C - 1);
+              const int ns = 16 * ((r >> 4) + 1);
+              float4 m = make_float4(0.f, 0.f, 0.f, 0.f), q = m;
+              if (c < ns) {
+                m = ld4(s + SC_M + 4 * i);
+                q = ld4(s + SC_P + 4 * i);
+              }
+              if (c + 0 >= r) m.x = 0.f;
+              if (c + 1 >= r) m.y = 0.f;
+              if (c + 2 >= r) m.z = 0.f;
+              if (c + 3 >= r) m.w = 0.f;
+              if (c + 0 > r) q.x = 0.f;
+              if (c + 1 > r) q.y = 0.f;
+              if (c + 2 > r) q.z = 0.f;
+              if (c + 3 > r) q.w = 0.f;
+              return F4x2{m, q};
+            },
+            [&](int i, F4x2 v) {
+              st4(s + SC_M + 4 * i, v.a);
+              st4(s + SC_P + 4 * i, v.b);
+              const int r = (4 * i) >> 6, c = (4 * i) & (C - 1);
+              const float b = s[SC_BETA + r];
+              sA[r * 65 + c] = b * v.a.x;
+              sA[r * 65 + c + 1] = b * v.a.y;
+              sA[r * 65 + c + 2] = b * v.a.z;
+              sA[r * 65 + c + 3] = b * v.a.w;
+              sT[r * 65 + c] = 0.f;
+              sT[r * 65 + c + 1] = 0.f;
+              sT[r * 65 + c + 2] = 0.f;
+              sT[r * 65 + c + 3] = 0.f;
+            });
+  __syncthreads();
+  // T = (I + A)^{-1}, A = diag(beta) M, in shared memory (leading dimension 65): diagonal 16 x 16
+  // blocks by substitution, then the blocks below them by distance, T_IJ = -T_II sum_K A_IK T_KJ
+  if (tid < 64) {
+    const int I = tid >> 4, j = tid & 15;
+    float x[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) x[m] = (m == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int m = 0; m < 15; ++m) {
+      const float xm = x[m];
+#pragma unroll
+      for (int i = m + 1; i < 16; ++i) x[i] = fmaf(-sA[(16 * I + i) * 65 + 16 * I + m], xm, x[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sT[(16 * I + i) * 65 + 16 * I + j] = x[i];
+  }
+  __syncthreads();
+  for (int dd = 1; dd < 4; ++dd) {
+    // Y_IJ = sum_{K=J}^{I-1} A_IK T_KJ for the 4 - dd blocks at this distance, parked in the (zero)
+    // blocks above the diagonal (row block J, column block I), which the result never reads
+    const int nb = 4 - dd;
+    for (int e = tid; e < nb * 256; e += kBwdThreads) {
+      const int J = e >> 8, I = J + dd, r = (e >> 4) & 15, c = e & 15;
+      float y = 0.f;
+      for (int k = 16 * J; k < 16 * I; ++k) y = fmaf(sA[(16 * I + r) * 65 + k], sT[k * 65 + 16 * J + c], y);
+      sT[(16 * J + r) * 65 + 16 * I + c] = y;
+    }
+    __syncthreads();
+    for (int e = tid; e < nb * 256; e += kBwdThreads) {
+      const int J = e >> 8, I = J + dd, r = (e >> 4) & 15, c = e & 15;
+      float t = 0.f;
+      for (int k = 0; k <= r; ++k) t = fmaf(sT[(16 * I + r) * 65 + 16 * I + k], sT[(16 * J + k) * 65 + 16 * I + c], t);
+      sT[(16 * I + r) * 65 + 16 * J + c] = -t;
+    }
+    __syncthreads();
+    for (int e = tid; e < nb * 256; e += kBwdThreads) {
+      const int J = e >> 8, I = J + dd, r = (e >> 4) & 15, c = e & 15;
+      sT[(16 * J + r) * 65 + 16 * I + c] = 0.f;
+    }
+    __syncthreads();
+  }
+  ew<kB2>(kQ4,
+            [&](int i) {
+              const int r = (4 * i) >> 6, c = (4 * i) & (C - 1);
+              const float4 t = make_float4(sT[r * 65 + c], sT[r * 65 + c + 1], sT[r * 65 + c + 2], sT[r * 65 + c + 3]);
+              return F4x2{t, mul4(t, ld4(s + SC_BETA + c))};
+            },
+            [&](int i, F4x2 v) {
+              st4(s + SC_T + 4 * i, v.a);
+              st4(s + SC_TB + 4 * i, v.b);
+            });
+  __syncthreads();
+}
 
-  for (int64_t wi = blockIdx.x; wi < work; wi += gridDim.x) {
-    const int64_t u = wi / kSlices;
-    const int sl = (int)(wi - u * kSlices);
-    const int n = (int)(u / H), h = (int)(u % H);
-    const int scol0 = sl * kSlice;         // the slice's first state column
-    const int col0 = scol0 + 4 * warp;     // this warp's first state column (v)
-    int64_t bos, eos;
-    seq_range(p, n, bos, eos);
-    if (!seqlens_ok) eos = bos;
-    const int64_t L = eos - bos;
-    const int nch = (int)((L + kBwdChunk - 1) / kBwdChunk);
-    const size_t soff = ((size_t)n * H + h) * kStateElems;
-    const int64_t ck0 = bos / kBwdChunk + n;  // this sequence's first checkpoint slot
-    const float ea = expf(p.A_log[h]);
-    const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
-    float S[4][4];  // S[4 lane + i][col0 + j]
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (p.initial_state) t = *reinterpret_cast<const float4*>(p.initial_state + soff + (size_t)(4 * lane + i) * D + col0);
-      S[i][0] = t.x; S[i][1] = t.y; S[i][2] = t.z; S[i][3] = t.w;
-    }
-    // checkpoint of chunk c: the whole state, transposed (S^T[v][k]), as the forward stores it
-    const float* ck_base = P.ckpt_in ? P.ckpt_in : P.ckpt;
-    auto ck_ptr = [&](int c) { return ck_base + ((size_t)(ck0 + c) * H + h) * kStateElems; };
-    auto load_ckpt = [&](const float* base) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 t = *reinterpret_cast<const float4*>(base + (size_t)(col0 + j) * D + 4 * lane);
-        S[0][j] = t.x; S[1][j] = t.y; S[2][j] = t.z; S[3][j] = t.w;
-      }
-    };
-    auto store_ckpt = [&](float* base) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        *reinterpret_cast<float4*>(base + (size_t)(col0 + j) * D + 4 * lane) = make_float4(S[0][j], S[1][j], S[2][j], S[3][j]);
-    };
-    float* const part_q = P.part + (size_t)sl * 3 * rows_total * D;
-    float* const part_b = P.part + (size_t)kSlices * 3 * rows_total * D + (size_t)sl * rows_total;
-
-    auto store_state = [&](float* base) {
-      float4* dst = reinterpret_cast<float4*>(base + (size_t)tid * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
-    };
-    auto load_state = [&](const float* base) {
-      const float4* src = reinterpret_cast<const float4*>(base + (size_t)tid * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 t = src[i];
-        S[i][0] = t.x; S[i][1] = t.y; S[i][2] = t.z; S[i][3] = t.w;
-      }
-    };
-    // the chunk's token i, this thread's rows and the warp's columns
-    auto row4 = [&](const float (*m)[D], int i) {
-      const float4 t = reinterpret_cast<const float4*>(m[i])[lane];
-      return t;
-    };
-    auto forward_token = [&](int i) {
-      const float4 a4 = row4(s.a, i), k4 = row4(s.k, i);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
-      const float4 v4 = reinterpret_cast<const float4*>(s.v[i])[warp];
-      const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-      const float b = s.b[i];
-      float pr[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          S[r][j] *= av[r];
-          pr[j] = fmaf(S[r][j], kv[r], pr[j]);
-        }
-      warp_allsum4(pr);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float d = b * (vv[j] - pr[j]);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) S[r][j] = fmaf(kv[r], d, S[r][j]);
-      }
-    };
-
-    // ---------------------------------------------------------------- forward with checkpoints
-    // (only without the forward's checkpoints; each CTA writes its own 32 columns of them)
-    if (!P.ckpt_in) {
-      for (int c = 0; c < nch; ++c) {
-        const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
-        const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
-        store_ckpt(P.ckpt + ((size_t)(ck0 + c) * H + h) * kStateElems);
-        for (int h0 = 0; h0 < len; h0 += kStage) {
-          const int hl = min(kStage, len - h0);
-          __syncthreads();  // the previously staged inputs are read
-          stage_chunk(P, s, t_begin + h0, hl, h, scol0, ea, dt, false);
-          __syncthreads();
-          for (int i = 0; i < hl; ++i) forward_token(i);
-        }
-      }
-    }
-
-    // ---------------------------------------------------------------- backward, chunk by chunk
-    float dS[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (P.d_final) t = *reinterpret_cast<const float4*>(P.d_final + soff + (size_t)(4 * lane + i) * D + col0);
-      dS[i][0] = t.x; dS[i][1] = t.y; dS[i][2] = t.z; dS[i][3] = t.w;
-    }
-    int buf = 0;
-    // one backward token: chunk token i (staged at si); S holds its S_{t-1}
-    auto backward_token = [&](int64_t t_begin, int i, int si) {
-        const size_t row = (size_t)(t_begin + i) * H + h;
-        const float4 a4 = row4(s.a, si), k4 = row4(s.k, si), q4 = row4(s.q, si);
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
-        const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-        const float4 v4 = reinterpret_cast<const float4*>(s.v[si])[warp];
-        const float4 d4 = reinterpret_cast<const float4*>(s.d[si])[warp];
-        const float vv[4] = {v4.x, v4.y, v4.z, v4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        const float b = s.b[si], scale = p.scale;
-        // p = Stil^T khat (columns), delta
-        float pj[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) pj[j] = fmaf(av[r] * S[r][j], kv[r], pj[j]);
-        warp_allsum4(pj);
-        float dl[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dl[j] = b * (vv[j] - pj[j]);
-        // dS += scale qhat do^T;  dqhat rows = scale S_t do;  ddelta = dS^T khat
-        float rq[4], dd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          float acc = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            acc = fmaf(fmaf(kv[r], dl[j], av[r] * S[r][j]), dv[j], acc);
-            dS[r][j] = fmaf(scale * qv[r], dv[j], dS[r][j]);
-            dd[j] = fmaf(dS[r][j], kv[r], dd[j]);
-          }
-          rq[r] = scale * acc;
-        }
-        warp_allsum4(dd);
-        float dp[4], db = 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          dp[j] = -b * dd[j];
-          db = fmaf(dd[j], vv[j] - pj[j], db);
-        }
-        if (lane == 0) st_bf16x4(P.dv + row * D + col0, b * dd[0], b * dd[1], b * dd[2], b * dd[3]);
-        // dkhat = dS delta + Stil dp;  dStil = dS + khat dp^T;  dalpha;  dS <- Diag(alpha) dStil
-        float rk[4], ra[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          float ak = 0.f, aa = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ak = fmaf(dS[r][j], dl[j], ak);
-            ak = fmaf(av[r] * S[r][j], dp[j], ak);
-            const float dst = fmaf(kv[r], dp[j], dS[r][j]);
-            aa = fmaf(dst, S[r][j], aa);
-            dS[r][j] = av[r] * dst;
-          }
-          rk[r] = ak;
-          ra[r] = aa;
-        }
-        if (i > 0) load_state(scr + (size_t)(i - 1) * kSliceElems);  // the next token's S_{t-1}
-        // the warps' row partials through shared memory, summed over the slice's 32 columns
-        reinterpret_cast<float4*>(part[buf][warp][0])[lane] = make_float4(rq[0], rq[1], rq[2], rq[3]);
-        reinterpret_cast<float4*>(part[buf][warp][1])[lane] = make_float4(rk[0], rk[1], rk[2], rk[3]);
-        reinterpret_cast<float4*>(part[buf][warp][2])[lane] = make_float4(ra[0], ra[1], ra[2], ra[3]);
-        if (lane == 0) part_beta[buf][warp] = db;
-        __syncthreads();
-        // 384 row sums: thread t sums entries t and t + 256 (of 3 x 128)
-        for (int e = tid; e < 3 * D; e += kBwdThreads) {
-          const int which = e / D, r = e % D;
-          float acc = 0.f;
-#pragma unroll
-          for (int w = 0; w < 8; ++w) acc += part[buf][w][which][r];
-          part_q[(size_t)which * rows_total * D + row * D + r] = acc;
-        }
-        if (tid == 0) {
-          float acc = 0.f;
-#pragma unroll
-          for (int w = 0; w < 8; ++w) acc += part_beta[buf][w];
-          part_b[row] = acc;
-        }
-        buf ^= 1;  // the next token writes the other buffer; this one is read until the next barrier
-    };
-    for (int c = nch - 1; c >= 0; --c) {
-      const int64_t t_begin = bos + (int64_t)c * kBwdChunk;
-      const int len = (int)min((int64_t)kBwdChunk, eos - t_begin);
-      const int len0 = min(kStage, len);  // tokens of the first staged half
-      // rerun the chunk's forward from its checkpoint, keeping the state before each token; the
-      // second half is staged with what the backward needs and walked backwards right away
-      load_ckpt(ck_ptr(c));
-      __syncthreads();  // the previously staged inputs and partials are read
-      stage_chunk(P, s, t_begin, len0, h, scol0, ea, dt, false);
-      __syncthreads();
-      for (int i = 0; i < len0; ++i) {
-        store_state(scr + (size_t)i * kSliceElems);
-        forward_token(i);
-      }
-      if (len > kStage) {
-        __syncthreads();
-        stage_chunk(P, s, t_begin + kStage, len - kStage, h, scol0, ea, dt, true);
-        __syncthreads();
-        for (int i = kStage; i < len; ++i) {
-          store_state(scr + (size_t)i * kSliceElems);
-          forward_token(i - kStage);
-        }
-        load_state(scr + (size_t)(len - 1) * kSliceElems);
-        for (int i = len - 1; i >= kStage; --i) backward_token(t_begin, i, i - kStage);
-      } else {
-        load_state(scr + (size_t)(len - 1) * kSliceElems);
-      }
-      // the first half backwards (S holds the state before its last token)
-      __syncthreads();
-      stage_chunk(P, s, t_begin, len0, h, scol0, ea, dt, true);
-      __syncthreads();
-      for (int i = len0 - 1; i >= 0; --i) backward_token(t_begin, i, i);
-    }
-    if (P.d_initial) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4*>(P.d_initial + soff + (size_t)(4 * lane + i) * D + col0) =
-            make_float4(dS[i][0], dS[i][1], dS[i][2], dS[i][3]);
-    }
-    __syncthreads();  // shared partials of this item are read before the next item writes them
+// out[r][c] (+)= f sum_{s} X[r][s] Y[s][c] e^{Gamma_rc - Gamma_sc} over s <= r (X lower triangular as
+// given), per row block I against rho_I = Gamma at the end of block I - 1.
+__device__ void gated_lower(float* s, float* out, const float* X, const float* Y, float f, bool acc, GemmSmem& gsm) {
+  for (int I = 0; I < 4; ++I) {
+    const int ns = 16 * (I + 1);
+    const float* rho = s + SC_G + (16 * I - 1) * D;
+    ew<kB1>(ns * D / 4,
+              [&](int i) {
+                const int c = (4 * i) & (D - 1);
+                const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
+                return mul4(ld4(Y + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + 4 * i))));
+              },
+              [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
+    __syncthreads();
+    gemm(s + SC_L, D, mat(X + 16 * I * C, C), mat(s + SC_R, D), 16, D, ns, 1.f, false, 0, gsm);
+    ew<kB1>(16 * D / 4,
+          [&](int i) {
+            const int c = (4 * i) & (D - 1), e = 16 * I * D + 4 * i;
+            const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
+            float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(ld4(s + SC_G + e), r4))), f);
+            if (acc) v = add4(v, ld4(out + e));
+            return v;
+          },
+          [&](int i, float4 v) { st4(out + 16 * I * D + 4 * i, v); });
+    __syncthreads();
   }
 }
 
-// Per (token, head) row: the slices' partial sums, then the derivatives of the transforms
-// (dq and dk through the L2 norms, dg through the gate, dbeta through the sigmoid).  A CTA takes one
-// head and a run of tokens (one warp per token at a time, a lane per 4 channels) and adds its sums
-// of the gate-parameter gradients with one atomic per value.
+// out[s][c] (+)= f sum_{r >= s} X[r][s] Y[r][c] e^{Gamma_rc - Gamma_sc} (X lower triangular as given),
+// per row block J of s against sigma_J = Gamma at the end of block J.
+__device__ void gated_upper(float* s, float* out, const float* X, const float* Y, float f, bool acc, GemmSmem& gsm) {
+  for (int J = 0; J < 4; ++J) {
+    const int r0 = 16 * J, nr = C - r0;
+    const float* sig = s + SC_G + (16 * J + 15) * D;
+    ew<kB1>(nr * D / 4,
+              [&](int i) {
+                const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
+                return mul4(ld4(Y + e), dexp4(sub4(ld4(s + SC_G + e), ld4(sig + c))));
+              },
+              [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
+    __syncthreads();
+    // (X[r0.., J cols])^T (rows s of block J) times R
+    gemm(s + SC_L, D, mat(X + r0 * C + r0, C, true), mat(s + SC_R, D), 16, D, nr, 1.f, false, 0, gsm);
+    ew<kB1>(16 * D / 4,
+          [&](int i) {
+            const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
+            float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(ld4(sig + c), ld4(s + SC_G + e)))), f);
+            if (acc) v = add4(v, ld4(out + e));
+            return v;
+          },
+          [&](int i, float4 v) { st4(out + r0 * D + 4 * i, v); });
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------- kernels
+__global__ void bwd_chunk_table_kernel(BwdParams P, int32_t* chunk_off) {
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t carry;
+  const FwdParams& p = P.f;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    carry = 0;
+    chunk_off[0] = 0;
+  }
+  bool bad = false;
+  for (int n = tid; n < p.num_seqs; n += 1024) bad |= !seq_entries_ok(p, n);
+  if (__syncthreads_or(bad)) {
+    for (int n = tid; n <= p.num_seqs; n += 1024) chunk_off[n] = 0;
+    if (tid == 0 && p.status) atomicOr(p.status, kStatusBadSeqlens);
+    return;
+  }
+  for (int base = 0; base < p.num_seqs; base += 1024) {
+    const int n = base + tid;
+    int32_t cnt = 0;
+    if (n < p.num_seqs) {
+      int64_t bos, eos;
+      seq_range(p, n, bos, eos);
+      cnt = (int32_t)((eos - bos + C - 1) / C);
+    }
+    int32_t x = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t w = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int32_t incl = carry + x + (warp > 0 ? warp_tot[warp - 1] : 0);
+    if (n < p.num_seqs) chunk_off[n + 1] = incl;
+    __syncthreads();
+    if (tid == 1023) carry = incl;
+    __syncthreads();
+  }
+}
+
+constexpr size_t kChunkSmem = sizeof(GemmSmem) + 2 * 64 * 65 * sizeof(float);
+
+// Per chunk: W, Kt, P^T dO, (Qt - P W)^T dO and e^gamma for the state-gradient walk.
+__global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, int64_t items) {
+  extern __shared__ float4 smem4[];
+  GemmSmem& gsm = *reinterpret_cast<GemmSmem*>(smem4);
+  float* sT = reinterpret_cast<float*>(smem4) + sizeof(GemmSmem) / 4;
+  float* sA = sT + 64 * 65;
+  float* s = P.scratch + (size_t)blockIdx.x * kScratchFloats;
+  const int tid = threadIdx.x;
+  const float scale = P.f.scale;
+  const int64_t n_items = min(items, (int64_t)P.chunk_off[P.f.num_seqs] * P.f.num_heads);
+  for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const Chunk ch = locate(P, it);
+    float* pr = P.prep + (size_t)it * kPrepFloats;
+    chunk_factors(P, ch, s, false, gsm, sT, sA);
+    // W = T_b Kg (to the output); Kt = khat e^{gamma - Gamma}; X = Qt - P W
+    gemm(pr + PR_W, D, mat(s + SC_TB, C), mat(s + SC_KG, D), C, D, C, 1.f, false, 0, gsm);
+    const float* gam = s + SC_G + (C - 1) * D;
+    ew<kB2>(kF4,
+              [&](int i) {
+                const int c = (4 * i) & (D - 1);
+                const float4 G = ld4(s + SC_G + 4 * i);
+                return F4x2{mul4(ld4(s + SC_KH + 4 * i), dexp4(sub4(ld4(gam + c), G))),
+                            scl4(mul4(ld4(s + SC_QH + 4 * i), dexp4(G)), scale)};
+              },
+              [&](int i, F4x2 v) {
+                st4(pr + PR_KT + 4 * i, v.a);
+                st4(s + SC_X + 4 * i, v.b);
+              });
+    if (tid < D) pr[PR_EG + tid] = s[SC_EG + tid];
+    __syncthreads();
+    gemm(s + SC_X, D, mat(s + SC_P, C), mat(pr + PR_W, D), C, D, C, -1.f, true, 0, gsm);
+    gemm(pr + PR_Y, D, mat(s + SC_X, D, true), mat(s + SC_DO, D), D, D, C, 1.f, false, 0, gsm);
+    gemm(pr + PR_PDO, D, mat(s + SC_P, C, true), mat(s + SC_DO, D), C, D, C, 1.f, false, 0, gsm);
+  }
+}
+
+// One CTA per (sequence, head): from the last chunk to the first, with dS' the gradient of the
+// chunk's end state (d_final, or 0, for the last chunk):
+//   E = Kt dS',  dDelta = P^T dO + E,  dS = Diag(e^gamma) dS' + (Qt - P W)^T dO - W^T E.
+// dS' of chunk j is kept in the chunk's slot (the input of bwd_grad_kernel); the dS of chunk 0 is
+// the initial state's gradient.
+__global__ void __launch_bounds__(kBwdThreads) bwd_state_kernel(BwdParams P) {
+  __shared__ GemmSmem gsm;
+  const FwdParams& p = P.f;
+  const int H = p.num_heads;
+  const int n = blockIdx.x / H, h = blockIdx.x - n * H;
+  const int tid = threadIdx.x;
+  int64_t bos, eos;
+  seq_range(p, n, bos, eos);
+  const int64_t c0 = P.chunk_off[n], nch = P.chunk_off[n + 1] - c0;
+  const int64_t slot0 = bos / C + n;
+  float* e_buf = P.scratch + (size_t)blockIdx.x * kF;  // E
+  const float* dfin = P.d_final ? P.d_final + ((size_t)n * H + h) * kStateElems : nullptr;
+  float* d_init = P.d_initial ? P.d_initial + ((size_t)n * H + h) * kStateElems : nullptr;
+  constexpr int kS4 = (int)kStateElems / 4;
+  auto copy_final = [&](float* dst) {
+    ew<kB1>(kS4, [&](int i) { return dfin ? ld4(dfin + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f); },
+              [&](int i, float4 v) { st4(dst + 4 * i, v); });
+  };
+  if (nch == 0) {
+    if (d_init) copy_final(d_init);
+    return;
+  }
+  copy_final(P.dsp + ((size_t)(slot0 + nch - 1) * H + h) * kStateElems);
+  __syncthreads();
+  for (int64_t j = nch - 1; j >= 0; --j) {
+    const int64_t it = (c0 + j) * H + h;
+    const float* pr = P.prep + (size_t)it * kPrepFloats;
+    if (j > 0) {
+      // the previous chunk's factors into L2 while this one runs
+      const char* nx = reinterpret_cast<const char*>(P.prep + (size_t)(it - H) * kPrepFloats);
+      for (int l = tid; l < (int)(kPrepFloats * sizeof(float) / 128); l += kBwdThreads)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + (size_t)l * 128));
+    }
+    const float* dsp = P.dsp + ((size_t)(slot0 + j) * H + h) * kStateElems;
+    float* nxt = j > 0 ? P.dsp + ((size_t)(slot0 + j - 1) * H + h) * kStateElems : d_init;
+    gemm(e_buf, D, mat(pr + PR_KT, D), mat(dsp, D), C, D, D, 1.f, false, 0, gsm);
+    float* dd = P.dd + (size_t)it * kF;
+    ew<kB1>(kF4, [&](int i) { return add4(ld4(pr + PR_PDO + 4 * i), ld4(e_buf + 4 * i)); },
+              [&](int i, float4 v) { st4(dd + 4 * i, v); });
+    if (nxt) {
+      ew<kB1>(kS4,
+                [&](int i) { return add4(scl4(ld4(dsp + 4 * i), pr[PR_EG + ((4 * i) >> 7)]), ld4(pr + PR_Y + 4 * i)); },
+                [&](int i, float4 v) { st4(nxt + 4 * i, v); });
+      __syncthreads();
+      gemm(nxt, D, mat(pr + PR_W, D, true), mat(e_buf, D), D, D, C, -1.f, true, 0, gsm);
+    }
+    __syncthreads();
+  }
+}
+
+// Per chunk: the gradients of khat, qhat, log alpha and beta (to the partial buffers) and dv.
+__global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, int64_t items) {
+  extern __shared__ float4 smem4[];
+  GemmSmem& gsm = *reinterpret_cast<GemmSmem*>(smem4);
+  float* sT = reinterpret_cast<float*>(smem4) + sizeof(GemmSmem) / 4;
+  float* sA = sT + 64 * 65;
+  float* s = P.scratch + (size_t)blockIdx.x * kScratchFloats;
+  const FwdParams& p = P.f;
+  const int H = p.num_heads;
+  const int tid = threadIdx.x;
+  const float scale = p.scale;
+  const int64_t rows_total = (p.cu_seqlens ? p.seqlen : p.seqlen * p.num_seqs) * H;
+  const int64_t n_items = min(items, (int64_t)P.chunk_off[p.num_seqs] * H);
+  for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const Chunk ch = locate(P, it);
+    chunk_factors(P, ch, s, true, gsm, sT, sA);
+    const float* S = P.ckpt + ((size_t)ch.slot * H + ch.h) * kStateElems;   // S^T [v][k]: S(k, v) = S[v * 128 + k]
+    const float* dSp = P.dsp + ((size_t)ch.slot * H + ch.h) * kStateElems;  // [k][v]
+    const float* dD = P.dd + (size_t)it * kF;
+    // W = T_b Kg; Delta = T_b V - W S
+    gemm(s + SC_W, D, mat(s + SC_TB, C), mat(s + SC_KG, D), C, D, C, 1.f, false, 0, gsm);
+    gemm(s + SC_D, D, mat(s + SC_TB, C), mat(s + SC_V, D), C, D, C, 1.f, false, 0, gsm);
+    gemm(s + SC_D, D, mat(s + SC_W, D), mat(S, D, true), C, D, D, -1.f, true, 0, gsm);
+    // dKt = Delta dS'^T;  dQs = dO S^T;  dW = -dDelta S^T;  dP = tril(dO Delta^T)
+    gemm(s + SC_DKT, D, mat(s + SC_D, D), mat(dSp, D, true), C, D, D, 1.f, false, 0, gsm);
+    gemm(s + SC_DQS, D, mat(s + SC_DO, D), mat(S, D), C, D, D, 1.f, false, 0, gsm);
+    gemm(s + SC_DW, D, mat(dD, D), mat(S, D), C, D, D, -1.f, false, 0, gsm);
+    gemm(s + SC_DP, C, mat(s + SC_DO, D), mat(s + SC_D, D, true), C, C, D, 1.f, false, 2, gsm);
+    // dgamma from the state: e^gamma_k sum_v S(k, v) dS'(k, v) (a warp per 16 channels, lanes over v)
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int k = 16 * warp; k < 16 * warp + 16; ++k) {
+        float acc = 0.f;
+#pragma unroll
+        for (int v = lane; v < D; v += 32) acc = fmaf(S[(size_t)v * D + k], dSp[(size_t)k * D + v], acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) s[SC_DGAM + k] = s[SC_EG + k] * acc;
+      }
+    }
+    // dT_b = dDelta V^T + dW Kg^T;  dv = T_b^T dDelta;  dKg = T_b^T dW
+    gemm(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
+    gemm(s + SC_DTB, C, mat(s + SC_DW, D), mat(s + SC_KG, D, true), C, C, D, 1.f, true, 0, gsm);
+    gemm(s + SC_X, D, mat(s + SC_TB, C, true), mat(dD, D), C, D, C, 1.f, false, 0, gsm);
+    ew<kB1>(ch.len * (D / 4), [&](int i) { return ld4(s + SC_X + 4 * i); },
+              [&](int i, float4 v) {
+                const int r = i >> 5, c4 = i & 31;
+                st_bf16x4(P.dv + ((size_t)(ch.t0 + r) * H + ch.h) * D + 4 * c4, v.x, v.y, v.z, v.w);
+              });
+    gemm(s + SC_DKG, D, mat(s + SC_TB, C, true), mat(s + SC_DW, D), C, D, C, 1.f, false, 0, gsm);
+    // dT = dT_b diag(beta); dbeta (columns) = colsum(dT_b o T); dA = strict_tril(-T^T dT T^T)
+    ew<kB1>(kQ4, [&](int i) { return mul4(ld4(s + SC_DTB + 4 * i), ld4(s + SC_BETA + ((4 * i) & (C - 1)))); },
+              [&](int i, float4 v) { st4(s + SC_DA + 4 * i, v); });
+    if (tid < C) {
+      float acc = 0.f;
+#pragma unroll 16
+      for (int r = 0; r < C; ++r) acc = fmaf(s[SC_DTB + r * C + tid], s[SC_T + r * C + tid], acc);
+      s[SC_DB + tid] = acc;
+    }
+    __syncthreads();
+    gemm(s + SC_TMP, C, mat(s + SC_T, C, true), mat(s + SC_DA, C), C, C, C, 1.f, false, 0, gsm);
+    gemm(s + SC_DA, C, mat(s + SC_TMP, C), mat(s + SC_T, C, true), C, C, C, -1.f, false, 1, gsm);
+    // dbeta (rows) += rowsum(dA o M); dM = diag(beta) dA (in place)
+    if (tid < C) {
+      float acc = 0.f;
+#pragma unroll 16
+      for (int c = 0; c < C; ++c) acc = fmaf(s[SC_DA + tid * C + c], s[SC_M + tid * C + c], acc);
+      s[SC_DB + tid] += acc;
+    }
+    __syncthreads();
+    ew<kB1>(kQ4, [&](int i) { return scl4(ld4(s + SC_DA + 4 * i), s[SC_BETA + ((4 * i) >> 6)]); },
+              [&](int i, float4 v) { st4(s + SC_DA + 4 * i, v); });
+    // the decay-weighted products: X1 = gated(dM, khat) and X3 = gated(dP, khat) (rows r), X2 = the
+    // transposed one of dM with khat and X4 = scale x that of dP with qhat (rows s)
+    float* dkh = s + SC_DKG;  // becomes dkhat: e^Gamma dKg first
+    float* dqh = s + SC_DQS;  // becomes dqhat / scale: e^Gamma dO S^T first
+    float* dG = s + SC_W;     // dGamma
+    const float* gam = s + SC_G + (C - 1) * D;
+    ew<kB4>(kF4,
+              [&](int i) {
+                const int c = (4 * i) & (D - 1);
+                const float4 G = ld4(s + SC_G + 4 * i), eG = dexp4(G);
+                const float4 a = mul4(ld4(dkh + 4 * i), eG);                                   // e^Gamma dKg
+                const float4 b = mul4(ld4(s + SC_DKT + 4 * i), dexp4(sub4(ld4(gam + c), G)));  // e^{gamma-Gamma} dKt
+                return F4x4{add4(a, b), mul4(ld4(s + SC_KH + 4 * i), sub4(a, b)), b, mul4(ld4(dqh + 4 * i), eG)};
+              },
+              [&](int i, F4x4 v) {
+                st4(dkh + 4 * i, v.a);
+                st4(dG + 4 * i, v.b);
+                st4(s + SC_DKT + 4 * i, v.c);
+                st4(dqh + 4 * i, v.d);
+              });
+    __syncthreads();
+    gated_lower(s, s + SC_X, s + SC_DA, s + SC_KH, 1.f, false, gsm);  // X1
+    ew<kB2>(kF4,
+              [&](int i) {
+                const float4 x = ld4(s + SC_X + 4 * i);
+                return F4x2{add4(ld4(dkh + 4 * i), x), add4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
+              },
+              [&](int i, F4x2 v) {
+                st4(dkh + 4 * i, v.a);
+                st4(dG + 4 * i, v.b);
+              });
+    __syncthreads();
+    gated_upper(s, s + SC_X, s + SC_DA, s + SC_KH, 1.f, false, gsm);   // X2
+    gated_upper(s, s + SC_X, s + SC_DP, s + SC_QH, scale, true, gsm);  // + X4
+    ew<kB2>(kF4,
+              [&](int i) {
+                const float4 x = ld4(s + SC_X + 4 * i);
+                return F4x2{add4(ld4(dkh + 4 * i), x), sub4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
+              },
+              [&](int i, F4x2 v) {
+                st4(dkh + 4 * i, v.a);
+                st4(dG + 4 * i, v.b);
+              });
+    __syncthreads();
+    gated_lower(s, dqh, s + SC_DP, s + SC_KH, 1.f, true, gsm);  // dqhat / scale
+    // dgamma: the state term plus sum_r khat e^{gamma-Gamma} dKt; then dlog alpha by a reverse running sum
+    if (tid < D) {
+      float acc = s[SC_DGAM + tid];
+#pragma unroll 16
+      for (int r = 0; r < C; ++r) acc = fmaf(s[SC_KH + r * D + tid], s[SC_DKT + r * D + tid], acc);
+      float run = 0.f;
+      for (int r0 = C - 16; r0 >= 0; r0 -= 16) {
+        float col[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const int e = (r0 + r) * D + tid;
+          col[r] = dG[e] + scale * s[SC_QH + e] * dqh[e];
+        }
+#pragma unroll
+        for (int r = 15; r >= 0; --r) {
+          run += col[r];
+          dG[(r0 + r) * D + tid] = run + acc;
+        }
+      }
+    }
+    __syncthreads();
+    // to the partial buffers: dqhat, dkhat, dlog alpha, dbeta
+    float* pq = P.part;
+    float* pk = P.part + (size_t)rows_total * D;
+    float* pa = P.part + 2 * (size_t)rows_total * D;
+    float* pb = P.part + 3 * (size_t)rows_total * D;
+    ew<kB4>(ch.len * (D / 4),
+              [&](int i) { return F4x4{scl4(ld4(dqh + 4 * i), scale), ld4(dkh + 4 * i), ld4(dG + 4 * i), {}}; },
+              [&](int i, F4x4 v) {
+                const int r = i >> 5, c4 = i & 31;
+                const size_t o = ((size_t)(ch.t0 + r) * H + ch.h) * D + 4 * c4;
+                st4(pq + o, v.a);
+                st4(pk + o, v.b);
+                st4(pa + o, v.c);
+              });
+    if (tid < ch.len) pb[(size_t)(ch.t0 + tid) * H + ch.h] = s[SC_DB + tid];
+    __syncthreads();
+  }
+}
+
+// Adds nothing up: applies the derivatives of the transforms to the per-token partials (dq and dk
+// through the L2 norms, dg through the gate, dbeta through the sigmoid).  A CTA takes one head and
+// a run of tokens (one warp per token at a time, a lane per 4 channels) and adds its sums of the
+// gate-parameter gradients with one atomic per value.
 __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t tokens, int tokens_per_cta) {
-  constexpr int D = kHeadDim;
   __shared__ __align__(16) float s_dt[8][D];
   __shared__ float s_dA[8];
   const FwdParams& p = P.f;
@@ -403,18 +874,13 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t to
   const int64_t t_end = min(t_begin + tokens_per_cta, tokens);
   for (int64_t t = t_begin + warp; t < t_end; t += 8) {
     const size_t row = (size_t)t * H + h;
-    float gq[4] = {0.f, 0.f, 0.f, 0.f}, gk[4] = {0.f, 0.f, 0.f, 0.f}, ga[4] = {0.f, 0.f, 0.f, 0.f}, gb = 0.f;
-#pragma unroll
-    for (int sl = 0; sl < kSlices; ++sl) {
-      const float* base = P.part + (size_t)sl * 3 * rows_total * D + row * D + 4 * lane;
-      const float4 a = *reinterpret_cast<const float4*>(base);
-      const float4 b = *reinterpret_cast<const float4*>(base + (size_t)rows_total * D);
-      const float4 c = *reinterpret_cast<const float4*>(base + 2 * (size_t)rows_total * D);
-      gq[0] += a.x; gq[1] += a.y; gq[2] += a.z; gq[3] += a.w;
-      gk[0] += b.x; gk[1] += b.y; gk[2] += b.z; gk[3] += b.w;
-      ga[0] += c.x; ga[1] += c.y; ga[2] += c.z; ga[3] += c.w;
-      gb += P.part[(size_t)kSlices * 3 * rows_total * D + (size_t)sl * rows_total + row];
-    }
+    const float* base = P.part + row * D + 4 * lane;
+    const float4 a4 = *reinterpret_cast<const float4*>(base);
+    const float4 b4 = *reinterpret_cast<const float4*>(base + (size_t)rows_total * D);
+    const float4 c4 = *reinterpret_cast<const float4*>(base + 2 * (size_t)rows_total * D);
+    const float gq[4] = {a4.x, a4.y, a4.z, a4.w}, gk[4] = {b4.x, b4.y, b4.z, b4.w};
+    const float ga[4] = {c4.x, c4.y, c4.z, c4.w};
+    const float gb = P.part[3 * (size_t)rows_total * D + row];
     // dq, dk: (dxhat - xhat (xhat . dxhat)) / n
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
@@ -435,7 +901,8 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t to
       for (int j = 0; j < 4; ++j) r[j] = (gx[j] - (xv[j] / nrm) * dot) / nrm;
       st_bf16x4((which == 0 ? P.dq : P.dk) + row * D + 4 * lane, r[0], r[1], r[2], r[3]);
     }
-    // dg through the gate; the sums for dt_bias and A_log
+    // dg through the gate (log alpha = lower_bound sigmoid(x), x = e^{A_log} (g + dt_bias)); the sums
+    // for dt_bias and A_log
     {
       const float4 g4 = ld_bf16x4(p.g + row * D + 4 * lane);
       const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
@@ -444,8 +911,7 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t to
       for (int j = 0; j < 4; ++j) {
         const float x = ea * (gv[j] + dts[j]);
         const float sg = sigmoid_acc(x);
-        const float al = expf(p.lower_bound * sg);
-        const float dx = ga[j] * al * p.lower_bound * sg * (1.f - sg);
+        const float dx = ga[j] * p.lower_bound * sg * (1.f - sg);
         dg[j] = dx * ea;
         ddt[j] += dg[j];
         dA = fmaf(dx, x, dA);
@@ -475,23 +941,53 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t to
   }
 }
 
-}  // namespace
+size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// At most this many persistent CTAs of the slice kernel (two per SM), so that the workspace size
-// depends only on the problem's sizes.
-constexpr int64_t kBwdMaxCtas = 512;
-constexpr int kFinishTokens = 64;  // tokens per CTA of the finishing kernel
+// Workspace regions (byte offsets), all 256-aligned: the forward's split workspace (its header holds
+// the status word), the checkpoints it writes, the chunk table, prep, dsp, dd, the partials, and the
+// CTA scratch.
+struct BwdLayout {
+  size_t fwd, ckpt, out, table, prep, dsp, dd, part, scratch, total;
+  int64_t chunk_cap;
+};
 
-size_t bwd_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+constexpr int64_t kBwdMaxCtas = 296;  // persistent CTAs of the chunk-parallel kernels (bounds the scratch)
+constexpr int kFinishTokens = 64;     // tokens per CTA of the finishing kernel
+
+BwdLayout bwd_layout(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
   const int64_t t = total_tokens > 0 ? total_tokens : 0, n = num_seqs > 0 ? num_seqs : 0;
   const int64_t hh = num_heads > 0 ? num_heads : 0;
-  const int64_t slots = t / kBwdChunk + n + 1;
-  const int64_t work = n * hh * kSlices;
-  const int64_t ctas = work < kBwdMaxCtas ? work : kBwdMaxCtas;
-  const size_t ckpt = (size_t)slots * hh * kStateElems;
-  const size_t scratch = (size_t)ctas * kBwdChunk * kSliceElems;
-  const size_t part = (size_t)kSlices * (3 * (size_t)t * hh * kHeadDim + (size_t)t * hh);
-  return (ckpt + scratch + part) * sizeof(float);
+  BwdLayout L;
+  L.chunk_cap = t / C + n;  // sum over sequences of ceil(len / 64)
+  const int64_t slots = t / C + n + 1;
+  size_t o = 0;
+  L.fwd = o;
+  o += align256(split_workspace_bytes(t, (int32_t)hh, (int32_t)n));
+  L.ckpt = o;
+  o += align256(checkpoint_bytes(t, (int32_t)hh, (int32_t)n));
+  L.out = o;  // the recomputed forward's output (not used)
+  o += align256((size_t)t * hh * D * sizeof(__nv_bfloat16));
+  L.table = o;
+  o += align256((size_t)(n + 1) * sizeof(int32_t));
+  L.prep = o;
+  o += align256((size_t)L.chunk_cap * hh * kPrepFloats * sizeof(float));
+  L.dsp = o;
+  o += align256((size_t)slots * hh * kStateElems * sizeof(float));
+  L.dd = o;
+  o += align256((size_t)L.chunk_cap * hh * kF * sizeof(float));
+  L.part = o;
+  o += align256((3 * (size_t)t * hh * D + (size_t)t * hh) * sizeof(float));
+  L.scratch = o;  // the chunk-parallel kernels' CTAs, or one E buffer per unit for the state kernel
+  const size_t sc = (size_t)kBwdMaxCtas * kScratchFloats, se = (size_t)(n * hh) * kF;
+  o += align256((sc > se ? sc : se) * sizeof(float));
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(int64_t total_tokens, int32_t num_heads, int32_t num_seqs) {
+  return bwd_layout(total_tokens, num_heads, num_seqs).total;
 }
 
 cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const float* d_final, __nv_bfloat16* dq,
@@ -500,19 +996,19 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
                        cudaStream_t stream) {
   const int64_t units = (int64_t)f.num_seqs * f.num_heads;
   int dev = 0, sms = 0;
-  cudaError_t qe = cudaGetDevice(&dev);
-  if (qe == cudaSuccess) qe = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (qe != cudaSuccess) return qe;
-  cudaError_t e = cudaMemsetAsync(dA_log, 0, sizeof(float) * f.num_heads, stream);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(dA_log, 0, sizeof(float) * f.num_heads, stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(ddt_bias, 0, sizeof(float) * f.num_heads * kHeadDim, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, kWorkspaceHeader, stream);  // status word, counters
   if (e != cudaSuccess || units == 0) return e;
   const int64_t tokens = f.cu_seqlens ? f.seqlen : f.seqlen * f.num_seqs;
-  const int64_t slots = tokens / kBwdChunk + f.num_seqs + 1;
-  const int64_t work = units * kSlices;
-  int64_t grid = work < 2 * (int64_t)sms ? work : 2 * (int64_t)sms;
-  if (grid > kBwdMaxCtas) grid = kBwdMaxCtas;
+  const BwdLayout L = bwd_layout(tokens, f.num_heads, f.num_seqs);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   BwdParams P;
   P.f = f;
+  P.f.status = reinterpret_cast<uint32_t*>(ws + L.fwd);
   P.d_out = d_out;
   P.d_final = d_final;
   P.dq = dq;
@@ -523,20 +1019,46 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
   P.dA_log = dA_log;
   P.ddt_bias = ddt_bias;
   P.d_initial = d_initial;
-  P.ckpt_in = checkpoints;
-  P.ckpt = static_cast<float*>(workspace);
-  P.scratch = P.ckpt + (size_t)slots * f.num_heads * kStateElems;
-  const int64_t work_cap = work < kBwdMaxCtas ? work : kBwdMaxCtas;
-  P.part = P.scratch + (size_t)work_cap * kBwdChunk * kSliceElems;
-  const size_t smem = sizeof(ChunkIn) + (2 * 8 * 3 * kHeadDim + 2 * 8) * sizeof(float);
+  P.chunk_off = reinterpret_cast<int32_t*>(ws + L.table);
+  P.prep = reinterpret_cast<float*>(ws + L.prep);
+  P.dsp = reinterpret_cast<float*>(ws + L.dsp);
+  P.dd = reinterpret_cast<float*>(ws + L.dd);
+  P.part = reinterpret_cast<float*>(ws + L.part);
+  P.scratch = reinterpret_cast<float*>(ws + L.scratch);
+  if (checkpoints || tokens == 0) {
+    P.ckpt = checkpoints;
+  } else {
+    // the forward, storing the chunk-start states (its outputs are not needed)
+    float* ck = reinterpret_cast<float*>(ws + L.ckpt);
+    FwdParams ff = P.f;
+    ff.out = reinterpret_cast<__nv_bfloat16*>(ws + L.out);
+    ff.final_state = nullptr;
+    if ((e = launch_split(ff, ws + L.fwd, stream, ck)) != cudaSuccess) return e;
+    P.ckpt = ck;
+  }
+  bwd_chunk_table_kernel<<<1, 1024, 0, stream>>>(P, const_cast<int32_t*>(P.chunk_off));
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t items = L.chunk_cap * f.num_heads;  // an upper bound; items past the last chunk are skipped
   static bool attr_done[64] = {};
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if ((e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChunkSmem)) !=
+            cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChunkSmem)) !=
+            cudaSuccess)
       return e;
     attr_done[dev] = true;
   }
-  bwd_kernel<<<(unsigned)grid, kBwdThreads, smem, stream>>>(P);
+  int64_t grid = 2 * (int64_t)sms;
+  if (grid > kBwdMaxCtas) grid = kBwdMaxCtas;
+  if (grid > items) grid = items;
+  if (tokens > 0) {
+    bwd_prep_kernel<<<(unsigned)grid, kBwdThreads, kChunkSmem, stream>>>(P, items);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  bwd_state_kernel<<<(unsigned)units, kBwdThreads, 0, stream>>>(P);  // also when every document is empty
   if ((e = cudaGetLastError()) != cudaSuccess || tokens == 0) return e;
+  bwd_grad_kernel<<<(unsigned)grid, kBwdThreads, kChunkSmem, stream>>>(P, items);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const dim3 fgrid((unsigned)((tokens + kFinishTokens - 1) / kFinishTokens), (unsigned)f.num_heads);
   bwd_finish_kernel<<<fgrid, 256, 0, stream>>>(P, tokens, kFinishTokens);
   return cudaGetLastError();

@@ -149,8 +149,9 @@ constexpr uint32_t I_RK = 16384;    // k tile (TMA); becomes QB once k sits in r
 constexpr uint32_t I_XK = 0;        // -Khat e^Gamma (pre-scaled to the chunk start), MN tile, B of MMA Xk
 constexpr uint32_t I_QB = 16384;    // Qtil, MN tile, B of the MMA that seeds [0; Qtil]
 constexpr uint32_t I_LKQ = 32768;   // [LK; LQ] K tile, 128 rows (A of MMA AP)
-constexpr uint32_t I_R = 65536;     // R_0..R_3 K tile, 160 rows (B of MMA AP)
-constexpr uint32_t I_RKBLK = 160 * 128;
+constexpr uint32_t I_R = 65536;     // R_1..R_3 K tile, 144 rows (B of MMA AP)
+constexpr uint32_t kRRows = 144;
+constexpr uint32_t I_RKBLK = kRRows * 128;
 constexpr uint32_t I_TP = 32768;    // after MMA AP: [T_b hi; P -> (P T_b) hi], 128 rows x 64
 constexpr uint32_t I_TL = 49152;    //               [T_b lo; (P T_b) lo]
 constexpr uint32_t I_AS = 65536;    //               A fp32 64 x 68 (then, over AS and TS, the
@@ -170,6 +171,12 @@ static_assert(I_YS + 4096 <= I_SC, "intra shared-memory map");
 static_assert(2 * (I_ALLOC + 1024) <= 233472, "two intra CTAs per SM");
 constexpr uint32_t kIntraTmemCols = 256;
 constexpr uint32_t kIdCol = 192;  // [0; I_64] as bf16 (32 columns), A of the MMA that seeds [0; Qtil]
+// Row of the R tile where the right operand of row block I starts.  Row block I >= 1 refers its
+// Gram entries to the decays at its own start, so R_I holds rows 0 .. 16 I + 15 of Khat scaled to
+// that reference; row block 0 refers to the start of block 1 (its left factors then lie in
+// [1, e^{80}], its right ones in [e^{-80}, 1]) and shares R_1.
+__host__ __device__ constexpr uint32_t r_seg(int I) { return I <= 1 ? 0u : 8u * I * (I + 1) - 16u; }
+static_assert(r_seg(3) + 64 == kRRows, "R tile rows");
 
 struct IntraMaps {
   CUtensorMap q, k, g;
@@ -186,8 +193,8 @@ __device__ __forceinline__ uint32_t bf16x2_of(float2 v) { return bf16x2(v.x, v.y
 // Per item (8 warps; warp iw owns rows 8 iw .. + 7 in the element-wise phases):
 //   prologue  norms, sigmoid(beta), the gate, per-warp decay products (q read, k kept in registers)
 //   pass 1    [LK; LQ] (Gram left operand), XK = -Khat e^Gamma and QB = Qtil (q read again)
-//   pass 2    R_0..R_3 (Gram right operand, one decay reference per row block) and Ktil (to the item)
-//   MMA AP    [LK; LQ] R^T (N = 160) -> assembly of A (fp32) and P (bf16)
+//   pass 2    R_1..R_3 (Gram right operand, one decay reference per row block) and Ktil (to the item)
+//   MMA AP    [LK; LQ] R^T (N = 144) -> assembly of A (fp32) and P (bf16)
 //   solve     diagonal 16 x 16 blocks by substitution (warps 0 and 5, which assembled them), then
 //             the off-diagonal blocks column by column on 3xTF32 mma.sync, warp-local levels
 //   T_b       hi + lo split; MMA PT: P T_b (hi + lo), read back as a hi + lo pair
@@ -292,7 +299,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
   const uint32_t a_r = sbase + I_R + kb * I_RKBLK;
   // matrix descriptors of the MMA operand tiles (thread 0 issues; k-steps are offsets)
   const uint64_t d_lkq = sdesc_sw128(sbase + I_LKQ, 16, 1024);   // K-major, 128 rows
-  const uint64_t d_r = sdesc_sw128(sbase + I_R, 16, 1024);       // K-major, 160 rows
+  const uint64_t d_r = sdesc_sw128(sbase + I_R, 16, 1024);       // K-major, 144 rows
   const uint64_t d_tpk = sdesc_sw128(sbase + I_TP, 16, 1024);    // [T; P] / [T; PT] as K-major A
   const uint64_t d_tlk = sdesc_sw128(sbase + I_TL, 16, 1024);
   const uint64_t d_tpm = sdesc_sw128(sbase + I_TP, 8192, 1024);  // T_b hi / lo as MN-major B
@@ -504,13 +511,26 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       }
     }
 
-    // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i.  XK is
+    // pass 1, rows ascending: e_i = prod of alpha from the sub-block start to row i.  Rows of
+    // sub-block J >= 1 refer to its start, rows of sub-block 0 to the start of sub-block 1 (e_i / b_0);
+    // XK = -Khat e^Gamma and QB = Qtil refer to the chunk start, where pre takes them.  XK is
     // written negated, so that MMA Xk subtracts [W; P W] from the [0; Qtil] it starts from
     {
-      const float2 npre[2] = {make_float2(-pre[0].x, -pre[0].y), make_float2(-pre[1].x, -pre[1].y)};
       float2 run[2];
 #pragma unroll
       for (int m = 0; m < 2; ++m) run[m] = upper_half ? pt[m] : make_float2(1.f, 1.f);
+      if (blk == 0) {
+        const float4 t0v = reinterpret_cast<const float4*>(sc_tot)[lane];
+        const float4 t1v = reinterpret_cast<const float4*>(sc_tot + 128)[lane];
+        const float2 b0[2] = {mul2(make_float2(t0v.x, t0v.y), make_float2(t1v.x, t1v.y)),
+                              mul2(make_float2(t0v.z, t0v.w), make_float2(t1v.z, t1v.w))};
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          run[m] = mul2(run[m], make_float2(1.0f / b0[m].x, 1.0f / b0[m].y));
+          pre[m] = b0[m];
+        }
+      }
+      const float2 npre[2] = {make_float2(-pre[0].x, -pre[0].y), make_float2(-pre[1].x, -pre[1].y)};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint2 qri = (8 * iw + i < len) ? lds64(a_rq + xo(i)) : make_uint2(0, 0);
@@ -534,13 +554,14 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     }
     // pass 2, rows descending: f_i = prod of alpha after row i to the sub-block end; Ktil goes
     // straight to the item (same swizzled image as a shared-memory MN tile).  Specialised on the
-    // warp's row block B, which writes R_B .. R_3
+    // warp's row block B, which writes R_max(B,1) .. R_3
     {
       float2 bJ[4][2];
       load_bJ(bJ);
       uint8_t* kt_dst = item + IT_KT + kb * 8192;
       auto pass2 = [&](auto nb) {
         constexpr int B = decltype(nb)::value;
+        constexpr int I0 = B < 1 ? 1 : B;
         float2 post[2], cI[4][2];
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
@@ -548,7 +569,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 #pragma unroll
           for (int J = B + 1; J < 4; ++J) z = mul2(z, bJ[J][m]);
           post[m] = z;
-          cI[B][m] = make_float2(1.0f / bJ[B][m].x, 1.0f / bJ[B][m].y);
+          if (B >= 1) cI[B][m] = make_float2(1.0f / bJ[B][m].x, 1.0f / bJ[B][m].y);
           float2 mm = make_float2(1.f, 1.f);
 #pragma unroll
           for (int I = B + 1; I < 4; ++I) {
@@ -570,8 +591,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
             kf[m] = mul2(kr_f[m], ik);      // khat * f
           }
 #pragma unroll
-          for (int I = B; I < 4; ++I)
-            sts64(a_r + row_off(I) * 128 + xo(i), bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
+          for (int I = I0; I < 4; ++I)
+            sts64(a_r + r_seg(I) * 128 + xo(i), bf16x2_of(mul2(kf[0], cI[I][0])), bf16x2_of(mul2(kf[1], cI[I][1])));
           *reinterpret_cast<uint2*>(kt_dst + xo(i)) =
               make_uint2(bf16x2_of(mul2(kr_f[0], post[0])), bf16x2_of(mul2(kr_f[1], post[1])));
 #pragma unroll
@@ -591,8 +612,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
     // ================================================================ MMA AP: [LK; LQ] x R_I^T
     if (itid == 0) {
       tc_fence_after();
-      // the four right operands R_0..R_3 are consecutive rows of one tile: a single N = 160 product
-      constexpr uint32_t idesc = idesc_bf16(128, 160, false, false);
+      // the right operands R_1..R_3 are consecutive rows of one tile: a single N = 144 product
+      constexpr uint32_t idesc = idesc_bf16(128, kRRows, false, false);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t ad = sdesc_add(d_lkq, (ks >> 2) * 16384 + (ks & 3) * 32);
@@ -613,10 +634,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
       const int q2 = quarter & 1;
       const bool skip = (ihalf == 1) && (q2 == 0);
       float d[32];
-      if (!skip) {
+      if (!skip && q2 == 0) {
+        tmem_ld32(tmem + lane_base + 32 * ihalf, d);  // row blocks 0 and 1 share R_1
+      } else if (!skip) {
         float d0[32], d1[32];
-        tmem_ld32(tmem + lane_base + row_off(2 * q2) + 32 * ihalf, d0);
-        tmem_ld32(tmem + lane_base + row_off(2 * q2 + 1) + 32 * ihalf, d1);
+        tmem_ld32(tmem + lane_base + r_seg(2) + 32 * ihalf, d0);
+        tmem_ld32(tmem + lane_base + r_seg(3) + 32 * ihalf, d1);
         const bool odd = Ib & 1;
 #pragma unroll
         for (int j = 0; j < 32; ++j) d[j] = odd ? d1[j] : d0[j];

@@ -116,3 +116,34 @@ def test_forward_checkpoints_are_chunk_start_states(cuda_device):
             got = np.swapaxes(ck[slot], -1, -2)
             err = rel_l2(got, s_ref[0])
             assert np.isfinite(got).all() and err <= 1e-2, (n, c, err)
+
+
+def test_bwd_long_sequence_few_heads(cuda_device):
+    """One 3000-token sequence over 2 heads: 47 chunks per (sequence, head), so the state gradient
+    crosses many chunk boundaries while the chunk-parallel kernels take the chunks side by side."""
+    x = kda_inputs.make_random("t", [3000], 2, seed=117, state_std=0.2)
+    x.g[:, :, :, 64:].fill_(-6.0)  # half the channels decay slowly
+    check_grads(*run_case(cuda_device, x, 6), "3000 tokens x 2 heads")
+
+
+def test_bwd_saturated_gates_and_empty_documents(cuda_device):
+    """Gates at the lower bound (raw gate 60: log alpha = -5 in every channel) and empty documents
+    between non-empty ones: the decay-weighted products then span e^{-80} .. e^{80} per sub-block."""
+    x = kda_inputs.make_random("t", [0, 150, 0, 0, 77], 2, seed=118, state_std=0.2)
+    x.g[:, :, 0, :].fill_(60.0)
+    check_grads(*run_case(cuda_device, x, 7), "saturated gate, empty documents")
+
+
+def test_bwd_malformed_offsets_report_and_pass_the_state_gradient_through(cuda_device):
+    """Out-of-order cu_seqlens: every document is empty, d_initial = d_final and the workspace's
+    status word says so."""
+    x = kda_inputs.make_random("t", [100, 200, 50], 2, seed=119, state_std=0.1).to(cuda_device)
+    cu_bad = torch.tensor([0, 200, 100, 350], dtype=torch.int32, device=cuda_device)
+    d_out = torch.randn(x.v.shape, device=cuda_device).to(torch.bfloat16)
+    d_final = torch.randn(3, 2, 128, 128, device=cuda_device)
+    ws = torch.empty(kda.bwd_workspace_size(350, 2, 3), dtype=torch.uint8, device=cuda_device)
+    got = kda.bwd(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, d_out,
+                  initial_state=x.initial_state, d_final=d_final, cu_seqlens=cu_bad, workspace=ws)
+    assert kda.read_device_status(ws) == 1
+    assert torch.equal(got["d_initial"], d_final)
+    assert torch.count_nonzero(got["dA_log"]) == 0 and torch.count_nonzero(got["ddt_bias"]) == 0
