@@ -31,6 +31,7 @@
 // kernels are persistent; each CTA keeps one chunk's intermediates in its own global scratch, which
 // stays in L2.  Arithmetic is fp32 on CUDA cores throughout.
 #include "kda_common.cuh"
+#include "sm100.cuh"
 
 namespace kda {
 namespace {
@@ -106,120 +107,158 @@ struct Mat {
 __device__ __forceinline__ Mat mat(const float* p, int ld, bool t = false) { return Mat{p, ld, t}; }
 
 constexpr int GB_K = 64;   // depth of one staged slice
+// Shared-memory rows padded by 8 floats, so that the tensor-core fragment reads (lane (g, t) reads
+// row k0 + t, column g) fall in 32 distinct banks.
+constexpr int SA_LD = 64 + 8, SB_LD = 128 + 8;
 struct GemmSmem {
-  float a[GB_K][64];
-  float b[GB_K][128];
+  float a[GB_K][SA_LD];
+  float b[GB_K][SB_LD];
 };
 
-// Loads the GB_K x W slice (k0.., i0..) of an operand into s[k][i] (zero outside rows x depth),
-// element (i, k) being p[k * ld + i] (memory along i) or p[i * ld + k] (kmaj: memory along k, the
-// slice transposed on the way in).
+// The GB_K x W slice (k0.., i0..) of an operand, element (i, k) being p[k * ld + i] (memory along
+// i) or p[i * ld + k] (kmaj: memory along k, transposed into s[k][i]), zero outside rows x depth:
+// fetched into registers, then put into shared memory as s[k][i].  A GEMM fetches both operands'
+// slices before it puts either, so that all of a thread's loads are in flight together (through
+// generic pointers the compiler would keep each shared-memory store ahead of the next load).
 template <int W>
-__device__ __forceinline__ void gemm_load(float (*s)[W], const float* p, int ld, bool kmaj, int i0, int k0, int rows,
-                                          int depth) {
+struct Slice {
+  static constexpr int kVec = GB_K * W / 4;  // float4s in the slice
+  static constexpr int kPer = (kVec + kBwdThreads - 1) / kBwdThreads;
+  float4 v[kPer];
+};
+
+template <int W>
+__device__ __forceinline__ void slice_fetch(Slice<W>& r, const float* p, int ld, bool kmaj, int i0, int k0, int rows,
+                                            int depth) {
+  constexpr int kVec = Slice<W>::kVec, kPer = Slice<W>::kPer;
   const int tid = threadIdx.x;
-  constexpr int kVec = GB_K * W / 4;  // float4s in the slice
-  if (!kmaj) {
 #pragma unroll
-    for (int e = 0; e < (kVec + kBwdThreads - 1) / kBwdThreads; ++e) {
-      const int idx = tid + e * kBwdThreads;
-      if (kVec % kBwdThreads != 0 && idx >= kVec) break;
+  for (int e = 0; e < kPer; ++e) {
+    const int idx = tid + e * kBwdThreads;
+    r.v[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (kVec % kBwdThreads != 0 && idx >= kVec) continue;
+    if (!kmaj) {
       const int i4 = idx % (W / 4), k = idx / (W / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (k0 + k < depth && i0 + 4 * i4 < rows)
-        v = *reinterpret_cast<const float4*>(p + (size_t)(k0 + k) * ld + i0 + 4 * i4);
-      *reinterpret_cast<float4*>(&s[k][4 * i4]) = v;
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < (kVec + kBwdThreads - 1) / kBwdThreads; ++e) {
-      const int idx = tid + e * kBwdThreads;
-      if (kVec % kBwdThreads != 0 && idx >= kVec) break;
+        r.v[e] = *reinterpret_cast<const float4*>(p + (size_t)(k0 + k) * ld + i0 + 4 * i4);
+    } else {
       const int i = idx % W, k4 = idx / W;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (i0 + i < rows && k0 + 4 * k4 < depth)
-        v = *reinterpret_cast<const float4*>(p + (size_t)(i0 + i) * ld + k0 + 4 * k4);
-      s[4 * k4 + 0][i] = v.x;
-      s[4 * k4 + 1][i] = v.y;
-      s[4 * k4 + 2][i] = v.z;
-      s[4 * k4 + 3][i] = v.w;
+        r.v[e] = *reinterpret_cast<const float4*>(p + (size_t)(i0 + i) * ld + k0 + 4 * k4);
+    }
+  }
+}
+
+template <int W, int LD>
+__device__ __forceinline__ void slice_put(float (*s)[LD], const Slice<W>& r, bool kmaj) {
+  constexpr int kVec = Slice<W>::kVec, kPer = Slice<W>::kPer;
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int idx = tid + e * kBwdThreads;
+    if (kVec % kBwdThreads != 0 && idx >= kVec) continue;
+    if (!kmaj) {
+      const int i4 = idx % (W / 4), k = idx / (W / 4);
+      *reinterpret_cast<float4*>(&s[k][4 * i4]) = r.v[e];
+    } else {
+      const int i = idx % W, k4 = idx / W;
+      s[4 * k4 + 0][i] = r.v[e].x;
+      s[4 * k4 + 1][i] = r.v[e].y;
+      s[4 * k4 + 2][i] = r.v[e].z;
+      s[4 * k4 + 3][i] = r.v[e].w;
     }
   }
 }
 
 // C[i][j] = alpha sum_k A(i, k) B(k, j) (+ C[i][j] when acc), i < M, j < N; mask 1 keeps j < i,
-// mask 2 keeps j <= i (the rest is written as 0).  Output tiles of (16 RM) x 128: thread (ty, tx)
-// holds rows RM ty .. + RM - 1 and columns 4 tx .. + 3 and 64 + 4 tx .. + 3 (conflict-free
-// 16-byte reads of the B slice).  M, N, K multiples of 4; operands 16-byte aligned with ld a
-// multiple of 4.  All threads of the CTA call it; it ends with a barrier.
+// mask 2 keeps j <= i (the rest is written as 0).  Output tiles of (16 RM) x 128 on the tensor cores:
+// mma.sync m16n8k8 with tf32 operands, each operand split into a high and a low tf32 part and the
+// three products hi hi, hi lo, lo hi accumulated in fp32 (about 2^-20 relative: fp32-level).  With
+// RM = 4 warp (wm, wn) holds rows 32 wm .. + 31 and columns 32 wn .. + 31 (2 x 4 fragments), with
+// RM = 1 warp w columns 16 w .. + 15 (1 x 2).  M, N, K multiples of 4 (K of 8 inside a slice);
+// operands 16-byte aligned with ld a multiple of 4.  All threads of the CTA call it; it ends with a
+// barrier.
 template <int RM>
 __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc, int mask,
                        GemmSmem& sm) {
   constexpr int BM = 16 * RM;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  float (*sa)[BM] = reinterpret_cast<float (*)[BM]>(&sm.a[0][0]);
+  constexpr int LDA = BM + 8;  // 72 or 24: (LDA t + g) mod 32 distinct over the lanes
+  constexpr int MT = RM == 4 ? 2 : 1, NT = RM == 4 ? 4 : 2;  // fragments per warp
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int wm = RM == 4 ? (warp & 1) : 0, wn = RM == 4 ? (warp >> 1) : warp;
+  const int row0 = RM == 4 ? 32 * wm : 0, col0 = RM == 4 ? 32 * wn : 16 * wn;
+  float (*sa)[LDA] = reinterpret_cast<float (*)[LDA]>(&sm.a[0][0]);
   for (int i0 = 0; i0 < M; i0 += BM) {
     for (int j0 = 0; j0 < N; j0 += 128) {
-      float c[RM][8];
+      float c[MT][NT][4];
 #pragma unroll
-      for (int a = 0; a < RM; ++a)
+      for (int a = 0; a < MT; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) c[a][b] = 0.f;
+        for (int b = 0; b < NT; ++b)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c[a][b][e] = 0.f;
       for (int k0 = 0; k0 < K; k0 += GB_K) {
         // A(i, k): memory along k when not transposed; B(k, j): memory along j when not transposed
-        gemm_load<BM>(sa, A.p, A.ld, !A.t, i0, k0, M, K);
-        gemm_load<128>(sm.b, B.p, B.ld, B.t, j0, k0, N, K);
+        {
+          Slice<BM> ra;
+          Slice<128> rb;
+          slice_fetch<BM>(ra, A.p, A.ld, !A.t, i0, k0, M, K);
+          slice_fetch<128>(rb, B.p, B.ld, B.t, j0, k0, N, K);
+          slice_put<BM, LDA>(sa, ra, !A.t);
+          slice_put<128, SB_LD>(sm.b, rb, B.t);
+        }
         __syncthreads();
         const int kn = K - k0 < GB_K ? K - k0 : GB_K;
-#pragma unroll 4
-        for (int k = 0; k < kn; ++k) {
-          float ar[RM];
-          if constexpr (RM == 4) {
-            const float4 av = *reinterpret_cast<const float4*>(&sa[k][4 * ty]);
-            ar[0] = av.x;
-            ar[1] = av.y;
-            ar[2] = av.z;
-            ar[3] = av.w;
-          } else {
+        for (int kk = 0; kk < kn; kk += 8) {
+          uint32_t ah[MT][4], al[MT][4];
 #pragma unroll
-            for (int a = 0; a < RM; ++a) ar[a] = sa[k][RM * ty + a];
+          for (int a = 0; a < MT; ++a) {
+            const int r = row0 + 16 * a + g;
+            sm100::tf32_split(sa[kk + t][r], ah[a][0], al[a][0]);
+            sm100::tf32_split(sa[kk + t][r + 8], ah[a][1], al[a][1]);
+            sm100::tf32_split(sa[kk + t + 4][r], ah[a][2], al[a][2]);
+            sm100::tf32_split(sa[kk + t + 4][r + 8], ah[a][3], al[a][3]);
           }
-          const float4 b0 = *reinterpret_cast<const float4*>(&sm.b[k][4 * tx]);
-          const float4 b1 = *reinterpret_cast<const float4*>(&sm.b[k][64 + 4 * tx]);
-          const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-          for (int a = 0; a < RM; ++a)
+          for (int b = 0; b < NT; ++b) {
+            const int n = col0 + 8 * b + g;
+            uint32_t bh0, bl0, bh1, bl1;
+            sm100::tf32_split(sm.b[kk + t][n], bh0, bl0);
+            sm100::tf32_split(sm.b[kk + t + 4][n], bh1, bl1);
 #pragma unroll
-            for (int b = 0; b < 8; ++b) c[a][b] = fmaf(ar[a], br[b], c[a][b]);
+            for (int a = 0; a < MT; ++a) {
+              sm100::mma_tf32(c[a][b], ah[a], bl0, bl1);
+              sm100::mma_tf32(c[a][b], al[a], bh0, bh1);
+              sm100::mma_tf32(c[a][b], ah[a], bh0, bh1);
+            }
+          }
         }
         __syncthreads();
       }
 #pragma unroll
-      for (int a = 0; a < RM; ++a) {
-        const int i = i0 + RM * ty + a;
-        if (i >= M) continue;
+      for (int a = 0; a < MT; ++a) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int j = j0 + 64 * hf + 4 * tx;
-          if (j >= N) continue;
-          float4* dst = reinterpret_cast<float4*>(Cp + (size_t)i * ldc + j);
-          float4 o = make_float4(alpha * c[a][4 * hf], alpha * c[a][4 * hf + 1], alpha * c[a][4 * hf + 2],
-                                 alpha * c[a][4 * hf + 3]);
-          if (acc) {
-            const float4 old = *dst;
-            o.x += old.x;
-            o.y += old.y;
-            o.z += old.z;
-            o.w += old.w;
+        for (int hr = 0; hr < 2; ++hr) {
+          const int i = i0 + row0 + 16 * a + g + 8 * hr;
+          if (i >= M) continue;
+#pragma unroll
+          for (int b = 0; b < NT; ++b) {
+            const int j = j0 + col0 + 8 * b + 2 * t;
+            if (j >= N) continue;
+            float2* dst = reinterpret_cast<float2*>(Cp + (size_t)i * ldc + j);
+            float2 o = make_float2(alpha * c[a][b][2 * hr], alpha * c[a][b][2 * hr + 1]);
+            if (acc) {
+              const float2 old = *dst;
+              o.x += old.x;
+              o.y += old.y;
+            }
+            if (mask) {
+              const int lim = mask == 1 ? i : i + 1;  // keep j < lim
+              if (j + 0 >= lim) o.x = 0.f;
+              if (j + 1 >= lim) o.y = 0.f;
+            }
+            *dst = o;
           }
-          if (mask) {
-            const int lim = mask == 1 ? i : i + 1;  // keep j < lim
-            if (j + 0 >= lim) o.x = 0.f;
-            if (j + 1 >= lim) o.y = 0.f;
-            if (j + 2 >= lim) o.z = 0.f;
-            if (j + 3 >= lim) o.w = 0.f;
-          }
-          *dst = o;
         }
       }
     }
@@ -380,68 +419,67 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   __syncthreads();
   ew<kB1>(kF4, [&](int i) { return mul4(ld4(s + SC_KH + 4 * i), dexp4(ld4(s + SC_G + 4 * i))); },
             [&](int i, float4 v) { st4(s + SC_KG + 4 * i, v); });
-  // M and P per row block I: (Y_r e^{Gamma_r - rho_I}) (khat_s e^{rho_I - Gamma_s})^T, rho_I = Gamma at
-  // the end of block I - 1 (0 for I = 0)
-  for (int I = 0; I < 4; ++I) {
-    const int ns = 16 * (I + 1);
-    const float* rho = s + SC_G + (16 * I - 1) * D;
-    ew<kB1>(ns * D / 4,
-              [&](int i) {
-                const int c = (4 * i) & (D - 1);
-                const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-                return mul4(ld4(s + SC_KH + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + 4 * i))));
-              },
-              [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
-    ew<kB2>(16 * D / 4,
+  // M and P: row r of block I = r / 16 takes khat_r e^{Gamma_r - rho_I} (qhat_r for P) against the
+  // rows s < 16 (I + 1) of R_I = khat_s e^{rho_I - Gamma_s}, rho_I = Gamma at the end of block I - 1
+  // (0 for I = 0).  One product [LK; LQ] (128 x 128) R_all^T, R_all the four R_I stacked (160 rows,
+  // R_I from row 8 I (I + 1)), of which each row keeps its own block's segment.
+  {
+    float* GL = s + SC_W;    // [LK; LQ]: 128 x 128
+    float* GR = s + SC_DKT;  // R_all: 160 x 128
+    float* GO = s + SC_DKG;  // [LK; LQ] R_all^T: 128 x 160
+    ew<kB1>(2 * kF4,
+            [&](int i) {
+              const int e = (4 * i) & (kF - 1), r = e >> 7, c = e & (D - 1), I = r >> 4;
+              const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(s + SC_G + (16 * I - 1) * D + c);
+              const float4 x = ld4(s + (4 * i < kF ? SC_KH : SC_QH) + e);
+              return mul4(x, dexp4(sub4(ld4(s + SC_G + e), r4)));
+            },
+            [&](int i, float4 v) { st4(GL + 4 * i, v); });
+    ew<kB1>(160 * D / 4,
+            [&](int i) {
+              const int q = (4 * i) >> 7, c = (4 * i) & (D - 1);
+              const int I = q < 16 ? 0 : (q < 48 ? 1 : (q < 96 ? 2 : 3)), srow = q - 8 * I * (I + 1);
+              const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(s + SC_G + (16 * I - 1) * D + c);
+              return mul4(ld4(s + SC_KH + srow * D + c), dexp4(sub4(r4, ld4(s + SC_G + srow * D + c))));
+            },
+            [&](int i, float4 v) { st4(GR + 4 * i, v); });
+    __syncthreads();
+    gemm(GO, 160, mat(GL, D), mat(GR, D, true), 2 * C, 160, D, 1.f, false, 0, gsm);
+  }
+  // M strictly lower, P (times scale) lower with its diagonal, each row from its block's segment
+  ew<kB2>(kQ4,
           [&](int i) {
-            const int c = (4 * i) & (D - 1), e = 16 * I * D + 4 * i;
-            const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-            const float4 f = dexp4(sub4(ld4(s + SC_G + e), r4));
-            return F4x2{mul4(ld4(s + SC_KH + e), f), mul4(ld4(s + SC_QH + e), f)};
+            const int r = (4 * i) >> 6, c = (4 * i) & (C - 1), I = r >> 4;
+            float4 m = make_float4(0.f, 0.f, 0.f, 0.f), q = m;
+            if (c < 16 * (I + 1)) {
+              const float* go = s + SC_DKG + r * 160 + 8 * I * (I + 1) + c;
+              m = ld4(go);
+              q = scl4(ld4(go + 64 * 160), p.scale);
+            }
+            if (c + 0 >= r) m.x = 0.f;
+            if (c + 1 >= r) m.y = 0.f;
+            if (c + 2 >= r) m.z = 0.f;
+            if (c + 3 >= r) m.w = 0.f;
+            if (c + 0 > r) q.x = 0.f;
+            if (c + 1 > r) q.y = 0.f;
+            if (c + 2 > r) q.z = 0.f;
+            if (c + 3 > r) q.w = 0.f;
+            return F4x2{m, q};
           },
           [&](int i, F4x2 v) {
-            st4(s + SC_L + 4 * i, v.a);
-            st4(s + SC_L + 16 * D + 4 * i, v.b);
+            st4(s + SC_M + 4 * i, v.a);
+            st4(s + SC_P + 4 * i, v.b);
+            const int r = (4 * i) >> 6, c = (4 * i) & (C - 1);
+            const float b = s[SC_BETA + r];
+            sA[r * 65 + c] = b * v.a.x;
+            sA[r * 65 + c + 1] = b * v.a.y;
+            sA[r * 65 + c + 2] = b * v.a.z;
+            sA[r * 65 + c + 3] = b * v.a.w;
+            sT[r * 65 + c] = 0.f;
+            sT[r * 65 + c + 1] = 0.f;
+            sT[r * 65 + c + 2] = 0.f;
+            sT[r * 65 + c + 3] = 0.f;
           });
-    __syncthreads();
-    gemm(s + SC_M + 16 * I * C, C, mat(s + SC_L, D), mat(s + SC_R, D, true), 16, ns, D, 1.f, false, 0, gsm);
-    gemm(s + SC_P + 16 * I * C, C, mat(s + SC_L + 16 * D, D), mat(s + SC_R, D, true), 16, ns, D, p.scale, false, 0,
-         gsm);
-  }
-  // M strictly lower, P lower with its diagonal: the entries right of each block's segment are zero
-  ew<kB2>(kQ4,
-            [&](int i) {
-              const int r = (4 * i) >> 6, c = (4 * i) & (C - 1);
-              const int ns = 16 * ((r >> 4) + 1);
-              float4 m = make_float4(0.f, 0.f, 0.f, 0.f), q = m;
-              if (c < ns) {
-                m = ld4(s + SC_M + 4 * i);
-                q = ld4(s + SC_P + 4 * i);
-              }
-              if (c + 0 >= r) m.x = 0.f;
-              if (c + 1 >= r) m.y = 0.f;
-              if (c + 2 >= r) m.z = 0.f;
-              if (c + 3 >= r) m.w = 0.f;
-              if (c + 0 > r) q.x = 0.f;
-              if (c + 1 > r) q.y = 0.f;
-              if (c + 2 > r) q.z = 0.f;
-              if (c + 3 > r) q.w = 0.f;
-              return F4x2{m, q};
-            },
-            [&](int i, F4x2 v) {
-              st4(s + SC_M + 4 * i, v.a);
-              st4(s + SC_P + 4 * i, v.b);
-              const int r = (4 * i) >> 6, c = (4 * i) & (C - 1);
-              const float b = s[SC_BETA + r];
-              sA[r * 65 + c] = b * v.a.x;
-              sA[r * 65 + c + 1] = b * v.a.y;
-              sA[r * 65 + c + 2] = b * v.a.z;
-              sA[r * 65 + c + 3] = b * v.a.w;
-              sT[r * 65 + c] = 0.f;
-              sT[r * 65 + c + 1] = 0.f;
-              sT[r * 65 + c + 2] = 0.f;
-              sT[r * 65 + c + 3] = 0.f;
-            });
   __syncthreads();
   // T = (I + A)^{-1}, A = diag(beta) M, in shared memory (leading dimension 65): diagonal 16 x 16
   // blocks by substitution, then the blocks below them by distance, T_IJ = -T_II sum_K A_IK T_KJ
@@ -497,57 +535,58 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   __syncthreads();
 }
 
-// out[r][c] (+)= f sum_{s} X[r][s] Y[s][c] e^{Gamma_rc - Gamma_sc} over s <= r (X lower triangular as
-// given), per row block I against rho_I = Gamma at the end of block I - 1.
+// out[r][c] (+)= f sum_{s <= r} X[r][s] Y[s][c] e^{Gamma_rc - Gamma_sc} (X lower triangular as given),
+// per block J of s against rho_J = Gamma at the end of block J: the rows r >= 16 J of
+// X[., J cols] (Y_J e^{rho_J - Gamma}) times e^{Gamma_r - rho_J}.
 __device__ void gated_lower(float* s, float* out, const float* X, const float* Y, float f, bool acc, GemmSmem& gsm) {
-  for (int I = 0; I < 4; ++I) {
-    const int ns = 16 * (I + 1);
-    const float* rho = s + SC_G + (16 * I - 1) * D;
-    ew<kB1>(ns * D / 4,
-              [&](int i) {
-                const int c = (4 * i) & (D - 1);
-                const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-                return mul4(ld4(Y + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + 4 * i))));
-              },
-              [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
-    __syncthreads();
-    gemm(s + SC_L, D, mat(X + 16 * I * C, C), mat(s + SC_R, D), 16, D, ns, 1.f, false, 0, gsm);
+  for (int J = 0; J < 4; ++J) {
+    const int r0 = 16 * J;
+    const float* rho = s + SC_G + (16 * J + 15) * D;
     ew<kB1>(16 * D / 4,
-          [&](int i) {
-            const int c = (4 * i) & (D - 1), e = 16 * I * D + 4 * i;
-            const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-            float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(ld4(s + SC_G + e), r4))), f);
-            if (acc) v = add4(v, ld4(out + e));
-            return v;
-          },
-          [&](int i, float4 v) { st4(out + 16 * I * D + 4 * i, v); });
+            [&](int i) {
+              const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
+              return mul4(ld4(Y + e), dexp4(sub4(ld4(rho + c), ld4(s + SC_G + e))));
+            },
+            [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
+    __syncthreads();
+    gemm(s + SC_L, D, mat(X + r0 * C + r0, C), mat(s + SC_R, D), C - r0, D, 16, 1.f, false, 0, gsm);
+    ew<kB1>((C - r0) * D / 4,
+            [&](int i) {
+              const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
+              float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(ld4(s + SC_G + e), ld4(rho + c)))), f);
+              if (acc || J > 0) v = add4(v, ld4(out + e));
+              return v;
+            },
+            [&](int i, float4 v) { st4(out + r0 * D + 4 * i, v); });
     __syncthreads();
   }
 }
 
 // out[s][c] (+)= f sum_{r >= s} X[r][s] Y[r][c] e^{Gamma_rc - Gamma_sc} (X lower triangular as given),
-// per row block J of s against sigma_J = Gamma at the end of block J.
+// per block K of r against rho_K = Gamma at the end of block K - 1 (0 for K = 0): the rows s <
+// 16 (K + 1) of X[K rows, .]^T (Y_K e^{Gamma - rho_K}) times e^{rho_K - Gamma_s}.
 __device__ void gated_upper(float* s, float* out, const float* X, const float* Y, float f, bool acc, GemmSmem& gsm) {
-  for (int J = 0; J < 4; ++J) {
-    const int r0 = 16 * J, nr = C - r0;
-    const float* sig = s + SC_G + (16 * J + 15) * D;
-    ew<kB1>(nr * D / 4,
-              [&](int i) {
-                const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
-                return mul4(ld4(Y + e), dexp4(sub4(ld4(s + SC_G + e), ld4(sig + c))));
-              },
-              [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
-    __syncthreads();
-    // (X[r0.., J cols])^T (rows s of block J) times R
-    gemm(s + SC_L, D, mat(X + r0 * C + r0, C, true), mat(s + SC_R, D), 16, D, nr, 1.f, false, 0, gsm);
+  for (int K = 3; K >= 0; --K) {
+    const int r0 = 16 * K, ns = 16 * (K + 1);
+    const float* rho = s + SC_G + (16 * K - 1) * D;
     ew<kB1>(16 * D / 4,
-          [&](int i) {
-            const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
-            float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(ld4(sig + c), ld4(s + SC_G + e)))), f);
-            if (acc) v = add4(v, ld4(out + e));
-            return v;
-          },
-          [&](int i, float4 v) { st4(out + r0 * D + 4 * i, v); });
+            [&](int i) {
+              const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
+              const float4 r4 = K == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
+              return mul4(ld4(Y + e), dexp4(sub4(ld4(s + SC_G + e), r4)));
+            },
+            [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
+    __syncthreads();
+    gemm(s + SC_L, D, mat(X + r0 * C, C, true), mat(s + SC_R, D), ns, D, 16, 1.f, false, 0, gsm);
+    ew<kB1>(ns * D / 4,
+            [&](int i) {
+              const int c = (4 * i) & (D - 1), e = 4 * i;
+              const float4 r4 = K == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
+              float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + e)))), f);
+              if (acc || K < 3) v = add4(v, ld4(out + e));
+              return v;
+            },
+            [&](int i, float4 v) { st4(out + 4 * i, v); });
     __syncthreads();
   }
 }
@@ -647,7 +686,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
 // dS' of chunk j is kept in the chunk's slot (the input of bwd_grad_kernel); the dS of chunk 0 is
 // the initial state's gradient.
 __global__ void __launch_bounds__(kBwdThreads) bwd_state_kernel(BwdParams P) {
-  __shared__ GemmSmem gsm;
+  extern __shared__ float4 smem4[];
+  GemmSmem& gsm = *reinterpret_cast<GemmSmem*>(smem4);
   const FwdParams& p = P.f;
   const int H = p.num_heads;
   const int n = blockIdx.x / H, h = blockIdx.x - n * H;
@@ -724,17 +764,16 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     gemm(s + SC_DQS, D, mat(s + SC_DO, D), mat(S, D), C, D, D, 1.f, false, 0, gsm);
     gemm(s + SC_DW, D, mat(dD, D), mat(S, D), C, D, D, -1.f, false, 0, gsm);
     gemm(s + SC_DP, C, mat(s + SC_DO, D), mat(s + SC_D, D, true), C, C, D, 1.f, false, 2, gsm);
-    // dgamma from the state: e^gamma_k sum_v S(k, v) dS'(k, v) (a warp per 16 channels, lanes over v)
+    // dgamma from the state: e^gamma_k sum_v S(k, v) dS'(k, v): thread k and half h of the v range
+    // (reads of S coalesced over k, each thread's row of dS' read in order)
     {
-      const int warp = tid >> 5, lane = tid & 31;
-      for (int k = 16 * warp; k < 16 * warp + 16; ++k) {
-        float acc = 0.f;
-#pragma unroll
-        for (int v = lane; v < D; v += 32) acc = fmaf(S[(size_t)v * D + k], dSp[(size_t)k * D + v], acc);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) s[SC_DGAM + k] = s[SC_EG + k] * acc;
-      }
+      const int k = tid & (D - 1), h = tid >> 7;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int v = 64 * h; v < 64 * h + 64; ++v) acc = fmaf(S[(size_t)v * D + k], dSp[(size_t)k * D + v], acc);
+      if (h == 1) s[SC_DGAM + k] = acc;
+      __syncthreads();
+      if (h == 0) s[SC_DGAM + k] = s[SC_EG + k] * (acc + s[SC_DGAM + k]);
     }
     // dT_b = dDelta V^T + dW Kg^T;  dv = T_b^T dDelta;  dKg = T_b^T dW
     gemm(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
@@ -1044,7 +1083,9 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
     if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChunkSmem)) !=
             cudaSuccess ||
         (e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChunkSmem)) !=
-            cudaSuccess)
+            cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sizeof(GemmSmem))) != cudaSuccess)
       return e;
     attr_done[dev] = true;
   }
@@ -1055,7 +1096,7 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
     bwd_prep_kernel<<<(unsigned)grid, kBwdThreads, kChunkSmem, stream>>>(P, items);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  bwd_state_kernel<<<(unsigned)units, kBwdThreads, 0, stream>>>(P);  // also when every document is empty
+  bwd_state_kernel<<<(unsigned)units, kBwdThreads, sizeof(GemmSmem), stream>>>(P);  // also when every document is empty
   if ((e = cudaGetLastError()) != cudaSuccess || tokens == 0) return e;
   bwd_grad_kernel<<<(unsigned)grid, kBwdThreads, kChunkSmem, stream>>>(P, items);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
