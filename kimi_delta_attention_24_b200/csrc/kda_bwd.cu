@@ -55,9 +55,10 @@ constexpr int kPrepFloats = PR_EG + D;
 constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_V = 4 * kF, SC_DO = 5 * kF;
 constexpr int SC_W = 6 * kF, SC_D = 7 * kF, SC_DKT = 8 * kF, SC_DQS = 9 * kF, SC_DW = 10 * kF;
 constexpr int SC_DKG = 11 * kF, SC_R = 12 * kF, SC_L = 13 * kF, SC_X = 14 * kF;
-constexpr int SC_M = 15 * kF, SC_P = SC_M + kQ, SC_T = SC_P + kQ, SC_TB = SC_T + kQ, SC_DP = SC_TB + kQ;
-constexpr int SC_DTB = SC_DP + kQ, SC_TMP = SC_DTB + kQ, SC_DA = SC_TMP + kQ;
-constexpr int SC_BETA = SC_DA + kQ, SC_EG = SC_BETA + C, SC_DGAM = SC_EG + D, SC_DB = SC_DGAM + D;
+constexpr int SC_M = 15 * kF, SC_P = SC_M + kQ, SC_T = SC_P + kQ, SC_TB = SC_T + kQ;
+constexpr int SC_DA = SC_TB + kQ, SC_DP = SC_DA + kQ;  // dA (then dM) and dP adjacent: [dM; dP] is 128 x 64
+constexpr int SC_DTB = SC_DP + kQ, SC_TMP = SC_DTB + kQ;
+constexpr int SC_BETA = SC_TMP + kQ, SC_EG = SC_BETA + C, SC_DGAM = SC_EG + D, SC_DB = SC_DGAM + D;
 constexpr int kScratchFloats = SC_DB + C + 64;
 
 struct BwdParams {
@@ -106,66 +107,47 @@ struct Mat {
 };
 __device__ __forceinline__ Mat mat(const float* p, int ld, bool t = false) { return Mat{p, ld, t}; }
 
-constexpr int GB_K = 64;   // depth of one staged slice
-// Shared-memory rows padded by 8 floats, so that the tensor-core fragment reads (lane (g, t) reads
-// row k0 + t, column g) fall in 32 distinct banks.
-constexpr int SA_LD = 64 + 8, SB_LD = 128 + 8;
+constexpr int GB_K = 32;  // depth of one staged slice
+// A slice keeps its operand's memory orientation in shared memory, rows padded so that the
+// tensor-core fragment reads (lane (g, t) reads row or column g, depth t) fall in 32 distinct banks:
+// along-i slices as [k][i] with 8 floats of padding (bank 8 t + g), along-k slices as [i][k] with 4
+// (bank 4 g + t).  Two stages, so that the next slice's copies overlap the current slice's products.
+constexpr int LD_K = GB_K + 4;  // [i][k] rows
+constexpr int kStageA = 64 * LD_K > GB_K * (64 + 8) ? 64 * LD_K : GB_K * (64 + 8);
+constexpr int kStageB = 128 * LD_K > GB_K * (128 + 8) ? 128 * LD_K : GB_K * (128 + 8);
 struct GemmSmem {
-  float a[GB_K][SA_LD];
-  float b[GB_K][SB_LD];
+  float a[2][kStageA];
+  float b[2][kStageB];
 };
 
-// The GB_K x W slice (k0.., i0..) of an operand, element (i, k) being p[k * ld + i] (memory along
-// i) or p[i * ld + k] (kmaj: memory along k, transposed into s[k][i]), zero outside rows x depth:
-// fetched into registers, then put into shared memory as s[k][i].  A GEMM fetches both operands'
-// slices before it puts either, so that all of a thread's loads are in flight together (through
-// generic pointers the compiler would keep each shared-memory store ahead of the next load).
-template <int W>
-struct Slice {
-  static constexpr int kVec = GB_K * W / 4;  // float4s in the slice
-  static constexpr int kPer = (kVec + kBwdThreads - 1) / kBwdThreads;
-  float4 v[kPer];
-};
-
-template <int W>
-__device__ __forceinline__ void slice_fetch(Slice<W>& r, const float* p, int ld, bool kmaj, int i0, int k0, int rows,
-                                            int depth) {
-  constexpr int kVec = Slice<W>::kVec, kPer = Slice<W>::kPer;
-  const int tid = threadIdx.x;
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    const int idx = tid + e * kBwdThreads;
-    r.v[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (kVec % kBwdThreads != 0 && idx >= kVec) continue;
-    if (!kmaj) {
-      const int i4 = idx % (W / 4), k = idx / (W / 4);
-      if (k0 + k < depth && i0 + 4 * i4 < rows)
-        r.v[e] = *reinterpret_cast<const float4*>(p + (size_t)(k0 + k) * ld + i0 + 4 * i4);
-    } else {
-      const int i = idx % W, k4 = idx / W;
-      if (i0 + i < rows && k0 + 4 * k4 < depth)
-        r.v[e] = *reinterpret_cast<const float4*>(p + (size_t)(i0 + i) * ld + k0 + 4 * k4);
-    }
-  }
+__device__ __forceinline__ void cp_async16(float* dst, const float* src, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int W, int LD>
-__device__ __forceinline__ void slice_put(float (*s)[LD], const Slice<W>& r, bool kmaj) {
-  constexpr int kVec = Slice<W>::kVec, kPer = Slice<W>::kPer;
+// Copies the GB_K x W slice (depth k0.., rows i0..) of an operand into shared memory, zero outside
+// rows x depth: element (i, k) is p[k * ld + i] (along i: to s[k][i], row length W + 8) or p[i * ld +
+// k] (kmaj: to s[i][k], row length LD_K).
+template <int W>
+__device__ __forceinline__ void slice_copy(float* s, const float* p, int ld, bool kmaj, int i0, int k0, int rows,
+                                           int depth) {
+  constexpr int kVec = GB_K * W / 4;
   const int tid = threadIdx.x;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) {
+  for (int e = 0; e < (kVec + kBwdThreads - 1) / kBwdThreads; ++e) {
     const int idx = tid + e * kBwdThreads;
-    if (kVec % kBwdThreads != 0 && idx >= kVec) continue;
+    if (kVec % kBwdThreads != 0 && idx >= kVec) break;
     if (!kmaj) {
       const int i4 = idx % (W / 4), k = idx / (W / 4);
-      *reinterpret_cast<float4*>(&s[k][4 * i4]) = r.v[e];
+      const bool ok = k0 + k < depth && i0 + 4 * i4 < rows;
+      cp_async16(s + k * (W + 8) + 4 * i4, ok ? p + (size_t)(k0 + k) * ld + i0 + 4 * i4 : p, ok);
     } else {
-      const int i = idx % W, k4 = idx / W;
-      s[4 * k4 + 0][i] = r.v[e].x;
-      s[4 * k4 + 1][i] = r.v[e].y;
-      s[4 * k4 + 2][i] = r.v[e].z;
-      s[4 * k4 + 3][i] = r.v[e].w;
+      const int k4 = idx % (GB_K / 4), i = idx / (GB_K / 4);
+      const bool ok = i0 + i < rows && k0 + 4 * k4 < depth;
+      cp_async16(s + i * LD_K + 4 * k4, ok ? p + (size_t)(i0 + i) * ld + k0 + 4 * k4 : p, ok);
     }
   }
 }
@@ -175,19 +157,21 @@ __device__ __forceinline__ void slice_put(float (*s)[LD], const Slice<W>& r, boo
 // mma.sync m16n8k8 with tf32 operands, each operand split into a high and a low tf32 part and the
 // three products hi hi, hi lo, lo hi accumulated in fp32 (about 2^-20 relative: fp32-level).  With
 // RM = 4 warp (wm, wn) holds rows 32 wm .. + 31 and columns 32 wn .. + 31 (2 x 4 fragments), with
-// RM = 1 warp w columns 16 w .. + 15 (1 x 2).  M, N, K multiples of 4 (K of 8 inside a slice);
-// operands 16-byte aligned with ld a multiple of 4.  All threads of the CTA call it; it ends with a
-// barrier.
+// RM = 1 warp w columns 16 w .. + 15 (1 x 2).  M, N multiples of 4, K of 8; operands 16-byte aligned
+// with ld a multiple of 4.  All threads of the CTA call it; it ends with a barrier.
 template <int RM>
 __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc, int mask,
                        GemmSmem& sm) {
   constexpr int BM = 16 * RM;
-  constexpr int LDA = BM + 8;  // 72 or 24: (LDA t + g) mod 32 distinct over the lanes
   constexpr int MT = RM == 4 ? 2 : 1, NT = RM == 4 ? 4 : 2;  // fragments per warp
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int wm = RM == 4 ? (warp & 1) : 0, wn = RM == 4 ? (warp >> 1) : warp;
   const int row0 = RM == 4 ? 32 * wm : 0, col0 = RM == 4 ? 32 * wn : 16 * wn;
-  float (*sa)[LDA] = reinterpret_cast<float (*)[LDA]>(&sm.a[0][0]);
+  const bool a_kmaj = !A.t, b_kmaj = B.t;  // A(i, k) runs along k unless transposed; B(k, j) along j unless transposed
+  const int nsl = (K + GB_K - 1) / GB_K;
+  // element (row, depth) of a stage's A slice and (column, depth) of its B slice
+  auto a_at = [&](const float* sa, int r, int k) { return a_kmaj ? sa[r * LD_K + k] : sa[k * (BM + 8) + r]; };
+  auto b_at = [&](const float* sb, int n, int k) { return b_kmaj ? sb[n * LD_K + k] : sb[k * (128 + 8) + n]; };
   for (int i0 = 0; i0 < M; i0 += BM) {
     for (int j0 = 0; j0 < N; j0 += 128) {
       float c[MT][NT][4];
@@ -197,34 +181,38 @@ __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, fl
         for (int b = 0; b < NT; ++b)
 #pragma unroll
           for (int e = 0; e < 4; ++e) c[a][b][e] = 0.f;
-      for (int k0 = 0; k0 < K; k0 += GB_K) {
-        // A(i, k): memory along k when not transposed; B(k, j): memory along j when not transposed
-        {
-          Slice<BM> ra;
-          Slice<128> rb;
-          slice_fetch<BM>(ra, A.p, A.ld, !A.t, i0, k0, M, K);
-          slice_fetch<128>(rb, B.p, B.ld, B.t, j0, k0, N, K);
-          slice_put<BM, LDA>(sa, ra, !A.t);
-          slice_put<128, SB_LD>(sm.b, rb, B.t);
+      slice_copy<BM>(sm.a[0], A.p, A.ld, a_kmaj, i0, 0, M, K);
+      slice_copy<128>(sm.b[0], B.p, B.ld, b_kmaj, j0, 0, N, K);
+      cp_async_commit();
+      for (int ks = 0; ks < nsl; ++ks) {
+        if (ks + 1 < nsl) {
+          slice_copy<BM>(sm.a[(ks + 1) & 1], A.p, A.ld, a_kmaj, i0, (ks + 1) * GB_K, M, K);
+          slice_copy<128>(sm.b[(ks + 1) & 1], B.p, B.ld, b_kmaj, j0, (ks + 1) * GB_K, N, K);
+          cp_async_commit();
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
         }
         __syncthreads();
-        const int kn = K - k0 < GB_K ? K - k0 : GB_K;
+        const float* sa = sm.a[ks & 1];
+        const float* sb = sm.b[ks & 1];
+        const int kn = K - ks * GB_K < GB_K ? K - ks * GB_K : GB_K;
         for (int kk = 0; kk < kn; kk += 8) {
           uint32_t ah[MT][4], al[MT][4];
 #pragma unroll
           for (int a = 0; a < MT; ++a) {
             const int r = row0 + 16 * a + g;
-            sm100::tf32_split(sa[kk + t][r], ah[a][0], al[a][0]);
-            sm100::tf32_split(sa[kk + t][r + 8], ah[a][1], al[a][1]);
-            sm100::tf32_split(sa[kk + t + 4][r], ah[a][2], al[a][2]);
-            sm100::tf32_split(sa[kk + t + 4][r + 8], ah[a][3], al[a][3]);
+            sm100::tf32_split(a_at(sa, r, kk + t), ah[a][0], al[a][0]);
+            sm100::tf32_split(a_at(sa, r + 8, kk + t), ah[a][1], al[a][1]);
+            sm100::tf32_split(a_at(sa, r, kk + t + 4), ah[a][2], al[a][2]);
+            sm100::tf32_split(a_at(sa, r + 8, kk + t + 4), ah[a][3], al[a][3]);
           }
 #pragma unroll
           for (int b = 0; b < NT; ++b) {
             const int n = col0 + 8 * b + g;
             uint32_t bh0, bl0, bh1, bl1;
-            sm100::tf32_split(sm.b[kk + t][n], bh0, bl0);
-            sm100::tf32_split(sm.b[kk + t + 4][n], bh1, bl1);
+            sm100::tf32_split(b_at(sb, n, kk + t), bh0, bl0);
+            sm100::tf32_split(b_at(sb, n, kk + t + 4), bh1, bl1);
 #pragma unroll
             for (int a = 0; a < MT; ++a) {
               sm100::mma_tf32(c[a][b], ah[a], bl0, bl1);
@@ -233,7 +221,7 @@ __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, fl
             }
           }
         }
-        __syncthreads();
+        __syncthreads();  // the stage is refilled two slices on
       }
 #pragma unroll
       for (int a = 0; a < MT; ++a) {
@@ -535,55 +523,67 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   __syncthreads();
 }
 
-// out[r][c] (+)= f sum_{s <= r} X[r][s] Y[s][c] e^{Gamma_rc - Gamma_sc} (X lower triangular as given),
-// per block J of s against rho_J = Gamma at the end of block J: the rows r >= 16 J of
-// X[., J cols] (Y_J e^{rho_J - Gamma}) times e^{Gamma_r - rho_J}.
-__device__ void gated_lower(float* s, float* out, const float* X, const float* Y, float f, bool acc, GemmSmem& gsm) {
+// The decay-weighted products of dM and dP (lower triangular, stored adjacent as XX = [dM; dP],
+// 128 x 64) with khat, for rows r:  out1[r] (+)= sum_{s<=r} dM[r][s] khat_s e^{Gamma_r - Gamma_s} and
+// out2[r] += sum_{s<=r} dP[r][s] khat_s e^{Gamma_r - Gamma_s}, per block J of s against rho_J = Gamma
+// at the end of block J: XX[., J cols] (khat_J e^{rho_J - Gamma}) times e^{Gamma_r - rho_J} (the rows
+// above block J add zeros).  T: a 128 x 128 temporary.
+__device__ void gated_lower2(float* s, float* out1, bool acc1, float* out2, const float* XX, float* T, GemmSmem& gsm) {
   for (int J = 0; J < 4; ++J) {
     const int r0 = 16 * J;
     const float* rho = s + SC_G + (16 * J + 15) * D;
     ew<kB1>(16 * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
-              return mul4(ld4(Y + e), dexp4(sub4(ld4(rho + c), ld4(s + SC_G + e))));
+              return mul4(ld4(s + SC_KH + e), dexp4(sub4(ld4(rho + c), ld4(s + SC_G + e))));
             },
             [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
     __syncthreads();
-    gemm(s + SC_L, D, mat(X + r0 * C + r0, C), mat(s + SC_R, D), C - r0, D, 16, 1.f, false, 0, gsm);
-    ew<kB1>((C - r0) * D / 4,
+    gemm(T, D, mat(XX + r0, C), mat(s + SC_R, D), 2 * C, D, 16, 1.f, false, 0, gsm);
+    ew<kB2>((C - r0) * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
-              float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(ld4(s + SC_G + e), ld4(rho + c)))), f);
-              if (acc || J > 0) v = add4(v, ld4(out + e));
-              return v;
+              const float4 f = dexp4(sub4(ld4(s + SC_G + e), ld4(rho + c)));
+              float4 v1 = mul4(ld4(T + e), f);
+              if (acc1 || J > 0) v1 = add4(v1, ld4(out1 + e));
+              return F4x2{v1, add4(mul4(ld4(T + C * D + e), f), ld4(out2 + e))};
             },
-            [&](int i, float4 v) { st4(out + r0 * D + 4 * i, v); });
+            [&](int i, F4x2 v) {
+              st4(out1 + r0 * D + 4 * i, v.a);
+              st4(out2 + r0 * D + 4 * i, v.b);
+            });
     __syncthreads();
   }
 }
 
-// out[s][c] (+)= f sum_{r >= s} X[r][s] Y[r][c] e^{Gamma_rc - Gamma_sc} (X lower triangular as given),
-// per block K of r against rho_K = Gamma at the end of block K - 1 (0 for K = 0): the rows s <
-// 16 (K + 1) of X[K rows, .]^T (Y_K e^{Gamma - rho_K}) times e^{rho_K - Gamma_s}.
-__device__ void gated_upper(float* s, float* out, const float* X, const float* Y, float f, bool acc, GemmSmem& gsm) {
+// The transposed decay-weighted products, for rows s:  out[s] = sum_{r>=s} (dM[r][s] khat_r + scale
+// dP[r][s] qhat_r) e^{Gamma_r - Gamma_s}, per block K of r against rho_K = Gamma at the end of block
+// K - 1 (0 for K = 0): the rows s < 16 (K + 1) of dM[K rows, .]^T (khat_K e^{Gamma - rho_K}) +
+// dP[K rows, .]^T (scale qhat_K e^{Gamma - rho_K}), times e^{rho_K - Gamma_s}.
+__device__ void gated_upper2(float* s, float* out, const float* dM, const float* dP, float scale, GemmSmem& gsm) {
   for (int K = 3; K >= 0; --K) {
     const int r0 = 16 * K, ns = 16 * (K + 1);
     const float* rho = s + SC_G + (16 * K - 1) * D;
-    ew<kB1>(16 * D / 4,
+    ew<kB2>(16 * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
               const float4 r4 = K == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-              return mul4(ld4(Y + e), dexp4(sub4(ld4(s + SC_G + e), r4)));
+              const float4 f = dexp4(sub4(ld4(s + SC_G + e), r4));
+              return F4x2{mul4(ld4(s + SC_KH + e), f), scl4(mul4(ld4(s + SC_QH + e), f), scale)};
             },
-            [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
+            [&](int i, F4x2 v) {
+              st4(s + SC_R + 4 * i, v.a);
+              st4(s + SC_R + 16 * D + 4 * i, v.b);
+            });
     __syncthreads();
-    gemm(s + SC_L, D, mat(X + r0 * C, C, true), mat(s + SC_R, D), ns, D, 16, 1.f, false, 0, gsm);
+    gemm(s + SC_L, D, mat(dM + r0 * C, C, true), mat(s + SC_R, D), ns, D, 16, 1.f, false, 0, gsm);
+    gemm(s + SC_L, D, mat(dP + r0 * C, C, true), mat(s + SC_R + 16 * D, D), ns, D, 16, 1.f, true, 0, gsm);
     ew<kB1>(ns * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = 4 * i;
               const float4 r4 = K == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-              float4 v = scl4(mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + e)))), f);
-              if (acc || K < 3) v = add4(v, ld4(out + e));
+              float4 v = mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + e))));
+              if (K < 3) v = add4(v, ld4(out + e));
               return v;
             },
             [&](int i, float4 v) { st4(out + 4 * i, v); });
@@ -828,30 +828,30 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
                 st4(dqh + 4 * i, v.d);
               });
     __syncthreads();
-    gated_lower(s, s + SC_X, s + SC_DA, s + SC_KH, 1.f, false, gsm);  // X1
+    // X1 (to SC_X) and X3 (added to dqhat / scale) in one pass; V and dO are dead: their 2 x 64 x 128
+    // floats hold the 128 x 128 temporary
+    gated_lower2(s, s + SC_X, false, dqh, s + SC_DA, s + SC_V, gsm);
     ew<kB2>(kF4,
-              [&](int i) {
-                const float4 x = ld4(s + SC_X + 4 * i);
-                return F4x2{add4(ld4(dkh + 4 * i), x), add4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
-              },
-              [&](int i, F4x2 v) {
-                st4(dkh + 4 * i, v.a);
-                st4(dG + 4 * i, v.b);
-              });
+            [&](int i) {
+              const float4 x = ld4(s + SC_X + 4 * i);
+              return F4x2{add4(ld4(dkh + 4 * i), x), add4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
+            },
+            [&](int i, F4x2 v) {
+              st4(dkh + 4 * i, v.a);
+              st4(dG + 4 * i, v.b);
+            });
     __syncthreads();
-    gated_upper(s, s + SC_X, s + SC_DA, s + SC_KH, 1.f, false, gsm);   // X2
-    gated_upper(s, s + SC_X, s + SC_DP, s + SC_QH, scale, true, gsm);  // + X4
+    gated_upper2(s, s + SC_X, s + SC_DA, s + SC_DP, scale, gsm);  // X2 + X4
     ew<kB2>(kF4,
-              [&](int i) {
-                const float4 x = ld4(s + SC_X + 4 * i);
-                return F4x2{add4(ld4(dkh + 4 * i), x), sub4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
-              },
-              [&](int i, F4x2 v) {
-                st4(dkh + 4 * i, v.a);
-                st4(dG + 4 * i, v.b);
-              });
+            [&](int i) {
+              const float4 x = ld4(s + SC_X + 4 * i);
+              return F4x2{add4(ld4(dkh + 4 * i), x), sub4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
+            },
+            [&](int i, F4x2 v) {
+              st4(dkh + 4 * i, v.a);
+              st4(dG + 4 * i, v.b);
+            });
     __syncthreads();
-    gated_lower(s, dqh, s + SC_DP, s + SC_KH, 1.f, true, gsm);  // dqhat / scale
     // dgamma: the state term plus sum_r khat e^{gamma-Gamma} dKt; then dlog alpha by a reverse running sum
     if (tid < D) {
       float acc = s[SC_DGAM + tid];
