@@ -379,7 +379,8 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
       const float gv[4] = {g4[u].x, g4[u].y, g4[u].z, g4[u].w};
       float la[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) la[j] = r < len ? p.lower_bound * sigmoid_acc(ea * (gv[j] + dts[j])) : 0.f;
+      for (int j = 0; j < 4; ++j)
+        la[j] = r < len ? p.lower_bound * __fdividef(1.f, 1.f + __expf(-ea * (gv[j] + dts[j]))) : 0.f;
       st4(s + SC_KH + r * D + 4 * lane, scl4(k4[u], ik));
       st4(s + SC_QH + r * D + 4 * lane, scl4(q4[u], iq));
       st4(s + SC_G + r * D + 4 * lane, make_float4(la[0], la[1], la[2], la[3]));
@@ -788,21 +789,29 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     // dT = dT_b diag(beta); dbeta (columns) = colsum(dT_b o T); dA = strict_tril(-T^T dT T^T)
     ew<kB1>(kQ4, [&](int i) { return mul4(ld4(s + SC_DTB + 4 * i), ld4(s + SC_BETA + ((4 * i) & (C - 1)))); },
               [&](int i, float4 v) { st4(s + SC_DA + 4 * i, v); });
-    if (tid < C) {
+    {
+      // thread (column c, quarter q of the rows), the quarters added by shuffles
+      const int c = tid >> 2, q = tid & 3;
       float acc = 0.f;
-#pragma unroll 16
-      for (int r = 0; r < C; ++r) acc = fmaf(s[SC_DTB + r * C + tid], s[SC_T + r * C + tid], acc);
-      s[SC_DB + tid] = acc;
+#pragma unroll
+      for (int r = 16 * q; r < 16 * q + 16; ++r) acc = fmaf(s[SC_DTB + r * C + c], s[SC_T + r * C + c], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (q == 0) s[SC_DB + c] = acc;
     }
     __syncthreads();
     gemm(s + SC_TMP, C, mat(s + SC_T, C, true), mat(s + SC_DA, C), C, C, C, 1.f, false, 0, gsm);
     gemm(s + SC_DA, C, mat(s + SC_TMP, C), mat(s + SC_T, C, true), C, C, C, -1.f, false, 1, gsm);
     // dbeta (rows) += rowsum(dA o M); dM = diag(beta) dA (in place)
-    if (tid < C) {
+    {
+      // thread (row r, quarter q of the columns)
+      const int r = tid >> 2, q = tid & 3;
       float acc = 0.f;
-#pragma unroll 16
-      for (int c = 0; c < C; ++c) acc = fmaf(s[SC_DA + tid * C + c], s[SC_M + tid * C + c], acc);
-      s[SC_DB + tid] += acc;
+#pragma unroll
+      for (int c = 16 * q; c < 16 * q + 16; ++c) acc = fmaf(s[SC_DA + r * C + c], s[SC_M + r * C + c], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (q == 0) s[SC_DB + r] += acc;
     }
     __syncthreads();
     ew<kB1>(kQ4, [&](int i) { return scl4(ld4(s + SC_DA + 4 * i), s[SC_BETA + ((4 * i) >> 6)]); },
@@ -853,22 +862,35 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
             });
     __syncthreads();
     // dgamma: the state term plus sum_r khat e^{gamma-Gamma} dKt; then dlog alpha by a reverse running sum
-    if (tid < D) {
-      float acc = s[SC_DGAM + tid];
-#pragma unroll 16
-      for (int r = 0; r < C; ++r) acc = fmaf(s[SC_KH + r * D + tid], s[SC_DKT + r * D + tid], acc);
-      float run = 0.f;
-      for (int r0 = C - 16; r0 >= 0; r0 -= 16) {
+    {
+      // thread (channel k, half h of the rows): the half's share of dgamma and the total of its
+      // dGamma (through shared memory, 2 x 2 x 128 floats in the dead solve buffer), then the reverse
+      // running sum over its half, the lower half starting from the upper half's total
+      const int k = tid & (D - 1), h = tid >> 7;
+      float* part = sT;
+      float pg = 0.f, tot = 0.f;
+#pragma unroll 8
+      for (int r = 32 * h; r < 32 * h + 32; ++r) {
+        const int e = r * D + k;
+        pg = fmaf(s[SC_KH + e], s[SC_DKT + e], pg);
+        tot += dG[e] + scale * s[SC_QH + e] * dqh[e];
+      }
+      part[h * D + k] = pg;
+      part[2 * D + h * D + k] = tot;
+      __syncthreads();
+      const float dgam = s[SC_DGAM + k] + part[k] + part[D + k];
+      float run = h == 0 ? part[3 * D + k] : 0.f;
+      for (int r0 = 32 * h + 16; r0 >= 32 * h; r0 -= 16) {
         float col[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-          const int e = (r0 + r) * D + tid;
+          const int e = (r0 + r) * D + k;
           col[r] = dG[e] + scale * s[SC_QH + e] * dqh[e];
         }
 #pragma unroll
         for (int r = 15; r >= 0; --r) {
           run += col[r];
-          dG[(r0 + r) * D + tid] = run + acc;
+          dG[(r0 + r) * D + k] = run + dgam;
         }
       }
     }
