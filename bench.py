@@ -215,7 +215,7 @@ BWD_FLOPS_PER_TOKEN_HEAD = 2 * _BWD_MACS_PER_CHUNK / _CB
 
 
 def bench_backward(dev, steps, warmup, seed=0, heads=HEADS):
-    """The backward pass (chunked, fp32 CUDA cores, from the checkpointing forward's states) on the
+    """The backward pass (chunked, from the checkpointing forward's states) on the
     prefill's heads with T = 4096 tokens: milliseconds per step, token-heads/s, HBM GB/s of its
     algorithmic bytes (inputs and d_out read once, the five token gradients written once) and
     TFLOP/s of its chunked-form FLOPs."""
@@ -271,8 +271,8 @@ def bench_backward(dev, steps, warmup, seed=0, heads=HEADS):
             "checkpointing_forward_ms": ms_fwd_ck,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
                          "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
-                         "note": "chunked form on fp32 CUDA cores: latency-bound per chunk (about a fifth of "
-                                 "the fp32 FMA rate), not bound by HBM"},
+                         "note": "chunked form, products on the tensor cores (mma.sync tf32, hi/lo operands): "
+                                 "latency-bound on each chunk's chain of steps, not bound by HBM"},
             "chunked_tflops": BWD_FLOPS_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e12,
             "gpu_launches": steps}
 

@@ -28,8 +28,9 @@
 // chunks last to first: dDelta and the state gradient at every chunk boundary); bwd_grad_kernel
 // (chunk-parallel: recomputes the factors and forms the gradients above); bwd_finish_kernel (the
 // transforms, and dA_log / dt_bias summed with one atomic per value per CTA).  The chunk-parallel
-// kernels are persistent; each CTA keeps one chunk's intermediates in its own global scratch, which
-// stays in L2.  Arithmetic is fp32 on CUDA cores throughout.
+// kernels are persistent; each CTA keeps one chunk's intermediates in its own global scratch (mostly
+// held by L2).  The products run on the tensor cores (mma.sync tf32 with hi/lo operands: fp32-level
+// accuracy), the element-wise work in fp32 on CUDA cores.
 #include "kda_common.cuh"
 #include "sm100.cuh"
 
