@@ -50,7 +50,9 @@ constexpr int PR_KT = kF;          // Kt [64][128]
 constexpr int PR_PDO = 2 * kF;     // P^T dO [64][128]
 constexpr int PR_Y = 3 * kF;       // (Qt - P W)^T dO [128][128]
 constexpr int PR_EG = 3 * kF + D * D;  // e^gamma [128]
-constexpr int kPrepFloats = PR_EG + D;
+constexpr int PR_M = PR_EG + D;        // M [64][64] (strict lower) and T = (I + A)^{-1} [64][64], for the gradient kernel
+constexpr int PR_T = PR_M + kQ;
+constexpr int kPrepFloats = PR_T + kQ;
 
 // per-CTA scratch (floats)
 constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_V = 4 * kF, SC_DO = 5 * kF;
@@ -337,7 +339,9 @@ __device__ Chunk locate(const BwdParams& P, int64_t item) {
 //   kh, qh, Gamma (G), beta, e^gamma, Kg; V and dO (fp32, rows past the chunk's end zero);
 //   M (strict lower), P (lower, with scale), T = (I + A)^{-1}, T_b.
 // need_v: also V (the gradient kernel).
-__device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, bool need_v, GemmSmem& gsm,
+// solve: also the Gram blocks and (I + A)^{-1} (M, P, T, T_b); otherwise only the element-wise factors
+// (the gradient kernel takes M and T from the prep kernel's output).
+__device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, bool need_v, bool solve, GemmSmem& gsm,
                               float* sT /* shared 64 x 65 */, float* sA /* shared 64 x 65 */) {
   const FwdParams& p = P.f;
   const int H = p.num_heads;
@@ -409,6 +413,10 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   __syncthreads();
   ew<kB1>(kF4, [&](int i) { return mul4(ld4(s + SC_KH + 4 * i), dexp4(ld4(s + SC_G + 4 * i))); },
             [&](int i, float4 v) { st4(s + SC_KG + 4 * i, v); });
+  if (!solve) {
+    __syncthreads();
+    return;
+  }
   // M and P: row r of block I = r / 16 takes khat_r e^{Gamma_r - rho_I} (qhat_r for P) against the
   // rows s < 16 (I + 1) of R_I = khat_s e^{rho_I - Gamma_s}, rho_I = Gamma at the end of block I - 1
   // (0 for I = 0).  One product [LK; LQ] (128 x 128) R_all^T, R_all the four R_I stacked (160 rows,
@@ -659,7 +667,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
     float* pr = P.prep + (size_t)it * kPrepFloats;
-    chunk_factors(P, ch, s, false, gsm, sT, sA);
+    chunk_factors(P, ch, s, false, true, gsm, sT, sA);
     // W = T_b Kg (to the output); Kt = khat e^{gamma - Gamma}; X = Qt - P W
     gemm(pr + PR_W, D, mat(s + SC_TB, C), mat(s + SC_KG, D), C, D, C, 1.f, false, 0, gsm);
     const float* gam = s + SC_G + (C - 1) * D;
@@ -675,6 +683,11 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
                 st4(s + SC_X + 4 * i, v.b);
               });
     if (tid < D) pr[PR_EG + tid] = s[SC_EG + tid];
+    ew<kB2>(kQ4, [&](int i) { return F4x2{ld4(s + SC_M + 4 * i), ld4(s + SC_T + 4 * i)}; },
+            [&](int i, F4x2 v) {
+              st4(pr + PR_M + 4 * i, v.a);
+              st4(pr + PR_T + 4 * i, v.b);
+            });
     __syncthreads();
     gemm(s + SC_X, D, mat(s + SC_P, C), mat(pr + PR_W, D), C, D, C, -1.f, true, 0, gsm);
     gemm(pr + PR_Y, D, mat(s + SC_X, D, true), mat(s + SC_DO, D), D, D, C, 1.f, false, 0, gsm);
@@ -718,7 +731,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_state_kernel(BwdParams P) {
     if (j > 0) {
       // the previous chunk's factors into L2 while this one runs
       const char* nx = reinterpret_cast<const char*>(P.prep + (size_t)(it - H) * kPrepFloats);
-      for (int l = tid; l < (int)(kPrepFloats * sizeof(float) / 128); l += kBwdThreads)
+      for (int l = tid; l < (int)(PR_M * sizeof(float) / 128); l += kBwdThreads)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + (size_t)l * 128));
     }
     const float* dsp = P.dsp + ((size_t)(slot0 + j) * H + h) * kStateElems;
@@ -753,7 +766,22 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
   const int64_t n_items = min(items, (int64_t)P.chunk_off[p.num_seqs] * H);
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
-    chunk_factors(P, ch, s, true, gsm, sT, sA);
+    chunk_factors(P, ch, s, true, false, gsm, sT, sA);
+    {
+      // M and T from the prep kernel; T_b = T diag(beta)
+      const float* pr = P.prep + (size_t)it * kPrepFloats;
+      ew<kB4>(kQ4,
+              [&](int i) {
+                const float4 t = ld4(pr + PR_T + 4 * i);
+                return F4x4{ld4(pr + PR_M + 4 * i), t, mul4(t, ld4(s + SC_BETA + ((4 * i) & (C - 1)))), {}};
+              },
+              [&](int i, F4x4 v) {
+                st4(s + SC_M + 4 * i, v.a);
+                st4(s + SC_T + 4 * i, v.b);
+                st4(s + SC_TB + 4 * i, v.c);
+              });
+      __syncthreads();
+    }
     const float* S = P.ckpt + ((size_t)ch.slot * H + ch.h) * kStateElems;   // S^T [v][k]: S(k, v) = S[v * 128 + k]
     const float* dSp = P.dsp + ((size_t)ch.slot * H + ch.h) * kStateElems;  // [k][v]
     const float* dD = P.dd + (size_t)it * kF;
