@@ -101,7 +101,7 @@ __device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, float a, float b, fl
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-// ------------------------------------------------------------------------- generic fp32 GEMM
+// ------------------------------------------------------------------------- the GEMM routine (fp32 operands)
 // An operand: element (i, j) is p[i * ld + j], or p[j * ld + i] when t (transposed).
 struct Mat {
   const float* p;
@@ -785,10 +785,9 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     const float* S = P.ckpt + ((size_t)ch.slot * H + ch.h) * kStateElems;   // S^T [v][k]: S(k, v) = S[v * 128 + k]
     const float* dSp = P.dsp + ((size_t)ch.slot * H + ch.h) * kStateElems;  // [k][v]
     const float* dD = P.dd + (size_t)it * kF;
-    // W = T_b Kg; Delta = T_b V - W S
-    gemm(s + SC_W, D, mat(s + SC_TB, C), mat(s + SC_KG, D), C, D, C, 1.f, false, 0, gsm);
+    // Delta = T_b V - W S (W = T_b Kg as the prep kernel stored it)
     gemm(s + SC_D, D, mat(s + SC_TB, C), mat(s + SC_V, D), C, D, C, 1.f, false, 0, gsm);
-    gemm(s + SC_D, D, mat(s + SC_W, D), mat(S, D, true), C, D, D, -1.f, true, 0, gsm);
+    gemm(s + SC_D, D, mat(P.prep + (size_t)it * kPrepFloats + PR_W, D), mat(S, D, true), C, D, D, -1.f, true, 0, gsm);
     // dKt = Delta dS'^T;  dQs = dO S^T;  dW = -dDelta S^T;  dP = tril(dO Delta^T)
     gemm(s + SC_DKT, D, mat(s + SC_D, D), mat(dSp, D, true), C, D, D, 1.f, false, 0, gsm);
     gemm(s + SC_DQS, D, mat(s + SC_DO, D), mat(S, D), C, D, D, 1.f, false, 0, gsm);
