@@ -147,3 +147,33 @@ def test_bwd_malformed_offsets_report_and_pass_the_state_gradient_through(cuda_d
     assert kda.read_device_status(ws) == 1
     assert torch.equal(got["d_initial"], d_final)
     assert torch.count_nonzero(got["dA_log"]) == 0 and torch.count_nonzero(got["ddt_bias"]) == 0
+
+
+def test_bwd_bench_workload_sampled_heads(cuda_device):
+    """The bench's backward at its full size and in its launch configuration (B = 1, T = 4096, 96
+    heads, from the checkpointing forward's states, inputs generated on the device as the bench does):
+    three heads against the oracle, which takes each head alone (heads are independent)."""
+    T, H = 4096, 96
+    dev = cuda_device
+    x = kda_inputs.make_random("bwd", [T], H, seed=0, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(11)
+    d_out = torch.randn(x.v.shape, generator=gen, device=dev).to(torch.bfloat16)
+    ck = torch.empty(kda.checkpoint_size(T, H, 1) // 4, dtype=torch.float32, device=dev)
+    ws = kda.new_workspace(T, H, 1, dev)
+    out = torch.empty_like(x.v)
+    kda.fwd_checkpointed(x.q, x.k, x.v, x.g, x.beta, x.scale, out, ws, x.A_log, x.dt_bias, x.lower_bound, ck,
+                         cu_seqlens=x.cu_seqlens)
+    got = kda.bwd(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, d_out,
+                  cu_seqlens=x.cu_seqlens, checkpoints=ck)
+    torch.cuda.synchronize()
+    assert kda.read_device_status(ws) == 0
+    for h in (0, 47, 95):
+        tok = lambda t: t[:, :, h:h + 1].contiguous().cpu()
+        ref = oracle.kda_bwd(tok(x.q), tok(x.k), tok(x.v), tok(x.g), tok(x.beta), x.scale,
+                             x.A_log[h:h + 1].cpu(), x.dt_bias[h:h + 1].cpu(), x.lower_bound, tok(d_out),
+                             cu_seqlens=x.cu_seqlens.cpu())
+        sub = {n: tok(got[n]) for n in ("dq", "dk", "dv", "dg", "dbeta")}
+        sub["dA_log"] = got["dA_log"][h:h + 1].cpu()
+        sub["ddt_bias"] = got["ddt_bias"][h:h + 1].cpu()
+        sub["d_initial"] = got["d_initial"][:, h:h + 1].cpu()
+        check_grads(sub, ref, f"bench workload T=4096 H=96, head {h}")
