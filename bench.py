@@ -216,9 +216,10 @@ BWD_FLOPS_PER_TOKEN_HEAD = 2 * _BWD_MACS_PER_CHUNK / _CB
 
 def bench_backward(dev, steps, warmup, seed=0, heads=HEADS):
     """The backward pass (chunked, from the checkpointing forward's states) on the
-    prefill's heads with T = 4096 tokens: milliseconds per step, token-heads/s, HBM GB/s of its
-    algorithmic bytes (inputs and d_out read once, the five token gradients written once) and
-    TFLOP/s of its chunked-form FLOPs."""
+    prefill's heads with T = 4096 tokens: milliseconds per step, token-heads/s, TFLOP/s of its
+    chunked-form FLOPs against the tf32 tensor peak (the binding roofline: about 193 FLOP per
+    algorithmic byte, above the tf32 ridge) and HBM GB/s of its algorithmic bytes (inputs and d_out
+    read once, the five token gradients written once)."""
     import kda_inputs
     import kimi_delta_attention_24_b200 as kda
 
@@ -262,18 +263,31 @@ def bench_backward(dev, steps, warmup, seed=0, heads=HEADS):
     ms_fwd_ck = e0.elapsed_time(e1) / steps
     th = BWD_TOKENS * HEADS
     alg = BWD_BYTES_PER_TOKEN_HEAD * th
-    hbm_peak, _, peak_kind = load_peaks()
+    flops = BWD_FLOPS_PER_TOKEN_HEAD * th
+    hbm_peak, bf16_peak, peak_kind = load_peaks()
+    # the products are tf32 contractions: the tf32 peak is the measured bf16 one times the nominal
+    # dense tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s); at 192 FLOP per byte the backward sits above the
+    # tf32 ridge, so the tensor roofline binds
+    tf32_peak = bf16_peak * 1.1 / 2.25
     gbs = alg / (ms * 1e-3) / 1e9
+    tflops = flops / (ms * 1e-3) / 1e12
+    bound = "tensor" if flops / (tf32_peak * 1e12) >= alg / (hbm_peak * 1e9) else "hbm"
+    roof = ({"bound": "tensor", "achieved": tflops, "peak": tf32_peak, "unit": "TFLOP/s", "frac": tflops / tf32_peak}
+            if bound == "tensor" else
+            {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak})
+    roof.update({"peak_source": f"{peak_kind} (tf32: measured bf16 x 1.1 / 2.25)" if bound == "tensor" else peak_kind,
+                 "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg,
+                 "hbm_achieved_gbs": gbs, "hbm_frac": gbs / hbm_peak,
+                 "note": "chunked form, products on the tensor cores (mma.sync tf32, each operand split hi + lo: "
+                         "three products per product of the form); latency-bound on each chunk's chain of "
+                         "steps"})
     return {"workload": f"backward: B=1 T={BWD_TOKENS} H={HEADS} K=V=128, gradients of every input, from the "
                         "chunk-start states the checkpointing forward stored",
             "ms_per_step": ms, "value": th / (ms * 1e-3) / 1e6, "unit": UNIT,
             "ms_per_step_without_checkpoints": ms_without,
             "checkpointing_forward_ms": ms_fwd_ck,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
-                         "note": "chunked form, products on the tensor cores (mma.sync tf32, hi/lo operands): "
-                                 "latency-bound on each chunk's chain of steps, not bound by HBM"},
-            "chunked_tflops": BWD_FLOPS_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e12,
+            "roofline": roof,
+            "chunked_tflops": tflops,
             "gpu_launches": steps}
 
 
