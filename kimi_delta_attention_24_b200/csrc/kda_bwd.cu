@@ -302,7 +302,9 @@ __device__ __forceinline__ void ew(int n4, F f, S st) {
   }
 }
 constexpr int kF4 = kF / 4, kQ4 = kQ / 4;  // float4s in a 64 x 128 / 64 x 64 matrix
-constexpr int kB1 = 8, kB2 = 4, kB4 = 2;  // batch sizes for results of 1, 2 and 4 float4s
+// batch sizes for results of 1, 2 and 4 float4s: small, since larger batches spill registers in the
+// chunk kernels (128 registers a thread at two CTAs per SM), which costs more than their latency hiding
+constexpr int kB1 = 2, kB2 = 1, kB4 = 1;
 
 // ------------------------------------------------------------------------- per-chunk recomputation
 struct Chunk {
@@ -350,12 +352,12 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   const float ea = expf(p.A_log[h]);
   const float4 dt = reinterpret_cast<const float4*>(p.dt_bias + (size_t)h * D)[lane];
   const float dts[4] = {dt.x, dt.y, dt.z, dt.w};
-  // prologue: warp per row, lane per 4 channels; each warp loads four rows before it stores any
-  for (int r0 = warp; r0 < C; r0 += 4 * (kBwdThreads / 32)) {
-    float4 k4[4], q4[4], g4[4], v4[4], o4[4];
-    float br[4];
+  // prologue: warp per row, lane per 4 channels; each warp loads two rows before it stores any
+  for (int r0 = warp; r0 < C; r0 += 2 * (kBwdThreads / 32)) {
+    float4 k4[2], q4[2], g4[2], v4[2], o4[2];
+    float br[2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int r = r0 + u * (kBwdThreads / 32);
       const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
       k4[u] = q4[u] = g4[u] = v4[u] = o4[u] = z;
@@ -371,7 +373,7 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int r = r0 + u * (kBwdThreads / 32);
       float sk = k4[u].x * k4[u].x + k4[u].y * k4[u].y + k4[u].z * k4[u].z + k4[u].w * k4[u].w;
       float sq = q4[u].x * q4[u].x + q4[u].y * q4[u].y + q4[u].z * q4[u].z + q4[u].w * q4[u].w;
@@ -652,7 +654,8 @@ __global__ void bwd_chunk_table_kernel(BwdParams P, int32_t* chunk_off) {
   }
 }
 
-constexpr size_t kChunkSmem = sizeof(GemmSmem) + 2 * 64 * 65 * sizeof(float);
+constexpr size_t kChunkSmem = sizeof(GemmSmem) + 2 * 64 * 65 * sizeof(float);  // the prep kernel
+constexpr size_t kGradSmem = sizeof(GemmSmem) + 4 * D * sizeof(float);        // + the dgamma partials
 
 // Per chunk: W, Kt, P^T dO, (Qt - P W)^T dO and e^gamma for the state-gradient walk.
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, int64_t items) {
@@ -755,8 +758,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_state_kernel(BwdParams P) {
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, int64_t items) {
   extern __shared__ float4 smem4[];
   GemmSmem& gsm = *reinterpret_cast<GemmSmem*>(smem4);
-  float* sT = reinterpret_cast<float*>(smem4) + sizeof(GemmSmem) / 4;
-  float* sA = sT + 64 * 65;
+  float* part = reinterpret_cast<float*>(smem4) + sizeof(GemmSmem) / 4;  // 4 x 128 floats
   float* s = P.scratch + (size_t)blockIdx.x * kScratchFloats;
   const FwdParams& p = P.f;
   const int H = p.num_heads;
@@ -766,7 +768,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
   const int64_t n_items = min(items, (int64_t)P.chunk_off[p.num_seqs] * H);
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
-    chunk_factors(P, ch, s, true, false, gsm, sT, sA);
+    chunk_factors(P, ch, s, true, false, gsm, nullptr, nullptr);
     {
       // M and T from the prep kernel; T_b = T diag(beta)
       const float* pr = P.prep + (size_t)it * kPrepFloats;
@@ -794,12 +796,18 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     gemm(s + SC_DW, D, mat(dD, D), mat(S, D), C, D, D, -1.f, false, 0, gsm);
     gemm(s + SC_DP, C, mat(s + SC_DO, D), mat(s + SC_D, D, true), C, C, D, 1.f, false, 2, gsm);
     // dgamma from the state: e^gamma_k sum_v S(k, v) dS'(k, v): thread k and half h of the v range
-    // (reads of S coalesced over k, each thread's row of dS' read in order)
+    // (reads of S coalesced over k, each thread's row of dS' read in order, 4 values a load)
     {
       const int k = tid & (D - 1), h = tid >> 7;
       float acc = 0.f;
-#pragma unroll 8
-      for (int v = 64 * h; v < 64 * h + 64; ++v) acc = fmaf(S[(size_t)v * D + k], dSp[(size_t)k * D + v], acc);
+#pragma unroll 4
+      for (int v = 64 * h; v < 64 * h + 64; v += 4) {
+        const float4 d = ld4(dSp + (size_t)k * D + v);
+        acc = fmaf(S[(size_t)v * D + k], d.x, acc);
+        acc = fmaf(S[(size_t)(v + 1) * D + k], d.y, acc);
+        acc = fmaf(S[(size_t)(v + 2) * D + k], d.z, acc);
+        acc = fmaf(S[(size_t)(v + 3) * D + k], d.w, acc);
+      }
       if (h == 1) s[SC_DGAM + k] = acc;
       __syncthreads();
       if (h == 0) s[SC_DGAM + k] = s[SC_EG + k] * (acc + s[SC_DGAM + k]);
@@ -892,10 +900,9 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     // dgamma: the state term plus sum_r khat e^{gamma-Gamma} dKt; then dlog alpha by a reverse running sum
     {
       // thread (channel k, half h of the rows): the half's share of dgamma and the total of its
-      // dGamma (through shared memory, 2 x 2 x 128 floats in the dead solve buffer), then the reverse
-      // running sum over its half, the lower half starting from the upper half's total
+      // dGamma (through shared memory, 2 x 2 x 128 floats), then the reverse running sum over its
+      // half, the lower half starting from the upper half's total
       const int k = tid & (D - 1), h = tid >> 7;
-      float* part = sT;
       float pg = 0.f, tot = 0.f;
 #pragma unroll 8
       for (int r = 32 * h; r < 32 * h + 32; ++r) {
@@ -1132,10 +1139,16 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChunkSmem)) !=
             cudaSuccess ||
-        (e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChunkSmem)) !=
+        (e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGradSmem)) !=
             cudaSuccess ||
         (e = cudaFuncSetAttribute(bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)sizeof(GemmSmem))) != cudaSuccess)
+      return e;
+    // the rest of each SM's 256 KB as L1: shared memory for exactly two CTAs (one for the walk)
+    auto carve = [](size_t bytes, int ctas) { return (int)((ctas * (bytes + 1024) * 100 + 232447) / 233472); };
+    if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve(kChunkSmem, 2))) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve(kGradSmem, 2))) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_state_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve(sizeof(GemmSmem), 1))) != cudaSuccess)
       return e;
     attr_done[dev] = true;
   }
@@ -1148,7 +1161,7 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
   }
   bwd_state_kernel<<<(unsigned)units, kBwdThreads, sizeof(GemmSmem), stream>>>(P);  // also when every document is empty
   if ((e = cudaGetLastError()) != cudaSuccess || tokens == 0) return e;
-  bwd_grad_kernel<<<(unsigned)grid, kBwdThreads, kChunkSmem, stream>>>(P, items);
+  bwd_grad_kernel<<<(unsigned)grid, kBwdThreads, kGradSmem, stream>>>(P, items);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const dim3 fgrid((unsigned)((tokens + kFinishTokens - 1) / kFinishTokens), (unsigned)f.num_heads);
   bwd_finish_kernel<<<fgrid, 256, 0, stream>>>(P, tokens, kFinishTokens);
