@@ -54,14 +54,21 @@ constexpr int PR_M = PR_EG + D;        // M [64][64] (strict lower) and T = (I +
 constexpr int PR_T = PR_M + kQ;
 constexpr int kPrepFloats = PR_T + kQ;
 
-// per-CTA scratch (floats)
-constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_V = 4 * kF, SC_DO = 5 * kF;
-constexpr int SC_W = 6 * kF, SC_D = 7 * kF, SC_DKT = 8 * kF, SC_DQS = 9 * kF, SC_DW = 10 * kF;
-constexpr int SC_DKG = 11 * kF, SC_R = 12 * kF, SC_L = 13 * kF, SC_X = 14 * kF;
-constexpr int SC_M = 15 * kF, SC_P = SC_M + kQ, SC_T = SC_P + kQ, SC_TB = SC_T + kQ;
+// per-CTA scratch (floats).  Each kernel reuses buffers once they are dead, so that the scratch of
+// all its CTAs (448 KB each) mostly stays in L2.  The prep kernel: the Gram product's operands and
+// output in V .. DKG (V is not needed there), Qt - P W in V after them.  The gradient kernel: dv's
+// temporary and the gated products' partial sums in D (Delta), their depth-16 right operands in DW,
+// the transposed ones' output in KG, the 128 x 128 temporary in dO and V, the product T^T dA in DTB;
+// M and T read from the prep kernel's output.
+constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_DO = 4 * kF, SC_V = 5 * kF;
+constexpr int SC_W = 6 * kF, SC_D = 7 * kF, SC_DKT = 8 * kF, SC_DQS = 9 * kF, SC_DW = 10 * kF, SC_DKG = 11 * kF;
+constexpr int SC_GL = SC_V, SC_GR = SC_D, SC_GO = SC_DQS + kF / 2;  // prep: 128 x 128, 160 x 128, 128 x 160
+constexpr int SC_X = SC_V;                                          // prep: Qt - P W
+constexpr int SC_M = 12 * kF, SC_P = SC_M + kQ, SC_T = SC_P + kQ, SC_TB = SC_T + kQ;
 constexpr int SC_DA = SC_TB + kQ, SC_DP = SC_DA + kQ;  // dA (then dM) and dP adjacent: [dM; dP] is 128 x 64
-constexpr int SC_DTB = SC_DP + kQ, SC_TMP = SC_DTB + kQ;
-constexpr int SC_BETA = SC_TMP + kQ, SC_EG = SC_BETA + C, SC_DGAM = SC_EG + D, SC_DB = SC_DGAM + D;
+constexpr int SC_DTB = SC_DP + kQ;
+constexpr int SC_BETA = SC_DTB + kQ, SC_EG = SC_BETA + C, SC_DGAM = SC_EG + D, SC_DB = SC_DGAM + D;
+static_assert(SC_GO + 160 * D <= SC_M, "the Gram product's output ends before M");
 constexpr int kScratchFloats = SC_DB + C + 64;
 
 struct BwdParams {
@@ -102,13 +109,19 @@ __device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, float a, float b, fl
 }
 
 // ------------------------------------------------------------------------- the GEMM routine (fp32 operands)
-// An operand: element (i, j) is p[i * ld + j], or p[j * ld + i] when t (transposed).
+// An operand: element (i, j) is p[i * ld + j], or p[j * ld + i] when t (transposed).  With p2, the
+// depth index k >= k2 reads the second operand p2 at depth k - k2 (two products summed in one).
 struct Mat {
   const float* p;
   int ld;
   bool t;
+  const float* p2;
+  int k2;
 };
-__device__ __forceinline__ Mat mat(const float* p, int ld, bool t = false) { return Mat{p, ld, t}; }
+__device__ __forceinline__ Mat mat(const float* p, int ld, bool t = false) { return Mat{p, ld, t, nullptr, 1 << 30}; }
+__device__ __forceinline__ Mat mat2(const float* p, const float* p2, int k2, int ld, bool t) {
+  return Mat{p, ld, t, p2, k2};
+}
 
 constexpr int GB_K = 32;  // depth of one staged slice
 // A slice keeps its operand's memory orientation in shared memory, rows padded so that the
@@ -135,8 +148,8 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // rows x depth: element (i, k) is p[k * ld + i] (along i: to s[k][i], row length W + 8) or p[i * ld +
 // k] (kmaj: to s[i][k], row length LD_K).
 template <int W>
-__device__ __forceinline__ void slice_copy(float* s, const float* p, int ld, bool kmaj, int i0, int k0, int rows,
-                                           int depth) {
+__device__ __forceinline__ void slice_copy(float* s, const Mat& m, bool kmaj, int i0, int k0, int rows, int depth) {
+  const int ld = m.ld;
   constexpr int kVec = GB_K * W / 4;
   const int tid = threadIdx.x;
 #pragma unroll
@@ -144,13 +157,15 @@ __device__ __forceinline__ void slice_copy(float* s, const float* p, int ld, boo
     const int idx = tid + e * kBwdThreads;
     if (kVec % kBwdThreads != 0 && idx >= kVec) break;
     if (!kmaj) {
-      const int i4 = idx % (W / 4), k = idx / (W / 4);
-      const bool ok = k0 + k < depth && i0 + 4 * i4 < rows;
-      cp_async16(s + k * (W + 8) + 4 * i4, ok ? p + (size_t)(k0 + k) * ld + i0 + 4 * i4 : p, ok);
+      const int i4 = idx % (W / 4), k = idx / (W / 4), kk = k0 + k;
+      const bool ok = kk < depth && i0 + 4 * i4 < rows;
+      const float* src = kk < m.k2 ? m.p + (size_t)kk * ld : m.p2 + (size_t)(kk - m.k2) * ld;
+      cp_async16(s + k * (W + 8) + 4 * i4, ok ? src + i0 + 4 * i4 : m.p, ok);
     } else {
-      const int k4 = idx % (GB_K / 4), i = idx / (GB_K / 4);
-      const bool ok = i0 + i < rows && k0 + 4 * k4 < depth;
-      cp_async16(s + i * LD_K + 4 * k4, ok ? p + (size_t)(i0 + i) * ld + k0 + 4 * k4 : p, ok);
+      const int k4 = idx % (GB_K / 4), i = idx / (GB_K / 4), kk = k0 + 4 * k4;
+      const bool ok = i0 + i < rows && kk < depth;
+      const float* src = kk < m.k2 ? m.p + kk : m.p2 + (kk - m.k2);
+      cp_async16(s + i * LD_K + 4 * k4, ok ? src + (size_t)(i0 + i) * ld : m.p, ok);
     }
   }
 }
@@ -184,13 +199,13 @@ __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, fl
         for (int b = 0; b < NT; ++b)
 #pragma unroll
           for (int e = 0; e < 4; ++e) c[a][b][e] = 0.f;
-      slice_copy<BM>(sm.a[0], A.p, A.ld, a_kmaj, i0, 0, M, K);
-      slice_copy<128>(sm.b[0], B.p, B.ld, b_kmaj, j0, 0, N, K);
+      slice_copy<BM>(sm.a[0], A, a_kmaj, i0, 0, M, K);
+      slice_copy<128>(sm.b[0], B, b_kmaj, j0, 0, N, K);
       cp_async_commit();
       for (int ks = 0; ks < nsl; ++ks) {
         if (ks + 1 < nsl) {
-          slice_copy<BM>(sm.a[(ks + 1) & 1], A.p, A.ld, a_kmaj, i0, (ks + 1) * GB_K, M, K);
-          slice_copy<128>(sm.b[(ks + 1) & 1], B.p, B.ld, b_kmaj, j0, (ks + 1) * GB_K, N, K);
+          slice_copy<BM>(sm.a[(ks + 1) & 1], A, a_kmaj, i0, (ks + 1) * GB_K, M, K);
+          slice_copy<128>(sm.b[(ks + 1) & 1], B, b_kmaj, j0, (ks + 1) * GB_K, N, K);
           cp_async_commit();
           cp_async_wait<1>();
         } else {
@@ -424,9 +439,9 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   // (0 for I = 0).  One product [LK; LQ] (128 x 128) R_all^T, R_all the four R_I stacked (160 rows,
   // R_I from row 8 I (I + 1)), of which each row keeps its own block's segment.
   {
-    float* GL = s + SC_W;    // [LK; LQ]: 128 x 128
-    float* GR = s + SC_DKT;  // R_all: 160 x 128
-    float* GO = s + SC_DKG;  // [LK; LQ] R_all^T: 128 x 160
+    float* GL = s + SC_GL;  // [LK; LQ]: 128 x 128
+    float* GR = s + SC_GR;  // R_all: 160 x 128
+    float* GO = s + SC_GO;  // [LK; LQ] R_all^T: 128 x 160
     ew<kB1>(2 * kF4,
             [&](int i) {
               const int e = (4 * i) & (kF - 1), r = e >> 7, c = e & (D - 1), I = r >> 4;
@@ -452,7 +467,7 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
             const int r = (4 * i) >> 6, c = (4 * i) & (C - 1), I = r >> 4;
             float4 m = make_float4(0.f, 0.f, 0.f, 0.f), q = m;
             if (c < 16 * (I + 1)) {
-              const float* go = s + SC_DKG + r * 160 + 8 * I * (I + 1) + c;
+              const float* go = s + SC_GO + r * 160 + 8 * I * (I + 1) + c;
               m = ld4(go);
               q = scl4(ld4(go + 64 * 160), p.scale);
             }
@@ -536,11 +551,14 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
 }
 
 // The decay-weighted products of dM and dP (lower triangular, stored adjacent as XX = [dM; dP],
-// 128 x 64) with khat, for rows r:  out1[r] (+)= sum_{s<=r} dM[r][s] khat_s e^{Gamma_r - Gamma_s} and
-// out2[r] += sum_{s<=r} dP[r][s] khat_s e^{Gamma_r - Gamma_s}, per block J of s against rho_J = Gamma
-// at the end of block J: XX[., J cols] (khat_J e^{rho_J - Gamma}) times e^{Gamma_r - rho_J} (the rows
-// above block J add zeros).  T: a 128 x 128 temporary.
-__device__ void gated_lower2(float* s, float* out1, bool acc1, float* out2, const float* XX, float* T, GemmSmem& gsm) {
+// 128 x 64) with khat, for rows r:  X1[r] = sum_{s<=r} dM[r][s] khat_s e^{Gamma_r - Gamma_s} and
+// X3[r] = sum_{s<=r} dP[r][s] khat_s e^{Gamma_r - Gamma_s}, per block J of s against rho_J = Gamma at
+// the end of block J: XX[., J cols] (khat_J e^{rho_J - Gamma}) times e^{Gamma_r - rho_J} (the rows
+// above block J add zeros).  X3 is added to out2; X1 is added to dkh and khat X1 to dG, row block J
+// as soon as block J of s (the last to reach it) is done, the later rows' partial sums kept in acc.
+// T: a 128 x 128 temporary.
+__device__ void gated_lower2(float* s, float* dkh, float* dG, float* acc, float* out2, const float* XX, float* T,
+                             float* R, GemmSmem& gsm) {
   for (int J = 0; J < 4; ++J) {
     const int r0 = 16 * J;
     const float* rho = s + SC_G + (16 * J + 15) * D;
@@ -549,30 +567,42 @@ __device__ void gated_lower2(float* s, float* out1, bool acc1, float* out2, cons
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
               return mul4(ld4(s + SC_KH + e), dexp4(sub4(ld4(rho + c), ld4(s + SC_G + e))));
             },
-            [&](int i, float4 v) { st4(s + SC_R + 4 * i, v); });
+            [&](int i, float4 v) { st4(R + 4 * i, v); });
     __syncthreads();
-    gemm(T, D, mat(XX + r0, C), mat(s + SC_R, D), 2 * C, D, 16, 1.f, false, 0, gsm);
-    ew<kB2>((C - r0) * D / 4,
+    gemm(T, D, mat(XX + r0, C), mat(R, D), 2 * C, D, 16, 1.f, false, 0, gsm);
+    ew<kB4>((C - r0) * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
               const float4 f = dexp4(sub4(ld4(s + SC_G + e), ld4(rho + c)));
               float4 v1 = mul4(ld4(T + e), f);
-              if (acc1 || J > 0) v1 = add4(v1, ld4(out1 + e));
-              return F4x2{v1, add4(mul4(ld4(T + C * D + e), f), ld4(out2 + e))};
+              if (J > 0) v1 = add4(v1, ld4(acc + e));
+              const float4 v3 = add4(mul4(ld4(T + C * D + e), f), ld4(out2 + e));
+              if (i < 16 * D / 4)  // row block J: X1 complete
+                return F4x4{add4(ld4(dkh + e), v1), add4(ld4(dG + e), mul4(ld4(s + SC_KH + e), v1)), v3, {}};
+              return F4x4{v1, {}, v3, {}};
             },
-            [&](int i, F4x2 v) {
-              st4(out1 + r0 * D + 4 * i, v.a);
-              st4(out2 + r0 * D + 4 * i, v.b);
+            [&](int i, F4x4 v) {
+              const int e = r0 * D + 4 * i;
+              if (i < 16 * D / 4) {
+                st4(dkh + e, v.a);
+                st4(dG + e, v.b);
+              } else {
+                st4(acc + e, v.a);
+              }
+              st4(out2 + e, v.c);
             });
     __syncthreads();
   }
 }
 
-// The transposed decay-weighted products, for rows s:  out[s] = sum_{r>=s} (dM[r][s] khat_r + scale
+// The transposed decay-weighted products, for rows s:  X[s] = sum_{r>=s} (dM[r][s] khat_r + scale
 // dP[r][s] qhat_r) e^{Gamma_r - Gamma_s}, per block K of r against rho_K = Gamma at the end of block
 // K - 1 (0 for K = 0): the rows s < 16 (K + 1) of dM[K rows, .]^T (khat_K e^{Gamma - rho_K}) +
-// dP[K rows, .]^T (scale qhat_K e^{Gamma - rho_K}), times e^{rho_K - Gamma_s}.
-__device__ void gated_upper2(float* s, float* out, const float* dM, const float* dP, float scale, GemmSmem& gsm) {
+// dP[K rows, .]^T (scale qhat_K e^{Gamma - rho_K}), times e^{rho_K - Gamma_s}.  X is added to dkh and
+// -khat X to dG, row block K as soon as block K of r (the last to reach it) is done, the earlier
+// rows' partial sums kept in acc.
+__device__ void gated_upper2(float* s, float* dkh, float* dG, float* acc, const float* dM, const float* dP,
+                             float scale, float* R, float* L, GemmSmem& gsm) {
   for (int K = 3; K >= 0; --K) {
     const int r0 = 16 * K, ns = 16 * (K + 1);
     const float* rho = s + SC_G + (16 * K - 1) * D;
@@ -584,21 +614,31 @@ __device__ void gated_upper2(float* s, float* out, const float* dM, const float*
               return F4x2{mul4(ld4(s + SC_KH + e), f), scl4(mul4(ld4(s + SC_QH + e), f), scale)};
             },
             [&](int i, F4x2 v) {
-              st4(s + SC_R + 4 * i, v.a);
-              st4(s + SC_R + 16 * D + 4 * i, v.b);
+              st4(R + 4 * i, v.a);
+              st4(R + 16 * D + 4 * i, v.b);
             });
     __syncthreads();
-    gemm(s + SC_L, D, mat(dM + r0 * C, C, true), mat(s + SC_R, D), ns, D, 16, 1.f, false, 0, gsm);
-    gemm(s + SC_L, D, mat(dP + r0 * C, C, true), mat(s + SC_R + 16 * D, D), ns, D, 16, 1.f, true, 0, gsm);
-    ew<kB1>(ns * D / 4,
+    // [dM[K rows, .]^T | dP[K rows, .]^T] [R_k; R_q]: one product of depth 32
+    gemm(L, D, mat2(dM + r0 * C, dP + r0 * C, 16, C, true), mat(R, D), ns, D, 32, 1.f, false, 0, gsm);
+    ew<kB2>(ns * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = 4 * i;
               const float4 r4 = K == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-              float4 v = mul4(ld4(s + SC_L + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + e))));
-              if (K < 3) v = add4(v, ld4(out + e));
-              return v;
+              float4 v = mul4(ld4(L + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + e))));
+              if (K < 3) v = add4(v, ld4(acc + e));
+              if (i >= r0 * D / 4)  // row block K: X complete
+                return F4x2{add4(ld4(dkh + e), v), sub4(ld4(dG + e), mul4(ld4(s + SC_KH + e), v))};
+              return F4x2{v, {}};
             },
-            [&](int i, float4 v) { st4(out + 4 * i, v); });
+            [&](int i, F4x2 v) {
+              const int e = 4 * i;
+              if (i >= r0 * D / 4) {
+                st4(dkh + e, v.a);
+                st4(dG + e, v.b);
+              } else {
+                st4(acc + e, v.a);
+              }
+            });
     __syncthreads();
   }
 }
@@ -769,27 +809,19 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
     chunk_factors(P, ch, s, true, false, gsm, nullptr, nullptr);
-    {
-      // M and T from the prep kernel; T_b = T diag(beta)
-      const float* pr = P.prep + (size_t)it * kPrepFloats;
-      ew<kB4>(kQ4,
-              [&](int i) {
-                const float4 t = ld4(pr + PR_T + 4 * i);
-                return F4x4{ld4(pr + PR_M + 4 * i), t, mul4(t, ld4(s + SC_BETA + ((4 * i) & (C - 1)))), {}};
-              },
-              [&](int i, F4x4 v) {
-                st4(s + SC_M + 4 * i, v.a);
-                st4(s + SC_T + 4 * i, v.b);
-                st4(s + SC_TB + 4 * i, v.c);
-              });
-      __syncthreads();
-    }
+    // M and T = (I + A)^{-1} as the prep kernel stored them; T_b = T diag(beta)
+    const float* pr = P.prep + (size_t)it * kPrepFloats;
+    const float* Mp = pr + PR_M;
+    const float* Tp = pr + PR_T;
+    ew<kB1>(kQ4, [&](int i) { return mul4(ld4(Tp + 4 * i), ld4(s + SC_BETA + ((4 * i) & (C - 1)))); },
+            [&](int i, float4 v) { st4(s + SC_TB + 4 * i, v); });
+    __syncthreads();
     const float* S = P.ckpt + ((size_t)ch.slot * H + ch.h) * kStateElems;   // S^T [v][k]: S(k, v) = S[v * 128 + k]
     const float* dSp = P.dsp + ((size_t)ch.slot * H + ch.h) * kStateElems;  // [k][v]
     const float* dD = P.dd + (size_t)it * kF;
     // Delta = T_b V - W S (W = T_b Kg as the prep kernel stored it)
     gemm(s + SC_D, D, mat(s + SC_TB, C), mat(s + SC_V, D), C, D, C, 1.f, false, 0, gsm);
-    gemm(s + SC_D, D, mat(P.prep + (size_t)it * kPrepFloats + PR_W, D), mat(S, D, true), C, D, D, -1.f, true, 0, gsm);
+    gemm(s + SC_D, D, mat(pr + PR_W, D), mat(S, D, true), C, D, D, -1.f, true, 0, gsm);
     // dKt = Delta dS'^T;  dQs = dO S^T;  dW = -dDelta S^T;  dP = tril(dO Delta^T)
     gemm(s + SC_DKT, D, mat(s + SC_D, D), mat(dSp, D, true), C, D, D, 1.f, false, 0, gsm);
     gemm(s + SC_DQS, D, mat(s + SC_DO, D), mat(S, D), C, D, D, 1.f, false, 0, gsm);
@@ -815,8 +847,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     // dT_b = dDelta V^T + dW Kg^T;  dv = T_b^T dDelta;  dKg = T_b^T dW
     gemm(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
     gemm(s + SC_DTB, C, mat(s + SC_DW, D), mat(s + SC_KG, D, true), C, C, D, 1.f, true, 0, gsm);
-    gemm(s + SC_X, D, mat(s + SC_TB, C, true), mat(dD, D), C, D, C, 1.f, false, 0, gsm);
-    ew<kB1>(ch.len * (D / 4), [&](int i) { return ld4(s + SC_X + 4 * i); },
+    gemm(s + SC_D, D, mat(s + SC_TB, C, true), mat(dD, D), C, D, C, 1.f, false, 0, gsm);  // Delta is dead
+    ew<kB1>(ch.len * (D / 4), [&](int i) { return ld4(s + SC_D + 4 * i); },
               [&](int i, float4 v) {
                 const int r = i >> 5, c4 = i & 31;
                 st_bf16x4(P.dv + ((size_t)(ch.t0 + r) * H + ch.h) * D + 4 * c4, v.x, v.y, v.z, v.w);
@@ -830,21 +862,22 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
       const int c = tid >> 2, q = tid & 3;
       float acc = 0.f;
 #pragma unroll
-      for (int r = 16 * q; r < 16 * q + 16; ++r) acc = fmaf(s[SC_DTB + r * C + c], s[SC_T + r * C + c], acc);
+      for (int r = 16 * q; r < 16 * q + 16; ++r) acc = fmaf(s[SC_DTB + r * C + c], Tp[r * C + c], acc);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       if (q == 0) s[SC_DB + c] = acc;
     }
     __syncthreads();
-    gemm(s + SC_TMP, C, mat(s + SC_T, C, true), mat(s + SC_DA, C), C, C, C, 1.f, false, 0, gsm);
-    gemm(s + SC_DA, C, mat(s + SC_TMP, C), mat(s + SC_T, C, true), C, C, C, -1.f, false, 1, gsm);
+    // T^T dT into DTB (dead)
+    gemm(s + SC_DTB, C, mat(Tp, C, true), mat(s + SC_DA, C), C, C, C, 1.f, false, 0, gsm);
+    gemm(s + SC_DA, C, mat(s + SC_DTB, C), mat(Tp, C, true), C, C, C, -1.f, false, 1, gsm);
     // dbeta (rows) += rowsum(dA o M); dM = diag(beta) dA (in place)
     {
       // thread (row r, quarter q of the columns)
       const int r = tid >> 2, q = tid & 3;
       float acc = 0.f;
 #pragma unroll
-      for (int c = 16 * q; c < 16 * q + 16; ++c) acc = fmaf(s[SC_DA + r * C + c], s[SC_M + r * C + c], acc);
+      for (int c = 16 * q; c < 16 * q + 16; ++c) acc = fmaf(s[SC_DA + r * C + c], Mp[r * C + c], acc);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       if (q == 0) s[SC_DB + r] += acc;
@@ -873,30 +906,10 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
                 st4(dqh + 4 * i, v.d);
               });
     __syncthreads();
-    // X1 (to SC_X) and X3 (added to dqhat / scale) in one pass; V and dO are dead: their 2 x 64 x 128
-    // floats hold the 128 x 128 temporary
-    gated_lower2(s, s + SC_X, false, dqh, s + SC_DA, s + SC_V, gsm);
-    ew<kB2>(kF4,
-            [&](int i) {
-              const float4 x = ld4(s + SC_X + 4 * i);
-              return F4x2{add4(ld4(dkh + 4 * i), x), add4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
-            },
-            [&](int i, F4x2 v) {
-              st4(dkh + 4 * i, v.a);
-              st4(dG + 4 * i, v.b);
-            });
-    __syncthreads();
-    gated_upper2(s, s + SC_X, s + SC_DA, s + SC_DP, scale, gsm);  // X2 + X4
-    ew<kB2>(kF4,
-            [&](int i) {
-              const float4 x = ld4(s + SC_X + 4 * i);
-              return F4x2{add4(ld4(dkh + 4 * i), x), sub4(ld4(dG + 4 * i), mul4(ld4(s + SC_KH + 4 * i), x))};
-            },
-            [&](int i, F4x2 v) {
-              st4(dkh + 4 * i, v.a);
-              st4(dG + 4 * i, v.b);
-            });
-    __syncthreads();
+    // X1 (into dkhat and dGamma) and X3 (added to dqhat / scale) in one pass; V and dO are dead: their
+    // 2 x 64 x 128 floats hold the 128 x 128 temporary.  Delta, dW and Kg are dead as well.
+    gated_lower2(s, dkh, dG, s + SC_D, dqh, s + SC_DA, s + SC_DO, s + SC_DW, gsm);
+    gated_upper2(s, dkh, dG, s + SC_D, s + SC_DA, s + SC_DP, scale, s + SC_DW, s + SC_KG, gsm);  // X2 + X4
     // dgamma: the state term plus sum_r khat e^{gamma-Gamma} dKt; then dlog alpha by a reverse running sum
     {
       // thread (channel k, half h of the rows): the half's share of dgamma and the total of its
