@@ -55,7 +55,7 @@ constexpr int PR_T = PR_M + kQ;
 constexpr int kPrepFloats = PR_T + kQ;
 
 // per-CTA scratch (floats).  Each kernel reuses buffers once they are dead, so that the scratch of
-// all its CTAs (448 KB each) mostly stays in L2.  The prep kernel: the Gram product's operands and
+// all its CTAs (at most 448 KB each) mostly stays in L2.  The prep kernel: the Gram product's operands and
 // output in V .. DKG (V is not needed there), Qt - P W in V after them.  The gradient kernel: dv's
 // temporary and the gated products' partial sums in D (Delta), their depth-16 right operands in DW,
 // the transposed ones' output in KG, the 128 x 128 temporary in dO and V, the product T^T dA in DTB;
@@ -64,11 +64,11 @@ constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_DO = 4 * 
 constexpr int SC_W = 6 * kF, SC_D = 7 * kF, SC_DKT = 8 * kF, SC_DQS = 9 * kF, SC_DW = 10 * kF, SC_DKG = 11 * kF;
 constexpr int SC_GL = SC_V, SC_GR = SC_D, SC_GO = SC_DQS + kF / 2;  // prep: 128 x 128, 160 x 128, 128 x 160
 constexpr int SC_X = SC_V;                                          // prep: Qt - P W
-constexpr int SC_M = 12 * kF, SC_P = SC_M + kQ, SC_T = SC_P + kQ, SC_TB = SC_T + kQ;
+constexpr int SC_P = 12 * kF, SC_TB = SC_P + kQ;  // prep: M and T go straight to its output
 constexpr int SC_DA = SC_TB + kQ, SC_DP = SC_DA + kQ;  // dA (then dM) and dP adjacent: [dM; dP] is 128 x 64
 constexpr int SC_DTB = SC_DP + kQ;
 constexpr int SC_BETA = SC_DTB + kQ, SC_EG = SC_BETA + C, SC_DGAM = SC_EG + D, SC_DB = SC_DGAM + D;
-static_assert(SC_GO + 160 * D <= SC_M, "the Gram product's output ends before M");
+static_assert(SC_GO + 160 * D <= SC_P, "the Gram product's output ends before P");
 constexpr int kScratchFloats = SC_DB + C + 64;
 
 struct BwdParams {
@@ -129,12 +129,15 @@ constexpr int GB_K = 32;  // depth of one staged slice
 // along-i slices as [k][i] with 8 floats of padding (bank 8 t + g), along-k slices as [i][k] with 4
 // (bank 4 g + t).  Two stages, so that the next slice's copies overlap the current slice's products.
 constexpr int LD_K = GB_K + 4;  // [i][k] rows
-constexpr int kStageA = 64 * LD_K > GB_K * (64 + 8) ? 64 * LD_K : GB_K * (64 + 8);
-constexpr int kStageB = 128 * LD_K > GB_K * (128 + 8) ? 128 * LD_K : GB_K * (128 + 8);
-struct GemmSmem {
+constexpr int stage_floats(int w) { return w * LD_K > GB_K * (w + 8) ? w * LD_K : GB_K * (w + 8); }
+constexpr int kStageA = stage_floats(64);
+// NB: the widest B tile (column block) the kernel's products use, 128 or 160
+template <int NB>
+struct GemmSmemT {
   float a[2][kStageA];
-  float b[2][kStageB];
+  float b[2][stage_floats(NB)];
 };
+using GemmSmem = GemmSmemT<128>;
 
 __device__ __forceinline__ void cp_async16(float* dst, const float* src, bool valid) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
@@ -171,27 +174,29 @@ __device__ __forceinline__ void slice_copy(float* s, const Mat& m, bool kmaj, in
 }
 
 // C[i][j] = alpha sum_k A(i, k) B(k, j) (+ C[i][j] when acc), i < M, j < N; mask 1 keeps j < i,
-// mask 2 keeps j <= i (the rest is written as 0).  Output tiles of (16 RM) x 128 on the tensor cores:
+// mask 2 keeps j <= i (the rest is written as 0).  Output tiles of (16 RM) x NW on the tensor cores:
 // mma.sync m16n8k8 with tf32 operands, each operand split into a high and a low tf32 part and the
 // three products hi hi, hi lo, lo hi accumulated in fp32 (about 2^-20 relative: fp32-level).  With
-// RM = 4 warp (wm, wn) holds rows 32 wm .. + 31 and columns 32 wn .. + 31 (2 x 4 fragments), with
-// RM = 1 warp w columns 16 w .. + 15 (1 x 2).  M, N multiples of 4, K of 8; operands 16-byte aligned
-// with ld a multiple of 4.  All threads of the CTA call it; it ends with a barrier.
-template <int RM>
+// RM = 4 warp (wm, wn) holds rows 32 wm .. + 31 and columns NW / 4 wn .. + NW / 4 - 1 (2 x NW / 32
+// fragments), with RM = 1 (NW = 128) warp w columns 16 w .. + 15 (1 x 2).  M, N multiples of 4, K of
+// 8; operands 16-byte aligned with ld a multiple of 4.  All threads of the CTA call it; it ends with
+// a barrier.
+template <int RM, int NW, int NB>
 __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc, int mask,
-                       GemmSmem& sm) {
+                       GemmSmemT<NB>& sm) {
+  static_assert(NW <= NB && (RM == 4 || NW == 128), "tile width");
   constexpr int BM = 16 * RM;
-  constexpr int MT = RM == 4 ? 2 : 1, NT = RM == 4 ? 4 : 2;  // fragments per warp
+  constexpr int MT = RM == 4 ? 2 : 1, NT = RM == 4 ? NW / 32 : 2;  // fragments per warp
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int wm = RM == 4 ? (warp & 1) : 0, wn = RM == 4 ? (warp >> 1) : warp;
-  const int row0 = RM == 4 ? 32 * wm : 0, col0 = RM == 4 ? 32 * wn : 16 * wn;
+  const int row0 = RM == 4 ? 32 * wm : 0, col0 = RM == 4 ? (NW / 4) * wn : 16 * wn;
   const bool a_kmaj = !A.t, b_kmaj = B.t;  // A(i, k) runs along k unless transposed; B(k, j) along j unless transposed
   const int nsl = (K + GB_K - 1) / GB_K;
   // element (row, depth) of a stage's A slice and (column, depth) of its B slice
   auto a_at = [&](const float* sa, int r, int k) { return a_kmaj ? sa[r * LD_K + k] : sa[k * (BM + 8) + r]; };
-  auto b_at = [&](const float* sb, int n, int k) { return b_kmaj ? sb[n * LD_K + k] : sb[k * (128 + 8) + n]; };
+  auto b_at = [&](const float* sb, int n, int k) { return b_kmaj ? sb[n * LD_K + k] : sb[k * (NW + 8) + n]; };
   for (int i0 = 0; i0 < M; i0 += BM) {
-    for (int j0 = 0; j0 < N; j0 += 128) {
+    for (int j0 = 0; j0 < N; j0 += NW) {
       float c[MT][NT][4];
 #pragma unroll
       for (int a = 0; a < MT; ++a)
@@ -200,12 +205,12 @@ __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, fl
 #pragma unroll
           for (int e = 0; e < 4; ++e) c[a][b][e] = 0.f;
       slice_copy<BM>(sm.a[0], A, a_kmaj, i0, 0, M, K);
-      slice_copy<128>(sm.b[0], B, b_kmaj, j0, 0, N, K);
+      slice_copy<NW>(sm.b[0], B, b_kmaj, j0, 0, N, K);
       cp_async_commit();
       for (int ks = 0; ks < nsl; ++ks) {
         if (ks + 1 < nsl) {
           slice_copy<BM>(sm.a[(ks + 1) & 1], A, a_kmaj, i0, (ks + 1) * GB_K, M, K);
-          slice_copy<128>(sm.b[(ks + 1) & 1], B, b_kmaj, j0, (ks + 1) * GB_K, N, K);
+          slice_copy<NW>(sm.b[(ks + 1) & 1], B, b_kmaj, j0, (ks + 1) * GB_K, N, K);
           cp_async_commit();
           cp_async_wait<1>();
         } else {
@@ -272,10 +277,11 @@ __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, fl
   __syncthreads();
 }
 
+template <int NB>
 __device__ __forceinline__ void gemm(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc,
-                                     int mask, GemmSmem& sm) {
-  if (M <= 16) gemm_t<1>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
-  else gemm_t<4>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
+                                     int mask, GemmSmemT<NB>& sm) {
+  if (M <= 16) gemm_t<1, 128, NB>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
+  else gemm_t<4, 128, NB>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
 }
 
 // ------------------------------------------------------------------------- element-wise passes
@@ -353,13 +359,16 @@ __device__ Chunk locate(const BwdParams& P, int64_t item) {
 }
 
 // The factors of a chunk that do not involve the state, into the CTA's scratch s:
-//   kh, qh, Gamma (G), beta, e^gamma, Kg; V and dO (fp32, rows past the chunk's end zero);
-//   M (strict lower), P (lower, with scale), T = (I + A)^{-1}, T_b.
+//   kh, qh, Gamma (G), beta, e^gamma, Kg; V and dO (fp32, rows past the chunk's end zero).
 // need_v: also V (the gradient kernel).
-// solve: also the Gram blocks and (I + A)^{-1} (M, P, T, T_b); otherwise only the element-wise factors
-// (the gradient kernel takes M and T from the prep kernel's output).
-__device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, bool need_v, bool solve, GemmSmem& gsm,
-                              float* sT /* shared 64 x 65 */, float* sA /* shared 64 x 65 */) {
+// solve: also the Gram blocks and (I + A)^{-1}: P (lower, with scale) and T_b into s, M (strict
+// lower) and T = (I + A)^{-1} to Mout and Tout (the prep kernel's output); otherwise only the
+// element-wise factors (the gradient kernel reads M and T from there).  sT, sA: the solve's two
+// 64 x 65 shared-memory tiles.
+template <int NB>
+__device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, bool need_v, bool solve, GemmSmemT<NB>& gsm,
+                              float* sT /* shared 64 x 65 */, float* sA /* shared 64 x 65 */, float* Mout = nullptr,
+                              float* Tout = nullptr) {
   const FwdParams& p = P.f;
   const int H = p.num_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -459,7 +468,8 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
             },
             [&](int i, float4 v) { st4(GR + 4 * i, v); });
     __syncthreads();
-    gemm(GO, 160, mat(GL, D), mat(GR, D, true), 2 * C, 160, D, 1.f, false, 0, gsm);
+    if constexpr (NB >= 160) gemm_t<4, 160, NB>(GO, 160, mat(GL, D), mat(GR, D, true), 2 * C, 160, D, 1.f, false, 0, gsm);
+    else gemm(GO, 160, mat(GL, D), mat(GR, D, true), 2 * C, 160, D, 1.f, false, 0, gsm);
   }
   // M strictly lower, P (times scale) lower with its diagonal, each row from its block's segment
   ew<kB2>(kQ4,
@@ -482,7 +492,7 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
             return F4x2{m, q};
           },
           [&](int i, F4x2 v) {
-            st4(s + SC_M + 4 * i, v.a);
+            st4(Mout + 4 * i, v.a);
             st4(s + SC_P + 4 * i, v.b);
             const int r = (4 * i) >> 6, c = (4 * i) & (C - 1);
             const float b = s[SC_BETA + r];
@@ -544,7 +554,7 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
               return F4x2{t, mul4(t, ld4(s + SC_BETA + c))};
             },
             [&](int i, F4x2 v) {
-              st4(s + SC_T + 4 * i, v.a);
+              st4(Tout + 4 * i, v.a);
               st4(s + SC_TB + 4 * i, v.b);
             });
   __syncthreads();
@@ -694,14 +704,18 @@ __global__ void bwd_chunk_table_kernel(BwdParams P, int32_t* chunk_off) {
   }
 }
 
-constexpr size_t kChunkSmem = sizeof(GemmSmem) + 2 * 64 * 65 * sizeof(float);  // the prep kernel
+// the prep kernel: the solve's two 64 x 65 tiles live in the staging buffer, which no product uses
+// between the Gram product and the W product
+using GemmSmemPrep = GemmSmemT<160>;
+constexpr size_t kChunkSmem = sizeof(GemmSmemPrep);
+static_assert(2 * 64 * 65 * sizeof(float) <= sizeof(GemmSmemPrep), "solve tiles");
 constexpr size_t kGradSmem = sizeof(GemmSmem) + 4 * D * sizeof(float);        // + the dgamma partials
 
 // Per chunk: W, Kt, P^T dO, (Qt - P W)^T dO and e^gamma for the state-gradient walk.
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, int64_t items) {
   extern __shared__ float4 smem4[];
-  GemmSmem& gsm = *reinterpret_cast<GemmSmem*>(smem4);
-  float* sT = reinterpret_cast<float*>(smem4) + sizeof(GemmSmem) / 4;
+  GemmSmemPrep& gsm = *reinterpret_cast<GemmSmemPrep*>(smem4);
+  float* sT = reinterpret_cast<float*>(smem4);  // the solve's tiles (see kChunkSmem)
   float* sA = sT + 64 * 65;
   float* s = P.scratch + (size_t)blockIdx.x * kScratchFloats;
   const int tid = threadIdx.x;
@@ -710,7 +724,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
     float* pr = P.prep + (size_t)it * kPrepFloats;
-    chunk_factors(P, ch, s, false, true, gsm, sT, sA);
+    chunk_factors(P, ch, s, false, true, gsm, sT, sA, pr + PR_M, pr + PR_T);
     // W = T_b Kg (to the output); Kt = khat e^{gamma - Gamma}; X = Qt - P W
     gemm(pr + PR_W, D, mat(s + SC_TB, C), mat(s + SC_KG, D), C, D, C, 1.f, false, 0, gsm);
     const float* gam = s + SC_G + (C - 1) * D;
@@ -726,11 +740,6 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
                 st4(s + SC_X + 4 * i, v.b);
               });
     if (tid < D) pr[PR_EG + tid] = s[SC_EG + tid];
-    ew<kB2>(kQ4, [&](int i) { return F4x2{ld4(s + SC_M + 4 * i), ld4(s + SC_T + 4 * i)}; },
-            [&](int i, F4x2 v) {
-              st4(pr + PR_M + 4 * i, v.a);
-              st4(pr + PR_T + 4 * i, v.b);
-            });
     __syncthreads();
     gemm(s + SC_X, D, mat(s + SC_P, C), mat(pr + PR_W, D), C, D, C, -1.f, true, 0, gsm);
     gemm(pr + PR_Y, D, mat(s + SC_X, D, true), mat(s + SC_DO, D), D, D, C, 1.f, false, 0, gsm);
