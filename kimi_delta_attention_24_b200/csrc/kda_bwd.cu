@@ -173,17 +173,41 @@ __device__ __forceinline__ void slice_copy(float* s, const Mat& m, bool kmaj, in
   }
 }
 
-// C[i][j] = alpha sum_k A(i, k) B(k, j) (+ C[i][j] when acc), i < M, j < N; mask 1 keeps j < i,
-// mask 2 keeps j <= i (the rest is written as 0).  Output tiles of (16 RM) x NW on the tensor cores:
+// The output of a product: load(i, j) reads what the result (i, j .. j + 1) combines with, store(i, j,
+// v, l) writes it from the product's value v and that l.  With kLoadsFirst a thread issues all of its
+// tile's loads before its stores (more registers; for outputs that combine with other buffers).  The
+// default: C[i][j] = alpha v (+ C[i][j] when acc); mask 1 keeps j < i, mask 2 keeps j <= i (the rest
+// is written as 0).
+struct EpiStore {
+  static constexpr bool kLoadsFirst = false;
+  float* C;
+  int ldc;
+  float alpha;
+  bool acc;
+  int mask;
+  __device__ __forceinline__ float2 load(int i, int j) const {
+    return acc ? *reinterpret_cast<const float2*>(C + (size_t)i * ldc + j) : make_float2(0.f, 0.f);
+  }
+  __device__ __forceinline__ void store(int i, int j, float2 v, float2 l) const {
+    float2 o = make_float2(fmaf(alpha, v.x, l.x), fmaf(alpha, v.y, l.y));
+    if (mask) {
+      const int lim = mask == 1 ? i : i + 1;  // keep j < lim
+      if (j + 0 >= lim) o.x = 0.f;
+      if (j + 1 >= lim) o.y = 0.f;
+    }
+    *reinterpret_cast<float2*>(C + (size_t)i * ldc + j) = o;
+  }
+};
+
+// sum_k A(i, k) B(k, j), i < M, j < N, to the output epi.  Output tiles of (16 RM) x NW on the tensor cores:
 // mma.sync m16n8k8 with tf32 operands, each operand split into a high and a low tf32 part and the
 // three products hi hi, hi lo, lo hi accumulated in fp32 (about 2^-20 relative: fp32-level).  With
 // RM = 4 warp (wm, wn) holds rows 32 wm .. + 31 and columns NW / 4 wn .. + NW / 4 - 1 (2 x NW / 32
 // fragments), with RM = 1 (NW = 128) warp w columns 16 w .. + 15 (1 x 2).  M, N multiples of 4, K of
 // 8; operands 16-byte aligned with ld a multiple of 4.  All threads of the CTA call it; it ends with
 // a barrier.
-template <int RM, int NW, int NB>
-__device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc, int mask,
-                       GemmSmemT<NB>& sm) {
+template <int RM, int NW, int NB, class Epi>
+__device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, const Epi& epi) {
   static_assert(NW <= NB && (RM == 4 || NW == 128), "tile width");
   constexpr int BM = 16 * RM;
   constexpr int MT = RM == 4 ? 2 : 1, NT = RM == 4 ? NW / 32 : 2;  // fragments per warp
@@ -246,42 +270,51 @@ __device__ void gemm_t(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, fl
         }
         __syncthreads();  // the stage is refilled two slices on
       }
+      if constexpr (Epi::kLoadsFirst) {
+        float2 l[MT][2][NT];
 #pragma unroll
-      for (int a = 0; a < MT; ++a) {
+        for (int a = 0; a < MT; ++a)
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int i = i0 + row0 + 16 * a + g + 8 * hr;
-          if (i >= M) continue;
+          for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
-          for (int b = 0; b < NT; ++b) {
-            const int j = j0 + col0 + 8 * b + 2 * t;
-            if (j >= N) continue;
-            float2* dst = reinterpret_cast<float2*>(Cp + (size_t)i * ldc + j);
-            float2 o = make_float2(alpha * c[a][b][2 * hr], alpha * c[a][b][2 * hr + 1]);
-            if (acc) {
-              const float2 old = *dst;
-              o.x += old.x;
-              o.y += old.y;
+            for (int b = 0; b < NT; ++b) {
+              const int i = i0 + row0 + 16 * a + g + 8 * hr, j = j0 + col0 + 8 * b + 2 * t;
+              if (i < M && j < N) l[a][hr][b] = epi.load(i, j);
             }
-            if (mask) {
-              const int lim = mask == 1 ? i : i + 1;  // keep j < lim
-              if (j + 0 >= lim) o.x = 0.f;
-              if (j + 1 >= lim) o.y = 0.f;
+#pragma unroll
+        for (int a = 0; a < MT; ++a)
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+            for (int b = 0; b < NT; ++b) {
+              const int i = i0 + row0 + 16 * a + g + 8 * hr, j = j0 + col0 + 8 * b + 2 * t;
+              if (i < M && j < N) epi.store(i, j, make_float2(c[a][b][2 * hr], c[a][b][2 * hr + 1]), l[a][hr][b]);
             }
-            *dst = o;
-          }
-        }
+      } else {
+#pragma unroll
+        for (int a = 0; a < MT; ++a)
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+            for (int b = 0; b < NT; ++b) {
+              const int i = i0 + row0 + 16 * a + g + 8 * hr, j = j0 + col0 + 8 * b + 2 * t;
+              if (i < M && j < N) epi.store(i, j, make_float2(c[a][b][2 * hr], c[a][b][2 * hr + 1]), epi.load(i, j));
+            }
       }
     }
   }
   __syncthreads();
 }
 
+template <int NB, class Epi>
+__device__ __forceinline__ void gemm_e(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, const Epi& epi) {
+  if (M <= 16) gemm_t<1, 128, NB>(A, B, M, N, K, sm, epi);
+  else gemm_t<4, 128, NB>(A, B, M, N, K, sm, epi);
+}
 template <int NB>
 __device__ __forceinline__ void gemm(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc,
                                      int mask, GemmSmemT<NB>& sm) {
-  if (M <= 16) gemm_t<1, 128, NB>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
-  else gemm_t<4, 128, NB>(Cp, ldc, A, B, M, N, K, alpha, acc, mask, sm);
+  gemm_e(A, B, M, N, K, sm, EpiStore{Cp, ldc, alpha, acc, mask});
 }
 
 // ------------------------------------------------------------------------- element-wise passes
@@ -468,7 +501,7 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
             },
             [&](int i, float4 v) { st4(GR + 4 * i, v); });
     __syncthreads();
-    if constexpr (NB >= 160) gemm_t<4, 160, NB>(GO, 160, mat(GL, D), mat(GR, D, true), 2 * C, 160, D, 1.f, false, 0, gsm);
+    if constexpr (NB >= 160) gemm_t<4, 160, NB>(mat(GL, D), mat(GR, D, true), 2 * C, 160, D, gsm, EpiStore{GO, 160, 1.f, false, 0});
     else gemm(GO, 160, mat(GL, D), mat(GR, D, true), 2 * C, 160, D, 1.f, false, 0, gsm);
   }
   // M strictly lower, P (times scale) lower with its diagonal, each row from its block's segment
@@ -747,6 +780,38 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
   }
 }
 
+// The state walk's outputs: E = Kt dS' (to e) and dDelta = P^T dO + E (to dd); the next dS' =
+// Diag(e^gamma) dS' + (Qt - P W)^T dO - W^T E.
+struct EpiE {
+  static constexpr bool kLoadsFirst = true;
+  float* e;
+  float* dd;
+  const float* pdo;
+  __device__ __forceinline__ float2 load(int i, int j) const {
+    return *reinterpret_cast<const float2*>(pdo + (size_t)i * D + j);
+  }
+  __device__ __forceinline__ void store(int i, int j, float2 v, float2 l) const {
+    *reinterpret_cast<float2*>(e + (size_t)i * D + j) = v;
+    *reinterpret_cast<float2*>(dd + (size_t)i * D + j) = make_float2(v.x + l.x, v.y + l.y);
+  }
+};
+struct EpiS {
+  static constexpr bool kLoadsFirst = true;
+  float* out;
+  const float* dsp;
+  const float* y;
+  const float* eg;
+  __device__ __forceinline__ float2 load(int i, int j) const {
+    const float2 a = *reinterpret_cast<const float2*>(dsp + (size_t)i * D + j);
+    const float2 b = *reinterpret_cast<const float2*>(y + (size_t)i * D + j);
+    const float e = eg[i];
+    return make_float2(fmaf(e, a.x, b.x), fmaf(e, a.y, b.y));
+  }
+  __device__ __forceinline__ void store(int i, int j, float2 v, float2 l) const {
+    *reinterpret_cast<float2*>(out + (size_t)i * D + j) = make_float2(l.x - v.x, l.y - v.y);
+  }
+};
+
 // One CTA per (sequence, head): from the last chunk to the first, with dS' the gradient of the
 // chunk's end state (d_final, or 0, for the last chunk):
 //   E = Kt dS',  dDelta = P^T dO + E,  dS = Diag(e^gamma) dS' + (Qt - P W)^T dO - W^T E.
@@ -788,20 +853,37 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_state_kernel(BwdParams P) {
     }
     const float* dsp = P.dsp + ((size_t)(slot0 + j) * H + h) * kStateElems;
     float* nxt = j > 0 ? P.dsp + ((size_t)(slot0 + j - 1) * H + h) * kStateElems : d_init;
-    gemm(e_buf, D, mat(pr + PR_KT, D), mat(dsp, D), C, D, D, 1.f, false, 0, gsm);
-    float* dd = P.dd + (size_t)it * kF;
-    ew<kB1>(kF4, [&](int i) { return add4(ld4(pr + PR_PDO + 4 * i), ld4(e_buf + 4 * i)); },
-              [&](int i, float4 v) { st4(dd + 4 * i, v); });
-    if (nxt) {
-      ew<kB1>(kS4,
-                [&](int i) { return add4(scl4(ld4(dsp + 4 * i), pr[PR_EG + ((4 * i) >> 7)]), ld4(pr + PR_Y + 4 * i)); },
-                [&](int i, float4 v) { st4(nxt + 4 * i, v); });
-      __syncthreads();
-      gemm(nxt, D, mat(pr + PR_W, D, true), mat(e_buf, D), D, D, C, -1.f, true, 0, gsm);
-    }
-    __syncthreads();
+    gemm_e(mat(pr + PR_KT, D), mat(dsp, D), C, D, D, gsm, EpiE{e_buf, P.dd + (size_t)it * kF, pr + PR_PDO});
+    if (nxt) gemm_e(mat(pr + PR_W, D, true), mat(e_buf, D), D, D, C, gsm, EpiS{nxt, dsp, pr + PR_Y, pr + PR_EG});
   }
 }
+
+// dT_b's second product, which also writes dT = dT_b diag(beta) (to da)
+struct EpiDtb {
+  static constexpr bool kLoadsFirst = false;
+  float* dtb;
+  float* da;
+  const float* beta;
+  __device__ __forceinline__ float2 load(int i, int j) const {
+    return *reinterpret_cast<const float2*>(dtb + (size_t)i * C + j);
+  }
+  __device__ __forceinline__ void store(int i, int j, float2 v, float2 l) const {
+    const float2 o = make_float2(v.x + l.x, v.y + l.y);
+    *reinterpret_cast<float2*>(dtb + (size_t)i * C + j) = o;
+    *reinterpret_cast<float2*>(da + (size_t)i * C + j) = make_float2(o.x * beta[j], o.y * beta[j + 1]);
+  }
+};
+// dv = T_b^T dDelta, rows of the chunk, as bf16 to the output
+struct EpiDv {
+  static constexpr bool kLoadsFirst = false;
+  __nv_bfloat16* dv;  // the chunk's first row of this head
+  int64_t row_stride;
+  int len;
+  __device__ __forceinline__ float2 load(int, int) const { return make_float2(0.f, 0.f); }
+  __device__ __forceinline__ void store(int i, int j, float2 v, float2) const {
+    if (i < len) *reinterpret_cast<__nv_bfloat162*>(dv + i * row_stride + j) = __floats2bfloat162_rn(v.x, v.y);
+  }
+};
 
 // Per chunk: the gradients of khat, qhat, log alpha and beta (to the partial buffers) and dv.
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, int64_t items) {
@@ -855,17 +937,12 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     }
     // dT_b = dDelta V^T + dW Kg^T;  dv = T_b^T dDelta;  dKg = T_b^T dW
     gemm(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
-    gemm(s + SC_DTB, C, mat(s + SC_DW, D), mat(s + SC_KG, D, true), C, C, D, 1.f, true, 0, gsm);
-    gemm(s + SC_D, D, mat(s + SC_TB, C, true), mat(dD, D), C, D, C, 1.f, false, 0, gsm);  // Delta is dead
-    ew<kB1>(ch.len * (D / 4), [&](int i) { return ld4(s + SC_D + 4 * i); },
-              [&](int i, float4 v) {
-                const int r = i >> 5, c4 = i & 31;
-                st_bf16x4(P.dv + ((size_t)(ch.t0 + r) * H + ch.h) * D + 4 * c4, v.x, v.y, v.z, v.w);
-              });
+    // with dT = dT_b diag(beta) (to DA)
+    gemm_e(mat(s + SC_DW, D), mat(s + SC_KG, D, true), C, C, D, gsm, EpiDtb{s + SC_DTB, s + SC_DA, s + SC_BETA});
+    gemm_e(mat(s + SC_TB, C, true), mat(dD, D), C, D, C, gsm,
+           EpiDv{P.dv + ((size_t)ch.t0 * H + ch.h) * D, (int64_t)H * D, ch.len});
     gemm(s + SC_DKG, D, mat(s + SC_TB, C, true), mat(s + SC_DW, D), C, D, C, 1.f, false, 0, gsm);
-    // dT = dT_b diag(beta); dbeta (columns) = colsum(dT_b o T); dA = strict_tril(-T^T dT T^T)
-    ew<kB1>(kQ4, [&](int i) { return mul4(ld4(s + SC_DTB + 4 * i), ld4(s + SC_BETA + ((4 * i) & (C - 1)))); },
-              [&](int i, float4 v) { st4(s + SC_DA + 4 * i, v); });
+    // dbeta (columns) = colsum(dT_b o T); dA = strict_tril(-T^T dT T^T)
     {
       // thread (column c, quarter q of the rows), the quarters added by shuffles
       const int c = tid >> 2, q = tid & 3;
