@@ -204,9 +204,10 @@ struct EpiStore {
 // three products hi hi, hi lo, lo hi accumulated in fp32 (about 2^-20 relative: fp32-level).  With
 // RM = 4 warp (wm, wn) holds rows 32 wm .. + 31 and columns NW / 4 wn .. + NW / 4 - 1 (2 x NW / 32
 // fragments), with RM = 1 (NW = 128) warp w columns 16 w .. + 15 (1 x 2).  M, N multiples of 4, K of
-// 8; operands 16-byte aligned with ld a multiple of 4.  All threads of the CTA call it; it ends with
-// a barrier.
-template <int RM, int NW, int NB, class Epi>
+// 8; operands 16-byte aligned with ld a multiple of 4.  X marks operands whose values are tf32
+// numbers already (bit 1: A, bit 2: B; bf16 inputs), whose low parts are zero: their products with
+// the other operand's high part are skipped.  All threads of the CTA call it; it ends with a barrier.
+template <int RM, int NW, int NB, class Epi, int X = 0>
 __device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, const Epi& epi) {
   static_assert(NW <= NB && (RM == 4 || NW == 128), "tile width");
   constexpr int BM = 16 * RM;
@@ -262,8 +263,8 @@ __device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, con
             sm100::tf32_split(b_at(sb, n, kk + t + 4), bh1, bl1);
 #pragma unroll
             for (int a = 0; a < MT; ++a) {
-              sm100::mma_tf32(c[a][b], ah[a], bl0, bl1);
-              sm100::mma_tf32(c[a][b], al[a], bh0, bh1);
+              if constexpr (!(X & 2)) sm100::mma_tf32(c[a][b], ah[a], bl0, bl1);
+              if constexpr (!(X & 1)) sm100::mma_tf32(c[a][b], al[a], bh0, bh1);
               sm100::mma_tf32(c[a][b], ah[a], bh0, bh1);
             }
           }
@@ -306,15 +307,15 @@ __device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, con
   __syncthreads();
 }
 
-template <int NB, class Epi>
+template <int X = 0, int NB, class Epi>
 __device__ __forceinline__ void gemm_e(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, const Epi& epi) {
-  if (M <= 16) gemm_t<1, 128, NB>(A, B, M, N, K, sm, epi);
-  else gemm_t<4, 128, NB>(A, B, M, N, K, sm, epi);
+  if (M <= 16) gemm_t<1, 128, NB, Epi, X>(A, B, M, N, K, sm, epi);
+  else gemm_t<4, 128, NB, Epi, X>(A, B, M, N, K, sm, epi);
 }
-template <int NB>
+template <int X = 0, int NB>
 __device__ __forceinline__ void gemm(float* Cp, int ldc, Mat A, Mat B, int M, int N, int K, float alpha, bool acc,
                                      int mask, GemmSmemT<NB>& sm) {
-  gemm_e(A, B, M, N, K, sm, EpiStore{Cp, ldc, alpha, acc, mask});
+  gemm_e<X>(A, B, M, N, K, sm, EpiStore{Cp, ldc, alpha, acc, mask});
 }
 
 // ------------------------------------------------------------------------- element-wise passes
@@ -775,8 +776,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
     if (tid < D) pr[PR_EG + tid] = s[SC_EG + tid];
     __syncthreads();
     gemm(s + SC_X, D, mat(s + SC_P, C), mat(pr + PR_W, D), C, D, C, -1.f, true, 0, gsm);
-    gemm(pr + PR_Y, D, mat(s + SC_X, D, true), mat(s + SC_DO, D), D, D, C, 1.f, false, 0, gsm);
-    gemm(pr + PR_PDO, D, mat(s + SC_P, C, true), mat(s + SC_DO, D), C, D, C, 1.f, false, 0, gsm);
+    gemm<2>(pr + PR_Y, D, mat(s + SC_X, D, true), mat(s + SC_DO, D), D, D, C, 1.f, false, 0, gsm);  // dO: bf16 values
+    gemm<2>(pr + PR_PDO, D, mat(s + SC_P, C, true), mat(s + SC_DO, D), C, D, C, 1.f, false, 0, gsm);
   }
 }
 
@@ -911,13 +912,13 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     const float* dSp = P.dsp + ((size_t)ch.slot * H + ch.h) * kStateElems;  // [k][v]
     const float* dD = P.dd + (size_t)it * kF;
     // Delta = T_b V - W S (W = T_b Kg as the prep kernel stored it)
-    gemm(s + SC_D, D, mat(s + SC_TB, C), mat(s + SC_V, D), C, D, C, 1.f, false, 0, gsm);
+    gemm<2>(s + SC_D, D, mat(s + SC_TB, C), mat(s + SC_V, D), C, D, C, 1.f, false, 0, gsm);  // V: bf16 values
     gemm(s + SC_D, D, mat(pr + PR_W, D), mat(S, D, true), C, D, D, -1.f, true, 0, gsm);
     // dKt = Delta dS'^T;  dQs = dO S^T;  dW = -dDelta S^T;  dP = tril(dO Delta^T)
     gemm(s + SC_DKT, D, mat(s + SC_D, D), mat(dSp, D, true), C, D, D, 1.f, false, 0, gsm);
-    gemm(s + SC_DQS, D, mat(s + SC_DO, D), mat(S, D), C, D, D, 1.f, false, 0, gsm);
+    gemm<1>(s + SC_DQS, D, mat(s + SC_DO, D), mat(S, D), C, D, D, 1.f, false, 0, gsm);  // dO: bf16 values
     gemm(s + SC_DW, D, mat(dD, D), mat(S, D), C, D, D, -1.f, false, 0, gsm);
-    gemm(s + SC_DP, C, mat(s + SC_DO, D), mat(s + SC_D, D, true), C, C, D, 1.f, false, 2, gsm);
+    gemm<1>(s + SC_DP, C, mat(s + SC_DO, D), mat(s + SC_D, D, true), C, C, D, 1.f, false, 2, gsm);
     // dgamma from the state: e^gamma_k sum_v S(k, v) dS'(k, v): thread k and half h of the v range
     // (reads of S coalesced over k, each thread's row of dS' read in order, 4 values a load)
     {
@@ -936,7 +937,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
       if (h == 0) s[SC_DGAM + k] = s[SC_EG + k] * (acc + s[SC_DGAM + k]);
     }
     // dT_b = dDelta V^T + dW Kg^T;  dv = T_b^T dDelta;  dKg = T_b^T dW
-    gemm(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
+    gemm<2>(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
     // with dT = dT_b diag(beta) (to DA)
     gemm_e(mat(s + SC_DW, D), mat(s + SC_KG, D, true), C, C, D, gsm, EpiDtb{s + SC_DTB, s + SC_DA, s + SC_BETA});
     gemm_e(mat(s + SC_TB, C, true), mat(dD, D), C, D, C, gsm,

@@ -48,11 +48,19 @@ def run_case(dev, x, seed, with_final=True, use_checkpoints=False):
     return got, ref
 
 
-def check_grads(got, ref, what):
+def check_grads(got, ref, what, sum_scale=None):
+    """Relative L2 per gradient; a gradient named in sum_scale (a sum whose terms cancel) is checked
+    element-wise against the sum of its terms' magnitudes instead: |got - ref| <= 1e-3 x scale."""
     worst = []
     for name in ("dq", "dk", "dv", "dg", "dbeta", "dA_log", "ddt_bias", "d_initial"):
         g = got[name].float().cpu().double().numpy()
         assert np.isfinite(g).all(), f"{what}: {name} not finite"
+        if sum_scale and name in sum_scale:
+            err = float(np.max(np.abs(g - ref[name]) / sum_scale[name]))
+            worst.append(f"{name} {err:.2e} of the terms' magnitude")
+            margins.note(f"backward {what} {name}: error / sum of |terms| {err:.2e} (tol 1e-03)")
+            assert err <= 1e-3, f"{what}: {name} error {err:.3e} of the sum of its terms' magnitudes"
+            continue
         err = rel_l2(g, ref[name])
         worst.append(f"{name} {err:.2e}")
         margins.note(f"backward {what} {name}: rel-L2 {err:.2e} (tol 1e-02)")
@@ -132,6 +140,23 @@ def test_bwd_saturated_gates_and_empty_documents(cuda_device):
     x = kda_inputs.make_random("t", [0, 150, 0, 0, 77], 2, seed=118, state_std=0.2)
     x.g[:, :, 0, :].fill_(60.0)
     check_grads(*run_case(cuda_device, x, 7), "saturated gate, empty documents")
+
+
+def test_bwd_near_collinear_keys(cuda_device):
+    """The forward's stress input (every key the same vector, beta = sigmoid(8), raw gate -12: alpha
+    close to 1, so (I + A) is close to I plus a strictly lower all-ones matrix) through the backward,
+    over six chunks with a ragged tail.  The queries are drawn at random here: with q = k, as in the
+    forward's case, every output depends on q only through khat . qhat = 1 and dq vanishes (the
+    oracle's is 1e-8), which a relative comparison cannot check."""
+    x = kda_inputs.make_collinear(336, seed=5)
+    x.q = torch.randn(x.q.shape, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    got, ref = run_case(cuda_device, x, 9)
+    # dA_log = sum over tokens and channels of dg (g + dt_bias) (the gate's chain rule); here those
+    # terms cancel to 2e-7 of their magnitudes (5.9e-7 against 3.1), below what any fp32 sum
+    # resolves, so dA_log is held to its terms' magnitude instead of to its own value
+    terms = ref["dg"].reshape(-1, x.num_heads, 128) * (x.g.double().numpy().reshape(-1, x.num_heads, 128)
+                                                       + x.dt_bias.double().numpy()[None])
+    check_grads(got, ref, "near-collinear keys", sum_scale={"dA_log": np.abs(terms).sum(axis=(0, 2))})
 
 
 def test_bwd_malformed_offsets_report_and_pass_the_state_gradient_through(cuda_device):

@@ -77,3 +77,18 @@ def test_adjoint_closed_form_frozen_state():
         np.testing.assert_allclose(g["d_initial"][n], want, rtol=1e-12, atol=1e-12)
     for name in ("dv", "dg", "dA_log", "ddt_bias"):
         assert np.all(g[name] == 0), name
+
+
+def test_gate_parameter_gradients_follow_from_dg():
+    """The gate is log alpha = lb sigmoid(e^A_log (g + dt_bias)): its derivatives in A_log and in
+    dt_bias are those in g times (g + dt_bias) and times 1, so dA_log[h] = sum_{t,c} dg (g + dt_bias)
+    and ddt_bias[h, c] = sum_t dg (the chain rule, independent of the adjoint's code)."""
+    x, d_out, d_final = _problem([9, 40, 17], 3, seed=104)
+    x.A_log.copy_(torch.tensor([-0.7, 0.0, 0.9]))
+    g = oracle.kda_bwd(x.q, x.k, x.v, x.g, x.beta, x.scale, x.A_log, x.dt_bias, x.lower_bound, d_out,
+                       initial_state=x.initial_state, d_final=d_final, cu_seqlens=x.cu_seqlens)
+    H = x.num_heads
+    dg = g["dg"].reshape(-1, H, 128)
+    gate = x.g.double().numpy().reshape(-1, H, 128) + x.dt_bias.double().numpy()[None]
+    np.testing.assert_allclose(g["dA_log"], (dg * gate).sum(axis=(0, 2)), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(g["ddt_bias"], dg.sum(axis=0), rtol=1e-10, atol=1e-14)
