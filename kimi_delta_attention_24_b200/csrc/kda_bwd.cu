@@ -150,11 +150,23 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Copies the GB_K x W slice (depth k0.., rows i0..) of an operand into shared memory, zero outside
 // rows x depth: element (i, k) is p[k * ld + i] (along i: to s[k][i], row length W + 8) or p[i * ld +
 // k] (kmaj: to s[i][k], row length LD_K).
-template <int W>
+// The threads that run a product together: the whole CTA of 256 threads, or one half of a CTA of 512
+// with its own named barrier.
+struct AllThreads {
+  __device__ static int tid() { return threadIdx.x; }
+  __device__ static void sync() { __syncthreads(); }
+};
+template <int kBar>
+struct HalfCta {
+  __device__ static int tid() { return threadIdx.x & (kBwdThreads - 1); }
+  __device__ static void sync() { asm volatile("bar.sync %0, %1;" ::"n"(kBar), "n"(kBwdThreads) : "memory"); }
+};
+
+template <int W, class Grp = AllThreads>
 __device__ __forceinline__ void slice_copy(float* s, const Mat& m, bool kmaj, int i0, int k0, int rows, int depth) {
   const int ld = m.ld;
   constexpr int kVec = GB_K * W / 4;
-  const int tid = threadIdx.x;
+  const int tid = Grp::tid();
 #pragma unroll
   for (int e = 0; e < (kVec + kBwdThreads - 1) / kBwdThreads; ++e) {
     const int idx = tid + e * kBwdThreads;
@@ -207,12 +219,12 @@ struct EpiStore {
 // 8; operands 16-byte aligned with ld a multiple of 4.  X marks operands whose values are tf32
 // numbers already (bit 1: A, bit 2: B; bf16 inputs), whose low parts are zero: their products with
 // the other operand's high part are skipped.  All threads of the CTA call it; it ends with a barrier.
-template <int RM, int NW, int NB, class Epi, int X = 0>
+template <int RM, int NW, int NB, class Epi, int X = 0, class Grp = AllThreads>
 __device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, const Epi& epi) {
   static_assert(NW <= NB && (RM == 4 || NW == 128), "tile width");
   constexpr int BM = 16 * RM;
   constexpr int MT = RM == 4 ? 2 : 1, NT = RM == 4 ? NW / 32 : 2;  // fragments per warp
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int tid = Grp::tid(), warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int wm = RM == 4 ? (warp & 1) : 0, wn = RM == 4 ? (warp >> 1) : warp;
   const int row0 = RM == 4 ? 32 * wm : 0, col0 = RM == 4 ? (NW / 4) * wn : 16 * wn;
   const bool a_kmaj = !A.t, b_kmaj = B.t;  // A(i, k) runs along k unless transposed; B(k, j) along j unless transposed
@@ -229,19 +241,19 @@ __device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, con
         for (int b = 0; b < NT; ++b)
 #pragma unroll
           for (int e = 0; e < 4; ++e) c[a][b][e] = 0.f;
-      slice_copy<BM>(sm.a[0], A, a_kmaj, i0, 0, M, K);
-      slice_copy<NW>(sm.b[0], B, b_kmaj, j0, 0, N, K);
+      slice_copy<BM, Grp>(sm.a[0], A, a_kmaj, i0, 0, M, K);
+      slice_copy<NW, Grp>(sm.b[0], B, b_kmaj, j0, 0, N, K);
       cp_async_commit();
       for (int ks = 0; ks < nsl; ++ks) {
         if (ks + 1 < nsl) {
-          slice_copy<BM>(sm.a[(ks + 1) & 1], A, a_kmaj, i0, (ks + 1) * GB_K, M, K);
-          slice_copy<NW>(sm.b[(ks + 1) & 1], B, b_kmaj, j0, (ks + 1) * GB_K, N, K);
+          slice_copy<BM, Grp>(sm.a[(ks + 1) & 1], A, a_kmaj, i0, (ks + 1) * GB_K, M, K);
+          slice_copy<NW, Grp>(sm.b[(ks + 1) & 1], B, b_kmaj, j0, (ks + 1) * GB_K, N, K);
           cp_async_commit();
           cp_async_wait<1>();
         } else {
           cp_async_wait<0>();
         }
-        __syncthreads();
+        Grp::sync();
         const float* sa = sm.a[ks & 1];
         const float* sb = sm.b[ks & 1];
         const int kn = K - ks * GB_K < GB_K ? K - ks * GB_K : GB_K;
@@ -269,7 +281,7 @@ __device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, con
             }
           }
         }
-        __syncthreads();  // the stage is refilled two slices on
+        Grp::sync();  // the stage is refilled two slices on
       }
       if constexpr (Epi::kLoadsFirst) {
         float2 l[MT][2][NT];
@@ -304,7 +316,7 @@ __device__ void gemm_t(Mat A, Mat B, int M, int N, int K, GemmSmemT<NB>& sm, con
       }
     }
   }
-  __syncthreads();
+  Grp::sync();
 }
 
 template <int X = 0, int NB, class Epi>
@@ -818,9 +830,11 @@ struct EpiS {
 //   E = Kt dS',  dDelta = P^T dO + E,  dS = Diag(e^gamma) dS' + (Qt - P W)^T dO - W^T E.
 // dS' of chunk j is kept in the chunk's slot (the input of bwd_grad_kernel); the dS of chunk 0 is
 // the initial state's gradient.
-__global__ void __launch_bounds__(kBwdThreads) bwd_state_kernel(BwdParams P) {
+// 512 threads: two groups of 8 warps, each with its own staging buffer, run the two halves of each
+// product at once (E by column halves, the next dS' by row halves).
+__global__ void __launch_bounds__(2 * kBwdThreads, 1) bwd_state_kernel(BwdParams P) {
   extern __shared__ float4 smem4[];
-  GemmSmem& gsm = *reinterpret_cast<GemmSmem*>(smem4);
+  GemmSmem* gsm = reinterpret_cast<GemmSmem*>(smem4);  // [2]
   const FwdParams& p = P.f;
   const int H = p.num_heads;
   const int n = blockIdx.x / H, h = blockIdx.x - n * H;
@@ -838,24 +852,42 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_state_kernel(BwdParams P) {
               [&](int i, float4 v) { st4(dst + 4 * i, v); });
   };
   if (nch == 0) {
-    if (d_init) copy_final(d_init);
+    if (d_init && tid < kBwdThreads) copy_final(d_init);
     return;
   }
-  copy_final(P.dsp + ((size_t)(slot0 + nch - 1) * H + h) * kStateElems);
+  if (tid < kBwdThreads) copy_final(P.dsp + ((size_t)(slot0 + nch - 1) * H + h) * kStateElems);
   __syncthreads();
+  const bool hi = tid >= kBwdThreads;  // the second group
   for (int64_t j = nch - 1; j >= 0; --j) {
     const int64_t it = (c0 + j) * H + h;
     const float* pr = P.prep + (size_t)it * kPrepFloats;
     if (j > 0) {
       // the previous chunk's factors into L2 while this one runs
       const char* nx = reinterpret_cast<const char*>(P.prep + (size_t)(it - H) * kPrepFloats);
-      for (int l = tid; l < (int)(PR_M * sizeof(float) / 128); l += kBwdThreads)
+      for (int l = tid; l < (int)(PR_M * sizeof(float) / 128); l += 2 * kBwdThreads)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + (size_t)l * 128));
     }
     const float* dsp = P.dsp + ((size_t)(slot0 + j) * H + h) * kStateElems;
     float* nxt = j > 0 ? P.dsp + ((size_t)(slot0 + j - 1) * H + h) * kStateElems : d_init;
-    gemm_e(mat(pr + PR_KT, D), mat(dsp, D), C, D, D, gsm, EpiE{e_buf, P.dd + (size_t)it * kF, pr + PR_PDO});
-    if (nxt) gemm_e(mat(pr + PR_W, D, true), mat(e_buf, D), D, D, C, gsm, EpiS{nxt, dsp, pr + PR_Y, pr + PR_EG});
+    float* dd = P.dd + (size_t)it * kF;
+    // E = Kt dS' and dDelta, columns 64 g .. + 63 by group g
+    if (!hi)
+      gemm_t<4, 64, 128, EpiE, 0, HalfCta<1>>(mat(pr + PR_KT, D), mat(dsp, D), C, 64, D, gsm[0],
+                                             EpiE{e_buf, dd, pr + PR_PDO});
+    else
+      gemm_t<4, 64, 128, EpiE, 0, HalfCta<2>>(mat(pr + PR_KT, D), mat(dsp + 64, D), C, 64, D, gsm[1],
+                                             EpiE{e_buf + 64, dd + 64, pr + PR_PDO + 64});
+    __syncthreads();
+    // the next dS', rows 64 g .. + 63 by group g
+    if (nxt) {
+      if (!hi)
+        gemm_t<4, 128, 128, EpiS, 0, HalfCta<1>>(mat(pr + PR_W, D, true), mat(e_buf, D), C, D, C, gsm[0],
+                                                EpiS{nxt, dsp, pr + PR_Y, pr + PR_EG});
+      else
+        gemm_t<4, 128, 128, EpiS, 0, HalfCta<2>>(mat(pr + PR_W + 64, D, true), mat(e_buf, D), C, D, C, gsm[1],
+                                                EpiS{nxt + 64 * D, dsp + 64 * D, pr + PR_Y + 64 * D, pr + PR_EG + 64});
+    }
+    __syncthreads();
   }
 }
 
@@ -1242,13 +1274,13 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
         (e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGradSmem)) !=
             cudaSuccess ||
         (e = cudaFuncSetAttribute(bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)sizeof(GemmSmem))) != cudaSuccess)
+                                  (int)(2 * sizeof(GemmSmem)))) != cudaSuccess)
       return e;
     // the rest of each SM's 256 KB as L1: shared memory for exactly two CTAs (one for the walk)
     auto carve = [](size_t bytes, int ctas) { return (int)((ctas * (bytes + 1024) * 100 + 232447) / 233472); };
     if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve(kChunkSmem, 2))) != cudaSuccess ||
         (e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve(kGradSmem, 2))) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(bwd_state_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve(sizeof(GemmSmem), 1))) != cudaSuccess)
+        (e = cudaFuncSetAttribute(bwd_state_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carve(2 * sizeof(GemmSmem), 1))) != cudaSuccess)
       return e;
     attr_done[dev] = true;
   }
@@ -1259,7 +1291,7 @@ cudaError_t launch_bwd(const FwdParams& f, const __nv_bfloat16* d_out, const flo
     bwd_prep_kernel<<<(unsigned)grid, kBwdThreads, kChunkSmem, stream>>>(P, items);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  bwd_state_kernel<<<(unsigned)units, kBwdThreads, sizeof(GemmSmem), stream>>>(P);  // also when every document is empty
+  bwd_state_kernel<<<(unsigned)units, 2 * kBwdThreads, 2 * sizeof(GemmSmem), stream>>>(P);  // also when every document is empty
   if ((e = cudaGetLastError()) != cudaSuccess || tokens == 0) return e;
   bwd_grad_kernel<<<(unsigned)grid, kBwdThreads, kGradSmem, stream>>>(P, items);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
