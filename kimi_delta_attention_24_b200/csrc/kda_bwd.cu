@@ -1100,40 +1100,54 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t to
   float ddt[4] = {0.f, 0.f, 0.f, 0.f}, dA = 0.f;
   const int64_t t_begin = (int64_t)blockIdx.x * tokens_per_cta;
   const int64_t t_end = min(t_begin + tokens_per_cta, tokens);
-  for (int64_t t = t_begin + warp; t < t_end; t += 8) {
-    const size_t row = (size_t)t * H + h;
-    const float* base = P.part + row * D + 4 * lane;
-    const float4 a4 = *reinterpret_cast<const float4*>(base);
-    const float4 b4 = *reinterpret_cast<const float4*>(base + (size_t)rows_total * D);
-    const float4 c4 = *reinterpret_cast<const float4*>(base + 2 * (size_t)rows_total * D);
-    const float gq[4] = {a4.x, a4.y, a4.z, a4.w}, gk[4] = {b4.x, b4.y, b4.z, b4.w};
-    const float ga[4] = {c4.x, c4.y, c4.z, c4.w};
-    const float gb = P.part[3 * (size_t)rows_total * D + row];
-    // dq, dk: (dxhat - xhat (xhat . dxhat)) / n
+  // a token per warp at a time, all of its loads issued before any store (the outputs may alias
+  // nothing the compiler can prove, so it would not hoist a load above an earlier store)
+  constexpr int kTok = 1;  // tokens per warp at a time (2 measured slower: 128 registers, fewer CTAs)
+  for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += 8 * kTok) {
+    float4 a4[kTok], b4[kTok], c4[kTok], q4[kTok], k4[kTok], g4[kTok];
+    float gb[kTok], bb[kTok];
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const float4 x4 = ld_bf16x4((which == 0 ? p.q : p.k) + row * D + 4 * lane);
-      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
-      float ss = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const float nrm = sqrtf(ss + kL2Eps);
-      const float* gx = which == 0 ? gq : gk;
-      float dot = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dot += (xv[j] / nrm) * gx[j];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      float r[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) r[j] = (gx[j] - (xv[j] / nrm) * dot) / nrm;
-      st_bf16x4((which == 0 ? P.dq : P.dk) + row * D + 4 * lane, r[0], r[1], r[2], r[3]);
+    for (int u = 0; u < kTok; ++u) {
+      const int64_t t = t0 + 8 * u;
+      const size_t row = (size_t)(t < t_end ? t : t0) * H + h;
+      const float* base = P.part + row * D + 4 * lane;
+      a4[u] = *reinterpret_cast<const float4*>(base);
+      b4[u] = *reinterpret_cast<const float4*>(base + (size_t)rows_total * D);
+      c4[u] = *reinterpret_cast<const float4*>(base + 2 * (size_t)rows_total * D);
+      gb[u] = P.part[3 * (size_t)rows_total * D + row];
+      q4[u] = ld_bf16x4(p.q + row * D + 4 * lane);
+      k4[u] = ld_bf16x4(p.k + row * D + 4 * lane);
+      g4[u] = ld_bf16x4(p.g + row * D + 4 * lane);
+      bb[u] = __bfloat162float(p.beta[row]);
     }
-    // dg through the gate (log alpha = lower_bound sigmoid(x), x = e^{A_log} (g + dt_bias)); the sums
-    // for dt_bias and A_log
-    {
-      const float4 g4 = ld_bf16x4(p.g + row * D + 4 * lane);
-      const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+    for (int u = 0; u < kTok; ++u) {
+      const int64_t t = t0 + 8 * u;
+      if (t >= t_end) break;
+      const size_t row = (size_t)t * H + h;
+      // dq, dk: (dxhat - xhat (xhat . dxhat)) / n
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const float4 x4 = which == 0 ? q4[u] : k4[u];
+        const float4 g = which == 0 ? a4[u] : b4[u];
+        const float xv[4] = {x4.x, x4.y, x4.z, x4.w}, gx[4] = {g.x, g.y, g.z, g.w};
+        float ss = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float nrm = sqrtf(ss + kL2Eps);
+        float dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dot += (xv[j] / nrm) * gx[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        float r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[j] = (gx[j] - (xv[j] / nrm) * dot) / nrm;
+        st_bf16x4((which == 0 ? P.dq : P.dk) + row * D + 4 * lane, r[0], r[1], r[2], r[3]);
+      }
+      // dg through the gate (log alpha = lower_bound sigmoid(x), x = e^{A_log} (g + dt_bias)); the
+      // sums for dt_bias and A_log
+      const float gv[4] = {g4[u].x, g4[u].y, g4[u].z, g4[u].w}, ga[4] = {c4[u].x, c4[u].y, c4[u].z, c4[u].w};
       float dg[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -1145,10 +1159,10 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams P, int64_t to
         dA = fmaf(dx, x, dA);
       }
       st_bf16x4(P.dg + row * D + 4 * lane, dg[0], dg[1], dg[2], dg[3]);
-    }
-    if (lane == 0) {
-      const float b = sigmoid_acc(__bfloat162float(p.beta[row]));
-      P.dbeta[row] = __float2bfloat16_rn(gb * b * (1.f - b));
+      if (lane == 0) {
+        const float b = sigmoid_acc(bb[u]);
+        P.dbeta[row] = __float2bfloat16_rn(gb[u] * b * (1.f - b));
+      }
     }
   }
 #pragma unroll
