@@ -263,9 +263,9 @@ kda_status_t kda_fwd_checkpointed(const void* q, const void* k, const void* v, c
 
 /* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): the forward's
  * workspace and the checkpoints and output it writes (used when the call is given no checkpoints),
- * per (64-token chunk, head) the factors of the reverse state walk (160 KB) and dDelta (32 KB), one
+ * per (64-token chunk, head) the factors of the reverse state walk (192.5 KB) and dDelta (32 KB), one
  * 128 x 128 state gradient per chunk slot and head, per-token partials (3 x 128 + 1 fp32 per token
- * and head), and a scratch of 624 KB per CTA of the chunk-parallel kernels (at most 296).  Depends
+ * and head), and a scratch of 466 KB per CTA of the chunk-parallel kernels (at most 296).  Depends
  * only on its arguments; its first 256 bytes hold the status word read by kda_read_device_status. */
 size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 
@@ -282,8 +282,9 @@ size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t n
  *                [batch, seqlen, H] (w.r.t. the raw beta, before the sigmoid; dg w.r.t. the raw gate)
  *   dA_log fp32 [H], ddt_bias fp32 [H, K]  (overwritten: zeroed, then summed over all tokens)
  *   d_initial    fp32 [N, H, K, V] or NULL (not written)
- * In the chunked form, on CUDA cores in fp32: (without checkpoints) the checkpointing forward; then
- * per 64-token chunk, in parallel, the chunk's factors (gate, norms, decay-weighted Gram products,
+ * In the chunked form, fp32 throughout (products on the tensor cores with tf32 operands split into
+ * high and low parts, fp32-level): (without checkpoints) the checkpointing forward; then per
+ * 64-token chunk, in parallel, the chunk's factors (gate, norms, decay-weighted Gram products,
  * (I + A)^{-1}); per (sequence, head), from the last chunk to the first, the gradient of the state at
  * every chunk boundary; per chunk, in parallel, the gradients of the chunk's inputs; and a last
  * kernel for the derivatives of the in-kernel transforms.  Gradient pointers are 16-byte aligned

@@ -24,9 +24,10 @@
 //
 // Launches: the checkpointing forward when no chunk-start states are given (the split path, which
 // stores S at every chunk start); bwd_prep_kernel (chunk-parallel: recomputes a chunk's factors and
-// stores W, Kt, P^T dO, (Qt - P W)^T dO and e^gamma); bwd_state_kernel (one CTA per (sequence, head),
-// chunks last to first: dDelta and the state gradient at every chunk boundary); bwd_grad_kernel
-// (chunk-parallel: recomputes the factors and forms the gradients above); bwd_finish_kernel (the
+// stores W, Kt, P^T dO, (Qt - P W)^T dO, e^gamma, M and T); bwd_state_kernel (one CTA per (sequence,
+// head), chunks last to first: dDelta and the state gradient at every chunk boundary);
+// bwd_grad_kernel (chunk-parallel: recomputes the element-wise factors, reads M and T, and forms the
+// gradients above); bwd_finish_kernel (the
 // transforms, and dA_log / dt_bias summed with one atomic per value per CTA).  The chunk-parallel
 // kernels are persistent; each CTA keeps one chunk's intermediates in its own global scratch (mostly
 // held by L2).  The products run on the tensor cores (mma.sync tf32 with hi/lo operands: fp32-level
