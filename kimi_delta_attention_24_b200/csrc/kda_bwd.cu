@@ -24,9 +24,9 @@
 //
 // Launches: the checkpointing forward when no chunk-start states are given (the split path, which
 // stores S at every chunk start); bwd_prep_kernel (chunk-parallel: recomputes a chunk's factors and
-// stores W, Kt, P^T dO, (Qt - P W)^T dO, e^gamma, M and T); bwd_state_kernel (one CTA per (sequence,
+// stores W, Kt, P^T dO, (Qt - P W)^T dO, e^gamma, M, T and T_b); bwd_state_kernel (one CTA per (sequence,
 // head), chunks last to first: dDelta and the state gradient at every chunk boundary);
-// bwd_grad_kernel (chunk-parallel: recomputes the element-wise factors, reads M and T, and forms the
+// bwd_grad_kernel (chunk-parallel: recomputes the element-wise factors, reads M, T and T_b, and forms the
 // gradients above); bwd_finish_kernel (the
 // transforms, and dA_log / dt_bias summed with one atomic per value per CTA).  The chunk-parallel
 // kernels are persistent; each CTA keeps one chunk's intermediates in its own global scratch (mostly
@@ -53,14 +53,15 @@ constexpr int PR_Y = 3 * kF;       // (Qt - P W)^T dO [128][128]
 constexpr int PR_EG = 3 * kF + D * D;  // e^gamma [128]
 constexpr int PR_M = PR_EG + D;        // M [64][64] (strict lower) and T = (I + A)^{-1} [64][64], for the gradient kernel
 constexpr int PR_T = PR_M + kQ;
-constexpr int kPrepFloats = PR_T + kQ;
+constexpr int PR_TB = PR_T + kQ;       // T_b = T diag(beta) [64][64]
+constexpr int kPrepFloats = PR_TB + kQ;
 
 // per-CTA scratch (floats).  Each kernel reuses buffers once they are dead, so that the scratch of
 // all its CTAs (at most 448 KB each) mostly stays in L2.  The prep kernel: the Gram product's operands and
 // output in V .. DKG (V is not needed there), Qt - P W in V after them.  The gradient kernel: dv's
 // temporary and the gated products' partial sums in D (Delta), their depth-16 right operands in DW,
 // the transposed ones' output in KG, the 128 x 128 temporary in dO and V, the product T^T dA in DTB;
-// M and T read from the prep kernel's output.
+// M, T and T_b read from the prep kernel's output.
 constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_DO = 4 * kF, SC_V = 5 * kF;
 constexpr int SC_W = 6 * kF, SC_D = 7 * kF, SC_DKT = 8 * kF, SC_DQS = 9 * kF, SC_DW = 10 * kF, SC_DKG = 11 * kF;
 constexpr int SC_GL = SC_V, SC_GR = SC_D, SC_GO = SC_DQS + kF / 2;  // prep: 128 x 128, 160 x 128, 128 x 160
@@ -409,13 +410,13 @@ __device__ Chunk locate(const BwdParams& P, int64_t item) {
 //   kh, qh, Gamma (G), beta, e^gamma, Kg; V and dO (fp32, rows past the chunk's end zero).
 // need_v: also V (the gradient kernel).
 // solve: also the Gram blocks and (I + A)^{-1}: P (lower, with scale) and T_b into s, M (strict
-// lower) and T = (I + A)^{-1} to Mout and Tout (the prep kernel's output); otherwise only the
-// element-wise factors (the gradient kernel reads M and T from there).  sT, sA: the solve's two
+// lower), T = (I + A)^{-1} and T_b to Mout, Tout and TBout (the prep kernel's output); otherwise
+// only the element-wise factors (the gradient kernel reads M, T and T_b from there).  sT, sA: the solve's two
 // 64 x 65 shared-memory tiles.
 template <int NB>
 __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, bool need_v, bool solve, GemmSmemT<NB>& gsm,
                               float* sT /* shared 64 x 65 */, float* sA /* shared 64 x 65 */, float* Mout = nullptr,
-                              float* Tout = nullptr) {
+                              float* Tout = nullptr, float* TBout = nullptr) {
   const FwdParams& p = P.f;
   const int H = p.num_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -603,6 +604,7 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
             [&](int i, F4x2 v) {
               st4(Tout + 4 * i, v.a);
               st4(s + SC_TB + 4 * i, v.b);
+              st4(TBout + 4 * i, v.b);
             });
   __syncthreads();
 }
@@ -771,7 +773,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
     float* pr = P.prep + (size_t)it * kPrepFloats;
-    chunk_factors(P, ch, s, false, true, gsm, sT, sA, pr + PR_M, pr + PR_T);
+    chunk_factors(P, ch, s, false, true, gsm, sT, sA, pr + PR_M, pr + PR_T, pr + PR_TB);
     // W = T_b Kg (to the output); Kt = khat e^{gamma - Gamma}; X = Qt - P W
     gemm(pr + PR_W, D, mat(s + SC_TB, C), mat(s + SC_KG, D), C, D, C, 1.f, false, 0, gsm);
     const float* gam = s + SC_G + (C - 1) * D;
@@ -934,18 +936,16 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
     chunk_factors(P, ch, s, true, false, gsm, nullptr, nullptr);
-    // M and T = (I + A)^{-1} as the prep kernel stored them; T_b = T diag(beta)
+    // M, T = (I + A)^{-1} and T_b = T diag(beta) as the prep kernel stored them
     const float* pr = P.prep + (size_t)it * kPrepFloats;
     const float* Mp = pr + PR_M;
     const float* Tp = pr + PR_T;
-    ew<kB1>(kQ4, [&](int i) { return mul4(ld4(Tp + 4 * i), ld4(s + SC_BETA + ((4 * i) & (C - 1)))); },
-            [&](int i, float4 v) { st4(s + SC_TB + 4 * i, v); });
-    __syncthreads();
+    const float* TBp = pr + PR_TB;
     const float* S = P.ckpt + ((size_t)ch.slot * H + ch.h) * kStateElems;   // S^T [v][k]: S(k, v) = S[v * 128 + k]
     const float* dSp = P.dsp + ((size_t)ch.slot * H + ch.h) * kStateElems;  // [k][v]
     const float* dD = P.dd + (size_t)it * kF;
     // Delta = T_b V - W S (W = T_b Kg as the prep kernel stored it)
-    gemm<2>(s + SC_D, D, mat(s + SC_TB, C), mat(s + SC_V, D), C, D, C, 1.f, false, 0, gsm);  // V: bf16 values
+    gemm<2>(s + SC_D, D, mat(TBp, C), mat(s + SC_V, D), C, D, C, 1.f, false, 0, gsm);  // V: bf16 values
     gemm(s + SC_D, D, mat(pr + PR_W, D), mat(S, D, true), C, D, D, -1.f, true, 0, gsm);
     // dKt = Delta dS'^T;  dQs = dO S^T;  dW = -dDelta S^T;  dP = tril(dO Delta^T)
     gemm(s + SC_DKT, D, mat(s + SC_D, D), mat(dSp, D, true), C, D, D, 1.f, false, 0, gsm);
@@ -973,9 +973,9 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     gemm<2>(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
     // with dT = dT_b diag(beta) (to DA)
     gemm_e(mat(s + SC_DW, D), mat(s + SC_KG, D, true), C, C, D, gsm, EpiDtb{s + SC_DTB, s + SC_DA, s + SC_BETA});
-    gemm_e(mat(s + SC_TB, C, true), mat(dD, D), C, D, C, gsm,
+    gemm_e(mat(TBp, C, true), mat(dD, D), C, D, C, gsm,
            EpiDv{P.dv + ((size_t)ch.t0 * H + ch.h) * D, (int64_t)H * D, ch.len});
-    gemm(s + SC_DKG, D, mat(s + SC_TB, C, true), mat(s + SC_DW, D), C, D, C, 1.f, false, 0, gsm);
+    gemm(s + SC_DKG, D, mat(TBp, C, true), mat(s + SC_DW, D), C, D, C, 1.f, false, 0, gsm);
     // dbeta (columns) = colsum(dT_b o T); dA = strict_tril(-T^T dT T^T)
     {
       // thread (column c, quarter q of the rows), the quarters added by shuffles
