@@ -263,9 +263,10 @@ kda_status_t kda_fwd_checkpointed(const void* q, const void* k, const void* v, c
 
 /* Bytes of device workspace kda_bwd needs for (total tokens T, heads H, sequences N): the forward's
  * workspace and the checkpoints and output it writes (used when the call is given no checkpoints),
- * per (64-token chunk, head) the factors of the reverse state walk (208.5 KB) and dDelta (32 KB), one
- * 128 x 128 state gradient per chunk slot and head, per-token partials (3 x 128 + 1 fp32 per token
- * and head), and a scratch of 466 KB per CTA of the chunk-parallel kernels (at most 296).  Depends
+ * per (64-token chunk, head) the chunk's factors for the reverse state walk and the gradient kernel
+ * (336.5 KB) and dDelta (32 KB), one 128 x 128 state gradient per chunk slot and head, per-token
+ * partials (3 x 128 + 1 fp32 per token and head), and a scratch of 369 KB per CTA of the
+ * chunk-parallel kernels (at most 296).  Depends
  * only on its arguments; its first 256 bytes hold the status word read by kda_read_device_status. */
 size_t kda_bwd_workspace_size(int64_t total_tokens, int32_t num_heads, int32_t num_seqs);
 

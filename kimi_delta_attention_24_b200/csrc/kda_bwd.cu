@@ -23,15 +23,15 @@
 // followed by the derivatives of the in-kernel transforms (L2 norms, sigmoid of beta, safe gate).
 //
 // Launches: the checkpointing forward when no chunk-start states are given (the split path, which
-// stores S at every chunk start); bwd_prep_kernel (chunk-parallel: recomputes a chunk's factors and
-// stores W, Kt, P^T dO, (Qt - P W)^T dO, e^gamma, M, T and T_b); bwd_state_kernel (one CTA per (sequence,
-// head), chunks last to first: dDelta and the state gradient at every chunk boundary);
-// bwd_grad_kernel (chunk-parallel: recomputes the element-wise factors, reads M, T and T_b, and forms the
-// gradients above); bwd_finish_kernel (the
-// transforms, and dA_log / dt_bias summed with one atomic per value per CTA).  The chunk-parallel
-// kernels are persistent; each CTA keeps one chunk's intermediates in its own global scratch (mostly
-// held by L2).  The products run on the tensor cores (mma.sync tf32 with hi/lo operands: fp32-level
-// accuracy), the element-wise work in fp32 on CUDA cores.
+// stores S at every chunk start); bwd_prep_kernel (chunk-parallel: forms a chunk's factors and stores
+// W, Kt, P^T dO, (Qt - P W)^T dO, e^gamma, M, T, T_b, khat, qhat, Gamma and Kg); bwd_state_kernel
+// (one CTA per (sequence, head), chunks last to first: dDelta and the state gradient at every chunk
+// boundary); bwd_grad_kernel (chunk-parallel: reads the chunk's factors from the prep output and
+// forms the gradients above); bwd_finish_kernel (the transforms, and dA_log / dt_bias summed with
+// one atomic per value per CTA).  The chunk-parallel kernels are persistent; each CTA keeps one
+// chunk's intermediates in its own global scratch (mostly held by L2).  The products run on the
+// tensor cores (mma.sync tf32 with hi/lo operands: fp32-level accuracy), the element-wise work in
+// fp32 on CUDA cores.
 #include "kda_common.cuh"
 #include "sm100.cuh"
 
@@ -54,23 +54,27 @@ constexpr int PR_EG = 3 * kF + D * D;  // e^gamma [128]
 constexpr int PR_M = PR_EG + D;        // M [64][64] (strict lower) and T = (I + A)^{-1} [64][64], for the gradient kernel
 constexpr int PR_T = PR_M + kQ;
 constexpr int PR_TB = PR_T + kQ;       // T_b = T diag(beta) [64][64]
-constexpr int kPrepFloats = PR_TB + kQ;
+constexpr int PR_KH = PR_TB + kQ;      // khat, qhat, Gamma, Kg [64][128] each: the chunk's element-wise factors
+constexpr int PR_QH = PR_KH + kF, PR_G = PR_QH + kF, PR_KG = PR_G + kF;
+constexpr int kPrepFloats = PR_KG + kF;
 
-// per-CTA scratch (floats).  Each kernel reuses buffers once they are dead, so that the scratch of
-// all its CTAs (at most 448 KB each) mostly stays in L2.  The prep kernel: the Gram product's operands and
-// output in V .. DKG (V is not needed there), Qt - P W in V after them.  The gradient kernel: dv's
-// temporary and the gated products' partial sums in D (Delta), their depth-16 right operands in DW,
-// the transposed ones' output in KG, the 128 x 128 temporary in dO and V, the product T^T dA in DTB;
-// M, T and T_b read from the prep kernel's output.
-constexpr int SC_KH = 0, SC_QH = kF, SC_G = 2 * kF, SC_KG = 3 * kF, SC_DO = 4 * kF, SC_V = 5 * kF;
-constexpr int SC_W = 6 * kF, SC_D = 7 * kF, SC_DKT = 8 * kF, SC_DQS = 9 * kF, SC_DW = 10 * kF, SC_DKG = 11 * kF;
+// per-CTA scratch (floats).  The chunk's element-wise factors (khat, qhat, Gamma, Kg) live in the
+// prep kernel's output, which both chunk kernels read.  Each kernel reuses buffers once they are dead,
+// so that the scratch of all its CTAs (at most 370 KB each) mostly stays in L2.  The prep kernel: the
+// Gram product's operands and output in V .. DKG (V is not needed there), Qt - P W in V after them.
+// The gradient kernel: dv's temporary and the gated products' partial sums in D (Delta), their
+// depth-16 right operands in DW, the 128 x 128 temporary in dO and V, the product T^T dA in DTB.
+constexpr int SC_L = 0;  // the gradient kernel: the transposed gated products' output
+constexpr int SC_DO = kF, SC_V = 2 * kF, SC_W = 3 * kF, SC_D = 4 * kF, SC_DKT = 5 * kF, SC_DQS = 6 * kF;
+constexpr int SC_DW = 7 * kF, SC_DKG = 8 * kF;
 constexpr int SC_GL = SC_V, SC_GR = SC_D, SC_GO = SC_DQS + kF / 2;  // prep: 128 x 128, 160 x 128, 128 x 160
 constexpr int SC_X = SC_V;                                          // prep: Qt - P W
-constexpr int SC_P = 12 * kF, SC_TB = SC_P + kQ;  // prep: M and T go straight to its output
+constexpr int SC_P = 9 * kF, SC_TB = SC_P + kQ;  // prep: M, T and T_b go straight to its output
 constexpr int SC_DA = SC_TB + kQ, SC_DP = SC_DA + kQ;  // dA (then dM) and dP adjacent: [dM; dP] is 128 x 64
 constexpr int SC_DTB = SC_DP + kQ;
 constexpr int SC_BETA = SC_DTB + kQ, SC_EG = SC_BETA + C, SC_DGAM = SC_EG + D, SC_DB = SC_DGAM + D;
 static_assert(SC_GO + 160 * D <= SC_P, "the Gram product's output ends before P");
+static_assert(SC_DO + kF == SC_V, "dO and V adjacent: the gradient kernel's 128 x 128 temporary");
 constexpr int kScratchFloats = SC_DB + C + 64;
 
 struct BwdParams {
@@ -406,15 +410,22 @@ __device__ Chunk locate(const BwdParams& P, int64_t item) {
   return c;
 }
 
-// The factors of a chunk that do not involve the state, into the CTA's scratch s:
-//   kh, qh, Gamma (G), beta, e^gamma, Kg; V and dO (fp32, rows past the chunk's end zero).
-// need_v: also V (the gradient kernel).
-// solve: also the Gram blocks and (I + A)^{-1}: P (lower, with scale) and T_b into s, M (strict
-// lower), T = (I + A)^{-1} and T_b to Mout, Tout and TBout (the prep kernel's output); otherwise
-// only the element-wise factors (the gradient kernel reads M, T and T_b from there).  sT, sA: the solve's two
-// 64 x 65 shared-memory tiles.
+// Where a chunk's element-wise factors live (the prep kernel's output).
+struct Fac {
+  float* kh;
+  float* qh;
+  float* G;
+  float* kg;
+};
+__device__ __forceinline__ Fac fac_of(float* pr) { return Fac{pr + PR_KH, pr + PR_QH, pr + PR_G, pr + PR_KG}; }
+
+// The factors of a chunk that do not involve the state (the prep kernel): khat, qhat, Gamma and Kg
+// to F; beta, e^gamma and dO (fp32, rows past the chunk's end zero) into the CTA's scratch s; the
+// Gram blocks and (I + A)^{-1}: P (lower, with scale) and T_b into s, M (strict lower),
+// T = (I + A)^{-1} and T_b to Mout, Tout and TBout (the prep kernel's output, which the gradient
+// kernel reads).  sT, sA: the solve's two 64 x 65 shared-memory tiles.
 template <int NB>
-__device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, bool need_v, bool solve, GemmSmemT<NB>& gsm,
+__device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, const Fac& F, GemmSmemT<NB>& gsm,
                               float* sT /* shared 64 x 65 */, float* sA /* shared 64 x 65 */, float* Mout = nullptr,
                               float* Tout = nullptr, float* TBout = nullptr) {
   const FwdParams& p = P.f;
@@ -426,20 +437,19 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   const float dts[4] = {dt.x, dt.y, dt.z, dt.w};
   // prologue: warp per row, lane per 4 channels; each warp loads two rows before it stores any
   for (int r0 = warp; r0 < C; r0 += 2 * (kBwdThreads / 32)) {
-    float4 k4[2], q4[2], g4[2], v4[2], o4[2];
+    float4 k4[2], q4[2], g4[2], o4[2];
     float br[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int r = r0 + u * (kBwdThreads / 32);
       const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      k4[u] = q4[u] = g4[u] = v4[u] = o4[u] = z;
+      k4[u] = q4[u] = g4[u] = o4[u] = z;
       br[u] = 0.f;
       if (r < len) {
         const size_t row = (size_t)(ch.t0 + r) * H + h;
         k4[u] = ld_bf16x4(p.k + row * D + 4 * lane);
         q4[u] = ld_bf16x4(p.q + row * D + 4 * lane);
         g4[u] = ld_bf16x4(p.g + row * D + 4 * lane);
-        if (need_v) v4[u] = ld_bf16x4(p.v + row * D + 4 * lane);
         o4[u] = ld_bf16x4(P.d_out + row * D + 4 * lane);
         br[u] = __bfloat162float(p.beta[row]);
       }
@@ -460,10 +470,9 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         la[j] = r < len ? p.lower_bound * __fdividef(1.f, 1.f + __expf(-ea * (gv[j] + dts[j]))) : 0.f;
-      st4(s + SC_KH + r * D + 4 * lane, scl4(k4[u], ik));
-      st4(s + SC_QH + r * D + 4 * lane, scl4(q4[u], iq));
-      st4(s + SC_G + r * D + 4 * lane, make_float4(la[0], la[1], la[2], la[3]));
-      if (need_v) st4(s + SC_V + r * D + 4 * lane, v4[u]);
+      st4(F.kh + r * D + 4 * lane, scl4(k4[u], ik));
+      st4(F.qh + r * D + 4 * lane, scl4(q4[u], iq));
+      st4(F.G + r * D + 4 * lane, make_float4(la[0], la[1], la[2], la[3]));
       st4(s + SC_DO + r * D + 4 * lane, o4[u]);
       if (lane == 0) s[SC_BETA + r] = r < len ? sigmoid_acc(br[u]) : 0.f;
     }
@@ -475,22 +484,18 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
     for (int r0 = 0; r0 < C; r0 += 16) {
       float col[16];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) col[r] = s[SC_G + (r0 + r) * D + tid];
+      for (int r = 0; r < 16; ++r) col[r] = F.G[(r0 + r) * D + tid];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
         acc += col[r];
-        s[SC_G + (r0 + r) * D + tid] = acc;
+        F.G[(r0 + r) * D + tid] = acc;
       }
     }
     s[SC_EG + tid] = dexp(acc);
   }
   __syncthreads();
-  ew<kB1>(kF4, [&](int i) { return mul4(ld4(s + SC_KH + 4 * i), dexp4(ld4(s + SC_G + 4 * i))); },
-            [&](int i, float4 v) { st4(s + SC_KG + 4 * i, v); });
-  if (!solve) {
-    __syncthreads();
-    return;
-  }
+  ew<kB1>(kF4, [&](int i) { return mul4(ld4(F.kh + 4 * i), dexp4(ld4(F.G + 4 * i))); },
+            [&](int i, float4 v) { st4(F.kg + 4 * i, v); });
   // M and P: row r of block I = r / 16 takes khat_r e^{Gamma_r - rho_I} (qhat_r for P) against the
   // rows s < 16 (I + 1) of R_I = khat_s e^{rho_I - Gamma_s}, rho_I = Gamma at the end of block I - 1
   // (0 for I = 0).  One product [LK; LQ] (128 x 128) R_all^T, R_all the four R_I stacked (160 rows,
@@ -502,17 +507,17 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
     ew<kB1>(2 * kF4,
             [&](int i) {
               const int e = (4 * i) & (kF - 1), r = e >> 7, c = e & (D - 1), I = r >> 4;
-              const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(s + SC_G + (16 * I - 1) * D + c);
-              const float4 x = ld4(s + (4 * i < kF ? SC_KH : SC_QH) + e);
-              return mul4(x, dexp4(sub4(ld4(s + SC_G + e), r4)));
+              const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(F.G + (16 * I - 1) * D + c);
+              const float4 x = ld4((4 * i < kF ? F.kh : F.qh) + e);
+              return mul4(x, dexp4(sub4(ld4(F.G + e), r4)));
             },
             [&](int i, float4 v) { st4(GL + 4 * i, v); });
     ew<kB1>(160 * D / 4,
             [&](int i) {
               const int q = (4 * i) >> 7, c = (4 * i) & (D - 1);
               const int I = q < 16 ? 0 : (q < 48 ? 1 : (q < 96 ? 2 : 3)), srow = q - 8 * I * (I + 1);
-              const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(s + SC_G + (16 * I - 1) * D + c);
-              return mul4(ld4(s + SC_KH + srow * D + c), dexp4(sub4(r4, ld4(s + SC_G + srow * D + c))));
+              const float4 r4 = I == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(F.G + (16 * I - 1) * D + c);
+              return mul4(ld4(F.kh + srow * D + c), dexp4(sub4(r4, ld4(F.G + srow * D + c))));
             },
             [&](int i, float4 v) { st4(GR + 4 * i, v); });
     __syncthreads();
@@ -609,6 +614,37 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
   __syncthreads();
 }
 
+// The gradient kernel's part of a chunk's prologue: V and dO (fp32, rows past the chunk's end zero)
+// and beta into the CTA's scratch; the other element-wise factors come from the prep kernel's output.
+__device__ void load_v_do_beta(const BwdParams& P, const Chunk& ch, float* s) {
+  const FwdParams& p = P.f;
+  const int H = p.num_heads, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r0 = warp; r0 < C; r0 += 2 * (kBwdThreads / 32)) {
+    float4 v4[2], o4[2];
+    float br[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = r0 + u * (kBwdThreads / 32);
+      v4[u] = o4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      br[u] = 0.f;
+      if (r < ch.len) {
+        const size_t row = (size_t)(ch.t0 + r) * H + ch.h;
+        v4[u] = ld_bf16x4(p.v + row * D + 4 * lane);
+        o4[u] = ld_bf16x4(P.d_out + row * D + 4 * lane);
+        br[u] = __bfloat162float(p.beta[row]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = r0 + u * (kBwdThreads / 32);
+      st4(s + SC_V + r * D + 4 * lane, v4[u]);
+      st4(s + SC_DO + r * D + 4 * lane, o4[u]);
+      if (lane == 0) s[SC_BETA + r] = r < ch.len ? sigmoid_acc(br[u]) : 0.f;
+    }
+  }
+  __syncthreads();
+}
+
 // The decay-weighted products of dM and dP (lower triangular, stored adjacent as XX = [dM; dP],
 // 128 x 64) with khat, for rows r:  X1[r] = sum_{s<=r} dM[r][s] khat_s e^{Gamma_r - Gamma_s} and
 // X3[r] = sum_{s<=r} dP[r][s] khat_s e^{Gamma_r - Gamma_s}, per block J of s against rho_J = Gamma at
@@ -616,15 +652,15 @@ __device__ void chunk_factors(const BwdParams& P, const Chunk& ch, float* s, boo
 // above block J add zeros).  X3 is added to out2; X1 is added to dkh and khat X1 to dG, row block J
 // as soon as block J of s (the last to reach it) is done, the later rows' partial sums kept in acc.
 // T: a 128 x 128 temporary.
-__device__ void gated_lower2(float* s, float* dkh, float* dG, float* acc, float* out2, const float* XX, float* T,
+__device__ void gated_lower2(const Fac& F, float* dkh, float* dG, float* acc, float* out2, const float* XX, float* T,
                              float* R, GemmSmem& gsm) {
   for (int J = 0; J < 4; ++J) {
     const int r0 = 16 * J;
-    const float* rho = s + SC_G + (16 * J + 15) * D;
+    const float* rho = F.G + (16 * J + 15) * D;
     ew<kB1>(16 * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
-              return mul4(ld4(s + SC_KH + e), dexp4(sub4(ld4(rho + c), ld4(s + SC_G + e))));
+              return mul4(ld4(F.kh + e), dexp4(sub4(ld4(rho + c), ld4(F.G + e))));
             },
             [&](int i, float4 v) { st4(R + 4 * i, v); });
     __syncthreads();
@@ -632,12 +668,12 @@ __device__ void gated_lower2(float* s, float* dkh, float* dG, float* acc, float*
     ew<kB4>((C - r0) * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
-              const float4 f = dexp4(sub4(ld4(s + SC_G + e), ld4(rho + c)));
+              const float4 f = dexp4(sub4(ld4(F.G + e), ld4(rho + c)));
               float4 v1 = mul4(ld4(T + e), f);
               if (J > 0) v1 = add4(v1, ld4(acc + e));
               const float4 v3 = add4(mul4(ld4(T + C * D + e), f), ld4(out2 + e));
               if (i < 16 * D / 4)  // row block J: X1 complete
-                return F4x4{add4(ld4(dkh + e), v1), add4(ld4(dG + e), mul4(ld4(s + SC_KH + e), v1)), v3, {}};
+                return F4x4{add4(ld4(dkh + e), v1), add4(ld4(dG + e), mul4(ld4(F.kh + e), v1)), v3, {}};
               return F4x4{v1, {}, v3, {}};
             },
             [&](int i, F4x4 v) {
@@ -660,17 +696,17 @@ __device__ void gated_lower2(float* s, float* dkh, float* dG, float* acc, float*
 // dP[K rows, .]^T (scale qhat_K e^{Gamma - rho_K}), times e^{rho_K - Gamma_s}.  X is added to dkh and
 // -khat X to dG, row block K as soon as block K of r (the last to reach it) is done, the earlier
 // rows' partial sums kept in acc.
-__device__ void gated_upper2(float* s, float* dkh, float* dG, float* acc, const float* dM, const float* dP,
+__device__ void gated_upper2(const Fac& F, float* dkh, float* dG, float* acc, const float* dM, const float* dP,
                              float scale, float* R, float* L, GemmSmem& gsm) {
   for (int K = 3; K >= 0; --K) {
     const int r0 = 16 * K, ns = 16 * (K + 1);
-    const float* rho = s + SC_G + (16 * K - 1) * D;
+    const float* rho = F.G + (16 * K - 1) * D;
     ew<kB2>(16 * D / 4,
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = r0 * D + 4 * i;
               const float4 r4 = K == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-              const float4 f = dexp4(sub4(ld4(s + SC_G + e), r4));
-              return F4x2{mul4(ld4(s + SC_KH + e), f), scl4(mul4(ld4(s + SC_QH + e), f), scale)};
+              const float4 f = dexp4(sub4(ld4(F.G + e), r4));
+              return F4x2{mul4(ld4(F.kh + e), f), scl4(mul4(ld4(F.qh + e), f), scale)};
             },
             [&](int i, F4x2 v) {
               st4(R + 4 * i, v.a);
@@ -683,10 +719,10 @@ __device__ void gated_upper2(float* s, float* dkh, float* dG, float* acc, const 
             [&](int i) {
               const int c = (4 * i) & (D - 1), e = 4 * i;
               const float4 r4 = K == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(rho + c);
-              float4 v = mul4(ld4(L + 4 * i), dexp4(sub4(r4, ld4(s + SC_G + e))));
+              float4 v = mul4(ld4(L + 4 * i), dexp4(sub4(r4, ld4(F.G + e))));
               if (K < 3) v = add4(v, ld4(acc + e));
               if (i >= r0 * D / 4)  // row block K: X complete
-                return F4x2{add4(ld4(dkh + e), v), sub4(ld4(dG + e), mul4(ld4(s + SC_KH + e), v))};
+                return F4x2{add4(ld4(dkh + e), v), sub4(ld4(dG + e), mul4(ld4(F.kh + e), v))};
               return F4x2{v, {}};
             },
             [&](int i, F4x2 v) {
@@ -773,16 +809,17 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_prep_kernel(BwdParams P, i
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
     float* pr = P.prep + (size_t)it * kPrepFloats;
-    chunk_factors(P, ch, s, false, true, gsm, sT, sA, pr + PR_M, pr + PR_T, pr + PR_TB);
+    const Fac F = fac_of(pr);  // khat, qhat, Gamma and Kg straight to the output (the gradient kernel reads them)
+    chunk_factors(P, ch, s, F, gsm, sT, sA, pr + PR_M, pr + PR_T, pr + PR_TB);
     // W = T_b Kg (to the output); Kt = khat e^{gamma - Gamma}; X = Qt - P W
-    gemm(pr + PR_W, D, mat(s + SC_TB, C), mat(s + SC_KG, D), C, D, C, 1.f, false, 0, gsm);
-    const float* gam = s + SC_G + (C - 1) * D;
+    gemm(pr + PR_W, D, mat(s + SC_TB, C), mat(F.kg, D), C, D, C, 1.f, false, 0, gsm);
+    const float* gam = F.G + (C - 1) * D;
     ew<kB2>(kF4,
               [&](int i) {
                 const int c = (4 * i) & (D - 1);
-                const float4 G = ld4(s + SC_G + 4 * i);
-                return F4x2{mul4(ld4(s + SC_KH + 4 * i), dexp4(sub4(ld4(gam + c), G))),
-                            scl4(mul4(ld4(s + SC_QH + 4 * i), dexp4(G)), scale)};
+                const float4 G = ld4(F.G + 4 * i);
+                return F4x2{mul4(ld4(F.kh + 4 * i), dexp4(sub4(ld4(gam + c), G))),
+                            scl4(mul4(ld4(F.qh + 4 * i), dexp4(G)), scale)};
               },
               [&](int i, F4x2 v) {
                 st4(pr + PR_KT + 4 * i, v.a);
@@ -935,9 +972,10 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
   const int64_t n_items = min(items, (int64_t)P.chunk_off[p.num_seqs] * H);
   for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
     const Chunk ch = locate(P, it);
-    chunk_factors(P, ch, s, true, false, gsm, nullptr, nullptr);
-    // M, T = (I + A)^{-1} and T_b = T diag(beta) as the prep kernel stored them
-    const float* pr = P.prep + (size_t)it * kPrepFloats;
+    // M, T = (I + A)^{-1}, T_b = T diag(beta), khat, qhat, Gamma and Kg as the prep kernel stored them
+    float* pr = P.prep + (size_t)it * kPrepFloats;
+    const Fac F = fac_of(pr);
+    load_v_do_beta(P, ch, s);
     const float* Mp = pr + PR_M;
     const float* Tp = pr + PR_T;
     const float* TBp = pr + PR_TB;
@@ -967,12 +1005,12 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
       }
       if (h == 1) s[SC_DGAM + k] = acc;
       __syncthreads();
-      if (h == 0) s[SC_DGAM + k] = s[SC_EG + k] * (acc + s[SC_DGAM + k]);
+      if (h == 0) s[SC_DGAM + k] = pr[PR_EG + k] * (acc + s[SC_DGAM + k]);
     }
     // dT_b = dDelta V^T + dW Kg^T;  dv = T_b^T dDelta;  dKg = T_b^T dW
     gemm<2>(s + SC_DTB, C, mat(dD, D), mat(s + SC_V, D, true), C, C, D, 1.f, false, 0, gsm);
     // with dT = dT_b diag(beta) (to DA)
-    gemm_e(mat(s + SC_DW, D), mat(s + SC_KG, D, true), C, C, D, gsm, EpiDtb{s + SC_DTB, s + SC_DA, s + SC_BETA});
+    gemm_e(mat(s + SC_DW, D), mat(F.kg, D, true), C, C, D, gsm, EpiDtb{s + SC_DTB, s + SC_DA, s + SC_BETA});
     gemm_e(mat(TBp, C, true), mat(dD, D), C, D, C, gsm,
            EpiDv{P.dv + ((size_t)ch.t0 * H + ch.h) * D, (int64_t)H * D, ch.len});
     gemm(s + SC_DKG, D, mat(TBp, C, true), mat(s + SC_DW, D), C, D, C, 1.f, false, 0, gsm);
@@ -1010,14 +1048,14 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
     float* dkh = s + SC_DKG;  // becomes dkhat: e^Gamma dKg first
     float* dqh = s + SC_DQS;  // becomes dqhat / scale: e^Gamma dO S^T first
     float* dG = s + SC_W;     // dGamma
-    const float* gam = s + SC_G + (C - 1) * D;
+    const float* gam = F.G + (C - 1) * D;
     ew<kB4>(kF4,
               [&](int i) {
                 const int c = (4 * i) & (D - 1);
-                const float4 G = ld4(s + SC_G + 4 * i), eG = dexp4(G);
+                const float4 G = ld4(F.G + 4 * i), eG = dexp4(G);
                 const float4 a = mul4(ld4(dkh + 4 * i), eG);                                   // e^Gamma dKg
                 const float4 b = mul4(ld4(s + SC_DKT + 4 * i), dexp4(sub4(ld4(gam + c), G)));  // e^{gamma-Gamma} dKt
-                return F4x4{add4(a, b), mul4(ld4(s + SC_KH + 4 * i), sub4(a, b)), b, mul4(ld4(dqh + 4 * i), eG)};
+                return F4x4{add4(a, b), mul4(ld4(F.kh + 4 * i), sub4(a, b)), b, mul4(ld4(dqh + 4 * i), eG)};
               },
               [&](int i, F4x4 v) {
                 st4(dkh + 4 * i, v.a);
@@ -1027,9 +1065,9 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
               });
     __syncthreads();
     // X1 (into dkhat and dGamma) and X3 (added to dqhat / scale) in one pass; V and dO are dead: their
-    // 2 x 64 x 128 floats hold the 128 x 128 temporary.  Delta, dW and Kg are dead as well.
-    gated_lower2(s, dkh, dG, s + SC_D, dqh, s + SC_DA, s + SC_DO, s + SC_DW, gsm);
-    gated_upper2(s, dkh, dG, s + SC_D, s + SC_DA, s + SC_DP, scale, s + SC_DW, s + SC_KG, gsm);  // X2 + X4
+    // 2 x 64 x 128 floats hold the 128 x 128 temporary.  Delta and dW are dead as well.
+    gated_lower2(F, dkh, dG, s + SC_D, dqh, s + SC_DA, s + SC_DO, s + SC_DW, gsm);
+    gated_upper2(F, dkh, dG, s + SC_D, s + SC_DA, s + SC_DP, scale, s + SC_DW, s + SC_L, gsm);  // X2 + X4
     // dgamma: the state term plus sum_r khat e^{gamma-Gamma} dKt; then dlog alpha by a reverse running sum
     {
       // thread (channel k, half h of the rows): the half's share of dgamma and the total of its
@@ -1040,8 +1078,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
 #pragma unroll 8
       for (int r = 32 * h; r < 32 * h + 32; ++r) {
         const int e = r * D + k;
-        pg = fmaf(s[SC_KH + e], s[SC_DKT + e], pg);
-        tot += dG[e] + scale * s[SC_QH + e] * dqh[e];
+        pg = fmaf(F.kh[e], s[SC_DKT + e], pg);
+        tot += dG[e] + scale * F.qh[e] * dqh[e];
       }
       part[h * D + k] = pg;
       part[2 * D + h * D + k] = tot;
@@ -1053,7 +1091,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_grad_kernel(BwdParams P, i
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
           const int e = (r0 + r) * D + k;
-          col[r] = dG[e] + scale * s[SC_QH + e] * dqh[e];
+          col[r] = dG[e] + scale * F.qh[e] * dqh[e];
         }
 #pragma unroll
         for (int r = 15; r >= 0; --r) {
