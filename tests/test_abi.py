@@ -80,6 +80,21 @@ def call(lib, name="kda_fwd", **kw):
                               a["H"], a["K"], a["V"], a["N"], a["transposed"], None)
 
 
+
+@pytest.mark.parametrize("T,H,N", [(4096, 96, 1), (350, 2, 3), (1, 1, 1), (100000, 8, 40)])
+def test_bwd_workspace_size_is_its_documented_parts(lib, T, H, N):
+    """kda_bwd_workspace_size as kda.h describes it: the forward's workspace, the checkpoints and the
+    recomputed output, the chunk table, per (chunk, head) the chunk's factors (336.5 KB) and dDelta
+    (32 KB), one 128 x 128 fp32 state gradient per chunk slot and head, the per-token partials
+    (3 x 128 + 1 fp32), and the larger of 296 CTAs' scratch (369.75 KB each) and one 64 x 128 fp32
+    buffer per (sequence, head); every region 256-byte aligned."""
+    a256 = lambda b: (b + 255) // 256 * 256
+    chunks, slots = T // 64 + N, T // 64 + N + 1
+    parts = [lib.kda_workspace_size(T, H, N), lib.kda_checkpoint_size(T, H, N), T * H * 128 * 2, (N + 1) * 4,
+             chunks * H * 344576, slots * H * 128 * 128 * 4, chunks * H * 64 * 128 * 4, (3 * 128 + 1) * 4 * T * H,
+             max(296 * 378624, N * H * 64 * 128 * 4)]
+    assert lib.kda_bwd_workspace_size(T, H, N) == sum(a256(p) for p in parts)
+
 @pytest.mark.parametrize("name", ["kda_fwd", "kda_fwd_recurrent"])
 def test_host_validation(lib, name):
     assert call(lib, name, K=64) == 2
